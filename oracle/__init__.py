@@ -1,0 +1,318 @@
+"""CPU oracle for the FourTune W4A4G4 triple-branch linear layer.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / reference leg of ``bench.py`` may import this package.  The
+CUDA library never loads it and shares no code with it.
+
+Sources (page "FourTune: Towards Fully 4-Bit Efficient Post-Training for
+Diffusion Models"):
+  * Eq. 1 (section 3.1): W ~ R + L_stab with L_stab = L1 L2 from the SVD.
+  * Eq. 2 (section 3.1): Y = GEMM4(Q(X), Q(R)) + X L_stab + X (A B).
+  * Eq. 3 (section 3.2): dX = GEMM4(Q(G), Q(R)^T) + G L_stab^T + G (A B)^T.
+  * Section 3.2, LoRA gradients: dB = (X A)^T G, dA = X^T (G B^T).
+  * Section 3.2: 16x16 weight blocks, so Q(R)^T is the transposed codes with
+    the same scales.
+
+Convention (PyTorch style, weights stored [out, in]):
+  W, W_res: [N, K];  U: [K, r_s];  V: [N, r_s];  A: [K, r_l];  B: [N, r_l]
+  Y = Q(X) Q(W_res)^T + (X U) V^T + s (X A) B^T
+so L_stab = (U V^T)^T in the page's notation and the page's R is W_res^T.
+
+The bit-level quantizer lives in ``ft_oracle.c`` (plain C, compiled with
+gcc -O2 -ffp-contract=off, no fast-math).  The contractions here use numpy's
+float64 matmul as a library primitive on the dequantized operands; nothing
+is blocked, fused or reordered beyond the equations above.
+
+Rounding points (the page is silent; plainest reading):
+  P   = [bf16(X U) | bf16(s * (X A))]          saved for the backward
+  Pg  = [bf16(dY V) | bf16(s * (dY B))]
+  Y, dX in float64;  dA = X^T Pg_lora,  dB = dY^T P_lora in float64.
+The low-rank branches read the unquantized bf16 X and dY (Eq. 2 and Eq. 3
+apply Q only inside GEMM4).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ft_oracle.c")
+_LIB_DIR = os.path.join(_HERE, "_build")
+_LIB = os.path.join(_LIB_DIR, "libft_oracle.so")
+
+_u8p = np.ctypeslib.ndpointer(dtype=np.uint8, flags="C_CONTIGUOUS")
+_u16p = np.ctypeslib.ndpointer(dtype=np.uint16, flags="C_CONTIGUOUS")
+_f64p = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
+_i64p = np.ctypeslib.ndpointer(dtype=np.int64, flags="C_CONTIGUOUS")
+
+
+def build(force: bool = False) -> str:
+    """Compile ft_oracle.c into a shared library (gcc, IEEE single, no FMA)."""
+    os.makedirs(_LIB_DIR, exist_ok=True)
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+               "-fno-fast-math", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        L.fto_e2m1_value.restype = ctypes.c_double
+        L.fto_e2m1_value.argtypes = [ctypes.c_uint8]
+        L.fto_e2m1_encode.restype = ctypes.c_uint8
+        L.fto_e2m1_encode.argtypes = [ctypes.c_float]
+        L.fto_e4m3_value.restype = ctypes.c_double
+        L.fto_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.fto_e4m3_encode.restype = ctypes.c_uint8
+        L.fto_e4m3_encode.argtypes = [ctypes.c_float]
+        L.fto_amax_bf16.restype = ctypes.c_float
+        L.fto_amax_bf16.argtypes = [_u16p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64]
+        L.fto_tensor_scale.restype = ctypes.c_float
+        L.fto_tensor_scale.argtypes = [ctypes.c_float]
+        L.fto_quantize_1x16.restype = None
+        L.fto_quantize_1x16.argtypes = [_u16p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                        ctypes.c_float, _u8p, _u8p,
+                                        ctypes.POINTER(ctypes.c_float)]
+        L.fto_quantize_16x16.restype = None
+        L.fto_quantize_16x16.argtypes = [_u16p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                         ctypes.c_float, _u8p, ctypes.c_void_p, _u8p,
+                                         ctypes.POINTER(ctypes.c_float)]
+        L.fto_dequant_1x16.restype = None
+        L.fto_dequant_1x16.argtypes = [_u8p, _u8p, ctypes.c_float, ctypes.c_int64,
+                                       ctypes.c_int64, _f64p]
+        L.fto_dequant_16x16.restype = None
+        L.fto_dequant_16x16.argtypes = [_u8p, _u8p, ctypes.c_float, ctypes.c_int64,
+                                        ctypes.c_int64, _f64p]
+        L.fto_gemm_nt_f64.restype = None
+        L.fto_gemm_nt_f64.argtypes = [_f64p, _f64p, ctypes.c_int64, ctypes.c_int64, _i64p,
+                                      ctypes.c_int64, _f64p]
+        _lib = L
+    return _lib
+
+
+# ------------------------------------------------------------------ formats
+
+def e2m1_value(code: int) -> float:
+    return lib().fto_e2m1_value(code)
+
+
+def e2m1_encode(q: float) -> int:
+    return lib().fto_e2m1_encode(q)
+
+
+def e4m3_value(byte: int) -> float:
+    return lib().fto_e4m3_value(byte)
+
+
+def e4m3_encode(v: float) -> int:
+    return lib().fto_e4m3_encode(v)
+
+
+# --------------------------------------------------------------------- bf16
+
+def bf16_to_f64(u16: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns."""
+    u32 = np.asarray(u16, dtype=np.uint16).astype(np.uint32) << 16
+    return u32.view(np.float32).astype(np.float64)
+
+
+def bf16_from_f64(v) -> np.ndarray:
+    """Round float64 values to bf16 (round-to-nearest-even), as bit patterns.
+
+    bf16 keeps 8 significant bits; the rounding quantum of a value with
+    binary exponent e (v = m 2^e, 0.5 <= |m| < 1) is 2^(e-8), and never finer
+    than the subnormal quantum 2^-133.  Scaling by powers of two is exact, so
+    np.rint performs exactly one RNE rounding.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    _, e = np.frexp(v)
+    q = np.maximum(e - 8, -133)
+    r = np.ldexp(np.rint(np.ldexp(v, -q)), q)
+    with np.errstate(over="ignore"):
+        f = r.astype(np.float32)
+    return (f.view(np.uint32) >> 16).astype(np.uint16)
+
+
+# ------------------------------------------------------------- quantization
+
+def amax_bf16(x: np.ndarray) -> float:
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    return float(lib().fto_amax_bf16(x, x.shape[0], x.shape[1], x.shape[1]))
+
+
+def tensor_scale(amax: float) -> float:
+    return float(lib().fto_tensor_scale(amax))
+
+
+def quantize_1x16(x: np.ndarray, amax: float | None = None):
+    """1x16 NVFP4 quantization along rows.  Returns (codes, scales, g)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    rows, cols = x.shape
+    assert cols % 16 == 0
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    scales = np.zeros((rows, cols // 16), np.uint8)
+    g = ctypes.c_float(0.0)
+    lib().fto_quantize_1x16(x, rows, cols, cols, -1.0 if amax is None else float(amax),
+                            codes, scales, ctypes.byref(g))
+    return codes, scales, float(np.float32(g.value))
+
+
+def quantize_16x16(x: np.ndarray, amax: float | None = None, want_col: bool = True):
+    """16x16 NVFP4 quantization.  Returns (codes_row, codes_col, scales, g);
+    codes_col holds the same codes packed along columns (the transpose)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    rows, cols = x.shape
+    assert rows % 16 == 0 and cols % 16 == 0
+    codes_row = np.zeros((rows, cols // 2), np.uint8)
+    codes_col = np.zeros((cols, rows // 2), np.uint8) if want_col else None
+    scales = np.zeros((rows // 16, cols // 16), np.uint8)
+    g = ctypes.c_float(0.0)
+    col_ptr = codes_col.ctypes.data_as(ctypes.c_void_p) if want_col else None
+    lib().fto_quantize_16x16(x, rows, cols, cols, -1.0 if amax is None else float(amax),
+                             codes_row, col_ptr, scales, ctypes.byref(g))
+    return codes_row, codes_col, scales, float(np.float32(g.value))
+
+
+def quantize_1x16_colwise(x: np.ndarray, amax: float | None = None):
+    """Column-wise copy: 1x16 quantization of x^T (blocks run along the rows
+    of x), sharing the tensor scale of x."""
+    if amax is None:
+        amax = amax_bf16(x)
+    return quantize_1x16(np.ascontiguousarray(np.asarray(x).T), amax)
+
+
+def dequant_1x16(codes, scales, g, rows, cols) -> np.ndarray:
+    out = np.empty((rows, cols), np.float64)
+    lib().fto_dequant_1x16(np.ascontiguousarray(codes), np.ascontiguousarray(scales),
+                           float(g), rows, cols, out)
+    return out
+
+
+def dequant_16x16(codes_row, scales, g, rows, cols) -> np.ndarray:
+    out = np.empty((rows, cols), np.float64)
+    lib().fto_dequant_16x16(np.ascontiguousarray(codes_row), np.ascontiguousarray(scales),
+                            float(g), rows, cols, out)
+    return out
+
+
+def gemm_nt_plain(A: np.ndarray, B: np.ndarray, rows=None) -> np.ndarray:
+    """C = A[rows] B^T by a plain triple loop in C (FP64)."""
+    A = np.ascontiguousarray(A, dtype=np.float64)
+    B = np.ascontiguousarray(B, dtype=np.float64)
+    idx = np.arange(A.shape[0], dtype=np.int64) if rows is None else np.asarray(rows, np.int64)
+    C = np.empty((len(idx), B.shape[0]), np.float64)
+    lib().fto_gemm_nt_f64(A, B, A.shape[1], B.shape[0], np.ascontiguousarray(idx), len(idx), C)
+    return C
+
+
+# -------------------------------------------------------------- weight prep
+
+def svd_split(W: np.ndarray, r_s: int):
+    """Eq. 1: W ~ W_res + V U^T with the top-r_s singular triplets.
+
+    The right singular vectors of W are the eigenvectors of W^T W; the top
+    r_s of them form U [K, r_s] and V = W U = (left vectors) * sigma
+    [N, r_s].  U and V are rounded to bf16 first and W_res = W - V U^T is
+    formed from the rounded factors, so W_res + V U^T reproduces W up to the
+    bf16 rounding of W_res.  Returns bf16 bit patterns (U, V, W_res).
+    """
+    Wd = bf16_to_f64(W)
+    if r_s == 0:
+        K, N = Wd.shape[1], Wd.shape[0]
+        return (np.zeros((K, 0), np.uint16), np.zeros((N, 0), np.uint16), np.asarray(W, np.uint16))
+    evals, evecs = np.linalg.eigh(Wd.T @ Wd)
+    top = evecs[:, np.argsort(evals)[::-1][:r_s]]
+    U = bf16_from_f64(top)
+    V = bf16_from_f64(Wd @ bf16_to_f64(U))
+    W_res = bf16_from_f64(Wd - bf16_to_f64(V) @ bf16_to_f64(U).T)
+    return U, V, W_res
+
+
+# -------------------------------------------------------------- layer math
+
+def _lowrank_down(Xd: np.ndarray, L1: np.ndarray, L2: np.ndarray, s: float):
+    """[bf16(X L1) | bf16(s (X L2))] from float64 values (bf16 inputs)."""
+    parts = []
+    if L1.shape[1]:
+        parts.append(bf16_from_f64(Xd @ bf16_to_f64(L1)))
+    if L2.shape[1]:
+        parts.append(bf16_from_f64(s * (Xd @ bf16_to_f64(L2))))
+    if not parts:
+        return np.zeros((Xd.shape[0], 0), np.uint16)
+    return np.concatenate(parts, axis=1)
+
+
+def linear_fwd(X, W_res, U, V, A, B, s: float, rows=None, amax_x=None, qw=None):
+    """Forward of the triple-branch layer (Eq. 2).
+
+    X: bf16 [M, K]; W_res: bf16 [N, K]; U [K, r_s]; V [N, r_s]; A [K, r_l];
+    B [N, r_l].  rows: optional row sample for Y (the quantization and P are
+    always computed on the full tensors).  qw: optional precomputed
+    quantize_16x16(W_res).  Returns a dict with Y (float64 [len(rows), N]),
+    P (bf16 [M, r_s + r_l]), qx = (codes, scales, g) and qw.
+    """
+    M, K = X.shape
+    N = W_res.shape[0]
+    rows = np.arange(M) if rows is None else np.asarray(rows)
+    qx = quantize_1x16(X, amax_x)
+    if qw is None:
+        qw = quantize_16x16(W_res)
+    Xq = dequant_1x16(qx[0], qx[1], qx[2], M, K)[rows]
+    Wq = dequant_16x16(qw[0], qw[2], qw[3], N, K)
+    Xd = bf16_to_f64(X)
+    P = _lowrank_down(Xd, U, A, s)
+    Pd = bf16_to_f64(P[rows])
+    LR = np.concatenate([bf16_to_f64(V), bf16_to_f64(B)], axis=1)  # [N, r_s + r_l]
+    Y = Xq @ Wq.T + Pd @ LR.T
+    return {"Y": Y, "P": P, "qx": qx, "qw": qw, "rows": rows}
+
+
+def linear_bwd(dY, X, W_res, U, V, A, B, s: float, P, rows=None, amax_dy=None, qw=None):
+    """Backward of the triple-branch layer (Eq. 3 and the LoRA gradients).
+
+    dY: bf16 [M, N]; X: bf16 [M, K]; P: the forward's saved bf16 [M, r_s+r_l].
+    Returns dX (float64 [len(rows), K]), dA (float64 [K, r_l]),
+    dB (float64 [N, r_l]), Pg (bf16 [M, r_s + r_l]) and qdy.
+    """
+    M, N = dY.shape
+    K = X.shape[1]
+    r_s, r_l = U.shape[1], A.shape[1]
+    rows = np.arange(M) if rows is None else np.asarray(rows)
+    qdy = quantize_1x16(dY, amax_dy)
+    if qw is None:
+        qw = quantize_16x16(W_res)
+    dYq = dequant_1x16(qdy[0], qdy[1], qdy[2], M, N)[rows]
+    Wq = dequant_16x16(qw[0], qw[2], qw[3], N, K)
+    dYd = bf16_to_f64(dY)
+    Pg = _lowrank_down(dYd, V, B, s)
+    Pgd = bf16_to_f64(Pg)
+    LR = np.concatenate([bf16_to_f64(U), bf16_to_f64(A)], axis=1)  # [K, r_s + r_l]
+    dX = dYq @ Wq + Pgd[rows] @ LR.T
+    P_lora = bf16_to_f64(np.asarray(P)[:, r_s:r_s + r_l])
+    Pg_lora = Pgd[:, r_s:r_s + r_l]
+    dB = dYd.T @ P_lora
+    dA = bf16_to_f64(X).T @ Pg_lora
+    return {"dX": dX, "dA": dA, "dB": dB, "Pg": Pg, "qdy": qdy, "rows": rows}
+
+
+def rel_fro(a: np.ndarray, b: np.ndarray) -> float:
+    """||a - b||_F / ||b||_F (0 when both are zero)."""
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    nb = np.linalg.norm(b)
+    na = np.linalg.norm(a - b)
+    if nb == 0.0:
+        return 0.0 if na == 0.0 else float("inf")
+    return float(na / nb)

@@ -1,0 +1,142 @@
+"""Pins of the oracle's triple-branch layer (Eq. 1-3 of the FourTune page and
+the LoRA gradients of section 3.2).
+
+The structure of the forward and backward (which operand is transposed,
+which branch reads the quantized tensors, where s sits, which terms dX sums)
+is pinned against torch autograd in float64 on inputs where every
+quantization and every bf16 rounding point is exact, so the oracle must equal
+the unquantized layer's true gradients.  The library matmul the oracle uses is
+pinned against a plain C triple loop, and the SVD split against numpy's SVD.
+"""
+import numpy as np
+import pytest
+import torch
+
+import ft_synth
+import oracle
+
+
+def test_numpy_matmul_matches_plain_loop():
+    rng = np.random.default_rng(20)
+    A = rng.standard_normal((37, 53))
+    B = rng.standard_normal((29, 53))
+    C = oracle.gemm_nt_plain(A, B)
+    np.testing.assert_allclose(A @ B.T, C, rtol=1e-12, atol=1e-12)
+    rows = [3, 0, 36]
+    np.testing.assert_allclose(oracle.gemm_nt_plain(A, B, rows), (A @ B.T)[rows], rtol=1e-12)
+
+
+def test_svd_split_reconstructs_w_and_is_best_rank_r():
+    rng = np.random.default_rng(21)
+    N, K, r = 96, 64, 8
+    W = ft_synth.to_bf16_bits(rng.standard_normal((N, K)) * 0.02
+                              + np.outer(rng.standard_normal(N), rng.standard_normal(K)) * 0.1)
+    U, V, Wr = oracle.svd_split(W, r)
+    assert U.shape == (K, r) and V.shape == (N, r) and Wr.shape == (N, K)
+    Wd = oracle.bf16_to_f64(W)
+    L = oracle.bf16_to_f64(V) @ oracle.bf16_to_f64(U).T
+    recon = oracle.bf16_to_f64(Wr) + L
+    # W_res is bf16(W - L): the reconstruction error is its rounding only
+    assert np.all(np.abs(recon - Wd) <= np.abs(oracle.bf16_to_f64(Wr)) * 2.0 ** -8 + 1e-30)
+    # V U^T is the best rank-r approximation (to bf16 precision of U, V)
+    u, sv, vt = np.linalg.svd(Wd)
+    best = (u[:, :r] * sv[:r]) @ vt[:r]
+    assert np.linalg.norm(L - best) <= 1e-2 * np.linalg.norm(best)
+    # r_s = 0 leaves W untouched
+    U0, V0, W0 = oracle.svd_split(W, 0)
+    assert U0.shape == (K, 0) and np.array_equal(W0, W)
+
+
+def _selection(rng, rows, cols):
+    """One non-zero (+-0.5, +-1, +-2) per column: products with lossless
+    operands stay exactly representable in bf16."""
+    m = np.zeros((rows, cols))
+    for j in range(cols):
+        m[rng.integers(rows), j] = rng.choice([-2.0, -1.0, -0.5, 0.5, 1.0, 2.0])
+    return ft_synth.to_bf16_bits(m)
+
+
+def _exact_case(seed, M=32, K=64, N=48, r_s=4, r_l=4, s=0.5):
+    rng = np.random.default_rng(seed)
+    X = ft_synth.lossless_fp4_operand(rng, M, K, 1, exp_range=(-2, 2))
+    Wr = ft_synth.lossless_fp4_operand(rng, N, K, 16, exp_range=(-2, 2))
+    dY = ft_synth.lossless_fp4_operand(rng, M, N, 1, exp_range=(-2, 2))
+    U = _selection(rng, K, r_s)
+    A = _selection(rng, K, r_l)
+    V = _selection(rng, N, r_s)
+    B = _selection(rng, N, r_l)
+    # amax 2688 * 4 -> g = 4: block maxima 6 * 2^e, e in [-2, 2], give exact
+    # power-of-two scales 2^(e-2)
+    amax = 2688.0 * 4.0
+    qw = oracle.quantize_16x16(Wr, amax)
+    return dict(X=X, Wr=Wr, dY=dY, U=U, V=V, A=A, B=B, s=s, amax=amax, qw=qw)
+
+
+def _torch_layer(c):
+    t = {k: torch.tensor(oracle.bf16_to_f64(c[k]), dtype=torch.float64, requires_grad=(k in "XAB"))
+         for k in ["X", "Wr", "U", "V", "A", "B", "dY"]}
+    Y = t["X"] @ t["Wr"].T + (t["X"] @ t["U"]) @ t["V"].T + c["s"] * (t["X"] @ t["A"]) @ t["B"].T
+    (Y * t["dY"]).sum().backward()
+    return Y.detach().numpy(), t["X"].grad.numpy(), t["A"].grad.numpy(), t["B"].grad.numpy()
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_layer_equals_autograd_when_quantization_is_exact(seed):
+    c = _exact_case(seed)
+    f = oracle.linear_fwd(c["X"], c["Wr"], c["U"], c["V"], c["A"], c["B"], c["s"],
+                          amax_x=c["amax"], qw=c["qw"])
+    b = oracle.linear_bwd(c["dY"], c["X"], c["Wr"], c["U"], c["V"], c["A"], c["B"], c["s"],
+                          f["P"], amax_dy=c["amax"], qw=c["qw"])
+    Y, dX, dA, dB = _torch_layer(c)
+    np.testing.assert_allclose(f["Y"], Y, rtol=1e-12, atol=1e-9)
+    np.testing.assert_allclose(b["dX"], dX, rtol=1e-12, atol=1e-9)
+    np.testing.assert_allclose(b["dA"], dA, rtol=1e-12, atol=1e-9)
+    np.testing.assert_allclose(b["dB"], dB, rtol=1e-12, atol=1e-9)
+    # each branch matters: dropping any one of them changes Y or dX
+    assert np.abs(Y).max() > 0 and np.abs(dA).max() > 0 and np.abs(dB).max() > 0
+
+
+def test_saved_p_layout():
+    c = _exact_case(5, r_s=3, r_l=5)
+    f = oracle.linear_fwd(c["X"], c["Wr"], c["U"], c["V"], c["A"], c["B"], c["s"],
+                          amax_x=c["amax"], qw=c["qw"])
+    Xd = oracle.bf16_to_f64(c["X"])
+    P = oracle.bf16_to_f64(f["P"])
+    assert P.shape == (32, 8)
+    np.testing.assert_array_equal(P[:, :3], Xd @ oracle.bf16_to_f64(c["U"]))
+    np.testing.assert_array_equal(P[:, 3:], c["s"] * (Xd @ oracle.bf16_to_f64(c["A"])))
+
+
+def test_no_low_rank_reduces_to_plain_nvfp4_gemm_and_zero_input():
+    rng = np.random.default_rng(22)
+    M, K, N = 32, 64, 48
+    X = ft_synth.to_bf16_bits(rng.standard_normal((M, K)))
+    W = ft_synth.to_bf16_bits(rng.standard_normal((N, K)) * 0.02)
+    z = lambda r, c: np.zeros((r, c), np.uint16)
+    f = oracle.linear_fwd(X, W, z(K, 0), z(N, 0), z(K, 0), z(N, 0), 1.0)
+    cx, sx, gx = oracle.quantize_1x16(X)
+    cw, _, sw, gw = oracle.quantize_16x16(W)
+    ref = oracle.dequant_1x16(cx, sx, gx, M, K) @ oracle.dequant_16x16(cw, sw, gw, N, K).T
+    np.testing.assert_array_equal(f["Y"], ref)
+    # X = 0 gives Y = 0 and P = 0 even with low-rank branches present
+    U = ft_synth.to_bf16_bits(rng.standard_normal((K, 4)))
+    V = ft_synth.to_bf16_bits(rng.standard_normal((N, 4)))
+    f0 = oracle.linear_fwd(z(M, K), W, U, V, U, V, 1.0)
+    assert not f0["Y"].any() and not f0["P"].any()
+
+
+def test_quantized_layer_is_close_to_unquantized_layer():
+    """Gross-error pin: NVFP4 with 1x16 / 16x16 blocks perturbs a Gaussian
+    GEMM by a few percent, not by a factor."""
+    rng = np.random.default_rng(23)
+    M, K, N = 64, 256, 128
+    X = ft_synth.to_bf16_bits(rng.standard_normal((M, K)))
+    W = ft_synth.to_bf16_bits(rng.standard_normal((N, K)) * 0.02)
+    U, V, Wr = oracle.svd_split(W, 8)
+    A = ft_synth.to_bf16_bits(rng.standard_normal((K, 8)) * 0.01)
+    B = ft_synth.to_bf16_bits(rng.standard_normal((N, 8)) * 0.01)
+    f = oracle.linear_fwd(X, Wr, U, V, A, B, 1.0)
+    Xd = oracle.bf16_to_f64(X)
+    exact = Xd @ oracle.bf16_to_f64(W).T + (Xd @ oracle.bf16_to_f64(A)) @ oracle.bf16_to_f64(B).T
+    err = oracle.rel_fro(f["Y"], exact)
+    assert 0.01 < err < 0.2
