@@ -56,6 +56,7 @@ double fto_e2m1_value(uint8_t code) {
 uint8_t fto_e2m1_encode(float q) {
     uint8_t sign = signbit(q) ? 8u : 0u;
     double a = fabs((double)q);
+    if (a >= 6.0) return (uint8_t)(sign | 7u); /* saturation, infinity included */
     int best = 0;
     double best_d = a; /* distance to magnitude 0 */
     for (int c = 1; c < 8; ++c) {
