@@ -1,0 +1,273 @@
+"""B200-native W4A4G4 triple-branch linear layer (FourTune).
+
+Thin Python binding over the C ABI of include/ft.h.  Every function here only
+marshals torch CUDA tensors into pointers and calls the CUDA library; all
+arithmetic of the hot path runs in the library's sm_100a kernels.  PyTorch is
+used for device memory and streams.
+
+    layer = prepare_layer(W, r_s=32, A=A, B=B, s=1.0)    # once per layer
+    Y, P  = ft_linear_fwd(layer, X)                       # Eq. 2
+    dX, dA, dB = ft_linear_bwd(layer, dY, X, P)           # Eq. 3 + adapter grads
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from ._lib import FtFp4, FtLinear, FtError, check, load
+
+BLK_1x16 = 0
+BLK_16x16 = 1
+BF16 = 0
+F32 = 1
+
+__all__ = [
+    "FP4", "Layer", "FtError", "BLK_1x16", "BLK_16x16", "BF16", "F32",
+    "ft_quantize", "ft_quantize_transpose", "ft_linear_fwd", "ft_linear_bwd",
+    "ft_workspace_bytes", "ft_quantize_workspace_bytes", "ft_device_error",
+    "prepare_layer", "svd_split", "Workspace", "timing",
+]
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _bf16(t: torch.Tensor, name: str) -> torch.Tensor:
+    if t.dtype != torch.bfloat16 or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA bfloat16 tensor")
+    return t
+
+
+@dataclass
+class FP4:
+    """NVFP4 tensor: codes [rows, cols/2] uint8, scales (E4M3 bytes) and the
+    decode tensor scale (1 float), all device tensors."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    tscale: torch.Tensor
+    rows: int
+    cols: int
+    blk: int
+
+    @staticmethod
+    def empty(rows: int, cols: int, blk: int, device, scales=None, tscale=None) -> "FP4":
+        codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=device)
+        if scales is None:
+            sshape = (rows, cols // 16) if blk == BLK_1x16 else (rows // 16, cols // 16)
+            scales = torch.empty(sshape, dtype=torch.uint8, device=device)
+        if tscale is None:
+            tscale = torch.empty(1, dtype=torch.float32, device=device)
+        return FP4(codes, scales, tscale, rows, cols, blk)
+
+    def view(self) -> FtFp4:
+        return FtFp4(self.codes.data_ptr(), _ptr(self.scales), _ptr(self.tscale), self.rows,
+                     self.cols, self.blk)
+
+
+class Workspace:
+    """Caller-owned scratch for the library (it never allocates)."""
+
+    def __init__(self):
+        self.buf = None
+
+    def get(self, nbytes: int, device) -> torch.Tensor:
+        if self.buf is None or self.buf.numel() < nbytes or self.buf.device != torch.device(device):
+            self.buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        return self.buf
+
+
+_default_ws: dict = {}
+
+
+def _ws(ws, nbytes, device):
+    if ws is None:
+        key = torch.device(device)
+        ws = _default_ws.setdefault(key, Workspace())
+    return ws.get(nbytes, device)
+
+
+def ft_workspace_bytes(M: int, N: int, K: int, r_s: int, r_l: int) -> int:
+    return load().ft_workspace_bytes(M, N, K, r_s, r_l)
+
+
+def ft_quantize_workspace_bytes() -> int:
+    return load().ft_quantize_workspace_bytes()
+
+
+def ft_quantize(x: torch.Tensor, blk: int = BLK_1x16, amax: torch.Tensor | None = None,
+                out: FP4 | None = None, ws: Workspace | None = None, stream=None) -> FP4:
+    """Q(x): NVFP4 block quantization of a 2-D bf16 CUDA tensor."""
+    _bf16(x, "x")
+    rows, cols = x.shape
+    if x.stride(1) != 1:
+        raise ValueError("x must have unit column stride")
+    out = out or FP4.empty(rows, cols, blk, x.device)
+    wbuf = _ws(ws, ft_quantize_workspace_bytes(), x.device) if amax is None else None
+    v = out.view()
+    check("ft_quantize", load().ft_quantize(
+        x.data_ptr(), rows, cols, x.stride(0), blk, _ptr(amax), ctypes.byref(v), _ptr(wbuf),
+        0 if wbuf is None else wbuf.numel(), _stream(stream)))
+    return out
+
+
+def ft_quantize_transpose(x: torch.Tensor, blk: int = BLK_16x16, amax: torch.Tensor | None = None,
+                          out_row: FP4 | None = None, out_col: FP4 | None = None,
+                          ws: Workspace | None = None, stream=None):
+    """Both layouts in one pass.  16x16: (codes packed along rows, the same
+    codes transposed) sharing one scale grid.  1x16: (Q(x), Q(x^T))."""
+    _bf16(x, "x")
+    rows, cols = x.shape
+    out_row = out_row or FP4.empty(rows, cols, blk, x.device)
+    if out_col is None:
+        if blk == BLK_16x16:
+            out_col = FP4.empty(cols, rows, blk, x.device, scales=out_row.scales, tscale=out_row.tscale)
+        else:
+            out_col = FP4.empty(cols, rows, blk, x.device)
+    wbuf = _ws(ws, ft_quantize_workspace_bytes(), x.device) if amax is None else None
+    vr, vc = out_row.view(), out_col.view()
+    check("ft_quantize_transpose", load().ft_quantize_transpose(
+        x.data_ptr(), rows, cols, x.stride(0), blk, _ptr(amax), ctypes.byref(vr), ctypes.byref(vc),
+        _ptr(wbuf), 0 if wbuf is None else wbuf.numel(), _stream(stream)))
+    return out_row, out_col
+
+
+@dataclass
+class Layer:
+    """One triple-branch linear: Q(W_res) in both code layouts (one scale
+    grid), the stabilizer factors U [K, r_s], V [N, r_s] and the adapter
+    A [K, r_l], B [N, r_l] (bf16), and the LoRA scale s."""
+    N: int
+    K: int
+    r_s: int
+    r_l: int
+    s: float
+    w_k: FP4
+    w_n: FP4
+    U: torch.Tensor | None
+    V: torch.Tensor | None
+    A: torch.Tensor | None
+    B: torch.Tensor | None
+
+    def view(self) -> FtLinear:
+        return FtLinear(self.N, self.K, self.r_s, self.r_l, self.s, self.w_k.view(), self.w_n.view(),
+                        _ptr(self.U), _ptr(self.V), _ptr(self.A), _ptr(self.B))
+
+
+def svd_split(W: torch.Tensor, r_s: int):
+    """Eq. 1 on the host side (untimed, once per layer): W ~ W_res + V U^T
+    with the top-r_s singular triplets, taken from the smaller Gram matrix in
+    float64 (eigenvectors of W^T W are the right singular vectors, those of
+    W W^T the left ones).  U = right vectors [K, r_s], V = W U [N, r_s], both
+    rounded to bf16, and W_res = W - V U^T from the rounded factors."""
+    Wd = W.to(torch.float64)
+    N, K = Wd.shape
+    if r_s == 0:
+        return None, None, W.to(torch.bfloat16).contiguous()
+    if K <= N:
+        evals, evecs = torch.linalg.eigh(Wd.T @ Wd)
+        vtop = evecs[:, torch.argsort(evals, descending=True)[:r_s]]
+    else:
+        evals, evecs = torch.linalg.eigh(Wd @ Wd.T)
+        order = torch.argsort(evals, descending=True)[:r_s]
+        sig = evals[order].clamp_min(0).sqrt()
+        vtop = (Wd.T @ evecs[:, order]) / torch.where(sig > 0, sig, torch.ones_like(sig))
+    U = vtop.to(torch.bfloat16).contiguous()
+    V = (Wd @ U.to(torch.float64)).to(torch.bfloat16).contiguous()
+    W_res = (Wd - V.to(torch.float64) @ U.to(torch.float64).T).to(torch.bfloat16).contiguous()
+    return U, V, W_res
+
+
+def prepare_layer(W: torch.Tensor | None = None, r_s: int = 0, A: torch.Tensor | None = None,
+                  B: torch.Tensor | None = None, s: float = 1.0, *, U=None, V=None, W_res=None,
+                  amax: torch.Tensor | None = None, ws: Workspace | None = None) -> Layer:
+    """Once-per-layer preparation: split W (or take a given U, V, W_res) and
+    quantize W_res with 16x16 blocks into both code layouts in one pass."""
+    if W_res is None:
+        U, V, W_res = svd_split(W, r_s)
+    _bf16(W_res, "W_res")
+    N, K = W_res.shape
+    r_s = 0 if U is None else U.shape[1]
+    r_l = 0 if A is None else A.shape[1]
+    w_k, w_n = ft_quantize_transpose(W_res.contiguous(), BLK_16x16, amax=amax, ws=ws)
+    return Layer(N, K, r_s, r_l, float(s), w_k, w_n, U, V,
+                 None if A is None else A.contiguous(), None if B is None else B.contiguous())
+
+
+def ft_linear_fwd(layer: Layer, X: torch.Tensor, amax_x: torch.Tensor | None = None,
+                  out_dtype: int = BF16, Y: torch.Tensor | None = None, P: torch.Tensor | None = None,
+                  ws: Workspace | None = None, stream=None):
+    """Y = Q(X) Q(W_res)^T + (X U) V^T + s (X A) B^T.  Returns (Y, P) where
+    P = [bf16(X U) | bf16(s X A)] is saved for the backward."""
+    _bf16(X, "X")
+    M = X.shape[0]
+    r = layer.r_s + layer.r_l
+    if Y is None:
+        Y = torch.empty(M, layer.N, device=X.device,
+                        dtype=torch.float32 if out_dtype == F32 else torch.bfloat16)
+    if P is None:
+        P = torch.empty(M, max(r, 0), device=X.device, dtype=torch.bfloat16)
+    wbuf = _ws(ws, ft_workspace_bytes(M, layer.N, layer.K, layer.r_s, layer.r_l), X.device)
+    v = layer.view()
+    check("ft_linear_fwd", load().ft_linear_fwd(
+        ctypes.byref(v), X.data_ptr(), M, _ptr(amax_x), Y.data_ptr(), out_dtype,
+        P.data_ptr() if r > 0 else None, wbuf.data_ptr(), wbuf.numel(), _stream(stream)))
+    return Y, P
+
+
+def ft_linear_bwd(layer: Layer, dY: torch.Tensor, X: torch.Tensor, P: torch.Tensor,
+                  amax_dy: torch.Tensor | None = None, out_dtype: int = BF16,
+                  dX: torch.Tensor | None = None, dA: torch.Tensor | None = None,
+                  dB: torch.Tensor | None = None, ws: Workspace | None = None, stream=None):
+    """dX = Q(dY) Q(W_res) + (dY V) U^T + s (dY B) A^T;  dB = dY^T P_lora,
+    dA = X^T Pg_lora (float32, overwritten).  Returns (dX, dA, dB)."""
+    _bf16(dY, "dY")
+    M = dY.shape[0]
+    r = layer.r_s + layer.r_l
+    if dX is None:
+        dX = torch.empty(M, layer.K, device=dY.device,
+                         dtype=torch.float32 if out_dtype == F32 else torch.bfloat16)
+    if layer.r_l > 0:
+        dA = dA if dA is not None else torch.empty(layer.K, layer.r_l, device=dY.device, dtype=torch.float32)
+        dB = dB if dB is not None else torch.empty(layer.N, layer.r_l, device=dY.device, dtype=torch.float32)
+    wbuf = _ws(ws, ft_workspace_bytes(M, layer.N, layer.K, layer.r_s, layer.r_l), dY.device)
+    v = layer.view()
+    check("ft_linear_bwd", load().ft_linear_bwd(
+        ctypes.byref(v), dY.data_ptr(), _ptr(X), P.data_ptr() if r > 0 else None, M, _ptr(amax_dy),
+        dX.data_ptr(), out_dtype, _ptr(dA), _ptr(dB), wbuf.data_ptr(), wbuf.numel(), _stream(stream)))
+    return dX, dA, dB
+
+
+def ft_device_error(stream=None) -> int:
+    """Reads and clears the device error word (0 = no kernel reported a
+    bounded wait that ran out)."""
+    code = ctypes.c_int(0)
+    load().ft_device_error(ctypes.byref(code), _stream(stream))
+    return code.value
+
+
+class timing:
+    """Per-kernel CUDA-event timing of the library's launches (measurement)."""
+
+    @staticmethod
+    def enable(on: bool = True) -> None:
+        check("ft_timing_enable", load().ft_timing_enable(1 if on else 0))
+
+    @staticmethod
+    def reset() -> None:
+        check("ft_timing_reset", load().ft_timing_reset())
+
+    @staticmethod
+    def read(kernel: str = "*"):
+        """(total milliseconds, launches) of one kernel since the last reset."""
+        ms = ctypes.c_double(0.0)
+        n = ctypes.c_int64(0)
+        check("ft_timing_read", load().ft_timing_read(kernel.encode(), ctypes.byref(ms), ctypes.byref(n)))
+        return ms.value, n.value

@@ -1,0 +1,682 @@
+// ft_api.cu -- the C ABI declared in include/ft.h.  Host-side argument
+// validation, workspace planning, TMA descriptor encoding and kernel
+// launches.  The kernels live in the included .cuh files (one translation
+// unit, so the device error word is a single symbol).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/ft.h"
+#include "ft_nvfp4.cuh"
+#include "ft_ptx.cuh"
+#include "k_gemm_fp4.cuh"
+#include "k_lora_grad.cuh"
+#include "k_qdown.cuh"
+#include "k_quant.cuh"
+
+namespace {
+
+using ft::gemm::Params;
+
+// ------------------------------------------------------------ device info
+struct DevInfo {
+    bool init = false;
+    bool ok = false;
+    int sms = 0;
+    bool attr_set = false;
+};
+DevInfo g_dev[64];
+std::mutex g_mu;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+ft_status device_info(DevInfo** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FT_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DevInfo& d = g_dev[dev];
+    if (!d.init) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return FT_ERR_CUDA;
+        d.ok = (major == 10 && minor == 0);
+        d.sms = sms;
+        d.init = true;
+    }
+    if (!d.ok) return FT_ERR_UNSUPPORTED;
+    if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return FT_ERR_CUDA;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    if (!d.attr_set) {
+        const int big = 227 * 1024;
+        if (cudaFuncSetAttribute(ft::gemm::k_gemm_fp4, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 big) != cudaSuccess ||
+            cudaFuncSetAttribute(ft::qdown::k_qdown, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)ft::qdown::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(ft::lgrad::k_lora_grad, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)ft::lgrad::smem_bytes(128)) != cudaSuccess)
+            return FT_ERR_CUDA;
+        d.attr_set = true;
+    }
+    *out = &d;
+    return FT_OK;
+}
+
+inline ft_status cuda_ok(cudaError_t e) { return e == cudaSuccess ? FT_OK : FT_ERR_CUDA; }
+inline ft_status last_launch() { return cuda_ok(cudaGetLastError()); }
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+inline int cdiv(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
+
+#define FT_TRY(expr)                 \
+    do {                             \
+        ft_status _s = (expr);       \
+        if (_s != FT_OK) return _s;  \
+    } while (0)
+
+// ------------------------------------------------------------ kernel timing
+// Optional measurement support: when enabled, every launch is bracketed by a
+// pair of CUDA events on its stream; ft_timing_read() adds up the elapsed
+// times per kernel.  Disabled by default (zero cost beyond a flag test).
+enum KernelId {
+    KID_AMAX = 0,
+    KID_QUANT_1X16,
+    KID_QUANT_TILE16,
+    KID_PACK_LT,
+    KID_QDOWN,
+    KID_LR_FINALIZE,
+    KID_GEMM,
+    KID_LORA_GRAD,
+    KID_LORA_REDUCE,
+    KID_COUNT
+};
+const char* const kKernelNames[KID_COUNT] = {
+    "k_amax_bf16", "k_quant_1x16", "k_quant_tile16", "k_pack_lt", "k_qdown",
+    "k_lowrank_finalize", "k_gemm_fp4", "k_lora_grad", "k_lora_grad_reduce"};
+
+struct TimingRec {
+    cudaEvent_t a, b;
+    int kid;
+};
+struct Timing {
+    bool on = false;
+    std::vector<TimingRec> recs;
+    std::vector<cudaEvent_t> pool;
+    double ms[KID_COUNT] = {};
+    int64_t launches[KID_COUNT] = {};
+    std::mutex mu;
+} g_timing;
+
+cudaEvent_t timing_event() {
+    if (!g_timing.pool.empty()) {
+        cudaEvent_t e = g_timing.pool.back();
+        g_timing.pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+// Brackets one launch: construct before it, call stop() after it.
+struct LaunchTimer {
+    int kid;
+    cudaStream_t st;
+    cudaEvent_t a = nullptr;
+    LaunchTimer(int k, cudaStream_t s) : kid(k), st(s) {
+        if (!g_timing.on) return;
+        std::lock_guard<std::mutex> lk(g_timing.mu);
+        a = timing_event();
+        cudaEventRecord(a, st);
+    }
+    void stop() {
+        if (!a) return;
+        std::lock_guard<std::mutex> lk(g_timing.mu);
+        cudaEvent_t b = timing_event();
+        cudaEventRecord(b, st);
+        g_timing.recs.push_back({a, b, kid});
+        a = nullptr;
+    }
+};
+
+// ------------------------------------------------------------ tensor maps
+ft_status encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                    uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                    CUtensorMapSwizzle swz) {
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_stride_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FT_OK : FT_ERR_CUDA;
+}
+
+// ------------------------------------------------------------ workspace
+constexpr int QD_MAX_SPLITS = 8;
+constexpr int LG_MAX_SPLITS = 16;
+
+struct WsPlan {
+    size_t amax, gact, codes, scales, lt, part, pg, lgpart, total;
+};
+
+WsPlan plan_ws(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t r_l) {
+    WsPlan w;
+    const int64_t C = std::max(N, K);
+    const int64_t r = r_s + r_l;
+    size_t o = 0;
+    w.amax = o;   o += 256;
+    w.gact = o;   o += 256;
+    w.codes = o;  o += up256((size_t)M * C / 2);
+    w.scales = o; o += up256((size_t)M * C / 16);
+    w.lt = o;     o += up256((size_t)128 * C * 2);
+    w.part = o;   o += up256((size_t)QD_MAX_SPLITS * M * r * 4);
+    w.pg = o;     o += up256((size_t)M * r * 2);
+    w.lgpart = o; o += up256((size_t)LG_MAX_SPLITS * (N + K) * r_l * 4);
+    w.total = o;
+    return w;
+}
+
+// ------------------------------------------------------------ pieces
+ft_status run_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, float* slot,
+                   const DevInfo* d, cudaStream_t st) {
+    FT_TRY(cuda_ok(cudaMemsetAsync(slot, 0, sizeof(float), st)));
+    const int64_t vecs = rows * (cols / 8);
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(vecs, 256), (int64_t)d->sms * 8));
+    {
+        LaunchTimer _lt(KID_AMAX, st);
+        ft::k_amax_bf16<<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(x), rows, cols, ld,
+                                              reinterpret_cast<unsigned int*>(slot));
+        _lt.stop();
+    }
+    return last_launch();
+}
+
+ft_status run_quant_1x16(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* amax,
+                         uint8_t* codes, uint8_t* scales, float* tscale, const DevInfo* d,
+                         cudaStream_t st) {
+    const int64_t blocks = rows * (cols / 16);
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(blocks, 256), (int64_t)d->sms * 16));
+    {
+        LaunchTimer _lt(KID_QUANT_1X16, st);
+        ft::k_quant_1x16<<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(x), rows, cols, ld, amax,
+                                               codes, scales, tscale);
+        _lt.stop();
+    }
+    return last_launch();
+}
+
+ft_status run_tile16(bool mode16x16, const void* x, int64_t rows, int64_t cols, int64_t ld,
+                     const float* amax, uint8_t* codes_row, uint8_t* scales_row, uint8_t* codes_col,
+                     uint8_t* scales_col, float* tscale, float* tscale2, cudaStream_t st) {
+    dim3 grid((unsigned)cdiv(cols / 16, 8), (unsigned)(rows / 16));
+    if (mode16x16)
+        {
+            LaunchTimer _lt(KID_QUANT_TILE16, st);
+            ft::k_quant_tile16<true><<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(x), rows, cols, ld,
+                                                           amax, codes_row, scales_row, codes_col,
+                                                           scales_col, tscale, tscale2);
+            _lt.stop();
+        }
+    else
+        {
+            LaunchTimer _lt(KID_QUANT_TILE16, st);
+            ft::k_quant_tile16<false><<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(x), rows, cols, ld,
+                                                            amax, codes_row, scales_row, codes_col,
+                                                            scales_col, tscale, tscale2);
+            _lt.stop();
+        }
+    return last_launch();
+}
+
+// Q(T) and P = [bf16(T L1) | bf16(s T L2)] in one pass over T [M, C].
+ft_status run_qdown(const void* T, int64_t M, int64_t C, const void* L1, int64_t r1, const void* L2,
+                    int64_t r2, float s, const float* amax, uint8_t* codes, uint8_t* scales,
+                    float* tscale, void* P, uint8_t* ws, const WsPlan& w, const DevInfo* d,
+                    cudaStream_t st) {
+    const int64_t r = r1 + r2;
+    if (r == 0) return run_quant_1x16(T, M, C, C, amax, codes, scales, tscale, d, st);
+    uint16_t* Lt = reinterpret_cast<uint16_t*>(ws + w.lt);
+    float* part = reinterpret_cast<float*>(ws + w.part);
+    {
+        const int grid = std::min(cdiv(128 * C, 256), d->sms * 8);
+        {
+            LaunchTimer _lt(KID_PACK_LT, st);
+            ft::k_pack_lt<<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(L1), (int)r1,
+                                                static_cast<const uint16_t*>(L2), (int)r2, (int)C, Lt);
+            _lt.stop();
+        }
+        FT_TRY(last_launch());
+    }
+    const int mt = cdiv(M, ft::qdown::BM);
+    int splits = std::max(1, std::min(QD_MAX_SPLITS, d->sms / std::max(1, mt)));
+    int cchunk = cdiv(C, (int64_t)splits * 64) * 64;
+    splits = cdiv(C, cchunk);
+    ft::qdown::Params p;
+    std::memset(&p, 0, sizeof(p));
+    FT_TRY(encode_2d(&p.mapT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, C, M, C * 2, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B));
+    FT_TRY(encode_2d(&p.mapLt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Lt, C, 128, C * 2, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B));
+    p.amax = amax;
+    p.tscale = tscale;
+    p.codes = codes;
+    p.scales = scales;
+    p.part = part;
+    p.M = (int)M;
+    p.C = (int)C;
+    p.r = (int)r;
+    p.cchunk = cchunk;
+    p.do_mma = 1;
+    {
+        LaunchTimer _lt(KID_QDOWN, st);
+        ft::qdown::k_qdown<<<dim3((unsigned)mt, (unsigned)splits), ft::qdown::NUM_THREADS,
+                             ft::qdown::SMEM_BYTES, st>>>(p);
+        _lt.stop();
+    }
+    FT_TRY(last_launch());
+    const int64_t tot = M * r;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(tot, 256), (int64_t)d->sms * 8));
+    {
+        LaunchTimer _lt(KID_LR_FINALIZE, st);
+        ft::k_lowrank_finalize<<<grid, 256, 0, st>>>(part, splits, (int)M, (int)r, (int)r1, s,
+                                                     static_cast<__nv_bfloat16*>(P));
+        _lt.stop();
+    }
+    return last_launch();
+}
+
+// out[M, Nout] = ga gb Q(A) Q(B)^T + P[:, :r1] L1^T + P[:, r1:] L2^T
+ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* ga, int64_t M,
+                   int64_t Kc, const uint8_t* b_codes, const uint8_t* grid_scales, const float* gb,
+                   int64_t Nout, bool sfb_trans, int64_t grid_rows, int64_t grid_cols,
+                   const void* P, const void* L1, int64_t r1, const void* L2, int64_t r2, void* out,
+                   ft_dtype ot, const DevInfo* d, cudaStream_t st) {
+    Params p;
+    std::memset(&p, 0, sizeof(p));
+    FT_TRY(encode_2d(&p.mapA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, Kc / 2, M, Kc / 2, 128, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B));
+    FT_TRY(encode_2d(&p.mapB, CU_TENSOR_MAP_DATA_TYPE_UINT8, b_codes, Kc / 2, Nout, Kc / 2, 128, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B));
+    FT_TRY(encode_2d(&p.mapSFA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_scales, Kc / 16, M, Kc / 16, 16, 128,
+                     CU_TENSOR_MAP_SWIZZLE_NONE));
+    // the 16x16 grid is [grid_rows, grid_cols] row-major
+    FT_TRY(encode_2d(&p.mapSFB, CU_TENSOR_MAP_DATA_TYPE_UINT8, grid_scales, grid_cols, grid_rows,
+                     grid_cols, 16, sfb_trans ? 16 : 8, CU_TENSOR_MAP_SWIZZLE_NONE));
+    const int64_t r = r1 + r2;
+    if (r > 0)
+        FT_TRY(encode_2d(&p.mapP, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P, r, M, r * 2, 64, 128,
+                         CU_TENSOR_MAP_SWIZZLE_128B));
+    if (r1 > 0)
+        FT_TRY(encode_2d(&p.mapL1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1, r1, Nout, r1 * 2, 64, 128,
+                         CU_TENSOR_MAP_SWIZZLE_128B));
+    if (r2 > 0)
+        FT_TRY(encode_2d(&p.mapL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2, r2, Nout, r2 * 2, 64, 128,
+                         CU_TENSOR_MAP_SWIZZLE_128B));
+    p.ga = ga;
+    p.gb = gb;
+    p.out = out;
+    p.out_f32 = (ot == FT_F32);
+    p.M = (int)M;
+    p.Nout = (int)Nout;
+    p.Kc = (int)Kc;
+    p.r1 = (int)r1;
+    p.r2 = (int)r2;
+    p.sfb_trans = sfb_trans ? 1 : 0;
+    int stages = ft::gemm::MAX_STAGES;
+    while (stages > 2 && ft::gemm::make_layout(stages, (int)r1, (int)r2).total > 227u * 1024u) --stages;
+    p.stages = stages;
+    const uint32_t smem = ft::gemm::make_layout(stages, (int)r1, (int)r2).total;
+    const int tiles = cdiv(M, ft::gemm::BM) * (int)(Nout / ft::gemm::BN);
+    const int grid = std::max(1, std::min(tiles, d->sms));
+    {
+        LaunchTimer _lt(KID_GEMM, st);
+        ft::gemm::k_gemm_fp4<<<grid, ft::gemm::NUM_THREADS, smem, st>>>(p);
+        _lt.stop();
+    }
+    return last_launch();
+}
+
+ft_status run_lora_grads(const void* dY, const void* X, const void* P, const void* Pg, int64_t M,
+                         int64_t N, int64_t K, int64_t r_s, int64_t r_l, float* dA, float* dB,
+                         uint8_t* ws, const WsPlan& w, const DevInfo* d, cudaStream_t st) {
+    const int64_t r = r_s + r_l;
+    ft::lgrad::Params p;
+    std::memset(&p, 0, sizeof(p));
+    FT_TRY(encode_2d(&p.mapT[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, N, M, N * 2, 64, 64,
+                     CU_TENSOR_MAP_SWIZZLE_128B));
+    FT_TRY(encode_2d(&p.mapT[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 64,
+                     CU_TENSOR_MAP_SWIZZLE_128B));
+    FT_TRY(encode_2d(&p.mapS[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P, r, M, r * 2, 64, 64,
+                     CU_TENSOR_MAP_SWIZZLE_128B));
+    FT_TRY(encode_2d(&p.mapS[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Pg, r, M, r * 2, 64, 64,
+                     CU_TENSOR_MAP_SWIZZLE_128B));
+    const int ctiles = (int)(N / ft::lgrad::BC + K / ft::lgrad::BC);
+    int splits = std::max(1, std::min(LG_MAX_SPLITS, d->sms / std::max(1, ctiles)));
+    int mrows = cdiv(M, (int64_t)splits * ft::lgrad::BMR) * ft::lgrad::BMR;
+    splits = std::max(1, cdiv(M, mrows));
+    float* partB = reinterpret_cast<float*>(ws + w.lgpart);
+    float* partA = partB + (size_t)splits * N * r_l;
+    p.part[0] = partB;
+    p.part[1] = partA;
+    p.C[0] = (int)N;
+    p.C[1] = (int)K;
+    p.M = (int)M;
+    p.r_s = (int)r_s;
+    p.r_l = (int)r_l;
+    p.n_pad = r_l <= 64 ? 64 : 128;
+    p.mrows = mrows;
+    dim3 grid((unsigned)(std::max(N, K) / ft::lgrad::BC), (unsigned)splits, 2);
+    {
+        LaunchTimer _lt(KID_LORA_GRAD, st);
+        ft::lgrad::k_lora_grad<<<grid, ft::lgrad::NUM_THREADS, ft::lgrad::smem_bytes(p.n_pad), st>>>(p);
+        _lt.stop();
+    }
+    FT_TRY(last_launch());
+    {
+        const int64_t n = N * r_l;
+        const int g = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(n, 256), (int64_t)d->sms * 4));
+        {
+            LaunchTimer _lt(KID_LORA_REDUCE, st);
+            ft::k_lora_grad_reduce<<<g, 256, 0, st>>>(partB, splits, n, dB);
+            _lt.stop();
+        }
+        FT_TRY(last_launch());
+    }
+    {
+        const int64_t n = K * r_l;
+        const int g = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(n, 256), (int64_t)d->sms * 4));
+        {
+            LaunchTimer _lt(KID_LORA_REDUCE, st);
+            ft::k_lora_grad_reduce<<<g, 256, 0, st>>>(partA, splits, n, dA);
+            _lt.stop();
+        }
+        FT_TRY(last_launch());
+    }
+    return FT_OK;
+}
+
+// ------------------------------------------------------------ validation
+ft_status check_fp4_view(const ft_fp4* v, int64_t rows, int64_t cols, ft_block blk) {
+    if (!v || !v->codes || !v->scales || !v->tscale) return FT_ERR_INVALID_ARG;
+    if (v->rows != rows || v->cols != cols || v->blk != blk) return FT_ERR_SHAPE;
+    if (!al16(v->codes) || !al16(v->scales) || (reinterpret_cast<uintptr_t>(v->tscale) & 3u))
+        return FT_ERR_ALIGN;
+    return FT_OK;
+}
+
+ft_status check_linear(const ft_linear* L) {
+    if (!L) return FT_ERR_INVALID_ARG;
+    if (L->N <= 0 || L->K <= 0 || L->r_s < 0 || L->r_l < 0) return FT_ERR_INVALID_ARG;
+    if (L->N % 256 || L->K % 256) return FT_ERR_SHAPE;
+    if (L->r_s % 16 || L->r_l % 16 || L->r_s + L->r_l > 128) return FT_ERR_SHAPE;
+    if (L->N > (1 << 20) || L->K > (1 << 20)) return FT_ERR_SHAPE;
+    FT_TRY(check_fp4_view(&L->w_k, L->N, L->K, FT_BLK_16x16));
+    if (!L->w_n.codes) return FT_ERR_INVALID_ARG;
+    if (L->w_n.rows != L->K || L->w_n.cols != L->N || L->w_n.blk != FT_BLK_16x16) return FT_ERR_SHAPE;
+    if (!al16(L->w_n.codes)) return FT_ERR_ALIGN;
+    if ((L->w_n.scales && L->w_n.scales != L->w_k.scales) ||
+        (L->w_n.tscale && L->w_n.tscale != L->w_k.tscale))
+        return FT_ERR_INVALID_ARG;
+    if (L->r_s > 0 && (!L->U || !L->V)) return FT_ERR_INVALID_ARG;
+    if (L->r_l > 0 && (!L->A || !L->B)) return FT_ERR_INVALID_ARG;
+    if ((L->U && !al16(L->U)) || (L->V && !al16(L->V)) || (L->A && !al16(L->A)) ||
+        (L->B && !al16(L->B)))
+        return FT_ERR_ALIGN;
+    return FT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ft_status_str(ft_status s) {
+    switch (s) {
+        case FT_OK: return "FT_OK";
+        case FT_ERR_INVALID_ARG: return "FT_ERR_INVALID_ARG";
+        case FT_ERR_SHAPE: return "FT_ERR_SHAPE";
+        case FT_ERR_ALIGN: return "FT_ERR_ALIGN";
+        case FT_ERR_CUDA: return "FT_ERR_CUDA";
+        case FT_ERR_TIMEOUT: return "FT_ERR_TIMEOUT";
+        case FT_ERR_WORKSPACE: return "FT_ERR_WORKSPACE";
+        case FT_ERR_UNSUPPORTED: return "FT_ERR_UNSUPPORTED";
+    }
+    return "FT_ERR_UNKNOWN";
+}
+
+size_t ft_quantize_workspace_bytes(void) { return 256; }
+
+size_t ft_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t r_l) {
+    if (M < 0 || N < 0 || K < 0 || r_s < 0 || r_l < 0) return 0;
+    return plan_ws(M, N, K, r_s, r_l).total;
+}
+
+ft_status ft_device_error(int* code, void* stream) {
+    if (!code) return FT_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int v = 0;
+    FT_TRY(cuda_ok(cudaMemcpyFromSymbolAsync(&v, ft::g_ft_error, sizeof(int), 0,
+                                             cudaMemcpyDeviceToHost, st)));
+    FT_TRY(cuda_ok(cudaStreamSynchronize(st)));
+    if (v) {
+        const int zero = 0;
+        FT_TRY(cuda_ok(cudaMemcpyToSymbolAsync(ft::g_ft_error, &zero, sizeof(int), 0,
+                                               cudaMemcpyHostToDevice, st)));
+        FT_TRY(cuda_ok(cudaStreamSynchronize(st)));
+    }
+    *code = v;
+    return v ? FT_ERR_TIMEOUT : FT_OK;
+}
+
+ft_status ft_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, ft_block blk,
+                      const float* amax, ft_fp4* out, void* ws, size_t ws_bytes, void* stream) {
+    if (!x || !out) return FT_ERR_INVALID_ARG;
+    if (blk != FT_BLK_1x16 && blk != FT_BLK_16x16) return FT_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 0 || ld < cols) return FT_ERR_INVALID_ARG;
+    if (cols % 16 || (blk == FT_BLK_16x16 && rows % 16)) return FT_ERR_SHAPE;
+    FT_TRY(check_fp4_view(out, rows, cols, blk));
+    if (!al16(x) || (ld % 8)) return FT_ERR_ALIGN;
+    if (!amax && (!ws || ws_bytes < ft_quantize_workspace_bytes())) return FT_ERR_WORKSPACE;
+    if (amax && (reinterpret_cast<uintptr_t>(amax) & 3u)) return FT_ERR_ALIGN;
+    if (rows == 0 || cols == 0) return FT_OK;
+    DevInfo* d;
+    FT_TRY(device_info(&d));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const float* a = amax;
+    if (!a) {
+        float* slot = static_cast<float*>(ws);
+        FT_TRY(run_amax(x, rows, cols, ld, slot, d, st));
+        a = slot;
+    }
+    if (blk == FT_BLK_1x16)
+        return run_quant_1x16(x, rows, cols, ld, a, out->codes, out->scales, out->tscale, d, st);
+    return run_tile16(true, x, rows, cols, ld, a, out->codes, out->scales, nullptr, nullptr,
+                      out->tscale, nullptr, st);
+}
+
+ft_status ft_quantize_transpose(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                ft_block blk, const float* amax, ft_fp4* out_row, ft_fp4* out_col,
+                                void* ws, size_t ws_bytes, void* stream) {
+    if (!x || !out_row || !out_col) return FT_ERR_INVALID_ARG;
+    if (blk != FT_BLK_1x16 && blk != FT_BLK_16x16) return FT_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 0 || ld < cols) return FT_ERR_INVALID_ARG;
+    if (rows % 16 || cols % 16) return FT_ERR_SHAPE;
+    FT_TRY(check_fp4_view(out_row, rows, cols, blk));
+    if (!out_col->codes) return FT_ERR_INVALID_ARG;
+    if (out_col->rows != cols || out_col->cols != rows || out_col->blk != blk) return FT_ERR_SHAPE;
+    if (!al16(out_col->codes)) return FT_ERR_ALIGN;
+    if (blk == FT_BLK_16x16) {
+        if ((out_col->scales && out_col->scales != out_row->scales) ||
+            (out_col->tscale && out_col->tscale != out_row->tscale))
+            return FT_ERR_INVALID_ARG;
+    } else {
+        if (!out_col->scales || !out_col->tscale) return FT_ERR_INVALID_ARG;
+        if (!al16(out_col->scales) || (reinterpret_cast<uintptr_t>(out_col->tscale) & 3u))
+            return FT_ERR_ALIGN;
+    }
+    if (!al16(x) || (ld % 8)) return FT_ERR_ALIGN;
+    if (!amax && (!ws || ws_bytes < ft_quantize_workspace_bytes())) return FT_ERR_WORKSPACE;
+    if (rows == 0 || cols == 0) return FT_OK;
+    DevInfo* d;
+    FT_TRY(device_info(&d));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const float* a = amax;
+    if (!a) {
+        float* slot = static_cast<float*>(ws);
+        FT_TRY(run_amax(x, rows, cols, ld, slot, d, st));
+        a = slot;
+    }
+    if (blk == FT_BLK_16x16)
+        return run_tile16(true, x, rows, cols, ld, a, out_row->codes, out_row->scales,
+                          out_col->codes, nullptr, out_row->tscale, nullptr, st);
+    return run_tile16(false, x, rows, cols, ld, a, out_row->codes, out_row->scales, out_col->codes,
+                      out_col->scales, out_row->tscale,
+                      out_col->tscale != out_row->tscale ? out_col->tscale : nullptr, st);
+}
+
+ft_status ft_linear_fwd(const ft_linear* L, const void* X, int64_t M, const float* amax_x, void* Y,
+                        ft_dtype yt, void* P_save, void* ws, size_t ws_bytes, void* stream) {
+    FT_TRY(check_linear(L));
+    if (M < 0) return FT_ERR_INVALID_ARG;
+    if (yt != FT_BF16 && yt != FT_F32) return FT_ERR_INVALID_ARG;
+    if (M > (1 << 24)) return FT_ERR_SHAPE;
+    const int64_t r = L->r_s + L->r_l;
+    if (M == 0) return FT_OK;
+    if (!X || !Y || (r > 0 && !P_save)) return FT_ERR_INVALID_ARG;
+    if (!al16(X) || !al16(Y) || (P_save && !al16(P_save))) return FT_ERR_ALIGN;
+    const WsPlan w = plan_ws(M, L->N, L->K, L->r_s, L->r_l);
+    if (!ws || ws_bytes < w.total || !al16(ws)) return FT_ERR_WORKSPACE;
+    DevInfo* d;
+    FT_TRY(device_info(&d));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    float* g_x = reinterpret_cast<float*>(wsb + w.gact);
+    const float* a = amax_x;
+    if (!a) {
+        FT_TRY(run_amax(X, M, L->K, L->K, reinterpret_cast<float*>(wsb + w.amax), d, st));
+        a = reinterpret_cast<float*>(wsb + w.amax);
+    }
+    uint8_t* codes = wsb + w.codes;
+    uint8_t* scales = wsb + w.scales;
+    FT_TRY(run_qdown(X, M, L->K, L->U, L->r_s, L->A, L->r_l, L->s, a, codes, scales, g_x, P_save,
+                     wsb, w, d, st));
+    return run_gemm(codes, scales, g_x, M, L->K, L->w_k.codes, L->w_k.scales, L->w_k.tscale, L->N,
+                    false, L->N / 16, L->K / 16, P_save, L->V, L->r_s, L->B, L->r_l, Y, yt, d, st);
+}
+
+ft_status ft_linear_bwd(const ft_linear* L, const void* dY, const void* X, const void* P_save,
+                        int64_t M, const float* amax_dy, void* dX, ft_dtype xt, float* dA,
+                        float* dB, void* ws, size_t ws_bytes, void* stream) {
+    FT_TRY(check_linear(L));
+    if (M < 0) return FT_ERR_INVALID_ARG;
+    if (xt != FT_BF16 && xt != FT_F32) return FT_ERR_INVALID_ARG;
+    if (M > (1 << 24)) return FT_ERR_SHAPE;
+    const int64_t r = L->r_s + L->r_l;
+    if (L->r_l > 0 && (!dA || !dB)) return FT_ERR_INVALID_ARG;
+    if ((dA && !al16(dA)) || (dB && !al16(dB))) return FT_ERR_ALIGN;
+    if (M == 0) {
+        // no tokens: dX is empty and the adapter gradients are exactly zero
+        if (L->r_l > 0) {
+            DevInfo* d0;
+            FT_TRY(device_info(&d0));
+            cudaStream_t st0 = static_cast<cudaStream_t>(stream);
+            FT_TRY(cuda_ok(cudaMemsetAsync(dA, 0, (size_t)L->K * L->r_l * 4, st0)));
+            FT_TRY(cuda_ok(cudaMemsetAsync(dB, 0, (size_t)L->N * L->r_l * 4, st0)));
+        }
+        return FT_OK;
+    }
+    if (!dY || !dX || (r > 0 && !P_save) || (L->r_l > 0 && !X)) return FT_ERR_INVALID_ARG;
+    if (!al16(dY) || !al16(dX) || (X && !al16(X)) || (P_save && !al16(P_save))) return FT_ERR_ALIGN;
+    const WsPlan w = plan_ws(M, L->N, L->K, L->r_s, L->r_l);
+    if (!ws || ws_bytes < w.total || !al16(ws)) return FT_ERR_WORKSPACE;
+    DevInfo* d;
+    FT_TRY(device_info(&d));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    float* g_dy = reinterpret_cast<float*>(wsb + w.gact);
+    const float* a = amax_dy;
+    if (!a) {
+        FT_TRY(run_amax(dY, M, L->N, L->N, reinterpret_cast<float*>(wsb + w.amax), d, st));
+        a = reinterpret_cast<float*>(wsb + w.amax);
+    }
+    uint8_t* codes = wsb + w.codes;
+    uint8_t* scales = wsb + w.scales;
+    void* Pg = wsb + w.pg;
+    FT_TRY(run_qdown(dY, M, L->N, L->V, L->r_s, L->B, L->r_l, L->s, a, codes, scales, g_dy, Pg, wsb,
+                     w, d, st));
+    FT_TRY(run_gemm(codes, scales, g_dy, M, L->N, L->w_n.codes, L->w_k.scales, L->w_k.tscale, L->K,
+                    true, L->N / 16, L->K / 16, Pg, L->U, L->r_s, L->A, L->r_l, dX, xt, d, st));
+    if (L->r_l > 0)
+        FT_TRY(run_lora_grads(dY, X, P_save, Pg, M, L->N, L->K, L->r_s, L->r_l, dA, dB, wsb, w, d, st));
+    return FT_OK;
+}
+
+ft_status ft_timing_enable(int on) {
+    std::lock_guard<std::mutex> lk(g_timing.mu);
+    g_timing.on = on != 0;
+    return FT_OK;
+}
+
+ft_status ft_timing_read(const char* kernel, double* total_ms, int64_t* launches) {
+    if (!kernel || !total_ms || !launches) return FT_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_timing.mu);
+    for (auto& r : g_timing.recs) {
+        float ms = 0.0f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess)
+            return FT_ERR_CUDA;
+        g_timing.ms[r.kid] += ms;
+        g_timing.launches[r.kid] += 1;
+        g_timing.pool.push_back(r.a);
+        g_timing.pool.push_back(r.b);
+    }
+    g_timing.recs.clear();
+    for (int k = 0; k < KID_COUNT; ++k)
+        if (std::strcmp(kernel, kKernelNames[k]) == 0) {
+            *total_ms = g_timing.ms[k];
+            *launches = g_timing.launches[k];
+            return FT_OK;
+        }
+    if (std::strcmp(kernel, "*") == 0) {
+        double t = 0.0;
+        int64_t n = 0;
+        for (int k = 0; k < KID_COUNT; ++k) {
+            t += g_timing.ms[k];
+            n += g_timing.launches[k];
+        }
+        *total_ms = t;
+        *launches = n;
+        return FT_OK;
+    }
+    return FT_ERR_INVALID_ARG;
+}
+
+ft_status ft_timing_reset(void) {
+    std::lock_guard<std::mutex> lk(g_timing.mu);
+    for (auto& r : g_timing.recs) {
+        cudaEventSynchronize(r.b);
+        g_timing.pool.push_back(r.a);
+        g_timing.pool.push_back(r.b);
+    }
+    g_timing.recs.clear();
+    for (int k = 0; k < KID_COUNT; ++k) {
+        g_timing.ms[k] = 0.0;
+        g_timing.launches[k] = 0;
+    }
+    return FT_OK;
+}
+
+}  // extern "C"

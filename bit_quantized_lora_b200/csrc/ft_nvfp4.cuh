@@ -1,0 +1,150 @@
+// ft_nvfp4.cuh -- the NVFP4 block encoder used by every quantizing kernel.
+//
+// Encoding (FourTune page, section 3.2 block quantization; the page names
+// NVFP4, whose elements are E2M1 with one E4M3 scale per block and an FP32
+// tensor scale):
+//   g   = amax_tensor / 2688              (1 when amax_tensor == 0)
+//   sd  = E4M3_rne_satfinite(amax_block / (6 g))
+//   q   = x / (sd g)                      (IEEE single, round to nearest even)
+//   code= E2M1_rne_satfinite(q), sign of x kept; 0 when sd == 0
+// Every FP32 step is an explicitly rounded intrinsic (no contraction), so the
+// codes and scales are bit-identical to a scalar IEEE implementation.
+#pragma once
+
+#include "ft_ptx.cuh"
+
+namespace ft {
+
+struct QTensor {
+    float g;      // decode tensor scale
+    float six_g;  // RN(6 g)
+};
+
+__device__ __forceinline__ QTensor make_qtensor(float amax) {
+    QTensor t;
+    t.g = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+    t.six_g = __fmul_rn(6.0f, t.g);
+    return t;
+}
+
+// RN(v) to E4M3 with saturation to 448; returns the byte.
+__device__ __forceinline__ uint32_t e4m3_encode(float v) {
+    uint16_t out;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(0.0f), "f"(v));
+    return out & 0xFFu;
+}
+
+// Exact value of an E4M3 byte.
+__device__ __forceinline__ float e4m3_decode(uint32_t b) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)b));
+    return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+// Eight non-negative values -> eight E2M1 magnitude codes (RNE, saturating
+// to 6), value i in nibble i.  In cvt...e2m1x2 the second source lands in the
+// low nibble.
+__device__ __forceinline__ uint32_t e2m1x8_encode(const float (&a)[8]) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(a[0]), "f"(a[1]), "f"(a[2]), "f"(a[3]), "f"(a[4]), "f"(a[5]), "f"(a[6]),
+          "f"(a[7]));
+    return out;
+}
+
+// RN(x / d) for d a normal float in [2^-60, 2^60] and x non-negative:
+// y = RN(1/d) is within half an ulp of 1/d and q0 = RN(x y) is faithful, so
+// one correction step with the exact remainder x - q0 d (an FMA) returns the
+// correctly rounded quotient (Markstein's theorem; see Muller et al.,
+// "Handbook of Floating-Point Arithmetic", division by Newton-Raphson).  The
+// range limit keeps the remainder clear of the subnormal range whenever the
+// quotient is large enough to matter for E2M1 (>= 2^-3).
+__device__ __forceinline__ float div_by_recip(float x, float d, float y) {
+    float q = __fmul_rn(x, y);
+    float r = __fmaf_rn(-q, d, x);
+    return __fmaf_rn(r, y, q);
+}
+
+// bf16 bit pattern (low 16 bits of w) -> |value| as float
+__device__ __forceinline__ float bf16_lo_abs(uint32_t w) { return __uint_as_float((w & 0x7FFFu) << 16); }
+__device__ __forceinline__ float bf16_hi_abs(uint32_t w) { return __uint_as_float(w & 0x7FFF0000u); }
+
+// Max of |x| over 8 packed bf16 pairs, as the bf16 magnitude bits << 16.
+__device__ __forceinline__ uint32_t amax_bits_16(const uint32_t (&w)[8]) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
+    m = max(m & 0xFFFFu, m >> 16);
+    return m << 16;
+}
+
+// Sign bits of 8 bf16 values (w[0..3]) placed at bit 3 of each nibble.
+__device__ __forceinline__ uint32_t sign_nibbles_8(uint32_t w0, uint32_t w1, uint32_t w2,
+                                                   uint32_t w3) {
+    uint32_t s = 0;
+    s |= (w0 >> 15) & 1u;
+    s |= ((w0 >> 31) & 1u) << 4;
+    s |= ((w1 >> 15) & 1u) << 8;
+    s |= ((w1 >> 31) & 1u) << 12;
+    s |= ((w2 >> 15) & 1u) << 16;
+    s |= ((w2 >> 31) & 1u) << 20;
+    s |= ((w3 >> 15) & 1u) << 24;
+    s |= ((w3 >> 31) & 1u) << 28;
+    return s << 3;
+}
+
+// Codes of 8 elements (w0..w3 = 4 bf16 pairs) for divisor d, as 8 nibbles.
+__device__ __forceinline__ uint32_t encode8(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3,
+                                            float d, float y, bool fast) {
+    float a[8] = {bf16_lo_abs(w0), bf16_hi_abs(w0), bf16_lo_abs(w1), bf16_hi_abs(w1),
+                  bf16_lo_abs(w2), bf16_hi_abs(w2), bf16_lo_abs(w3), bf16_hi_abs(w3)};
+    float q[8];
+    if (fast) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = div_by_recip(a[i], d, y);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(a[i], d);
+    }
+    return e2m1x8_encode(q) | sign_nibbles_8(w0, w1, w2, w3);
+}
+
+// Per-block divisor setup.  Returns false when the block is all zero scale
+// (sd == 0: every code is 0).
+struct BlockDiv {
+    float d, y;
+    bool fast;
+};
+
+__device__ __forceinline__ bool block_divisor(float amax_b, const QTensor& t, uint32_t& sbyte,
+                                              BlockDiv& bd) {
+    float sf = __fdiv_rn(amax_b, t.six_g);
+    sbyte = e4m3_encode(sf);
+    float sd = e4m3_decode(sbyte);
+    if (sd == 0.0f) return false;
+    bd.d = __fmul_rn(sd, t.g);
+    bd.fast = (bd.d >= 0x1p-60f) && (bd.d <= 0x1p60f);
+    bd.y = bd.fast ? __frcp_rn(bd.d) : 0.0f;
+    return true;
+}
+
+// Quantize one 1x16 block held as 8 bf16 pairs.  Returns 16 codes packed in
+// 8 bytes (element 0 in the low nibble of byte 0) and the scale byte.
+__device__ __forceinline__ uint2 quant_block16(const uint32_t (&w)[8], const QTensor& t,
+                                               uint32_t& sbyte) {
+    float amax_b = __uint_as_float(amax_bits_16(w));
+    BlockDiv bd;
+    if (!block_divisor(amax_b, t, sbyte, bd)) return make_uint2(0u, 0u);
+    uint2 r;
+    r.x = encode8(w[0], w[1], w[2], w[3], bd.d, bd.y, bd.fast);
+    r.y = encode8(w[4], w[5], w[6], w[7], bd.d, bd.y, bd.fast);
+    return r;
+}
+
+}  // namespace ft

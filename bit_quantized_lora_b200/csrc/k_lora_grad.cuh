@@ -1,0 +1,177 @@
+// k_lora_grad.cuh -- adapter weight gradients (FourTune page, section 3.2:
+// weight gradients only for the trainable branch, dB = (X A)^T G and
+// dA = X^T (G B^T) in the page's notation).  With the saved, already scaled
+// P_lora = bf16(s X A) and Pg_lora = bf16(s dY B):
+//     dB[n, j] = sum_m dY[m, n] P_lora[m, j]        (z = 0)
+//     dA[k, j] = sum_m X[m, k]  Pg_lora[m, j]       (z = 1)
+// Both are out[c, j] = sum_m T[m, c] S[m, j]: a reduction over the token
+// dimension, HBM-bound on reading T.  Each CTA takes 128 columns c and a
+// slice of m, runs tcgen05 kind::f16 with both operands MN-major straight
+// from the TMA tiles (T^T as A, S as B), and writes an FP32 partial;
+// k_lora_grad_reduce adds the slices in a fixed order.
+#pragma once
+
+#include <cuda.h>
+
+#include "ft_ptx.cuh"
+
+namespace ft {
+namespace lgrad {
+
+constexpr int BC = 128;    // output rows (columns of T) per CTA
+constexpr int BMR = 64;    // token rows per stage
+constexpr int STAGES = 4;
+constexpr int NUM_THREADS = 192;
+constexpr int T_BYTES = BMR * BC * 2;    // 16 KiB: two 64-column boxes
+constexpr int S_CHUNK = BMR * 64 * 2;    // 8 KiB: one 64-column box
+constexpr uint32_t TMEM_COLS = 128;
+
+struct Params {
+    CUtensorMap mapT[2];  // bf16 [M, C_z], box {64, 64}, 128 B swizzle
+    CUtensorMap mapS[2];  // bf16 [M, r],   box {64, 64}, 128 B swizzle
+    float* part[2];       // [splits, C_z, r_l]
+    int C[2];
+    int M, r_s, r_l, n_pad, mrows;
+};
+
+constexpr uint32_t smem_bytes(int n_pad) {
+    return STAGES * (T_BYTES + (n_pad / 64) * S_CHUNK) + 256 + 1024;
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1) k_lora_grad(const __grid_constant__ Params p) {
+    const int z = blockIdx.z;
+    const int c0 = blockIdx.x * BC;
+    if (c0 >= p.C[z]) return;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = smem_u32(smem_raw);
+    const uint32_t base = (raw_base + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (base - raw_base);
+    const int nsc = p.n_pad / 64;
+    const uint32_t s_bytes = nsc * S_CHUNK;
+    const uint32_t off_t = 0, off_s = STAGES * T_BYTES, off_bar = STAGES * (T_BYTES + s_bytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + off_bar);
+    uint64_t* empty = full + STAGES;
+    uint64_t* accfull = empty + STAGES;
+    uint64_t* drain = accfull + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = warp_id(), lane = lane_id();
+    const int split = blockIdx.y;
+    const int mbeg = split * p.mrows;
+    const int mend = min(p.M, mbeg + p.mrows);
+    const int nst = mend > mbeg ? (mend - mbeg + BMR - 1) / BMR : 0;
+    const CUtensorMap* mapT = &p.mapT[z];
+    const CUtensorMap* mapS = &p.mapS[z];
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        mbar_init(accfull, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int st = 0;
+            for (; st < nst; ++st) {
+                const int s = st % STAGES;
+                const uint32_t ph = (st / STAGES) & 1;
+                if (!mbar_wait(&empty[s], ph ^ 1, ERR_WAIT_EMPTY, abort_flag)) break;
+                const int m = mbeg + st * BMR;
+                mbar_arrive_expect_tx(&full[s], T_BYTES + s_bytes);
+                uint8_t* tdst = smem + off_t + s * T_BYTES;
+                tma_load_2d(tdst, mapT, &full[s], c0, m);
+                tma_load_2d(tdst + T_BYTES / 2, mapT, &full[s], c0 + 64, m);
+                uint8_t* sdst = smem + off_s + s * s_bytes;
+                for (int h = 0; h < nsc; ++h)
+                    tma_load_2d(sdst + h * S_CHUNK, mapS, &full[s], p.r_s + 64 * h, m);
+            }
+            if (st < nst) {
+                for (int d = 0; d < STAGES && d < st; ++d) {
+                    int j = st - 1 - d;
+                    volatile int no_abort = 0;
+                    mbar_wait(&full[j % STAGES], (j / STAGES) & 1, ERR_WAIT_DRAIN, &no_abort);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // A = T^T (M = 128 columns c, MN-major: two 64-wide swizzle atoms
+            // 8 KiB apart), B = S (N = n_pad, MN-major), K = 16 token rows.
+            const uint32_t idesc = idesc_bf16(BC, p.n_pad, 1, 1);
+            bool ok = true;
+            for (int st = 0; st < nst; ++st) {
+                const int s = st % STAGES;
+                const uint32_t ph = (st / STAGES) & 1;
+                if (!mbar_wait(&full[s], ph, ERR_WAIT_FULL, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a = base + off_t + s * T_BYTES;
+                const uint32_t b = base + off_s + s * s_bytes;
+#pragma unroll
+                for (int k = 0; k < BMR / 16; ++k)
+                    umma_bf16(tmem, smem_desc(a + 2048 * k, T_BYTES / 2, 1024, SWZ_128B),
+                              smem_desc(b + 2048 * k, S_CHUNK, 1024, SWZ_128B), idesc, (st | k) != 0);
+                tc_commit(&empty[s]);
+            }
+            if (ok && nst > 0) tc_commit(accfull);
+            tc_commit(drain);
+            volatile int no_abort = 0;
+            mbar_wait(drain, 0, ERR_WAIT_DRAIN, &no_abort);
+        }
+        __syncwarp();
+    } else {
+        const int sp = warp & 3;
+        const int c = c0 + 32 * sp + lane;
+        float* out = p.part[z] + ((int64_t)split * p.C[z] + c) * p.r_l;
+        bool have = nst > 0 && mbar_wait(accfull, 0, ERR_WAIT_ACC_FULL, abort_flag);
+        if (have) tc_fence_after();
+        const uint32_t lane_addr = (uint32_t)(32 * sp) << 16;
+        for (int j0 = 0; j0 < p.r_l; j0 += 32) {
+            uint32_t v[32];
+            if (have) {
+                tmem_ld_32x32b_x32(tmem + lane_addr + j0, v);
+                tmem_ld_wait();
+            }
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+                if (j0 + k < p.r_l) out[j0 + k] = have ? __uint_as_float(v[k]) : 0.0f;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+}  // namespace lgrad
+
+// out[c, j] = sum over splits of part[split, c, j], in increasing split order.
+__global__ void __launch_bounds__(256) k_lora_grad_reduce(const float* __restrict__ part, int splits,
+                                                          int64_t n, float* __restrict__ out) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        float acc = 0.0f;
+        for (int k = 0; k < splits; ++k) acc = __fadd_rn(acc, part[(int64_t)k * n + i]);
+        out[i] = acc;
+    }
+}
+
+}  // namespace ft

@@ -1,0 +1,191 @@
+// k_quant.cuh -- HBM-bound NVFP4 kernels: tensor amax, 1x16 quantization of
+// activations / gradients, and the tile kernel that emits both layouts in one
+// pass (16x16 weight blocks: codes packed along rows and along columns with
+// one scale grid; 1x16: Q(X) and Q(X^T) sharing the tensor scale).
+//
+// FourTune page, section 3.2 (block-wise 16x16 weight quantization so the
+// transposed weight needs no re-quantization) and section 4.3, Table 5 (1x16
+// group-wise granularity).
+#pragma once
+
+#include "ft_nvfp4.cuh"
+
+namespace ft {
+
+// ------------------------------------------------------------------ amax
+// max|x| over a bf16 matrix (cols % 8 == 0, rows 16-byte aligned).  Each
+// block reduces its share and folds it into *out with an integer atomicMax on
+// the float bits (non-negative floats order like their bit patterns), so the
+// result is exact and independent of scheduling.  *out must be 0 on entry.
+__global__ void __launch_bounds__(256) k_amax_bf16(const uint16_t* __restrict__ x, int64_t rows,
+                                                   int64_t cols, int64_t ld,
+                                                   unsigned int* __restrict__ out) {
+    const int64_t vec_per_row = cols / 8;
+    const int64_t total = rows * vec_per_row;
+    uint32_t m = 0;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        int64_t r = i / vec_per_row, c = i - r * vec_per_row;
+        uint4 v = ld_nc_v4(x + r * ld + c * 8);
+        m = __vmaxu2(m, v.x & 0x7FFF7FFFu);
+        m = __vmaxu2(m, v.y & 0x7FFF7FFFu);
+        m = __vmaxu2(m, v.z & 0x7FFF7FFFu);
+        m = __vmaxu2(m, v.w & 0x7FFF7FFFu);
+    }
+    m = max(m & 0xFFFFu, m >> 16);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    __shared__ uint32_t red[8];
+    if (lane_id() == 0) red[warp_id()] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t b = 0;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) b = max(b, red[w]);
+        if (b) atomicMax(out, b << 16);
+    }
+}
+
+// ------------------------------------------------------- 1x16 row-wise
+// One thread per 16-element block of a row.  Loads are two 16-byte vectors,
+// stores are 8 bytes of codes and one scale byte; consecutive threads touch
+// consecutive blocks, so every access is coalesced.
+__global__ void __launch_bounds__(256) k_quant_1x16(const uint16_t* __restrict__ x, int64_t rows,
+                                                    int64_t cols, int64_t ld,
+                                                    const float* __restrict__ amax,
+                                                    uint8_t* __restrict__ codes,
+                                                    uint8_t* __restrict__ scales,
+                                                    float* __restrict__ tscale) {
+    const QTensor t = make_qtensor(*amax);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *tscale = t.g;
+    const int64_t nb = cols / 16;
+    const int64_t total = rows * nb;
+    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < total;
+         b += (int64_t)gridDim.x * blockDim.x) {
+        int64_t r = b / nb, c = b - r * nb;
+        const uint16_t* p = x + r * ld + c * 16;
+        uint4 v0 = ld_nc_v4(p), v1 = ld_nc_v4(p + 8);
+        uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        uint32_t s;
+        uint2 q = quant_block16(w, t, s);
+        *reinterpret_cast<uint2*>(codes + r * (cols / 2) + c * 8) = q;
+        scales[r * nb + c] = (uint8_t)s;
+    }
+}
+
+// ---------------------------------------------------- 16x16 tile kernel
+// One warp per 16x16 tile.  Lane l holds row (l & 15), columns 8*(l >> 4)
+// .. +7 of the tile (one 16-byte load).
+//
+// kMode16x16 = true : one scale per tile (weights).  Writes codes packed
+//   along rows (codes_row, [rows, cols/2]) and, if codes_col != nullptr,
+//   the same codes packed along columns ([cols, rows/2]); scale grid
+//   [rows/16, cols/16].
+// kMode16x16 = false: 1x16 blocks (activations).  Row blocks -> codes_row /
+//   scales_row ([rows, cols/16]); column blocks (16 consecutive rows of one
+//   column) -> codes_col / scales_col ([cols, rows/16]); both share g.
+template <bool kMode16x16>
+__global__ void __launch_bounds__(256) k_quant_tile16(
+    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+    const float* __restrict__ amax, uint8_t* __restrict__ codes_row,
+    uint8_t* __restrict__ scales_row, uint8_t* __restrict__ codes_col,
+    uint8_t* __restrict__ scales_col, float* __restrict__ tscale, float* __restrict__ tscale2) {
+    __shared__ uint32_t tile[8][16][9];  // per warp: 16 rows x 8 bf16 pairs (+1 pad)
+    const QTensor t = make_qtensor(*amax);
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+        *tscale = t.g;
+        if (tscale2) *tscale2 = t.g;
+    }
+    const int w = warp_id(), l = lane_id();
+    const int64_t tiles_c = cols / 16;
+    const int64_t tr = blockIdx.y;                            // tile row
+    const int64_t tc = (int64_t)blockIdx.x * 8 + w;           // tile column
+    if (tc >= tiles_c) return;
+    const int r = l & 15, h = l >> 4;
+    const int64_t row = tr * 16 + r;
+    const int64_t col = tc * 16 + h * 8;
+    uint4 v = ld_nc_v4(x + row * ld + col);
+    uint32_t mine[4] = {v.x, v.y, v.z, v.w};
+
+    if (kMode16x16) {
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m = __vmaxu2(m, mine[i] & 0x7FFF7FFFu);
+        m = max(m & 0xFFFFu, m >> 16);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        float amax_b = __uint_as_float(m << 16);
+        uint32_t s;
+        BlockDiv bd;
+        uint32_t code8 = 0;
+        if (block_divisor(amax_b, t, s, bd))
+            code8 = encode8(mine[0], mine[1], mine[2], mine[3], bd.d, bd.y, bd.fast);
+        *reinterpret_cast<uint32_t*>(codes_row + row * (cols / 2) + col / 2) = code8;
+        if (l == 0) scales_row[tr * tiles_c + tc] = (uint8_t)s;
+        if (codes_col) {
+            // transpose the 16x16 nibble tile through shared memory
+            uint32_t* tw = &tile[w][0][0];
+            tw[r * 9 + h] = code8;  // row r, columns 8h..8h+7 (nibbles)
+            __syncwarp();
+            // lane l: column c = l & 15, rows 8*(l>>4) .. +7
+            const int c = l & 15, rh = l >> 4;
+            uint32_t out = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                int rr = rh * 8 + i;
+                uint32_t word = tw[rr * 9 + (c >> 3)];
+                uint32_t nib = (word >> (4 * (c & 7))) & 0xFu;
+                out |= nib << (4 * i);
+            }
+            *reinterpret_cast<uint32_t*>(codes_col + (tc * 16 + c) * (rows / 2) + tr * 8 + rh * 4) =
+                out;
+        }
+    } else {
+        // row blocks: lanes r and r+16 hold the two halves of row r
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m = __vmaxu2(m, mine[i] & 0x7FFF7FFFu);
+        m = max(m & 0xFFFFu, m >> 16);
+        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 16));
+        {
+            float amax_b = __uint_as_float(m << 16);
+            uint32_t s;
+            BlockDiv bd;
+            uint32_t code8 = 0;
+            if (block_divisor(amax_b, t, s, bd))
+                code8 = encode8(mine[0], mine[1], mine[2], mine[3], bd.d, bd.y, bd.fast);
+            *reinterpret_cast<uint32_t*>(codes_row + row * (cols / 2) + col / 2) = code8;
+            if (h == 0) scales_row[row * tiles_c + tc] = (uint8_t)s;
+        }
+        // column blocks: gather column c (rows 8h'..8h'+7) through shared memory
+        uint32_t* tw = &tile[w][0][0];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tw[r * 9 + h * 4 + i] = mine[i];
+        __syncwarp();
+        const int c = l & 15, rh = l >> 4;
+        uint32_t cw[4];  // 8 bf16 of column c, rows rh*8 .. +7, packed in pairs
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            int r0 = rh * 8 + 2 * i;
+            uint32_t a = tw[r0 * 9 + (c >> 1)];
+            uint32_t b = tw[(r0 + 1) * 9 + (c >> 1)];
+            uint32_t ea = (c & 1) ? (a >> 16) : (a & 0xFFFFu);
+            uint32_t eb = (c & 1) ? (b >> 16) : (b & 0xFFFFu);
+            cw[i] = ea | (eb << 16);
+        }
+        uint32_t mc = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mc = __vmaxu2(mc, cw[i] & 0x7FFF7FFFu);
+        mc = max(mc & 0xFFFFu, mc >> 16);
+        mc = max(mc, __shfl_xor_sync(0xFFFFFFFFu, mc, 16));
+        float amax_c = __uint_as_float(mc << 16);
+        uint32_t s;
+        BlockDiv bd;
+        uint32_t code8 = 0;
+        if (block_divisor(amax_c, t, s, bd)) code8 = encode8(cw[0], cw[1], cw[2], cw[3], bd.d, bd.y, bd.fast);
+        const int64_t ccol = tc * 16 + c;
+        *reinterpret_cast<uint32_t*>(codes_col + ccol * (rows / 2) + tr * 8 + rh * 4) = code8;
+        if (rh == 0) scales_col[ccol * (rows / 16) + tr] = (uint8_t)s;
+    }
+}
+
+}  // namespace ft

@@ -1,0 +1,187 @@
+/*
+ * ft.h -- C ABI of the B200 (sm_100a) W4A4G4 triple-branch linear layer.
+ *
+ * The method is FourTune ("FourTune: Towards Fully 4-Bit Efficient
+ * Post-Training for Diffusion Models"): every linear layer of a diffusion
+ * transformer is split into three branches that read the same input and whose
+ * outputs are summed (section 3.1, Eq. 2):
+ *
+ *     Y  = GEMM4(Q(X), Q(W_res))  +  (X U) V^T  +  s (X A) B^T
+ *          frozen 4-bit backbone     frozen        trainable LoRA
+ *                                    stabilizer
+ *
+ * and the backward pass propagates through all three (section 3.2, Eq. 3):
+ *
+ *     dX = GEMM4(Q(dY), Q(W_res)^T) + (dY V) U^T + s (dY B) A^T
+ *     dB = s dY^T (X A)          dA = s X^T (dY B)
+ *
+ * Notation (PyTorch convention, weights stored [out, in]):
+ *   X  [M, K] bf16      W_res [N, K] (the SVD residual of the weight, Eq. 1)
+ *   U  [K, r_s] bf16    V [N, r_s] bf16   (V U^T = the top-r_s SVD part of W)
+ *   A  [K, r_l] bf16    B [N, r_l] bf16   (the adapter; s its scale)
+ *
+ * Q() is NVFP4 block quantization: E2M1 4-bit codes, one E4M3 scale per
+ * block, one FP32 tensor scale g.  Activations and gradients use 1x16 blocks
+ * along the contiguous axis; weights use 16x16 blocks so that Q(W_res)^T is
+ * the same codes read transposed with the same scale grid (section 3.2,
+ * "block-wise quantization ... efficient online transposition").  Encoding,
+ * with IEEE FP32 round-to-nearest-even at every step:
+ *     g   = amax(tensor) / 2688          (g = 1 for an all-zero tensor)
+ *     sd  = E4M3_rne_satfinite(amax(block) / (6 g))
+ *     code= E2M1_rne_satfinite(x / (sd g)),  sign kept; code 0 when sd == 0
+ *     deq = e2m1(code) * sd * g
+ * Two codes per byte, the lower-index element in the low nibble.
+ *
+ * Conventions for every call:
+ *   - All pointers are DEVICE pointers unless stated; the caller owns every
+ *     buffer (inputs, outputs, workspace).  The library never allocates.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream).  Arguments are validated on the host
+ *     first: on any FT_ERR_* return nothing has been launched.
+ *   - bf16 matrices are row-major with a leading dimension in elements.
+ *     Device pointers of bf16 inputs and of code/scale outputs must be 16-byte
+ *     aligned and leading dimensions must keep rows 16-byte aligned
+ *     (FT_ERR_ALIGN otherwise).
+ *   - Empty inputs (zero rows) return FT_OK and launch nothing.
+ *   - NaN or Inf inputs are outside the contract; results are unspecified.
+ *   - Device-side failures (a bounded wait inside a kernel that ran out) set a
+ *     device error word; read and clear it with ft_device_error().
+ */
+#ifndef FT_H_
+#define FT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FT_OK = 0,
+    FT_ERR_INVALID_ARG = 1, /* null pointer, bad enum, negative size          */
+    FT_ERR_SHAPE = 2,       /* a size is not a supported multiple             */
+    FT_ERR_ALIGN = 3,       /* pointer or leading dimension misaligned        */
+    FT_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed            */
+    FT_ERR_TIMEOUT = 5,     /* a kernel's bounded wait ran out (device word)  */
+    FT_ERR_WORKSPACE = 6,   /* workspace missing or smaller than required     */
+    FT_ERR_UNSUPPORTED = 7  /* the current device is not sm_100               */
+} ft_status;
+
+typedef enum { FT_BLK_1x16 = 0, FT_BLK_16x16 = 1 } ft_block;
+typedef enum { FT_BF16 = 0, FT_F32 = 1 } ft_dtype;
+
+/* Non-owning view of an NVFP4 tensor of logical shape rows x cols.
+ *   codes : rows x cols/2 bytes, row-major, two E2M1 codes per byte packed
+ *           along the row (column 2i in the low nibble of byte i).
+ *   scales: E4M3 bytes, row-major.  FT_BLK_1x16: rows x cols/16 (one per 16
+ *           consecutive elements of a row).  FT_BLK_16x16: rows/16 x cols/16.
+ *   tscale: one float, the decode tensor scale g.                          */
+typedef struct {
+    uint8_t* codes;
+    uint8_t* scales;
+    float* tscale;
+    int64_t rows;
+    int64_t cols;
+    ft_block blk;
+} ft_fp4;
+
+/* Non-owning description of one triple-branch linear layer (Eq. 2).
+ *   w_k : Q(W_res), FT_BLK_16x16, rows = N, cols = K (codes packed along K).
+ *   w_n : the same codes transposed, rows = K, cols = N (codes packed along
+ *         N).  Its scales/tscale pointers must equal w_k's: one scale grid
+ *         [N/16, K/16] serves both layouts (section 3.2).
+ *   U [K, r_s], V [N, r_s], A [K, r_l], B [N, r_l]: bf16, row-major, dense.
+ *   r_s, r_l: multiples of 16 with r_s + r_l <= 128 (either may be 0).
+ *   s: the LoRA scale.                                                     */
+typedef struct {
+    int64_t N, K, r_s, r_l;
+    float s;
+    ft_fp4 w_k;
+    ft_fp4 w_n;
+    const void* U;
+    const void* V;
+    const void* A;
+    const void* B;
+} ft_linear;
+
+/* ft_quantize -- Q(x) for a bf16 matrix (section 3.2 block quantization).
+ *   x     : bf16 [rows, cols], leading dimension ld (elements, ld >= cols).
+ *   blk   : FT_BLK_1x16 (cols % 16 == 0) or FT_BLK_16x16 (rows % 16 == 0 and
+ *           cols % 16 == 0).
+ *   amax  : device float holding max|x| to use for the tensor scale, or NULL
+ *           to compute it (needs ws_bytes >= ft_quantize_workspace_bytes()).
+ *   out   : out->codes / scales / tscale receive the result; out->rows,
+ *           out->cols and out->blk must equal rows, cols, blk.
+ * Codes and scales match the encoding above bit for bit.                   */
+ft_status ft_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, ft_block blk,
+                      const float* amax, ft_fp4* out, void* ws, size_t ws_bytes, void* stream);
+
+/* ft_quantize_transpose -- both layouts in one pass over x.
+ *   FT_BLK_16x16: out_row = codes packed along rows of x ([rows, cols/2]);
+ *     out_col = the same codes transposed ([cols, rows/2]); one scale grid
+ *     [rows/16, cols/16] and one tensor scale, written through out_row
+ *     (out_col->scales / tscale must be equal to out_row's or NULL).
+ *   FT_BLK_1x16: out_row = Q(x) with blocks along rows; out_col = Q(x^T),
+ *     an independent 1x16 quantization of the columns of x (blocks of 16
+ *     consecutive rows), codes [cols, rows/2], scales [cols, rows/16].  Both
+ *     share the tensor scale of x (written to both tscale pointers).
+ *     Needs rows % 16 == 0 and cols % 16 == 0.                             */
+ft_status ft_quantize_transpose(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                ft_block blk, const float* amax, ft_fp4* out_row,
+                                ft_fp4* out_col, void* ws, size_t ws_bytes, void* stream);
+
+/* ft_linear_fwd -- Eq. 2 with LoRA fusion (section 3.3): one pass over X
+ * emits Q(X) and the down-projections P = [bf16(X U) | bf16(s X A)]; one
+ * FP4 GEMM on tcgen05 block-scaled tensor cores adds P [V | B]^T in its
+ * epilogue and writes Y once.
+ *   X      : bf16 [M, K] dense (ld = K).  M >= 0, any value.
+ *   amax_x : device float max|X|, or NULL to compute it.
+ *   Y      : [M, N] dense, FT_BF16 or FT_F32 (yt).
+ *   P_save : bf16 [M, r_s + r_l] dense, written; the backward reads it.
+ *   N, K   : multiples of 256 (the scale rows stay 16-byte aligned for TMA).
+ *   ws     : at least ft_workspace_bytes(M, N, K, r_s, r_l) bytes.         */
+ft_status ft_linear_fwd(const ft_linear* L, const void* X, int64_t M, const float* amax_x,
+                        void* Y, ft_dtype yt, void* P_save, void* ws, size_t ws_bytes,
+                        void* stream);
+
+/* ft_linear_bwd -- Eq. 3 and the adapter gradients (section 3.2).
+ *   dY      : bf16 [M, N] dense; X: the forward's bf16 [M, K];
+ *   P_save  : the forward's P.
+ *   amax_dy : device float max|dY|, or NULL to compute it.
+ *   dX      : [M, K], FT_BF16 or FT_F32 (xt).
+ *   dA [K, r_l], dB [N, r_l]: float32, overwritten (not accumulated); may be
+ *   NULL when r_l == 0.                                                    */
+ft_status ft_linear_bwd(const ft_linear* L, const void* dY, const void* X, const void* P_save,
+                        int64_t M, const float* amax_dy, void* dX, ft_dtype xt, float* dA,
+                        float* dB, void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace sizes (bytes) for the calls above. */
+size_t ft_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t r_l);
+size_t ft_quantize_workspace_bytes(void);
+
+/* Reads and clears the device error word of the current device (a host-
+ * synchronous copy on `stream`).  *code receives 0 when no kernel reported a
+ * failure; otherwise a nonzero code naming the wait that ran out.  Returns
+ * FT_ERR_TIMEOUT when *code != 0.                                          */
+ft_status ft_device_error(int* code, void* stream);
+
+/* Human-readable name of a status. */
+const char* ft_status_str(ft_status s);
+
+/* Measurement support (no counterpart in the method; used to report each
+ * kernel's roofline fraction from inside a real step).  While enabled, every
+ * kernel launch of the library is bracketed by two CUDA events on its
+ * stream.  ft_timing_read() waits for the recorded events, adds their
+ * elapsed times to per-kernel totals and returns the total milliseconds and
+ * launch count of one kernel (by name, e.g. "k_gemm_fp4"; "*" = all
+ * kernels).  ft_timing_reset() clears the totals.  Host-synchronous; not
+ * for use inside stream capture.                                          */
+ft_status ft_timing_enable(int on);
+ft_status ft_timing_read(const char* kernel, double* total_ms, int64_t* launches);
+ft_status ft_timing_reset(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FT_H_ */

@@ -222,19 +222,28 @@ def gemm_nt_plain(A: np.ndarray, B: np.ndarray, rows=None) -> np.ndarray:
 def svd_split(W: np.ndarray, r_s: int):
     """Eq. 1: W ~ W_res + V U^T with the top-r_s singular triplets.
 
-    The right singular vectors of W are the eigenvectors of W^T W; the top
-    r_s of them form U [K, r_s] and V = W U = (left vectors) * sigma
-    [N, r_s].  U and V are rounded to bf16 first and W_res = W - V U^T is
-    formed from the rounded factors, so W_res + V U^T reproduces W up to the
-    bf16 rounding of W_res.  Returns bf16 bit patterns (U, V, W_res).
+    The top singular subspace comes from the smaller Gram matrix: with
+    W = sum_i sigma_i u_i v_i^T, the eigenvectors of W^T W are the v_i and
+    those of W W^T the u_i (eigenvalues sigma_i^2).  U = [v_i] [K, r_s] and
+    V = [sigma_i u_i] = W U [N, r_s].  U and V are rounded to bf16 first and
+    W_res = W - V U^T is formed from the rounded factors, so W_res + V U^T
+    reproduces W up to the bf16 rounding of W_res.  Returns bf16 bit patterns
+    (U, V, W_res).
     """
     Wd = bf16_to_f64(W)
+    N, K = Wd.shape
     if r_s == 0:
-        K, N = Wd.shape[1], Wd.shape[0]
         return (np.zeros((K, 0), np.uint16), np.zeros((N, 0), np.uint16), np.asarray(W, np.uint16))
-    evals, evecs = np.linalg.eigh(Wd.T @ Wd)
-    top = evecs[:, np.argsort(evals)[::-1][:r_s]]
-    U = bf16_from_f64(top)
+    if K <= N:
+        evals, evecs = np.linalg.eigh(Wd.T @ Wd)
+        vtop = evecs[:, np.argsort(evals)[::-1][:r_s]]
+    else:
+        evals, evecs = np.linalg.eigh(Wd @ Wd.T)
+        order = np.argsort(evals)[::-1][:r_s]
+        utop = evecs[:, order]
+        sig = np.sqrt(np.maximum(evals[order], 0.0))
+        vtop = (Wd.T @ utop) / np.where(sig > 0, sig, 1.0)
+    U = bf16_from_f64(vtop)
     V = bf16_from_f64(Wd @ bf16_to_f64(U))
     W_res = bf16_from_f64(Wd - bf16_to_f64(V) @ bf16_to_f64(U).T)
     return U, V, W_res

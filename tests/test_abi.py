@@ -1,0 +1,118 @@
+"""Host-only checks of the C ABI: the library builds for sm_100a, loads, and
+exports every entry point include/ft.h declares; argument validation rejects
+bad calls before anything touches the GPU (these calls never reach CUDA)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_quantized_lora_b200 import _lib
+from bit_quantized_lora_b200._lib import FtFp4, FtLinear
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ft.h")
+
+FT_OK, FT_ERR_INVALID_ARG, FT_ERR_SHAPE, FT_ERR_ALIGN = 0, 1, 2, 3
+FT_ERR_WORKSPACE = 6
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ft_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    return _lib.load(build_if_missing=True)
+
+
+def test_every_declared_symbol_is_exported_and_bound(L):
+    names = declared_functions()
+    assert len(names) >= 8
+    for n in names:
+        assert hasattr(L, n), n
+        assert n in _lib.SIGNATURES, n
+    assert set(_lib.SIGNATURES) == set(names)
+
+
+def test_struct_layouts_match_c():
+    # int64 x4, float (+4 pad), two 48-byte views, four pointers
+    assert ctypes.sizeof(FtFp4) == 48
+    assert ctypes.sizeof(FtLinear) == 32 + 8 + 2 * 48 + 4 * 8
+
+
+def test_status_strings(L):
+    assert L.ft_status_str(0) == b"FT_OK"
+    assert L.ft_status_str(2) == b"FT_ERR_SHAPE"
+    assert L.ft_status_str(99) == b"FT_ERR_UNKNOWN"
+
+
+def test_workspace_sizes_are_deterministic_and_monotone(L):
+    a = L.ft_workspace_bytes(4608, 3072, 3072, 32, 16)
+    b = L.ft_workspace_bytes(4608, 3072, 3072, 32, 16)
+    c = L.ft_workspace_bytes(9216, 3072, 3072, 32, 16)
+    assert a == b and c > a > 0
+    assert L.ft_workspace_bytes(-1, 1, 1, 0, 0) == 0
+    assert L.ft_quantize_workspace_bytes() == 256
+
+
+def _view(rows, cols, blk, p=0x1000):
+    return FtFp4(p, p, p, rows, cols, blk)
+
+
+def test_quantize_validation_happens_on_the_host(L):
+    v = _view(32, 64, 0)
+    x = 0x10000
+    # null input
+    assert L.ft_quantize(None, 32, 64, 64, 0, None, ctypes.byref(v), x, 256, None) == FT_ERR_INVALID_ARG
+    # bad block enum
+    assert L.ft_quantize(x, 32, 64, 64, 7, None, ctypes.byref(v), x, 256, None) == FT_ERR_INVALID_ARG
+    # cols not a multiple of 16
+    v2 = _view(32, 60, 0)
+    assert L.ft_quantize(x, 32, 60, 64, 0, None, ctypes.byref(v2), x, 256, None) == FT_ERR_SHAPE
+    # 16x16 needs rows % 16 == 0
+    v3 = _view(30, 64, 1)
+    assert L.ft_quantize(x, 30, 64, 64, 1, None, ctypes.byref(v3), x, 256, None) == FT_ERR_SHAPE
+    # view shape must match
+    assert L.ft_quantize(x, 16, 64, 64, 0, None, ctypes.byref(v), x, 256, None) == FT_ERR_SHAPE
+    # misaligned input pointer / leading dimension
+    assert L.ft_quantize(x + 2, 32, 64, 64, 0, None, ctypes.byref(v), x, 256, None) == FT_ERR_ALIGN
+    assert L.ft_quantize(x, 32, 64, 68, 0, None, ctypes.byref(v), x, 256, None) == FT_ERR_ALIGN
+    # amax to compute but no workspace
+    assert L.ft_quantize(x, 32, 64, 64, 0, None, ctypes.byref(v), None, 0, None) == FT_ERR_WORKSPACE
+    # empty input: nothing to do, no launch
+    v0 = _view(0, 64, 0)
+    assert L.ft_quantize(x, 0, 64, 64, 0, None, ctypes.byref(v0), x, 256, None) == FT_OK
+
+
+def _linear(N=256, K=256, r_s=16, r_l=16):
+    p = 0x100000
+    wk = FtFp4(p, p, p, N, K, 1)
+    wn = FtFp4(p, p, p, K, N, 1)
+    return FtLinear(N, K, r_s, r_l, 1.0, wk, wn, p, p, p, p)
+
+
+def test_linear_validation_happens_on_the_host(L):
+    x = 0x200000
+    ws = L.ft_workspace_bytes(128, 256, 256, 16, 16)
+    ok = _linear()
+    bad_n = _linear(N=320)
+    assert L.ft_linear_fwd(ctypes.byref(bad_n), x, 128, None, x, 0, x, x, ws, None) == FT_ERR_SHAPE
+    bad_r = _linear(r_s=8)
+    assert L.ft_linear_fwd(ctypes.byref(bad_r), x, 128, None, x, 0, x, x, ws, None) == FT_ERR_SHAPE
+    big_r = _linear(r_s=80, r_l=64)
+    assert L.ft_linear_fwd(ctypes.byref(big_r), x, 128, None, x, 0, x, x, ws, None) == FT_ERR_SHAPE
+    assert L.ft_linear_fwd(None, x, 128, None, x, 0, x, x, ws, None) == FT_ERR_INVALID_ARG
+    assert L.ft_linear_fwd(ctypes.byref(ok), x, 128, None, x, 5, x, x, ws, None) == FT_ERR_INVALID_ARG
+    assert L.ft_linear_fwd(ctypes.byref(ok), x, 128, None, x, 0, x, x, ws - 1, None) == FT_ERR_WORKSPACE
+    assert L.ft_linear_fwd(ctypes.byref(ok), x + 8, 128, None, x, 0, x, x, ws, None) == FT_ERR_ALIGN
+    # the transposed weight view must share the scale grid
+    shared = _linear()
+    shared.w_n.scales = 0x300000
+    assert L.ft_linear_fwd(ctypes.byref(shared), x, 128, None, x, 0, x, x, ws, None) == FT_ERR_INVALID_ARG
+    # M = 0: nothing to do
+    assert L.ft_linear_fwd(ctypes.byref(ok), x, 0, None, x, 0, x, x, ws, None) == FT_OK
+    assert L.ft_linear_bwd(ctypes.byref(bad_n), x, x, x, 128, None, x, 0, x, x, x, ws, None) == FT_ERR_SHAPE
+    assert L.ft_linear_bwd(ctypes.byref(ok), x, x, x, 128, None, x, 9, x, x, x, ws, None) == FT_ERR_INVALID_ARG

@@ -1,0 +1,117 @@
+"""GPU parity of the NVFP4 quantize kernels against the CPU oracle.
+
+Codes, scales and the tensor scale must match bit for bit (integer work)."""
+import numpy as np
+import pytest
+import torch
+
+import ft_synth
+import oracle
+import bit_quantized_lora_b200 as ft
+from gpu_util import dev_bf16, host, scalar_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_1x16(x_u16, amax=None):
+    x = dev_bf16(x_u16)
+    q = ft.ft_quantize(x, ft.BLK_1x16, amax=None if amax is None else scalar_dev(amax))
+    torch.cuda.synchronize()
+    codes, scales, g = oracle.quantize_1x16(x_u16, amax)
+    assert np.float32(host(q.tscale)[0]) == np.float32(g)
+    np.testing.assert_array_equal(host(q.scales), scales)
+    np.testing.assert_array_equal(host(q.codes), codes)
+
+
+@pytest.mark.parametrize("wl", [0, 1, 3])
+def test_quantize_1x16_workload_activations_and_gradients(wl):
+    shape = ft_synth.WORKLOADS[wl]
+    inp = ft_synth.make_inputs(shape, seed=wl)
+    _check_1x16(inp["X"])
+    _check_1x16(inp["dY"])
+
+
+def test_quantize_1x16_every_bf16_value():
+    # all finite bf16 patterns, shuffled into 16-element blocks, under several
+    # tensor scales (computed, larger, smaller than the true amax)
+    rng = np.random.default_rng(30)
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    f = (bits.astype(np.uint32) << 16).view(np.float32)
+    finite = bits[np.isfinite(f)]
+    x = rng.permutation(finite)
+    x = x[: (len(x) // 256) * 256].reshape(-1, 256)
+    _check_1x16(x)
+    for amax in [1.0, 3.0e38, 1e-30, 448.0 * 6.0]:
+        _check_1x16(x, amax)
+    # small-magnitude tensor: exercises subnormal divisors
+    small = rng.permutation(finite[(np.abs(f[np.isfinite(f)]) < 1e-30)])
+    small = small[: (len(small) // 256) * 256].reshape(-1, 256)
+    _check_1x16(small)
+
+
+def test_quantize_1x16_ragged_strided_zero():
+    rng = np.random.default_rng(31)
+    x = ft_synth.to_bf16_bits(rng.standard_normal((37, 80)))
+    _check_1x16(x)
+    # strided input (ld > cols): quantize a column slice
+    big = ft_synth.to_bf16_bits(rng.standard_normal((40, 96)))
+    xd = dev_bf16(big)[:, :64]
+    q = ft.ft_quantize(xd, ft.BLK_1x16)
+    torch.cuda.synchronize()
+    codes, scales, g = oracle.quantize_1x16(np.ascontiguousarray(big[:, :64]))
+    np.testing.assert_array_equal(host(q.codes), codes)
+    np.testing.assert_array_equal(host(q.scales), scales)
+    # all zero: g = 1, zero codes and scales
+    z = np.zeros((16, 32), np.uint16)
+    q = ft.ft_quantize(dev_bf16(z), ft.BLK_1x16)
+    torch.cuda.synchronize()
+    assert host(q.tscale)[0] == 1.0 and not host(q.codes).any() and not host(q.scales).any()
+
+
+@pytest.mark.parametrize("wl", [0, 1, 2, 3])
+def test_quantize_transpose_16x16_weights(wl):
+    shape = ft_synth.WORKLOADS[wl]
+    W = ft_synth.make_inputs(shape, seed=wl)["W"]
+    cr, cc, s, g = oracle.quantize_16x16(W)
+    w_k, w_n = ft.ft_quantize_transpose(dev_bf16(W), ft.BLK_16x16)
+    torch.cuda.synchronize()
+    assert np.float32(host(w_k.tscale)[0]) == np.float32(g)
+    assert w_n.scales.data_ptr() == w_k.scales.data_ptr()
+    np.testing.assert_array_equal(host(w_k.scales), s)
+    np.testing.assert_array_equal(host(w_k.codes), cr)
+    np.testing.assert_array_equal(host(w_n.codes), cc)
+    # ft_quantize with 16x16 blocks emits the row layout alone, identically
+    q = ft.ft_quantize(dev_bf16(W), ft.BLK_16x16)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host(q.codes), cr)
+    np.testing.assert_array_equal(host(q.scales), s)
+
+
+@pytest.mark.parametrize("wl", [0, 2])
+def test_quantize_transpose_1x16_activations(wl):
+    shape = ft_synth.WORKLOADS[wl]
+    inp = ft_synth.make_inputs(shape, seed=wl)
+    for key in ["X", "dY"]:
+        x = inp[key]
+        r, c = ft.ft_quantize_transpose(dev_bf16(x), ft.BLK_1x16)
+        torch.cuda.synchronize()
+        cr, sr, g = oracle.quantize_1x16(x)
+        cc, sc, gc = oracle.quantize_1x16_colwise(x)
+        assert gc == g
+        assert np.float32(host(r.tscale)[0]) == np.float32(g)
+        assert np.float32(host(c.tscale)[0]) == np.float32(g)
+        np.testing.assert_array_equal(host(r.codes), cr)
+        np.testing.assert_array_equal(host(r.scales), sr)
+        np.testing.assert_array_equal(host(c.codes), cc)
+        np.testing.assert_array_equal(host(c.scales), sc)
+
+
+def test_supplied_amax_matches_computed():
+    rng = np.random.default_rng(32)
+    x = ft_synth.to_bf16_bits(rng.standard_normal((64, 128)) * 3)
+    a = oracle.amax_bf16(x)
+    q1 = ft.ft_quantize(dev_bf16(x), ft.BLK_1x16)
+    q2 = ft.ft_quantize(dev_bf16(x), ft.BLK_1x16, amax=scalar_dev(a))
+    torch.cuda.synchronize()
+    assert torch.equal(q1.codes, q2.codes) and torch.equal(q1.scales, q2.scales)
+    assert torch.equal(q1.tscale, q2.tscale)
