@@ -53,6 +53,9 @@ SIGNATURES = {
     "ft_quantize_workspace_bytes": (ctypes.c_size_t, []),
     "ft_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int), c_vp]),
     "ft_status_str": (ctypes.c_char_p, [ctypes.c_int]),
+    "ft_linear_fwd_noalloc": (ctypes.c_int, [ctypes.POINTER(FtLinear), c_vp, c_i64, c_vp, c_vp,
+                                             ctypes.c_int, c_vp, c_vp]),
+    "ft_linear_fwd_noalloc_max_bytes": (ctypes.c_size_t, []),
     "ft_timing_enable": (ctypes.c_int, [ctypes.c_int]),
     "ft_timing_read": (ctypes.c_int, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),
                                       ctypes.POINTER(c_i64)]),

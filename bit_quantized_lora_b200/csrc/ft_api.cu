@@ -680,3 +680,50 @@ ft_status ft_timing_reset(void) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- forward without allocation
+// Some callers cannot hand the library a workspace: a C host that has no
+// device allocator wired in, a plug-in living inside another framework that
+// owns all device memory through its own pool and forbids cudaMalloc from
+// third-party code, or code that must not allocate while it builds up work
+// on a stream.  ft_linear_fwd_noalloc serves them: it runs the same forward
+// as ft_linear_fwd with its workspace in the array below, which lives in the
+// library's device image.  Every GPU that loads the library holds these
+// bytes until the process exits.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+void* g_noalloc_scratch_dev[64] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of g_noalloc_scratch on the current device.  The host
+// symbol is only a stand-in; the address has to be looked up, once per
+// device, with that device current.
+ft_status noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FT_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_scratch_dev[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return FT_ERR_CUDA;
+        g_noalloc_scratch_dev[dev] = p;
+    }
+    *out = g_noalloc_scratch_dev[dev];
+    return FT_OK;
+}
+
+}  // namespace
+
+extern "C" ft_status ft_linear_fwd_noalloc(const ft_linear* L, const void* X, int64_t M,
+                                           const float* amax_x, void* Y, ft_dtype yt, void* P_save,
+                                           void* stream) {
+    if (!L || M < 0 || L->N < 0 || L->K < 0 || L->r_s < 0 || L->r_l < 0) return FT_ERR_INVALID_ARG;
+    if (ft_workspace_bytes(M, L->N, L->K, L->r_s, L->r_l) > kNoAllocScratchBytes) return FT_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    FT_TRY(noalloc_scratch(&scratch));
+    return ft_linear_fwd(L, X, M, amax_x, Y, yt, P_save, scratch, kNoAllocScratchBytes, stream);
+}
+
+extern "C" size_t ft_linear_fwd_noalloc_max_bytes(void) { return kNoAllocScratchBytes; }

@@ -169,6 +169,29 @@ ft_status ft_device_error(int* code, void* stream);
 /* Human-readable name of a status. */
 const char* ft_status_str(ft_status s);
 
+/* ft_linear_fwd_noalloc -- the forward of ft_linear_fwd for callers that
+ * cannot allocate device memory or hand over a workspace (a C host with no
+ * device allocator, a plug-in inside a framework that owns all device memory
+ * through its own pool, code that must not allocate while queueing work).
+ * The paper has no counterpart: this is a deployment convenience.
+ *   Arguments, results and errors are those of ft_linear_fwd, without ws.
+ *   Scratch: a fixed array inside the library's device image,
+ *   ft_linear_fwd_noalloc_max_bytes() = 32 MiB, held on every GPU that
+ *   loads the library until the process exits.  A layer/batch whose
+ *   ft_workspace_bytes() exceeds it returns FT_ERR_WORKSPACE, nothing
+ *   launched.  The function itself allocates nothing.
+ *   The first call on a device looks up the array's device address (once
+ *   per device, with that device current); make that first call before any
+ *   stream capture.
+ *   All calls on a device share its one copy of the array, which keeps the
+ *   last call's contents (each call clears what must start at zero itself).
+ *   Calls whose work overlaps on the same GPU (two streams, two host
+ *   threads) race on the array: the caller must serialise them.  Calls on
+ *   different GPUs use different copies.                                  */
+ft_status ft_linear_fwd_noalloc(const ft_linear* L, const void* X, int64_t M, const float* amax_x,
+                                void* Y, ft_dtype yt, void* P_save, void* stream);
+size_t ft_linear_fwd_noalloc_max_bytes(void);
+
 /* Measurement support (no counterpart in the method; used to report each
  * kernel's roofline fraction from inside a real step).  While enabled, every
  * kernel launch of the library is bracketed by two CUDA events on its
