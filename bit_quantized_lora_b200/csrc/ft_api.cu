@@ -171,7 +171,8 @@ constexpr int QD_MAX_SPLITS = 8;
 constexpr int LG_MAX_SPLITS = 16;
 
 struct WsPlan {
-    size_t amax, gact, codes, scales, lt, part, pg, lgpart, total;
+    size_t amax, gact, codes, scales, lt, part, pg, lgpart, counters, total;
+    int n_qd_counters, lg_ctiles, n_counters;
 };
 
 WsPlan plan_ws(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t r_l) {
@@ -187,6 +188,12 @@ WsPlan plan_ws(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t r_l) {
     w.part = o;   o += up256((size_t)QD_MAX_SPLITS * M * r * 4);
     w.pg = o;     o += up256((size_t)M * r * 2);
     w.lgpart = o; o += up256((size_t)LG_MAX_SPLITS * (N + K) * r_l * 4);
+    // completion counters: one per row tile of the fused quantize/down-proj,
+    // one per (gradient, column tile) of the adapter gradients
+    w.n_qd_counters = (int)((M + 127) / 128);
+    w.lg_ctiles = (int)((C + 127) / 128);
+    w.n_counters = w.n_qd_counters + 2 * w.lg_ctiles;
+    w.counters = o; o += up256((size_t)w.n_counters * 4);
     w.total = o;
     return w;
 }
@@ -196,7 +203,8 @@ ft_status run_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, float*
                    const DevInfo* d, cudaStream_t st) {
     FT_TRY(cuda_ok(cudaMemsetAsync(slot, 0, sizeof(float), st)));
     const int64_t vecs = rows * (cols / 8);
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(vecs, 256), (int64_t)d->sms * 8));
+    // one round of four 16-byte loads per thread covers a dense tensor
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(vecs, 4 * 256), 1 << 30));
     {
         LaunchTimer _lt(KID_AMAX, st);
         ft::k_amax_bf16<<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(x), rows, cols, ld,
@@ -244,16 +252,30 @@ ft_status run_tile16(bool mode16x16, const void* x, int64_t rows, int64_t cols, 
 }
 
 // Q(T) and P = [bf16(T L1) | bf16(s T L2)] in one pass over T [M, C].
+// Also zeroes the completion counters (qdown and adapter-gradient tiles) the
+// kernels of this call use.
 ft_status run_qdown(const void* T, int64_t M, int64_t C, const void* L1, int64_t r1, const void* L2,
                     int64_t r2, float s, const float* amax, uint8_t* codes, uint8_t* scales,
                     float* tscale, void* P, uint8_t* ws, const WsPlan& w, const DevInfo* d,
                     cudaStream_t st) {
     const int64_t r = r1 + r2;
     if (r == 0) return run_quant_1x16(T, M, C, C, amax, codes, scales, tscale, d, st);
-    uint16_t* Lt = reinterpret_cast<uint16_t*>(ws + w.lt);
     float* part = reinterpret_cast<float*>(ws + w.part);
-    {
-        const int grid = std::min(cdiv(128 * C, 256), d->sms * 8);
+    unsigned int* counters = reinterpret_cast<unsigned int*>(ws + w.counters);
+    FT_TRY(cuda_ok(cudaMemsetAsync(counters, 0, (size_t)w.n_counters * 4, st)));
+    ft::qdown::Params p;
+    std::memset(&p, 0, sizeof(p));
+    p.direct = (r1 <= 64 && r2 <= 64) ? 1 : 0;
+    if (p.direct) {
+        if (r1 > 0)
+            FT_TRY(encode_2d(&p.mapL1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1, r1, C, r1 * 2, 64, 64,
+                             CU_TENSOR_MAP_SWIZZLE_128B));
+        if (r2 > 0)
+            FT_TRY(encode_2d(&p.mapL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2, r2, C, r2 * 2, 64, 64,
+                             CU_TENSOR_MAP_SWIZZLE_128B));
+    } else {
+        uint16_t* Lt = reinterpret_cast<uint16_t*>(ws + w.lt);
+        dim3 grid((unsigned)cdiv(C, 256), 128);
         {
             LaunchTimer _lt(KID_PACK_LT, st);
             ft::k_pack_lt<<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(L1), (int)r1,
@@ -261,40 +283,34 @@ ft_status run_qdown(const void* T, int64_t M, int64_t C, const void* L1, int64_t
             _lt.stop();
         }
         FT_TRY(last_launch());
+        FT_TRY(encode_2d(&p.mapL1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Lt, C, 128, C * 2, 64, 128,
+                         CU_TENSOR_MAP_SWIZZLE_128B));
     }
     const int mt = cdiv(M, ft::qdown::BM);
     int splits = std::max(1, std::min(QD_MAX_SPLITS, d->sms / std::max(1, mt)));
     int cchunk = cdiv(C, (int64_t)splits * 64) * 64;
     splits = cdiv(C, cchunk);
-    ft::qdown::Params p;
-    std::memset(&p, 0, sizeof(p));
     FT_TRY(encode_2d(&p.mapT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, C, M, C * 2, 64, 128,
-                     CU_TENSOR_MAP_SWIZZLE_128B));
-    FT_TRY(encode_2d(&p.mapLt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Lt, C, 128, C * 2, 64, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B));
     p.amax = amax;
     p.tscale = tscale;
     p.codes = codes;
     p.scales = scales;
     p.part = part;
+    p.P = static_cast<__nv_bfloat16*>(P);
+    p.counters = counters;
     p.M = (int)M;
     p.C = (int)C;
     p.r = (int)r;
+    p.r1 = (int)r1;
     p.cchunk = cchunk;
+    p.splits = splits;
+    p.s = s;
     p.do_mma = 1;
     {
         LaunchTimer _lt(KID_QDOWN, st);
         ft::qdown::k_qdown<<<dim3((unsigned)mt, (unsigned)splits), ft::qdown::NUM_THREADS,
                              ft::qdown::SMEM_BYTES, st>>>(p);
-        _lt.stop();
-    }
-    FT_TRY(last_launch());
-    const int64_t tot = M * r;
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(tot, 256), (int64_t)d->sms * 8));
-    {
-        LaunchTimer _lt(KID_LR_FINALIZE, st);
-        ft::k_lowrank_finalize<<<grid, 256, 0, st>>>(part, splits, (int)M, (int)r, (int)r1, s,
-                                                     static_cast<__nv_bfloat16*>(P));
         _lt.stop();
     }
     return last_launch();
@@ -373,6 +389,9 @@ ft_status run_lora_grads(const void* dY, const void* X, const void* P, const voi
     float* partA = partB + (size_t)splits * N * r_l;
     p.part[0] = partB;
     p.part[1] = partA;
+    p.out[0] = dB;
+    p.out[1] = dA;
+    p.counters = reinterpret_cast<unsigned int*>(ws + w.counters) + w.n_qd_counters;
     p.C[0] = (int)N;
     p.C[1] = (int)K;
     p.M = (int)M;
@@ -380,34 +399,15 @@ ft_status run_lora_grads(const void* dY, const void* X, const void* P, const voi
     p.r_l = (int)r_l;
     p.n_pad = r_l <= 64 ? 64 : 128;
     p.mrows = mrows;
+    p.splits = splits;
+    p.ctiles_max = w.lg_ctiles;
     dim3 grid((unsigned)(std::max(N, K) / ft::lgrad::BC), (unsigned)splits, 2);
     {
         LaunchTimer _lt(KID_LORA_GRAD, st);
         ft::lgrad::k_lora_grad<<<grid, ft::lgrad::NUM_THREADS, ft::lgrad::smem_bytes(p.n_pad), st>>>(p);
         _lt.stop();
     }
-    FT_TRY(last_launch());
-    {
-        const int64_t n = N * r_l;
-        const int g = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(n, 256), (int64_t)d->sms * 4));
-        {
-            LaunchTimer _lt(KID_LORA_REDUCE, st);
-            ft::k_lora_grad_reduce<<<g, 256, 0, st>>>(partB, splits, n, dB);
-            _lt.stop();
-        }
-        FT_TRY(last_launch());
-    }
-    {
-        const int64_t n = K * r_l;
-        const int g = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(n, 256), (int64_t)d->sms * 4));
-        {
-            LaunchTimer _lt(KID_LORA_REDUCE, st);
-            ft::k_lora_grad_reduce<<<g, 256, 0, st>>>(partA, splits, n, dA);
-            _lt.stop();
-        }
-        FT_TRY(last_launch());
-    }
-    return FT_OK;
+    return last_launch();
 }
 
 // ------------------------------------------------------------ validation

@@ -147,4 +147,134 @@ __device__ __forceinline__ uint2 quant_block16(const uint32_t (&w)[8], const QTe
     return r;
 }
 
+
+// ------------------------------------------------------------------------
+// Throughput path.  The divisor d = RN(sd g) of a block depends only on its
+// scale byte, so each CTA tabulates d and y = RN(1/d) for the 126 positive
+// finite E4M3 values once (QTable, in shared memory); per element the exact
+// quotient then costs one packed multiply and two packed FMAs on f32x2
+// pairs.  The sign of x is ORed back after the division (the correction step
+// turns -0 / d into +0), and cvt...e2m1x2 encodes sign and magnitude.
+// Bit-identical to quant_block16 (same IEEE definition).
+
+struct QTable {
+    float d[128];
+    float y[128];  // 0 marks a divisor outside [2^-60, 2^60]: use IEEE division
+};
+
+struct QTensorFast {
+    float g, six_g, y6;  // y6 = RN(1/six_g), 0 when six_g is outside the safe range
+};
+
+__device__ __forceinline__ QTensorFast make_qtensor_fast(float amax) {
+    QTensor t = make_qtensor(amax);
+    QTensorFast f;
+    f.g = t.g;
+    f.six_g = t.six_g;
+    f.y6 = (t.six_g >= 0x1p-60f && t.six_g <= 0x1p60f) ? __frcp_rn(t.six_g) : 0.0f;
+    return f;
+}
+
+// Fill the table cooperatively (threads tid of nthreads).  Call before a
+// barrier that precedes the first lookup.
+__device__ __forceinline__ void build_qtable(QTable& tab, float g, int tid, int nthreads) {
+    for (int s = tid; s < 128; s += nthreads) {
+        float d = 0.0f, y = 0.0f;
+        if (s >= 1 && s <= 0x7E) {
+            d = __fmul_rn(e4m3_decode((uint32_t)s), g);
+            y = (d >= 0x1p-60f && d <= 0x1p60f) ? __frcp_rn(d) : 0.0f;
+        }
+        tab.d[s] = d;
+        tab.y[s] = y;
+    }
+}
+
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// Scale byte of a block from its amax (Markstein quotient when y6 != 0).
+__device__ __forceinline__ uint32_t scale_byte_fast(float amax_b, const QTensorFast& t) {
+    float sf;
+    const float q = __fmul_rn(amax_b, t.y6);
+    if (t.y6 != 0.0f && q < 0x1p100f) {
+        const float r = __fmaf_rn(-q, t.six_g, amax_b);
+        sf = __fmaf_rn(r, t.y6, q);
+    } else {
+        // no reciprocal, or a quotient far beyond the E4M3 range (a caller
+        // amax below the true one): IEEE division, which saturates cleanly
+        sf = __fdiv_rn(amax_b, t.six_g);
+    }
+    return e4m3_encode(sf);
+}
+
+// Codes of 8 elements (4 bf16 pairs) given the block divisor d and y.
+__device__ __forceinline__ uint32_t encode8_fast(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3,
+                                                 float d, float y) {
+    const uint32_t w[4] = {w0, w1, w2, w3};
+    const uint64_t Y = f2pack(y, y);
+    const uint64_t ND = f2pack(-d, -d);
+    uint32_t out;
+    float q[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t lo = w[i] << 16, hi = w[i] & 0xFFFF0000u;
+        const uint64_t X = f2pack(__uint_as_float(lo), __uint_as_float(hi));
+        uint64_t Q = mul_f32x2(X, Y);
+        const uint64_t R = fma_f32x2(Q, ND, X);
+        Q = fma_f32x2(R, Y, Q);
+        float qa, qb;
+        f2unpack(Q, qa, qb);
+        q[2 * i] = __uint_as_float(__float_as_uint(qa) | (lo & 0x80000000u));
+        q[2 * i + 1] = __uint_as_float(__float_as_uint(qb) | (hi & 0x80000000u));
+    }
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(q[0]), "f"(q[1]), "f"(q[2]), "f"(q[3]), "f"(q[4]), "f"(q[5]), "f"(q[6]), "f"(q[7]));
+    return out;
+}
+
+// One 1x16 block through the table.  Returns the 8 code bytes; *sbyte the scale.
+__device__ __forceinline__ uint2 quant_block16_fast(const uint32_t (&w)[8], const QTensorFast& t,
+                                                    const QTable& tab, uint32_t& sbyte) {
+    const float amax_b = __uint_as_float(amax_bits_16(w));
+    sbyte = scale_byte_fast(amax_b, t);
+    const float d = tab.d[sbyte];
+    const float y = tab.y[sbyte];
+    uint2 r;
+    if (sbyte == 0) {
+        r = make_uint2(0u, 0u);
+    } else if (y != 0.0f && sbyte != 0x7Eu) {
+        // below the top scale every quotient stays under ~13, so x * y cannot
+        // overflow; the saturated top scale (a tensor's largest block, or a
+        // caller amax below the true one) takes the IEEE path
+        r.x = encode8_fast(w[0], w[1], w[2], w[3], d, y);
+        r.y = encode8_fast(w[4], w[5], w[6], w[7], d, y);
+    } else {
+        r.x = encode8(w[0], w[1], w[2], w[3], d, 0.0f, false);
+        r.y = encode8(w[4], w[5], w[6], w[7], d, 0.0f, false);
+    }
+    return r;
+}
+
 }  // namespace ft

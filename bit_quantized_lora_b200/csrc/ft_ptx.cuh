@@ -19,6 +19,10 @@ namespace ft {
 // that ran out.  One per device per process (module scope).
 __device__ int g_ft_error = 0;
 
+// Suspend-time hint of one mbarrier.try_wait (the thread resumes earlier
+// when the phase completes).
+constexpr uint32_t kTryWaitHintNs = 1000000;
+
 // A wait gives up after this many nanoseconds of %globaltimer.
 constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
 
@@ -70,10 +74,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kTryWaitHintNs)
         : "memory");
     return ok != 0;
 }
@@ -180,6 +184,11 @@ __device__ __forceinline__ void umma_nvfp4(uint32_t d_tmem, uint64_t adesc, uint
 __device__ __forceinline__ void tc_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
     asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
                  : "memory");
+}
+
+// 64-bit descriptor from its two 32-bit words.
+__device__ __forceinline__ uint64_t make_desc(uint32_t lo, uint32_t hi) {
+    return ((uint64_t)hi << 32) | lo;
 }
 
 // Each thread of the warp reads 32 consecutive 32-bit columns of its TMEM

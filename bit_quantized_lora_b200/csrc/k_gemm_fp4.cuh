@@ -17,17 +17,24 @@
 // Blackwell mapping: one CTA per SM, persistent over 128x128 output tiles.
 //   warp 0  TMA producer: FP4 code tiles (128 B swizzle), raw scale rows,
 //           the tile's P / L1 / L2 panels.
-//   warp 1  TMEM owner and UMMA issuer: tcgen05.cp of the block scales into
-//           TMEM, tcgen05.mma.kind::mxf4nvf4.block16 (K = 64 per instruction)
-//           into a double-buffered FP32 accumulator, then tcgen05.mma
-//           kind::f16 for the low-rank panels into a separate accumulator.
+//   warp 1  TMEM owner and UMMA issuer: per stage one tcgen05.cp of each
+//           operand's block scales into TMEM and four
+//           tcgen05.mma.kind::mxf4nvf4.block16 (K = 64 each) into a
+//           double-buffered FP32 accumulator, then tcgen05.mma kind::f16 for
+//           the low-rank panels into a separate accumulator.  Descriptors
+//           are precomputed words, so the issue loop is a few integer adds.
 //   warp 2  scale-factor warp: rearranges each stage's scale bytes into the
-//           32x128-bit layout tcgen05.cp expects (row r of a 128-row slab in
-//           32-bit slot (r % 32) * 4 + r / 32), expanding 16x16 weight
-//           scales to one per row.
+//           slab layout below, expanding 16x16 weight scales to one per row.
 //   warps 4-7 epilogue: tcgen05.ld both accumulators, combine, store.
 // TMEM columns: [0,128) acc0, [128,256) acc1, [256,384) low-rank acc,
 // [384,400) A scales, [400,416) B scales.
+//
+// Scale factors in TMEM: the MMA reads the four scale bytes of row m (one
+// per 16 K-elements of its K = 64) from TMEM lane m at column c + m/32, c
+// being the (4-column aligned) scale address the instruction names.  Each
+// K-step's scales are one 32-row x 16-byte slab in shared memory (row m % 32
+// holds rows m % 32 + 32 q at bytes 4q..4q+3) that tcgen05.cp.32x128b.warpx4
+// replicates into all four lane quarters; K-step j uses columns c = base + 4j.
 #pragma once
 
 #include <cuda.h>
@@ -46,7 +53,7 @@ constexpr int NUM_THREADS = 256;
 constexpr int TILE_BYTES = BM * BK_BYTES;      // 16 KiB, A or B stage
 constexpr int SFA_RAW_BYTES = BM * 16;         // 128 rows x 16 scale bytes
 constexpr int SFB_RAW_BYTES = 256;             // 8 x 16 (fwd) or 16 x 16 (dgrad)
-constexpr int SF_ATOM_BYTES = KSTEPS * 512;    // 4 x (32 x 16 B)
+constexpr int SF_ATOM_BYTES = KSTEPS * 512;    // 4 x (32 rows x 16 B)
 constexpr int PANEL_BYTES = 128 * 64 * 2;      // a 128-row x 64-col bf16 panel
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL0 = 0, LR_COL = 256, SFA_COL = 384, SFB_COL = 400;
@@ -213,6 +220,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
         if (lane == 0) {
             const uint32_t idesc = idesc_nvfp4(BM, BN);
             const uint32_t idesc_lr = idesc_bf16(BM, BN, 0, 0);
+            // descriptor words: lo = start >> 4 | (LBO >> 4) << 16;
+            // hi = SBO >> 4 | version 1 << 14 | layout << 29
+            const uint32_t hi_sw128 = (1024u >> 4) | (1u << 14) | (SWZ_128B << 29);
+            const uint32_t hi_sf = (128u >> 4) | (1u << 14);  // 8-row groups 128 B apart
+            const uint32_t a_lo0 = ((base + L.a) >> 4) | (1u << 16);
+            const uint32_t b_lo0 = ((base + L.b) >> 4) | (1u << 16);
+            const uint32_t sfa_lo0 = (base + L.sfa) >> 4;  // one 16-byte column: LBO unused
+            const uint32_t sfb_lo0 = (base + L.sfb) >> 4;
             uint32_t it = 0;
             bool ok = true;
             int local = 0;
@@ -233,21 +248,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sfa_s = base + L.sfa + s * SF_ATOM_BYTES;
-                    const uint32_t sfb_s = base + L.sfb + s * SF_ATOM_BYTES;
+                    const uint32_t sfa_lo = sfa_lo0 + s * (SF_ATOM_BYTES >> 4);
+                    const uint32_t sfb_lo = sfb_lo0 + s * (SF_ATOM_BYTES >> 4);
 #pragma unroll
                     for (int j = 0; j < KSTEPS; ++j) {
-                        tc_cp_32x128b_x4(tmem + SFA_COL + 4 * j, smem_desc(sfa_s + 512 * j, 0, 128, SWZ_NONE));
-                        tc_cp_32x128b_x4(tmem + SFB_COL + 4 * j, smem_desc(sfb_s + 512 * j, 0, 128, SWZ_NONE));
+                        tc_cp_32x128b_x4(tmem + SFA_COL + 4 * j, make_desc(sfa_lo + 32 * j, hi_sf));
+                        tc_cp_32x128b_x4(tmem + SFB_COL + 4 * j, make_desc(sfb_lo + 32 * j, hi_sf));
                     }
-                    const uint32_t a_s = base + L.a + s * TILE_BYTES;
-                    const uint32_t b_s = base + L.b + s * TILE_BYTES;
+                    const uint32_t a_lo = a_lo0 + s * (TILE_BYTES >> 4);
+                    const uint32_t b_lo = b_lo0 + s * (TILE_BYTES >> 4);
 #pragma unroll
-                    for (int j = 0; j < KSTEPS; ++j) {
-                        umma_nvfp4(acc, desc_kmajor_sw128(a_s + 32 * j), desc_kmajor_sw128(b_s + 32 * j),
-                                   idesc, tmem + SFA_COL + 4 * j, tmem + SFB_COL + 4 * j,
-                                   (kt | j) != 0);
-                    }
+                    for (int j = 0; j < KSTEPS; ++j)
+                        umma_nvfp4(acc, make_desc(a_lo + 2 * j, hi_sw128), make_desc(b_lo + 2 * j, hi_sw128),
+                                   idesc, tmem + SFA_COL + 4 * j, tmem + SFB_COL + 4 * j, (kt | j) != 0);
                     tc_commit(&bars[B_EMPTY + s]);
                 }
                 if (!ok) break;
@@ -300,25 +313,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                 const uint32_t raw_b = base + L.sfb_raw + s * SFB_RAW_BYTES;
                 const uint32_t at_a = base + L.sfa + s * SF_ATOM_BYTES;
                 const uint32_t at_b = base + L.sfb + s * SF_ATOM_BYTES;
-                // A: rows lane, lane+32, lane+64, lane+96; 16 bytes = 4 K-steps each
-                uint4 ra[4];
+                // Rows handled by this lane: m = lane + 32 i (i = 0..3, so m / 32 = i).
+                // wa[i][j] / wb[i][j]: the scale word of row m for K-step j.
+                uint32_t wa[4][4], wb[4][4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) ra[i] = ld_shared_v4(raw_a + (lane + 32 * i) * 16);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    uint32_t w0 = (&ra[0].x)[j], w1 = (&ra[1].x)[j], w2 = (&ra[2].x)[j],
-                             w3 = (&ra[3].x)[j];
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(at_a + 512 * j + lane * 16),
-                                 "r"(w0), "r"(w1), "r"(w2), "r"(w3)
-                                 : "memory");
+                for (int i = 0; i < 4; ++i) {
+                    const uint4 v = ld_shared_v4(raw_a + (lane + 32 * i) * 16);
+                    wa[i][0] = v.x; wa[i][1] = v.y; wa[i][2] = v.z; wa[i][3] = v.w;
                 }
-                // B: one scale per 16x16 weight block, expanded to one per row
-                uint32_t wb[4][4];  // [i = row group][j = K-step]
                 if (!p.sfb_trans) {
                     // raw row y (16 bytes) = scales of rows n0+16y .. +15, 16 K-blocks
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        uint4 g = ld_shared_v4(raw_b + ((lane >> 4) + 2 * i) * 16);
+                        const uint4 g = ld_shared_v4(raw_b + ((lane >> 4) + 2 * i) * 16);
                         wb[i][0] = g.x; wb[i][1] = g.y; wb[i][2] = g.z; wb[i][3] = g.w;
                     }
                 } else {
@@ -343,11 +350,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                         }
                     }
                 }
+                // slab j (512 B) = K-step j: row (lane) at lane * 16 holds the
+                // words of rows lane + 32 i, i = 0..3
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(at_a + 512 * j + lane * 16),
+                                 "r"(wa[0][j]), "r"(wa[1][j]), "r"(wa[2][j]), "r"(wa[3][j]) : "memory");
                     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(at_b + 512 * j + lane * 16),
-                                 "r"(wb[0][j]), "r"(wb[1][j]), "r"(wb[2][j]), "r"(wb[3][j])
-                                 : "memory");
+                                 "r"(wb[0][j]), "r"(wb[1][j]), "r"(wb[2][j]), "r"(wb[3][j]) : "memory");
                 }
                 fence_proxy_async_smem();
                 __syncwarp();

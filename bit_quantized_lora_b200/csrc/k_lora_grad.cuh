@@ -7,8 +7,9 @@
 // Both are out[c, j] = sum_m T[m, c] S[m, j]: a reduction over the token
 // dimension, HBM-bound on reading T.  Each CTA takes 128 columns c and a
 // slice of m, runs tcgen05 kind::f16 with both operands MN-major straight
-// from the TMA tiles (T^T as A, S as B), and writes an FP32 partial;
-// k_lora_grad_reduce adds the slices in a fixed order.
+// from the TMA tiles (T^T as A, S as B), and writes an FP32 partial; the last
+// CTA of a column tile (completion counter) adds the slices in split order
+// into the output.
 #pragma once
 
 #include <cuda.h>
@@ -30,8 +31,10 @@ struct Params {
     CUtensorMap mapT[2];  // bf16 [M, C_z], box {64, 64}, 128 B swizzle
     CUtensorMap mapS[2];  // bf16 [M, r],   box {64, 64}, 128 B swizzle
     float* part[2];       // [splits, C_z, r_l]
+    float* out[2];        // dB [N, r_l], dA [K, r_l]
+    unsigned int* counters;  // [2][ctiles_max], zero on entry; left zero on exit
     int C[2];
-    int M, r_s, r_l, n_pad, mrows;
+    int M, r_s, r_l, n_pad, mrows, splits, ctiles_max;
 };
 
 constexpr uint32_t smem_bytes(int n_pad) {
@@ -55,6 +58,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_lora_grad(const __grid_const
     uint64_t* drain = accfull + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* last_flag = abort_flag + 1;
 
     const int warp = warp_id(), lane = lane_id();
     const int split = blockIdx.y;
@@ -153,25 +157,59 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_lora_grad(const __grid_const
                 if (j0 + k < p.r_l) out[j0 + k] = have ? __uint_as_float(v[k]) : 0.0f;
         }
     }
+    // every thread's partial writes become visible device-wide before the
+    // completion counter below is bumped
+    __threadfence();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
+    if (*abort_flag) return;
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned prev = atomicAdd(&p.counters[z * p.ctiles_max + blockIdx.x], 1u);
+        *last_flag = (prev == (unsigned)(p.splits - 1)) ? 1 : 0;
+    }
+    __syncthreads();
+    if (!*last_flag) return;
+    __threadfence();
+    // the tile's partials, 4 floats at a time, every split's load of a batch
+    // in flight together
+    const int n4 = BC * p.r_l / 4;
+    const int64_t stride4 = (int64_t)p.C[z] * p.r_l / 4;
+    const float4* part4 = reinterpret_cast<const float4*>(p.part[z]) + (int64_t)c0 * p.r_l / 4;
+    float4* out4 = reinterpret_cast<float4*>(p.out[z]) + (int64_t)c0 * p.r_l / 4;
+    constexpr int UNR = 4;
+    for (int i0 = threadIdx.x; i0 < n4; i0 += UNR * NUM_THREADS) {
+        float4 acc[UNR];
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int k = 0; k < p.splits; ++k) {
+            float4 v[UNR];
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const int i = i0 + u * NUM_THREADS;
+                v[u] = i < n4 ? __ldcg(part4 + k * stride4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                acc[u].x = __fadd_rn(acc[u].x, v[u].x);
+                acc[u].y = __fadd_rn(acc[u].y, v[u].y);
+                acc[u].z = __fadd_rn(acc[u].z, v[u].z);
+                acc[u].w = __fadd_rn(acc[u].w, v[u].w);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
+            const int i = i0 + u * NUM_THREADS;
+            if (i < n4) out4[i] = acc[u];
+        }
+    }
+    if (threadIdx.x == 0) p.counters[z * p.ctiles_max + blockIdx.x] = 0u;
 }
 
 }  // namespace lgrad
-
-// out[c, j] = sum over splits of part[split, c, j], in increasing split order.
-__global__ void __launch_bounds__(256) k_lora_grad_reduce(const float* __restrict__ part, int splits,
-                                                          int64_t n, float* __restrict__ out) {
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        float acc = 0.0f;
-        for (int k = 0; k < splits; ++k) acc = __fadd_rn(acc, part[(int64_t)k * n + i]);
-        out[i] = acc;
-    }
-}
 
 }  // namespace ft

@@ -22,9 +22,29 @@ __global__ void __launch_bounds__(256) k_amax_bf16(const uint16_t* __restrict__ 
                                                    unsigned int* __restrict__ out) {
     const int64_t vec_per_row = cols / 8;
     const int64_t total = rows * vec_per_row;
+    const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
     uint32_t m = 0;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-         i += (int64_t)gridDim.x * blockDim.x) {
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (ld == cols) {
+        // dense rows: four independent (predicated) 16-byte loads in flight
+        // per thread; the launch sizes the grid so one round covers the tensor
+        const uint4* xv = reinterpret_cast<const uint4*>(x);
+        for (; i < total; i += 4 * nthr) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                v[u] = (i + u * nthr < total) ? ld_nc_v4(xv + i + u * nthr) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                m = __vmaxu2(m, v[u].x & 0x7FFF7FFFu);
+                m = __vmaxu2(m, v[u].y & 0x7FFF7FFFu);
+                m = __vmaxu2(m, v[u].z & 0x7FFF7FFFu);
+                m = __vmaxu2(m, v[u].w & 0x7FFF7FFFu);
+            }
+        }
+        i = total;
+    }
+    for (; i < total; i += nthr) {
         int64_t r = i / vec_per_row, c = i - r * vec_per_row;
         uint4 v = ld_nc_v4(x + r * ld + c * 8);
         m = __vmaxu2(m, v.x & 0x7FFF7FFFu);
@@ -46,29 +66,43 @@ __global__ void __launch_bounds__(256) k_amax_bf16(const uint16_t* __restrict__ 
 }
 
 // ------------------------------------------------------- 1x16 row-wise
-// One thread per 16-element block of a row.  Loads are two 16-byte vectors,
-// stores are 8 bytes of codes and one scale byte; consecutive threads touch
-// consecutive blocks, so every access is coalesced.
+// Two 16-element blocks per thread per iteration (four 16-byte loads in
+// flight); stores are 8 bytes of codes and one scale byte per block;
+// consecutive threads touch consecutive blocks, so accesses are coalesced.
 __global__ void __launch_bounds__(256) k_quant_1x16(const uint16_t* __restrict__ x, int64_t rows,
                                                     int64_t cols, int64_t ld,
                                                     const float* __restrict__ amax,
                                                     uint8_t* __restrict__ codes,
                                                     uint8_t* __restrict__ scales,
                                                     float* __restrict__ tscale) {
-    const QTensor t = make_qtensor(*amax);
+    __shared__ QTable tab;
+    const QTensorFast t = make_qtensor_fast(*amax);
+    build_qtable(tab, t.g, threadIdx.x, blockDim.x);
+    __syncthreads();
     if (blockIdx.x == 0 && threadIdx.x == 0) *tscale = t.g;
     const int64_t nb = cols / 16;
     const int64_t total = rows * nb;
-    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < total;
-         b += (int64_t)gridDim.x * blockDim.x) {
-        int64_t r = b / nb, c = b - r * nb;
+    const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < total; b += 2 * nthr) {
+        const int64_t b2 = b + nthr;
+        const bool two = b2 < total;
+        const int64_t r = b / nb, c = b - r * nb;
+        const int64_t r2 = two ? b2 / nb : r, c2 = two ? b2 - r2 * nb : c;
         const uint16_t* p = x + r * ld + c * 16;
-        uint4 v0 = ld_nc_v4(p), v1 = ld_nc_v4(p + 8);
+        const uint16_t* p2 = x + r2 * ld + c2 * 16;
+        const uint4 v0 = ld_nc_v4(p), v1 = ld_nc_v4(p + 8);
+        const uint4 u0 = ld_nc_v4(p2), u1 = ld_nc_v4(p2 + 8);
         uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
         uint32_t s;
-        uint2 q = quant_block16(w, t, s);
+        const uint2 q = quant_block16_fast(w, t, tab, s);
         *reinterpret_cast<uint2*>(codes + r * (cols / 2) + c * 8) = q;
         scales[r * nb + c] = (uint8_t)s;
+        if (two) {
+            uint32_t w2[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+            const uint2 q2 = quant_block16_fast(w2, t, tab, s);
+            *reinterpret_cast<uint2*>(codes + r2 * (cols / 2) + c2 * 8) = q2;
+            scales[r2 * nb + c2] = (uint8_t)s;
+        }
     }
 }
 

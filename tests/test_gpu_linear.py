@@ -146,3 +146,22 @@ def test_empty_batch_is_a_no_op():
     torch.cuda.synchronize()
     assert Y.shape == (0, 256) and dX.shape == (0, 256)
     assert not dA.any() and not dB.any()
+
+
+def test_repeated_runs_are_bitwise_identical():
+    """Every reduction (split down-projection, adapter gradients, amax) adds
+    in a fixed order, so repeated forward/backward passes must agree bit for
+    bit; a cross-CTA ordering race would show up here."""
+    inp, U, V, Wr, layer = _prep(ft_synth.ATTN, 21)
+    X, dY = dev_bf16(inp["X"]), dev_bf16(inp["dY"])
+    ref = None
+    for _ in range(6):
+        Y, P = ft.ft_linear_fwd(layer, X, out_dtype=ft.F32)
+        dX, dA, dB = ft.ft_linear_bwd(layer, dY, X, P, out_dtype=ft.F32)
+        torch.cuda.synchronize()
+        outs = [t.clone() for t in (Y, P, dX, dA, dB)]
+        if ref is None:
+            ref = outs
+        else:
+            for a, b in zip(outs, ref):
+                assert torch.equal(a, b)
