@@ -102,6 +102,16 @@ def ft_quantize_workspace_bytes() -> int:
     return load().ft_quantize_workspace_bytes()
 
 
+def ft_workspace_qact(M: int, N: int, K: int, r_s: int, r_l: int) -> tuple[int, int, int]:
+    """Byte offsets (codes, scales, tensor scale) of the quantized
+    activation that ft_linear_fwd (Q(X)) or ft_linear_bwd (Q(dY)) leaves in
+    its workspace."""
+    c, s, g = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    check("ft_workspace_qact", load().ft_workspace_qact(M, N, K, r_s, r_l, ctypes.byref(c),
+                                                        ctypes.byref(s), ctypes.byref(g)))
+    return c.value, s.value, g.value
+
+
 def ft_quantize(x: torch.Tensor, blk: int = BLK_1x16, amax: torch.Tensor | None = None,
                 out: FP4 | None = None, ws: Workspace | None = None, stream=None) -> FP4:
     """Q(x): NVFP4 block quantization of a 2-D bf16 CUDA tensor."""

@@ -51,6 +51,9 @@ SIGNATURES = {
                                      ctypes.c_int, c_vp, c_vp, c_vp, ctypes.c_size_t, c_vp]),
     "ft_workspace_bytes": (ctypes.c_size_t, [c_i64, c_i64, c_i64, c_i64, c_i64]),
     "ft_quantize_workspace_bytes": (ctypes.c_size_t, []),
+    "ft_workspace_qact": (ctypes.c_int, [c_i64, c_i64, c_i64, c_i64, c_i64,
+                                         ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t),
+                                         ctypes.POINTER(ctypes.c_size_t)]),
     "ft_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int), c_vp]),
     "ft_status_str": (ctypes.c_char_p, [ctypes.c_int]),
     "ft_linear_fwd_noalloc": (ctypes.c_int, [ctypes.POINTER(FtLinear), c_vp, c_i64, c_vp, c_vp,

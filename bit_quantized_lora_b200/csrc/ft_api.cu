@@ -18,6 +18,7 @@
 #include "k_gemm_fp4.cuh"
 #include "k_lora_grad.cuh"
 #include "k_qdown.cuh"
+#include "k_qres.cuh"
 #include "k_quant.cuh"
 
 namespace {
@@ -30,6 +31,7 @@ struct DevInfo {
     bool ok = false;
     int sms = 0;
     bool attr_set = false;
+    int qres_ctas = 0;  // CTAs of k_qres that fit on the device at once
 };
 DevInfo g_dev[64];
 std::mutex g_mu;
@@ -67,8 +69,18 @@ ft_status device_info(DevInfo** out) {
             cudaFuncSetAttribute(ft::qdown::k_qdown, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)ft::qdown::SMEM_BYTES) != cudaSuccess ||
             cudaFuncSetAttribute(ft::lgrad::k_lora_grad, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)ft::lgrad::smem_bytes(128)) != cudaSuccess)
+                                 (int)ft::lgrad::smem_bytes(128)) != cudaSuccess ||
+            cudaFuncSetAttribute(ft::qres::k_qres, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 big) != cudaSuccess)
             return FT_ERR_CUDA;
+        // the resident quantizer's grid barrier needs every CTA resident at
+        // once; size its grids by the occupancy at its largest footprint
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                &per_sm, ft::qres::k_qres, ft::qres::NUM_THREADS,
+                ft::qres::make_layout(ft::qres::MAX_ST, 1).total) != cudaSuccess)
+            return FT_ERR_CUDA;
+        d.qres_ctas = per_sm * d.sms;
         d.attr_set = true;
     }
     *out = &d;
@@ -101,11 +113,12 @@ enum KernelId {
     KID_GEMM,
     KID_LORA_GRAD,
     KID_LORA_REDUCE,
+    KID_QRES,
     KID_COUNT
 };
 const char* const kKernelNames[KID_COUNT] = {
     "k_amax_bf16", "k_quant_1x16", "k_quant_tile16", "k_pack_lt", "k_qdown",
-    "k_lowrank_finalize", "k_gemm_fp4", "k_lora_grad", "k_lora_grad_reduce"};
+    "k_lowrank_finalize", "k_gemm_fp4", "k_lora_grad", "k_lora_grad_reduce", "k_qres"};
 
 struct TimingRec {
     cudaEvent_t a, b;
@@ -173,6 +186,10 @@ constexpr int LG_MAX_SPLITS = 16;
 struct WsPlan {
     size_t amax, gact, codes, scales, lt, part, pg, lgpart, counters, total;
     int n_qd_counters, lg_ctiles, n_counters;
+    // counters region: [0] tensor-amax bits and [1] grid-barrier arrivals of
+    // the resident quantizer, then the row-tile counters of the fused
+    // quantize/down-projection, then the adapter-gradient tile counters
+    int qd_cnt, lg_cnt;
 };
 
 WsPlan plan_ws(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t r_l) {
@@ -192,7 +209,9 @@ WsPlan plan_ws(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t r_l) {
     // one per (gradient, column tile) of the adapter gradients
     w.n_qd_counters = (int)((M + 127) / 128);
     w.lg_ctiles = (int)((C + 127) / 128);
-    w.n_counters = w.n_qd_counters + 2 * w.lg_ctiles;
+    w.qd_cnt = 2;
+    w.lg_cnt = 2 + w.n_qd_counters;
+    w.n_counters = 2 + w.n_qd_counters + 2 * w.lg_ctiles;
     w.counters = o; o += up256((size_t)w.n_counters * 4);
     w.total = o;
     return w;
@@ -298,7 +317,7 @@ ft_status run_qdown(const void* T, int64_t M, int64_t C, const void* L1, int64_t
     p.scales = scales;
     p.part = part;
     p.P = static_cast<__nv_bfloat16*>(P);
-    p.counters = counters;
+    p.counters = counters + w.qd_cnt;
     p.M = (int)M;
     p.C = (int)C;
     p.r = (int)r;
@@ -314,6 +333,137 @@ ft_status run_qdown(const void* T, int64_t M, int64_t C, const void* L1, int64_t
         _lt.stop();
     }
     return last_launch();
+}
+
+// Grid of the resident quantizer for T [M, C]: 128-row tiles x C-splits of
+// at most 768 columns; false when it does not fit the device at once.
+bool qres_grid(int64_t M, int64_t C, const DevInfo* d, int* mt, int* splits, int* cchunk) {
+    namespace Q = ft::qres;
+    if (C % Q::BKC) return false;
+    *mt = cdiv(M, Q::BM);
+    int sp = std::max(1, std::min(QD_MAX_SPLITS, d->sms / std::max(1, *mt)));
+    sp = std::max(sp, cdiv(C, (int64_t)Q::MAX_ST * Q::BKC));
+    *cchunk = cdiv(C, (int64_t)sp * Q::BKC) * Q::BKC;
+    *splits = cdiv(C, *cchunk);
+    return *splits <= QD_MAX_SPLITS && *cchunk <= Q::MAX_ST * Q::BKC &&
+           (int64_t)(*mt) * (*splits) <= d->qres_ctas;
+}
+
+// Launches k_qres; cooperative (all CTAs co-resident) when it computes the
+// tensor amax itself, since its grid barrier waits on every CTA.
+ft_status launch_qres(const ft::qres::Params& p, int mt, int splits, cudaStream_t st) {
+    namespace Q = ft::qres;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)mt, (unsigned)splits, 1);
+    cfg.blockDim = dim3(Q::NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = Q::make_layout(p.cchunk / Q::BKC, p.do_mma).total;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = p.amax_in ? 0 : 1;
+    {
+        LaunchTimer _lt(KID_QRES, st);
+        FT_TRY(cuda_ok(cudaLaunchKernelEx(&cfg, Q::k_qres, p)));
+        _lt.stop();
+    }
+    return last_launch();
+}
+
+// Q(T), g_T and P = [bf16(T L1) | bf16(s T L2)] for T [M, C], with the
+// tensor amax computed on the way (amax_in == null) or taken from the caller.
+// When the CTAs' chunks fit in shared memory all at once, one cooperative
+// launch of k_qres reads T from HBM once; otherwise the amax pass (if
+// needed) is followed by k_qdown (or the plain 1x16 quantizer when r == 0).
+ft_status run_quant_down(const void* T, int64_t M, int64_t C, const void* L1, int64_t r1,
+                         const void* L2, int64_t r2, float s, const float* amax_in, uint8_t* codes,
+                         uint8_t* scales, float* tscale, void* P, uint8_t* ws, const WsPlan& w,
+                         const DevInfo* d, cudaStream_t st) {
+    namespace Q = ft::qres;
+    const int64_t r = r1 + r2;
+    int mt = 0, splits = 0, cchunk = 0;
+    if (!qres_grid(M, C, d, &mt, &splits, &cchunk)) {
+        const float* a = amax_in;
+        if (!a) {
+            FT_TRY(run_amax(T, M, C, C, reinterpret_cast<float*>(ws + w.amax), d, st));
+            a = reinterpret_cast<float*>(ws + w.amax);
+        }
+        return run_qdown(T, M, C, L1, r1, L2, r2, s, a, codes, scales, tscale, P, ws, w, d, st);
+    }
+    unsigned int* counters = reinterpret_cast<unsigned int*>(ws + w.counters);
+    FT_TRY(cuda_ok(cudaMemsetAsync(counters, 0, (size_t)w.n_counters * 4, st)));
+    Q::Params p;
+    std::memset(&p, 0, sizeof(p));
+    p.do_mma = r > 0 ? 1 : 0;
+    p.direct = (r1 <= 64 && r2 <= 64) ? 1 : 0;
+    if (p.do_mma && p.direct) {
+        if (r1 > 0)
+            FT_TRY(encode_2d(&p.mapL1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1, r1, C, r1 * 2, 64, 64,
+                             CU_TENSOR_MAP_SWIZZLE_128B));
+        if (r2 > 0)
+            FT_TRY(encode_2d(&p.mapL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2, r2, C, r2 * 2, 64, 64,
+                             CU_TENSOR_MAP_SWIZZLE_128B));
+    } else if (p.do_mma) {
+        uint16_t* Lt = reinterpret_cast<uint16_t*>(ws + w.lt);
+        dim3 grid((unsigned)cdiv(C, 256), 128);
+        {
+            LaunchTimer _lt(KID_PACK_LT, st);
+            ft::k_pack_lt<<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(L1), (int)r1,
+                                                static_cast<const uint16_t*>(L2), (int)r2, (int)C, Lt);
+            _lt.stop();
+        }
+        FT_TRY(last_launch());
+        FT_TRY(encode_2d(&p.mapL1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Lt, C, 128, C * 2, 64, 128,
+                         CU_TENSOR_MAP_SWIZZLE_128B));
+    }
+    FT_TRY(encode_2d(&p.mapT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, C, M, C * 2, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B));
+    p.amax_in = amax_in;
+    p.amax_bits = counters;
+    p.arrivals = counters + 1;
+    p.tscale = tscale;
+    p.codes = codes;
+    p.scales = scales;
+    p.part = reinterpret_cast<float*>(ws + w.part);
+    p.P = static_cast<__nv_bfloat16*>(P);
+    p.counters = counters + w.qd_cnt;
+    p.M = (int)M;
+    p.C = (int)C;
+    p.r = (int)r;
+    p.r1 = (int)r1;
+    p.cchunk = cchunk;
+    p.splits = splits;
+    p.s = s;
+    p.num_ctas = (unsigned)(mt * splits);
+    return launch_qres(p, mt, splits, st);
+}
+
+// 1x16 quantization of a dense T [M, C] through the resident kernel (no
+// down-projection).  sync: two zeroed words when amax_in is null.
+ft_status run_quant_1x16_resident(const void* T, int64_t M, int64_t C, const float* amax_in,
+                                  unsigned int* sync, uint8_t* codes, uint8_t* scales,
+                                  float* tscale, int mt, int splits, int cchunk, cudaStream_t st) {
+    namespace Q = ft::qres;
+    if (!amax_in) FT_TRY(cuda_ok(cudaMemsetAsync(sync, 0, 2 * sizeof(unsigned int), st)));
+    Q::Params p;
+    std::memset(&p, 0, sizeof(p));
+    FT_TRY(encode_2d(&p.mapT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, C, M, C * 2, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B));
+    p.amax_in = amax_in;
+    p.amax_bits = sync;
+    p.arrivals = sync ? sync + 1 : nullptr;
+    p.tscale = tscale;
+    p.codes = codes;
+    p.scales = scales;
+    p.M = (int)M;
+    p.C = (int)C;
+    p.cchunk = cchunk;
+    p.splits = splits;
+    p.s = 1.0f;
+    p.num_ctas = (unsigned)(mt * splits);
+    return launch_qres(p, mt, splits, st);
 }
 
 // out[M, Nout] = ga gb Q(A) Q(B)^T + P[:, :r1] L1^T + P[:, r1:] L2^T
@@ -391,7 +541,7 @@ ft_status run_lora_grads(const void* dY, const void* X, const void* P, const voi
     p.part[1] = partA;
     p.out[0] = dB;
     p.out[1] = dA;
-    p.counters = reinterpret_cast<unsigned int*>(ws + w.counters) + w.n_qd_counters;
+    p.counters = reinterpret_cast<unsigned int*>(ws + w.counters) + w.lg_cnt;
     p.C[0] = (int)N;
     p.C[1] = (int)K;
     p.M = (int)M;
@@ -465,6 +615,17 @@ size_t ft_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t 
     return plan_ws(M, N, K, r_s, r_l).total;
 }
 
+ft_status ft_workspace_qact(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t r_l,
+                            size_t* codes_off, size_t* scales_off, size_t* tscale_off) {
+    if (M < 0 || N < 0 || K < 0 || r_s < 0 || r_l < 0) return FT_ERR_INVALID_ARG;
+    if (!codes_off || !scales_off || !tscale_off) return FT_ERR_INVALID_ARG;
+    const WsPlan w = plan_ws(M, N, K, r_s, r_l);
+    *codes_off = w.codes;
+    *scales_off = w.scales;
+    *tscale_off = w.gact;
+    return FT_OK;
+}
+
 ft_status ft_device_error(int* code, void* stream) {
     if (!code) return FT_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -496,6 +657,10 @@ ft_status ft_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, ft_
     DevInfo* d;
     FT_TRY(device_info(&d));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int mt = 0, splits = 0, cchunk = 0;
+    if (blk == FT_BLK_1x16 && ld == cols && qres_grid(rows, cols, d, &mt, &splits, &cchunk))
+        return run_quant_1x16_resident(x, rows, cols, amax, static_cast<unsigned int*>(ws),
+                                       out->codes, out->scales, out->tscale, mt, splits, cchunk, st);
     const float* a = amax;
     if (!a) {
         float* slot = static_cast<float*>(ws);
@@ -565,15 +730,10 @@ ft_status ft_linear_fwd(const ft_linear* L, const void* X, int64_t M, const floa
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     float* g_x = reinterpret_cast<float*>(wsb + w.gact);
-    const float* a = amax_x;
-    if (!a) {
-        FT_TRY(run_amax(X, M, L->K, L->K, reinterpret_cast<float*>(wsb + w.amax), d, st));
-        a = reinterpret_cast<float*>(wsb + w.amax);
-    }
     uint8_t* codes = wsb + w.codes;
     uint8_t* scales = wsb + w.scales;
-    FT_TRY(run_qdown(X, M, L->K, L->U, L->r_s, L->A, L->r_l, L->s, a, codes, scales, g_x, P_save,
-                     wsb, w, d, st));
+    FT_TRY(run_quant_down(X, M, L->K, L->U, L->r_s, L->A, L->r_l, L->s, amax_x, codes, scales, g_x,
+                          P_save, wsb, w, d, st));
     return run_gemm(codes, scales, g_x, M, L->K, L->w_k.codes, L->w_k.scales, L->w_k.tscale, L->N,
                     false, L->N / 16, L->K / 16, P_save, L->V, L->r_s, L->B, L->r_l, Y, yt, d, st);
 }
@@ -608,16 +768,11 @@ ft_status ft_linear_bwd(const ft_linear* L, const void* dY, const void* X, const
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     float* g_dy = reinterpret_cast<float*>(wsb + w.gact);
-    const float* a = amax_dy;
-    if (!a) {
-        FT_TRY(run_amax(dY, M, L->N, L->N, reinterpret_cast<float*>(wsb + w.amax), d, st));
-        a = reinterpret_cast<float*>(wsb + w.amax);
-    }
     uint8_t* codes = wsb + w.codes;
     uint8_t* scales = wsb + w.scales;
     void* Pg = wsb + w.pg;
-    FT_TRY(run_qdown(dY, M, L->N, L->V, L->r_s, L->B, L->r_l, L->s, a, codes, scales, g_dy, Pg, wsb,
-                     w, d, st));
+    FT_TRY(run_quant_down(dY, M, L->N, L->V, L->r_s, L->B, L->r_l, L->s, amax_dy, codes, scales, g_dy,
+                          Pg, wsb, w, d, st));
     FT_TRY(run_gemm(codes, scales, g_dy, M, L->N, L->w_n.codes, L->w_k.scales, L->w_k.tscale, L->K,
                     true, L->N / 16, L->K / 16, Pg, L->U, L->r_s, L->A, L->r_l, dX, xt, d, st));
     if (L->r_l > 0)

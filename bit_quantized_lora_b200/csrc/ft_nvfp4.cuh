@@ -254,10 +254,13 @@ __device__ __forceinline__ uint32_t encode8_fast(uint32_t w0, uint32_t w1, uint3
     return out;
 }
 
-// One 1x16 block through the table.  Returns the 8 code bytes; *sbyte the scale.
-__device__ __forceinline__ uint2 quant_block16_fast(const uint32_t (&w)[8], const QTensorFast& t,
-                                                    const QTable& tab, uint32_t& sbyte) {
-    const float amax_b = __uint_as_float(amax_bits_16(w));
+// One 1x16 block through the table, its max|x| given as float bits
+// (amax_bits_16 of the same block).  Returns the 8 code bytes; *sbyte the
+// scale.
+__device__ __forceinline__ uint2 quant_block16_fast_m(const uint32_t (&w)[8], uint32_t amax_bits,
+                                                      const QTensorFast& t, const QTable& tab,
+                                                      uint32_t& sbyte) {
+    const float amax_b = __uint_as_float(amax_bits);
     sbyte = scale_byte_fast(amax_b, t);
     const float d = tab.d[sbyte];
     const float y = tab.y[sbyte];
@@ -275,6 +278,12 @@ __device__ __forceinline__ uint2 quant_block16_fast(const uint32_t (&w)[8], cons
         r.y = encode8(w[4], w[5], w[6], w[7], d, 0.0f, false);
     }
     return r;
+}
+
+// One 1x16 block through the table.  Returns the 8 code bytes; *sbyte the scale.
+__device__ __forceinline__ uint2 quant_block16_fast(const uint32_t (&w)[8], const QTensorFast& t,
+                                                    const QTable& tab, uint32_t& sbyte) {
+    return quant_block16_fast_m(w, amax_bits_16(w), t, tab, sbyte);
 }
 
 }  // namespace ft

@@ -34,6 +34,7 @@ enum : int {
     ERR_WAIT_ACC_EMPTY = 5,
     ERR_WAIT_LR = 6,
     ERR_WAIT_DRAIN = 7,
+    ERR_GRID_SYNC = 8,
 };
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
@@ -248,6 +249,22 @@ __host__ __device__ constexpr uint32_t idesc_nvfp4(int M, int N) {
            | ((uint32_t)(N >> 3) << 17)  // N / 8
            | (0u << 23)                  // scale format UE4M3
            | ((uint32_t)(M >> 4) << 24); // M / 16
+}
+
+// ---------------------------------------------------------------- grid-wide flags
+__device__ __forceinline__ void red_add_release_gpu(unsigned int* p, unsigned int v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Named barrier over `nthreads` threads (a multiple of 32) with id `id`
+// (0 is __syncthreads' barrier).
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // ---------------------------------------------------------------- misc

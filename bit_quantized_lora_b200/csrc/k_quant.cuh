@@ -17,25 +17,26 @@ namespace ft {
 // block reduces its share and folds it into *out with an integer atomicMax on
 // the float bits (non-negative floats order like their bit patterns), so the
 // result is exact and independent of scheduling.  *out must be 0 on entry.
+// The grid is kept to a few blocks per SM (same-address atomics serialise in
+// L2); each thread keeps eight independent 16-byte loads in flight.
 __global__ void __launch_bounds__(256) k_amax_bf16(const uint16_t* __restrict__ x, int64_t rows,
                                                    int64_t cols, int64_t ld,
                                                    unsigned int* __restrict__ out) {
+    constexpr int U = 8;
     const int64_t vec_per_row = cols / 8;
     const int64_t total = rows * vec_per_row;
     const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
     uint32_t m = 0;
     int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (ld == cols) {
-        // dense rows: four independent (predicated) 16-byte loads in flight
-        // per thread; the launch sizes the grid so one round covers the tensor
         const uint4* xv = reinterpret_cast<const uint4*>(x);
-        for (; i < total; i += 4 * nthr) {
-            uint4 v[4];
+        for (; i < total; i += U * nthr) {
+            uint4 v[U];
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
+            for (int u = 0; u < U; ++u)
                 v[u] = (i + u * nthr < total) ? ld_nc_v4(xv + i + u * nthr) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < U; ++u) {
                 m = __vmaxu2(m, v[u].x & 0x7FFF7FFFu);
                 m = __vmaxu2(m, v[u].y & 0x7FFF7FFFu);
                 m = __vmaxu2(m, v[u].z & 0x7FFF7FFFu);

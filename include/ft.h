@@ -160,6 +160,21 @@ ft_status ft_linear_bwd(const ft_linear* L, const void* dY, const void* X, const
 size_t ft_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t r_l);
 size_t ft_quantize_workspace_bytes(void);
 
+/* ft_workspace_qact -- where the quantized activation of the last
+ * ft_linear_fwd / ft_linear_bwd call lies inside its workspace (byte
+ * offsets from the workspace start, for the same M, N, K, r_s, r_l).  Once
+ * the call's work has finished on its stream, the workspace holds Q(X) after
+ * a forward and Q(dY) after a backward, in the layout of an FT_BLK_1x16
+ * ft_fp4 view: codes [M, C/2] at *codes_off, scales [M, C/16] at
+ * *scales_off, the tensor scale (one float) at *tscale_off, C = K after a
+ * forward and N after a backward.  It is the operand of the 4-bit GEMM
+ * (section 3.1, Eq. 2 / section 3.2, Eq. 3), the same bytes ft_quantize
+ * would produce; a caller may reuse it (e.g. for a quantized weight
+ * gradient) until its next call on the workspace.  Pure host arithmetic.
+ * FT_ERR_INVALID_ARG for negative sizes or null outputs.                  */
+ft_status ft_workspace_qact(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t r_l,
+                            size_t* codes_off, size_t* scales_off, size_t* tscale_off);
+
 /* Reads and clears the device error word of the current device (a host-
  * synchronous copy on `stream`).  *code receives 0 when no kernel reported a
  * failure; otherwise a nonzero code naming the wait that ran out.  Returns

@@ -116,3 +116,20 @@ def test_linear_validation_happens_on_the_host(L):
     assert L.ft_linear_fwd(ctypes.byref(ok), x, 0, None, x, 0, x, x, ws, None) == FT_OK
     assert L.ft_linear_bwd(ctypes.byref(bad_n), x, x, x, 128, None, x, 0, x, x, x, ws, None) == FT_ERR_SHAPE
     assert L.ft_linear_bwd(ctypes.byref(ok), x, x, x, 128, None, x, 9, x, x, x, ws, None) == FT_ERR_INVALID_ARG
+
+
+def test_workspace_qact_offsets_lie_inside_the_workspace(L):
+    for M, N, K, rs, rl in [(4608, 3072, 3072, 32, 16), (128, 256, 256, 16, 16), (37, 512, 256, 0, 0)]:
+        c, s, g = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+        assert L.ft_workspace_qact(M, N, K, rs, rl, ctypes.byref(c), ctypes.byref(s), ctypes.byref(g)) == FT_OK
+        total = L.ft_workspace_bytes(M, N, K, rs, rl)
+        C = max(N, K)
+        # codes, scales and the tensor scale do not overlap and fit the workspace
+        spans = sorted([(c.value, M * C // 2), (s.value, M * C // 16), (g.value, 4)])
+        for (a, n), (b, _) in zip(spans, spans[1:]):
+            assert a + n <= b
+        assert spans[-1][0] + spans[-1][1] <= total
+        assert c.value % 16 == 0 and s.value % 16 == 0
+    bad = ctypes.c_size_t()
+    assert L.ft_workspace_qact(-1, 1, 1, 0, 0, ctypes.byref(bad), ctypes.byref(bad), ctypes.byref(bad)) == FT_ERR_INVALID_ARG
+    assert L.ft_workspace_qact(1, 1, 1, 0, 0, None, ctypes.byref(bad), ctypes.byref(bad)) == FT_ERR_INVALID_ARG

@@ -165,3 +165,56 @@ def test_repeated_runs_are_bitwise_identical():
         else:
             for a, b in zip(outs, ref):
                 assert torch.equal(a, b)
+
+
+def _ws_qact(ws, M, N, K, r_s, r_l, C):
+    co, so, go = ft.ft_workspace_qact(M, N, K, r_s, r_l)
+    raw = ws.buf
+    assert raw.numel() >= ft.ft_workspace_bytes(M, N, K, r_s, r_l)
+    codes = host(raw[co:co + M * C // 2]).reshape(M, C // 2)
+    scales = host(raw[so:so + M * C // 16]).reshape(M, C // 16)
+    g = host(raw[go:go + 4]).view(np.float32)[0]
+    return codes, scales, g
+
+
+@pytest.mark.parametrize("case", ["tiny", "attn", "ragged300", "packed16_112", "rank0", "amax_given"])
+def test_fused_quantizer_output_is_bit_exact(case):
+    """The operand the 4-bit GEMM consumes, Q(X) after the forward and Q(dY)
+    after the backward, read back from the workspace: codes, scales and the
+    tensor scale equal the oracle's bit for bit (integer work).  Covers the
+    single-pass resident path with its grid-wide amax (attention shape), the
+    split reductions, a ragged token count, the packed-factor mode (a rank
+    above 64), no low-rank branch, and a caller-supplied amax."""
+    shape, seed, M, r_s, r_l, amax = ft_synth.TINY, 50, None, None, None, None
+    if case == "attn":
+        shape, seed = ft_synth.ATTN, 51
+    elif case == "ragged300":
+        M = 300
+    elif case == "packed16_112":
+        M, r_s, r_l = 256, 16, 112
+    elif case == "rank0":
+        M, r_s, r_l = 256, 0, 0
+    elif case == "amax_given":
+        amax = 7.25
+    inp, U, V, Wr, layer = _prep(shape, seed, M, r_s, r_l)
+    X, dY = inp["X"], inp["dY"]
+    Mr = X.shape[0]
+    ws = ft.Workspace()
+    Y, P = ft.ft_linear_fwd(layer, dev_bf16(X), out_dtype=ft.F32, ws=ws,
+                            amax_x=None if amax is None else scalar_dev(amax))
+    torch.cuda.synchronize()
+    assert ft.ft_device_error() == 0
+    codes, scales, g = _ws_qact(ws, Mr, layer.N, layer.K, layer.r_s, layer.r_l, layer.K)
+    rc, rs_, rg = oracle.quantize_1x16(X, amax)
+    assert np.float32(g) == np.float32(rg)
+    np.testing.assert_array_equal(scales, rs_)
+    np.testing.assert_array_equal(codes, rc)
+    ft.ft_linear_bwd(layer, dev_bf16(dY), dev_bf16(X), P, out_dtype=ft.F32, ws=ws,
+                     amax_dy=None if amax is None else scalar_dev(amax))
+    torch.cuda.synchronize()
+    assert ft.ft_device_error() == 0
+    codes, scales, g = _ws_qact(ws, Mr, layer.N, layer.K, layer.r_s, layer.r_l, layer.N)
+    rc, rs_, rg = oracle.quantize_1x16(dY, amax)
+    assert np.float32(g) == np.float32(rg)
+    np.testing.assert_array_equal(scales, rs_)
+    np.testing.assert_array_equal(codes, rc)
