@@ -77,8 +77,7 @@ ft_status device_info(DevInfo** out) {
         // once; size its grids by the occupancy at its largest footprint
         int per_sm = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-                &per_sm, ft::qres::k_qres, ft::qres::NUM_THREADS,
-                ft::qres::make_layout(ft::qres::MAX_ST, 1).total) != cudaSuccess)
+                &per_sm, ft::qres::k_qres, ft::qres::NUM_THREADS, ft::qres::SMEM_LIMIT) != cudaSuccess)
             return FT_ERR_CUDA;
         d.qres_ctas = per_sm * d.sms;
         d.attr_set = true;
@@ -335,18 +334,58 @@ ft_status run_qdown(const void* T, int64_t M, int64_t C, const void* L1, int64_t
     return last_launch();
 }
 
-// Grid of the resident quantizer for T [M, C]: 128-row tiles x C-splits of
-// at most 768 columns; false when it does not fit the device at once.
-bool qres_grid(int64_t M, int64_t C, const DevInfo* d, int* mt, int* splits, int* cchunk) {
+// Factor tile of the resident quantizer for a rank rf: boxes of 16, 32 or
+// 64 columns (swizzle = the box's row bytes), two 64-wide atoms above 64.
+ft::qres::Factor qres_factor(int64_t rf) {
+    ft::qres::Factor f;
+    std::memset(&f, 0, sizeof(f));
+    f.rf = (int)rf;
+    if (rf <= 0) return f;
+    f.wbox = rf <= 16 ? 16 : rf <= 32 ? 32 : 64;
+    f.natoms = rf <= 64 ? 1 : 2;
+    f.sbo = 8u * (uint32_t)f.wbox * 2u;
+    f.swz = f.wbox == 16 ? ft::SWZ_32B : f.wbox == 32 ? ft::SWZ_64B : ft::SWZ_128B;
+    return f;
+}
+uint32_t qres_factor_bytes(const ft::qres::Factor& f) {
+    return f.rf > 0 ? (uint32_t)f.natoms * 64u * (uint32_t)f.wbox * 2u : 0u;
+}
+
+// Ring of factor tiles: as many stages of both tiles as fit in 31 KiB (the
+// room left beside 12 resident 16 KiB stages; at least 2 stages), and at
+// least the 6 KiB the staged scales need.
+void qres_ring(ft::qres::Params& p) {
     namespace Q = ft::qres;
-    if (C % Q::BKC) return false;
+    p.f1.off = 0;
+    p.f2.off = qres_factor_bytes(p.f1);
+    p.fstage_bytes = qres_factor_bytes(p.f1) + qres_factor_bytes(p.f2);
+    p.fs = 2;
+    if (p.fstage_bytes > 0)
+        p.fs = (int)std::max<uint32_t>(2u, std::min<uint32_t>((uint32_t)Q::MAX_FS, 31744u / p.fstage_bytes));
+    p.ring_bytes = std::max<uint32_t>((uint32_t)p.fs * p.fstage_bytes, Q::BM * Q::SROW);
+    p.ring_bytes = (p.ring_bytes + 1023u) & ~1023u;
+}
+
+// Grid of the resident quantizer for T [M, C]: 128-row tiles x C-splits of
+// at most max_st 64-column stages; false when the chunks do not all fit on
+// the device at once.
+bool qres_grid(int64_t M, int64_t C, int max_st, const DevInfo* d, int* mt, int* splits, int* cchunk) {
+    namespace Q = ft::qres;
+    if (C % Q::BKC || max_st < 1) return false;
     *mt = cdiv(M, Q::BM);
     int sp = std::max(1, std::min(QD_MAX_SPLITS, d->sms / std::max(1, *mt)));
-    sp = std::max(sp, cdiv(C, (int64_t)Q::MAX_ST * Q::BKC));
+    sp = std::max(sp, cdiv(C, (int64_t)max_st * Q::BKC));
     *cchunk = cdiv(C, (int64_t)sp * Q::BKC) * Q::BKC;
     *splits = cdiv(C, *cchunk);
-    return *splits <= QD_MAX_SPLITS && *cchunk <= Q::MAX_ST * Q::BKC &&
+    return *splits <= QD_MAX_SPLITS && *cchunk <= max_st * Q::BKC &&
            (int64_t)(*mt) * (*splits) <= d->qres_ctas;
+}
+
+// Resident stages that fit next to the ring, the table and the barriers.
+int qres_max_stages(uint32_t ring_bytes) {
+    namespace Q = ft::qres;
+    const int64_t avail = (int64_t)Q::SMEM_LIMIT - Q::make_layout(0, ring_bytes).total;
+    return (int)std::min<int64_t>(Q::MAX_ST, std::max<int64_t>(0, avail / Q::TILE_BYTES));
 }
 
 // Launches k_qres; cooperative (all CTAs co-resident) when it computes the
@@ -357,7 +396,7 @@ ft_status launch_qres(const ft::qres::Params& p, int mt, int splits, cudaStream_
     std::memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3((unsigned)mt, (unsigned)splits, 1);
     cfg.blockDim = dim3(Q::NUM_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = Q::make_layout(p.cchunk / Q::BKC, p.do_mma).total;
+    cfg.dynamicSmemBytes = Q::make_layout(p.cchunk / Q::BKC, p.ring_bytes).total;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeCooperative;
@@ -383,8 +422,14 @@ ft_status run_quant_down(const void* T, int64_t M, int64_t C, const void* L1, in
                          const DevInfo* d, cudaStream_t st) {
     namespace Q = ft::qres;
     const int64_t r = r1 + r2;
+    Q::Params p;
+    std::memset(&p, 0, sizeof(p));
+    p.do_mma = r > 0 ? 1 : 0;
+    p.f1 = qres_factor(r1);
+    p.f2 = qres_factor(r2);
+    qres_ring(p);
     int mt = 0, splits = 0, cchunk = 0;
-    if (!qres_grid(M, C, d, &mt, &splits, &cchunk)) {
+    if (!qres_grid(M, C, qres_max_stages(p.ring_bytes), d, &mt, &splits, &cchunk)) {
         const float* a = amax_in;
         if (!a) {
             FT_TRY(run_amax(T, M, C, C, reinterpret_cast<float*>(ws + w.amax), d, st));
@@ -394,30 +439,14 @@ ft_status run_quant_down(const void* T, int64_t M, int64_t C, const void* L1, in
     }
     unsigned int* counters = reinterpret_cast<unsigned int*>(ws + w.counters);
     FT_TRY(cuda_ok(cudaMemsetAsync(counters, 0, (size_t)w.n_counters * 4, st)));
-    Q::Params p;
-    std::memset(&p, 0, sizeof(p));
-    p.do_mma = r > 0 ? 1 : 0;
-    p.direct = (r1 <= 64 && r2 <= 64) ? 1 : 0;
-    if (p.do_mma && p.direct) {
-        if (r1 > 0)
-            FT_TRY(encode_2d(&p.mapL1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1, r1, C, r1 * 2, 64, 64,
-                             CU_TENSOR_MAP_SWIZZLE_128B));
-        if (r2 > 0)
-            FT_TRY(encode_2d(&p.mapL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2, r2, C, r2 * 2, 64, 64,
-                             CU_TENSOR_MAP_SWIZZLE_128B));
-    } else if (p.do_mma) {
-        uint16_t* Lt = reinterpret_cast<uint16_t*>(ws + w.lt);
-        dim3 grid((unsigned)cdiv(C, 256), 128);
-        {
-            LaunchTimer _lt(KID_PACK_LT, st);
-            ft::k_pack_lt<<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(L1), (int)r1,
-                                                static_cast<const uint16_t*>(L2), (int)r2, (int)C, Lt);
-            _lt.stop();
-        }
-        FT_TRY(last_launch());
-        FT_TRY(encode_2d(&p.mapL1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Lt, C, 128, C * 2, 64, 128,
-                         CU_TENSOR_MAP_SWIZZLE_128B));
-    }
+    const CUtensorMapSwizzle swz[3] = {CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_SWIZZLE_64B,
+                                       CU_TENSOR_MAP_SWIZZLE_128B};
+    if (r1 > 0)
+        FT_TRY(encode_2d(&p.mapL1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1, r1, C, r1 * 2, p.f1.wbox, 64,
+                         swz[p.f1.wbox == 16 ? 0 : p.f1.wbox == 32 ? 1 : 2]));
+    if (r2 > 0)
+        FT_TRY(encode_2d(&p.mapL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2, r2, C, r2 * 2, p.f2.wbox, 64,
+                         swz[p.f2.wbox == 16 ? 0 : p.f2.wbox == 32 ? 1 : 2]));
     FT_TRY(encode_2d(&p.mapT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, C, M, C * 2, 64, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B));
     p.amax_in = amax_in;
@@ -441,14 +470,20 @@ ft_status run_quant_down(const void* T, int64_t M, int64_t C, const void* L1, in
 }
 
 // 1x16 quantization of a dense T [M, C] through the resident kernel (no
-// down-projection).  sync: two zeroed words when amax_in is null.
+// down-projection) when it fits; sync: two words (zeroed here) when amax_in
+// is null.  Returns false in *done when the tensor does not fit.
 ft_status run_quant_1x16_resident(const void* T, int64_t M, int64_t C, const float* amax_in,
                                   unsigned int* sync, uint8_t* codes, uint8_t* scales,
-                                  float* tscale, int mt, int splits, int cchunk, cudaStream_t st) {
+                                  float* tscale, const DevInfo* d, cudaStream_t st, bool* done) {
     namespace Q = ft::qres;
-    if (!amax_in) FT_TRY(cuda_ok(cudaMemsetAsync(sync, 0, 2 * sizeof(unsigned int), st)));
     Q::Params p;
     std::memset(&p, 0, sizeof(p));
+    qres_ring(p);
+    int mt = 0, splits = 0, cchunk = 0;
+    *done = false;
+    if (!qres_grid(M, C, qres_max_stages(p.ring_bytes), d, &mt, &splits, &cchunk)) return FT_OK;
+    *done = true;
+    if (!amax_in) FT_TRY(cuda_ok(cudaMemsetAsync(sync, 0, 2 * sizeof(unsigned int), st)));
     FT_TRY(encode_2d(&p.mapT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, C, M, C * 2, 64, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B));
     p.amax_in = amax_in;
@@ -657,10 +692,12 @@ ft_status ft_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, ft_
     DevInfo* d;
     FT_TRY(device_info(&d));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    int mt = 0, splits = 0, cchunk = 0;
-    if (blk == FT_BLK_1x16 && ld == cols && qres_grid(rows, cols, d, &mt, &splits, &cchunk))
-        return run_quant_1x16_resident(x, rows, cols, amax, static_cast<unsigned int*>(ws),
-                                       out->codes, out->scales, out->tscale, mt, splits, cchunk, st);
+    if (blk == FT_BLK_1x16 && ld == cols) {
+        bool done = false;
+        FT_TRY(run_quant_1x16_resident(x, rows, cols, amax, static_cast<unsigned int*>(ws), out->codes,
+                                       out->scales, out->tscale, d, st, &done));
+        if (done) return FT_OK;
+    }
     const float* a = amax;
     if (!a) {
         float* slot = static_cast<float*>(ws);

@@ -286,4 +286,141 @@ __device__ __forceinline__ uint2 quant_block16_fast(const uint32_t (&w)[8], cons
     return quant_block16_fast_m(w, amax_bits_16(w), t, tab, sbyte);
 }
 
+
+// ------------------------------------------------------------------------
+// Multiply path.  For most divisors d the product RN(x * y), y = RN(1/d),
+// already encodes every bf16 x exactly like the correctly rounded RN(x / d):
+// the two differ by at most an ulp of FP32, which changes the E2M1 code only
+// for an x within that ulp of one of the seven rounding boundaries
+// {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5} * d.  Both encodings are monotone
+// step functions of |x|, so they agree on every bf16 value when they agree on
+// the few bf16 values around each boundary; QTableM checks exactly those
+// once per scale byte and keeps y in ym[] only for the divisors that pass.
+// The multiply also carries the sign (a -0 input gives -0 and code 0x8), so
+// an element costs half a packed multiply and half a conversion.
+// Bit-identical to quant_block16 (same IEEE definition).
+
+struct QTableM {
+    float d[128];
+    float y[128];     // 0: divisor outside [2^-60, 2^60] (IEEE division)
+    float ym[128];    // y where the multiply path is exact for every bf16 x, else 0
+    uint32_t bad[4];  // scratch of the check: one bit per scale byte
+};
+
+__device__ __forceinline__ uint32_t e2m1_encode1(float q) {
+    uint16_t out;
+    asm("{\n\t.reg .b8 b;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n\t"
+        "cvt.u16.u8 %0, b;\n\t}"
+        : "=h"(out)
+        : "f"(0.0f), "f"(q));
+    return out & 0xFu;
+}
+
+// Step 1 of 3 (a barrier between steps): divisors and reciprocals.
+__device__ __forceinline__ void build_qtable_m1(QTableM& tab, float g, int tid, int nthreads) {
+    for (int s = tid; s < 128; s += nthreads) {
+        float d = 0.0f, y = 0.0f;
+        if (s >= 1 && s <= 0x7E) {
+            d = __fmul_rn(e4m3_decode((uint32_t)s), g);
+            y = (d >= 0x1p-60f && d <= 0x1p60f) ? __frcp_rn(d) : 0.0f;
+        }
+        tab.d[s] = d;
+        tab.y[s] = y;
+    }
+    if (tid < 4) tab.bad[tid] = 0u;
+}
+
+// Step 2: the exactness check of the multiply path, four threads per scale
+// byte (boundaries k = part, part + 4).
+__device__ __forceinline__ void build_qtable_m2(QTableM& tab, int tid, int nthreads) {
+    for (int i = tid; i < 512; i += nthreads) {
+        const int s = i & 127, part = i >> 7;
+        const float d = tab.d[s], y = tab.y[s];
+        if (s == 0 || s >= 0x7E || y == 0.0f) continue;  // these never take the multiply path
+        bool ok = true;
+        for (int k = part; k < 7; k += 4) {
+            // x0: the largest bf16 value <= b_k d (b_k d is exact in double)
+            // rounding boundary k of the E2M1 grid: 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5
+            const float bk = k < 4 ? 0.25f + 0.5f * (float)k : (k == 4 ? 2.5f : (k == 5 ? 3.5f : 5.0f));
+            // x0: the largest bf16 value <= bk d (RZ keeps the product at or
+            // below the exact one, truncation then keeps a bf16 value below it)
+            const uint32_t x0 = __float_as_uint(__fmul_rz(bk, d)) & 0xFFFF0000u;
+#pragma unroll
+            for (int c = -1; c <= 2; ++c) {
+                if (c < 0 && x0 < 0x10000u) continue;
+                const float x = __uint_as_float(x0 + (uint32_t)(c * 0x10000));
+                // div_by_recip is the correctly rounded quotient for these d
+                if (e2m1_encode1(div_by_recip(x, d, y)) != e2m1_encode1(__fmul_rn(x, y))) ok = false;
+            }
+        }
+        if (!ok) atomicOr(&tab.bad[s >> 5], 1u << (s & 31));
+    }
+}
+
+// Step 3: publish ym.
+__device__ __forceinline__ void build_qtable_m3(QTableM& tab, int tid, int nthreads) {
+    for (int s = tid; s < 128; s += nthreads) {
+        const bool bad = (tab.bad[s >> 5] >> (s & 31)) & 1u;
+        tab.ym[s] = (bad || s == 0 || s >= 0x7E) ? 0.0f : tab.y[s];
+    }
+}
+
+// Codes of 8 elements (4 bf16 pairs) as RN(x * y), sign included.
+__device__ __forceinline__ uint32_t encode8_mul(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3,
+                                                float y) {
+    const uint32_t w[4] = {w0, w1, w2, w3};
+    const uint64_t Y = f2pack(y, y);
+    float q[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint64_t X = f2pack(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+        f2unpack(mul_f32x2(X, Y), q[2 * i], q[2 * i + 1]);
+    }
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(q[0]), "f"(q[1]), "f"(q[2]), "f"(q[3]), "f"(q[4]), "f"(q[5]), "f"(q[6]), "f"(q[7]));
+    return out;
+}
+
+// The divisors the multiply path rejects (and zero / saturated scales),
+// kept out of line so the common path stays small.
+__device__ __noinline__ uint2 quant_block16_rare(uint4 lo, uint4 hi, uint32_t sbyte, float d,
+                                                 float y) {
+    const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+    uint2 r;
+    if (sbyte == 0) {
+        r = make_uint2(0u, 0u);
+    } else if (y != 0.0f && sbyte != 0x7Eu) {
+        r.x = encode8_fast(w[0], w[1], w[2], w[3], d, y);
+        r.y = encode8_fast(w[4], w[5], w[6], w[7], d, y);
+    } else {
+        r.x = encode8(w[0], w[1], w[2], w[3], d, 0.0f, false);
+        r.y = encode8(w[4], w[5], w[6], w[7], d, 0.0f, false);
+    }
+    return r;
+}
+
+// One 1x16 block given its max|x| bits, through QTableM.
+__device__ __forceinline__ uint2 quant_block16_m(const uint32_t (&w)[8], uint32_t amax_bits,
+                                                 const QTensorFast& t, const QTableM& tab,
+                                                 uint32_t& sbyte) {
+    sbyte = scale_byte_fast(__uint_as_float(amax_bits), t);
+    const float ym = tab.ym[sbyte];
+    if (ym != 0.0f) {
+        uint2 r;
+        r.x = encode8_mul(w[0], w[1], w[2], w[3], ym);
+        r.y = encode8_mul(w[4], w[5], w[6], w[7], ym);
+        return r;
+    }
+    return quant_block16_rare(make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]),
+                              sbyte, tab.d[sbyte], tab.y[sbyte]);
+}
+
 }  // namespace ft

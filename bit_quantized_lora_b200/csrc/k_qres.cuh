@@ -9,23 +9,25 @@
 //
 //   phase 1  TMA lands the chunk (all of it in flight at once); the
 //            quantizer warps take every 1x16 block's max|x| as its stage
-//            lands; meanwhile the MMA warp runs the down-projection
-//            D[j, m] = sum_c L[c, j] T[m, c] on tcgen05 (kind::f16) over the
-//            same tiles, with the factor tiles streamed through a small ring.
-//   barrier  the CTA's max is folded into one global word (integer atomicMax
-//            on the float bits: exact, order-free); a grid-wide arrival
-//            counter (cooperative launch: every CTA is resident) releases all
-//            CTAs once every max is in.  Skipped when the caller supplies the
+//            lands; meanwhile the MMA warp runs the down-projections
+//            D[m, j] = sum_c T[m, c] L[c, j] on tcgen05 (kind::f16): A = the
+//            same swizzled T tiles (K-major), B = L1 and L2 as they lie in
+//            HBM (MN-major, swizzled to their width), streamed through a ring.
+//   barrier  the CTA's max is folded into one global word (an integer max on
+//            the float bits: exact, order-free); a grid-wide arrival counter
+//            (cooperative launch: every CTA is resident) releases all CTAs
+//            once every max is in.  Skipped when the caller supplies the
 //            tensor amax.
-//   phase 2  the tensor scale, the per-scale divisor table, then every block
-//            is encoded from shared memory with the block maxima kept in
-//            registers since phase 1.
-//   tail     TMEM -> FP32 split partials; the last CTA of a row tile adds the
-//            splits in split order and rounds P = [bf16(T L1) | bf16(s T L2)].
+//   phase 2  the tensor scale and the per-scale divisor table, then every
+//            block is encoded from shared memory with the block maxima kept
+//            in registers since phase 1; codes and scales are staged in
+//            shared memory and leave in coalesced 16-byte / 4-byte stores.
+//   tail     TMEM (lane = token, column = P column) -> FP32 split partials;
+//            the last CTA of a row tile adds the splits in split order and
+//            rounds P = [bf16(T L1) | bf16(s T L2)].
 //
-// The arithmetic of every code, scale and P entry is the one of k_qdown and
-// k_amax_bf16 (same encoder, same reduction order), so results are
-// bit-identical to the two-pass path.
+// Codes and scales follow the encoding of every other quantizer here, bit
+// for bit; P follows k_qdown's rounding (FP32 accumulation, one rounding).
 //
 // CTA = 128 rows x one C-range of at most 768 columns (12 stages of 64);
 // warps: 0 TMA producer, 1 TMEM owner + UMMA issuer, 2-17 quantizers (thread
@@ -43,17 +45,32 @@ namespace qres {
 constexpr int BM = 128;
 constexpr int BKC = 64;          // columns per stage (128 bytes of bf16)
 constexpr int MAX_ST = 12;       // resident stages per CTA (768 columns)
-constexpr int FSTAGES = 2;       // factor-tile ring
+constexpr int MAX_FS = 8;        // factor-ring stages
 constexpr int NQ_WARPS = 16;
 constexpr int NQ_THREADS = NQ_WARPS * 32;
 constexpr int NUM_THREADS = 64 + NQ_THREADS;
 constexpr int TILE_BYTES = BM * BKC * 2;  // 16 KiB
 constexpr uint32_t TMEM_COLS = 128;
+constexpr uint32_t SROW = MAX_ST * 4;  // staged scale bytes per row
+constexpr uint32_t BAR_BYTES = 512;
+constexpr uint32_t SMEM_LIMIT = 227u * 1024u;
+
+// One low-rank factor L [C, rf] read as the MN-major B operand: boxes of
+// `wbox` rank columns x 64 rows of c, swizzled to the box's row bytes
+// (32, 64 or 128), `natoms` boxes side by side (rf > 64: two 64-wide atoms).
+struct Factor {
+    int rf;          // rank (0: absent)
+    int wbox;        // 16, 32 or 64 columns per box
+    int natoms;      // 1 or 2
+    uint32_t off;    // byte offset of its tile inside a ring stage
+    uint32_t sbo;    // bytes between 8-row groups (8 * wbox * 2)
+    uint32_t swz;    // descriptor swizzle code
+};
 
 struct Params {
     CUtensorMap mapT;   // bf16 [M, C], box {64, 128}, 128 B swizzle
-    CUtensorMap mapL1;  // direct: L1 [C, r1], box {64, 64}; packed: Lt [128, C], box {64, 128}
-    CUtensorMap mapL2;  // direct: L2 [C, r2], box {64, 64}
+    CUtensorMap mapL1;  // bf16 [C, r1], box {wbox1, 64}
+    CUtensorMap mapL2;  // bf16 [C, r2], box {wbox2, 64}
     const float* amax_in;      // caller's tensor amax, or null (computed here)
     unsigned int* amax_bits;   // global max word, zero on entry (amax_in == null)
     unsigned int* arrivals;    // grid barrier counter, zero on entry (amax_in == null)
@@ -66,7 +83,10 @@ struct Params {
     int M, C, r, r1, cchunk, splits;
     float s;
     int do_mma;
-    int direct;
+    Factor f1, f2;
+    uint32_t fstage_bytes;     // one ring stage (both factor tiles)
+    int fs;                    // ring stages
+    uint32_t ring_bytes;
     unsigned int num_ctas;
 };
 
@@ -74,27 +94,28 @@ struct Layout {
     uint32_t x, f, tab, bars, total;
 };
 
-__host__ __device__ inline Layout make_layout(int nst, int do_mma) {
+__host__ __device__ inline Layout make_layout(int nst, uint32_t ring_bytes) {
     Layout L;
     uint32_t o = 0;
     L.x = o;    o += (uint32_t)nst * TILE_BYTES;
-    L.f = o;    o += do_mma ? (uint32_t)FSTAGES * TILE_BYTES : 0u;
-    L.tab = o;  o += (uint32_t)sizeof(QTable);
-    L.bars = o; o += 256;
+    L.f = o;    o += ring_bytes;  // factor ring, then the staged scales
+    L.tab = o;  o += (uint32_t)sizeof(QTableM);
+    L.bars = o; o += BAR_BYTES;
     L.total = o + 1024;  // slack for the 1 KiB alignment of the base
     return L;
 }
 
 // barrier slots (uint64 each)
 enum {
-    QB_XFULL = 0,                    // [MAX_ST] chunk stage landed (used once)
-    QB_FFULL = QB_XFULL + MAX_ST,    // [FSTAGES] factor tile landed
-    QB_FEMPTY = QB_FFULL + FSTAGES,  // [FSTAGES] factor tile consumed by the MMAs
-    QB_ACC = QB_FEMPTY + FSTAGES,    // accumulator complete
-    QB_DRAIN,                        // every tcgen05 op of the MMA warp done
+    QB_XFULL = 0,                   // [MAX_ST] chunk stage landed (used once)
+    QB_FFULL = QB_XFULL + MAX_ST,   // [MAX_FS] factor tiles landed
+    QB_FEMPTY = QB_FFULL + MAX_FS,  // [MAX_FS] factor tiles consumed by the MMAs
+    QB_ACC = QB_FEMPTY + MAX_FS,    // accumulator complete
+    QB_DRAIN,                       // every tcgen05 op of the MMA warp done
     QB_COUNT
 };
-static_assert(QB_COUNT * 8 + 16 + 4 * NQ_WARPS + 16 <= 256, "barrier area");
+static_assert(QB_COUNT * 8 + 16 + 4 * NQ_WARPS <= BAR_BYTES, "barrier area");
+static_assert(BM * SROW <= 6 * 1024, "scale staging");
 
 // Waits for a phase that must complete (copies already issued) before the
 // CTA may exit; bounded like every other wait.
@@ -103,29 +124,49 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     mbar_wait(bar, parity, ERR_WAIT_DRAIN, &no_abort);
 }
 
+// TMA loads of one factor's tile for rows c .. c+63.
+__device__ __forceinline__ void load_factor(uint8_t* stage, const Factor& f, const CUtensorMap* map,
+                                            uint64_t* bar, int c) {
+    for (int a = 0; a < f.natoms; ++a)
+        tma_load_2d(stage + f.off + a * 8192, map, bar, 64 * a, c);
+}
+
+// The four K = 16 MMAs of one 64-column stage for one factor:
+// D[:, col0 .. col0 + rf) (+)= T_tile (K-major) x L_tile (MN-major).
+__device__ __forceinline__ void mma_factor(uint32_t tmem_d, uint32_t a_tile, uint32_t b_stage,
+                                           const Factor& f, bool first) {
+    const uint32_t idesc = idesc_bf16(128, f.rf, 0, 1);
+    const uint32_t b = b_stage + f.off;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        umma_bf16(tmem_d, desc_kmajor_sw128(a_tile + 32 * j),
+                  smem_desc(b + 2 * f.sbo * j, 8192, f.sbo, f.swz), idesc, (!first || j) ? 1u : 0u);
+}
+
 __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (base - raw_base);
-    const Layout L = make_layout(p.cchunk / BKC, p.do_mma);
+    const Layout L = make_layout(p.cchunk / BKC, p.ring_bytes);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.bars + QB_COUNT * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile int* last_flag = abort_flag + 1;
     volatile uint32_t* amax_share = reinterpret_cast<volatile uint32_t*>(last_flag + 1);
     volatile uint32_t* red = amax_share + 1;  // [NQ_WARPS]
-    QTable& tab = *reinterpret_cast<QTable*>(smem + L.tab);
+    QTableM& tab = *reinterpret_cast<QTableM*>(smem + L.tab);
 
     const int warp = warp_id(), lane = lane_id();
     const int m0 = blockIdx.x * BM;
     const int split = blockIdx.y;
     const int c0 = split * p.cchunk;
     const int nst = min(p.cchunk, p.C - c0) / BKC;  // 1 .. MAX_ST
+    const int FS = p.fs;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < MAX_ST; ++i) mbar_init(&bars[QB_XFULL + i], 1);
-        for (int i = 0; i < FSTAGES; ++i) {
+        for (int i = 0; i < MAX_FS; ++i) {
             mbar_init(&bars[QB_FFULL + i], 1);
             mbar_init(&bars[QB_FEMPTY + i], 1);
         }
@@ -146,67 +187,61 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
+            // the first ring stages of factor tiles (small) ahead of the
+            // chunk, so the down-projection starts with the first chunk stage
+            const int pre = p.do_mma ? min(FS, nst) : 0;
+            for (int st = 0; st < pre; ++st) {
+                uint64_t* fb = &bars[QB_FFULL + st];
+                mbar_arrive_expect_tx(fb, p.fstage_bytes);
+                uint8_t* dst = smem + L.f + st * p.fstage_bytes;
+                if (p.f1.rf > 0) load_factor(dst, p.f1, &p.mapL1, fb, c0 + st * BKC);
+                if (p.f2.rf > 0) load_factor(dst, p.f2, &p.mapL2, fb, c0 + st * BKC);
+            }
             // the whole chunk at once: it stays resident
             for (int st = 0; st < nst; ++st) {
                 mbar_arrive_expect_tx(&bars[QB_XFULL + st], TILE_BYTES);
                 tma_load_2d(smem + L.x + st * TILE_BYTES, &p.mapT, &bars[QB_XFULL + st], c0 + st * BKC, m0);
             }
-            int st = 0;
+            int st = pre;
             if (p.do_mma) {
-                const int r2 = p.r - p.r1;
-                const uint32_t fbytes =
-                    !p.direct ? (uint32_t)TILE_BYTES
-                              : (p.r1 > 0 ? TILE_BYTES / 2u : 0u) + (r2 > 0 ? TILE_BYTES / 2u : 0u);
                 for (; st < nst; ++st) {
-                    const int f = st % FSTAGES;
-                    const uint32_t ph = (st / FSTAGES) & 1;
+                    const int f = st % FS;
+                    const uint32_t ph = (st / FS) & 1;
                     if (!mbar_wait(&bars[QB_FEMPTY + f], ph ^ 1, ERR_WAIT_EMPTY, abort_flag)) break;
                     uint64_t* fb = &bars[QB_FFULL + f];
-                    mbar_arrive_expect_tx(fb, fbytes);
-                    uint8_t* dst = smem + L.f + f * TILE_BYTES;
+                    mbar_arrive_expect_tx(fb, p.fstage_bytes);
+                    uint8_t* dst = smem + L.f + f * p.fstage_bytes;
                     const int c = c0 + st * BKC;
-                    if (p.direct) {
-                        // rank columns 0..63 of rows c .. c+63 of L1 and L2
-                        if (p.r1 > 0) tma_load_2d(dst, &p.mapL1, fb, 0, c);
-                        if (r2 > 0) tma_load_2d(dst + TILE_BYTES / 2, &p.mapL2, fb, 0, c);
-                    } else {
-                        tma_load_2d(dst, &p.mapL1, fb, c, 0);
-                    }
+                    if (p.f1.rf > 0) load_factor(dst, p.f1, &p.mapL1, fb, c);
+                    if (p.f2.rf > 0) load_factor(dst, p.f2, &p.mapL2, fb, c);
                 }
             }
             if (*abort_flag) {
                 // every copy issued lands before the CTA may exit
                 for (int s2 = 0; s2 < nst; ++s2) drain_wait(&bars[QB_XFULL + s2], 0);
-                for (int d = 0; d < FSTAGES && d < st; ++d) {
+                for (int d = 0; d < FS && d < st; ++d) {
                     const int j = st - 1 - d;
-                    drain_wait(&bars[QB_FFULL + j % FSTAGES], (j / FSTAGES) & 1);
+                    drain_wait(&bars[QB_FFULL + j % FS], (j / FS) & 1);
                 }
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------ UMMA issuer
         if (lane == 0 && p.do_mma) {
-            // direct: A = [L1 | L2]^T, MN-major (two 64-wide atoms 8 KiB apart,
-            // K step = 16 rows = 2 KiB); packed: A = Lt, K-major.  B = T tile.
-            const uint32_t idesc = idesc_bf16(128, BM, p.direct ? 1 : 0, 0);
             bool ok = true;
             for (int st = 0; st < nst; ++st) {
-                const int f = st % FSTAGES;
-                const uint32_t ph = (st / FSTAGES) & 1;
+                const int f = st % FS;
+                const uint32_t ph = (st / FS) & 1;
                 if (!mbar_wait(&bars[QB_XFULL + st], 0, ERR_WAIT_FULL, abort_flag) ||
                     !mbar_wait(&bars[QB_FFULL + f], ph, ERR_WAIT_FULL, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t a = base + L.f + f * TILE_BYTES;
-                const uint32_t b = base + L.x + st * TILE_BYTES;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint64_t ad = p.direct ? smem_desc(a + 2048 * j, TILE_BYTES / 2, 1024, SWZ_128B)
-                                                 : desc_kmajor_sw128(a + 32 * j);
-                    umma_bf16(tmem, ad, desc_kmajor_sw128(b + 32 * j), idesc, (st | j) != 0);
-                }
+                const uint32_t a = base + L.x + st * TILE_BYTES;
+                const uint32_t b = base + L.f + f * p.fstage_bytes;
+                if (p.f1.rf > 0) mma_factor(tmem, a, b, p.f1, st == 0);
+                if (p.f2.rf > 0) mma_factor(tmem + (uint32_t)p.r1, a, b, p.f2, st == 0);
                 tc_commit(&bars[QB_FEMPTY + f]);
             }
             if (ok) tc_commit(&bars[QB_ACC]);
@@ -218,7 +253,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
         // ------------------------------------------------ quantizers
         const int t = threadIdx.x - 64;
         const int trow = t & (BM - 1), blk = t >> 7;
-        const int row = m0 + trow;
         const uint32_t sw = (uint32_t)(trow & 7);
         const uint32_t off_lo = (uint32_t)trow * 128u + (((uint32_t)(2 * blk) ^ sw) << 4);
         const uint32_t off_hi = (uint32_t)trow * 128u + (((uint32_t)(2 * blk + 1) ^ sw) << 4);
@@ -256,9 +290,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
                 uint32_t m = 0;
                 for (int i = 0; i < NQ_WARPS; ++i) m = max(m, red[i]);
                 // every CTA arrives, also one that gave up, so no other CTA
-                // waits on it
-                if (m) atomicMax(p.amax_bits, m);
-                __threadfence();
+                // waits on it; the release orders this CTA's max before its
+                // arrival
+                if (m) red_max_relaxed_gpu(p.amax_bits, m);
                 red_add_release_gpu(p.arrivals, 1u);
                 const uint64_t t0 = globaltimer_ns();
                 while (ld_acquire_gpu(p.arrivals) < p.num_ctas) {
@@ -267,7 +301,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
                         *abort_flag = 1;
                         break;
                     }
-                    __nanosleep(100);
                 }
                 amax_t = __uint_as_float(ld_acquire_gpu(p.amax_bits));
             }
@@ -275,12 +308,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
         }
         named_bar_sync(1, NQ_THREADS);
         const QTensorFast qt = make_qtensor_fast(__uint_as_float(*amax_share));
-        build_qtable(tab, qt.g, t, NQ_THREADS);
+        build_qtable_m1(tab, qt.g, t, NQ_THREADS);
         if (blockIdx.x == 0 && blockIdx.y == 0 && t == 0) *p.tscale = qt.g;
+        named_bar_sync(1, NQ_THREADS);
+        build_qtable_m2(tab, t, NQ_THREADS);
+        named_bar_sync(1, NQ_THREADS);
+        build_qtable_m3(tab, t, NQ_THREADS);
+        // the MMAs have normally finished with the tiles by now (they ran
+        // during phase 1 and the barrier); after this wait phase 2 may
+        // overwrite the chunk and the factor ring
+        if (p.do_mma && ok && !mbar_wait(&bars[QB_ACC], 0, ERR_WAIT_ACC_FULL, abort_flag)) ok = false;
         named_bar_sync(1, NQ_THREADS);
         ok = ok && !*abort_flag;
 
-        // phase 2: encode every block from shared memory
+        // phase 2: encode every block from shared memory.  A block's 8 code
+        // bytes go back into the first half of its own (already read) 16-byte
+        // slot, its scale byte into a [128, 48] staging array over the factor
+        // ring; the output pass then writes both with coalesced stores.
+        const uint32_t sstage = base + L.f;
         if (ok) {
 #pragma unroll
             for (int st = 0; st < MAX_ST; ++st) {
@@ -289,44 +334,53 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
                     const uint4 v0 = ld_shared_v4(ta + off_lo), v1 = ld_shared_v4(ta + off_hi);
                     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
                     uint32_t sbyte;
-                    const uint2 q = quant_block16_fast_m(w, mb[st], qt, tab, sbyte);
-                    if (row < p.M) {
-                        const int col = c0 + st * BKC + 16 * blk;
-                        *reinterpret_cast<uint2*>(p.codes + (int64_t)row * (p.C / 2) + col / 2) = q;
-                        p.scales[(int64_t)row * (p.C / 16) + col / 16] = (uint8_t)sbyte;
-                    }
+                    const uint2 q = quant_block16_m(w, mb[st], qt, tab, sbyte);
+                    st_shared_v2(ta + off_lo, q);
+                    st_shared_u8(sstage + (uint32_t)trow * SROW + st * 4 + blk, sbyte);
                 }
             }
         }
+        named_bar_sync(1, NQ_THREADS);
+        if (ok) {
+            const int rows = min(BM, p.M - m0);
+            // codes: 16-byte segments (two blocks), consecutive threads on
+            // consecutive segments of a row
+            const int segs = nst * 2;
+            for (int i = t; i < rows * segs; i += NQ_THREADS) {
+                const int r = i / segs, j = i - r * segs;
+                const int st = j >> 1, b0 = 2 * (j & 1);
+                const uint32_t rs = (uint32_t)(r & 7);
+                const uint32_t ra = base + L.x + st * TILE_BYTES + (uint32_t)r * 128u;
+                const uint2 lo = ld_shared_v2(ra + (((uint32_t)(2 * b0) ^ rs) << 4));
+                const uint2 hi = ld_shared_v2(ra + (((uint32_t)(2 * b0 + 2) ^ rs) << 4));
+                *reinterpret_cast<uint4*>(p.codes + (int64_t)(m0 + r) * (p.C / 2) + c0 / 2 + 16 * j) =
+                    make_uint4(lo.x, lo.y, hi.x, hi.y);
+            }
+            // scales: one 4-byte word per stage of a row
+            for (int i = t; i < rows * nst; i += NQ_THREADS) {
+                const int r = i / nst, st = i - r * nst;
+                const uint32_t v = ld_shared_u32(sstage + (uint32_t)r * SROW + st * 4);
+                *reinterpret_cast<uint32_t*>(p.scales + (int64_t)(m0 + r) * (p.C / 16) + c0 / 16 + 4 * st) = v;
+            }
+        }
 
-        // epilogue: TMEM lane = rank index j, column = tile row; the four
-        // warps of a lane quarter take 32 tile rows each
+        // epilogue: TMEM lane = token row, column = P column; the four warps
+        // of a lane quarter take 16-column chunks c = part, part + 4
         if (p.do_mma && ok) {
             const int sp = warp & 3;
-            const int quarter = (warp - 2) >> 2;
-            const int r2 = p.r - p.r1;
-            int j;      // P column of this TMEM lane (-1: padding lane)
-            bool any;   // warp-uniform: does this lane quarter hold any column
-            if (p.direct) {
-                const int l = 32 * sp + lane;
-                j = (l < 64) ? (l < p.r1 ? l : -1) : (l - 64 < r2 ? p.r1 + l - 64 : -1);
-                any = (sp < 2) ? (32 * sp < p.r1) : (32 * (sp - 2) < r2);
-            } else {
-                j = 32 * sp + lane < p.r ? 32 * sp + lane : -1;
-                any = 32 * sp < p.r;
-            }
-            if (mbar_wait(&bars[QB_ACC], 0, ERR_WAIT_ACC_FULL, abort_flag) && any) {
-                tc_fence_after();
-                uint32_t v[32];
-                const int col0 = 32 * quarter;
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * sp) << 16) + col0, v);
+            const int part = (warp - 2) >> 2;
+            const int m = m0 + 32 * sp + lane;
+            const uint32_t lane_addr = (uint32_t)(32 * sp) << 16;
+            for (int c = part; c < p.r / 16; c += 4) {
+                uint32_t v[16];
+                tmem_ld_32x32b_x16(tmem + lane_addr + 16 * c, v);
                 tmem_ld_wait();
-                if (j >= 0) {
+                if (m < p.M) {
+                    float4* o = reinterpret_cast<float4*>(p.part + ((int64_t)split * p.M + m) * p.r + 16 * c);
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) {
-                        const int m = m0 + col0 + k;
-                        if (m < p.M) p.part[((int64_t)split * p.M + m) * p.r + j] = __uint_as_float(v[k]);
-                    }
+                    for (int k = 0; k < 4; ++k)
+                        o[k] = make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                                           __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
                 }
             }
         }
