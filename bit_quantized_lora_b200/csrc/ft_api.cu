@@ -183,7 +183,7 @@ constexpr int QD_MAX_SPLITS = 8;
 constexpr int LG_MAX_SPLITS = 16;
 
 struct WsPlan {
-    size_t amax, gact, codes, scales, lt, part, pg, lgpart, counters, total;
+    size_t amax, gact, codes, scales, sfslab, lt, part, pg, lgpart, counters, total;
     int n_qd_counters, lg_ctiles, n_counters;
     // counters region: [0] tensor-amax bits and [1] grid-barrier arrivals of
     // the resident quantizer, then the row-tile counters of the fused
@@ -200,6 +200,7 @@ WsPlan plan_ws(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t r_l) {
     w.gact = o;   o += 256;
     w.codes = o;  o += up256((size_t)M * C / 2);
     w.scales = o; o += up256((size_t)M * C / 16);
+    w.sfslab = o; o += up256((size_t)((M + 127) / 128) * 128 * C / 16);  // GEMM scale slabs
     w.lt = o;     o += up256((size_t)128 * C * 2);
     w.part = o;   o += up256((size_t)QD_MAX_SPLITS * M * r * 4);
     w.pg = o;     o += up256((size_t)M * r * 2);
@@ -233,14 +234,14 @@ ft_status run_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, float*
 }
 
 ft_status run_quant_1x16(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* amax,
-                         uint8_t* codes, uint8_t* scales, float* tscale, const DevInfo* d,
-                         cudaStream_t st) {
+                         uint8_t* codes, uint8_t* scales, float* tscale, uint8_t* slab,
+                         const DevInfo* d, cudaStream_t st) {
     const int64_t blocks = rows * (cols / 16);
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(blocks, 256), (int64_t)d->sms * 16));
     {
         LaunchTimer _lt(KID_QUANT_1X16, st);
         ft::k_quant_1x16<<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(x), rows, cols, ld, amax,
-                                               codes, scales, tscale);
+                                               codes, scales, tscale, slab);
         _lt.stop();
     }
     return last_launch();
@@ -277,7 +278,8 @@ ft_status run_qdown(const void* T, int64_t M, int64_t C, const void* L1, int64_t
                     float* tscale, void* P, uint8_t* ws, const WsPlan& w, const DevInfo* d,
                     cudaStream_t st) {
     const int64_t r = r1 + r2;
-    if (r == 0) return run_quant_1x16(T, M, C, C, amax, codes, scales, tscale, d, st);
+    uint8_t* slab = ws + w.sfslab;
+    if (r == 0) return run_quant_1x16(T, M, C, C, amax, codes, scales, tscale, slab, d, st);
     float* part = reinterpret_cast<float*>(ws + w.part);
     unsigned int* counters = reinterpret_cast<unsigned int*>(ws + w.counters);
     FT_TRY(cuda_ok(cudaMemsetAsync(counters, 0, (size_t)w.n_counters * 4, st)));
@@ -314,6 +316,7 @@ ft_status run_qdown(const void* T, int64_t M, int64_t C, const void* L1, int64_t
     p.tscale = tscale;
     p.codes = codes;
     p.scales = scales;
+    p.slab = slab;
     p.part = part;
     p.P = static_cast<__nv_bfloat16*>(P);
     p.counters = counters + w.qd_cnt;
@@ -455,6 +458,7 @@ ft_status run_quant_down(const void* T, int64_t M, int64_t C, const void* L1, in
     p.tscale = tscale;
     p.codes = codes;
     p.scales = scales;
+    p.slab = ws + w.sfslab;
     p.part = reinterpret_cast<float*>(ws + w.part);
     p.P = static_cast<__nv_bfloat16*>(P);
     p.counters = counters + w.qd_cnt;
@@ -501,33 +505,55 @@ ft_status run_quant_1x16_resident(const void* T, int64_t M, int64_t C, const flo
     return launch_qres(p, mt, splits, st);
 }
 
-// out[M, Nout] = ga gb Q(A) Q(B)^T + P[:, :r1] L1^T + P[:, r1:] L2^T
-ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* ga, int64_t M,
-                   int64_t Kc, const uint8_t* b_codes, const uint8_t* grid_scales, const float* gb,
-                   int64_t Nout, bool sfb_trans, int64_t grid_rows, int64_t grid_cols,
-                   const void* P, const void* L1, int64_t r1, const void* L2, int64_t r2, void* out,
-                   ft_dtype ot, const DevInfo* d, cudaStream_t st) {
+// Panels of one low-rank factor in the GEMM: K-major, swizzled to the
+// factor's width (16, 32 or 64 columns; two 64-wide atoms above 64).
+ft::gemm::LrFactor gemm_factor(int64_t rf, int64_t pcol) {
+    ft::gemm::LrFactor f;
+    std::memset(&f, 0, sizeof(f));
+    f.rf = (int)rf;
+    f.pcol = (int)pcol;
+    if (rf <= 0) return f;
+    f.wbox = rf <= 16 ? 16 : rf <= 32 ? 32 : 64;
+    f.natoms = rf <= 64 ? 1 : 2;
+    f.swz = f.wbox == 16 ? ft::SWZ_32B : f.wbox == 32 ? ft::SWZ_64B : ft::SWZ_128B;
+    f.atom_bytes = 128u * (uint32_t)f.wbox * 2u;
+    return f;
+}
+
+CUtensorMapSwizzle swizzle_for(int wbox) {
+    return wbox == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : wbox == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                               : CU_TENSOR_MAP_SWIZZLE_128B;
+}
+
+// out[M, Nout] = ga gb Q(A) Q(B)^T + P[:, :r1] L1^T + P[:, r1:] L2^T, the
+// block scales of A and B given as slabs ([rows/128][Kc/64][512]).
+ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_slab, const float* ga, int64_t M,
+                   int64_t Kc, const uint8_t* b_codes, const uint8_t* b_slab, const float* gb,
+                   int64_t Nout, const void* P, const void* L1, int64_t r1, const void* L2, int64_t r2,
+                   void* out, ft_dtype ot, const DevInfo* d, cudaStream_t st) {
     Params p;
     std::memset(&p, 0, sizeof(p));
     FT_TRY(encode_2d(&p.mapA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, Kc / 2, M, Kc / 2, 128, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B));
     FT_TRY(encode_2d(&p.mapB, CU_TENSOR_MAP_DATA_TYPE_UINT8, b_codes, Kc / 2, Nout, Kc / 2, 128, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B));
-    FT_TRY(encode_2d(&p.mapSFA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_scales, Kc / 16, M, Kc / 16, 16, 128,
-                     CU_TENSOR_MAP_SWIZZLE_NONE));
-    // the 16x16 grid is [grid_rows, grid_cols] row-major
-    FT_TRY(encode_2d(&p.mapSFB, CU_TENSOR_MAP_DATA_TYPE_UINT8, grid_scales, grid_cols, grid_rows,
-                     grid_cols, 16, sfb_trans ? 16 : 8, CU_TENSOR_MAP_SWIZZLE_NONE));
     const int64_t r = r1 + r2;
-    if (r > 0)
-        FT_TRY(encode_2d(&p.mapP, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P, r, M, r * 2, 64, 128,
-                         CU_TENSOR_MAP_SWIZZLE_128B));
-    if (r1 > 0)
-        FT_TRY(encode_2d(&p.mapL1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1, r1, Nout, r1 * 2, 64, 128,
-                         CU_TENSOR_MAP_SWIZZLE_128B));
-    if (r2 > 0)
-        FT_TRY(encode_2d(&p.mapL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2, r2, Nout, r2 * 2, 64, 128,
-                         CU_TENSOR_MAP_SWIZZLE_128B));
+    p.f1 = gemm_factor(r1, 0);
+    p.f2 = gemm_factor(r2, r1);
+    if (r1 > 0) {
+        FT_TRY(encode_2d(&p.mapP1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P, r, M, r * 2, p.f1.wbox, 128,
+                         swizzle_for(p.f1.wbox)));
+        FT_TRY(encode_2d(&p.mapL1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1, r1, Nout, r1 * 2, p.f1.wbox, 128,
+                         swizzle_for(p.f1.wbox)));
+    }
+    if (r2 > 0) {
+        FT_TRY(encode_2d(&p.mapP2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P, r, M, r * 2, p.f2.wbox, 128,
+                         swizzle_for(p.f2.wbox)));
+        FT_TRY(encode_2d(&p.mapL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2, r2, Nout, r2 * 2, p.f2.wbox, 128,
+                         swizzle_for(p.f2.wbox)));
+    }
+    p.sfa = a_slab;
+    p.sfb = b_slab;
     p.ga = ga;
     p.gb = gb;
     p.out = out;
@@ -535,13 +561,10 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float*
     p.M = (int)M;
     p.Nout = (int)Nout;
     p.Kc = (int)Kc;
-    p.r1 = (int)r1;
-    p.r2 = (int)r2;
-    p.sfb_trans = sfb_trans ? 1 : 0;
     int stages = ft::gemm::MAX_STAGES;
-    while (stages > 2 && ft::gemm::make_layout(stages, (int)r1, (int)r2).total > 227u * 1024u) --stages;
+    while (stages > 2 && ft::gemm::make_layout(stages, p.f1, p.f2).total > 227u * 1024u) --stages;
     p.stages = stages;
-    const uint32_t smem = ft::gemm::make_layout(stages, (int)r1, (int)r2).total;
+    const uint32_t smem = ft::gemm::make_layout(stages, p.f1, p.f2).total;
     const int tiles = cdiv(M, ft::gemm::BM) * (int)(Nout / ft::gemm::BN);
     const int grid = std::max(1, std::min(tiles, d->sms));
     {
@@ -622,6 +645,8 @@ ft_status check_linear(const ft_linear* L) {
     if ((L->U && !al16(L->U)) || (L->V && !al16(L->V)) || (L->A && !al16(L->A)) ||
         (L->B && !al16(L->B)))
         return FT_ERR_ALIGN;
+    if (!L->sf_k || !L->sf_n) return FT_ERR_INVALID_ARG;
+    if (!al16(L->sf_k) || !al16(L->sf_n)) return FT_ERR_ALIGN;
     return FT_OK;
 }
 
@@ -644,6 +669,26 @@ const char* ft_status_str(ft_status s) {
 }
 
 size_t ft_quantize_workspace_bytes(void) { return 256; }
+
+size_t ft_weight_scales_bytes(int64_t N, int64_t K) {
+    if (N < 0 || K < 0) return 0;
+    return (size_t)N * (size_t)K / 16;
+}
+
+ft_status ft_expand_weight_scales(const uint8_t* grid, int64_t N, int64_t K, uint8_t* sf_k,
+                                  uint8_t* sf_n, void* stream) {
+    if (!grid || !sf_k || !sf_n || N < 0 || K < 0) return FT_ERR_INVALID_ARG;
+    if (N % 256 || K % 256) return FT_ERR_SHAPE;
+    if (!al16(sf_k) || !al16(sf_n)) return FT_ERR_ALIGN;
+    if (N == 0 || K == 0) return FT_OK;
+    DevInfo* d;
+    FT_TRY(device_info(&d));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t rows = (N / 128) * (K / 64) * 32 * 2;  // 16-byte slab rows, both layouts
+    const int grid_n = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(rows, 256), (int64_t)d->sms * 8));
+    ft::k_expand_wsf<<<grid_n, 256, 0, st>>>(grid, N, K, sf_k, sf_n);
+    return last_launch();
+}
 
 size_t ft_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t r_l) {
     if (M < 0 || N < 0 || K < 0 || r_s < 0 || r_l < 0) return 0;
@@ -705,7 +750,7 @@ ft_status ft_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, ft_
         a = slot;
     }
     if (blk == FT_BLK_1x16)
-        return run_quant_1x16(x, rows, cols, ld, a, out->codes, out->scales, out->tscale, d, st);
+        return run_quant_1x16(x, rows, cols, ld, a, out->codes, out->scales, out->tscale, nullptr, d, st);
     return run_tile16(true, x, rows, cols, ld, a, out->codes, out->scales, nullptr, nullptr,
                       out->tscale, nullptr, st);
 }
@@ -771,8 +816,8 @@ ft_status ft_linear_fwd(const ft_linear* L, const void* X, int64_t M, const floa
     uint8_t* scales = wsb + w.scales;
     FT_TRY(run_quant_down(X, M, L->K, L->U, L->r_s, L->A, L->r_l, L->s, amax_x, codes, scales, g_x,
                           P_save, wsb, w, d, st));
-    return run_gemm(codes, scales, g_x, M, L->K, L->w_k.codes, L->w_k.scales, L->w_k.tscale, L->N,
-                    false, L->N / 16, L->K / 16, P_save, L->V, L->r_s, L->B, L->r_l, Y, yt, d, st);
+    return run_gemm(codes, wsb + w.sfslab, g_x, M, L->K, L->w_k.codes, L->sf_k, L->w_k.tscale, L->N,
+                    P_save, L->V, L->r_s, L->B, L->r_l, Y, yt, d, st);
 }
 
 ft_status ft_linear_bwd(const ft_linear* L, const void* dY, const void* X, const void* P_save,
@@ -810,8 +855,8 @@ ft_status ft_linear_bwd(const ft_linear* L, const void* dY, const void* X, const
     void* Pg = wsb + w.pg;
     FT_TRY(run_quant_down(dY, M, L->N, L->V, L->r_s, L->B, L->r_l, L->s, amax_dy, codes, scales, g_dy,
                           Pg, wsb, w, d, st));
-    FT_TRY(run_gemm(codes, scales, g_dy, M, L->N, L->w_n.codes, L->w_k.scales, L->w_k.tscale, L->K,
-                    true, L->N / 16, L->K / 16, Pg, L->U, L->r_s, L->A, L->r_l, dX, xt, d, st));
+    FT_TRY(run_gemm(codes, wsb + w.sfslab, g_dy, M, L->N, L->w_n.codes, L->sf_n, L->w_k.tscale, L->K,
+                    Pg, L->U, L->r_s, L->A, L->r_l, dX, xt, d, st));
     if (L->r_l > 0)
         FT_TRY(run_lora_grads(dY, X, P_save, Pg, M, L->N, L->K, L->r_s, L->r_l, dA, dB, wsb, w, d, st));
     return FT_OK;

@@ -15,6 +15,13 @@
 
 namespace ft {
 
+// Byte offset of the scale of (row r, 16-column block b) in the slab layout
+// the FP4 GEMM copies into tensor memory: [ceil(rows/128)][cols/64][512],
+// byte 16 l + 4 i + (b % 4) of slab (r / 128, b / 4) with r % 128 = 32 i + l.
+__host__ __device__ __forceinline__ int64_t slab_offset(int64_t r, int64_t b, int64_t cols) {
+    return ((r >> 7) * (cols >> 6) + (b >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (b & 3);
+}
+
 struct QTensor {
     float g;      // decode tensor scale
     float six_g;  // RN(6 g)

@@ -9,32 +9,37 @@
 //
 // Forward : A = Q(X) [M, K] 1x16,  B = Q(W_res) codes packed along K,
 //           P = [X U | s X A], L1 = V, L2 = B.
-// Dgrad   : A = Q(dY) [M, N] 1x16, B = Q(W_res)^T codes packed along N with
-//           the 16x16 scale grid read transposed (section 3.2: the scale of a
-//           16x16 block is the same for W and W^T), P = [dY V | s dY B],
-//           L1 = U, L2 = A.
+// Dgrad   : A = Q(dY) [M, N] 1x16, B = Q(W_res)^T codes packed along N,
+//           P = [dY V | s dY B], L1 = U, L2 = A.
+//
+// Block scales arrive in the tensor-memory slab layout (below): the
+// activation quantizers write it next to the row-major scales, and the
+// weight's 16x16 grid is expanded into it once, for both code layouts, when
+// the weight is prepared (section 3.2: one grid serves W and W^T; the
+// expansion repeats each 16x16 scale for its 16 rows and changes no code).
+// Slab layout of an operand with R rows and Kc contraction columns:
+// [ceil(R/128)][Kc/64][512 B], byte 16 l + 4 i + b of slab (t, s) = the
+// scale of row 128 t + 32 i + l, 16-column block 4 s + b.  One slab is
+// exactly what tcgen05.cp.32x128b.warpx4 turns into the scale layout the
+// MMA reads (row m at TMEM lane m % 32 of every lane quarter, column
+// c + m / 32), so the MMA warp copies it straight from the TMA buffer.
 //
 // Blackwell mapping: one CTA per SM, persistent over 128x128 output tiles.
-//   warp 0  TMA producer: FP4 code tiles (128 B swizzle), raw scale rows,
-//           the tile's P / L1 / L2 panels.
-//   warp 1  TMEM owner and UMMA issuer: per stage one tcgen05.cp of each
-//           operand's block scales into TMEM and four
-//           tcgen05.mma.kind::mxf4nvf4.block16 (K = 64 each) into a
+//   warp 0  TMA producer: FP4 code tiles (128 B swizzle) and the two scale
+//           slabs of each stage (bulk copies), the tile's P / L1 / L2 panels.
+//   warp 1  TMEM owner and UMMA issuer: per K-step one tcgen05.cp of each
+//           operand's slab into TMEM and one
+//           tcgen05.mma.kind::mxf4nvf4.block16 (K = 64) into a
 //           double-buffered FP32 accumulator, then tcgen05.mma kind::f16 for
-//           the low-rank panels into a separate accumulator.  Descriptors
-//           are precomputed words, so the issue loop is a few integer adds.
-//   warp 2  scale-factor warp: rearranges each stage's scale bytes into the
-//           slab layout below, expanding 16x16 weight scales to one per row.
+//           the low-rank panels into a separate accumulator.
 //   warps 4-7 epilogue: tcgen05.ld both accumulators, combine, store.
 // TMEM columns: [0,128) acc0, [128,256) acc1, [256,384) low-rank acc,
 // [384,400) A scales, [400,416) B scales.
 //
-// Scale factors in TMEM: the MMA reads the four scale bytes of row m (one
-// per 16 K-elements of its K = 64) from TMEM lane m at column c + m/32, c
-// being the (4-column aligned) scale address the instruction names.  Each
-// K-step's scales are one 32-row x 16-byte slab in shared memory (row m % 32
-// holds rows m % 32 + 32 q at bytes 4q..4q+3) that tcgen05.cp.32x128b.warpx4
-// replicates into all four lane quarters; K-step j uses columns c = base + 4j.
+// Low-rank panels are K-major with the rank as K, each factor's part of P
+// and the factor itself swizzled to its own width (16, 32 or 64 columns per
+// 32, 64 or 128-byte row; two 64-column atoms above 64), so a rank-16
+// factor costs 4 KiB of shared memory, not a padded 16 KiB panel.
 #pragma once
 
 #include <cuda.h>
@@ -48,90 +53,108 @@ constexpr int BM = 128;
 constexpr int BN = 128;
 constexpr int BK_BYTES = 128;  // 256 FP4 elements of K per stage
 constexpr int KSTEPS = 4;      // MMAs of K = 64 per stage
-constexpr int MAX_STAGES = 4;
+constexpr int MAX_STAGES = 6;
 constexpr int NUM_THREADS = 256;
 constexpr int TILE_BYTES = BM * BK_BYTES;      // 16 KiB, A or B stage
-constexpr int SFA_RAW_BYTES = BM * 16;         // 128 rows x 16 scale bytes
-constexpr int SFB_RAW_BYTES = 256;             // 8 x 16 (fwd) or 16 x 16 (dgrad)
-constexpr int SF_ATOM_BYTES = KSTEPS * 512;    // 4 x (32 rows x 16 B)
-constexpr int PANEL_BYTES = 128 * 64 * 2;      // a 128-row x 64-col bf16 panel
+constexpr int SF_STAGE_BYTES = KSTEPS * 512;   // four slabs of one operand
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL0 = 0, LR_COL = 256, SFA_COL = 384, SFB_COL = 400;
 
+// One low-rank factor's panels: P columns [pcol, pcol + rf) for the tile's
+// 128 rows (A operand) and L [128 output rows, rf] (B operand), both K-major.
+struct LrFactor {
+    int rf;        // rank (0: absent)
+    int wbox;      // 16, 32 or 64 elements per swizzled row
+    int natoms;    // 1, or 2 above 64
+    int pcol;      // first column of P
+    uint32_t swz;  // descriptor swizzle code
+    uint32_t atom_bytes;  // 128 rows x wbox x 2
+};
+
 struct Params {
-    CUtensorMap mapA, mapB, mapSFA, mapSFB, mapP, mapL1, mapL2;
+    CUtensorMap mapA, mapB, mapP1, mapP2, mapL1, mapL2;
+    const uint8_t* sfa;  // activation scale slabs [ceil(M/128)][Kc/64][512]
+    const uint8_t* sfb;  // weight scale slabs [Nout/128][Kc/64][512]
     const float* ga;
     const float* gb;
     void* out;
     int out_f32;
     int M, Nout, Kc;
-    int r1, r2;
-    int sfb_trans;
+    LrFactor f1, f2;
     int stages;
 };
 
 struct Layout {
-    uint32_t a, b, p, l1, l2, sfa_raw, sfb_raw, sfa, sfb, bars, total;
-    int np, n1, n2;
+    uint32_t a, b, sfa, sfb, p1, p2, l1, l2, bars, total;
 };
 
-__host__ __device__ inline Layout make_layout(int stages, int r1, int r2) {
+__host__ __device__ inline uint32_t lr_bytes(const LrFactor& f) {
+    return f.rf > 0 ? (uint32_t)f.natoms * f.atom_bytes : 0u;
+}
+
+__host__ __device__ inline Layout make_layout(int stages, const LrFactor& f1, const LrFactor& f2) {
     Layout L;
-    int r = r1 + r2;
-    L.np = (r + 63) / 64;
-    L.n1 = (r1 + 63) / 64;
-    L.n2 = (r2 + 63) / 64;
     uint32_t o = 0;
-    L.a = o;        o += stages * TILE_BYTES;
-    L.b = o;        o += stages * TILE_BYTES;
-    L.p = o;        o += L.np * PANEL_BYTES;
-    L.l1 = o;       o += L.n1 * PANEL_BYTES;
-    L.l2 = o;       o += L.n2 * PANEL_BYTES;
-    L.sfa = o;      o += stages * SF_ATOM_BYTES;
-    L.sfb = o;      o += stages * SF_ATOM_BYTES;
-    L.sfa_raw = o;  o += stages * SFA_RAW_BYTES;
-    L.sfb_raw = o;  o += stages * SFB_RAW_BYTES;
-    L.bars = o;     o += 256;  // barriers, TMEM slot, abort flag
-    L.total = o + 1024;        // slack for 1 KiB alignment of the base
+    L.a = o;    o += stages * TILE_BYTES;
+    L.b = o;    o += stages * TILE_BYTES;
+    L.p1 = o;   o += lr_bytes(f1);
+    L.l1 = o;   o += lr_bytes(f1);
+    L.p2 = o;   o += lr_bytes(f2);
+    L.l2 = o;   o += lr_bytes(f2);
+    L.sfa = o;  o += stages * SF_STAGE_BYTES;
+    L.sfb = o;  o += stages * SF_STAGE_BYTES;
+    L.bars = o; o += 256;  // barriers, TMEM slot, abort flag
+    L.total = o + 1024;    // slack for 1 KiB alignment of the base
     return L;
 }
 
 // barrier slots (uint64 each) inside the 256-byte barrier area
 enum {
-    B_FULL = 0,                 // [MAX_STAGES] TMA landed
-    B_SF = B_FULL + MAX_STAGES,  // [MAX_STAGES] scale atoms ready
-    B_EMPTY = B_SF + MAX_STAGES, // [MAX_STAGES] stage consumed by the MMAs
-    B_ACC_FULL = B_EMPTY + MAX_STAGES,  // [2]
-    B_ACC_EMPTY = B_ACC_FULL + 2,       // [2]
+    B_FULL = 0,                           // [MAX_STAGES] TMA landed
+    B_EMPTY = B_FULL + MAX_STAGES,        // [MAX_STAGES] stage consumed by the MMAs
+    B_ACC_FULL = B_EMPTY + MAX_STAGES,    // [2]
+    B_ACC_EMPTY = B_ACC_FULL + 2,         // [2]
     B_LR_FULL = B_ACC_EMPTY + 2,
     B_LR_SMEM_EMPTY,
     B_LR_ACC_EMPTY,
     B_DRAIN,
     B_COUNT
 };
+static_assert(B_COUNT * 8 + 8 <= 256, "barrier area");
+
+// The K = 16 MMAs of one factor's up-projection: D (+)= P_f x L_f^T.
+__device__ __forceinline__ void lr_mma(uint32_t tmem_d, uint32_t pa, uint32_t pb, const LrFactor& f,
+                                       uint32_t idesc, int& q) {
+    const uint32_t sbo = 8u * (uint32_t)f.wbox * 2u;
+    for (int j = 0; j < f.rf; j += 16, ++q) {
+        const uint32_t off = (uint32_t)(j / 64) * f.atom_bytes + (uint32_t)(j % f.wbox) * 2u;
+        umma_bf16(tmem_d, smem_desc(pa + off, 16, sbo, f.swz), smem_desc(pb + off, 16, sbo, f.swz), idesc,
+                  q != 0);
+    }
+}
 
 __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (base - raw_base);
-    const Layout L = make_layout(p.stages, p.r1, p.r2);
+    const Layout L = make_layout(p.stages, p.f1, p.f2);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.bars + B_COUNT * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.bars + B_COUNT * 8 + 4);
 
     const int warp = warp_id(), lane = lane_id();
     const int S = p.stages;
-    const int r = p.r1 + p.r2;
+    const bool has_lr = p.f1.rf + p.f2.rf > 0;
     const int tiles_m = (p.M + BM - 1) / BM;
     const int tiles_n = p.Nout / BN;
     const int num_tiles = tiles_m * tiles_n;
-    const int KT = (p.Kc + 255) / 256;
+    const int KT = p.Kc / 256;       // stages per tile
+    const int KS = p.Kc / 64;        // slabs per 128-row tile
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < MAX_STAGES; ++i) {
             mbar_init(&bars[B_FULL + i], 1);
-            mbar_init(&bars[B_SF + i], 1);
             mbar_init(&bars[B_EMPTY + i], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -148,8 +171,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&p.mapA);
         tma_prefetch_desc(&p.mapB);
-        tma_prefetch_desc(&p.mapSFA);
-        tma_prefetch_desc(&p.mapSFB);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, TMEM_COLS);
@@ -163,15 +184,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            const uint32_t stage_bytes =
-                2 * TILE_BYTES + SFA_RAW_BYTES + (p.sfb_trans ? 256u : 128u);
-            const uint32_t lr_bytes = (uint32_t)(L.np + L.n1 + L.n2) * PANEL_BYTES;
+            const uint32_t stage_bytes = 2 * TILE_BYTES + 2 * SF_STAGE_BYTES;
+            const uint32_t lr_total = 2 * (lr_bytes(p.f1) + lr_bytes(p.f2));
             uint32_t it = 0;
             bool ok = true;
             int local = 0;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
-                const int m0 = (tile / tiles_n) * BM;
-                const int n0 = (tile % tiles_n) * BN;
+                const int tm = tile / tiles_n, tn = tile % tiles_n;
+                const int m0 = tm * BM, n0 = tn * BN;
+                const uint8_t* sfa = p.sfa + (size_t)tm * KS * 512;
+                const uint8_t* sfb = p.sfb + (size_t)tn * KS * 512;
                 for (int kt = 0; kt < KT; ++kt, ++it) {
                     const int s = it % S;
                     const uint32_t ph = (it / S) & 1;
@@ -183,28 +205,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     mbar_arrive_expect_tx(fb, stage_bytes);
                     tma_load_2d(smem + L.a + s * TILE_BYTES, &p.mapA, fb, kt * BK_BYTES, m0);
                     tma_load_2d(smem + L.b + s * TILE_BYTES, &p.mapB, fb, kt * BK_BYTES, n0);
-                    tma_load_2d(smem + L.sfa_raw + s * SFA_RAW_BYTES, &p.mapSFA, fb, kt * 16, m0);
-                    if (!p.sfb_trans)
-                        tma_load_2d(smem + L.sfb_raw + s * SFB_RAW_BYTES, &p.mapSFB, fb, kt * 16,
-                                    n0 / 16);
-                    else
-                        tma_load_2d(smem + L.sfb_raw + s * SFB_RAW_BYTES, &p.mapSFB, fb,
-                                    (n0 / 16) & ~15, kt * 16);
+                    bulk_load(smem + L.sfa + s * SF_STAGE_BYTES, sfa + (size_t)kt * SF_STAGE_BYTES,
+                              SF_STAGE_BYTES, fb);
+                    bulk_load(smem + L.sfb + s * SF_STAGE_BYTES, sfb + (size_t)kt * SF_STAGE_BYTES,
+                              SF_STAGE_BYTES, fb);
                 }
-                if (!ok || r == 0) continue;
+                if (!ok || !has_lr) continue;
                 // low-rank panels of this tile, after its mainloop loads
                 if (!mbar_wait(&bars[B_LR_SMEM_EMPTY], (local & 1) ^ 1, ERR_WAIT_LR, abort_flag)) {
                     ok = false;
                     break;
                 }
                 uint64_t* lb = &bars[B_LR_FULL];
-                mbar_arrive_expect_tx(lb, lr_bytes);
-                for (int c = 0; c < L.np; ++c)
-                    tma_load_2d(smem + L.p + c * PANEL_BYTES, &p.mapP, lb, c * 64, m0);
-                for (int c = 0; c < L.n1; ++c)
-                    tma_load_2d(smem + L.l1 + c * PANEL_BYTES, &p.mapL1, lb, c * 64, n0);
-                for (int c = 0; c < L.n2; ++c)
-                    tma_load_2d(smem + L.l2 + c * PANEL_BYTES, &p.mapL2, lb, c * 64, n0);
+                mbar_arrive_expect_tx(lb, lr_total);
+                for (int a = 0; a < (p.f1.rf > 0 ? p.f1.natoms : 0); ++a) {
+                    tma_load_2d(smem + L.p1 + a * p.f1.atom_bytes, &p.mapP1, lb, p.f1.pcol + 64 * a, m0);
+                    tma_load_2d(smem + L.l1 + a * p.f1.atom_bytes, &p.mapL1, lb, 64 * a, n0);
+                }
+                for (int a = 0; a < (p.f2.rf > 0 ? p.f2.natoms : 0); ++a) {
+                    tma_load_2d(smem + L.p2 + a * p.f2.atom_bytes, &p.mapP2, lb, p.f2.pcol + 64 * a, m0);
+                    tma_load_2d(smem + L.l2 + a * p.f2.atom_bytes, &p.mapL2, lb, 64 * a, n0);
+                }
             }
             if (!ok) {
                 // let copies already issued land before the CTA exits
@@ -243,20 +264,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                 for (int kt = 0; kt < KT; ++kt, ++it) {
                     const int s = it % S;
                     const uint32_t ph = (it / S) & 1;
-                    if (!mbar_wait(&bars[B_SF + s], ph, ERR_WAIT_SF, abort_flag)) {
+                    if (!mbar_wait(&bars[B_FULL + s], ph, ERR_WAIT_FULL, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sfa_lo = sfa_lo0 + s * (SF_ATOM_BYTES >> 4);
-                    const uint32_t sfb_lo = sfb_lo0 + s * (SF_ATOM_BYTES >> 4);
+                    const uint32_t sfa_lo = sfa_lo0 + s * (SF_STAGE_BYTES >> 4);
+                    const uint32_t sfb_lo = sfb_lo0 + s * (SF_STAGE_BYTES >> 4);
+                    const uint32_t a_lo = a_lo0 + s * (TILE_BYTES >> 4);
+                    const uint32_t b_lo = b_lo0 + s * (TILE_BYTES >> 4);
 #pragma unroll
                     for (int j = 0; j < KSTEPS; ++j) {
                         tc_cp_32x128b_x4(tmem + SFA_COL + 4 * j, make_desc(sfa_lo + 32 * j, hi_sf));
                         tc_cp_32x128b_x4(tmem + SFB_COL + 4 * j, make_desc(sfb_lo + 32 * j, hi_sf));
                     }
-                    const uint32_t a_lo = a_lo0 + s * (TILE_BYTES >> 4);
-                    const uint32_t b_lo = b_lo0 + s * (TILE_BYTES >> 4);
 #pragma unroll
                     for (int j = 0; j < KSTEPS; ++j)
                         umma_nvfp4(acc, make_desc(a_lo + 2 * j, hi_sw128), make_desc(b_lo + 2 * j, hi_sw128),
@@ -264,28 +285,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     tc_commit(&bars[B_EMPTY + s]);
                 }
                 if (!ok) break;
-                if (r > 0) {
+                if (has_lr) {
                     if (!mbar_wait(&bars[B_LR_FULL], local & 1, ERR_WAIT_LR, abort_flag) ||
                         !mbar_wait(&bars[B_LR_ACC_EMPTY], (local & 1) ^ 1, ERR_WAIT_LR, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t pP = base + L.p, pL1 = base + L.l1, pL2 = base + L.l2;
                     int q = 0;
-                    for (int j = 0; j < p.r1; j += 16, ++q) {
-                        uint32_t pa = pP + (j >> 6) * PANEL_BYTES + (j & 63) * 2;
-                        uint32_t pb = pL1 + (j >> 6) * PANEL_BYTES + (j & 63) * 2;
-                        umma_bf16(tmem + LR_COL, desc_kmajor_sw128(pa), desc_kmajor_sw128(pb), idesc_lr,
-                                  q != 0);
-                    }
-                    for (int j = 0; j < p.r2; j += 16, ++q) {
-                        int jp = p.r1 + j;
-                        uint32_t pa = pP + (jp >> 6) * PANEL_BYTES + (jp & 63) * 2;
-                        uint32_t pb = pL2 + (j >> 6) * PANEL_BYTES + (j & 63) * 2;
-                        umma_bf16(tmem + LR_COL, desc_kmajor_sw128(pa), desc_kmajor_sw128(pb), idesc_lr,
-                                  q != 0);
-                    }
+                    if (p.f1.rf > 0) lr_mma(tmem + LR_COL, base + L.p1, base + L.l1, p.f1, idesc_lr, q);
+                    if (p.f2.rf > 0) lr_mma(tmem + LR_COL, base + L.p2, base + L.l2, p.f2, idesc_lr, q);
                     tc_commit(&bars[B_LR_SMEM_EMPTY]);
                 }
                 tc_commit(&bars[B_ACC_FULL + b]);
@@ -296,74 +305,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             mbar_wait(&bars[B_DRAIN], 0, ERR_WAIT_DRAIN, &no_abort);
         }
         __syncwarp();
-    } else if (warp == 2) {
-        // ------------------------------------------------ scale-factor warp
-        uint32_t it = 0;
-        bool ok = true;
-        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-            const int n0 = (tile % tiles_n) * BN;
-            for (int kt = 0; kt < KT; ++kt, ++it) {
-                const int s = it % S;
-                const uint32_t ph = (it / S) & 1;
-                if (!mbar_wait(&bars[B_FULL + s], ph, ERR_WAIT_FULL, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t raw_a = base + L.sfa_raw + s * SFA_RAW_BYTES;
-                const uint32_t raw_b = base + L.sfb_raw + s * SFB_RAW_BYTES;
-                const uint32_t at_a = base + L.sfa + s * SF_ATOM_BYTES;
-                const uint32_t at_b = base + L.sfb + s * SF_ATOM_BYTES;
-                // Rows handled by this lane: m = lane + 32 i (i = 0..3, so m / 32 = i).
-                // wa[i][j] / wb[i][j]: the scale word of row m for K-step j.
-                uint32_t wa[4][4], wb[4][4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint4 v = ld_shared_v4(raw_a + (lane + 32 * i) * 16);
-                    wa[i][0] = v.x; wa[i][1] = v.y; wa[i][2] = v.z; wa[i][3] = v.w;
-                }
-                if (!p.sfb_trans) {
-                    // raw row y (16 bytes) = scales of rows n0+16y .. +15, 16 K-blocks
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint4 g = ld_shared_v4(raw_b + ((lane >> 4) + 2 * i) * 16);
-                        wb[i][0] = g.x; wb[i][1] = g.y; wb[i][2] = g.z; wb[i][3] = g.w;
-                    }
-                } else {
-                    // raw[y][x]: y = contraction block (16 per stage), x = output
-                    // row block starting at (n0/16) & ~15
-                    const int xo = (n0 / 16) & 15;
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int col = xo + (lane >> 4) + 2 * i;
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            uint32_t v = 0;
-#pragma unroll
-                            for (int kb = 0; kb < 4; ++kb) {
-                                uint32_t byte;
-                                asm volatile("ld.shared.u8 %0, [%1];"
-                                             : "=r"(byte)
-                                             : "r"(raw_b + (4 * j + kb) * 16 + col));
-                                v |= (byte & 0xFFu) << (8 * kb);
-                            }
-                            wb[i][j] = v;
-                        }
-                    }
-                }
-                // slab j (512 B) = K-step j: row (lane) at lane * 16 holds the
-                // words of rows lane + 32 i, i = 0..3
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(at_a + 512 * j + lane * 16),
-                                 "r"(wa[0][j]), "r"(wa[1][j]), "r"(wa[2][j]), "r"(wa[3][j]) : "memory");
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(at_b + 512 * j + lane * 16),
-                                 "r"(wb[0][j]), "r"(wb[1][j]), "r"(wb[2][j]), "r"(wb[3][j]) : "memory");
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars[B_SF + s]);
-            }
-        }
     } else if (warp >= 4) {
         // ------------------------------------------------ epilogue
         const int sp = warp & 3;  // TMEM sub-partition = rows 32*sp .. +31
@@ -385,12 +326,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t v[32], lr[32];
                 tmem_ld_32x32b_x32(tmem + lane_addr + ACC_COL0 + b * BN + 32 * c, v);
-                if (r > 0) tmem_ld_32x32b_x32(tmem + lane_addr + LR_COL + 32 * c, lr);
+                if (has_lr) tmem_ld_32x32b_x32(tmem + lane_addr + LR_COL + 32 * c, lr);
                 tmem_ld_wait();
                 float y[32];
 #pragma unroll
                 for (int k = 0; k < 32; ++k)
-                    y[k] = __fmaf_rn(gab, __uint_as_float(v[k]), r > 0 ? __uint_as_float(lr[k]) : 0.0f);
+                    y[k] = __fmaf_rn(gab, __uint_as_float(v[k]), has_lr ? __uint_as_float(lr[k]) : 0.0f);
                 if (row < p.M) {
                     if (p.out_f32) {
                         float* o = reinterpret_cast<float*>(p.out) + (int64_t)row * p.Nout + n0 + 32 * c;
@@ -420,7 +361,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&bars[B_ACC_EMPTY + b]);
-                if (r > 0) mbar_arrive(&bars[B_LR_ACC_EMPTY]);
+                if (has_lr) mbar_arrive(&bars[B_LR_ACC_EMPTY]);
             }
         }
     }

@@ -45,6 +45,7 @@ struct Params {
     float* tscale;
     uint8_t* codes;
     uint8_t* scales;
+    uint8_t* slab;             // the scales again in the GEMM slab layout
     float* part;               // [splits, M, r] FP32 partial down-projections
     __nv_bfloat16* P;          // [M, r] result
     unsigned int* counters;    // [row tiles], zero on entry; left zero on exit
@@ -197,6 +198,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qdown(const __grid_constant_
                 *reinterpret_cast<uint4*>(p.codes + (int64_t)row * (p.C / 2) + col / 2) =
                     make_uint4(q0.x, q0.y, q1.x, q1.y);
                 *reinterpret_cast<uint16_t*>(p.scales + (int64_t)row * (p.C / 16) + col / 16) =
+                    (uint16_t)(s0 | (s1 << 8));
+                *reinterpret_cast<uint16_t*>(p.slab + slab_offset(row, col / 16, p.C)) =
                     (uint16_t)(s0 | (s1 << 8));
             }
         }

@@ -77,6 +77,7 @@ struct Params {
     float* tscale;
     uint8_t* codes;
     uint8_t* scales;
+    uint8_t* slab;             // null, or the scales again in the GEMM slab layout
     float* part;               // [splits, M, r] FP32 partial down-projections
     __nv_bfloat16* P;          // [M, r]
     unsigned int* counters;    // [row tiles], zero on entry; left zero on exit
@@ -361,6 +362,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
                 const int r = i / nst, st = i - r * nst;
                 const uint32_t v = ld_shared_u32(sstage + (uint32_t)r * SROW + st * 4);
                 *reinterpret_cast<uint32_t*>(p.scales + (int64_t)(m0 + r) * (p.C / 16) + c0 / 16 + 4 * st) = v;
+            }
+            // the GEMM's scale slabs: slab (row tile, K-step c0 / 64 + st),
+            // 16-byte row l = the words of tile rows l, 32 + l, 64 + l, 96 + l
+            // (rows past M hold zero scales)
+            if (p.slab) {
+                for (int i = t; i < nst * 32; i += NQ_THREADS) {
+                    const int st = i >> 5, l = i & 31;
+                    const uint32_t sa = sstage + (uint32_t)l * SROW + st * 4;
+                    const uint4 v = make_uint4(ld_shared_u32(sa), ld_shared_u32(sa + 32 * SROW),
+                                               ld_shared_u32(sa + 64 * SROW), ld_shared_u32(sa + 96 * SROW));
+                    *reinterpret_cast<uint4*>(p.slab + ((int64_t)blockIdx.x * (p.C / 64) + c0 / 64 + st) * 512 +
+                                              l * 16) = v;
+                }
             }
         }
 

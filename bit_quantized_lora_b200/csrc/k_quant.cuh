@@ -66,16 +66,54 @@ __global__ void __launch_bounds__(256) k_amax_bf16(const uint16_t* __restrict__ 
     }
 }
 
+// ---------------------------------------------------- scale slabs
+// Expands a weight's 16x16 scale grid [N/16, K/16] into the slab layout of
+// both code layouts: sf_k for W_res (rows N, contraction K) and sf_n for
+// W_res^T (rows K, contraction N).  Each 16x16 scale is repeated for its 16
+// rows; no scale is recomputed.  One thread per 16-byte slab row.
+__global__ void __launch_bounds__(256) k_expand_wsf(const uint8_t* __restrict__ grid, int64_t N,
+                                                    int64_t K, uint8_t* __restrict__ sf_k,
+                                                    uint8_t* __restrict__ sf_n) {
+    const int64_t gc = K / 16;
+    const int64_t rows_k = (N / 128) * (K / 64) * 32;  // slab rows of sf_k
+    const int64_t rows_n = (K / 128) * (N / 64) * 32;
+    const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < rows_k + rows_n; i += nthr) {
+        const bool trans = i >= rows_k;
+        const int64_t j = trans ? i - rows_k : i;
+        const int64_t l = j & 31, slab = j >> 5;
+        const int64_t ks_per = trans ? N / 64 : K / 64;
+        const int64_t t = slab / ks_per, ks = slab - t * ks_per;
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int64_t row = 128 * t + 32 * q + l;  // row of this operand
+            uint32_t v = 0;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int64_t kb = 4 * ks + b;  // 16-column block of the contraction
+                const uint32_t sb = trans ? grid[kb * gc + row / 16] : grid[(row / 16) * gc + kb];
+                v |= sb << (8 * b);
+            }
+            w[q] = v;
+        }
+        uint8_t* dst = (trans ? sf_n : sf_k) + slab * 512 + l * 16;
+        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
 // ------------------------------------------------------- 1x16 row-wise
 // Two 16-element blocks per thread per iteration (four 16-byte loads in
 // flight); stores are 8 bytes of codes and one scale byte per block;
 // consecutive threads touch consecutive blocks, so accesses are coalesced.
+// slab (optional, cols % 64 == 0): the scales again in the GEMM slab layout.
 __global__ void __launch_bounds__(256) k_quant_1x16(const uint16_t* __restrict__ x, int64_t rows,
                                                     int64_t cols, int64_t ld,
                                                     const float* __restrict__ amax,
                                                     uint8_t* __restrict__ codes,
                                                     uint8_t* __restrict__ scales,
-                                                    float* __restrict__ tscale) {
+                                                    float* __restrict__ tscale,
+                                                    uint8_t* __restrict__ slab) {
     __shared__ QTable tab;
     const QTensorFast t = make_qtensor_fast(*amax);
     build_qtable(tab, t.g, threadIdx.x, blockDim.x);
@@ -98,11 +136,13 @@ __global__ void __launch_bounds__(256) k_quant_1x16(const uint16_t* __restrict__
         const uint2 q = quant_block16_fast(w, t, tab, s);
         *reinterpret_cast<uint2*>(codes + r * (cols / 2) + c * 8) = q;
         scales[r * nb + c] = (uint8_t)s;
+        if (slab) slab[slab_offset(r, c, cols)] = (uint8_t)s;
         if (two) {
             uint32_t w2[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
             const uint2 q2 = quant_block16_fast(w2, t, tab, s);
             *reinterpret_cast<uint2*>(codes + r2 * (cols / 2) + c2 * 8) = q2;
             scales[r2 * nb + c2] = (uint8_t)s;
+            if (slab) slab[slab_offset(r2, c2, cols)] = (uint8_t)s;
         }
     }
 }

@@ -93,7 +93,11 @@ typedef struct {
  *         [N/16, K/16] serves both layouts (section 3.2).
  *   U [K, r_s], V [N, r_s], A [K, r_l], B [N, r_l]: bf16, row-major, dense.
  *   r_s, r_l: multiples of 16 with r_s + r_l <= 128 (either may be 0).
- *   s: the LoRA scale.                                                     */
+ *   s: the LoRA scale.
+ *   sf_k, sf_n: the scale grid expanded for the tensor cores, one scale per
+ *         row of w_k and of w_n (ft_expand_weight_scales fills them from
+ *         w_k.scales; ft_weight_scales_bytes(N, K) bytes each, 16-byte
+ *         aligned).  A layout of the same scales, not a new quantization.  */
 typedef struct {
     int64_t N, K, r_s, r_l;
     float s;
@@ -103,6 +107,8 @@ typedef struct {
     const void* V;
     const void* A;
     const void* B;
+    const uint8_t* sf_k;
+    const uint8_t* sf_n;
 } ft_linear;
 
 /* ft_quantize -- Q(x) for a bf16 matrix (section 3.2 block quantization).
@@ -130,6 +136,23 @@ ft_status ft_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, ft_
 ft_status ft_quantize_transpose(const void* x, int64_t rows, int64_t cols, int64_t ld,
                                 ft_block blk, const float* amax, ft_fp4* out_row,
                                 ft_fp4* out_col, void* ws, size_t ws_bytes, void* stream);
+
+/* ft_expand_weight_scales -- once per weight, after its 16x16 quantization:
+ * writes the per-row scale layouts the 4-bit GEMMs read (section 3.2: the
+ * grid of a 16x16 block serves W_res and W_res^T alike, so each grid entry
+ * is repeated for the 16 rows of its block in either orientation; no value
+ * changes).
+ *   grid : the [N/16, K/16] E4M3 scale grid of Q(W_res) (w_k.scales).
+ *   sf_k : ft_weight_scales_bytes(N, K) bytes, for w_k (rows N, along K).
+ *   sf_n : as many bytes, for w_n (rows K, along N).
+ *   N, K : multiples of 256.  Both outputs 16-byte aligned.
+ * Layout (for a matrix of R rows and C columns): [R/128][C/64][512 B];
+ * byte 16 l + 4 i + b of block (t, s) holds the scale of row 128 t + 32 i + l
+ * for columns 64 s + 16 b .. + 15 -- the order tcgen05.cp copies into the
+ * tensor memory's scale-factor layout.                                     */
+size_t ft_weight_scales_bytes(int64_t N, int64_t K);
+ft_status ft_expand_weight_scales(const uint8_t* grid, int64_t N, int64_t K, uint8_t* sf_k,
+                                  uint8_t* sf_n, void* stream);
 
 /* ft_linear_fwd -- Eq. 2 with LoRA fusion (section 3.3): one pass over X
  * emits Q(X) and the down-projections P = [bf16(X U) | bf16(s X A)]; one

@@ -38,9 +38,9 @@ def test_every_declared_symbol_is_exported_and_bound(L):
 
 
 def test_struct_layouts_match_c():
-    # int64 x4, float (+4 pad), two 48-byte views, four pointers
+    # int64 x4, float (+4 pad), two 48-byte views, six pointers
     assert ctypes.sizeof(FtFp4) == 48
-    assert ctypes.sizeof(FtLinear) == 32 + 8 + 2 * 48 + 4 * 8
+    assert ctypes.sizeof(FtLinear) == 32 + 8 + 2 * 48 + 6 * 8
 
 
 def test_status_strings(L):
@@ -91,7 +91,7 @@ def _linear(N=256, K=256, r_s=16, r_l=16):
     p = 0x100000
     wk = FtFp4(p, p, p, N, K, 1)
     wn = FtFp4(p, p, p, K, N, 1)
-    return FtLinear(N, K, r_s, r_l, 1.0, wk, wn, p, p, p, p)
+    return FtLinear(N, K, r_s, r_l, 1.0, wk, wn, p, p, p, p, p, p)
 
 
 def test_linear_validation_happens_on_the_host(L):
@@ -112,6 +112,13 @@ def test_linear_validation_happens_on_the_host(L):
     shared = _linear()
     shared.w_n.scales = 0x300000
     assert L.ft_linear_fwd(ctypes.byref(shared), x, 128, None, x, 0, x, x, ws, None) == FT_ERR_INVALID_ARG
+    # the expanded weight scales are required and 16-byte aligned
+    no_sf = _linear()
+    no_sf.sf_n = None
+    assert L.ft_linear_fwd(ctypes.byref(no_sf), x, 128, None, x, 0, x, x, ws, None) == FT_ERR_INVALID_ARG
+    odd_sf = _linear()
+    odd_sf.sf_k = 0x100008
+    assert L.ft_linear_fwd(ctypes.byref(odd_sf), x, 128, None, x, 0, x, x, ws, None) == FT_ERR_ALIGN
     # M = 0: nothing to do
     assert L.ft_linear_fwd(ctypes.byref(ok), x, 0, None, x, 0, x, x, ws, None) == FT_OK
     assert L.ft_linear_bwd(ctypes.byref(bad_n), x, x, x, 128, None, x, 0, x, x, x, ws, None) == FT_ERR_SHAPE
@@ -133,3 +140,13 @@ def test_workspace_qact_offsets_lie_inside_the_workspace(L):
     bad = ctypes.c_size_t()
     assert L.ft_workspace_qact(-1, 1, 1, 0, 0, ctypes.byref(bad), ctypes.byref(bad), ctypes.byref(bad)) == FT_ERR_INVALID_ARG
     assert L.ft_workspace_qact(1, 1, 1, 0, 0, None, ctypes.byref(bad), ctypes.byref(bad)) == FT_ERR_INVALID_ARG
+
+
+def test_weight_scale_expansion_validation(L):
+    assert L.ft_weight_scales_bytes(3072, 3072) == 3072 * 3072 // 16
+    assert L.ft_weight_scales_bytes(-1, 256) == 0
+    g = 0x100000
+    assert L.ft_expand_weight_scales(None, 256, 256, g, g, None) == FT_ERR_INVALID_ARG
+    assert L.ft_expand_weight_scales(g, 320, 256, g, g, None) == FT_ERR_SHAPE
+    assert L.ft_expand_weight_scales(g, 256, 256, g + 8, g, None) == FT_ERR_ALIGN
+    assert L.ft_expand_weight_scales(g, 0, 256, g, g, None) == FT_OK
