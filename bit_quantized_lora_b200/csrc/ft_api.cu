@@ -516,7 +516,7 @@ ft::gemm::LrFactor gemm_factor(int64_t rf, int64_t pcol) {
     f.wbox = rf <= 16 ? 16 : rf <= 32 ? 32 : 64;
     f.natoms = rf <= 64 ? 1 : 2;
     f.swz = f.wbox == 16 ? ft::SWZ_32B : f.wbox == 32 ? ft::SWZ_64B : ft::SWZ_128B;
-    f.atom_bytes = 128u * (uint32_t)f.wbox * 2u;
+    f.row_bytes = (uint32_t)f.wbox * 2u;
     return f;
 }
 
@@ -535,22 +535,22 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_slab, const float* g
     std::memset(&p, 0, sizeof(p));
     FT_TRY(encode_2d(&p.mapA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, Kc / 2, M, Kc / 2, 128, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B));
-    FT_TRY(encode_2d(&p.mapB, CU_TENSOR_MAP_DATA_TYPE_UINT8, b_codes, Kc / 2, Nout, Kc / 2, 128, 128,
-                     CU_TENSOR_MAP_SWIZZLE_128B));
+    FT_TRY(encode_2d(&p.mapB, CU_TENSOR_MAP_DATA_TYPE_UINT8, b_codes, Kc / 2, Nout, Kc / 2, 128,
+                     ft::gemm::BN, CU_TENSOR_MAP_SWIZZLE_128B));
     const int64_t r = r1 + r2;
     p.f1 = gemm_factor(r1, 0);
     p.f2 = gemm_factor(r2, r1);
     if (r1 > 0) {
         FT_TRY(encode_2d(&p.mapP1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P, r, M, r * 2, p.f1.wbox, 128,
                          swizzle_for(p.f1.wbox)));
-        FT_TRY(encode_2d(&p.mapL1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1, r1, Nout, r1 * 2, p.f1.wbox, 128,
-                         swizzle_for(p.f1.wbox)));
+        FT_TRY(encode_2d(&p.mapL1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1, r1, Nout, r1 * 2, p.f1.wbox,
+                         ft::gemm::BN, swizzle_for(p.f1.wbox)));
     }
     if (r2 > 0) {
         FT_TRY(encode_2d(&p.mapP2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P, r, M, r * 2, p.f2.wbox, 128,
                          swizzle_for(p.f2.wbox)));
-        FT_TRY(encode_2d(&p.mapL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2, r2, Nout, r2 * 2, p.f2.wbox, 128,
-                         swizzle_for(p.f2.wbox)));
+        FT_TRY(encode_2d(&p.mapL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2, r2, Nout, r2 * 2, p.f2.wbox,
+                         ft::gemm::BN, swizzle_for(p.f2.wbox)));
     }
     p.sfa = a_slab;
     p.sfb = b_slab;

@@ -24,22 +24,25 @@
 // MMA reads (row m at TMEM lane m % 32 of every lane quarter, column
 // c + m / 32), so the MMA warp copies it straight from the TMA buffer.
 //
-// Blackwell mapping: one CTA per SM, persistent over 128x128 output tiles.
-//   warp 0  TMA producer: FP4 code tiles (128 B swizzle) and the two scale
-//           slabs of each stage (bulk copies), the tile's P / L1 / L2 panels.
-//   warp 1  TMEM owner and UMMA issuer: per K-step one tcgen05.cp of each
-//           operand's slab into TMEM and one
-//           tcgen05.mma.kind::mxf4nvf4.block16 (K = 64) into a
-//           double-buffered FP32 accumulator, then tcgen05.mma kind::f16 for
-//           the low-rank panels into a separate accumulator.
-//   warps 4-7 epilogue: tcgen05.ld both accumulators, combine, store.
-// TMEM columns: [0,128) acc0, [128,256) acc1, [256,384) low-rank acc,
-// [384,400) A scales, [400,416) B scales.
+// Blackwell mapping: one CTA per SM, persistent over 128x256 output tiles
+// (a tcgen05 MMA costs about the same for N = 128 as for N = 256, so the
+// wide tile doubles the work per instruction).
+//   warp 0  TMA producer: FP4 code tiles (128 B swizzle) and the scale slabs
+//           of each stage (bulk copies), the tile's P / L1 / L2 panels.
+//   warp 1  TMEM owner and UMMA issuer: four
+//           tcgen05.mma.kind::mxf4nvf4.block16 (K = 64, N = 256) per stage
+//           into the FP32 accumulator, then the low-rank up-projection
+//           (kind::f16) in two 128-column halves into its own accumulator.
+//   warp 2  scale warp: tcgen05.cp of each stage's slabs into a two-deep
+//           ring of scale columns, ahead of the MMAs (copies issued by
+//           another warp overlap the MMAs instead of queueing behind them).
+//   warps 4-7 epilogue: tcgen05.ld both accumulators, combine, store Y once.
+// TMEM columns: [0,256) accumulator, [256,384) low-rank half,
+// [384,480) scale ring (per slot: A 16 columns, B 32 columns).
 //
 // Low-rank panels are K-major with the rank as K, each factor's part of P
 // and the factor itself swizzled to its own width (16, 32 or 64 columns per
-// 32, 64 or 128-byte row; two 64-column atoms above 64), so a rank-16
-// factor costs 4 KiB of shared memory, not a padded 16 KiB panel.
+// 32, 64 or 128-byte row; two 64-column atoms above 64).
 #pragma once
 
 #include <cuda.h>
@@ -50,25 +53,27 @@ namespace ft {
 namespace gemm {
 
 constexpr int BM = 128;
-constexpr int BN = 128;
+constexpr int BN = 256;
 constexpr int BK_BYTES = 128;  // 256 FP4 elements of K per stage
 constexpr int KSTEPS = 4;      // MMAs of K = 64 per stage
-constexpr int MAX_STAGES = 6;
+constexpr int MAX_STAGES = 4;
 constexpr int NUM_THREADS = 256;
-constexpr int TILE_BYTES = BM * BK_BYTES;      // 16 KiB, A or B stage
-constexpr int SF_STAGE_BYTES = KSTEPS * 512;   // four slabs of one operand
+constexpr int A_BYTES = BM * BK_BYTES;         // 16 KiB
+constexpr int B_BYTES = BN * BK_BYTES;         // 32 KiB
+constexpr int SFA_STAGE_BYTES = KSTEPS * 512;  // four slabs (128 rows)
+constexpr int SFB_STAGE_BYTES = 2 * KSTEPS * 512;  // two row halves x four slabs
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t ACC_COL0 = 0, LR_COL = 256, SFA_COL = 384, SFB_COL = 400;
+constexpr uint32_t ACC_COL = 0, LR_COL = 256, SF_COL = 384, SF_SLOT_COLS = 48;
 
 // One low-rank factor's panels: P columns [pcol, pcol + rf) for the tile's
-// 128 rows (A operand) and L [128 output rows, rf] (B operand), both K-major.
+// 128 rows (A operand) and L [256 output rows, rf] (B operand), both K-major.
 struct LrFactor {
     int rf;        // rank (0: absent)
     int wbox;      // 16, 32 or 64 elements per swizzled row
     int natoms;    // 1, or 2 above 64
     int pcol;      // first column of P
     uint32_t swz;  // descriptor swizzle code
-    uint32_t atom_bytes;  // 128 rows x wbox x 2
+    uint32_t row_bytes;  // wbox x 2
 };
 
 struct Params {
@@ -88,21 +93,25 @@ struct Layout {
     uint32_t a, b, sfa, sfb, p1, p2, l1, l2, bars, total;
 };
 
-__host__ __device__ inline uint32_t lr_bytes(const LrFactor& f) {
-    return f.rf > 0 ? (uint32_t)f.natoms * f.atom_bytes : 0u;
+// bytes of a factor's P panel (128 rows) and L panel (256 rows)
+__host__ __device__ inline uint32_t p_bytes(const LrFactor& f) {
+    return f.rf > 0 ? (uint32_t)f.natoms * 128u * f.row_bytes : 0u;
+}
+__host__ __device__ inline uint32_t l_bytes(const LrFactor& f) {
+    return f.rf > 0 ? (uint32_t)f.natoms * 256u * f.row_bytes : 0u;
 }
 
 __host__ __device__ inline Layout make_layout(int stages, const LrFactor& f1, const LrFactor& f2) {
     Layout L;
     uint32_t o = 0;
-    L.a = o;    o += stages * TILE_BYTES;
-    L.b = o;    o += stages * TILE_BYTES;
-    L.p1 = o;   o += lr_bytes(f1);
-    L.l1 = o;   o += lr_bytes(f1);
-    L.p2 = o;   o += lr_bytes(f2);
-    L.l2 = o;   o += lr_bytes(f2);
-    L.sfa = o;  o += stages * SF_STAGE_BYTES;
-    L.sfb = o;  o += stages * SF_STAGE_BYTES;
+    L.a = o;    o += stages * A_BYTES;
+    L.b = o;    o += stages * B_BYTES;
+    L.p1 = o;   o += p_bytes(f1);
+    L.l1 = o;   o += l_bytes(f1);
+    L.p2 = o;   o += p_bytes(f2);
+    L.l2 = o;   o += l_bytes(f2);
+    L.sfa = o;  o += stages * SFA_STAGE_BYTES;
+    L.sfb = o;  o += stages * SFB_STAGE_BYTES;
     L.bars = o; o += 256;  // barriers, TMEM slot, abort flag
     L.total = o + 1024;    // slack for 1 KiB alignment of the base
     return L;
@@ -110,25 +119,32 @@ __host__ __device__ inline Layout make_layout(int stages, const LrFactor& f1, co
 
 // barrier slots (uint64 each) inside the 256-byte barrier area
 enum {
-    B_FULL = 0,                           // [MAX_STAGES] TMA landed
-    B_EMPTY = B_FULL + MAX_STAGES,        // [MAX_STAGES] stage consumed by the MMAs
-    B_ACC_FULL = B_EMPTY + MAX_STAGES,    // [2]
-    B_ACC_EMPTY = B_ACC_FULL + 2,         // [2]
-    B_LR_FULL = B_ACC_EMPTY + 2,
-    B_LR_SMEM_EMPTY,
-    B_LR_ACC_EMPTY,
+    B_FULL = 0,                        // [MAX_STAGES] TMA landed
+    B_EMPTY = B_FULL + MAX_STAGES,     // [MAX_STAGES] stage consumed by the MMAs
+    B_SF_READY = B_EMPTY + MAX_STAGES, // [2] scale slot copied into TMEM
+    B_SF_FREE = B_SF_READY + 2,        // [2] scale slot read by its MMAs
+    B_ACC_FULL = B_SF_FREE + 2,
+    B_ACC_EMPTY,                       // 4 epilogue warps
+    B_LR_FULL,                         // panels landed
+    B_LR_SMEM_EMPTY,                   // panels consumed
+    B_LR_READY,                        // low-rank half computed
+    B_LR_EMPTY,                        // low-rank half read (4 epilogue warps)
     B_DRAIN,
+    B_DRAIN_SF,
     B_COUNT
 };
 static_assert(B_COUNT * 8 + 8 <= 256, "barrier area");
 
-// The K = 16 MMAs of one factor's up-projection: D (+)= P_f x L_f^T.
-__device__ __forceinline__ void lr_mma(uint32_t tmem_d, uint32_t pa, uint32_t pb, const LrFactor& f,
+// The K = 16 MMAs of one factor's up-projection for output rows
+// [128 h, 128 h + 128) of the tile: D (+)= P_f x L_f[half h]^T.
+__device__ __forceinline__ void lr_mma(uint32_t tmem_d, uint32_t pa, uint32_t pb, const LrFactor& f, int h,
                                        uint32_t idesc, int& q) {
-    const uint32_t sbo = 8u * (uint32_t)f.wbox * 2u;
+    const uint32_t sbo = 8u * f.row_bytes;
     for (int j = 0; j < f.rf; j += 16, ++q) {
-        const uint32_t off = (uint32_t)(j / 64) * f.atom_bytes + (uint32_t)(j % f.wbox) * 2u;
-        umma_bf16(tmem_d, smem_desc(pa + off, 16, sbo, f.swz), smem_desc(pb + off, 16, sbo, f.swz), idesc,
+        const uint32_t a = (uint32_t)(j / 64), k = (uint32_t)(j % f.wbox) * 2u;
+        const uint32_t ao = a * 128u * f.row_bytes + k;
+        const uint32_t bo = a * 256u * f.row_bytes + (uint32_t)h * 128u * f.row_bytes + k;
+        umma_bf16(tmem_d, smem_desc(pa + ao, 16, sbo, f.swz), smem_desc(pb + bo, 16, sbo, f.swz), idesc,
                   q != 0);
     }
 }
@@ -149,8 +165,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
     const int tiles_m = (p.M + BM - 1) / BM;
     const int tiles_n = p.Nout / BN;
     const int num_tiles = tiles_m * tiles_n;
-    const int KT = p.Kc / 256;       // stages per tile
-    const int KS = p.Kc / 64;        // slabs per 128-row tile
+    const int KT = p.Kc / 256;  // stages per tile
+    const int KS = p.Kc / 64;   // slabs per 128-row tile
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < MAX_STAGES; ++i) {
@@ -158,13 +174,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             mbar_init(&bars[B_EMPTY + i], 1);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&bars[B_ACC_FULL + i], 1);
-            mbar_init(&bars[B_ACC_EMPTY + i], 4);
+            mbar_init(&bars[B_SF_READY + i], 1);
+            mbar_init(&bars[B_SF_FREE + i], 1);
         }
+        mbar_init(&bars[B_ACC_FULL], 1);
+        mbar_init(&bars[B_ACC_EMPTY], 4);
         mbar_init(&bars[B_LR_FULL], 1);
         mbar_init(&bars[B_LR_SMEM_EMPTY], 1);
-        mbar_init(&bars[B_LR_ACC_EMPTY], 4);
+        mbar_init(&bars[B_LR_READY], 1);
+        mbar_init(&bars[B_LR_EMPTY], 4);
         mbar_init(&bars[B_DRAIN], 1);
+        mbar_init(&bars[B_DRAIN_SF], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -184,8 +204,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            const uint32_t stage_bytes = 2 * TILE_BYTES + 2 * SF_STAGE_BYTES;
-            const uint32_t lr_total = 2 * (lr_bytes(p.f1) + lr_bytes(p.f2));
+            const uint32_t stage_bytes = A_BYTES + B_BYTES + SFA_STAGE_BYTES + SFB_STAGE_BYTES;
+            const uint32_t lr_total = p_bytes(p.f1) + l_bytes(p.f1) + p_bytes(p.f2) + l_bytes(p.f2);
             uint32_t it = 0;
             bool ok = true;
             int local = 0;
@@ -193,7 +213,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                 const int tm = tile / tiles_n, tn = tile % tiles_n;
                 const int m0 = tm * BM, n0 = tn * BN;
                 const uint8_t* sfa = p.sfa + (size_t)tm * KS * 512;
-                const uint8_t* sfb = p.sfb + (size_t)tn * KS * 512;
+                const uint8_t* sfb0 = p.sfb + (size_t)(2 * tn) * KS * 512;
+                const uint8_t* sfb1 = sfb0 + (size_t)KS * 512;
                 for (int kt = 0; kt < KT; ++kt, ++it) {
                     const int s = it % S;
                     const uint32_t ph = (it / S) & 1;
@@ -203,12 +224,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     }
                     uint64_t* fb = &bars[B_FULL + s];
                     mbar_arrive_expect_tx(fb, stage_bytes);
-                    tma_load_2d(smem + L.a + s * TILE_BYTES, &p.mapA, fb, kt * BK_BYTES, m0);
-                    tma_load_2d(smem + L.b + s * TILE_BYTES, &p.mapB, fb, kt * BK_BYTES, n0);
-                    bulk_load(smem + L.sfa + s * SF_STAGE_BYTES, sfa + (size_t)kt * SF_STAGE_BYTES,
-                              SF_STAGE_BYTES, fb);
-                    bulk_load(smem + L.sfb + s * SF_STAGE_BYTES, sfb + (size_t)kt * SF_STAGE_BYTES,
-                              SF_STAGE_BYTES, fb);
+                    tma_load_2d(smem + L.a + s * A_BYTES, &p.mapA, fb, kt * BK_BYTES, m0);
+                    tma_load_2d(smem + L.b + s * B_BYTES, &p.mapB, fb, kt * BK_BYTES, n0);
+                    const size_t so = (size_t)kt * SFA_STAGE_BYTES;
+                    bulk_load(smem + L.sfa + s * SFA_STAGE_BYTES, sfa + so, SFA_STAGE_BYTES, fb);
+                    bulk_load(smem + L.sfb + s * SFB_STAGE_BYTES, sfb0 + so, SFA_STAGE_BYTES, fb);
+                    bulk_load(smem + L.sfb + s * SFB_STAGE_BYTES + SFA_STAGE_BYTES, sfb1 + so, SFA_STAGE_BYTES, fb);
                 }
                 if (!ok || !has_lr) continue;
                 // low-rank panels of this tile, after its mainloop loads
@@ -219,12 +240,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                 uint64_t* lb = &bars[B_LR_FULL];
                 mbar_arrive_expect_tx(lb, lr_total);
                 for (int a = 0; a < (p.f1.rf > 0 ? p.f1.natoms : 0); ++a) {
-                    tma_load_2d(smem + L.p1 + a * p.f1.atom_bytes, &p.mapP1, lb, p.f1.pcol + 64 * a, m0);
-                    tma_load_2d(smem + L.l1 + a * p.f1.atom_bytes, &p.mapL1, lb, 64 * a, n0);
+                    tma_load_2d(smem + L.p1 + a * 128 * p.f1.row_bytes, &p.mapP1, lb, p.f1.pcol + 64 * a, m0);
+                    tma_load_2d(smem + L.l1 + a * 256 * p.f1.row_bytes, &p.mapL1, lb, 64 * a, n0);
                 }
                 for (int a = 0; a < (p.f2.rf > 0 ? p.f2.natoms : 0); ++a) {
-                    tma_load_2d(smem + L.p2 + a * p.f2.atom_bytes, &p.mapP2, lb, p.f2.pcol + 64 * a, m0);
-                    tma_load_2d(smem + L.l2 + a * p.f2.atom_bytes, &p.mapL2, lb, 64 * a, n0);
+                    tma_load_2d(smem + L.p2 + a * 128 * p.f2.row_bytes, &p.mapP2, lb, p.f2.pcol + 64 * a, m0);
+                    tma_load_2d(smem + L.l2 + a * 256 * p.f2.row_bytes, &p.mapL2, lb, 64 * a, n0);
                 }
             }
             if (!ok) {
@@ -240,69 +261,104 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
         // ------------------------------------------------ UMMA issuer
         if (lane == 0) {
             const uint32_t idesc = idesc_nvfp4(BM, BN);
-            const uint32_t idesc_lr = idesc_bf16(BM, BN, 0, 0);
+            const uint32_t idesc_lr = idesc_bf16(BM, 128, 0, 0);
             // descriptor words: lo = start >> 4 | (LBO >> 4) << 16;
             // hi = SBO >> 4 | version 1 << 14 | layout << 29
             const uint32_t hi_sw128 = (1024u >> 4) | (1u << 14) | (SWZ_128B << 29);
-            const uint32_t hi_sf = (128u >> 4) | (1u << 14);  // 8-row groups 128 B apart
             const uint32_t a_lo0 = ((base + L.a) >> 4) | (1u << 16);
             const uint32_t b_lo0 = ((base + L.b) >> 4) | (1u << 16);
-            const uint32_t sfa_lo0 = (base + L.sfa) >> 4;  // one 16-byte column: LBO unused
-            const uint32_t sfb_lo0 = (base + L.sfb) >> 4;
             uint32_t it = 0;
             bool ok = true;
             int local = 0;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
-                const int b = local & 1;
-                const uint32_t acc = tmem + ACC_COL0 + b * BN;
-                if (!mbar_wait(&bars[B_ACC_EMPTY + b], ((local >> 1) & 1) ^ 1, ERR_WAIT_ACC_EMPTY,
-                               abort_flag)) {
+                if (!mbar_wait(&bars[B_ACC_EMPTY], (local & 1) ^ 1, ERR_WAIT_ACC_EMPTY, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 for (int kt = 0; kt < KT; ++kt, ++it) {
                     const int s = it % S;
-                    const uint32_t ph = (it / S) & 1;
-                    if (!mbar_wait(&bars[B_FULL + s], ph, ERR_WAIT_FULL, abort_flag)) {
+                    const int sb = it & 1;
+                    if (!mbar_wait(&bars[B_FULL + s], (it / S) & 1, ERR_WAIT_FULL, abort_flag) ||
+                        !mbar_wait(&bars[B_SF_READY + sb], (it >> 1) & 1, ERR_WAIT_SF, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sfa_lo = sfa_lo0 + s * (SF_STAGE_BYTES >> 4);
-                    const uint32_t sfb_lo = sfb_lo0 + s * (SF_STAGE_BYTES >> 4);
-                    const uint32_t a_lo = a_lo0 + s * (TILE_BYTES >> 4);
-                    const uint32_t b_lo = b_lo0 + s * (TILE_BYTES >> 4);
-#pragma unroll
-                    for (int j = 0; j < KSTEPS; ++j) {
-                        tc_cp_32x128b_x4(tmem + SFA_COL + 4 * j, make_desc(sfa_lo + 32 * j, hi_sf));
-                        tc_cp_32x128b_x4(tmem + SFB_COL + 4 * j, make_desc(sfb_lo + 32 * j, hi_sf));
-                    }
+                    const uint32_t a_lo = a_lo0 + s * (A_BYTES >> 4);
+                    const uint32_t b_lo = b_lo0 + s * (B_BYTES >> 4);
+                    const uint32_t sf = tmem + SF_COL + sb * SF_SLOT_COLS;
 #pragma unroll
                     for (int j = 0; j < KSTEPS; ++j)
-                        umma_nvfp4(acc, make_desc(a_lo + 2 * j, hi_sw128), make_desc(b_lo + 2 * j, hi_sw128),
-                                   idesc, tmem + SFA_COL + 4 * j, tmem + SFB_COL + 4 * j, (kt | j) != 0);
+                        umma_nvfp4(tmem + ACC_COL, make_desc(a_lo + 2 * j, hi_sw128),
+                                   make_desc(b_lo + 2 * j, hi_sw128), idesc, sf + 4 * j, sf + 16 + 8 * j,
+                                   (kt | j) != 0);
                     tc_commit(&bars[B_EMPTY + s]);
+                    tc_commit(&bars[B_SF_FREE + sb]);
                 }
                 if (!ok) break;
+                tc_commit(&bars[B_ACC_FULL]);
                 if (has_lr) {
-                    if (!mbar_wait(&bars[B_LR_FULL], local & 1, ERR_WAIT_LR, abort_flag) ||
-                        !mbar_wait(&bars[B_LR_ACC_EMPTY], (local & 1) ^ 1, ERR_WAIT_LR, abort_flag)) {
+                    if (!mbar_wait(&bars[B_LR_FULL], local & 1, ERR_WAIT_LR, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
-                    int q = 0;
-                    if (p.f1.rf > 0) lr_mma(tmem + LR_COL, base + L.p1, base + L.l1, p.f1, idesc_lr, q);
-                    if (p.f2.rf > 0) lr_mma(tmem + LR_COL, base + L.p2, base + L.l2, p.f2, idesc_lr, q);
+                    for (int h = 0; h < 2 && ok; ++h) {
+                        const int u = 2 * local + h;  // use of the low-rank columns
+                        if (!mbar_wait(&bars[B_LR_EMPTY], (u & 1) ^ 1, ERR_WAIT_LR, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        int q = 0;
+                        if (p.f1.rf > 0) lr_mma(tmem + LR_COL, base + L.p1, base + L.l1, p.f1, h, idesc_lr, q);
+                        if (p.f2.rf > 0) lr_mma(tmem + LR_COL, base + L.p2, base + L.l2, p.f2, h, idesc_lr, q);
+                        tc_commit(&bars[B_LR_READY]);
+                    }
                     tc_commit(&bars[B_LR_SMEM_EMPTY]);
                 }
-                tc_commit(&bars[B_ACC_FULL + b]);
             }
             // every tcgen05 op issued by this thread completes before TMEM is freed
             tc_commit(&bars[B_DRAIN]);
             volatile int no_abort = 0;
             mbar_wait(&bars[B_DRAIN], 0, ERR_WAIT_DRAIN, &no_abort);
+        }
+        __syncwarp();
+    } else if (warp == 2) {
+        // ------------------------------------------------ scale warp
+        if (lane == 0) {
+            const uint32_t hi_sf = (128u >> 4) | (1u << 14);  // 8-row groups 128 B apart
+            const uint32_t sfa_lo0 = (base + L.sfa) >> 4;     // one 16-byte column: LBO unused
+            const uint32_t sfb_lo0 = (base + L.sfb) >> 4;
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                for (int kt = 0; kt < KT; ++kt, ++it) {
+                    const int s = it % S;
+                    const int sb = it & 1;
+                    if (!mbar_wait(&bars[B_FULL + s], (it / S) & 1, ERR_WAIT_FULL, abort_flag) ||
+                        !mbar_wait(&bars[B_SF_FREE + sb], ((it >> 1) & 1) ^ 1, ERR_WAIT_SF, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sfa_lo = sfa_lo0 + s * (SFA_STAGE_BYTES >> 4);
+                    const uint32_t sfb_lo = sfb_lo0 + s * (SFB_STAGE_BYTES >> 4);
+                    const uint32_t sf = tmem + SF_COL + sb * SF_SLOT_COLS;
+#pragma unroll
+                    for (int j = 0; j < KSTEPS; ++j) {
+                        // A: rows 0-127; B: rows 0-127 then 128-255 (four columns each)
+                        tc_cp_32x128b_x4(sf + 4 * j, make_desc(sfa_lo + 32 * j, hi_sf));
+                        tc_cp_32x128b_x4(sf + 16 + 8 * j, make_desc(sfb_lo + 32 * j, hi_sf));
+                        tc_cp_32x128b_x4(sf + 20 + 8 * j,
+                                         make_desc(sfb_lo + (SFA_STAGE_BYTES >> 4) + 32 * j, hi_sf));
+                    }
+                    tc_commit(&bars[B_SF_READY + sb]);
+                }
+            }
+            tc_commit(&bars[B_DRAIN_SF]);
+            volatile int no_abort = 0;
+            mbar_wait(&bars[B_DRAIN_SF], 0, ERR_WAIT_DRAIN, &no_abort);
         }
         __syncwarp();
     } else if (warp >= 4) {
@@ -312,57 +368,66 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
         int local = 0;
         const float gab = __fmul_rn(*p.ga, *p.gb);
         for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
-            const int b = local & 1;
             const int m0 = (tile / tiles_n) * BM;
             const int n0 = (tile % tiles_n) * BN;
-            if (!mbar_wait(&bars[B_ACC_FULL + b], (local >> 1) & 1, ERR_WAIT_ACC_FULL, abort_flag)) {
+            if (!mbar_wait(&bars[B_ACC_FULL], local & 1, ERR_WAIT_ACC_FULL, abort_flag)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             const int row = m0 + 32 * sp + lane;
             const uint32_t lane_addr = (uint32_t)(32 * sp) << 16;
+            for (int h = 0; h < 2 && ok; ++h) {
+                if (has_lr) {
+                    if (!mbar_wait(&bars[B_LR_READY], (2 * local + h) & 1, ERR_WAIT_LR, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                }
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t v[32], lr[32];
-                tmem_ld_32x32b_x32(tmem + lane_addr + ACC_COL0 + b * BN + 32 * c, v);
-                if (has_lr) tmem_ld_32x32b_x32(tmem + lane_addr + LR_COL + 32 * c, lr);
-                tmem_ld_wait();
-                float y[32];
+                for (int c = 0; c < 4; ++c) {
+                    const int col = 128 * h + 32 * c;  // tile column
+                    uint32_t v[32], lr[32];
+                    tmem_ld_32x32b_x32(tmem + lane_addr + ACC_COL + col, v);
+                    if (has_lr) tmem_ld_32x32b_x32(tmem + lane_addr + LR_COL + 32 * c, lr);
+                    tmem_ld_wait();
+                    float y[32];
 #pragma unroll
-                for (int k = 0; k < 32; ++k)
-                    y[k] = __fmaf_rn(gab, __uint_as_float(v[k]), has_lr ? __uint_as_float(lr[k]) : 0.0f);
-                if (row < p.M) {
-                    if (p.out_f32) {
-                        float* o = reinterpret_cast<float*>(p.out) + (int64_t)row * p.Nout + n0 + 32 * c;
+                    for (int k = 0; k < 32; ++k)
+                        y[k] = __fmaf_rn(gab, __uint_as_float(v[k]), has_lr ? __uint_as_float(lr[k]) : 0.0f);
+                    if (row < p.M) {
+                        if (p.out_f32) {
+                            float* o = reinterpret_cast<float*>(p.out) + (int64_t)row * p.Nout + n0 + col;
 #pragma unroll
-                        for (int k = 0; k < 32; k += 4)
-                            *reinterpret_cast<float4*>(o + k) = make_float4(y[k], y[k + 1], y[k + 2], y[k + 3]);
-                    } else {
-                        __nv_bfloat16* o =
-                            reinterpret_cast<__nv_bfloat16*>(p.out) + (int64_t)row * p.Nout + n0 + 32 * c;
+                            for (int k = 0; k < 32; k += 4)
+                                *reinterpret_cast<float4*>(o + k) = make_float4(y[k], y[k + 1], y[k + 2], y[k + 3]);
+                        } else {
+                            __nv_bfloat16* o =
+                                reinterpret_cast<__nv_bfloat16*>(p.out) + (int64_t)row * p.Nout + n0 + col;
 #pragma unroll
-                        for (int k = 0; k < 32; k += 8) {
-                            uint4 u;
-                            __nv_bfloat162 t0 = __floats2bfloat162_rn(y[k], y[k + 1]);
-                            __nv_bfloat162 t1 = __floats2bfloat162_rn(y[k + 2], y[k + 3]);
-                            __nv_bfloat162 t2 = __floats2bfloat162_rn(y[k + 4], y[k + 5]);
-                            __nv_bfloat162 t3 = __floats2bfloat162_rn(y[k + 6], y[k + 7]);
-                            u.x = *reinterpret_cast<uint32_t*>(&t0);
-                            u.y = *reinterpret_cast<uint32_t*>(&t1);
-                            u.z = *reinterpret_cast<uint32_t*>(&t2);
-                            u.w = *reinterpret_cast<uint32_t*>(&t3);
-                            *reinterpret_cast<uint4*>(o + k) = u;
+                            for (int k = 0; k < 32; k += 8) {
+                                uint4 u;
+                                __nv_bfloat162 t0 = __floats2bfloat162_rn(y[k], y[k + 1]);
+                                __nv_bfloat162 t1 = __floats2bfloat162_rn(y[k + 2], y[k + 3]);
+                                __nv_bfloat162 t2 = __floats2bfloat162_rn(y[k + 4], y[k + 5]);
+                                __nv_bfloat162 t3 = __floats2bfloat162_rn(y[k + 6], y[k + 7]);
+                                u.x = *reinterpret_cast<uint32_t*>(&t0);
+                                u.y = *reinterpret_cast<uint32_t*>(&t1);
+                                u.z = *reinterpret_cast<uint32_t*>(&t2);
+                                u.w = *reinterpret_cast<uint32_t*>(&t3);
+                                *reinterpret_cast<uint4*>(o + k) = u;
+                            }
                         }
                     }
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0 && has_lr) mbar_arrive(&bars[B_LR_EMPTY]);
             }
-            tc_fence_before();
+            if (!ok) break;
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&bars[B_ACC_EMPTY + b]);
-                if (has_lr) mbar_arrive(&bars[B_LR_ACC_EMPTY]);
-            }
+            if (lane == 0) mbar_arrive(&bars[B_ACC_EMPTY]);
         }
     }
 
