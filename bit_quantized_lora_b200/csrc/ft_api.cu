@@ -552,17 +552,21 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_slab, const float* g
         FT_TRY(encode_2d(&p.mapL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2, r2, Nout, r2 * 2, p.f2.wbox,
                          ft::gemm::BN, swizzle_for(p.f2.wbox)));
     }
+    // output chunks of 64 bytes per row (32 bf16 / 16 f32 columns) x 128 rows
+    const int64_t esize = (ot == FT_F32) ? 4 : 2;
+    FT_TRY(encode_2d(&p.mapY, ot == FT_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                     out, Nout, M, Nout * esize, (uint32_t)(64 / esize), 128, CU_TENSOR_MAP_SWIZZLE_64B));
     p.sfa = a_slab;
     p.sfb = b_slab;
     p.ga = ga;
     p.gb = gb;
-    p.out = out;
     p.out_f32 = (ot == FT_F32);
     p.M = (int)M;
     p.Nout = (int)Nout;
     p.Kc = (int)Kc;
     int stages = ft::gemm::MAX_STAGES;
-    while (stages > 2 && ft::gemm::make_layout(stages, p.f1, p.f2).total > 227u * 1024u) --stages;
+    while (stages > 1 && ft::gemm::make_layout(stages, p.f1, p.f2).total > 227u * 1024u) --stages;
+    if (ft::gemm::make_layout(stages, p.f1, p.f2).total > 227u * 1024u) return FT_ERR_SHAPE;
     p.stages = stages;
     const uint32_t smem = ft::gemm::make_layout(stages, p.f1, p.f2).total;
     const int tiles = cdiv(M, ft::gemm::BM) * (int)(Nout / ft::gemm::BN);

@@ -78,11 +78,11 @@ struct LrFactor {
 
 struct Params {
     CUtensorMap mapA, mapB, mapP1, mapP2, mapL1, mapL2;
+    CUtensorMap mapY;    // output [M, Nout], box {64 bytes of columns, 128 rows}, 64 B swizzle
     const uint8_t* sfa;  // activation scale slabs [ceil(M/128)][Kc/64][512]
     const uint8_t* sfb;  // weight scale slabs [Nout/128][Kc/64][512]
     const float* ga;
     const float* gb;
-    void* out;
     int out_f32;
     int M, Nout, Kc;
     LrFactor f1, f2;
@@ -90,8 +90,9 @@ struct Params {
 };
 
 struct Layout {
-    uint32_t a, b, sfa, sfb, p1, p2, l1, l2, bars, total;
+    uint32_t a, b, sfa, sfb, p1, p2, l1, l2, stg, bars, total;
 };
+constexpr uint32_t STG_BYTES = 128 * 64;  // one staged output chunk: 128 rows x 64 bytes
 
 // bytes of a factor's P panel (128 rows) and L panel (256 rows)
 __host__ __device__ inline uint32_t p_bytes(const LrFactor& f) {
@@ -112,6 +113,7 @@ __host__ __device__ inline Layout make_layout(int stages, const LrFactor& f1, co
     L.l2 = o;   o += l_bytes(f2);
     L.sfa = o;  o += stages * SFA_STAGE_BYTES;
     L.sfb = o;  o += stages * SFB_STAGE_BYTES;
+    L.stg = o;  o += 2 * STG_BYTES;  // double-buffered output staging
     L.bars = o; o += 256;  // barriers, TMEM slot, abort flag
     L.total = o + 1024;    // slack for 1 KiB alignment of the base
     return L;
@@ -215,6 +217,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                 const uint8_t* sfa = p.sfa + (size_t)tm * KS * 512;
                 const uint8_t* sfb0 = p.sfb + (size_t)(2 * tn) * KS * 512;
                 const uint8_t* sfb1 = sfb0 + (size_t)KS * 512;
+                if (has_lr) {
+                    // low-rank panels first: the first half of the
+                    // up-projection runs before the tile's mainloop
+                    if (!mbar_wait(&bars[B_LR_SMEM_EMPTY], (local & 1) ^ 1, ERR_WAIT_LR, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    uint64_t* lb = &bars[B_LR_FULL];
+                    mbar_arrive_expect_tx(lb, lr_total);
+                    for (int a = 0; a < (p.f1.rf > 0 ? p.f1.natoms : 0); ++a) {
+                        tma_load_2d(smem + L.p1 + a * 128 * p.f1.row_bytes, &p.mapP1, lb, p.f1.pcol + 64 * a, m0);
+                        tma_load_2d(smem + L.l1 + a * 256 * p.f1.row_bytes, &p.mapL1, lb, 64 * a, n0);
+                    }
+                    for (int a = 0; a < (p.f2.rf > 0 ? p.f2.natoms : 0); ++a) {
+                        tma_load_2d(smem + L.p2 + a * 128 * p.f2.row_bytes, &p.mapP2, lb, p.f2.pcol + 64 * a, m0);
+                        tma_load_2d(smem + L.l2 + a * 256 * p.f2.row_bytes, &p.mapL2, lb, 64 * a, n0);
+                    }
+                }
                 for (int kt = 0; kt < KT; ++kt, ++it) {
                     const int s = it % S;
                     const uint32_t ph = (it / S) & 1;
@@ -230,22 +250,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     bulk_load(smem + L.sfa + s * SFA_STAGE_BYTES, sfa + so, SFA_STAGE_BYTES, fb);
                     bulk_load(smem + L.sfb + s * SFB_STAGE_BYTES, sfb0 + so, SFA_STAGE_BYTES, fb);
                     bulk_load(smem + L.sfb + s * SFB_STAGE_BYTES + SFA_STAGE_BYTES, sfb1 + so, SFA_STAGE_BYTES, fb);
-                }
-                if (!ok || !has_lr) continue;
-                // low-rank panels of this tile, after its mainloop loads
-                if (!mbar_wait(&bars[B_LR_SMEM_EMPTY], (local & 1) ^ 1, ERR_WAIT_LR, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                uint64_t* lb = &bars[B_LR_FULL];
-                mbar_arrive_expect_tx(lb, lr_total);
-                for (int a = 0; a < (p.f1.rf > 0 ? p.f1.natoms : 0); ++a) {
-                    tma_load_2d(smem + L.p1 + a * 128 * p.f1.row_bytes, &p.mapP1, lb, p.f1.pcol + 64 * a, m0);
-                    tma_load_2d(smem + L.l1 + a * 256 * p.f1.row_bytes, &p.mapL1, lb, 64 * a, n0);
-                }
-                for (int a = 0; a < (p.f2.rf > 0 ? p.f2.natoms : 0); ++a) {
-                    tma_load_2d(smem + L.p2 + a * 128 * p.f2.row_bytes, &p.mapP2, lb, p.f2.pcol + 64 * a, m0);
-                    tma_load_2d(smem + L.l2 + a * 256 * p.f2.row_bytes, &p.mapL2, lb, 64 * a, n0);
                 }
             }
             if (!ok) {
@@ -271,6 +275,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             bool ok = true;
             int local = 0;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+                if (has_lr) {
+                    // first half of the up-projection, ahead of the mainloop
+                    // (the tensor pipe would otherwise idle waiting for data)
+                    if (!mbar_wait(&bars[B_LR_FULL], local & 1, ERR_WAIT_LR, abort_flag) ||
+                        !mbar_wait(&bars[B_LR_EMPTY], ((2 * local) & 1) ^ 1, ERR_WAIT_LR, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    int q = 0;
+                    if (p.f1.rf > 0) lr_mma(tmem + LR_COL, base + L.p1, base + L.l1, p.f1, 0, idesc_lr, q);
+                    if (p.f2.rf > 0) lr_mma(tmem + LR_COL, base + L.p2, base + L.l2, p.f2, 0, idesc_lr, q);
+                    tc_commit(&bars[B_LR_READY]);
+                }
                 if (!mbar_wait(&bars[B_ACC_EMPTY], (local & 1) ^ 1, ERR_WAIT_ACC_EMPTY, abort_flag)) {
                     ok = false;
                     break;
@@ -299,22 +317,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                 if (!ok) break;
                 tc_commit(&bars[B_ACC_FULL]);
                 if (has_lr) {
-                    if (!mbar_wait(&bars[B_LR_FULL], local & 1, ERR_WAIT_LR, abort_flag)) {
+                    // second half once the epilogue has read the first
+                    if (!mbar_wait(&bars[B_LR_EMPTY], ((2 * local + 1) & 1) ^ 1, ERR_WAIT_LR, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    for (int h = 0; h < 2 && ok; ++h) {
-                        const int u = 2 * local + h;  // use of the low-rank columns
-                        if (!mbar_wait(&bars[B_LR_EMPTY], (u & 1) ^ 1, ERR_WAIT_LR, abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        int q = 0;
-                        if (p.f1.rf > 0) lr_mma(tmem + LR_COL, base + L.p1, base + L.l1, p.f1, h, idesc_lr, q);
-                        if (p.f2.rf > 0) lr_mma(tmem + LR_COL, base + L.p2, base + L.l2, p.f2, h, idesc_lr, q);
-                        tc_commit(&bars[B_LR_READY]);
-                    }
+                    tc_fence_after();
+                    int q = 0;
+                    if (p.f1.rf > 0) lr_mma(tmem + LR_COL, base + L.p1, base + L.l1, p.f1, 1, idesc_lr, q);
+                    if (p.f2.rf > 0) lr_mma(tmem + LR_COL, base + L.p2, base + L.l2, p.f2, 1, idesc_lr, q);
+                    tc_commit(&bars[B_LR_READY]);
                     tc_commit(&bars[B_LR_SMEM_EMPTY]);
                 }
             }
@@ -363,9 +375,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
         __syncwarp();
     } else if (warp >= 4) {
         // ------------------------------------------------ epilogue
+        // Each thread owns one tile row (its TMEM lane).  Output leaves in
+        // chunks of 64 bytes per row (32 bf16 or 16 f32 columns): the rows
+        // are written into a 64-byte-swizzled staging buffer (two buffers,
+        // alternating) and one thread stores the 128-row chunk with TMA, so
+        // global writes are whole lines instead of one 16-byte piece per row.
         const int sp = warp & 3;  // TMEM sub-partition = rows 32*sp .. +31
+        const int et = threadIdx.x - 128;  // tile row
+        const bool leader = et == 0;
+        const int cw = p.out_f32 ? 16 : 32;  // columns per chunk
+        const int nch = 128 / cw;            // chunks per half tile
+        const uint32_t rsw = (uint32_t)((et >> 1) & 3);
         bool ok = true;
         int local = 0;
+        uint32_t nstore = 0;
         const float gab = __fmul_rn(*p.ga, *p.gb);
         for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
             const int m0 = (tile / tiles_n) * BM;
@@ -375,7 +398,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                 break;
             }
             tc_fence_after();
-            const int row = m0 + 32 * sp + lane;
             const uint32_t lane_addr = (uint32_t)(32 * sp) << 16;
             for (int h = 0; h < 2 && ok; ++h) {
                 if (has_lr) {
@@ -386,40 +408,59 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     tc_fence_after();
                 }
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    const int col = 128 * h + 32 * c;  // tile column
-                    uint32_t v[32], lr[32];
-                    tmem_ld_32x32b_x32(tmem + lane_addr + ACC_COL + col, v);
-                    if (has_lr) tmem_ld_32x32b_x32(tmem + lane_addr + LR_COL + 32 * c, lr);
-                    tmem_ld_wait();
+                for (int c = 0; c < nch; ++c) {
+                    const int col = 128 * h + cw * c;  // tile column
                     float y[32];
+                    if (cw == 32) {
+                        uint32_t v[32], lr[32];
+                        tmem_ld_32x32b_x32(tmem + lane_addr + ACC_COL + col, v);
+                        if (has_lr) tmem_ld_32x32b_x32(tmem + lane_addr + LR_COL + cw * c, lr);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int k = 0; k < 32; ++k)
-                        y[k] = __fmaf_rn(gab, __uint_as_float(v[k]), has_lr ? __uint_as_float(lr[k]) : 0.0f);
-                    if (row < p.M) {
-                        if (p.out_f32) {
-                            float* o = reinterpret_cast<float*>(p.out) + (int64_t)row * p.Nout + n0 + col;
+                        for (int k = 0; k < 32; ++k)
+                            y[k] = __fmaf_rn(gab, __uint_as_float(v[k]), has_lr ? __uint_as_float(lr[k]) : 0.0f);
+                    } else {
+                        uint32_t v[16], lr[16];
+                        tmem_ld_32x32b_x16(tmem + lane_addr + ACC_COL + col, v);
+                        if (has_lr) tmem_ld_32x32b_x16(tmem + lane_addr + LR_COL + cw * c, lr);
+                        tmem_ld_wait();
 #pragma unroll
-                            for (int k = 0; k < 32; k += 4)
-                                *reinterpret_cast<float4*>(o + k) = make_float4(y[k], y[k + 1], y[k + 2], y[k + 3]);
-                        } else {
-                            __nv_bfloat16* o =
-                                reinterpret_cast<__nv_bfloat16*>(p.out) + (int64_t)row * p.Nout + n0 + col;
-#pragma unroll
-                            for (int k = 0; k < 32; k += 8) {
-                                uint4 u;
-                                __nv_bfloat162 t0 = __floats2bfloat162_rn(y[k], y[k + 1]);
-                                __nv_bfloat162 t1 = __floats2bfloat162_rn(y[k + 2], y[k + 3]);
-                                __nv_bfloat162 t2 = __floats2bfloat162_rn(y[k + 4], y[k + 5]);
-                                __nv_bfloat162 t3 = __floats2bfloat162_rn(y[k + 6], y[k + 7]);
-                                u.x = *reinterpret_cast<uint32_t*>(&t0);
-                                u.y = *reinterpret_cast<uint32_t*>(&t1);
-                                u.z = *reinterpret_cast<uint32_t*>(&t2);
-                                u.w = *reinterpret_cast<uint32_t*>(&t3);
-                                *reinterpret_cast<uint4*>(o + k) = u;
-                            }
-                        }
+                        for (int k = 0; k < 16; ++k)
+                            y[k] = __fmaf_rn(gab, __uint_as_float(v[k]), has_lr ? __uint_as_float(lr[k]) : 0.0f);
                     }
+                    // the buffer written two chunks ago has been read by its store
+                    if (leader && nstore >= 2) bulk_wait_group_read<1>();
+                    named_bar_sync(1, 128);
+                    const uint32_t buf = base + L.stg + (nstore & 1) * STG_BYTES;
+                    const uint32_t rowa = buf + (uint32_t)et * 64u;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 u;
+                        if (cw == 32) {
+                            __nv_bfloat162 t0 = __floats2bfloat162_rn(y[8 * q], y[8 * q + 1]);
+                            __nv_bfloat162 t1 = __floats2bfloat162_rn(y[8 * q + 2], y[8 * q + 3]);
+                            __nv_bfloat162 t2 = __floats2bfloat162_rn(y[8 * q + 4], y[8 * q + 5]);
+                            __nv_bfloat162 t3 = __floats2bfloat162_rn(y[8 * q + 6], y[8 * q + 7]);
+                            u.x = *reinterpret_cast<uint32_t*>(&t0);
+                            u.y = *reinterpret_cast<uint32_t*>(&t1);
+                            u.z = *reinterpret_cast<uint32_t*>(&t2);
+                            u.w = *reinterpret_cast<uint32_t*>(&t3);
+                        } else {
+                            u = make_uint4(__float_as_uint(y[4 * q]), __float_as_uint(y[4 * q + 1]),
+                                           __float_as_uint(y[4 * q + 2]), __float_as_uint(y[4 * q + 3]));
+                        }
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
+                                         rowa + (((uint32_t)q ^ rsw) << 4)),
+                                     "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w)
+                                     : "memory");
+                    }
+                    fence_proxy_async_smem();
+                    named_bar_sync(1, 128);
+                    if (leader) {
+                        tma_store_2d(&p.mapY, smem + (buf - base), n0 + col, m0);
+                        bulk_commit_group();
+                    }
+                    ++nstore;
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -429,6 +470,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[B_ACC_EMPTY]);
         }
+        // every store has finished before the CTA exits
+        if (leader) bulk_wait_group_all();
     }
 
     tc_fence_before();

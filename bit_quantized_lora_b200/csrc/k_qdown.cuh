@@ -84,7 +84,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qdown(const __grid_constant_
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], NQ_WARPS + (p.do_mma ? 1 : 0));
+            // every quantizer thread releases the stage after its own loads
+            // (behind a proxy fence, see below), plus the MMA commit
+            mbar_init(&empty[i], NQ_WARPS * 32 + (p.do_mma ? 1 : 0));
         }
         mbar_init(accfull, 1);
         mbar_init(drain, 1);
@@ -186,8 +188,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qdown(const __grid_constant_
             uint4 v[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c) v[c] = ld_shared_v4(rowaddr + (((uint32_t)(4 * h + c) ^ sw) << 4));
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
+            // the next TMA copy into this stage is an async-proxy write: the
+            // generic-proxy loads above must be ordered before it explicitly
+            // (without this fence the copy was seen to overtake them)
+            fence_proxy_async_smem();
+            mbar_arrive(&empty[s]);
             uint32_t w0[8] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w};
             uint32_t w1[8] = {v[2].x, v[2].y, v[2].z, v[2].w, v[3].x, v[3].y, v[3].z, v[3].w};
             uint32_t s0, s1;

@@ -148,14 +148,19 @@ def test_empty_batch_is_a_no_op():
     assert not dA.any() and not dB.any()
 
 
-def test_repeated_runs_are_bitwise_identical():
+@pytest.mark.parametrize("wl", [1, 2])
+def test_repeated_runs_are_bitwise_identical(wl):
     """Every reduction (split down-projection, adapter gradients, amax) adds
-    in a fixed order, so repeated forward/backward passes must agree bit for
-    bit; a cross-CTA ordering race would show up here."""
-    inp, U, V, Wr, layer = _prep(ft_synth.ATTN, 21)
+    in a fixed order and every shared-memory stage is released only after
+    all of its readers are done, so repeated forward/backward passes must
+    agree bit for bit; a cross-CTA ordering race or a stage overwritten
+    under a reader would show up here.  The attention shape runs the
+    single-pass resident quantizer; the MLP up-projection's backward
+    (dY [4608, 12288]) runs the streaming two-pass one."""
+    inp, U, V, Wr, layer = _prep(ft_synth.WORKLOADS[wl], 21)
     X, dY = dev_bf16(inp["X"]), dev_bf16(inp["dY"])
     ref = None
-    for _ in range(6):
+    for _ in range(6 if wl == 1 else 4):
         Y, P = ft.ft_linear_fwd(layer, X, out_dtype=ft.F32)
         dX, dA, dB = ft.ft_linear_bwd(layer, dY, X, P, out_dtype=ft.F32)
         torch.cuda.synchronize()
@@ -177,17 +182,22 @@ def _ws_qact(ws, M, N, K, r_s, r_l, C):
     return codes, scales, g
 
 
-@pytest.mark.parametrize("case", ["tiny", "attn", "ragged300", "packed16_112", "rank0", "amax_given"])
+@pytest.mark.parametrize("case", ["tiny", "attn", "ragged300", "packed16_112", "rank0", "amax_given",
+                                  "streaming"])
 def test_fused_quantizer_output_is_bit_exact(case):
     """The operand the 4-bit GEMM consumes, Q(X) after the forward and Q(dY)
     after the backward, read back from the workspace: codes, scales and the
     tensor scale equal the oracle's bit for bit (integer work).  Covers the
     single-pass resident path with its grid-wide amax (attention shape), the
     split reductions, a ragged token count, the packed-factor mode (a rank
-    above 64), no low-rank branch, and a caller-supplied amax."""
+    above 64), no low-rank branch, a caller-supplied amax, and the streaming
+    two-pass path (the MLP up-projection's dY [4608, 12288] is too large to
+    keep resident)."""
     shape, seed, M, r_s, r_l, amax = ft_synth.TINY, 50, None, None, None, None
     if case == "attn":
         shape, seed = ft_synth.ATTN, 51
+    elif case == "streaming":
+        shape, seed = ft_synth.WORKLOADS[2], 52
     elif case == "ragged300":
         M = 300
     elif case == "packed16_112":
