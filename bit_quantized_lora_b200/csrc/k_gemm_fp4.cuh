@@ -29,16 +29,19 @@
 // wide tile doubles the work per instruction).
 //   warp 0  TMA producer: FP4 code tiles (128 B swizzle) and the scale slabs
 //           of each stage (bulk copies), the tile's P / L1 / L2 panels.
-//   warp 1  TMEM owner and UMMA issuer: four
+//   warp 1  TMEM owner and UMMA issuer: half 0 of the low-rank
+//           up-projection (kind::f16, N = 128), then four
 //           tcgen05.mma.kind::mxf4nvf4.block16 (K = 64, N = 256) per stage
-//           into the FP32 accumulator, then the low-rank up-projection
-//           (kind::f16) in two 128-column halves into its own accumulator.
+//           into the FP32 accumulator, then low-rank half 1.
 //   warp 2  scale warp: tcgen05.cp of each stage's slabs into a two-deep
 //           ring of scale columns, ahead of the MMAs (copies issued by
 //           another warp overlap the MMAs instead of queueing behind them).
-//   warps 4-7 epilogue: tcgen05.ld both accumulators, combine, store Y once.
-// TMEM columns: [0,256) accumulator, [256,384) low-rank half,
-// [384,480) scale ring (per slot: A 16 columns, B 32 columns).
+//   warps 4-11 epilogue, two groups working on the two column halves at
+//           once: tcgen05.ld accumulator and low-rank half, combine, store
+//           Y once.
+// TMEM columns: [0,256) accumulator, [256,384) low-rank half 0, [384,512)
+// the scale ring (per slot: A 16 columns, B 32 columns) during the mainloop
+// and low-rank half 1 after it.
 //
 // Low-rank panels are K-major with the rank as K, each factor's part of P
 // and the factor itself swizzled to its own width (16, 32 or 64 columns per
@@ -57,13 +60,17 @@ constexpr int BN = 256;
 constexpr int BK_BYTES = 128;  // 256 FP4 elements of K per stage
 constexpr int KSTEPS = 4;      // MMAs of K = 64 per stage
 constexpr int MAX_STAGES = 4;
-constexpr int NUM_THREADS = 256;
+constexpr int NUM_EPI_WARPS = 8;  // two column groups of four lane-quarter warps
+constexpr int NUM_THREADS = 128 + 32 * NUM_EPI_WARPS;
 constexpr int A_BYTES = BM * BK_BYTES;         // 16 KiB
 constexpr int B_BYTES = BN * BK_BYTES;         // 32 KiB
 constexpr int SFA_STAGE_BYTES = KSTEPS * 512;  // four slabs (128 rows)
 constexpr int SFB_STAGE_BYTES = 2 * KSTEPS * 512;  // two row halves x four slabs
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t ACC_COL = 0, LR_COL = 256, SF_COL = 384, SF_SLOT_COLS = 48;
+// TMEM columns: [0,256) accumulator; [256,384) low-rank half 0; [384,512)
+// shared in time: the scale ring while the mainloop runs, low-rank half 1
+// after it (the next tile's first scale copy waits for the epilogue).
+constexpr uint32_t ACC_COL = 0, LR0_COL = 256, R2_COL = 384, SF_SLOT_COLS = 48;
 
 // One low-rank factor's panels: P columns [pcol, pcol + rf) for the tile's
 // 128 rows (A operand) and L [256 output rows, rf] (B operand), both K-major.
@@ -113,7 +120,7 @@ __host__ __device__ inline Layout make_layout(int stages, const LrFactor& f1, co
     L.l2 = o;   o += l_bytes(f2);
     L.sfa = o;  o += stages * SFA_STAGE_BYTES;
     L.sfb = o;  o += stages * SFB_STAGE_BYTES;
-    L.stg = o;  o += 2 * STG_BYTES;  // double-buffered output staging
+    L.stg = o;  o += 2 * STG_BYTES;  // output staging, one buffer per column group
     L.bars = o; o += 256;  // barriers, TMEM slot, abort flag
     L.total = o + 1024;    // slack for 1 KiB alignment of the base
     return L;
@@ -126,11 +133,11 @@ enum {
     B_SF_READY = B_EMPTY + MAX_STAGES, // [2] scale slot copied into TMEM
     B_SF_FREE = B_SF_READY + 2,        // [2] scale slot read by its MMAs
     B_ACC_FULL = B_SF_FREE + 2,
-    B_ACC_EMPTY,                       // 4 epilogue warps
+    B_ACC_EMPTY,                       // every epilogue warp done with the tile
     B_LR_FULL,                         // panels landed
     B_LR_SMEM_EMPTY,                   // panels consumed
-    B_LR_READY,                        // low-rank half computed
-    B_LR_EMPTY,                        // low-rank half read (4 epilogue warps)
+    B_LR0_READY,                       // low-rank half 0 computed
+    B_LR1_READY,                       // low-rank half 1 computed
     B_DRAIN,
     B_DRAIN_SF,
     B_COUNT
@@ -180,11 +187,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             mbar_init(&bars[B_SF_FREE + i], 1);
         }
         mbar_init(&bars[B_ACC_FULL], 1);
-        mbar_init(&bars[B_ACC_EMPTY], 4);
+        mbar_init(&bars[B_ACC_EMPTY], NUM_EPI_WARPS);
         mbar_init(&bars[B_LR_FULL], 1);
         mbar_init(&bars[B_LR_SMEM_EMPTY], 1);
-        mbar_init(&bars[B_LR_READY], 1);
-        mbar_init(&bars[B_LR_EMPTY], 4);
+        mbar_init(&bars[B_LR0_READY], 1);
+        mbar_init(&bars[B_LR1_READY], 1);
         mbar_init(&bars[B_DRAIN], 1);
         mbar_init(&bars[B_DRAIN_SF], 1);
         *abort_flag = 0;
@@ -275,23 +282,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             bool ok = true;
             int local = 0;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
-                if (has_lr) {
-                    // first half of the up-projection, ahead of the mainloop
-                    // (the tensor pipe would otherwise idle waiting for data)
-                    if (!mbar_wait(&bars[B_LR_FULL], local & 1, ERR_WAIT_LR, abort_flag) ||
-                        !mbar_wait(&bars[B_LR_EMPTY], ((2 * local) & 1) ^ 1, ERR_WAIT_LR, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    int q = 0;
-                    if (p.f1.rf > 0) lr_mma(tmem + LR_COL, base + L.p1, base + L.l1, p.f1, 0, idesc_lr, q);
-                    if (p.f2.rf > 0) lr_mma(tmem + LR_COL, base + L.p2, base + L.l2, p.f2, 0, idesc_lr, q);
-                    tc_commit(&bars[B_LR_READY]);
-                }
-                if (!mbar_wait(&bars[B_ACC_EMPTY], (local & 1) ^ 1, ERR_WAIT_ACC_EMPTY, abort_flag)) {
+                if ((has_lr && !mbar_wait(&bars[B_LR_FULL], local & 1, ERR_WAIT_LR, abort_flag)) ||
+                    !mbar_wait(&bars[B_ACC_EMPTY], (local & 1) ^ 1, ERR_WAIT_ACC_EMPTY, abort_flag)) {
                     ok = false;
                     break;
+                }
+                tc_fence_after();
+                if (has_lr) {
+                    // half 0 of the up-projection ahead of the mainloop (the
+                    // tensor pipe would otherwise idle waiting for data)
+                    int q = 0;
+                    if (p.f1.rf > 0) lr_mma(tmem + LR0_COL, base + L.p1, base + L.l1, p.f1, 0, idesc_lr, q);
+                    if (p.f2.rf > 0) lr_mma(tmem + LR0_COL, base + L.p2, base + L.l2, p.f2, 0, idesc_lr, q);
+                    tc_commit(&bars[B_LR0_READY]);
                 }
                 tc_fence_after();
                 for (int kt = 0; kt < KT; ++kt, ++it) {
@@ -305,7 +308,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     tc_fence_after();
                     const uint32_t a_lo = a_lo0 + s * (A_BYTES >> 4);
                     const uint32_t b_lo = b_lo0 + s * (B_BYTES >> 4);
-                    const uint32_t sf = tmem + SF_COL + sb * SF_SLOT_COLS;
+                    const uint32_t sf = tmem + R2_COL + sb * SF_SLOT_COLS;
 #pragma unroll
                     for (int j = 0; j < KSTEPS; ++j)
                         umma_nvfp4(tmem + ACC_COL, make_desc(a_lo + 2 * j, hi_sw128),
@@ -317,16 +320,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                 if (!ok) break;
                 tc_commit(&bars[B_ACC_FULL]);
                 if (has_lr) {
-                    // second half once the epilogue has read the first
-                    if (!mbar_wait(&bars[B_LR_EMPTY], ((2 * local + 1) & 1) ^ 1, ERR_WAIT_LR, abort_flag)) {
+                    // half 1 into the scale ring's columns once the mainloop's
+                    // MMAs (the last readers of the scales) have completed
+                    if (!mbar_wait(&bars[B_ACC_FULL], local & 1, ERR_WAIT_ACC_FULL, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     int q = 0;
-                    if (p.f1.rf > 0) lr_mma(tmem + LR_COL, base + L.p1, base + L.l1, p.f1, 1, idesc_lr, q);
-                    if (p.f2.rf > 0) lr_mma(tmem + LR_COL, base + L.p2, base + L.l2, p.f2, 1, idesc_lr, q);
-                    tc_commit(&bars[B_LR_READY]);
+                    if (p.f1.rf > 0) lr_mma(tmem + R2_COL, base + L.p1, base + L.l1, p.f1, 1, idesc_lr, q);
+                    if (p.f2.rf > 0) lr_mma(tmem + R2_COL, base + L.p2, base + L.l2, p.f2, 1, idesc_lr, q);
+                    tc_commit(&bars[B_LR1_READY]);
                     tc_commit(&bars[B_LR_SMEM_EMPTY]);
                 }
             }
@@ -344,7 +348,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             const uint32_t sfb_lo0 = (base + L.sfb) >> 4;
             uint32_t it = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            int local = 0;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+                // the ring's columns hold the previous tile's low-rank half 1
+                // until its epilogue is done
+                if (has_lr && local > 0 &&
+                    !mbar_wait(&bars[B_ACC_EMPTY], (local - 1) & 1, ERR_WAIT_SF, abort_flag)) {
+                    ok = false;
+                    break;
+                }
                 for (int kt = 0; kt < KT; ++kt, ++it) {
                     const int s = it % S;
                     const int sb = it & 1;
@@ -356,7 +368,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     tc_fence_after();
                     const uint32_t sfa_lo = sfa_lo0 + s * (SFA_STAGE_BYTES >> 4);
                     const uint32_t sfb_lo = sfb_lo0 + s * (SFB_STAGE_BYTES >> 4);
-                    const uint32_t sf = tmem + SF_COL + sb * SF_SLOT_COLS;
+                    const uint32_t sf = tmem + R2_COL + sb * SF_SLOT_COLS;
 #pragma unroll
                     for (int j = 0; j < KSTEPS; ++j) {
                         // A: rows 0-127; B: rows 0-127 then 128-255 (four columns each)
@@ -375,98 +387,95 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
         __syncwarp();
     } else if (warp >= 4) {
         // ------------------------------------------------ epilogue
-        // Each thread owns one tile row (its TMEM lane).  Output leaves in
-        // chunks of 64 bytes per row (32 bf16 or 16 f32 columns): the rows
-        // are written into a 64-byte-swizzled staging buffer (two buffers,
-        // alternating) and one thread stores the 128-row chunk with TMA, so
-        // global writes are whole lines instead of one 16-byte piece per row.
+        // Each thread owns one tile row (its TMEM lane) within one of two
+        // column groups working concurrently: warps 4-7 take columns 0-127
+        // (with low-rank half 0), warps 8-11 columns 128-255 (half 1).
+        // Output leaves in chunks of 64 bytes per row (32 bf16 or 16 f32
+        // columns): the group's rows are written into its 64-byte-swizzled
+        // staging buffer and one thread of the group stores the 128-row chunk
+        // with TMA, so global writes are whole lines instead of one 16-byte
+        // piece per row.
         const int sp = warp & 3;  // TMEM sub-partition = rows 32*sp .. +31
-        const int et = threadIdx.x - 128;  // tile row
+        const int grp = (warp - 4) >> 2;
+        const int et = (threadIdx.x - 128) & 127;  // tile row
         const bool leader = et == 0;
         const int cw = p.out_f32 ? 16 : 32;  // columns per chunk
-        const int nch = 128 / cw;            // chunks per half tile
+        const int nch = 128 / cw;            // chunks per group per tile
         const uint32_t rsw = (uint32_t)((et >> 1) & 3);
+        const uint32_t buf = base + L.stg + (uint32_t)grp * STG_BYTES;
+        const uint32_t lr_col = grp == 0 ? LR0_COL : R2_COL;
+        uint64_t* lr_ready = &bars[grp == 0 ? B_LR0_READY : B_LR1_READY];
         bool ok = true;
         int local = 0;
-        uint32_t nstore = 0;
+        bool pending = false;  // this group's buffer is being read by a store
         const float gab = __fmul_rn(*p.ga, *p.gb);
         for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
             const int m0 = (tile / tiles_n) * BM;
             const int n0 = (tile % tiles_n) * BN;
-            if (!mbar_wait(&bars[B_ACC_FULL], local & 1, ERR_WAIT_ACC_FULL, abort_flag)) {
+            if (!mbar_wait(&bars[B_ACC_FULL], local & 1, ERR_WAIT_ACC_FULL, abort_flag) ||
+                (has_lr && !mbar_wait(lr_ready, local & 1, ERR_WAIT_LR, abort_flag))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             const uint32_t lane_addr = (uint32_t)(32 * sp) << 16;
-            for (int h = 0; h < 2 && ok; ++h) {
-                if (has_lr) {
-                    if (!mbar_wait(&bars[B_LR_READY], (2 * local + h) & 1, ERR_WAIT_LR, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                }
 #pragma unroll 1
-                for (int c = 0; c < nch; ++c) {
-                    const int col = 128 * h + cw * c;  // tile column
-                    float y[32];
-                    if (cw == 32) {
-                        uint32_t v[32], lr[32];
-                        tmem_ld_32x32b_x32(tmem + lane_addr + ACC_COL + col, v);
-                        if (has_lr) tmem_ld_32x32b_x32(tmem + lane_addr + LR_COL + cw * c, lr);
-                        tmem_ld_wait();
+            for (int c = 0; c < nch; ++c) {
+                const int lcol = cw * c;              // column within the group's half
+                const int col = 128 * grp + lcol;     // tile column
+                float y[32];
+                if (cw == 32) {
+                    uint32_t v[32], lr[32];
+                    tmem_ld_32x32b_x32(tmem + lane_addr + ACC_COL + col, v);
+                    if (has_lr) tmem_ld_32x32b_x32(tmem + lane_addr + lr_col + lcol, lr);
+                    tmem_ld_wait();
 #pragma unroll
-                        for (int k = 0; k < 32; ++k)
-                            y[k] = __fmaf_rn(gab, __uint_as_float(v[k]), has_lr ? __uint_as_float(lr[k]) : 0.0f);
-                    } else {
-                        uint32_t v[16], lr[16];
-                        tmem_ld_32x32b_x16(tmem + lane_addr + ACC_COL + col, v);
-                        if (has_lr) tmem_ld_32x32b_x16(tmem + lane_addr + LR_COL + cw * c, lr);
-                        tmem_ld_wait();
+                    for (int k = 0; k < 32; ++k)
+                        y[k] = __fmaf_rn(gab, __uint_as_float(v[k]), has_lr ? __uint_as_float(lr[k]) : 0.0f);
+                } else {
+                    uint32_t v[16], lr[16];
+                    tmem_ld_32x32b_x16(tmem + lane_addr + ACC_COL + col, v);
+                    if (has_lr) tmem_ld_32x32b_x16(tmem + lane_addr + lr_col + lcol, lr);
+                    tmem_ld_wait();
 #pragma unroll
-                        for (int k = 0; k < 16; ++k)
-                            y[k] = __fmaf_rn(gab, __uint_as_float(v[k]), has_lr ? __uint_as_float(lr[k]) : 0.0f);
-                    }
-                    // the buffer written two chunks ago has been read by its store
-                    if (leader && nstore >= 2) bulk_wait_group_read<1>();
-                    named_bar_sync(1, 128);
-                    const uint32_t buf = base + L.stg + (nstore & 1) * STG_BYTES;
-                    const uint32_t rowa = buf + (uint32_t)et * 64u;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint4 u;
-                        if (cw == 32) {
-                            __nv_bfloat162 t0 = __floats2bfloat162_rn(y[8 * q], y[8 * q + 1]);
-                            __nv_bfloat162 t1 = __floats2bfloat162_rn(y[8 * q + 2], y[8 * q + 3]);
-                            __nv_bfloat162 t2 = __floats2bfloat162_rn(y[8 * q + 4], y[8 * q + 5]);
-                            __nv_bfloat162 t3 = __floats2bfloat162_rn(y[8 * q + 6], y[8 * q + 7]);
-                            u.x = *reinterpret_cast<uint32_t*>(&t0);
-                            u.y = *reinterpret_cast<uint32_t*>(&t1);
-                            u.z = *reinterpret_cast<uint32_t*>(&t2);
-                            u.w = *reinterpret_cast<uint32_t*>(&t3);
-                        } else {
-                            u = make_uint4(__float_as_uint(y[4 * q]), __float_as_uint(y[4 * q + 1]),
-                                           __float_as_uint(y[4 * q + 2]), __float_as_uint(y[4 * q + 3]));
-                        }
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
-                                         rowa + (((uint32_t)q ^ rsw) << 4)),
-                                     "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w)
-                                     : "memory");
-                    }
-                    fence_proxy_async_smem();
-                    named_bar_sync(1, 128);
-                    if (leader) {
-                        tma_store_2d(&p.mapY, smem + (buf - base), n0 + col, m0);
-                        bulk_commit_group();
-                    }
-                    ++nstore;
+                    for (int k = 0; k < 16; ++k)
+                        y[k] = __fmaf_rn(gab, __uint_as_float(v[k]), has_lr ? __uint_as_float(lr[k]) : 0.0f);
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0 && has_lr) mbar_arrive(&bars[B_LR_EMPTY]);
+                // the group's previous chunk has been read out of the buffer
+                if (leader && pending) bulk_wait_group_read<0>();
+                named_bar_sync(1 + grp, 128);
+                const uint32_t rowa = buf + (uint32_t)et * 64u;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint4 u;
+                    if (cw == 32) {
+                        __nv_bfloat162 t0 = __floats2bfloat162_rn(y[8 * q], y[8 * q + 1]);
+                        __nv_bfloat162 t1 = __floats2bfloat162_rn(y[8 * q + 2], y[8 * q + 3]);
+                        __nv_bfloat162 t2 = __floats2bfloat162_rn(y[8 * q + 4], y[8 * q + 5]);
+                        __nv_bfloat162 t3 = __floats2bfloat162_rn(y[8 * q + 6], y[8 * q + 7]);
+                        u.x = *reinterpret_cast<uint32_t*>(&t0);
+                        u.y = *reinterpret_cast<uint32_t*>(&t1);
+                        u.z = *reinterpret_cast<uint32_t*>(&t2);
+                        u.w = *reinterpret_cast<uint32_t*>(&t3);
+                    } else {
+                        u = make_uint4(__float_as_uint(y[4 * q]), __float_as_uint(y[4 * q + 1]),
+                                       __float_as_uint(y[4 * q + 2]), __float_as_uint(y[4 * q + 3]));
+                    }
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(rowa + (((uint32_t)q ^ rsw) << 4)),
+                                 "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w)
+                                 : "memory");
+                }
+                fence_proxy_async_smem();
+                named_bar_sync(1 + grp, 128);
+                if (leader) {
+                    tma_store_2d(&p.mapY, smem + (buf - base), n0 + col, m0);
+                    bulk_commit_group();
+                }
+                pending = true;
             }
-            if (!ok) break;
+            // every TMEM read of this tile is done: the MMA warp may overwrite
+            // the accumulator and both low-rank halves
+            tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[B_ACC_EMPTY]);
         }
