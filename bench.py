@@ -244,9 +244,13 @@ class ClockSampler:
 
 
 def kernel_source_sha(name: str) -> str:
-    path = os.path.join(ROOT, "bit_quantized_lora_b200", "csrc", name)
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of a kernel's source file and the device headers every kernel
+    includes, so a recorded ncu figure lapses when any of them changes."""
+    h = hashlib.sha256()
+    for part in (name, "ft_ptx.cuh", "ft_nvfp4.cuh"):
+        with open(os.path.join(ROOT, "bit_quantized_lora_b200", "csrc", part), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def ncu_traffic(kernel: str, source: str):
