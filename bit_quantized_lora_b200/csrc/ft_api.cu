@@ -73,6 +73,21 @@ ft_status device_info(DevInfo** out) {
             cudaFuncSetAttribute(ft::qres::k_qres, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  big) != cudaSuccess)
             return FT_ERR_CUDA;
+        // one shared-memory carveout (the largest) for every kernel of a
+        // step, so that no SM has to re-partition L1 between two of them
+        const void* kernels[] = {
+            reinterpret_cast<const void*>(ft::gemm::k_gemm_fp4),
+            reinterpret_cast<const void*>(ft::qres::k_qres),
+            reinterpret_cast<const void*>(ft::qdown::k_qdown),
+            reinterpret_cast<const void*>(ft::lgrad::k_lora_grad),
+            reinterpret_cast<const void*>(ft::k_amax_bf16),
+            reinterpret_cast<const void*>(ft::k_quant_1x16),
+            reinterpret_cast<const void*>(ft::k_pack_lt),
+        };
+        for (const void* k : kernels)
+            if (cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+                return FT_ERR_CUDA;
         // the resident quantizer's grid barrier needs every CTA resident at
         // once; size its grids by the occupancy at its largest footprint
         int per_sm = 0;
@@ -181,6 +196,7 @@ ft_status encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, ui
 // ------------------------------------------------------------ workspace
 constexpr int QD_MAX_SPLITS = 8;
 constexpr int LG_MAX_SPLITS = 16;
+static_assert(QD_MAX_SPLITS <= ft::qres::MAX_SPLITS, "k_qres reduces at most MAX_SPLITS partials");
 
 struct WsPlan {
     size_t amax, gact, codes, scales, sfslab, lt, part, pg, lgpart, counters, total;
@@ -362,11 +378,12 @@ void qres_ring(ft::qres::Params& p) {
     p.f1.off = 0;
     p.f2.off = qres_factor_bytes(p.f1);
     p.fstage_bytes = qres_factor_bytes(p.f1) + qres_factor_bytes(p.f2);
+    // 24 KB of ring leaves room for twelve resident 16 KB stages (a
+    // [128, 768] chunk) next to the scale staging, the table and the barriers
     p.fs = 2;
     if (p.fstage_bytes > 0)
-        p.fs = (int)std::max<uint32_t>(2u, std::min<uint32_t>((uint32_t)Q::MAX_FS, 31744u / p.fstage_bytes));
-    p.ring_bytes = std::max<uint32_t>((uint32_t)p.fs * p.fstage_bytes, Q::BM * Q::SROW);
-    p.ring_bytes = (p.ring_bytes + 1023u) & ~1023u;
+        p.fs = (int)std::max<uint32_t>(2u, std::min<uint32_t>((uint32_t)Q::MAX_FS, 24576u / p.fstage_bytes));
+    p.ring_bytes = ((uint32_t)p.fs * p.fstage_bytes + 1023u) & ~1023u;
 }
 
 // Grid of the resident quantizer for T [M, C]: 128-row tiles x C-splits of

@@ -302,16 +302,21 @@ __device__ __forceinline__ uint2 quant_block16_fast(const uint32_t (&w)[8], cons
 // {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5} * d.  Both encodings are monotone
 // step functions of |x|, so they agree on every bf16 value when they agree on
 // the few bf16 values around each boundary; QTableM checks exactly those
-// once per scale byte and keeps y in ym[] only for the divisors that pass.
+// once per scale byte.  When RN(1/d) fails, its two FP32 neighbours are
+// tried: they move the product by one more ulp at most, far less than the
+// spacing of bf16 values, so the same few candidates still decide.  ym[]
+// keeps the first multiplier that passes (0: none does, IEEE division).
 // The multiply also carries the sign (a -0 input gives -0 and code 0x8), so
 // an element costs half a packed multiply and half a conversion.
 // Bit-identical to quant_block16 (same IEEE definition).
 
+constexpr int QT_NY = 3;  // multipliers tried: RN(1/d), then one ulp below and above
+
 struct QTableM {
     float d[128];
-    float y[128];     // 0: divisor outside [2^-60, 2^60] (IEEE division)
-    float ym[128];    // y where the multiply path is exact for every bf16 x, else 0
-    uint32_t bad[4];  // scratch of the check: one bit per scale byte
+    float y[128];           // 0: divisor outside [2^-60, 2^60] (IEEE division)
+    float ym[128];          // the multiplier that is exact for every bf16 x, else 0
+    uint32_t bad[QT_NY][4]; // scratch of the check: one bit per (multiplier, scale byte)
 };
 
 __device__ __forceinline__ uint32_t e2m1_encode1(float q) {
@@ -322,6 +327,12 @@ __device__ __forceinline__ uint32_t e2m1_encode1(float q) {
         : "=h"(out)
         : "f"(0.0f), "f"(q));
     return out & 0xFu;
+}
+
+// Candidate multiplier j of a positive normal y: y, y - 1 ulp, y + 1 ulp.
+__device__ __forceinline__ float qt_multiplier(float y, int j) {
+    const uint32_t u = __float_as_uint(y);
+    return __uint_as_float(j == 0 ? u : (j == 1 ? u - 1u : u + 1u));
 }
 
 // Step 1 of 3 (a barrier between steps): divisors and reciprocals.
@@ -335,19 +346,19 @@ __device__ __forceinline__ void build_qtable_m1(QTableM& tab, float g, int tid, 
         tab.d[s] = d;
         tab.y[s] = y;
     }
-    if (tid < 4) tab.bad[tid] = 0u;
+    if (tid < QT_NY * 4) (&tab.bad[0][0])[tid] = 0u;
 }
 
-// Step 2: the exactness check of the multiply path, four threads per scale
-// byte (boundaries k = part, part + 4).
+// Step 2: the exactness check of the multiply path, for each candidate
+// multiplier, four threads per scale byte (boundaries k = part, part + 4).
 __device__ __forceinline__ void build_qtable_m2(QTableM& tab, int tid, int nthreads) {
-    for (int i = tid; i < 512; i += nthreads) {
-        const int s = i & 127, part = i >> 7;
+    for (int i = tid; i < QT_NY * 512; i += nthreads) {
+        const int j = i >> 9, s = i & 127, part = (i >> 7) & 3;
         const float d = tab.d[s], y = tab.y[s];
         if (s == 0 || s >= 0x7E || y == 0.0f) continue;  // these never take the multiply path
+        const float yj = qt_multiplier(y, j);
         bool ok = true;
         for (int k = part; k < 7; k += 4) {
-            // x0: the largest bf16 value <= b_k d (b_k d is exact in double)
             // rounding boundary k of the E2M1 grid: 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5
             const float bk = k < 4 ? 0.25f + 0.5f * (float)k : (k == 4 ? 2.5f : (k == 5 ? 3.5f : 5.0f));
             // x0: the largest bf16 value <= bk d (RZ keeps the product at or
@@ -358,18 +369,22 @@ __device__ __forceinline__ void build_qtable_m2(QTableM& tab, int tid, int nthre
                 if (c < 0 && x0 < 0x10000u) continue;
                 const float x = __uint_as_float(x0 + (uint32_t)(c * 0x10000));
                 // div_by_recip is the correctly rounded quotient for these d
-                if (e2m1_encode1(div_by_recip(x, d, y)) != e2m1_encode1(__fmul_rn(x, y))) ok = false;
+                if (e2m1_encode1(div_by_recip(x, d, y)) != e2m1_encode1(__fmul_rn(x, yj))) ok = false;
             }
         }
-        if (!ok) atomicOr(&tab.bad[s >> 5], 1u << (s & 31));
+        if (!ok) atomicOr(&tab.bad[j][s >> 5], 1u << (s & 31));
     }
 }
 
-// Step 3: publish ym.
+// Step 3: publish ym, the first multiplier that passed.
 __device__ __forceinline__ void build_qtable_m3(QTableM& tab, int tid, int nthreads) {
     for (int s = tid; s < 128; s += nthreads) {
-        const bool bad = (tab.bad[s >> 5] >> (s & 31)) & 1u;
-        tab.ym[s] = (bad || s == 0 || s >= 0x7E) ? 0.0f : tab.y[s];
+        float ym = 0.0f;
+        if (s != 0 && s < 0x7E && tab.y[s] != 0.0f) {
+            for (int j = QT_NY - 1; j >= 0; --j)
+                if (!((tab.bad[j][s >> 5] >> (s & 31)) & 1u)) ym = qt_multiplier(tab.y[s], j);
+        }
+        tab.ym[s] = ym;
     }
 }
 

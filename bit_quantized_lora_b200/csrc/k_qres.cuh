@@ -46,12 +46,15 @@ constexpr int BM = 128;
 constexpr int BKC = 64;          // columns per stage (128 bytes of bf16)
 constexpr int MAX_ST = 12;       // resident stages per CTA (768 columns)
 constexpr int MAX_FS = 8;        // factor-ring stages
+constexpr int MAX_SPLITS = 8;    // C-splits of one row tile
 constexpr int NQ_WARPS = 16;
 constexpr int NQ_THREADS = NQ_WARPS * 32;
 constexpr int NUM_THREADS = 64 + NQ_THREADS;
 constexpr int TILE_BYTES = BM * BKC * 2;  // 16 KiB
 constexpr uint32_t TMEM_COLS = 128;
-constexpr uint32_t SROW = MAX_ST * 4;  // staged scale bytes per row
+// staged scale bytes per row: MAX_ST words plus one, so that the byte
+// stores of 32 consecutive rows fall in 32 different banks
+constexpr uint32_t SROW = MAX_ST * 4 + 4;
 constexpr uint32_t BAR_BYTES = 512;
 constexpr uint32_t SMEM_LIMIT = 227u * 1024u;
 
@@ -92,14 +95,15 @@ struct Params {
 };
 
 struct Layout {
-    uint32_t x, f, tab, bars, total;
+    uint32_t x, f, sst, tab, bars, total;
 };
 
 __host__ __device__ inline Layout make_layout(int nst, uint32_t ring_bytes) {
     Layout L;
     uint32_t o = 0;
     L.x = o;    o += (uint32_t)nst * TILE_BYTES;
-    L.f = o;    o += ring_bytes;  // factor ring, then the staged scales
+    L.f = o;    o += ring_bytes;  // factor ring
+    L.sst = o;  o += BM * SROW;   // staged scale bytes
     L.tab = o;  o += (uint32_t)sizeof(QTableM);
     L.bars = o; o += BAR_BYTES;
     L.total = o + 1024;  // slack for the 1 KiB alignment of the base
@@ -111,12 +115,12 @@ enum {
     QB_XFULL = 0,                   // [MAX_ST] chunk stage landed (used once)
     QB_FFULL = QB_XFULL + MAX_ST,   // [MAX_FS] factor tiles landed
     QB_FEMPTY = QB_FFULL + MAX_FS,  // [MAX_FS] factor tiles consumed by the MMAs
-    QB_ACC = QB_FEMPTY + MAX_FS,    // accumulator complete
+    QB_XDONE = QB_FEMPTY + MAX_FS,  // [MAX_ST] the MMAs are done with a chunk stage
+    QB_ACC = QB_XDONE + MAX_ST,     // accumulator complete
     QB_DRAIN,                       // every tcgen05 op of the MMA warp done
     QB_COUNT
 };
 static_assert(QB_COUNT * 8 + 16 + 4 * NQ_WARPS <= BAR_BYTES, "barrier area");
-static_assert(BM * SROW <= 6 * 1024, "scale staging");
 
 // Waits for a phase that must complete (copies already issued) before the
 // CTA may exit; bounded like every other wait.
@@ -166,7 +170,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
     const int FS = p.fs;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < MAX_ST; ++i) mbar_init(&bars[QB_XFULL + i], 1);
+        for (int i = 0; i < MAX_ST; ++i) {
+            mbar_init(&bars[QB_XFULL + i], 1);
+            mbar_init(&bars[QB_XDONE + i], 1);
+        }
         for (int i = 0; i < MAX_FS; ++i) {
             mbar_init(&bars[QB_FFULL + i], 1);
             mbar_init(&bars[QB_FEMPTY + i], 1);
@@ -244,6 +251,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
                 if (p.f1.rf > 0) mma_factor(tmem, a, b, p.f1, st == 0);
                 if (p.f2.rf > 0) mma_factor(tmem + (uint32_t)p.r1, a, b, p.f2, st == 0);
                 tc_commit(&bars[QB_FEMPTY + f]);
+                tc_commit(&bars[QB_XDONE + st]);
             }
             if (ok) tc_commit(&bars[QB_ACC]);
             tc_commit(&bars[QB_DRAIN]);
@@ -315,50 +323,66 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
         build_qtable_m2(tab, t, NQ_THREADS);
         named_bar_sync(1, NQ_THREADS);
         build_qtable_m3(tab, t, NQ_THREADS);
-        // the MMAs have normally finished with the tiles by now (they ran
-        // during phase 1 and the barrier); after this wait phase 2 may
-        // overwrite the chunk and the factor ring
-        if (p.do_mma && ok && !mbar_wait(&bars[QB_ACC], 0, ERR_WAIT_ACC_FULL, abort_flag)) ok = false;
         named_bar_sync(1, NQ_THREADS);
         ok = ok && !*abort_flag;
 
-        // phase 2: encode every block from shared memory.  A block's 8 code
-        // bytes go back into the first half of its own (already read) 16-byte
-        // slot, its scale byte into a [128, 48] staging array over the factor
-        // ring; the output pass then writes both with coalesced stores.
-        const uint32_t sstage = base + L.f;
+        // phase 2: encode every block from shared memory, the loads one
+        // stage ahead.  A block's 8 code bytes go back into the first half of
+        // its own 16-byte slot once the MMAs are done with that stage (they
+        // run during phase 1 and mostly finish during the barrier), its scale
+        // byte into the [128, SROW] staging array; the output pass then
+        // writes both with coalesced stores.
+        const uint32_t sstage = base + L.sst;
         if (ok) {
+            uint4 n0 = ld_shared_v4(base + L.x + off_lo), n1 = ld_shared_v4(base + L.x + off_hi);
 #pragma unroll
             for (int st = 0; st < MAX_ST; ++st) {
-                if (st < nst) {
+                if (st < nst && ok) {
                     const uint32_t ta = base + L.x + st * TILE_BYTES;
-                    const uint4 v0 = ld_shared_v4(ta + off_lo), v1 = ld_shared_v4(ta + off_hi);
-                    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                    const uint32_t w[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
+                    if (st + 1 < nst) {
+                        n0 = ld_shared_v4(ta + TILE_BYTES + off_lo);
+                        n1 = ld_shared_v4(ta + TILE_BYTES + off_hi);
+                    }
                     uint32_t sbyte;
                     const uint2 q = quant_block16_m(w, mb[st], qt, tab, sbyte);
-                    st_shared_v2(ta + off_lo, q);
-                    st_shared_u8(sstage + (uint32_t)trow * SROW + st * 4 + blk, sbyte);
+                    if (p.do_mma && !mbar_wait(&bars[QB_XDONE + st], 0, ERR_WAIT_ACC_FULL, abort_flag)) {
+                        ok = false;
+                    } else {
+                        st_shared_v2(ta + off_lo, q);
+                        st_shared_u8(sstage + (uint32_t)trow * SROW + st * 4 + blk, sbyte);
+                    }
                 }
             }
         }
         named_bar_sync(1, NQ_THREADS);
-        if (ok) {
+        ok = ok && !*abort_flag;
+
+        // With the down-projections, warps 2-5 (one per TMEM lane quarter)
+        // take the epilogue while the other twelve write the outputs.
+        const bool epi_warp = p.do_mma && warp < 6;
+        if (ok && !epi_warp) {
+            const int ot = p.do_mma ? t - 128 : t;
+            const int on = p.do_mma ? NQ_THREADS - 128 : NQ_THREADS;
             const int rows = min(BM, p.M - m0);
-            // codes: 16-byte segments (two blocks), consecutive threads on
-            // consecutive segments of a row
-            const int segs = nst * 2;
-            for (int i = t; i < rows * segs; i += NQ_THREADS) {
-                const int r = i / segs, j = i - r * segs;
-                const int st = j >> 1, b0 = 2 * (j & 1);
-                const uint32_t rs = (uint32_t)(r & 7);
-                const uint32_t ra = base + L.x + st * TILE_BYTES + (uint32_t)r * 128u;
-                const uint2 lo = ld_shared_v2(ra + (((uint32_t)(2 * b0) ^ rs) << 4));
-                const uint2 hi = ld_shared_v2(ra + (((uint32_t)(2 * b0 + 2) ^ rs) << 4));
-                *reinterpret_cast<uint4*>(p.codes + (int64_t)(m0 + r) * (p.C / 2) + c0 / 2 + 16 * j) =
-                    make_uint4(lo.x, lo.y, hi.x, hi.y);
+            // codes: 8-byte pieces (one block), a warp on 8 rows x the 4
+            // blocks of one stage: the pieces sit at the start of 16-byte
+            // slots whose swizzle differs from row to row, so the warp's
+            // shared loads spread over all banks (2 ways), and every row
+            // gets one full 32-byte sector
+            const int ngroups = nst * ((rows + 7) >> 3);
+            for (int i = ot; i < ngroups * 32; i += on) {
+                const int g = i >> 5, l = i & 31;
+                const int rg = g / nst, st = g - rg * nst;
+                const int r = rg * 8 + (l >> 2), b = l & 3;
+                if (r < rows) {
+                    const uint2 v = ld_shared_v2(base + L.x + st * TILE_BYTES + (uint32_t)r * 128u +
+                                                 (((uint32_t)(2 * b) ^ (uint32_t)(r & 7)) << 4));
+                    *reinterpret_cast<uint2*>(p.codes + (int64_t)(m0 + r) * (p.C / 2) + c0 / 2 + 32 * st + 8 * b) = v;
+                }
             }
             // scales: one 4-byte word per stage of a row
-            for (int i = t; i < rows * nst; i += NQ_THREADS) {
+            for (int i = ot; i < rows * nst; i += on) {
                 const int r = i / nst, st = i - r * nst;
                 const uint32_t v = ld_shared_u32(sstage + (uint32_t)r * SROW + st * 4);
                 *reinterpret_cast<uint32_t*>(p.scales + (int64_t)(m0 + r) * (p.C / 16) + c0 / 16 + 4 * st) = v;
@@ -367,7 +391,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
             // 16-byte row l = the words of tile rows l, 32 + l, 64 + l, 96 + l
             // (rows past M hold zero scales)
             if (p.slab) {
-                for (int i = t; i < nst * 32; i += NQ_THREADS) {
+                for (int i = ot; i < nst * 32; i += on) {
                     const int st = i >> 5, l = i & 31;
                     const uint32_t sa = sstage + (uint32_t)l * SROW + st * 4;
                     const uint4 v = make_uint4(ld_shared_u32(sa), ld_shared_u32(sa + 32 * SROW),
@@ -378,82 +402,90 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
             }
         }
 
-        // epilogue: TMEM lane = token row, column = P column; the four warps
-        // of a lane quarter take 16-column chunks c = part, part + 4
-        if (p.do_mma && ok) {
-            const int sp = warp & 3;
-            const int part = (warp - 2) >> 2;
-            const int m = m0 + 32 * sp + lane;
-            const uint32_t lane_addr = (uint32_t)(32 * sp) << 16;
-            for (int c = part; c < p.r / 16; c += 4) {
-                uint32_t v[16];
-                tmem_ld_32x32b_x16(tmem + lane_addr + 16 * c, v);
-                tmem_ld_wait();
-                if (m < p.M) {
-                    float4* o = reinterpret_cast<float4*>(p.part + ((int64_t)split * p.M + m) * p.r + 16 * c);
+        // epilogue: TMEM lane = token row, column = P column.  The partials
+        // are published (a fence, then one arrival on the row tile's
+        // counter) while the other warps are still writing codes and scales.
+        if (epi_warp) {
+            if (ok && __all_sync(0xFFFFFFFFu, mbar_wait(&bars[QB_ACC], 0, ERR_WAIT_ACC_FULL, abort_flag))) {
+                tc_fence_after();
+                const int sp = warp & 3;
+                const int m = m0 + 32 * sp + lane;
+                const uint32_t lane_addr = (uint32_t)(32 * sp) << 16;
+                for (int c = 0; c < p.r / 16; ++c) {
+                    uint32_t v[16];
+                    tmem_ld_32x32b_x16(tmem + lane_addr + 16 * c, v);
+                    tmem_ld_wait();
+                    if (m < p.M) {
+                        float4* o = reinterpret_cast<float4*>(p.part + ((int64_t)split * p.M + m) * p.r + 16 * c);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        o[k] = make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
-                                           __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
+                        for (int k = 0; k < 4; ++k)
+                            o[k] = make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                                               __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
+                    }
                 }
+            }
+            __threadfence();
+            named_bar_sync(2, 128);
+            if (warp == 2 && lane == 0) {
+                // the last CTA of the row tile to arrive adds the splits
+                int last = 0;
+                if (!*abort_flag) {
+                    const unsigned prev = atomicAdd(&p.counters[blockIdx.x], 1u);
+                    last = (prev == (unsigned)(p.splits - 1)) ? 1 : 0;
+                }
+                *last_flag = last;
             }
         }
     }
-    // every thread's partial writes become visible device-wide before the
-    // completion counter below is bumped
-    __threadfence();
     tc_fence_before();
     __syncthreads();
     if (warp == 1 && p.do_mma) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
-    if (!p.do_mma || *abort_flag) return;
+    if (!p.do_mma || *abort_flag || !*last_flag) return;
 
-    // The last CTA of this row tile to finish adds the splits' partials in
-    // split order (deterministic) and rounds P = [bf16(T L1) | bf16(s T L2)].
-    if (threadIdx.x == 0) {
-        __threadfence();
-        const unsigned prev = atomicAdd(&p.counters[blockIdx.x], 1u);
-        *last_flag = (prev == (unsigned)(p.splits - 1)) ? 1 : 0;
-    }
-    __syncthreads();
-    if (!*last_flag) return;
+    // The last CTA of this row tile adds the splits' partials in split order
+    // (deterministic) and rounds P = [bf16(T L1) | bf16(s T L2)].
     __threadfence();
     const int rows = min(BM, p.M - m0);
     const int n4 = rows * p.r / 4;
     const int64_t stride4 = (int64_t)p.M * p.r / 4;
     const float4* part4 = reinterpret_cast<const float4*>(p.part) + (int64_t)m0 * p.r / 4;
-    constexpr int UNR = 4;
+    // every split's loads are issued before the first add (one L2 round trip
+    // per pass instead of one per split); the adds then run in split order
+    constexpr int UNR = 2;
     for (int i0 = threadIdx.x; i0 < n4; i0 += UNR * NUM_THREADS) {
-        float4 acc[UNR];
+        float4 v[UNR][MAX_SPLITS];
 #pragma unroll
-        for (int u = 0; u < UNR; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int k = 0; k < p.splits; ++k) {
-            float4 v[UNR];
+        for (int k = 0; k < MAX_SPLITS; ++k) {
 #pragma unroll
             for (int u = 0; u < UNR; ++u) {
                 const int i = i0 + u * NUM_THREADS;
-                v[u] = i < n4 ? __ldcg(part4 + k * stride4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-            for (int u = 0; u < UNR; ++u) {
-                acc[u].x = __fadd_rn(acc[u].x, v[u].x);
-                acc[u].y = __fadd_rn(acc[u].y, v[u].y);
-                acc[u].z = __fadd_rn(acc[u].z, v[u].z);
-                acc[u].w = __fadd_rn(acc[u].w, v[u].w);
+                v[u][k] = (k < p.splits && i < n4) ? __ldcg(part4 + k * stride4 + i)
+                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
 #pragma unroll
         for (int u = 0; u < UNR; ++u) {
             const int i = i0 + u * NUM_THREADS;
             if (i >= n4) continue;
+            float4 acc = v[u][0];
+#pragma unroll
+            for (int k = 1; k < MAX_SPLITS; ++k) {
+                if (k < p.splits) {
+                    acc.x = __fadd_rn(acc.x, v[u][k].x);
+                    acc.y = __fadd_rn(acc.y, v[u][k].y);
+                    acc.z = __fadd_rn(acc.z, v[u][k].z);
+                    acc.w = __fadd_rn(acc.w, v[u][k].w);
+                }
+            }
             const int j = (4 * i) % p.r;  // first of the four columns; r1 % 16 == 0
             const bool lora = j >= p.r1;
-            const float a0 = lora ? __fmul_rn(acc[u].x, p.s) : acc[u].x;
-            const float a1 = lora ? __fmul_rn(acc[u].y, p.s) : acc[u].y;
-            const float a2 = lora ? __fmul_rn(acc[u].z, p.s) : acc[u].z;
-            const float a3 = lora ? __fmul_rn(acc[u].w, p.s) : acc[u].w;
+            const float a0 = lora ? __fmul_rn(acc.x, p.s) : acc.x;
+            const float a1 = lora ? __fmul_rn(acc.y, p.s) : acc.y;
+            const float a2 = lora ? __fmul_rn(acc.z, p.s) : acc.z;
+            const float a3 = lora ? __fmul_rn(acc.w, p.s) : acc.w;
             __nv_bfloat162 lo = __floats2bfloat162_rn(a0, a1), hi = __floats2bfloat162_rn(a2, a3);
             uint2 o;
             o.x = *reinterpret_cast<uint32_t*>(&lo);

@@ -115,3 +115,46 @@ def test_supplied_amax_matches_computed():
     torch.cuda.synchronize()
     assert torch.equal(q1.codes, q2.codes) and torch.equal(q1.scales, q2.scales)
     assert torch.equal(q1.tscale, q2.tscale)
+
+
+def _boundary_probe(amax: float) -> np.ndarray:
+    """bf16 tensor whose tensor amax is `amax` and whose 1x16 blocks, for
+    every scale byte, hold the bf16 values next to each E2M1 rounding boundary
+    (0.25, 0.75, ..., 5) times that byte's divisor: the inputs on which a
+    quantizer that multiplies by a reciprocal instead of dividing would err."""
+    g = np.float32(np.float32(amax) / np.float32(2688.0))
+    bounds = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+    rows = []
+    for s in range(1, 0x7E):
+        e, m = (s >> 3) & 0xF, s & 7
+        sd = (m / 8.0) * 2.0**-6 if e == 0 else (1 + m / 8.0) * 2.0 ** (e - 7)
+        d = np.float32(np.float32(sd) * g)
+        vals = []
+        for bk in bounds:
+            x0 = int(np.array([np.float32(bk) * d], dtype=np.float32).view(np.uint32)[0]) >> 16
+            vals += [x0 - 1, x0, x0 + 1, x0 + 2]
+        # the block max that selects this byte: 6 * sd * g, to bf16
+        top = ft_synth.to_bf16_bits(np.array([6.0 * sd * float(g)]))[0]
+        blk = np.array(vals[:15] + [top], dtype=np.uint32)
+        blk2 = np.array(vals[15:] + [top] * (16 - len(vals[15:])), dtype=np.uint32)
+        for b in (blk, blk2):
+            b = np.clip(b, 0, 0x7F7F).astype(np.uint16)
+            rows.append(b)
+            rows.append(b | np.uint16(0x8000))  # the same magnitudes negative
+    x = np.concatenate(rows)
+    x = np.concatenate([x, ft_synth.to_bf16_bits(np.array([amax] * 16))])
+    pad = (-len(x)) % 256
+    x = np.concatenate([x, np.zeros(pad, dtype=np.uint16)])
+    return x.reshape(-1, 256)
+
+
+@pytest.mark.parametrize("amax", [5.40625, 1.0, 135.0, 0.0123, 7.3e-3, 2.2e4])
+def test_quantize_1x16_rounding_boundaries_every_scale(amax):
+    # 5.40625 is a tensor amax for which RN(1/d) misencodes one bf16 value for
+    # every scale byte with mantissa 4: the quantizer must still match the
+    # correctly rounded division bit for bit
+    x = _boundary_probe(amax)
+    a_bf16 = ft_synth.bf16_bits_to_f32(ft_synth.to_bf16_bits(np.array([amax])))[0]
+    assert oracle.amax_bf16(x) == a_bf16
+    _check_1x16(x)
+    _check_1x16(x, float(oracle.amax_bf16(x)))
