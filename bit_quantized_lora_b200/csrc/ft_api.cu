@@ -193,6 +193,20 @@ ft_status encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, ui
     return r == CUDA_SUCCESS ? FT_OK : FT_ERR_CUDA;
 }
 
+// Scale slabs [tiles][k-steps][512 B] as a 3-D byte tensor {256, 2 * k-steps,
+// tiles} with boxes of {256, 8, depth}: one stage's four slabs of `depth`
+// consecutive 128-row tiles per copy.
+ft_status encode_slabs(CUtensorMap* m, const uint8_t* slabs, int64_t ksteps, int64_t tiles, uint32_t depth) {
+    cuuint64_t dims[3] = {256, (cuuint64_t)(2 * ksteps), (cuuint64_t)tiles};
+    cuuint64_t strides[2] = {256, (cuuint64_t)(ksteps * 512)};
+    cuuint32_t box[3] = {256, 8, depth};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(slabs), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FT_OK : FT_ERR_CUDA;
+}
+
 // ------------------------------------------------------------ workspace
 constexpr int QD_MAX_SPLITS = 8;
 constexpr int LG_MAX_SPLITS = 16;
@@ -571,10 +585,11 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_slab, const float* g
     }
     // output chunks of 64 bytes per row (32 bf16 / 16 f32 columns) x 128 rows
     const int64_t esize = (ot == FT_F32) ? 4 : 2;
-    FT_TRY(encode_2d(&p.mapY, ot == FT_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                     out, Nout, M, Nout * esize, (uint32_t)(64 / esize), 128, CU_TENSOR_MAP_SWIZZLE_64B));
+    p.out = static_cast<uint8_t*>(out);
     p.sfa = a_slab;
     p.sfb = b_slab;
+    FT_TRY(encode_slabs(&p.mapSFA, a_slab, Kc / 64, cdiv(M, 128), 1));
+    FT_TRY(encode_slabs(&p.mapSFB, b_slab, Kc / 64, cdiv(Nout, 128), 2));
     p.ga = ga;
     p.gb = gb;
     p.out_f32 = (ot == FT_F32);

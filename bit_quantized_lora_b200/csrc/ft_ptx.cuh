@@ -125,6 +125,16 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* map, uint64_t
         : "memory");
 }
 
+// 3-D tiled load of one box, completion on `bar` (same rules as the 2-D form).
+__device__ __forceinline__ void tma_load_3d(void* dst, const void* map, uint64_t* bar, int c0, int c1,
+                                            int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
 // 2-D tiled store of one box from shared memory (bulk-group completion);
 // the coordinates must not be negative (x 16-byte aligned); elements past
 // the tensor's extent are not written.
@@ -342,6 +352,10 @@ __device__ __forceinline__ uint32_t ld_shared_u32(uint32_t saddr) {
 }
 __device__ __forceinline__ void st_shared_v2(uint32_t saddr, uint2 v) {
     asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(saddr), "r"(v.x), "r"(v.y) : "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
 }
 __device__ __forceinline__ void st_shared_u8(uint32_t saddr, uint32_t v) {
     asm volatile("st.shared.u8 [%0], %1;" ::"r"(saddr), "r"(v) : "memory");

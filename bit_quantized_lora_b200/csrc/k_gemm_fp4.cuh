@@ -85,11 +85,14 @@ struct LrFactor {
 
 struct Params {
     CUtensorMap mapA, mapB, mapP1, mapP2, mapL1, mapL2;
-    CUtensorMap mapY;    // output [M, Nout], box {64 bytes of columns, 128 rows}, 64 B swizzle
     const uint8_t* sfa;  // activation scale slabs [ceil(M/128)][Kc/64][512]
     const uint8_t* sfb;  // weight scale slabs [Nout/128][Kc/64][512]
+    // the same slabs as 3-D tensors {256 B, 2 * Kc / 64, tiles}: one stage's
+    // four slabs are one box (8 x 256 B) of one tile (A) or of two (B)
+    CUtensorMap mapSFA, mapSFB;
     const float* ga;
     const float* gb;
+    uint8_t* out;        // output [M, Nout], bf16 or FP32, rows contiguous
     int out_f32;
     int M, Nout, Kc;
     LrFactor f1, f2;
@@ -130,7 +133,8 @@ __host__ __device__ inline Layout make_layout(int stages, const LrFactor& f1, co
 enum {
     B_FULL = 0,                        // [MAX_STAGES] TMA landed
     B_EMPTY = B_FULL + MAX_STAGES,     // [MAX_STAGES] stage consumed by the MMAs
-    B_SF_READY = B_EMPTY + MAX_STAGES, // [2] scale slot copied into TMEM
+    B_SFFULL = B_EMPTY + MAX_STAGES,   // [MAX_STAGES] the stage's scale slabs landed
+    B_SF_READY = B_SFFULL + MAX_STAGES, // [2] scale slot copied into TMEM
     B_SF_FREE = B_SF_READY + 2,        // [2] scale slot read by its MMAs
     B_ACC_FULL = B_SF_FREE + 2,
     B_ACC_EMPTY,                       // every epilogue warp done with the tile
@@ -175,11 +179,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
     const int tiles_n = p.Nout / BN;
     const int num_tiles = tiles_m * tiles_n;
     const int KT = p.Kc / 256;  // stages per tile
-    const int KS = p.Kc / 64;   // slabs per 128-row tile
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < MAX_STAGES; ++i) {
             mbar_init(&bars[B_FULL + i], 1);
+            mbar_init(&bars[B_SFFULL + i], 1);
             mbar_init(&bars[B_EMPTY + i], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -200,6 +204,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&p.mapA);
         tma_prefetch_desc(&p.mapB);
+        tma_prefetch_desc(&p.mapSFA);
+        tma_prefetch_desc(&p.mapSFB);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, TMEM_COLS);
@@ -213,7 +219,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            const uint32_t stage_bytes = A_BYTES + B_BYTES + SFA_STAGE_BYTES + SFB_STAGE_BYTES;
+            const uint32_t stage_bytes = A_BYTES + B_BYTES;
             const uint32_t lr_total = p_bytes(p.f1) + l_bytes(p.f1) + p_bytes(p.f2) + l_bytes(p.f2);
             uint32_t it = 0;
             bool ok = true;
@@ -221,9 +227,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
                 const int tm = tile / tiles_n, tn = tile % tiles_n;
                 const int m0 = tm * BM, n0 = tn * BN;
-                const uint8_t* sfa = p.sfa + (size_t)tm * KS * 512;
-                const uint8_t* sfb0 = p.sfb + (size_t)(2 * tn) * KS * 512;
-                const uint8_t* sfb1 = sfb0 + (size_t)KS * 512;
                 if (has_lr) {
                     // low-rank panels first: the first half of the
                     // up-projection runs before the tile's mainloop
@@ -249,14 +252,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                         ok = false;
                         break;
                     }
+                    // the scale slabs first, on their own barrier: the scale
+                    // warp copies them into tensor memory while the code
+                    // tiles are still on their way
+                    uint64_t* sfb_bar = &bars[B_SFFULL + s];
+                    mbar_arrive_expect_tx(sfb_bar, SFA_STAGE_BYTES + SFB_STAGE_BYTES);
+                    tma_load_3d(smem + L.sfa + s * SFA_STAGE_BYTES, &p.mapSFA, sfb_bar, 0, 8 * kt, tm);
+                    tma_load_3d(smem + L.sfb + s * SFB_STAGE_BYTES, &p.mapSFB, sfb_bar, 0, 8 * kt, 2 * tn);
                     uint64_t* fb = &bars[B_FULL + s];
                     mbar_arrive_expect_tx(fb, stage_bytes);
                     tma_load_2d(smem + L.a + s * A_BYTES, &p.mapA, fb, kt * BK_BYTES, m0);
                     tma_load_2d(smem + L.b + s * B_BYTES, &p.mapB, fb, kt * BK_BYTES, n0);
-                    const size_t so = (size_t)kt * SFA_STAGE_BYTES;
-                    bulk_load(smem + L.sfa + s * SFA_STAGE_BYTES, sfa + so, SFA_STAGE_BYTES, fb);
-                    bulk_load(smem + L.sfb + s * SFB_STAGE_BYTES, sfb0 + so, SFA_STAGE_BYTES, fb);
-                    bulk_load(smem + L.sfb + s * SFB_STAGE_BYTES + SFA_STAGE_BYTES, sfb1 + so, SFA_STAGE_BYTES, fb);
                 }
             }
             if (!ok) {
@@ -264,6 +270,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                 for (int d = 0; d < S && d < (int)it; ++d) {
                     uint32_t j = it - 1 - d;
                     volatile int no_abort = 0;
+                    mbar_wait(&bars[B_SFFULL + (j % S)], (j / S) & 1, ERR_WAIT_DRAIN, &no_abort);
                     mbar_wait(&bars[B_FULL + (j % S)], (j / S) & 1, ERR_WAIT_DRAIN, &no_abort);
                 }
             }
@@ -360,7 +367,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                 for (int kt = 0; kt < KT; ++kt, ++it) {
                     const int s = it % S;
                     const int sb = it & 1;
-                    if (!mbar_wait(&bars[B_FULL + s], (it / S) & 1, ERR_WAIT_FULL, abort_flag) ||
+                    if (!mbar_wait(&bars[B_SFFULL + s], (it / S) & 1, ERR_WAIT_FULL, abort_flag) ||
                         !mbar_wait(&bars[B_SF_FREE + sb], ((it >> 1) & 1) ^ 1, ERR_WAIT_SF, abort_flag)) {
                         ok = false;
                         break;
@@ -392,22 +399,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
         // (with low-rank half 0), warps 8-11 columns 128-255 (half 1).
         // Output leaves in chunks of 64 bytes per row (32 bf16 or 16 f32
         // columns): the group's rows are written into its 64-byte-swizzled
-        // staging buffer and one thread of the group stores the 128-row chunk
-        // with TMA, so global writes are whole lines instead of one 16-byte
-        // piece per row.
+        // staging buffer, then the group copies the 128-row chunk out with
+        // 16-byte stores, four threads per row, so every warp store covers
+        // whole sectors of eight rows.  (A TMA store per chunk would queue
+        // in the same copy engine as the next tile's operand loads.)
         const int sp = warp & 3;  // TMEM sub-partition = rows 32*sp .. +31
         const int grp = (warp - 4) >> 2;
         const int et = (threadIdx.x - 128) & 127;  // tile row
-        const bool leader = et == 0;
-        const int cw = p.out_f32 ? 16 : 32;  // columns per chunk
-        const int nch = 128 / cw;            // chunks per group per tile
         const uint32_t rsw = (uint32_t)((et >> 1) & 3);
         const uint32_t buf = base + L.stg + (uint32_t)grp * STG_BYTES;
         const uint32_t lr_col = grp == 0 ? LR0_COL : R2_COL;
         uint64_t* lr_ready = &bars[grp == 0 ? B_LR0_READY : B_LR1_READY];
         bool ok = true;
         int local = 0;
-        bool pending = false;  // this group's buffer is being read by a store
+        const int64_t ldo = (int64_t)p.Nout * (p.out_f32 ? 4 : 2);  // output row bytes
         const float gab = __fmul_rn(*p.ga, *p.gb);
         for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
             const int m0 = (tile / tiles_n) * BM;
@@ -419,68 +424,86 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             }
             tc_fence_after();
             const uint32_t lane_addr = (uint32_t)(32 * sp) << 16;
-#pragma unroll 1
-            for (int c = 0; c < nch; ++c) {
-                const int lcol = cw * c;              // column within the group's half
-                const int col = 128 * grp + lcol;     // tile column
-                float y[32];
-                if (cw == 32) {
+            const uint32_t rowa = buf + (uint32_t)et * 64u;
+            // the staged chunk at tile column `col` leaves the buffer: piece
+            // i is row i / 4, 16-byte column i % 4
+            auto copy_out = [&](int col) {
+                uint8_t* obase = p.out + (int64_t)m0 * ldo + (int64_t)(n0 + col) * (p.out_f32 ? 4 : 2);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int i = et + 128 * k;
+                    const int row = i >> 2, q = i & 3;
+                    const uint4 v =
+                        ld_shared_v4(buf + (uint32_t)row * 64u + (((uint32_t)q ^ (uint32_t)((row >> 1) & 3)) << 4));
+                    if (m0 + row < p.M) *reinterpret_cast<uint4*>(obase + (int64_t)row * ldo + 16 * q) = v;
+                }
+            };
+            if (!p.out_f32) {
+                // bf16: the group's 128 columns of this row are read out of
+                // tensor memory and packed first, so the accumulator is
+                // released before the stores and the next tile's MMAs run
+                // while they drain
+                uint32_t pk[4][16];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
                     uint32_t v[32], lr[32];
-                    tmem_ld_32x32b_x32(tmem + lane_addr + ACC_COL + col, v);
-                    if (has_lr) tmem_ld_32x32b_x32(tmem + lane_addr + lr_col + lcol, lr);
+                    tmem_ld_32x32b_x32(tmem + lane_addr + ACC_COL + 128 * grp + 32 * c, v);
+                    if (has_lr) tmem_ld_32x32b_x32(tmem + lane_addr + lr_col + 32 * c, lr);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int k = 0; k < 32; ++k)
-                        y[k] = __fmaf_rn(gab, __uint_as_float(v[k]), has_lr ? __uint_as_float(lr[k]) : 0.0f);
-                } else {
+                    for (int k = 0; k < 16; ++k) {
+                        const float y0 = __fmaf_rn(gab, __uint_as_float(v[2 * k]), has_lr ? __uint_as_float(lr[2 * k]) : 0.0f);
+                        const float y1 =
+                            __fmaf_rn(gab, __uint_as_float(v[2 * k + 1]), has_lr ? __uint_as_float(lr[2 * k + 1]) : 0.0f);
+                        __nv_bfloat162 t = __floats2bfloat162_rn(y0, y1);
+                        pk[c][k] = *reinterpret_cast<uint32_t*>(&t);
+                    }
+                }
+                // every TMEM read of this tile is done: the MMA warp may
+                // overwrite the accumulator and both low-rank halves
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[B_ACC_EMPTY]);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    // the group's previous chunk has been copied out of the buffer
+                    named_bar_sync(1 + grp, 128);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        st_shared_v4(rowa + (((uint32_t)q ^ rsw) << 4),
+                                     make_uint4(pk[c][4 * q], pk[c][4 * q + 1], pk[c][4 * q + 2], pk[c][4 * q + 3]));
+                    named_bar_sync(1 + grp, 128);
+                    copy_out(128 * grp + 32 * c);
+                }
+            } else {
+                // FP32: eight chunks of 16 columns, the accumulator released
+                // after the last
+#pragma unroll 1
+                for (int c = 0; c < 8; ++c) {
+                    const int lcol = 16 * c;          // column within the group's half
+                    const int col = 128 * grp + lcol; // tile column
                     uint32_t v[16], lr[16];
                     tmem_ld_32x32b_x16(tmem + lane_addr + ACC_COL + col, v);
                     if (has_lr) tmem_ld_32x32b_x16(tmem + lane_addr + lr_col + lcol, lr);
                     tmem_ld_wait();
+                    float y[16];
 #pragma unroll
                     for (int k = 0; k < 16; ++k)
                         y[k] = __fmaf_rn(gab, __uint_as_float(v[k]), has_lr ? __uint_as_float(lr[k]) : 0.0f);
-                }
-                // the group's previous chunk has been read out of the buffer
-                if (leader && pending) bulk_wait_group_read<0>();
-                named_bar_sync(1 + grp, 128);
-                const uint32_t rowa = buf + (uint32_t)et * 64u;
+                    named_bar_sync(1 + grp, 128);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint4 u;
-                    if (cw == 32) {
-                        __nv_bfloat162 t0 = __floats2bfloat162_rn(y[8 * q], y[8 * q + 1]);
-                        __nv_bfloat162 t1 = __floats2bfloat162_rn(y[8 * q + 2], y[8 * q + 3]);
-                        __nv_bfloat162 t2 = __floats2bfloat162_rn(y[8 * q + 4], y[8 * q + 5]);
-                        __nv_bfloat162 t3 = __floats2bfloat162_rn(y[8 * q + 6], y[8 * q + 7]);
-                        u.x = *reinterpret_cast<uint32_t*>(&t0);
-                        u.y = *reinterpret_cast<uint32_t*>(&t1);
-                        u.z = *reinterpret_cast<uint32_t*>(&t2);
-                        u.w = *reinterpret_cast<uint32_t*>(&t3);
-                    } else {
-                        u = make_uint4(__float_as_uint(y[4 * q]), __float_as_uint(y[4 * q + 1]),
-                                       __float_as_uint(y[4 * q + 2]), __float_as_uint(y[4 * q + 3]));
-                    }
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(rowa + (((uint32_t)q ^ rsw) << 4)),
-                                 "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w)
-                                 : "memory");
+                    for (int q = 0; q < 4; ++q)
+                        st_shared_v4(rowa + (((uint32_t)q ^ rsw) << 4),
+                                     make_uint4(__float_as_uint(y[4 * q]), __float_as_uint(y[4 * q + 1]),
+                                                __float_as_uint(y[4 * q + 2]), __float_as_uint(y[4 * q + 3])));
+                    named_bar_sync(1 + grp, 128);
+                    copy_out(col);
                 }
-                fence_proxy_async_smem();
-                named_bar_sync(1 + grp, 128);
-                if (leader) {
-                    tma_store_2d(&p.mapY, smem + (buf - base), n0 + col, m0);
-                    bulk_commit_group();
-                }
-                pending = true;
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[B_ACC_EMPTY]);
             }
-            // every TMEM read of this tile is done: the MMA warp may overwrite
-            // the accumulator and both low-rank halves
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[B_ACC_EMPTY]);
         }
-        // every store has finished before the CTA exits
-        if (leader) bulk_wait_group_all();
     }
 
     tc_fence_before();
