@@ -103,6 +103,25 @@ ft_status device_info(DevInfo** out) {
 
 inline ft_status cuda_ok(cudaError_t e) { return e == cudaSuccess ? FT_OK : FT_ERR_CUDA; }
 inline ft_status last_launch() { return cuda_ok(cudaGetLastError()); }
+
+// Launches `kernel` so that it may begin while the previous kernel on the
+// stream finishes (programmatic stream serialization): the kernel waits for
+// that kernel's results itself (grid_dep_wait) after its setup.
+template <typename P>
+ft_status launch_overlapped(void (*kernel)(P), dim3 grid, dim3 block, size_t smem, cudaStream_t st, const P& p) {
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cuda_ok(cudaLaunchKernelEx(&cfg, kernel, p));
+}
 inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 inline int cdiv(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
@@ -193,6 +212,21 @@ ft_status encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, ui
     return r == CUDA_SUCCESS ? FT_OK : FT_ERR_CUDA;
 }
 
+// A row-major bf16 matrix [rows, cols] as the 3-D tensor {64, rows, cols / 64}
+// (64-column blocks as the outer dimension), boxes {64, box_rows, depth}:
+// `depth` side-by-side 128-byte-swizzled 64-column tiles in one copy.
+ft_status encode_colblocks(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_rows,
+                           uint32_t depth) {
+    cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)(cols / 64)};
+    cuuint64_t strides[2] = {(cuuint64_t)(cols * 2), 128};
+    cuuint32_t box[3] = {64, box_rows, depth};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FT_OK : FT_ERR_CUDA;
+}
+
 // Scale slabs [tiles][k-steps][512 B] as a 3-D byte tensor {256, 2 * k-steps,
 // tiles} with boxes of {256, 8, depth}: one stage's four slabs of `depth`
 // consecutive 128-row tiles per copy.
@@ -211,6 +245,7 @@ ft_status encode_slabs(CUtensorMap* m, const uint8_t* slabs, int64_t ksteps, int
 constexpr int QD_MAX_SPLITS = 8;
 constexpr int LG_MAX_SPLITS = 16;
 static_assert(QD_MAX_SPLITS <= ft::qres::MAX_SPLITS, "k_qres reduces at most MAX_SPLITS partials");
+static_assert(LG_MAX_SPLITS <= ft::lgrad::MAX_SPLITS, "k_lora_grad reduces at most MAX_SPLITS partials");
 
 struct WsPlan {
     size_t amax, gact, codes, scales, sfslab, lt, part, pg, lgpart, counters, total;
@@ -605,7 +640,7 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_slab, const float* g
     const int grid = std::max(1, std::min(tiles, d->sms));
     {
         LaunchTimer _lt(KID_GEMM, st);
-        ft::gemm::k_gemm_fp4<<<grid, ft::gemm::NUM_THREADS, smem, st>>>(p);
+        FT_TRY(launch_overlapped(ft::gemm::k_gemm_fp4, dim3((unsigned)grid), dim3(ft::gemm::NUM_THREADS), smem, st, p));
         _lt.stop();
     }
     return last_launch();
@@ -617,13 +652,12 @@ ft_status run_lora_grads(const void* dY, const void* X, const void* P, const voi
     const int64_t r = r_s + r_l;
     ft::lgrad::Params p;
     std::memset(&p, 0, sizeof(p));
-    FT_TRY(encode_2d(&p.mapT[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, N, M, N * 2, 64, 64,
+    namespace LG = ft::lgrad;
+    FT_TRY(encode_colblocks(&p.mapT[0], dY, M, N, LG::BMR, 2));
+    FT_TRY(encode_colblocks(&p.mapT[1], X, M, K, LG::BMR, 2));
+    FT_TRY(encode_2d(&p.mapS[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P, r, M, r * 2, 64, LG::BMR,
                      CU_TENSOR_MAP_SWIZZLE_128B));
-    FT_TRY(encode_2d(&p.mapT[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 64,
-                     CU_TENSOR_MAP_SWIZZLE_128B));
-    FT_TRY(encode_2d(&p.mapS[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P, r, M, r * 2, 64, 64,
-                     CU_TENSOR_MAP_SWIZZLE_128B));
-    FT_TRY(encode_2d(&p.mapS[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Pg, r, M, r * 2, 64, 64,
+    FT_TRY(encode_2d(&p.mapS[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Pg, r, M, r * 2, 64, LG::BMR,
                      CU_TENSOR_MAP_SWIZZLE_128B));
     const int ctiles = (int)(N / ft::lgrad::BC + K / ft::lgrad::BC);
     int splits = std::max(1, std::min(LG_MAX_SPLITS, d->sms / std::max(1, ctiles)));
@@ -642,13 +676,15 @@ ft_status run_lora_grads(const void* dY, const void* X, const void* P, const voi
     p.r_s = (int)r_s;
     p.r_l = (int)r_l;
     p.n_pad = r_l <= 64 ? 64 : 128;
+    p.stages = LG::stages_for(p.n_pad);
     p.mrows = mrows;
     p.splits = splits;
     p.ctiles_max = w.lg_ctiles;
     dim3 grid((unsigned)(std::max(N, K) / ft::lgrad::BC), (unsigned)splits, 2);
     {
         LaunchTimer _lt(KID_LORA_GRAD, st);
-        ft::lgrad::k_lora_grad<<<grid, ft::lgrad::NUM_THREADS, ft::lgrad::smem_bytes(p.n_pad), st>>>(p);
+        FT_TRY(launch_overlapped(ft::lgrad::k_lora_grad, grid, dim3(ft::lgrad::NUM_THREADS),
+                                 ft::lgrad::smem_bytes(p.n_pad), st, p));
         _lt.stop();
     }
     return last_launch();

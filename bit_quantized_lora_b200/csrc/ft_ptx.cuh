@@ -104,6 +104,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int co
     }
 }
 
+// ---------------------------------------------------------------- dependent launches
+// A kernel launched with programmatic stream serialization may start while
+// the previous kernel on the stream is still running: it waits here, after
+// its own setup, until that kernel has completed and its writes are
+// visible (a no-op for an ordinary launch) ...
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// ... and lets the next kernel on the stream begin its setup early.
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

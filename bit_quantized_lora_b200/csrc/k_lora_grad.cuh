@@ -9,7 +9,9 @@
 // slice of m, runs tcgen05 kind::f16 with both operands MN-major straight
 // from the TMA tiles (T^T as A, S as B), and writes an FP32 partial; the last
 // CTA of a column tile (completion counter) adds the slices in split order
-// into the output.
+// into the output.  A stage is 128 token rows: T arrives as one 32 KB 3-D
+// box (both 64-column halves) and S as one 16 KB box per 64 columns, since
+// the copy engine's cost is per copy far more than per byte.
 #pragma once
 
 #include <cuda.h>
@@ -20,25 +22,33 @@ namespace ft {
 namespace lgrad {
 
 constexpr int BC = 128;    // output rows (columns of T) per CTA
-constexpr int BMR = 64;    // token rows per stage
-constexpr int STAGES = 4;
+constexpr int BMR = 128;   // token rows per stage
+constexpr int MAX_STAGES = 4;
+constexpr int MAX_SPLITS = 16;  // token slices of one column tile
 constexpr int NUM_THREADS = 192;
-constexpr int T_BYTES = BMR * BC * 2;    // 16 KiB: two 64-column boxes
-constexpr int S_CHUNK = BMR * 64 * 2;    // 8 KiB: one 64-column box
+constexpr int T_BYTES = BMR * BC * 2;    // 32 KiB: two 64-column swizzle atoms
+constexpr int S_CHUNK = BMR * 64 * 2;    // 16 KiB: one 64-column box
 constexpr uint32_t TMEM_COLS = 128;
 
 struct Params {
-    CUtensorMap mapT[2];  // bf16 [M, C_z], box {64, 64}, 128 B swizzle
-    CUtensorMap mapS[2];  // bf16 [M, r],   box {64, 64}, 128 B swizzle
+    CUtensorMap mapT[2];  // bf16 [M, C_z] as {64, M, C_z / 64}, box {64, 128, 2}, 128 B swizzle
+    CUtensorMap mapS[2];  // bf16 [M, r],   box {64, 128}, 128 B swizzle
     float* part[2];       // [splits, C_z, r_l]
     float* out[2];        // dB [N, r_l], dA [K, r_l]
     unsigned int* counters;  // [2][ctiles_max], zero on entry; left zero on exit
     int C[2];
     int M, r_s, r_l, n_pad, mrows, splits, ctiles_max;
+    int stages;
 };
 
+// Stages that fit 192 KiB of ring: four with one S box, three with two.
+constexpr int stages_for(int n_pad) {
+    return (192 * 1024) / (T_BYTES + (n_pad / 64) * S_CHUNK) > MAX_STAGES
+               ? MAX_STAGES
+               : (192 * 1024) / (T_BYTES + (n_pad / 64) * S_CHUNK);
+}
 constexpr uint32_t smem_bytes(int n_pad) {
-    return STAGES * (T_BYTES + (n_pad / 64) * S_CHUNK) + 256 + 1024;
+    return stages_for(n_pad) * (T_BYTES + (n_pad / 64) * S_CHUNK) + 256 + 1024;
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1) k_lora_grad(const __grid_constant__ Params p) {
@@ -51,10 +61,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_lora_grad(const __grid_const
     uint8_t* smem = smem_raw + (base - raw_base);
     const int nsc = p.n_pad / 64;
     const uint32_t s_bytes = nsc * S_CHUNK;
+    const int STAGES = p.stages;
     const uint32_t off_t = 0, off_s = STAGES * T_BYTES, off_bar = STAGES * (T_BYTES + s_bytes);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + off_bar);
-    uint64_t* empty = full + STAGES;
-    uint64_t* accfull = empty + STAGES;
+    uint64_t* empty = full + MAX_STAGES;
+    uint64_t* accfull = empty + MAX_STAGES;
     uint64_t* drain = accfull + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -86,6 +97,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_lora_grad(const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // the previous kernel's outputs are complete from here on; the next
+    // kernel may start its own setup
+    grid_dep_wait();
+    grid_dep_launch();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -96,9 +111,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_lora_grad(const __grid_const
                 if (!mbar_wait(&empty[s], ph ^ 1, ERR_WAIT_EMPTY, abort_flag)) break;
                 const int m = mbeg + st * BMR;
                 mbar_arrive_expect_tx(&full[s], T_BYTES + s_bytes);
-                uint8_t* tdst = smem + off_t + s * T_BYTES;
-                tma_load_2d(tdst, mapT, &full[s], c0, m);
-                tma_load_2d(tdst + T_BYTES / 2, mapT, &full[s], c0 + 64, m);
+                tma_load_3d(smem + off_t + s * T_BYTES, mapT, &full[s], 0, m, c0 / 64);
                 uint8_t* sdst = smem + off_s + s * s_bytes;
                 for (int h = 0; h < nsc; ++h)
                     tma_load_2d(sdst + h * S_CHUNK, mapS, &full[s], p.r_s + 64 * h, m);
@@ -175,37 +188,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_lora_grad(const __grid_const
     __syncthreads();
     if (!*last_flag) return;
     __threadfence();
-    // the tile's partials, 4 floats at a time, every split's load of a batch
-    // in flight together
+    // the tile's partials, 4 floats at a time: every split's load of an
+    // element is issued before the first add (one L2 round trip per pass),
+    // then the adds run in split order
     const int n4 = BC * p.r_l / 4;
     const int64_t stride4 = (int64_t)p.C[z] * p.r_l / 4;
     const float4* part4 = reinterpret_cast<const float4*>(p.part[z]) + (int64_t)c0 * p.r_l / 4;
     float4* out4 = reinterpret_cast<float4*>(p.out[z]) + (int64_t)c0 * p.r_l / 4;
-    constexpr int UNR = 4;
-    for (int i0 = threadIdx.x; i0 < n4; i0 += UNR * NUM_THREADS) {
-        float4 acc[UNR];
+    for (int i = threadIdx.x; i < n4; i += NUM_THREADS) {
+        float4 v[MAX_SPLITS];
 #pragma unroll
-        for (int u = 0; u < UNR; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int k = 0; k < p.splits; ++k) {
-            float4 v[UNR];
+        for (int k = 0; k < MAX_SPLITS; ++k)
+            v[k] = k < p.splits ? __ldcg(part4 + k * stride4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 acc = v[0];
 #pragma unroll
-            for (int u = 0; u < UNR; ++u) {
-                const int i = i0 + u * NUM_THREADS;
-                v[u] = i < n4 ? __ldcg(part4 + k * stride4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-            for (int u = 0; u < UNR; ++u) {
-                acc[u].x = __fadd_rn(acc[u].x, v[u].x);
-                acc[u].y = __fadd_rn(acc[u].y, v[u].y);
-                acc[u].z = __fadd_rn(acc[u].z, v[u].z);
-                acc[u].w = __fadd_rn(acc[u].w, v[u].w);
+        for (int k = 1; k < MAX_SPLITS; ++k) {
+            if (k < p.splits) {
+                acc.x = __fadd_rn(acc.x, v[k].x);
+                acc.y = __fadd_rn(acc.y, v[k].y);
+                acc.z = __fadd_rn(acc.z, v[k].z);
+                acc.w = __fadd_rn(acc.w, v[k].w);
             }
         }
-#pragma unroll
-        for (int u = 0; u < UNR; ++u) {
-            const int i = i0 + u * NUM_THREADS;
-            if (i < n4) out4[i] = acc[u];
-        }
+        out4[i] = acc;
     }
     if (threadIdx.x == 0) p.counters[z * p.ctiles_max + blockIdx.x] = 0u;
 }

@@ -191,6 +191,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = p.do_mma ? *tmem_slot : 0u;
+    // the previous kernel's outputs are complete from here on; the next
+    // kernel may start its own setup
+    grid_dep_wait();
+    grid_dep_launch();
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
