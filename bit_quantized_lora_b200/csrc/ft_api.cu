@@ -250,10 +250,18 @@ static_assert(LG_MAX_SPLITS <= ft::lgrad::MAX_SPLITS, "k_lora_grad reduces at mo
 struct WsPlan {
     size_t amax, gact, codes, scales, sfslab, lt, part, pg, lgpart, counters, total;
     int n_qd_counters, lg_ctiles, n_counters;
-    // counters region: [0] tensor-amax bits and [1] grid-barrier arrivals of
-    // the resident quantizer, then the row-tile counters of the fused
-    // quantize/down-projection, then the adapter-gradient tile counters
+    // counters region: [0] tensor-amax bits, [1] grid-barrier arrivals and
+    // [2] finished CTAs of the resident quantizer, [3] unused, then the
+    // row-tile counters of the fused quantize/down-projection, then the
+    // adapter-gradient tile counters
     int qd_cnt, lg_cnt;
+};
+
+// A kernel whose every CTA counts itself into `done` when its writes are
+// finished; the kernel after it waits for `count` instead of the grid's end.
+struct DepFlag {
+    const unsigned int* done = nullptr;
+    unsigned int count = 0;
 };
 
 WsPlan plan_ws(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t r_l) {
@@ -274,9 +282,9 @@ WsPlan plan_ws(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t r_l) {
     // one per (gradient, column tile) of the adapter gradients
     w.n_qd_counters = (int)((M + 127) / 128);
     w.lg_ctiles = (int)((C + 127) / 128);
-    w.qd_cnt = 2;
-    w.lg_cnt = 2 + w.n_qd_counters;
-    w.n_counters = 2 + w.n_qd_counters + 2 * w.lg_ctiles;
+    w.qd_cnt = 4;
+    w.lg_cnt = 4 + w.n_qd_counters;
+    w.n_counters = 4 + w.n_qd_counters + 2 * w.lg_ctiles;
     w.counters = o; o += up256((size_t)w.n_counters * 4);
     w.total = o;
     return w;
@@ -488,7 +496,8 @@ ft_status launch_qres(const ft::qres::Params& p, int mt, int splits, cudaStream_
 ft_status run_quant_down(const void* T, int64_t M, int64_t C, const void* L1, int64_t r1,
                          const void* L2, int64_t r2, float s, const float* amax_in, uint8_t* codes,
                          uint8_t* scales, float* tscale, void* P, uint8_t* ws, const WsPlan& w,
-                         const DevInfo* d, cudaStream_t st) {
+                         const DevInfo* d, cudaStream_t st, DepFlag* dep) {
+    *dep = DepFlag();
     namespace Q = ft::qres;
     const int64_t r = r1 + r2;
     Q::Params p;
@@ -528,6 +537,7 @@ ft_status run_quant_down(const void* T, int64_t M, int64_t C, const void* L1, in
     p.part = reinterpret_cast<float*>(ws + w.part);
     p.P = static_cast<__nv_bfloat16*>(P);
     p.counters = counters + w.qd_cnt;
+    p.done = counters + 2;
     p.M = (int)M;
     p.C = (int)C;
     p.r = (int)r;
@@ -536,7 +546,10 @@ ft_status run_quant_down(const void* T, int64_t M, int64_t C, const void* L1, in
     p.splits = splits;
     p.s = s;
     p.num_ctas = (unsigned)(mt * splits);
-    return launch_qres(p, mt, splits, st);
+    FT_TRY(launch_qres(p, mt, splits, st));
+    dep->done = p.done;
+    dep->count = p.num_ctas;
+    return FT_OK;
 }
 
 // 1x16 quantization of a dense T [M, C] through the resident kernel (no
@@ -596,7 +609,7 @@ CUtensorMapSwizzle swizzle_for(int wbox) {
 ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_slab, const float* ga, int64_t M,
                    int64_t Kc, const uint8_t* b_codes, const uint8_t* b_slab, const float* gb,
                    int64_t Nout, const void* P, const void* L1, int64_t r1, const void* L2, int64_t r2,
-                   void* out, ft_dtype ot, const DevInfo* d, cudaStream_t st) {
+                   void* out, ft_dtype ot, const DevInfo* d, cudaStream_t st, DepFlag dep) {
     Params p;
     std::memset(&p, 0, sizeof(p));
     FT_TRY(encode_2d(&p.mapA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, Kc / 2, M, Kc / 2, 128, 128,
@@ -621,6 +634,8 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_slab, const float* g
     // output chunks of 64 bytes per row (32 bf16 / 16 f32 columns) x 128 rows
     const int64_t esize = (ot == FT_F32) ? 4 : 2;
     p.out = static_cast<uint8_t*>(out);
+    p.dep_done = dep.done;
+    p.dep_count = dep.count;
     p.sfa = a_slab;
     p.sfb = b_slab;
     FT_TRY(encode_slabs(&p.mapSFA, a_slab, Kc / 64, cdiv(M, 128), 1));
@@ -648,7 +663,7 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_slab, const float* g
 
 ft_status run_lora_grads(const void* dY, const void* X, const void* P, const void* Pg, int64_t M,
                          int64_t N, int64_t K, int64_t r_s, int64_t r_l, float* dA, float* dB,
-                         uint8_t* ws, const WsPlan& w, const DevInfo* d, cudaStream_t st) {
+                         uint8_t* ws, const WsPlan& w, const DevInfo* d, cudaStream_t st, DepFlag dep) {
     const int64_t r = r_s + r_l;
     ft::lgrad::Params p;
     std::memset(&p, 0, sizeof(p));
@@ -680,6 +695,8 @@ ft_status run_lora_grads(const void* dY, const void* X, const void* P, const voi
     p.mrows = mrows;
     p.splits = splits;
     p.ctiles_max = w.lg_ctiles;
+    p.dep_done = dep.done;
+    p.dep_count = dep.count;
     dim3 grid((unsigned)(std::max(N, K) / ft::lgrad::BC), (unsigned)splits, 2);
     {
         LaunchTimer _lt(KID_LORA_GRAD, st);
@@ -886,10 +903,11 @@ ft_status ft_linear_fwd(const ft_linear* L, const void* X, int64_t M, const floa
     float* g_x = reinterpret_cast<float*>(wsb + w.gact);
     uint8_t* codes = wsb + w.codes;
     uint8_t* scales = wsb + w.scales;
+    DepFlag dep;
     FT_TRY(run_quant_down(X, M, L->K, L->U, L->r_s, L->A, L->r_l, L->s, amax_x, codes, scales, g_x,
-                          P_save, wsb, w, d, st));
+                          P_save, wsb, w, d, st, &dep));
     return run_gemm(codes, wsb + w.sfslab, g_x, M, L->K, L->w_k.codes, L->sf_k, L->w_k.tscale, L->N,
-                    P_save, L->V, L->r_s, L->B, L->r_l, Y, yt, d, st);
+                    P_save, L->V, L->r_s, L->B, L->r_l, Y, yt, d, st, dep);
 }
 
 ft_status ft_linear_bwd(const ft_linear* L, const void* dY, const void* X, const void* P_save,
@@ -925,12 +943,16 @@ ft_status ft_linear_bwd(const ft_linear* L, const void* dY, const void* X, const
     uint8_t* codes = wsb + w.codes;
     uint8_t* scales = wsb + w.scales;
     void* Pg = wsb + w.pg;
+    DepFlag dep;
     FT_TRY(run_quant_down(dY, M, L->N, L->V, L->r_s, L->B, L->r_l, L->s, amax_dy, codes, scales, g_dy,
-                          Pg, wsb, w, d, st));
+                          Pg, wsb, w, d, st, &dep));
     FT_TRY(run_gemm(codes, wsb + w.sfslab, g_dy, M, L->N, L->w_n.codes, L->sf_n, L->w_k.tscale, L->K,
-                    Pg, L->U, L->r_s, L->A, L->r_l, dX, xt, d, st));
+                    Pg, L->U, L->r_s, L->A, L->r_l, dX, xt, d, st, dep));
+    // the adapter gradients read dY, X, P_save and Pg: nothing the dgrad GEMM
+    // (the kernel they overlap) writes, so they wait on the quantizer's
+    // counter for Pg, not on the GEMM
     if (L->r_l > 0)
-        FT_TRY(run_lora_grads(dY, X, P_save, Pg, M, L->N, L->K, L->r_s, L->r_l, dA, dB, wsb, w, d, st));
+        FT_TRY(run_lora_grads(dY, X, P_save, Pg, M, L->N, L->K, L->r_s, L->r_l, dA, dB, wsb, w, d, st, dep));
     return FT_OK;
 }
 

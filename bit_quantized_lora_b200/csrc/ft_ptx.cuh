@@ -35,6 +35,7 @@ enum : int {
     ERR_WAIT_LR = 6,
     ERR_WAIT_DRAIN = 7,
     ERR_GRID_SYNC = 8,
+    ERR_WAIT_DEP = 9,
 };
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
@@ -112,6 +113,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int co
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 // ... and lets the next kernel on the stream begin its setup early.
 __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Waits, in thread 0, until `*done` (released by each CTA of the kernel that
+// produced this kernel's inputs) reaches `count`, then orders the copy
+// engine's later reads after it; a bounded wait (the error word records
+// ERR_WAIT_DEP).  Without a counter it is the plain grid dependency wait.
+// Either way the CTA continues past a barrier, and the next kernel may start
+// its setup.  With a counter, this kernel must read nothing but the counted
+// kernel's outputs and buffers of kernels that completed before it launched,
+// and share no buffer with the kernel it overlaps.
+__device__ __forceinline__ void wait_inputs(const unsigned int* done, unsigned int count,
+                                            volatile int* abort_flag);
 
 // ---------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -325,10 +337,34 @@ __device__ __forceinline__ void red_add_release_gpu(unsigned int* p, unsigned in
 __device__ __forceinline__ void red_max_relaxed_gpu(unsigned int* p, unsigned int v) {
     asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
 __device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
     unsigned int v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+
+__device__ __forceinline__ void wait_inputs(const unsigned int* done, unsigned int count,
+                                            volatile int* abort_flag) {
+    if (done) {
+        if (threadIdx.x == 0) {
+            const uint64_t t0 = globaltimer_ns();
+            while (ld_acquire_gpu(done) < count) {
+                if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                    report_error(ERR_WAIT_DEP);
+                    *abort_flag = 1;
+                    break;
+                }
+            }
+            fence_proxy_async_global();
+        }
+    } else {
+        grid_dep_wait();
+    }
+    __syncthreads();
+    grid_dep_launch();
 }
 
 // Named barrier over `nthreads` threads (a multiple of 32) with id `id`

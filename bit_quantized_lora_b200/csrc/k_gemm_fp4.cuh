@@ -93,6 +93,8 @@ struct Params {
     const float* ga;
     const float* gb;
     uint8_t* out;        // output [M, Nout], bf16 or FP32, rows contiguous
+    const unsigned int* dep_done;  // null, or the producer's finished-CTA counter ...
+    unsigned int dep_count;        // ... and its grid size
     int out_f32;
     int M, Nout, Kc;
     LrFactor f1, f2;
@@ -215,10 +217,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // the previous kernel's outputs are complete from here on; the next
-    // kernel may start its own setup
-    grid_dep_wait();
-    grid_dep_launch();
+    // the inputs written by the previous kernel are complete from here on;
+    // the next kernel may start its own setup
+    wait_inputs(p.dep_done, p.dep_count, abort_flag);
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer

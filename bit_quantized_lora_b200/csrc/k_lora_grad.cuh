@@ -36,6 +36,8 @@ struct Params {
     float* part[2];       // [splits, C_z, r_l]
     float* out[2];        // dB [N, r_l], dA [K, r_l]
     unsigned int* counters;  // [2][ctiles_max], zero on entry; left zero on exit
+    const unsigned int* dep_done;  // null, or the finished-CTA counter of the kernel that wrote S ...
+    unsigned int dep_count;        // ... and its grid size
     int C[2];
     int M, r_s, r_l, n_pad, mrows, splits, ctiles_max;
     int stages;
@@ -97,10 +99,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_lora_grad(const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // the previous kernel's outputs are complete from here on; the next
-    // kernel may start its own setup
-    grid_dep_wait();
-    grid_dep_launch();
+    // the inputs written by the previous kernel are complete from here on;
+    // the next kernel may start its own setup
+    wait_inputs(p.dep_done, p.dep_count, abort_flag);
 
     if (warp == 0) {
         if (lane == 0) {

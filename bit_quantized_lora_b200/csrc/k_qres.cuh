@@ -84,6 +84,8 @@ struct Params {
     float* part;               // [splits, M, r] FP32 partial down-projections
     __nv_bfloat16* P;          // [M, r]
     unsigned int* counters;    // [row tiles], zero on entry; left zero on exit
+    unsigned int* done;        // null, or counts finished CTAs (zero on entry): the next
+                               // kernel may wait on it instead of on this grid's end
     int M, C, r, r1, cchunk, splits;
     float s;
     int do_mma;
@@ -121,6 +123,16 @@ enum {
     QB_COUNT
 };
 static_assert(QB_COUNT * 8 + 16 + 4 * NQ_WARPS <= BAR_BYTES, "barrier area");
+
+// Every global write of this CTA is done: count it (release) for a kernel
+// that waits on the counter rather than on this grid's completion.
+__device__ __forceinline__ void signal_done(unsigned int* done) {
+    __syncthreads();
+    if (threadIdx.x == 0 && done) {
+        __threadfence();
+        red_add_release_gpu(done, 1u);
+    }
+}
 
 // Waits for a phase that must complete (copies already issued) before the
 // CTA may exit; bounded like every other wait.
@@ -447,7 +459,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
-    if (!p.do_mma || *abort_flag || !*last_flag) return;
+    if (!p.do_mma || *abort_flag || !*last_flag) {
+        signal_done(p.done);
+        return;
+    }
 
     // The last CTA of this row tile adds the splits' partials in split order
     // (deterministic) and rounds P = [bf16(T L1) | bf16(s T L2)].
@@ -498,6 +513,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
         }
     }
     if (threadIdx.x == 0) p.counters[blockIdx.x] = 0u;
+    signal_done(p.done);
 }
 
 }  // namespace qres
