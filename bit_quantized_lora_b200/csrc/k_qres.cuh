@@ -160,6 +160,52 @@ __device__ __forceinline__ void mma_factor(uint32_t tmem_d, uint32_t a_tile, uin
                   smem_desc(b + 2 * f.sbo * j, 8192, f.sbo, f.swz), idesc, (!first || j) ? 1u : 0u);
 }
 
+// P rows of one row tile from the splits' FP32 partials: every split's
+// loads of UNR float4s are issued before the first add (one L2 round trip per
+// pass instead of one per split), then the adds run in split order.
+template <int MAXS, int UNR>
+__device__ __forceinline__ void reduce_splits(const Params& p, const float4* part4, int64_t stride4, int n4,
+                                              int m0) {
+    for (int i0 = threadIdx.x; i0 < n4; i0 += UNR * NUM_THREADS) {
+        float4 v[UNR][MAXS];
+#pragma unroll
+        for (int k = 0; k < MAXS; ++k) {
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const int i = i0 + u * NUM_THREADS;
+                v[u][k] = (k < p.splits && i < n4) ? __ldcg(part4 + k * stride4 + i)
+                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
+            const int i = i0 + u * NUM_THREADS;
+            if (i >= n4) continue;
+            float4 acc = v[u][0];
+#pragma unroll
+            for (int k = 1; k < MAXS; ++k) {
+                if (k < p.splits) {
+                    acc.x = __fadd_rn(acc.x, v[u][k].x);
+                    acc.y = __fadd_rn(acc.y, v[u][k].y);
+                    acc.z = __fadd_rn(acc.z, v[u][k].z);
+                    acc.w = __fadd_rn(acc.w, v[u][k].w);
+                }
+            }
+            const int j = (4 * i) % p.r;  // first of the four columns; r1 % 16 == 0
+            const bool lora = j >= p.r1;
+            const float a0 = lora ? __fmul_rn(acc.x, p.s) : acc.x;
+            const float a1 = lora ? __fmul_rn(acc.y, p.s) : acc.y;
+            const float a2 = lora ? __fmul_rn(acc.z, p.s) : acc.z;
+            const float a3 = lora ? __fmul_rn(acc.w, p.s) : acc.w;
+            __nv_bfloat162 lo = __floats2bfloat162_rn(a0, a1), hi = __floats2bfloat162_rn(a2, a3);
+            uint2 o;
+            o.x = *reinterpret_cast<uint32_t*>(&lo);
+            o.y = *reinterpret_cast<uint32_t*>(&hi);
+            *reinterpret_cast<uint2*>(p.P + (int64_t)m0 * p.r + 4 * i) = o;
+        }
+    }
+}
+
 __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
@@ -471,47 +517,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
     const int n4 = rows * p.r / 4;
     const int64_t stride4 = (int64_t)p.M * p.r / 4;
     const float4* part4 = reinterpret_cast<const float4*>(p.part) + (int64_t)m0 * p.r / 4;
-    // every split's loads are issued before the first add (one L2 round trip
-    // per pass instead of one per split); the adds then run in split order
-    constexpr int UNR = 2;
-    for (int i0 = threadIdx.x; i0 < n4; i0 += UNR * NUM_THREADS) {
-        float4 v[UNR][MAX_SPLITS];
-#pragma unroll
-        for (int k = 0; k < MAX_SPLITS; ++k) {
-#pragma unroll
-            for (int u = 0; u < UNR; ++u) {
-                const int i = i0 + u * NUM_THREADS;
-                v[u][k] = (k < p.splits && i < n4) ? __ldcg(part4 + k * stride4 + i)
-                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < UNR; ++u) {
-            const int i = i0 + u * NUM_THREADS;
-            if (i >= n4) continue;
-            float4 acc = v[u][0];
-#pragma unroll
-            for (int k = 1; k < MAX_SPLITS; ++k) {
-                if (k < p.splits) {
-                    acc.x = __fadd_rn(acc.x, v[u][k].x);
-                    acc.y = __fadd_rn(acc.y, v[u][k].y);
-                    acc.z = __fadd_rn(acc.z, v[u][k].z);
-                    acc.w = __fadd_rn(acc.w, v[u][k].w);
-                }
-            }
-            const int j = (4 * i) % p.r;  // first of the four columns; r1 % 16 == 0
-            const bool lora = j >= p.r1;
-            const float a0 = lora ? __fmul_rn(acc.x, p.s) : acc.x;
-            const float a1 = lora ? __fmul_rn(acc.y, p.s) : acc.y;
-            const float a2 = lora ? __fmul_rn(acc.z, p.s) : acc.z;
-            const float a3 = lora ? __fmul_rn(acc.w, p.s) : acc.w;
-            __nv_bfloat162 lo = __floats2bfloat162_rn(a0, a1), hi = __floats2bfloat162_rn(a2, a3);
-            uint2 o;
-            o.x = *reinterpret_cast<uint32_t*>(&lo);
-            o.y = *reinterpret_cast<uint32_t*>(&hi);
-            *reinterpret_cast<uint2*>(p.P + (int64_t)m0 * p.r + 4 * i) = o;
-        }
-    }
+    if (p.splits <= 4)
+        reduce_splits<4, 3>(p, part4, stride4, n4, m0);
+    else
+        reduce_splits<MAX_SPLITS, 2>(p, part4, stride4, n4, m0);
     if (threadIdx.x == 0) p.counters[blockIdx.x] = 0u;
     signal_done(p.done);
 }
