@@ -80,7 +80,8 @@ class Workspace:
 
     def get(self, nbytes: int, device) -> torch.Tensor:
         if self.buf is None or self.buf.numel() < nbytes or self.buf.device != torch.device(device):
-            self.buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+            # zero-filled once: the library's synchronisation words live here
+            self.buf = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
         return self.buf
 
 

@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
+#include <chrono>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -243,32 +245,52 @@ ft_status encode_slabs(CUtensorMap* m, const uint8_t* slabs, int64_t ksteps, int
 
 // ------------------------------------------------------------ workspace
 constexpr int QD_MAX_SPLITS = 8;
+constexpr int QRES_MAX_ROW_TILES = 1024;  // row tiles the resident quantizer's counters cover
+constexpr int LG_MAX_CTILES = 8192;       // column tiles of the adapter gradients (C <= 2^20)
 constexpr int LG_MAX_SPLITS = 16;
 static_assert(QD_MAX_SPLITS <= ft::qres::MAX_SPLITS, "k_qres reduces at most MAX_SPLITS partials");
 static_assert(LG_MAX_SPLITS <= ft::lgrad::MAX_SPLITS, "k_lora_grad reduces at most MAX_SPLITS partials");
 
 struct WsPlan {
-    size_t amax, gact, codes, scales, sfslab, lt, part, pg, lgpart, counters, total;
-    int n_qd_counters, lg_ctiles, n_counters;
-    // counters region: [0] tensor-amax bits, [1] grid-barrier arrivals and
-    // [2] finished CTAs of the resident quantizer, [3] unused, then the
-    // row-tile counters of the fused quantize/down-projection, then the
-    // adapter-gradient tile counters
-    int qd_cnt, lg_cnt;
+    size_t amax, gact, codes, scales, sfslab, lt, part, pg, lgpart, sync, qcnt, lgcnt, counters, total;
+    int n_qd_counters, lg_ctiles;
+    // sync: the resident quantizer's epoch-tagged words (grid-barrier
+    // arrivals, tensor amax, finished CTAs); qcnt: its row-tile counters;
+    // lgcnt: the adapter-gradient tile counters (all epoch-tagged: no reset);
+    // counters: the streaming quantizer's row-tile counters (zeroed per call)
 };
 
-// A kernel whose every CTA counts itself into `done` when its writes are
-// finished; the kernel after it waits for `count` instead of the grid's end.
+// A kernel whose every CTA counts itself into the epoch-tagged word `done`
+// when its writes are finished; the kernel after it waits for `count` at
+// `epoch` instead of the grid's end.
 struct DepFlag {
-    const unsigned int* done = nullptr;
+    const unsigned long long* done = nullptr;
+    unsigned long long epoch = 0;
     unsigned int count = 0;
 };
+
+// Epochs for the epoch-tagged counters: increasing across every launch of
+// the process.  The start is taken from the clock (below 2^28) so that a
+// word holding a foreign value is unlikely to match; the amax word keeps
+// 33 bits of epoch, about 8e9 launches.
+unsigned long long next_epoch() {
+    static std::atomic<unsigned long long> e{
+        (unsigned long long)(std::chrono::steady_clock::now().time_since_epoch().count() >> 10) &
+        ((1ull << 28) - 1)};
+    return ++e;
+}
 
 WsPlan plan_ws(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t r_l) {
     WsPlan w;
     const int64_t C = std::max(N, K);
     const int64_t r = r_s + r_l;
     size_t o = 0;
+    // The epoch-tagged words come first, at offsets no shape changes, so a
+    // workspace shared by calls of different shapes only ever holds epoch
+    // counters there (their content from any earlier call is valid).
+    w.sync = o;   o += 256;
+    w.qcnt = o;   o += (size_t)QRES_MAX_ROW_TILES * 8;
+    w.lgcnt = o;  o += (size_t)2 * LG_MAX_CTILES * 8;
     w.amax = o;   o += 256;
     w.gact = o;   o += 256;
     w.codes = o;  o += up256((size_t)M * C / 2);
@@ -282,10 +304,7 @@ WsPlan plan_ws(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t r_l) {
     // one per (gradient, column tile) of the adapter gradients
     w.n_qd_counters = (int)((M + 127) / 128);
     w.lg_ctiles = (int)((C + 127) / 128);
-    w.qd_cnt = 4;
-    w.lg_cnt = 4 + w.n_qd_counters;
-    w.n_counters = 4 + w.n_qd_counters + 2 * w.lg_ctiles;
-    w.counters = o; o += up256((size_t)w.n_counters * 4);
+    w.counters = o; o += up256((size_t)w.n_qd_counters * 4);
     w.total = o;
     return w;
 }
@@ -344,8 +363,7 @@ ft_status run_tile16(bool mode16x16, const void* x, int64_t rows, int64_t cols, 
 }
 
 // Q(T) and P = [bf16(T L1) | bf16(s T L2)] in one pass over T [M, C].
-// Also zeroes the completion counters (qdown and adapter-gradient tiles) the
-// kernels of this call use.
+// Also zeroes its row-tile completion counters.
 ft_status run_qdown(const void* T, int64_t M, int64_t C, const void* L1, int64_t r1, const void* L2,
                     int64_t r2, float s, const float* amax, uint8_t* codes, uint8_t* scales,
                     float* tscale, void* P, uint8_t* ws, const WsPlan& w, const DevInfo* d,
@@ -355,7 +373,7 @@ ft_status run_qdown(const void* T, int64_t M, int64_t C, const void* L1, int64_t
     if (r == 0) return run_quant_1x16(T, M, C, C, amax, codes, scales, tscale, slab, d, st);
     float* part = reinterpret_cast<float*>(ws + w.part);
     unsigned int* counters = reinterpret_cast<unsigned int*>(ws + w.counters);
-    FT_TRY(cuda_ok(cudaMemsetAsync(counters, 0, (size_t)w.n_counters * 4, st)));
+    FT_TRY(cuda_ok(cudaMemsetAsync(counters, 0, (size_t)w.n_qd_counters * 4, st)));
     ft::qdown::Params p;
     std::memset(&p, 0, sizeof(p));
     p.direct = (r1 <= 64 && r2 <= 64) ? 1 : 0;
@@ -392,7 +410,7 @@ ft_status run_qdown(const void* T, int64_t M, int64_t C, const void* L1, int64_t
     p.slab = slab;
     p.part = part;
     p.P = static_cast<__nv_bfloat16*>(P);
-    p.counters = counters + w.qd_cnt;
+    p.counters = counters;
     p.M = (int)M;
     p.C = (int)C;
     p.r = (int)r;
@@ -475,11 +493,16 @@ ft_status launch_qres(const ft::qres::Params& p, int mt, int splits, cudaStream_
     cfg.blockDim = dim3(Q::NUM_THREADS, 1, 1);
     cfg.dynamicSmemBytes = Q::make_layout(p.cchunk / Q::BKC, p.ring_bytes).total;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
+    // it may start its setup while the previous kernel finishes (it waits
+    // for that kernel's results on the device); cooperative when its grid
+    // barrier must see every CTA resident
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeCooperative;
+    attr[1].val.cooperative = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = p.amax_in ? 0 : 1;
+    cfg.numAttrs = p.amax_in ? 1 : 2;
     {
         LaunchTimer _lt(KID_QRES, st);
         FT_TRY(cuda_ok(cudaLaunchKernelEx(&cfg, Q::k_qres, p)));
@@ -507,7 +530,7 @@ ft_status run_quant_down(const void* T, int64_t M, int64_t C, const void* L1, in
     p.f2 = qres_factor(r2);
     qres_ring(p);
     int mt = 0, splits = 0, cchunk = 0;
-    if (!qres_grid(M, C, qres_max_stages(p.ring_bytes), d, &mt, &splits, &cchunk)) {
+    if (!qres_grid(M, C, qres_max_stages(p.ring_bytes), d, &mt, &splits, &cchunk) || mt > QRES_MAX_ROW_TILES) {
         const float* a = amax_in;
         if (!a) {
             FT_TRY(run_amax(T, M, C, C, reinterpret_cast<float*>(ws + w.amax), d, st));
@@ -515,8 +538,6 @@ ft_status run_quant_down(const void* T, int64_t M, int64_t C, const void* L1, in
         }
         return run_qdown(T, M, C, L1, r1, L2, r2, s, a, codes, scales, tscale, P, ws, w, d, st);
     }
-    unsigned int* counters = reinterpret_cast<unsigned int*>(ws + w.counters);
-    FT_TRY(cuda_ok(cudaMemsetAsync(counters, 0, (size_t)w.n_counters * 4, st)));
     const CUtensorMapSwizzle swz[3] = {CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_SWIZZLE_64B,
                                        CU_TENSOR_MAP_SWIZZLE_128B};
     if (r1 > 0)
@@ -528,16 +549,16 @@ ft_status run_quant_down(const void* T, int64_t M, int64_t C, const void* L1, in
     FT_TRY(encode_2d(&p.mapT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, C, M, C * 2, 64, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B));
     p.amax_in = amax_in;
-    p.amax_bits = counters;
-    p.arrivals = counters + 1;
+    p.sync = reinterpret_cast<unsigned long long*>(ws + w.sync);
+    p.epoch = next_epoch();
     p.tscale = tscale;
     p.codes = codes;
     p.scales = scales;
     p.slab = ws + w.sfslab;
     p.part = reinterpret_cast<float*>(ws + w.part);
     p.P = static_cast<__nv_bfloat16*>(P);
-    p.counters = counters + w.qd_cnt;
-    p.done = counters + 2;
+    p.counters = reinterpret_cast<unsigned long long*>(ws + w.qcnt);
+    p.count_done = 1;
     p.M = (int)M;
     p.C = (int)C;
     p.r = (int)r;
@@ -547,16 +568,17 @@ ft_status run_quant_down(const void* T, int64_t M, int64_t C, const void* L1, in
     p.s = s;
     p.num_ctas = (unsigned)(mt * splits);
     FT_TRY(launch_qres(p, mt, splits, st));
-    dep->done = p.done;
+    dep->done = p.sync + 2;
+    dep->epoch = p.epoch;
     dep->count = p.num_ctas;
     return FT_OK;
 }
 
 // 1x16 quantization of a dense T [M, C] through the resident kernel (no
-// down-projection) when it fits; sync: two words (zeroed here) when amax_in
-// is null.  Returns false in *done when the tensor does not fit.
+// down-projection) when it fits; sync: three epoch-tagged words (any content
+// left by earlier calls).  Returns false in *done when the tensor does not fit.
 ft_status run_quant_1x16_resident(const void* T, int64_t M, int64_t C, const float* amax_in,
-                                  unsigned int* sync, uint8_t* codes, uint8_t* scales,
+                                  unsigned long long* sync, uint8_t* codes, uint8_t* scales,
                                   float* tscale, const DevInfo* d, cudaStream_t st, bool* done) {
     namespace Q = ft::qres;
     Q::Params p;
@@ -566,12 +588,11 @@ ft_status run_quant_1x16_resident(const void* T, int64_t M, int64_t C, const flo
     *done = false;
     if (!qres_grid(M, C, qres_max_stages(p.ring_bytes), d, &mt, &splits, &cchunk)) return FT_OK;
     *done = true;
-    if (!amax_in) FT_TRY(cuda_ok(cudaMemsetAsync(sync, 0, 2 * sizeof(unsigned int), st)));
     FT_TRY(encode_2d(&p.mapT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, C, M, C * 2, 64, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B));
     p.amax_in = amax_in;
-    p.amax_bits = sync;
-    p.arrivals = sync ? sync + 1 : nullptr;
+    p.sync = sync;
+    p.epoch = next_epoch();
     p.tscale = tscale;
     p.codes = codes;
     p.scales = scales;
@@ -635,6 +656,7 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_slab, const float* g
     const int64_t esize = (ot == FT_F32) ? 4 : 2;
     p.out = static_cast<uint8_t*>(out);
     p.dep_done = dep.done;
+    p.dep_epoch = dep.epoch;
     p.dep_count = dep.count;
     p.sfa = a_slab;
     p.sfb = b_slab;
@@ -684,7 +706,8 @@ ft_status run_lora_grads(const void* dY, const void* X, const void* P, const voi
     p.part[1] = partA;
     p.out[0] = dB;
     p.out[1] = dA;
-    p.counters = reinterpret_cast<unsigned int*>(ws + w.counters) + w.lg_cnt;
+    p.counters = reinterpret_cast<unsigned long long*>(ws + w.lgcnt);
+    p.epoch = next_epoch();
     p.C[0] = (int)N;
     p.C[1] = (int)K;
     p.M = (int)M;
@@ -694,8 +717,9 @@ ft_status run_lora_grads(const void* dY, const void* X, const void* P, const voi
     p.stages = LG::stages_for(p.n_pad);
     p.mrows = mrows;
     p.splits = splits;
-    p.ctiles_max = w.lg_ctiles;
+    p.ctiles_max = LG_MAX_CTILES;
     p.dep_done = dep.done;
+    p.dep_epoch = dep.epoch;
     p.dep_count = dep.count;
     dim3 grid((unsigned)(std::max(N, K) / ft::lgrad::BC), (unsigned)splits, 2);
     {
@@ -828,13 +852,16 @@ ft_status ft_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, ft_
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (blk == FT_BLK_1x16 && ld == cols) {
         bool done = false;
-        FT_TRY(run_quant_1x16_resident(x, rows, cols, amax, static_cast<unsigned int*>(ws), out->codes,
+        // the amax slot sits at the start of the workspace, the
+        // synchronisation words 64 bytes in
+        unsigned long long* sync = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(ws) + 64);
+        FT_TRY(run_quant_1x16_resident(x, rows, cols, amax, sync, out->codes,
                                        out->scales, out->tscale, d, st, &done));
         if (done) return FT_OK;
     }
     const float* a = amax;
     if (!a) {
-        float* slot = static_cast<float*>(ws);
+        float* slot = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + 128);
         FT_TRY(run_amax(x, rows, cols, ld, slot, d, st));
         a = slot;
     }
@@ -872,7 +899,7 @@ ft_status ft_quantize_transpose(const void* x, int64_t rows, int64_t cols, int64
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const float* a = amax;
     if (!a) {
-        float* slot = static_cast<float*>(ws);
+        float* slot = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + 128);
         FT_TRY(run_amax(x, rows, cols, ld, slot, d, st));
         a = slot;
     }

@@ -114,16 +114,17 @@ __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.w
 // ... and lets the next kernel on the stream begin its setup early.
 __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
-// Waits, in thread 0, until `*done` (released by each CTA of the kernel that
-// produced this kernel's inputs) reaches `count`, then orders the copy
-// engine's later reads after it; a bounded wait (the error word records
-// ERR_WAIT_DEP).  Without a counter it is the plain grid dependency wait.
-// Either way the CTA continues past a barrier, and the next kernel may start
-// its setup.  With a counter, this kernel must read nothing but the counted
-// kernel's outputs and buffers of kernels that completed before it launched,
-// and share no buffer with the kernel it overlaps.
-__device__ __forceinline__ void wait_inputs(const unsigned int* done, unsigned int count,
-                                            volatile int* abort_flag);
+// Waits, in thread 0, until the epoch-tagged counter `done` (released by each
+// CTA of the kernel that produced this kernel's inputs) reaches `count` for
+// `epoch`, then orders the copy engine's later reads after it; a bounded wait
+// (the error word records ERR_WAIT_DEP).  Without a counter it is the plain
+// grid dependency wait.  Either way the CTA continues past a barrier, and
+// the next kernel may start its setup.  With a counter, this kernel must read
+// nothing but the counted kernel's outputs and buffers of kernels that
+// completed before that kernel passed its own dependency wait, and share no
+// buffer with the kernel it overlaps.
+__device__ __forceinline__ void wait_inputs(const unsigned long long* done, unsigned long long epoch,
+                                            unsigned int count, volatile int* abort_flag);
 
 // ---------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -337,6 +338,44 @@ __device__ __forceinline__ void red_add_release_gpu(unsigned int* p, unsigned in
 __device__ __forceinline__ void red_max_relaxed_gpu(unsigned int* p, unsigned int v) {
     asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+// ---------------------------------------------------------------- epoch-tagged counters
+// A 64-bit counter word holds (epoch << 20) + count.  Every launch that uses
+// it gets a new, larger epoch from the host, so a word left by any earlier
+// launch (finished or not) reads as older and needs no reset: a user first
+// raises it to (epoch << 20) with an atomic max, then counts.  Waiters compare
+// for equality, so a word holding a foreign value makes them time out rather
+// than pass.
+constexpr int kEpochShift = 20;
+__device__ __forceinline__ unsigned long long epoch_base(unsigned long long epoch) {
+    return epoch << kEpochShift;
+}
+// Joins the epoch and counts one (relaxed); returns the count before.
+__device__ __forceinline__ unsigned long long epoch_count(unsigned long long* w, unsigned long long epoch) {
+    atomicMax(w, epoch_base(epoch));
+    return atomicAdd(w, 1ull) - epoch_base(epoch);
+}
+// Joins the epoch and counts one, releasing this thread's earlier writes (and
+// those it has observed) to whoever acquires the count.
+__device__ __forceinline__ void epoch_count_release(unsigned long long* w, unsigned long long epoch) {
+    atomicMax(w, epoch_base(epoch));
+    asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(w), "l"(1ull) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+// Waits until the word reads (epoch << 20) + count exactly; false on timeout.
+__device__ __forceinline__ bool epoch_wait(const unsigned long long* w, unsigned long long epoch,
+                                           unsigned long long count) {
+    const unsigned long long target = epoch_base(epoch) + count;
+    if (ld_acquire_gpu_u64(w) == target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire_gpu_u64(w) != target)
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    return true;
+}
+
 __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
@@ -346,17 +385,13 @@ __device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
     return v;
 }
 
-__device__ __forceinline__ void wait_inputs(const unsigned int* done, unsigned int count,
-                                            volatile int* abort_flag) {
+__device__ __forceinline__ void wait_inputs(const unsigned long long* done, unsigned long long epoch,
+                                            unsigned int count, volatile int* abort_flag) {
     if (done) {
         if (threadIdx.x == 0) {
-            const uint64_t t0 = globaltimer_ns();
-            while (ld_acquire_gpu(done) < count) {
-                if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                    report_error(ERR_WAIT_DEP);
-                    *abort_flag = 1;
-                    break;
-                }
+            if (!epoch_wait(done, epoch, count)) {
+                report_error(ERR_WAIT_DEP);
+                *abort_flag = 1;
             }
             fence_proxy_async_global();
         }

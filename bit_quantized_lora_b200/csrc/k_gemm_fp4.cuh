@@ -93,8 +93,9 @@ struct Params {
     const float* ga;
     const float* gb;
     uint8_t* out;        // output [M, Nout], bf16 or FP32, rows contiguous
-    const unsigned int* dep_done;  // null, or the producer's finished-CTA counter ...
-    unsigned int dep_count;        // ... and its grid size
+    const unsigned long long* dep_done;  // null, or the producer's finished-CTA counter,
+    unsigned long long dep_epoch;        // its epoch
+    unsigned int dep_count;              // and its grid size
     int out_f32;
     int M, Nout, Kc;
     LrFactor f1, f2;
@@ -219,7 +220,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
     const uint32_t tmem = *tmem_slot;
     // the inputs written by the previous kernel are complete from here on;
     // the next kernel may start its own setup
-    wait_inputs(p.dep_done, p.dep_count, abort_flag);
+    wait_inputs(p.dep_done, p.dep_epoch, p.dep_count, abort_flag);
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer

@@ -35,9 +35,11 @@ struct Params {
     CUtensorMap mapS[2];  // bf16 [M, r],   box {64, 128}, 128 B swizzle
     float* part[2];       // [splits, C_z, r_l]
     float* out[2];        // dB [N, r_l], dA [K, r_l]
-    unsigned int* counters;  // [2][ctiles_max], zero on entry; left zero on exit
-    const unsigned int* dep_done;  // null, or the finished-CTA counter of the kernel that wrote S ...
-    unsigned int dep_count;        // ... and its grid size
+    unsigned long long* counters;  // [2][ctiles_max] epoch-tagged arrivals of the splits
+    unsigned long long epoch;      // this launch's epoch (host-issued, increasing)
+    const unsigned long long* dep_done;  // null, or the finished-CTA counter of the kernel that wrote S,
+    unsigned long long dep_epoch;        // its epoch
+    unsigned int dep_count;              // and its grid size
     int C[2];
     int M, r_s, r_l, n_pad, mrows, splits, ctiles_max;
     int stages;
@@ -101,7 +103,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_lora_grad(const __grid_const
     const uint32_t tmem = *tmem_slot;
     // the inputs written by the previous kernel are complete from here on;
     // the next kernel may start its own setup
-    wait_inputs(p.dep_done, p.dep_count, abort_flag);
+    wait_inputs(p.dep_done, p.dep_epoch, p.dep_count, abort_flag);
 
     if (warp == 0) {
         if (lane == 0) {
@@ -183,8 +185,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_lora_grad(const __grid_const
     if (*abort_flag) return;
     if (threadIdx.x == 0) {
         __threadfence();
-        const unsigned prev = atomicAdd(&p.counters[z * p.ctiles_max + blockIdx.x], 1u);
-        *last_flag = (prev == (unsigned)(p.splits - 1)) ? 1 : 0;
+        const unsigned long long prev = epoch_count(&p.counters[z * p.ctiles_max + blockIdx.x], p.epoch);
+        *last_flag = (prev == (unsigned long long)(p.splits - 1)) ? 1 : 0;
     }
     __syncthreads();
     if (!*last_flag) return;
@@ -213,7 +215,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_lora_grad(const __grid_const
         }
         out4[i] = acc;
     }
-    if (threadIdx.x == 0) p.counters[z * p.ctiles_max + blockIdx.x] = 0u;
 }
 
 }  // namespace lgrad

@@ -75,17 +75,19 @@ struct Params {
     CUtensorMap mapL1;  // bf16 [C, r1], box {wbox1, 64}
     CUtensorMap mapL2;  // bf16 [C, r2], box {wbox2, 64}
     const float* amax_in;      // caller's tensor amax, or null (computed here)
-    unsigned int* amax_bits;   // global max word, zero on entry (amax_in == null)
-    unsigned int* arrivals;    // grid barrier counter, zero on entry (amax_in == null)
+    // epoch-tagged words (any earlier content is fine): [0] grid-barrier
+    // arrivals, [1] tensor amax as (epoch << 31) | bits, [2] finished CTAs
+    unsigned long long* sync;
+    unsigned long long epoch;  // this launch's epoch (host-issued, increasing)
     float* tscale;
     uint8_t* codes;
     uint8_t* scales;
     uint8_t* slab;             // null, or the scales again in the GEMM slab layout
     float* part;               // [splits, M, r] FP32 partial down-projections
     __nv_bfloat16* P;          // [M, r]
-    unsigned int* counters;    // [row tiles], zero on entry; left zero on exit
-    unsigned int* done;        // null, or counts finished CTAs (zero on entry): the next
-                               // kernel may wait on it instead of on this grid's end
+    unsigned long long* counters;  // [row tiles] epoch-tagged arrivals of the splits
+    int count_done;            // count finished CTAs into sync[2]: the next kernel
+                               // may wait on it instead of on this grid's end
     int M, C, r, r1, cchunk, splits;
     float s;
     int do_mma;
@@ -126,11 +128,11 @@ static_assert(QB_COUNT * 8 + 16 + 4 * NQ_WARPS <= BAR_BYTES, "barrier area");
 
 // Every global write of this CTA is done: count it (release) for a kernel
 // that waits on the counter rather than on this grid's completion.
-__device__ __forceinline__ void signal_done(unsigned int* done) {
+__device__ __forceinline__ void signal_done(const Params& p) {
     __syncthreads();
-    if (threadIdx.x == 0 && done) {
+    if (threadIdx.x == 0 && p.count_done) {
         __threadfence();
-        red_add_release_gpu(done, 1u);
+        epoch_count_release(&p.sync[2], p.epoch);
     }
 }
 
@@ -363,17 +365,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
                 // every CTA arrives, also one that gave up, so no other CTA
                 // waits on it; the release orders this CTA's max before its
                 // arrival
-                if (m) red_max_relaxed_gpu(p.amax_bits, m);
-                red_add_release_gpu(p.arrivals, 1u);
-                const uint64_t t0 = globaltimer_ns();
-                while (ld_acquire_gpu(p.arrivals) < p.num_ctas) {
-                    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                atomicMax(&p.sync[1], (p.epoch << 31) | m);
+                epoch_count_release(&p.sync[0], p.epoch);
+                amax_t = 0.0f;
+                if (!epoch_wait(&p.sync[0], p.epoch, p.num_ctas)) {
+                    report_error(ERR_GRID_SYNC);
+                    *abort_flag = 1;
+                } else {
+                    const unsigned long long a = ld_acquire_gpu_u64(&p.sync[1]);
+                    if ((a >> 31) != p.epoch) {
+                        // the word held a value no earlier launch writes
                         report_error(ERR_GRID_SYNC);
                         *abort_flag = 1;
-                        break;
                     }
+                    amax_t = __uint_as_float((uint32_t)(a & 0x7FFFFFFFull));
                 }
-                amax_t = __uint_as_float(ld_acquire_gpu(p.amax_bits));
             }
             *amax_share = __float_as_uint(amax_t);
         }
@@ -492,8 +498,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
                 // the last CTA of the row tile to arrive adds the splits
                 int last = 0;
                 if (!*abort_flag) {
-                    const unsigned prev = atomicAdd(&p.counters[blockIdx.x], 1u);
-                    last = (prev == (unsigned)(p.splits - 1)) ? 1 : 0;
+                    const unsigned long long prev = epoch_count(&p.counters[blockIdx.x], p.epoch);
+                    last = (prev == (unsigned long long)(p.splits - 1)) ? 1 : 0;
                 }
                 *last_flag = last;
             }
@@ -506,7 +512,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
         tmem_dealloc(tmem, TMEM_COLS);
     }
     if (!p.do_mma || *abort_flag || !*last_flag) {
-        signal_done(p.done);
+        signal_done(p);
         return;
     }
 
@@ -521,8 +527,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
         reduce_splits<4, 3>(p, part4, stride4, n4, m0);
     else
         reduce_splits<MAX_SPLITS, 2>(p, part4, stride4, n4, m0);
-    if (threadIdx.x == 0) p.counters[blockIdx.x] = 0u;
-    signal_done(p.done);
+    signal_done(p);
 }
 
 }  // namespace qres

@@ -179,7 +179,12 @@ ft_status ft_linear_bwd(const ft_linear* L, const void* dY, const void* X, const
                         int64_t M, const float* amax_dy, void* dX, ft_dtype xt, float* dA,
                         float* dB, void* ws, size_t ws_bytes, void* stream);
 
-/* Workspace sizes (bytes) for the calls above. */
+/* Workspace sizes (bytes) for the calls above.  Zero-fill a workspace once
+ * after allocating it (e.g. cudaMemsetAsync); calls keep their
+ * synchronisation words in it and never need it cleared again, whatever
+ * earlier calls (finished, failed or of other shapes) left behind.  A
+ * workspace holding arbitrary bytes can make a call's device waits run out
+ * (reported by ft_device_error as a timeout) instead of computing. */
 size_t ft_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t r_l);
 size_t ft_quantize_workspace_bytes(void);
 
