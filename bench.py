@@ -473,6 +473,7 @@ def run_ours(args):
             "launch_ms": qd_ms / qd_n,
             "amax_gbs": am_gbs,
             "lora_grad_gbs": lg_gbs,
+            "lora_grad_traffic": ncu_traffic("k_lora_grad", "k_lora_grad.cuh"),
             "traffic": ncu_traffic(qd_kernel, qd_kernel + ".cuh"),
         },
         "kernels_ms_per_step": {k: v[0] / args.steps for k, v in kt.items()},
