@@ -228,3 +228,27 @@ def test_fused_quantizer_output_is_bit_exact(case):
     assert np.float32(g) == np.float32(rg)
     np.testing.assert_array_equal(scales, rs_)
     np.testing.assert_array_equal(codes, rc)
+
+
+def test_foreign_sync_words_time_out_then_zeroing_recovers():
+    """The workspace's synchronisation words are epoch-tagged: anything an
+    earlier call left is valid, but a value no call writes (here all ones)
+    must make the bounded device waits run out and report it through the
+    error word -- not pass early and compute from a wrong tensor amax -- and
+    zero-filling the workspace once must restore bit-identical results."""
+    inp, U, V, Wr, layer = _prep(ft_synth.WORKLOADS[1], 22, M=512)
+    X = dev_bf16(inp["X"])
+    ws = ft.Workspace()
+    ws.get(ft.ft_workspace_bytes(X.shape[0], layer.N, layer.K, layer.r_s, layer.r_l), X.device)
+    Y0, P0 = ft.ft_linear_fwd(layer, X, out_dtype=ft.F32, ws=ws)
+    torch.cuda.synchronize()
+    assert ft.ft_device_error() == 0
+    ws.buf[:256].fill_(0xFF)
+    ft.ft_linear_fwd(layer, X, out_dtype=ft.F32, ws=ws)
+    torch.cuda.synchronize()
+    assert ft.ft_device_error() != 0
+    ws.buf.zero_()
+    Y1, P1 = ft.ft_linear_fwd(layer, X, out_dtype=ft.F32, ws=ws)
+    torch.cuda.synchronize()
+    assert ft.ft_device_error() == 0
+    assert torch.equal(Y0, Y1) and torch.equal(P0, P1)
