@@ -55,6 +55,40 @@ constexpr uint32_t smem_bytes(int n_pad) {
     return stages_for(n_pad) * (T_BYTES + (n_pad / 64) * S_CHUNK) + 256 + 1024;
 }
 
+// out = the sum over splits of the partials, in split order, for n4 float4
+// elements; every split's loads of UNR elements are in flight together.
+template <int MAXS, int UNR>
+__device__ __forceinline__ void reduce_splits(const float4* part4, int64_t stride4, int n4, int splits,
+                                              float4* out4) {
+    for (int i0 = threadIdx.x; i0 < n4; i0 += UNR * NUM_THREADS) {
+        float4 v[UNR][MAXS];
+#pragma unroll
+        for (int k = 0; k < MAXS; ++k) {
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const int i = i0 + u * NUM_THREADS;
+                v[u][k] = (k < splits && i < n4) ? __ldcg(part4 + k * stride4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
+            const int i = i0 + u * NUM_THREADS;
+            if (i >= n4) continue;
+            float4 acc = v[u][0];
+#pragma unroll
+            for (int k = 1; k < MAXS; ++k) {
+                if (k < splits) {
+                    acc.x = __fadd_rn(acc.x, v[u][k].x);
+                    acc.y = __fadd_rn(acc.y, v[u][k].y);
+                    acc.z = __fadd_rn(acc.z, v[u][k].z);
+                    acc.w = __fadd_rn(acc.w, v[u][k].w);
+                }
+            }
+            out4[i] = acc;
+        }
+    }
+}
+
 __global__ void __launch_bounds__(NUM_THREADS, 1) k_lora_grad(const __grid_constant__ Params p) {
     const int z = blockIdx.z;
     const int c0 = blockIdx.x * BC;
@@ -191,30 +225,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_lora_grad(const __grid_const
     __syncthreads();
     if (!*last_flag) return;
     __threadfence();
-    // the tile's partials, 4 floats at a time: every split's load of an
-    // element is issued before the first add (one L2 round trip per pass),
+    // the tile's partials, 4 floats at a time: every split's load of UNR
+    // elements is issued before the first add (one L2 round trip per pass),
     // then the adds run in split order
     const int n4 = BC * p.r_l / 4;
     const int64_t stride4 = (int64_t)p.C[z] * p.r_l / 4;
     const float4* part4 = reinterpret_cast<const float4*>(p.part[z]) + (int64_t)c0 * p.r_l / 4;
     float4* out4 = reinterpret_cast<float4*>(p.out[z]) + (int64_t)c0 * p.r_l / 4;
-    for (int i = threadIdx.x; i < n4; i += NUM_THREADS) {
-        float4 v[MAX_SPLITS];
-#pragma unroll
-        for (int k = 0; k < MAX_SPLITS; ++k)
-            v[k] = k < p.splits ? __ldcg(part4 + k * stride4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-        float4 acc = v[0];
-#pragma unroll
-        for (int k = 1; k < MAX_SPLITS; ++k) {
-            if (k < p.splits) {
-                acc.x = __fadd_rn(acc.x, v[k].x);
-                acc.y = __fadd_rn(acc.y, v[k].y);
-                acc.z = __fadd_rn(acc.z, v[k].z);
-                acc.w = __fadd_rn(acc.w, v[k].w);
-            }
-        }
-        out4[i] = acc;
-    }
+    if (p.splits <= 4)
+        reduce_splits<4, 3>(part4, stride4, n4, p.splits, out4);
+    else
+        reduce_splits<MAX_SPLITS, 1>(part4, stride4, n4, p.splits, out4);
 }
 
 }  // namespace lgrad
