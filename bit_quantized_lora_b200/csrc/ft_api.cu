@@ -658,8 +658,6 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_slab, const float* g
     p.dep_done = dep.done;
     p.dep_epoch = dep.epoch;
     p.dep_count = dep.count;
-    p.sfa = a_slab;
-    p.sfb = b_slab;
     FT_TRY(encode_slabs(&p.mapSFA, a_slab, Kc / 64, cdiv(M, 128), 1));
     FT_TRY(encode_slabs(&p.mapSFB, b_slab, Kc / 64, cdiv(Nout, 128), 2));
     p.ga = ga;

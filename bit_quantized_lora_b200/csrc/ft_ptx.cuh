@@ -157,36 +157,7 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* map, uint64_t
         : "memory");
 }
 
-// 2-D tiled store of one box from shared memory (bulk-group completion);
-// the coordinates must not be negative (x 16-byte aligned); elements past
-// the tensor's extent are not written.
-__device__ __forceinline__ void tma_store_2d(const void* map, const void* src, int c0, int c1) {
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
-                 "r"(smem_u32(src)), "r"(c0), "r"(c1)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_commit_group() {
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-// Waits until at most N committed bulk groups still read shared memory.
-template <int N>
-__device__ __forceinline__ void bulk_wait_group_read() {
-    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-// Waits until every committed bulk group has completed.
-__device__ __forceinline__ void bulk_wait_group_all() {
-    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
 
-// 1-D bulk copy of `bytes` (a multiple of 16; both addresses 16-byte
-// aligned) from global into shared memory; completes `bar`'s tx count.
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
 
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
@@ -271,13 +242,6 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
           "=r"(r[31])
         : "r"(taddr));
 }
-// Each thread of the warp reads 8 consecutive 32-bit columns of its lane.
-__device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, uint32_t (&r)[8]) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-                   "=r"(r[7])
-                 : "r"(taddr));
-}
 // Each thread of the warp reads 16 consecutive 32-bit columns of its lane.
 __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
@@ -331,13 +295,6 @@ __host__ __device__ constexpr uint32_t idesc_nvfp4(int M, int N) {
            | ((uint32_t)(M >> 4) << 24); // M / 16
 }
 
-// ---------------------------------------------------------------- grid-wide flags
-__device__ __forceinline__ void red_add_release_gpu(unsigned int* p, unsigned int v) {
-    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ void red_max_relaxed_gpu(unsigned int* p, unsigned int v) {
-    asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
 // ---------------------------------------------------------------- epoch-tagged counters
 // A 64-bit counter word holds (epoch << 20) + count.  Every launch that uses
 // it gets a new, larger epoch from the host, so a word left by any earlier
@@ -378,11 +335,6 @@ __device__ __forceinline__ bool epoch_wait(const unsigned long long* w, unsigned
 
 __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
-    unsigned int v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
 }
 
 __device__ __forceinline__ void wait_inputs(const unsigned long long* done, unsigned long long epoch,

@@ -85,10 +85,9 @@ struct LrFactor {
 
 struct Params {
     CUtensorMap mapA, mapB, mapP1, mapP2, mapL1, mapL2;
-    const uint8_t* sfa;  // activation scale slabs [ceil(M/128)][Kc/64][512]
-    const uint8_t* sfb;  // weight scale slabs [Nout/128][Kc/64][512]
-    // the same slabs as 3-D tensors {256 B, 2 * Kc / 64, tiles}: one stage's
-    // four slabs are one box (8 x 256 B) of one tile (A) or of two (B)
+    // the block-scale slabs ([tiles][Kc/64][512 B], activations and weights)
+    // as 3-D tensors {256 B, 2 * Kc / 64, tiles}: one stage's four slabs are
+    // one box (8 x 256 B) of one tile (A) or of two (B)
     CUtensorMap mapSFA, mapSFB;
     const float* ga;
     const float* gb;
