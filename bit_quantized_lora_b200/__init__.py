@@ -166,13 +166,13 @@ class Layer:
     V: torch.Tensor | None
     A: torch.Tensor | None
     B: torch.Tensor | None
-    sf_k: torch.Tensor | None = None  # the scale grid expanded per row of w_k
-    sf_n: torch.Tensor | None = None  # ... and per row of w_n
+    op_k: torch.Tensor | None = None  # the GEMM's image of w_k (codes + per-row scales)
+    op_n: torch.Tensor | None = None  # ... and of w_n
 
     def view(self) -> FtLinear:
         return FtLinear(self.N, self.K, self.r_s, self.r_l, self.s, self.w_k.view(), self.w_n.view(),
-                        _ptr(self.U), _ptr(self.V), _ptr(self.A), _ptr(self.B), _ptr(self.sf_k),
-                        _ptr(self.sf_n))
+                        _ptr(self.U), _ptr(self.V), _ptr(self.A), _ptr(self.B), _ptr(self.op_k),
+                        _ptr(self.op_n))
 
 
 def svd_split(W: torch.Tensor, r_s: int):
@@ -211,20 +211,22 @@ def prepare_layer(W: torch.Tensor | None = None, r_s: int = 0, A: torch.Tensor |
     r_s = 0 if U is None else U.shape[1]
     r_l = 0 if A is None else A.shape[1]
     w_k, w_n = ft_quantize_transpose(W_res.contiguous(), BLK_16x16, amax=amax, ws=ws)
-    sf_k, sf_n = ft_expand_weight_scales(w_k.scales, N, K)
+    op_k, op_n = ft_pack_weight_operands(w_k, w_n, N, K)
     return Layer(N, K, r_s, r_l, float(s), w_k, w_n, U, V,
-                 None if A is None else A.contiguous(), None if B is None else B.contiguous(), sf_k, sf_n)
+                 None if A is None else A.contiguous(), None if B is None else B.contiguous(), op_k, op_n)
 
 
-def ft_expand_weight_scales(grid: torch.Tensor, N: int, K: int, stream=None):
-    """The 16x16 scale grid of Q(W_res) laid out per row for both code
-    layouts, as the 4-bit GEMMs read it.  Returns (sf_k, sf_n), uint8."""
-    nbytes = load().ft_weight_scales_bytes(N, K)
-    sf_k = torch.empty(nbytes, dtype=torch.uint8, device=grid.device)
-    sf_n = torch.empty(nbytes, dtype=torch.uint8, device=grid.device)
-    check("ft_expand_weight_scales", load().ft_expand_weight_scales(
-        grid.data_ptr(), N, K, sf_k.data_ptr(), sf_n.data_ptr(), _stream(stream)))
-    return sf_k, sf_n
+def ft_pack_weight_operands(w_k, w_n, N: int, K: int, stream=None):
+    """The 4-bit GEMMs' images of Q(W_res) in both orientations: codes and the
+    16x16 scales repeated per row, side by side per 256 x 256 block.  Returns
+    (op_k, op_n), uint8."""
+    nbytes = load().ft_weight_operand_bytes(N, K)
+    op_k = torch.empty(nbytes, dtype=torch.uint8, device=w_k.codes.device)
+    op_n = torch.empty(nbytes, dtype=torch.uint8, device=w_k.codes.device)
+    check("ft_pack_weight_operands", load().ft_pack_weight_operands(
+        w_k.codes.data_ptr(), w_n.codes.data_ptr(), w_k.scales.data_ptr(), N, K, op_k.data_ptr(),
+        op_n.data_ptr(), _stream(stream)))
+    return op_k, op_n
 
 
 def ft_linear_fwd(layer: Layer, X: torch.Tensor, amax_x: torch.Tensor | None = None,

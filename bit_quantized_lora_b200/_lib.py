@@ -35,8 +35,8 @@ class FtLinear(ctypes.Structure):
         ("V", c_vp),
         ("A", c_vp),
         ("B", c_vp),
-        ("sf_k", c_vp),
-        ("sf_n", c_vp),
+        ("op_k", c_vp),
+        ("op_n", c_vp),
     ]
 
 
@@ -53,8 +53,8 @@ SIGNATURES = {
                                      ctypes.c_int, c_vp, c_vp, c_vp, ctypes.c_size_t, c_vp]),
     "ft_workspace_bytes": (ctypes.c_size_t, [c_i64, c_i64, c_i64, c_i64, c_i64]),
     "ft_quantize_workspace_bytes": (ctypes.c_size_t, []),
-    "ft_weight_scales_bytes": (ctypes.c_size_t, [c_i64, c_i64]),
-    "ft_expand_weight_scales": (ctypes.c_int, [c_vp, c_i64, c_i64, c_vp, c_vp, c_vp]),
+    "ft_weight_operand_bytes": (ctypes.c_size_t, [c_i64, c_i64]),
+    "ft_pack_weight_operands": (ctypes.c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_vp]),
     "ft_workspace_qact": (ctypes.c_int, [c_i64, c_i64, c_i64, c_i64, c_i64,
                                          ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t),
                                          ctypes.POINTER(ctypes.c_size_t)]),

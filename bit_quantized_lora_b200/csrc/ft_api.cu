@@ -628,15 +628,26 @@ CUtensorMapSwizzle swizzle_for(int wbox) {
 // out[M, Nout] = ga gb Q(A) Q(B)^T + P[:, :r1] L1^T + P[:, r1:] L2^T, the
 // block scales of A and B given as slabs ([rows/128][Kc/64][512]).
 ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_slab, const float* ga, int64_t M,
-                   int64_t Kc, const uint8_t* b_codes, const uint8_t* b_slab, const float* gb,
+                   int64_t Kc, const uint8_t* b_op, const float* gb,
                    int64_t Nout, const void* P, const void* L1, int64_t r1, const void* L2, int64_t r2,
                    void* out, ft_dtype ot, const DevInfo* d, cudaStream_t st, DepFlag dep) {
     Params p;
     std::memset(&p, 0, sizeof(p));
     FT_TRY(encode_2d(&p.mapA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, Kc / 2, M, Kc / 2, 128, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B));
-    FT_TRY(encode_2d(&p.mapB, CU_TENSOR_MAP_DATA_TYPE_UINT8, b_codes, Kc / 2, Nout, Kc / 2, 128,
-                     ft::gemm::BN, CU_TENSOR_MAP_SWIZZLE_128B));
+    {
+        // the weight's operand image (ft_pack_weight_operands) as a 3-D byte
+        // tensor {128, 144, 2 * blocks}: one block (codes + scales of a
+        // 256-row tile for one stage) is one box of {128, 144, 2}
+        cuuint64_t dims[3] = {128, 144, (cuuint64_t)((Nout / 256) * (Kc / 256) * 2)};
+        cuuint64_t strides[2] = {128, 144 * 128};
+        cuuint32_t box[3] = {128, 144, 2};
+        cuuint32_t estr[3] = {1, 1, 1};
+        if (g_encode(&p.mapB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(b_op), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return FT_ERR_CUDA;
+    }
     const int64_t r = r1 + r2;
     p.f1 = gemm_factor(r1, 0);
     p.f2 = gemm_factor(r2, r1);
@@ -652,14 +663,11 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_slab, const float* g
         FT_TRY(encode_2d(&p.mapL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2, r2, Nout, r2 * 2, p.f2.wbox,
                          ft::gemm::BN, swizzle_for(p.f2.wbox)));
     }
-    // output chunks of 64 bytes per row (32 bf16 / 16 f32 columns) x 128 rows
-    const int64_t esize = (ot == FT_F32) ? 4 : 2;
     p.out = static_cast<uint8_t*>(out);
     p.dep_done = dep.done;
     p.dep_epoch = dep.epoch;
     p.dep_count = dep.count;
     FT_TRY(encode_slabs(&p.mapSFA, a_slab, Kc / 64, cdiv(M, 128), 1));
-    FT_TRY(encode_slabs(&p.mapSFB, b_slab, Kc / 64, cdiv(Nout, 128), 2));
     p.ga = ga;
     p.gb = gb;
     p.out_f32 = (ot == FT_F32);
@@ -756,8 +764,8 @@ ft_status check_linear(const ft_linear* L) {
     if ((L->U && !al16(L->U)) || (L->V && !al16(L->V)) || (L->A && !al16(L->A)) ||
         (L->B && !al16(L->B)))
         return FT_ERR_ALIGN;
-    if (!L->sf_k || !L->sf_n) return FT_ERR_INVALID_ARG;
-    if (!al16(L->sf_k) || !al16(L->sf_n)) return FT_ERR_ALIGN;
+    if (!L->op_k || !L->op_n) return FT_ERR_INVALID_ARG;
+    if (!al16(L->op_k) || !al16(L->op_n)) return FT_ERR_ALIGN;
     return FT_OK;
 }
 
@@ -781,23 +789,25 @@ const char* ft_status_str(ft_status s) {
 
 size_t ft_quantize_workspace_bytes(void) { return 256; }
 
-size_t ft_weight_scales_bytes(int64_t N, int64_t K) {
+size_t ft_weight_operand_bytes(int64_t N, int64_t K) {
     if (N < 0 || K < 0) return 0;
-    return (size_t)N * (size_t)K / 16;
+    return (size_t)(N / 256) * (size_t)(K / 256) * 288u * 128u;
 }
 
-ft_status ft_expand_weight_scales(const uint8_t* grid, int64_t N, int64_t K, uint8_t* sf_k,
-                                  uint8_t* sf_n, void* stream) {
-    if (!grid || !sf_k || !sf_n || N < 0 || K < 0) return FT_ERR_INVALID_ARG;
+ft_status ft_pack_weight_operands(const uint8_t* codes_k, const uint8_t* codes_n, const uint8_t* grid,
+                                  int64_t N, int64_t K, uint8_t* op_k, uint8_t* op_n, void* stream) {
+    if (!codes_k || !codes_n || !grid || !op_k || !op_n || N < 0 || K < 0) return FT_ERR_INVALID_ARG;
     if (N % 256 || K % 256) return FT_ERR_SHAPE;
-    if (!al16(sf_k) || !al16(sf_n)) return FT_ERR_ALIGN;
+    if (!al16(codes_k) || !al16(codes_n) || !al16(op_k) || !al16(op_n)) return FT_ERR_ALIGN;
     if (N == 0 || K == 0) return FT_OK;
     DevInfo* d;
     FT_TRY(device_info(&d));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int64_t rows = (N / 128) * (K / 64) * 32 * 2;  // 16-byte slab rows, both layouts
-    const int grid_n = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(rows, 256), (int64_t)d->sms * 8));
-    ft::k_expand_wsf<<<grid_n, 256, 0, st>>>(grid, N, K, sf_k, sf_n);
+    const int64_t chunks = (int64_t)ft_weight_operand_bytes(N, K) / 16;
+    const int grid_n = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(chunks, 256), (int64_t)d->sms * 16));
+    ft::k_pack_wop<<<grid_n, 256, 0, st>>>(codes_k, grid, N, K, 0, op_k);
+    FT_TRY(last_launch());
+    ft::k_pack_wop<<<grid_n, 256, 0, st>>>(codes_n, grid, N, K, 1, op_n);
     return last_launch();
 }
 
@@ -931,7 +941,7 @@ ft_status ft_linear_fwd(const ft_linear* L, const void* X, int64_t M, const floa
     DepFlag dep;
     FT_TRY(run_quant_down(X, M, L->K, L->U, L->r_s, L->A, L->r_l, L->s, amax_x, codes, scales, g_x,
                           P_save, wsb, w, d, st, &dep));
-    return run_gemm(codes, wsb + w.sfslab, g_x, M, L->K, L->w_k.codes, L->sf_k, L->w_k.tscale, L->N,
+    return run_gemm(codes, wsb + w.sfslab, g_x, M, L->K, L->op_k, L->w_k.tscale, L->N,
                     P_save, L->V, L->r_s, L->B, L->r_l, Y, yt, d, st, dep);
 }
 
@@ -971,7 +981,7 @@ ft_status ft_linear_bwd(const ft_linear* L, const void* dY, const void* X, const
     DepFlag dep;
     FT_TRY(run_quant_down(dY, M, L->N, L->V, L->r_s, L->B, L->r_l, L->s, amax_dy, codes, scales, g_dy,
                           Pg, wsb, w, d, st, &dep));
-    FT_TRY(run_gemm(codes, wsb + w.sfslab, g_dy, M, L->N, L->w_n.codes, L->sf_n, L->w_k.tscale, L->K,
+    FT_TRY(run_gemm(codes, wsb + w.sfslab, g_dy, M, L->N, L->op_n, L->w_k.tscale, L->K,
                     Pg, L->U, L->r_s, L->A, L->r_l, dX, xt, d, st, dep));
     // the adapter gradients read dY, X, P_save and Pg: nothing the dgrad GEMM
     // (the kernel they overlap) writes, so they wait on the quantizer's

@@ -63,9 +63,12 @@ constexpr int MAX_STAGES = 4;
 constexpr int NUM_EPI_WARPS = 8;  // two column groups of four lane-quarter warps
 constexpr int NUM_THREADS = 128 + 32 * NUM_EPI_WARPS;
 constexpr int A_BYTES = BM * BK_BYTES;         // 16 KiB
-constexpr int B_BYTES = BN * BK_BYTES;         // 32 KiB
+constexpr int B_BYTES = BN * BK_BYTES;         // 32 KiB of codes
 constexpr int SFA_STAGE_BYTES = KSTEPS * 512;  // four slabs (128 rows)
 constexpr int SFB_STAGE_BYTES = 2 * KSTEPS * 512;  // two row halves x four slabs
+// one block of the weight's operand image: the B tile's codes, then its
+// scale slabs (they arrive in one copy)
+constexpr int B_SLOT = B_BYTES + SFB_STAGE_BYTES;  // 36 KiB
 constexpr uint32_t TMEM_COLS = 512;
 // TMEM columns: [0,256) accumulator; [256,384) low-rank half 0; [384,512)
 // shared in time: the scale ring while the mainloop runs, low-rank half 1
@@ -88,7 +91,7 @@ struct Params {
     // the block-scale slabs ([tiles][Kc/64][512 B], activations and weights)
     // as 3-D tensors {256 B, 2 * Kc / 64, tiles}: one stage's four slabs are
     // one box (8 x 256 B) of one tile (A) or of two (B)
-    CUtensorMap mapSFA, mapSFB;
+    CUtensorMap mapSFA;
     const float* ga;
     const float* gb;
     uint8_t* out;        // output [M, Nout], bf16 or FP32, rows contiguous
@@ -102,7 +105,7 @@ struct Params {
 };
 
 struct Layout {
-    uint32_t a, b, sfa, sfb, p1, p2, l1, l2, stg, bars, total;
+    uint32_t a, b, sfa, p1, p2, l1, l2, stg, bars, total;
 };
 constexpr uint32_t STG_BYTES = 128 * 64;  // one staged output chunk: 128 rows x 64 bytes
 
@@ -118,13 +121,12 @@ __host__ __device__ inline Layout make_layout(int stages, const LrFactor& f1, co
     Layout L;
     uint32_t o = 0;
     L.a = o;    o += stages * A_BYTES;
-    L.b = o;    o += stages * B_BYTES;
+    L.b = o;    o += stages * B_SLOT;
     L.p1 = o;   o += p_bytes(f1);
     L.l1 = o;   o += l_bytes(f1);
     L.p2 = o;   o += p_bytes(f2);
     L.l2 = o;   o += l_bytes(f2);
     L.sfa = o;  o += stages * SFA_STAGE_BYTES;
-    L.sfb = o;  o += stages * SFB_STAGE_BYTES;
     L.stg = o;  o += 2 * STG_BYTES;  // output staging, one buffer per column group
     L.bars = o; o += 256;  // barriers, TMEM slot, abort flag
     L.total = o + 1024;    // slack for 1 KiB alignment of the base
@@ -207,7 +209,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
         tma_prefetch_desc(&p.mapA);
         tma_prefetch_desc(&p.mapB);
         tma_prefetch_desc(&p.mapSFA);
-        tma_prefetch_desc(&p.mapSFB);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, TMEM_COLS);
@@ -224,7 +225,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            const uint32_t stage_bytes = A_BYTES + B_BYTES;
+            const uint32_t stage_bytes = A_BYTES;
             const uint32_t lr_total = p_bytes(p.f1) + l_bytes(p.f1) + p_bytes(p.f2) + l_bytes(p.f2);
             uint32_t it = 0;
             bool ok = true;
@@ -257,17 +258,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                         ok = false;
                         break;
                     }
-                    // the scale slabs first, on their own barrier: the scale
-                    // warp copies them into tensor memory while the code
-                    // tiles are still on their way
+                    // the weight block (codes and scales in one copy) and the
+                    // activation scale slabs first, on their own barrier: the
+                    // scale warp copies the scales into tensor memory while
+                    // the activation codes are still on their way
                     uint64_t* sfb_bar = &bars[B_SFFULL + s];
-                    mbar_arrive_expect_tx(sfb_bar, SFA_STAGE_BYTES + SFB_STAGE_BYTES);
+                    mbar_arrive_expect_tx(sfb_bar, B_SLOT + SFA_STAGE_BYTES);
+                    tma_load_3d(smem + L.b + s * B_SLOT, &p.mapB, sfb_bar, 0, 0, 2 * (tn * KT + kt));
                     tma_load_3d(smem + L.sfa + s * SFA_STAGE_BYTES, &p.mapSFA, sfb_bar, 0, 8 * kt, tm);
-                    tma_load_3d(smem + L.sfb + s * SFB_STAGE_BYTES, &p.mapSFB, sfb_bar, 0, 8 * kt, 2 * tn);
                     uint64_t* fb = &bars[B_FULL + s];
                     mbar_arrive_expect_tx(fb, stage_bytes);
                     tma_load_2d(smem + L.a + s * A_BYTES, &p.mapA, fb, kt * BK_BYTES, m0);
-                    tma_load_2d(smem + L.b + s * B_BYTES, &p.mapB, fb, kt * BK_BYTES, n0);
                 }
             }
             if (!ok) {
@@ -313,13 +314,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     const int s = it % S;
                     const int sb = it & 1;
                     if (!mbar_wait(&bars[B_FULL + s], (it / S) & 1, ERR_WAIT_FULL, abort_flag) ||
+                        !mbar_wait(&bars[B_SFFULL + s], (it / S) & 1, ERR_WAIT_FULL, abort_flag) ||
                         !mbar_wait(&bars[B_SF_READY + sb], (it >> 1) & 1, ERR_WAIT_SF, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t a_lo = a_lo0 + s * (A_BYTES >> 4);
-                    const uint32_t b_lo = b_lo0 + s * (B_BYTES >> 4);
+                    const uint32_t b_lo = b_lo0 + s * (B_SLOT >> 4);
                     const uint32_t sf = tmem + R2_COL + sb * SF_SLOT_COLS;
 #pragma unroll
                     for (int j = 0; j < KSTEPS; ++j)
@@ -357,7 +359,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
         if (lane == 0) {
             const uint32_t hi_sf = (128u >> 4) | (1u << 14);  // 8-row groups 128 B apart
             const uint32_t sfa_lo0 = (base + L.sfa) >> 4;     // one 16-byte column: LBO unused
-            const uint32_t sfb_lo0 = (base + L.sfb) >> 4;
+            const uint32_t sfb_lo0 = (base + L.b + B_BYTES) >> 4;  // the scales behind each B tile
             uint32_t it = 0;
             bool ok = true;
             int local = 0;
@@ -379,7 +381,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     }
                     tc_fence_after();
                     const uint32_t sfa_lo = sfa_lo0 + s * (SFA_STAGE_BYTES >> 4);
-                    const uint32_t sfb_lo = sfb_lo0 + s * (SFB_STAGE_BYTES >> 4);
+                    const uint32_t sfb_lo = sfb_lo0 + s * (B_SLOT >> 4);
                     const uint32_t sf = tmem + R2_COL + sb * SF_SLOT_COLS;
 #pragma unroll
                     for (int j = 0; j < KSTEPS; ++j) {

@@ -66,39 +66,56 @@ __global__ void __launch_bounds__(256) k_amax_bf16(const uint16_t* __restrict__ 
     }
 }
 
-// ---------------------------------------------------- scale slabs
-// Expands a weight's 16x16 scale grid [N/16, K/16] into the slab layout of
-// both code layouts: sf_k for W_res (rows N, contraction K) and sf_n for
-// W_res^T (rows K, contraction N).  Each 16x16 scale is repeated for its 16
-// rows; no scale is recomputed.  One thread per 16-byte slab row.
-__global__ void __launch_bounds__(256) k_expand_wsf(const uint8_t* __restrict__ grid, int64_t N,
-                                                    int64_t K, uint8_t* __restrict__ sf_k,
-                                                    uint8_t* __restrict__ sf_n) {
-    const int64_t gc = K / 16;
-    const int64_t rows_k = (N / 128) * (K / 64) * 32;  // slab rows of sf_k
-    const int64_t rows_n = (K / 128) * (N / 64) * 32;
+// ---------------------------------------------------- weight operand images
+// The GEMM's image of one orientation of Q(W_res): for every 256-row tile t
+// of the operand and every 256-deep stage kt of the contraction, one block
+// of 288 rows of 128 bytes (36 KB): rows 0-255 hold the codes of operand
+// rows 256t .. 256t + 255, contraction bytes [128 kt, 128 kt + 128); rows
+// 256-287 hold the block scales of those rows for the stage in the slab
+// order tensor memory wants (two 128-row halves x four 64-deep steps x 512
+// bytes; byte 16l + 4i + b of a slab is the scale of half-row 32i + l, block
+// b), each 16-byte chunk c of slab row p stored at chunk c ^ (p % 8) so that
+// a 128-byte-swizzled copy lands it in natural order.  One copy per stage
+// then brings a tile and its scales.
+//   codes: the operand's codes [R, Kc/2]; grid: the 16x16 scale grid
+//   [N/16, K/16]; trans = 0: operand rows are N (op_k, Kc = K), trans = 1:
+//   operand rows are K (op_n, Kc = N) and the grid is read transposed.
+__global__ void __launch_bounds__(256) k_pack_wop(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ grid,
+                                                  int64_t N, int64_t K, int trans, uint8_t* __restrict__ op) {
+    const int64_t R = trans ? K : N, Kc = trans ? N : K;
+    const int64_t KT = Kc / 256, gc = K / 16;
+    const int64_t chunks = (R / 256) * KT * 288 * 8;
     const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < rows_k + rows_n; i += nthr) {
-        const bool trans = i >= rows_k;
-        const int64_t j = trans ? i - rows_k : i;
-        const int64_t l = j & 31, slab = j >> 5;
-        const int64_t ks_per = trans ? N / 64 : K / 64;
-        const int64_t t = slab / ks_per, ks = slab - t * ks_per;
-        uint32_t w[4];
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < chunks; i += nthr) {
+        const int64_t blk = i / (288 * 8);
+        const int rc = (int)(i - blk * 288 * 8);
+        const int row = rc >> 3, c = rc & 7;
+        const int64_t t = blk / KT, kt = blk - t * KT;
+        uint4 v;
+        if (row < 256) {
+            v = *reinterpret_cast<const uint4*>(codes + (256 * t + row) * (Kc / 2) + 128 * kt + 16 * c);
+        } else {
+            const int pr = row - 256;
+            const int nat = pr * 128 + 16 * (c ^ (pr & 7));  // natural byte offset in the scale image
+            uint32_t w[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int64_t row = 128 * t + 32 * q + l;  // row of this operand
-            uint32_t v = 0;
+            for (int q = 0; q < 4; ++q) {
+                uint32_t acc = 0;
 #pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const int64_t kb = 4 * ks + b;  // 16-column block of the contraction
-                const uint32_t sb = trans ? grid[kb * gc + row / 16] : grid[(row / 16) * gc + kb];
-                v |= sb << (8 * b);
+                for (int bb = 0; bb < 4; ++bb) {
+                    const int beta = nat + 4 * q + bb;
+                    const int h = beta >> 11, j = (beta >> 9) & 3, e = beta & 511;
+                    const int l = e >> 4, ii = (e >> 2) & 3, b = e & 3;
+                    const int64_t orow = 256 * t + 128 * h + 32 * ii + l;  // operand row
+                    const int64_t kb = 16 * kt + 4 * j + b;                // 16-wide contraction block
+                    const uint32_t sb = trans ? grid[kb * gc + orow / 16] : grid[(orow / 16) * gc + kb];
+                    acc |= sb << (8 * bb);
+                }
+                w[q] = acc;
             }
-            w[q] = v;
+            v = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        uint8_t* dst = (trans ? sf_n : sf_k) + slab * 512 + l * 16;
-        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(op + i * 16) = v;
     }
 }
 

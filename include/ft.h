@@ -94,10 +94,11 @@ typedef struct {
  *   U [K, r_s], V [N, r_s], A [K, r_l], B [N, r_l]: bf16, row-major, dense.
  *   r_s, r_l: multiples of 16 with r_s + r_l <= 128 (either may be 0).
  *   s: the LoRA scale.
- *   sf_k, sf_n: the scale grid expanded for the tensor cores, one scale per
- *         row of w_k and of w_n (ft_expand_weight_scales fills them from
- *         w_k.scales; ft_weight_scales_bytes(N, K) bytes each, 16-byte
- *         aligned).  A layout of the same scales, not a new quantization.  */
+ *   op_k, op_n: the 4-bit GEMMs' images of w_k and of w_n: codes and
+ *         scales of each 256 x 256 block side by side, the scales one per
+ *         row (ft_pack_weight_operands fills them from w_k, w_n and the
+ *         grid; ft_weight_operand_bytes(N, K) bytes each, 16-byte aligned).
+ *         A layout of the same codes and scales, not a new quantization.  */
 typedef struct {
     int64_t N, K, r_s, r_l;
     float s;
@@ -107,8 +108,8 @@ typedef struct {
     const void* V;
     const void* A;
     const void* B;
-    const uint8_t* sf_k;
-    const uint8_t* sf_n;
+    const uint8_t* op_k;
+    const uint8_t* op_n;
 } ft_linear;
 
 /* ft_quantize -- Q(x) for a bf16 matrix (section 3.2 block quantization).
@@ -137,22 +138,28 @@ ft_status ft_quantize_transpose(const void* x, int64_t rows, int64_t cols, int64
                                 ft_block blk, const float* amax, ft_fp4* out_row,
                                 ft_fp4* out_col, void* ws, size_t ws_bytes, void* stream);
 
-/* ft_expand_weight_scales -- once per weight, after its 16x16 quantization:
- * writes the per-row scale layouts the 4-bit GEMMs read (section 3.2: the
- * grid of a 16x16 block serves W_res and W_res^T alike, so each grid entry
- * is repeated for the 16 rows of its block in either orientation; no value
- * changes).
- *   grid : the [N/16, K/16] E4M3 scale grid of Q(W_res) (w_k.scales).
- *   sf_k : ft_weight_scales_bytes(N, K) bytes, for w_k (rows N, along K).
- *   sf_n : as many bytes, for w_n (rows K, along N).
- *   N, K : multiples of 256.  Both outputs 16-byte aligned.
- * Layout (for a matrix of R rows and C columns): [R/128][C/64][512 B];
- * byte 16 l + 4 i + b of block (t, s) holds the scale of row 128 t + 32 i + l
- * for columns 64 s + 16 b .. + 15 -- the order tcgen05.cp copies into the
- * tensor memory's scale-factor layout.                                     */
-size_t ft_weight_scales_bytes(int64_t N, int64_t K);
-ft_status ft_expand_weight_scales(const uint8_t* grid, int64_t N, int64_t K, uint8_t* sf_k,
-                                  uint8_t* sf_n, void* stream);
+/* ft_pack_weight_operands -- once per weight, after its 16x16 quantization:
+ * writes the operand images the 4-bit GEMMs read, one per orientation
+ * (section 3.2: the grid of a 16x16 block serves W_res and W_res^T alike,
+ * so each grid entry is repeated for the 16 rows of its block in either
+ * orientation; no value changes).
+ *   codes_k : w_k.codes [N, K/2];  codes_n : w_n.codes [K, N/2].
+ *   grid    : the [N/16, K/16] E4M3 scale grid of Q(W_res) (w_k.scales).
+ *   op_k, op_n: ft_weight_operand_bytes(N, K) bytes each, 16-byte aligned.
+ *   N, K    : multiples of 256.
+ * Layout (an operand of R rows and C contraction columns): for each 256-row
+ * tile t and 256-deep stage kt, a block of 288 rows of 128 bytes: rows
+ * 0-255 = the codes of rows 256 t .. + 255, contraction bytes 128 kt ..
+ * + 127; rows 256-287 = their scales for the stage, as two 128-row halves x
+ * four 64-deep steps x 512 bytes, byte 16 l + 4 i + b of a step holding the
+ * scale of half-row 32 i + l, columns 64 s + 16 b .. + 15 (the order
+ * tcgen05.cp copies into the tensor memory's scale-factor layout), with
+ * 16-byte chunk c of scale row p stored at chunk c ^ (p % 8) (undone by the
+ * 128-byte swizzle of the copy that loads a block).  Blocks are ordered
+ * (t, kt) with kt fastest.                                                 */
+size_t ft_weight_operand_bytes(int64_t N, int64_t K);
+ft_status ft_pack_weight_operands(const uint8_t* codes_k, const uint8_t* codes_n, const uint8_t* grid,
+                                  int64_t N, int64_t K, uint8_t* op_k, uint8_t* op_n, void* stream);
 
 /* ft_linear_fwd -- Eq. 2 with LoRA fusion (section 3.3): one pass over X
  * emits Q(X) and the down-projections P = [bf16(X U) | bf16(s X A)]; one

@@ -112,12 +112,12 @@ def test_linear_validation_happens_on_the_host(L):
     shared = _linear()
     shared.w_n.scales = 0x300000
     assert L.ft_linear_fwd(ctypes.byref(shared), x, 128, None, x, 0, x, x, ws, None) == FT_ERR_INVALID_ARG
-    # the expanded weight scales are required and 16-byte aligned
+    # the weight operand images are required and 16-byte aligned
     no_sf = _linear()
-    no_sf.sf_n = None
+    no_sf.op_n = None
     assert L.ft_linear_fwd(ctypes.byref(no_sf), x, 128, None, x, 0, x, x, ws, None) == FT_ERR_INVALID_ARG
     odd_sf = _linear()
-    odd_sf.sf_k = 0x100008
+    odd_sf.op_k = 0x100008
     assert L.ft_linear_fwd(ctypes.byref(odd_sf), x, 128, None, x, 0, x, x, ws, None) == FT_ERR_ALIGN
     # M = 0: nothing to do
     assert L.ft_linear_fwd(ctypes.byref(ok), x, 0, None, x, 0, x, x, ws, None) == FT_OK
@@ -142,11 +142,14 @@ def test_workspace_qact_offsets_lie_inside_the_workspace(L):
     assert L.ft_workspace_qact(1, 1, 1, 0, 0, None, ctypes.byref(bad), ctypes.byref(bad)) == FT_ERR_INVALID_ARG
 
 
-def test_weight_scale_expansion_validation(L):
-    assert L.ft_weight_scales_bytes(3072, 3072) == 3072 * 3072 // 16
-    assert L.ft_weight_scales_bytes(-1, 256) == 0
+def test_weight_operand_packing_validation(L):
+    # one 288 x 128-byte block (codes + scales) per 256 x 256 tile of the weight
+    assert L.ft_weight_operand_bytes(3072, 3072) == 12 * 12 * 288 * 128
+    assert L.ft_weight_operand_bytes(3072, 3072) == 3072 * 3072 // 2 * 9 // 8
+    assert L.ft_weight_operand_bytes(-1, 256) == 0
     g = 0x100000
-    assert L.ft_expand_weight_scales(None, 256, 256, g, g, None) == FT_ERR_INVALID_ARG
-    assert L.ft_expand_weight_scales(g, 320, 256, g, g, None) == FT_ERR_SHAPE
-    assert L.ft_expand_weight_scales(g, 256, 256, g + 8, g, None) == FT_ERR_ALIGN
-    assert L.ft_expand_weight_scales(g, 0, 256, g, g, None) == FT_OK
+    assert L.ft_pack_weight_operands(None, g, g, 256, 256, g, g, None) == FT_ERR_INVALID_ARG
+    assert L.ft_pack_weight_operands(g, g, None, 256, 256, g, g, None) == FT_ERR_INVALID_ARG
+    assert L.ft_pack_weight_operands(g, g, g, 320, 256, g, g, None) == FT_ERR_SHAPE
+    assert L.ft_pack_weight_operands(g, g, g, 256, 256, g + 8, g, None) == FT_ERR_ALIGN
+    assert L.ft_pack_weight_operands(g, g, g, 0, 256, g, g, None) == FT_OK
