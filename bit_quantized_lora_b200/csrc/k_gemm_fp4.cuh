@@ -13,22 +13,25 @@
 //           P = [dY V | s dY B], L1 = U, L2 = A.
 //
 // Block scales arrive in the tensor-memory slab layout (below): the
-// activation quantizers write it next to the row-major scales, and the
-// weight's 16x16 grid is expanded into it once, for both code layouts, when
-// the weight is prepared (section 3.2: one grid serves W and W^T; the
-// expansion repeats each 16x16 scale for its 16 rows and changes no code).
+// activation quantizers write it next to the row-major scales; the weight's
+// 16x16 grid is expanded into it once per layer, for both code layouts, and
+// stored behind each 256 x 256 block of codes in the weight's operand image
+// (section 3.2: one grid serves W and W^T; the expansion repeats each 16x16
+// scale for its 16 rows and changes no code).
 // Slab layout of an operand with R rows and Kc contraction columns:
 // [ceil(R/128)][Kc/64][512 B], byte 16 l + 4 i + b of slab (t, s) = the
 // scale of row 128 t + 32 i + l, 16-column block 4 s + b.  One slab is
 // exactly what tcgen05.cp.32x128b.warpx4 turns into the scale layout the
 // MMA reads (row m at TMEM lane m % 32 of every lane quarter, column
-// c + m / 32), so the MMA warp copies it straight from the TMA buffer.
+// c + m / 32).
 //
 // Blackwell mapping: one CTA per SM, persistent over 128x256 output tiles
 // (a tcgen05 MMA costs about the same for N = 128 as for N = 256, so the
 // wide tile doubles the work per instruction).
-//   warp 0  TMA producer: FP4 code tiles (128 B swizzle) and the scale slabs
-//           of each stage (bulk copies), the tile's P / L1 / L2 panels.
+//   warp 0  TMA producer: per stage, the weight block (codes + scales, one
+//           3-D box) and the activation scale slabs on one barrier, the
+//           activation code tile (128 B swizzle) on another; per tile the
+//           P / L1 / L2 panels.
 //   warp 1  TMEM owner and UMMA issuer: half 0 of the low-rank
 //           up-projection (kind::f16, N = 128), then four
 //           tcgen05.mma.kind::mxf4nvf4.block16 (K = 64, N = 256) per stage
@@ -37,8 +40,8 @@
 //           ring of scale columns, ahead of the MMAs (copies issued by
 //           another warp overlap the MMAs instead of queueing behind them).
 //   warps 4-11 epilogue, two groups working on the two column halves at
-//           once: tcgen05.ld accumulator and low-rank half, combine, store
-//           Y once.
+//           once: tcgen05.ld accumulator and low-rank half into registers,
+//           release tensor memory, combine, stage and store Y once.
 // TMEM columns: [0,256) accumulator, [256,384) low-rank half 0, [384,512)
 // the scale ring (per slot: A 16 columns, B 32 columns) during the mainloop
 // and low-rank half 1 after it.
