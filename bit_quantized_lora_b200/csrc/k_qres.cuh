@@ -22,17 +22,19 @@
 //            block is encoded from shared memory with the block maxima kept
 //            in registers since phase 1; codes and scales are staged in
 //            shared memory and leave in coalesced 16-byte / 4-byte stores.
-//   tail     TMEM (lane = token, column = P column) -> FP32 split partials;
-//            the last CTA of a row tile adds the splits in split order and
-//            rounds P = [bf16(T L1) | bf16(s T L2)].
+//   P        as soon as the accumulator is complete (during the barrier),
+//            four helper warps move TMEM (lane = token, column = P column)
+//            to FP32 split partials; in the last CTA of a row tile they add
+//            the splits in split order and round P = [bf16(T L1) |
+//            bf16(s T L2)] while the quantizer warps are still encoding.
 //
 // Codes and scales follow the encoding of every other quantizer here, bit
 // for bit; P follows k_qdown's rounding (FP32 accumulation, one rounding).
 //
 // CTA = 128 rows x one C-range of at most 768 columns (12 stages of 64);
-// warps: 0 TMA producer, 1 TMEM owner + UMMA issuer, 2-17 quantizers (thread
-// t owns row t % 128 and block t / 128 of every 64-column stage) and then
-// the epilogue.
+// warps: 0 TMA producer, 1 TMEM owner + UMMA issuer, 0-3 then the P path
+// (one TMEM lane quarter each), 4-19 quantizers (thread t owns row t % 128
+// and block t / 128 of every 64-column stage) and then the outputs.
 #pragma once
 
 #include <cuda.h>
@@ -49,7 +51,9 @@ constexpr int MAX_FS = 8;        // factor-ring stages
 constexpr int MAX_SPLITS = 8;    // C-splits of one row tile
 constexpr int NQ_WARPS = 16;
 constexpr int NQ_THREADS = NQ_WARPS * 32;
-constexpr int NUM_THREADS = 64 + NQ_THREADS;
+constexpr int NH_WARPS = 4;      // producer, MMA issuer and two more: the P path
+constexpr int NH_THREADS = NH_WARPS * 32;
+constexpr int NUM_THREADS = NH_THREADS + NQ_THREADS;
 constexpr int TILE_BYTES = BM * BKC * 2;  // 16 KiB
 constexpr uint32_t TMEM_COLS = 128;
 // staged scale bytes per row: MAX_ST words plus one, so that the byte
@@ -162,26 +166,27 @@ __device__ __forceinline__ void mma_factor(uint32_t tmem_d, uint32_t a_tile, uin
                   smem_desc(b + 2 * f.sbo * j, 8192, f.sbo, f.swz), idesc, (!first || j) ? 1u : 0u);
 }
 
-// P rows of one row tile from the splits' FP32 partials: every split's
-// loads of UNR float4s are issued before the first add (one L2 round trip per
-// pass instead of one per split), then the adds run in split order.
+// P rows of one row tile from the splits' FP32 partials, by threads
+// tid = 0 .. NH_THREADS - 1: every split's loads of UNR float4s are issued
+// before the first add (one L2 round trip per pass instead of one per
+// split), then the adds run in split order.
 template <int MAXS, int UNR>
 __device__ __forceinline__ void reduce_splits(const Params& p, const float4* part4, int64_t stride4, int n4,
-                                              int m0) {
-    for (int i0 = threadIdx.x; i0 < n4; i0 += UNR * NUM_THREADS) {
+                                              int m0, int tid) {
+    for (int i0 = tid; i0 < n4; i0 += UNR * NH_THREADS) {
         float4 v[UNR][MAXS];
 #pragma unroll
         for (int k = 0; k < MAXS; ++k) {
 #pragma unroll
             for (int u = 0; u < UNR; ++u) {
-                const int i = i0 + u * NUM_THREADS;
+                const int i = i0 + u * NH_THREADS;
                 v[u][k] = (k < p.splits && i < n4) ? __ldcg(part4 + k * stride4 + i)
                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
 #pragma unroll
         for (int u = 0; u < UNR; ++u) {
-            const int i = i0 + u * NUM_THREADS;
+            const int i = i0 + u * NH_THREADS;
             if (i >= n4) continue;
             float4 acc = v[u][0];
 #pragma unroll
@@ -256,75 +261,126 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
     grid_dep_wait();
     grid_dep_launch();
 
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer
-        if (lane == 0) {
-            // the first ring stages of factor tiles (small) ahead of the
-            // chunk, so the down-projection starts with the first chunk stage
-            const int pre = p.do_mma ? min(FS, nst) : 0;
-            for (int st = 0; st < pre; ++st) {
-                uint64_t* fb = &bars[QB_FFULL + st];
-                mbar_arrive_expect_tx(fb, p.fstage_bytes);
-                uint8_t* dst = smem + L.f + st * p.fstage_bytes;
-                if (p.f1.rf > 0) load_factor(dst, p.f1, &p.mapL1, fb, c0 + st * BKC);
-                if (p.f2.rf > 0) load_factor(dst, p.f2, &p.mapL2, fb, c0 + st * BKC);
+    if (warp < NH_WARPS) {
+        if (warp == 0) {
+            // ------------------------------------------------ TMA producer
+            if (lane == 0) {
+                // the first ring stages of factor tiles (small) ahead of the
+                // chunk, so the down-projection starts with the first chunk stage
+                const int pre = p.do_mma ? min(FS, nst) : 0;
+                for (int st = 0; st < pre; ++st) {
+                    uint64_t* fb = &bars[QB_FFULL + st];
+                    mbar_arrive_expect_tx(fb, p.fstage_bytes);
+                    uint8_t* dst = smem + L.f + st * p.fstage_bytes;
+                    if (p.f1.rf > 0) load_factor(dst, p.f1, &p.mapL1, fb, c0 + st * BKC);
+                    if (p.f2.rf > 0) load_factor(dst, p.f2, &p.mapL2, fb, c0 + st * BKC);
+                }
+                // the whole chunk at once: it stays resident
+                for (int st = 0; st < nst; ++st) {
+                    mbar_arrive_expect_tx(&bars[QB_XFULL + st], TILE_BYTES);
+                    tma_load_2d(smem + L.x + st * TILE_BYTES, &p.mapT, &bars[QB_XFULL + st], c0 + st * BKC, m0);
+                }
+                int st = pre;
+                if (p.do_mma) {
+                    for (; st < nst; ++st) {
+                        const int f = st % FS;
+                        const uint32_t ph = (st / FS) & 1;
+                        if (!mbar_wait(&bars[QB_FEMPTY + f], ph ^ 1, ERR_WAIT_EMPTY, abort_flag)) break;
+                        uint64_t* fb = &bars[QB_FFULL + f];
+                        mbar_arrive_expect_tx(fb, p.fstage_bytes);
+                        uint8_t* dst = smem + L.f + f * p.fstage_bytes;
+                        const int c = c0 + st * BKC;
+                        if (p.f1.rf > 0) load_factor(dst, p.f1, &p.mapL1, fb, c);
+                        if (p.f2.rf > 0) load_factor(dst, p.f2, &p.mapL2, fb, c);
+                    }
+                }
+                if (*abort_flag) {
+                    // every copy issued lands before the CTA may exit
+                    for (int s2 = 0; s2 < nst; ++s2) drain_wait(&bars[QB_XFULL + s2], 0);
+                    for (int d = 0; d < FS && d < st; ++d) {
+                        const int j = st - 1 - d;
+                        drain_wait(&bars[QB_FFULL + j % FS], (j / FS) & 1);
+                    }
+                }
             }
-            // the whole chunk at once: it stays resident
-            for (int st = 0; st < nst; ++st) {
-                mbar_arrive_expect_tx(&bars[QB_XFULL + st], TILE_BYTES);
-                tma_load_2d(smem + L.x + st * TILE_BYTES, &p.mapT, &bars[QB_XFULL + st], c0 + st * BKC, m0);
-            }
-            int st = pre;
-            if (p.do_mma) {
-                for (; st < nst; ++st) {
+        } else if (warp == 1) {
+            // ------------------------------------------------ UMMA issuer
+            if (lane == 0 && p.do_mma) {
+                bool ok = true;
+                for (int st = 0; st < nst; ++st) {
                     const int f = st % FS;
                     const uint32_t ph = (st / FS) & 1;
-                    if (!mbar_wait(&bars[QB_FEMPTY + f], ph ^ 1, ERR_WAIT_EMPTY, abort_flag)) break;
-                    uint64_t* fb = &bars[QB_FFULL + f];
-                    mbar_arrive_expect_tx(fb, p.fstage_bytes);
-                    uint8_t* dst = smem + L.f + f * p.fstage_bytes;
-                    const int c = c0 + st * BKC;
-                    if (p.f1.rf > 0) load_factor(dst, p.f1, &p.mapL1, fb, c);
-                    if (p.f2.rf > 0) load_factor(dst, p.f2, &p.mapL2, fb, c);
+                    if (!mbar_wait(&bars[QB_XFULL + st], 0, ERR_WAIT_FULL, abort_flag) ||
+                        !mbar_wait(&bars[QB_FFULL + f], ph, ERR_WAIT_FULL, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a = base + L.x + st * TILE_BYTES;
+                    const uint32_t b = base + L.f + f * p.fstage_bytes;
+                    if (p.f1.rf > 0) mma_factor(tmem, a, b, p.f1, st == 0);
+                    if (p.f2.rf > 0) mma_factor(tmem + (uint32_t)p.r1, a, b, p.f2, st == 0);
+                    tc_commit(&bars[QB_FEMPTY + f]);
+                    tc_commit(&bars[QB_XDONE + st]);
                 }
+                if (ok) tc_commit(&bars[QB_ACC]);
+                tc_commit(&bars[QB_DRAIN]);
+                drain_wait(&bars[QB_DRAIN], 0);
             }
-            if (*abort_flag) {
-                // every copy issued lands before the CTA may exit
-                for (int s2 = 0; s2 < nst; ++s2) drain_wait(&bars[QB_XFULL + s2], 0);
-                for (int d = 0; d < FS && d < st; ++d) {
-                    const int j = st - 1 - d;
-                    drain_wait(&bars[QB_FFULL + j % FS], (j / FS) & 1);
-                }
-            }
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------ UMMA issuer
-        if (lane == 0 && p.do_mma) {
-            bool ok = true;
-            for (int st = 0; st < nst; ++st) {
-                const int f = st % FS;
-                const uint32_t ph = (st / FS) & 1;
-                if (!mbar_wait(&bars[QB_XFULL + st], 0, ERR_WAIT_FULL, abort_flag) ||
-                    !mbar_wait(&bars[QB_FFULL + f], ph, ERR_WAIT_FULL, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t a = base + L.x + st * TILE_BYTES;
-                const uint32_t b = base + L.f + f * p.fstage_bytes;
-                if (p.f1.rf > 0) mma_factor(tmem, a, b, p.f1, st == 0);
-                if (p.f2.rf > 0) mma_factor(tmem + (uint32_t)p.r1, a, b, p.f2, st == 0);
-                tc_commit(&bars[QB_FEMPTY + f]);
-                tc_commit(&bars[QB_XDONE + st]);
-            }
-            if (ok) tc_commit(&bars[QB_ACC]);
-            tc_commit(&bars[QB_DRAIN]);
-            drain_wait(&bars[QB_DRAIN], 0);
         }
         __syncwarp();
+
+        // ------------------------------------------------ P path
+        // Warp w holds TMEM lanes 32w .. 32w + 31 (token rows).  The split
+        // partial leaves as soon as the MMAs are done, which is during the
+        // grid barrier; the last CTA of the row tile then adds the splits
+        // while its quantizer warps encode.
+        if (p.do_mma) {
+            if (__all_sync(0xFFFFFFFFu, mbar_wait(&bars[QB_ACC], 0, ERR_WAIT_ACC_FULL, abort_flag))) {
+                tc_fence_after();
+                const int m = m0 + 32 * warp + lane;
+                const uint32_t lane_addr = (uint32_t)(32 * warp) << 16;
+                for (int c = 0; c < p.r / 16; ++c) {
+                    uint32_t v[16];
+                    tmem_ld_32x32b_x16(tmem + lane_addr + 16 * c, v);
+                    tmem_ld_wait();
+                    if (m < p.M) {
+                        float4* o = reinterpret_cast<float4*>(p.part + ((int64_t)split * p.M + m) * p.r + 16 * c);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            o[k] = make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                                               __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
+                    }
+                }
+            }
+            __threadfence();
+            named_bar_sync(2, NH_THREADS);
+            if (threadIdx.x == 0) {
+                // the last CTA of the row tile to arrive adds the splits
+                int last = 0;
+                if (!*abort_flag) {
+                    const unsigned long long prev = epoch_count(&p.counters[blockIdx.x], p.epoch);
+                    last = (prev == (unsigned long long)(p.splits - 1)) ? 1 : 0;
+                }
+                *last_flag = last;
+            }
+            named_bar_sync(2, NH_THREADS);
+            if (*last_flag) {
+                // P = [bf16(T L1) | bf16(s T L2)], splits added in split order
+                __threadfence();
+                const int rows = min(BM, p.M - m0);
+                const int n4 = rows * p.r / 4;
+                const int64_t stride4 = (int64_t)p.M * p.r / 4;
+                const float4* part4 = reinterpret_cast<const float4*>(p.part) + (int64_t)m0 * p.r / 4;
+                if (p.splits <= 4)
+                    reduce_splits<4, 3>(p, part4, stride4, n4, m0, threadIdx.x);
+                else
+                    reduce_splits<MAX_SPLITS, 2>(p, part4, stride4, n4, m0, threadIdx.x);
+            }
+        }
     } else {
         // ------------------------------------------------ quantizers
-        const int t = threadIdx.x - 64;
+        const int t = threadIdx.x - NH_THREADS;
         const int trow = t & (BM - 1), blk = t >> 7;
         const uint32_t sw = (uint32_t)(trow & 7);
         const uint32_t off_lo = (uint32_t)trow * 128u + (((uint32_t)(2 * blk) ^ sw) << 4);
@@ -353,7 +409,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
         // tensor amax: CTA max, then the grid-wide max (or the caller's value)
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) cmax = max(cmax, __shfl_xor_sync(0xFFFFFFFFu, cmax, o));
-        if (lane == 0) red[warp - 2] = cmax;
+        if (lane == 0) red[warp - NH_WARPS] = cmax;
         named_bar_sync(1, NQ_THREADS);
         if (t == 0) {
             float amax_t;
@@ -426,12 +482,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
         named_bar_sync(1, NQ_THREADS);
         ok = ok && !*abort_flag;
 
-        // With the down-projections, warps 2-5 (one per TMEM lane quarter)
-        // take the epilogue while the other twelve write the outputs.
-        const bool epi_warp = p.do_mma && warp < 6;
-        if (ok && !epi_warp) {
-            const int ot = p.do_mma ? t - 128 : t;
-            const int on = p.do_mma ? NQ_THREADS - 128 : NQ_THREADS;
+        if (ok) {
+            const int ot = t, on = NQ_THREADS;
             const int rows = min(BM, p.M - m0);
             // codes: 8-byte pieces (one block), a warp on 8 rows x the 4
             // blocks of one stage: the pieces sit at the start of 16-byte
@@ -469,41 +521,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
                 }
             }
         }
-
-        // epilogue: TMEM lane = token row, column = P column.  The partials
-        // are published (a fence, then one arrival on the row tile's
-        // counter) while the other warps are still writing codes and scales.
-        if (epi_warp) {
-            if (ok && __all_sync(0xFFFFFFFFu, mbar_wait(&bars[QB_ACC], 0, ERR_WAIT_ACC_FULL, abort_flag))) {
-                tc_fence_after();
-                const int sp = warp & 3;
-                const int m = m0 + 32 * sp + lane;
-                const uint32_t lane_addr = (uint32_t)(32 * sp) << 16;
-                for (int c = 0; c < p.r / 16; ++c) {
-                    uint32_t v[16];
-                    tmem_ld_32x32b_x16(tmem + lane_addr + 16 * c, v);
-                    tmem_ld_wait();
-                    if (m < p.M) {
-                        float4* o = reinterpret_cast<float4*>(p.part + ((int64_t)split * p.M + m) * p.r + 16 * c);
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            o[k] = make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
-                                               __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
-                    }
-                }
-            }
-            __threadfence();
-            named_bar_sync(2, 128);
-            if (warp == 2 && lane == 0) {
-                // the last CTA of the row tile to arrive adds the splits
-                int last = 0;
-                if (!*abort_flag) {
-                    const unsigned long long prev = epoch_count(&p.counters[blockIdx.x], p.epoch);
-                    last = (prev == (unsigned long long)(p.splits - 1)) ? 1 : 0;
-                }
-                *last_flag = last;
-            }
-        }
     }
     tc_fence_before();
     __syncthreads();
@@ -511,22 +528,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
-    if (!p.do_mma || *abort_flag || !*last_flag) {
-        signal_done(p);
-        return;
-    }
-
-    // The last CTA of this row tile adds the splits' partials in split order
-    // (deterministic) and rounds P = [bf16(T L1) | bf16(s T L2)].
-    __threadfence();
-    const int rows = min(BM, p.M - m0);
-    const int n4 = rows * p.r / 4;
-    const int64_t stride4 = (int64_t)p.M * p.r / 4;
-    const float4* part4 = reinterpret_cast<const float4*>(p.part) + (int64_t)m0 * p.r / 4;
-    if (p.splits <= 4)
-        reduce_splits<4, 3>(p, part4, stride4, n4, m0);
-    else
-        reduce_splits<MAX_SPLITS, 2>(p, part4, stride4, n4, m0);
     signal_done(p);
 }
 
