@@ -428,21 +428,29 @@ ft_status run_qdown(const void* T, int64_t M, int64_t C, const void* L1, int64_t
     return last_launch();
 }
 
-// Factor tile of the resident quantizer for a rank rf: boxes of 16, 32 or
-// 64 columns (swizzle = the box's row bytes), two 64-wide atoms above 64.
+// Factor tile of the resident quantizer for a rank rf (a multiple of 16):
+// rf / 16 atoms of 16 columns x 64 rows.
 ft::qres::Factor qres_factor(int64_t rf) {
     ft::qres::Factor f;
     std::memset(&f, 0, sizeof(f));
-    f.rf = (int)rf;
-    if (rf <= 0) return f;
-    f.wbox = rf <= 16 ? 16 : rf <= 32 ? 32 : 64;
-    f.natoms = rf <= 64 ? 1 : 2;
-    f.sbo = 8u * (uint32_t)f.wbox * 2u;
-    f.swz = f.wbox == 16 ? ft::SWZ_32B : f.wbox == 32 ? ft::SWZ_64B : ft::SWZ_128B;
+    f.rf = (int)std::max<int64_t>(rf, 0);
     return f;
 }
 uint32_t qres_factor_bytes(const ft::qres::Factor& f) {
-    return f.rf > 0 ? (uint32_t)f.natoms * 64u * (uint32_t)f.wbox * 2u : 0u;
+    return (uint32_t)(f.rf / 16) * ft::qres::ATOM_BYTES;
+}
+
+// L [C, rf] row-major as the 3-D tensor {16, C, rf / 16} (16-column atoms as
+// the outer dimension), boxes {16, 64, rf / 16}: a stage's atoms in one copy.
+ft_status encode_factor_atoms(CUtensorMap* m, const void* L, int64_t C, int64_t rf) {
+    cuuint64_t dims[3] = {16, (cuuint64_t)C, (cuuint64_t)(rf / 16)};
+    cuuint64_t strides[2] = {(cuuint64_t)(rf * 2), 32};
+    cuuint32_t box[3] = {16, 64, (cuuint32_t)(rf / 16)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(L), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FT_OK : FT_ERR_CUDA;
 }
 
 // Ring of factor tiles: as many stages of both tiles as fit in 31 KiB (the
@@ -538,14 +546,8 @@ ft_status run_quant_down(const void* T, int64_t M, int64_t C, const void* L1, in
         }
         return run_qdown(T, M, C, L1, r1, L2, r2, s, a, codes, scales, tscale, P, ws, w, d, st);
     }
-    const CUtensorMapSwizzle swz[3] = {CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_SWIZZLE_64B,
-                                       CU_TENSOR_MAP_SWIZZLE_128B};
-    if (r1 > 0)
-        FT_TRY(encode_2d(&p.mapL1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1, r1, C, r1 * 2, p.f1.wbox, 64,
-                         swz[p.f1.wbox == 16 ? 0 : p.f1.wbox == 32 ? 1 : 2]));
-    if (r2 > 0)
-        FT_TRY(encode_2d(&p.mapL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2, r2, C, r2 * 2, p.f2.wbox, 64,
-                         swz[p.f2.wbox == 16 ? 0 : p.f2.wbox == 32 ? 1 : 2]));
+    if (r1 > 0) FT_TRY(encode_factor_atoms(&p.mapL1, L1, C, r1));
+    if (r2 > 0) FT_TRY(encode_factor_atoms(&p.mapL2, L2, C, r2));
     FT_TRY(encode_2d(&p.mapT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, C, M, C * 2, 64, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B));
     p.amax_in = amax_in;

@@ -11,8 +11,9 @@
 //            quantizer warps take every 1x16 block's max|x| as its stage
 //            lands; meanwhile the MMA warp runs the down-projections
 //            D[m, j] = sum_c T[m, c] L[c, j] on tcgen05 (kind::f16): A = the
-//            same swizzled T tiles (K-major), B = L1 and L2 as they lie in
-//            HBM (MN-major, swizzled to their width), streamed through a ring.
+//            same swizzled T tiles (K-major), B = [L1 | L2] as they lie in
+//            HBM (MN-major), streamed through a ring: one MMA of N = r per
+//            K = 16 step.
 //   barrier  the CTA's max is folded into one global word (an integer max on
 //            the float bits: exact, order-free); a grid-wide arrival counter
 //            (cooperative launch: every CTA is resident) releases all CTAs
@@ -62,22 +63,20 @@ constexpr uint32_t SROW = MAX_ST * 4 + 4;
 constexpr uint32_t BAR_BYTES = 512;
 constexpr uint32_t SMEM_LIMIT = 227u * 1024u;
 
-// One low-rank factor L [C, rf] read as the MN-major B operand: boxes of
-// `wbox` rank columns x 64 rows of c, swizzled to the box's row bytes
-// (32, 64 or 128), `natoms` boxes side by side (rf > 64: two 64-wide atoms).
+// One low-rank factor L [C, rf] in a ring stage: rf / 16 atoms of 16 rank
+// columns x 64 rows of c (32-byte rows, 32-byte swizzle, 2 KiB each), one
+// 3-D box per stage.  The second factor's atoms follow the first's, so the
+// stage is one MN-major B operand [64, r] whose atoms are ATOM_BYTES apart.
 struct Factor {
     int rf;          // rank (0: absent)
-    int wbox;        // 16, 32 or 64 columns per box
-    int natoms;      // 1 or 2
-    uint32_t off;    // byte offset of its tile inside a ring stage
-    uint32_t sbo;    // bytes between 8-row groups (8 * wbox * 2)
-    uint32_t swz;    // descriptor swizzle code
+    uint32_t off;    // byte offset of its atoms inside a ring stage
 };
+constexpr uint32_t ATOM_BYTES = 64 * 16 * 2;
 
 struct Params {
     CUtensorMap mapT;   // bf16 [M, C], box {64, 128}, 128 B swizzle
-    CUtensorMap mapL1;  // bf16 [C, r1], box {wbox1, 64}
-    CUtensorMap mapL2;  // bf16 [C, r2], box {wbox2, 64}
+    CUtensorMap mapL1;  // bf16 [C, r1] as {16, C, r1 / 16}, box {16, 64, r1 / 16}, 32 B swizzle
+    CUtensorMap mapL2;  // bf16 [C, r2] likewise
     const float* amax_in;      // caller's tensor amax, or null (computed here)
     // epoch-tagged words (any earlier content is fine): [0] grid-barrier
     // arrivals, [1] tensor amax as (epoch << 31) | bits, [2] finished CTAs
@@ -147,23 +146,10 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     mbar_wait(bar, parity, ERR_WAIT_DRAIN, &no_abort);
 }
 
-// TMA loads of one factor's tile for rows c .. c+63.
+// TMA load of one factor's atoms for rows c .. c+63 (one 3-D box).
 __device__ __forceinline__ void load_factor(uint8_t* stage, const Factor& f, const CUtensorMap* map,
                                             uint64_t* bar, int c) {
-    for (int a = 0; a < f.natoms; ++a)
-        tma_load_2d(stage + f.off + a * 8192, map, bar, 64 * a, c);
-}
-
-// The four K = 16 MMAs of one 64-column stage for one factor:
-// D[:, col0 .. col0 + rf) (+)= T_tile (K-major) x L_tile (MN-major).
-__device__ __forceinline__ void mma_factor(uint32_t tmem_d, uint32_t a_tile, uint32_t b_stage,
-                                           const Factor& f, bool first) {
-    const uint32_t idesc = idesc_bf16(128, f.rf, 0, 1);
-    const uint32_t b = b_stage + f.off;
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-        umma_bf16(tmem_d, desc_kmajor_sw128(a_tile + 32 * j),
-                  smem_desc(b + 2 * f.sbo * j, 8192, f.sbo, f.swz), idesc, (!first || j) ? 1u : 0u);
+    tma_load_3d(stage + f.off, map, bar, 0, c, 0);
 }
 
 // P rows of one row tile from the splits' FP32 partials, by threads
@@ -306,6 +292,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
         } else if (warp == 1) {
             // ------------------------------------------------ UMMA issuer
             if (lane == 0 && p.do_mma) {
+                // D[:, 0 .. r) (+)= T_tile[:, 16 j ..) (K-major, 128-byte
+                // swizzle) x [L1 | L2][16 j .., :) (MN-major 16-column atoms,
+                // 32-byte swizzle).  Descriptor words built once: lo = start
+                // >> 4 | (LBO >> 4) << 16, hi = SBO >> 4 | version 1 << 14 |
+                // swizzle << 29; a K step adds 32 bytes (A) or 16 rows (B).
+                const uint32_t idesc = idesc_bf16(128, p.r, 0, 1);
+                const uint32_t a_hi = (1024u >> 4) | (1u << 14) | (SWZ_128B << 29);
+                const uint32_t b_hi = (256u >> 4) | (1u << 14) | (SWZ_32B << 29);
+                const uint32_t a_lo0 = ((base + L.x) >> 4) | (1u << 16);
+                const uint32_t b_lo0 = ((base + L.f) >> 4) | ((ATOM_BYTES >> 4) << 16);
                 bool ok = true;
                 for (int st = 0; st < nst; ++st) {
                     const int f = st % FS;
@@ -316,10 +312,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a = base + L.x + st * TILE_BYTES;
-                    const uint32_t b = base + L.f + f * p.fstage_bytes;
-                    if (p.f1.rf > 0) mma_factor(tmem, a, b, p.f1, st == 0);
-                    if (p.f2.rf > 0) mma_factor(tmem + (uint32_t)p.r1, a, b, p.f2, st == 0);
+                    const uint32_t a_lo = a_lo0 + (uint32_t)st * (TILE_BYTES >> 4);
+                    const uint32_t b_lo = b_lo0 + (uint32_t)f * (p.fstage_bytes >> 4);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        umma_bf16(tmem, make_desc(a_lo + 2 * j, a_hi), make_desc(b_lo + 32 * j, b_hi), idesc,
+                                  (st | j) != 0);
                     tc_commit(&bars[QB_FEMPTY + f]);
                     tc_commit(&bars[QB_XDONE + st]);
                 }
