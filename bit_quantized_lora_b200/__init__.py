@@ -27,7 +27,7 @@ __all__ = [
     "FP4", "Layer", "FtError", "BLK_1x16", "BLK_16x16", "BF16", "F32",
     "ft_quantize", "ft_quantize_transpose", "ft_linear_fwd", "ft_linear_bwd",
     "ft_workspace_bytes", "ft_quantize_workspace_bytes", "ft_device_error",
-    "prepare_layer", "svd_split", "Workspace", "timing",
+    "ft_set_cooperative_quantizer", "prepare_layer", "svd_split", "Workspace", "timing",
 ]
 
 
@@ -279,6 +279,13 @@ def ft_device_error(stream=None) -> int:
     code = ctypes.c_int(0)
     load().ft_device_error(ctypes.byref(code), _stream(stream))
     return code.value
+
+
+def ft_set_cooperative_quantizer(on: bool) -> None:
+    """Launch mode of the single-pass quantizer's grid barrier: False (the
+    default) = plain launch, True = cooperative launch (safe next to other
+    streams' long-running kernels, ~3 us later start per call)."""
+    check("ft_set_cooperative_quantizer", load().ft_set_cooperative_quantizer(1 if on else 0))
 
 
 class timing:

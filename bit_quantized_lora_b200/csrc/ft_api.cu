@@ -491,8 +491,14 @@ int qres_max_stages(uint32_t ring_bytes) {
     return (int)std::min<int64_t>(Q::MAX_ST, std::max<int64_t>(0, avail / Q::TILE_BYTES));
 }
 
-// Launches k_qres; cooperative (all CTAs co-resident) when it computes the
-// tensor amax itself, since its grid barrier waits on every CTA.
+// Launch mode of k_qres when it computes the tensor amax (its grid barrier
+// waits on every CTA): 0 = plain launch (every CTA resident once the
+// previous kernel ends, the grid being at most one CTA per SM), 1 =
+// cooperative.  See ft_set_cooperative_quantizer.
+std::atomic<int> g_qres_cooperative{0};
+
+// Launches k_qres with programmatic stream serialization; cooperative when
+// requested and the kernel computes the tensor amax itself.
 ft_status launch_qres(const ft::qres::Params& p, int mt, int splits, cudaStream_t st) {
     namespace Q = ft::qres;
     cudaLaunchConfig_t cfg;
@@ -502,15 +508,14 @@ ft_status launch_qres(const ft::qres::Params& p, int mt, int splits, cudaStream_
     cfg.dynamicSmemBytes = Q::make_layout(p.cchunk / Q::BKC, p.ring_bytes).total;
     cfg.stream = st;
     // it may start its setup while the previous kernel finishes (it waits
-    // for that kernel's results on the device); cooperative when its grid
-    // barrier must see every CTA resident
+    // for that kernel's results on the device)
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     attr[1].id = cudaLaunchAttributeCooperative;
     attr[1].val.cooperative = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = p.amax_in ? 1 : 2;
+    cfg.numAttrs = (!p.amax_in && g_qres_cooperative.load(std::memory_order_relaxed)) ? 2 : 1;
     {
         LaunchTimer _lt(KID_QRES, st);
         FT_TRY(cuda_ok(cudaLaunchKernelEx(&cfg, Q::k_qres, p)));
@@ -826,6 +831,11 @@ ft_status ft_workspace_qact(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_
     *codes_off = w.codes;
     *scales_off = w.scales;
     *tscale_off = w.gact;
+    return FT_OK;
+}
+
+ft_status ft_set_cooperative_quantizer(int on) {
+    g_qres_cooperative.store(on ? 1 : 0, std::memory_order_relaxed);
     return FT_OK;
 }
 

@@ -157,14 +157,18 @@ static_assert(B_COUNT * 8 + 8 <= 256, "barrier area");
 
 // The K = 16 MMAs of one factor's up-projection for output rows
 // [128 h, 128 h + 128) of the tile: D (+)= P_f x L_f[half h]^T.
+// Descriptor words are built once per call (lo = start >> 4 | 1 << 16,
+// hi = SBO >> 4 | version 1 << 14 | swizzle << 29); a K step adds 32 bytes
+// inside an atom, the second 64-wide atom (rf > 64) starts a panel later.
 __device__ __forceinline__ void lr_mma(uint32_t tmem_d, uint32_t pa, uint32_t pb, const LrFactor& f, int h,
                                        uint32_t idesc, int& q) {
-    const uint32_t sbo = 8u * f.row_bytes;
+    const uint32_t hi = ((8u * f.row_bytes) >> 4) | (1u << 14) | (f.swz << 29);
+    const uint32_t a_lo = (pa >> 4) | (1u << 16);
+    const uint32_t b_lo = ((pb + (uint32_t)h * 128u * f.row_bytes) >> 4) | (1u << 16);
+    const uint32_t a_atom = (128u * f.row_bytes) >> 4, b_atom = (256u * f.row_bytes) >> 4;
     for (int j = 0; j < f.rf; j += 16, ++q) {
-        const uint32_t a = (uint32_t)(j / 64), k = (uint32_t)(j % f.wbox) * 2u;
-        const uint32_t ao = a * 128u * f.row_bytes + k;
-        const uint32_t bo = a * 256u * f.row_bytes + (uint32_t)h * 128u * f.row_bytes + k;
-        umma_bf16(tmem_d, smem_desc(pa + ao, 16, sbo, f.swz), smem_desc(pb + bo, 16, sbo, f.swz), idesc,
+        const uint32_t a = (uint32_t)(j >> 6), k = ((uint32_t)(j & (f.wbox - 1)) * 2u) >> 4;
+        umma_bf16(tmem_d, make_desc(a_lo + a * a_atom + k, hi), make_desc(b_lo + a * b_atom + k, hi), idesc,
                   q != 0);
     }
 }

@@ -166,6 +166,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_lora_grad(const __grid_const
             // A = T^T (M = 128 columns c, MN-major: two 64-wide swizzle atoms
             // 8 KiB apart), B = S (N = n_pad, MN-major), K = 16 token rows.
             const uint32_t idesc = idesc_bf16(BC, p.n_pad, 1, 1);
+            // descriptor words built once (lo = start >> 4 | (LBO >> 4) << 16,
+            // hi = SBO >> 4 | version 1 << 14 | swizzle << 29): atoms / boxes
+            // LBO apart, 8-row groups 1 KiB apart; a K step is 16 rows (2 KiB)
+            const uint32_t hi = (1024u >> 4) | (1u << 14) | (SWZ_128B << 29);
+            const uint32_t a_lo0 = ((base + off_t) >> 4) | ((uint32_t)((T_BYTES / 2) >> 4) << 16);
+            const uint32_t b_lo0 = ((base + off_s) >> 4) | ((uint32_t)(S_CHUNK >> 4) << 16);
             bool ok = true;
             for (int st = 0; st < nst; ++st) {
                 const int s = st % STAGES;
@@ -175,12 +181,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_lora_grad(const __grid_const
                     break;
                 }
                 tc_fence_after();
-                const uint32_t a = base + off_t + s * T_BYTES;
-                const uint32_t b = base + off_s + s * s_bytes;
+                const uint32_t a_lo = a_lo0 + (uint32_t)s * (T_BYTES >> 4);
+                const uint32_t b_lo = b_lo0 + (uint32_t)s * (s_bytes >> 4);
 #pragma unroll
                 for (int k = 0; k < BMR / 16; ++k)
-                    umma_bf16(tmem, smem_desc(a + 2048 * k, T_BYTES / 2, 1024, SWZ_128B),
-                              smem_desc(b + 2048 * k, S_CHUNK, 1024, SWZ_128B), idesc, (st | k) != 0);
+                    umma_bf16(tmem, make_desc(a_lo + 128 * k, hi), make_desc(b_lo + 128 * k, hi), idesc,
+                              (st | k) != 0);
                 tc_commit(&empty[s]);
             }
             if (ok && nst > 0) tc_commit(accfull);

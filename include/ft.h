@@ -216,6 +216,25 @@ ft_status ft_workspace_qact(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_
  * FT_ERR_TIMEOUT when *code != 0.                                          */
 ft_status ft_device_error(int* code, void* stream);
 
+/* ft_set_cooperative_quantizer -- launch mode of the single-pass quantizer
+ * (the kernel that keeps the whole activation in shared memory and finds
+ * the tensor amax through a grid-wide barrier, section 3.3's fused down
+ * side).  Its barrier needs every CTA of its grid resident at once; the grid
+ * never has more CTAs than the device holds at once (one per SM).
+ *   on = 0 (the default): a plain launch with programmatic stream
+ *     serialization.  Its CTAs take SMs as the previous kernel's CTAs
+ *     retire and wait on the device for that kernel's results; all of them
+ *     are resident once it ends, unless a kernel of another stream or
+ *     process keeps SMs busy meanwhile.  If that lasts longer than the
+ *     barrier's wait limit (1 s) the call's results are invalid and
+ *     ft_device_error() reports the timeout (code 8); nothing hangs.
+ *   on = 1: a cooperative launch: the driver starts the grid only when all
+ *     of its CTAs fit at once, which is safe next to other streams' kernels
+ *     but starts it only after the previous kernel has fully ended (about
+ *     3 us later per call on a B200).
+ * Process-wide, for calls made after it returns.  Host-only; always FT_OK. */
+ft_status ft_set_cooperative_quantizer(int on);
+
 /* Human-readable name of a status. */
 const char* ft_status_str(ft_status s);
 

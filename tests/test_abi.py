@@ -153,3 +153,13 @@ def test_weight_operand_packing_validation(L):
     assert L.ft_pack_weight_operands(g, g, g, 320, 256, g, g, None) == FT_ERR_SHAPE
     assert L.ft_pack_weight_operands(g, g, g, 256, 256, g + 8, g, None) == FT_ERR_ALIGN
     assert L.ft_pack_weight_operands(g, g, g, 0, 256, g, g, None) == FT_OK
+
+
+def test_cooperative_quantizer_switch_is_host_only(L):
+    """The launch-mode switch touches no device: it answers FT_OK on a host
+    without a GPU and accepts any int (nonzero = cooperative)."""
+    try:
+        for on in (1, 0, 7, 0):
+            assert L.ft_set_cooperative_quantizer(on) == 0
+    finally:
+        L.ft_set_cooperative_quantizer(0)

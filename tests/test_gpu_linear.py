@@ -252,3 +252,26 @@ def test_foreign_sync_words_time_out_then_zeroing_recovers():
     torch.cuda.synchronize()
     assert ft.ft_device_error() == 0
     assert torch.equal(Y0, Y1) and torch.equal(P0, P1)
+
+
+def test_cooperative_and_plain_quantizer_launches_agree():
+    """The single-pass quantizer's grid barrier works under both launch
+    modes: a plain launch (the default; its CTAs start as the previous
+    kernel's CTAs retire) and a cooperative one.  Both compute the same
+    bytes, so forward and backward outputs agree bit for bit."""
+    inp, U, V, Wr, layer = _prep(ft_synth.ATTN, 23)
+    X, dY = dev_bf16(inp["X"]), dev_bf16(inp["dY"])
+    outs = []
+    try:
+        for coop in (False, True, False):
+            ft.ft_set_cooperative_quantizer(coop)
+            Y, P = ft.ft_linear_fwd(layer, X, out_dtype=ft.F32)
+            dX, dA, dB = ft.ft_linear_bwd(layer, dY, X, P, out_dtype=ft.F32)
+            torch.cuda.synchronize()
+            assert ft.ft_device_error() == 0
+            outs.append([t.clone() for t in (Y, P, dX, dA, dB)])
+    finally:
+        ft.ft_set_cooperative_quantizer(False)
+    for o in outs[1:]:
+        for a, b in zip(o, outs[0]):
+            assert torch.equal(a, b)
