@@ -350,12 +350,10 @@ __device__ __forceinline__ void build_qtable_m1(QTableM& tab, float g, int tid, 
 }
 
 // Step 2: the exactness check of the multiply path, for each candidate
-// multiplier, four threads per scale byte (boundaries k = part, part + 4),
-// over the scale bytes s_lo .. s_hi that the caller's blocks can take.
-__device__ __forceinline__ void build_qtable_m2(QTableM& tab, int tid, int nthreads, int s_lo, int s_hi) {
-    const int ns = s_hi - s_lo + 1;
-    for (int i = tid; i < QT_NY * 4 * ns; i += nthreads) {
-        const int j = i / (4 * ns), rest = i - j * 4 * ns, part = rest / ns, s = s_lo + (rest - part * ns);
+// multiplier, four threads per scale byte (boundaries k = part, part + 4).
+__device__ __forceinline__ void build_qtable_m2(QTableM& tab, int tid, int nthreads) {
+    for (int i = tid; i < QT_NY * 512; i += nthreads) {
+        const int j = i >> 9, s = i & 127, part = (i >> 7) & 3;
         const float d = tab.d[s], y = tab.y[s];
         if (s == 0 || s >= 0x7E || y == 0.0f) continue;  // these never take the multiply path
         const float yj = qt_multiplier(y, j);
@@ -378,12 +376,11 @@ __device__ __forceinline__ void build_qtable_m2(QTableM& tab, int tid, int nthre
     }
 }
 
-// Step 3: publish ym, the first multiplier that passed; bytes outside the
-// checked range s_lo .. s_hi get none (they would take the exact division).
-__device__ __forceinline__ void build_qtable_m3(QTableM& tab, int tid, int nthreads, int s_lo, int s_hi) {
+// Step 3: publish ym, the first multiplier that passed.
+__device__ __forceinline__ void build_qtable_m3(QTableM& tab, int tid, int nthreads) {
     for (int s = tid; s < 128; s += nthreads) {
         float ym = 0.0f;
-        if (s >= s_lo && s <= s_hi && s != 0 && s < 0x7E && tab.y[s] != 0.0f) {
+        if (s != 0 && s < 0x7E && tab.y[s] != 0.0f) {
             for (int j = QT_NY - 1; j >= 0; --j)
                 if (!((tab.bad[j][s >> 5] >> (s & 31)) & 1u)) ym = qt_multiplier(tab.y[s], j);
         }

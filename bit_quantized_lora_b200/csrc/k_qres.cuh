@@ -127,7 +127,7 @@ enum {
     QB_DRAIN,                       // every tcgen05 op of the MMA warp done
     QB_COUNT
 };
-static_assert(QB_COUNT * 8 + 16 + 8 * NQ_WARPS <= BAR_BYTES, "barrier area");
+static_assert(QB_COUNT * 8 + 16 + 4 * NQ_WARPS <= BAR_BYTES, "barrier area");
 
 // Every global write of this CTA is done: count it (release) for a kernel
 // that waits on the counter rather than on this grid's completion.
@@ -210,8 +210,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile int* last_flag = abort_flag + 1;
     volatile uint32_t* amax_share = reinterpret_cast<volatile uint32_t*>(last_flag + 1);
-    volatile uint32_t* red = amax_share + 1;  // [NQ_WARPS] block-max maxima
-    volatile uint32_t* redmin = red + NQ_WARPS;  // [NQ_WARPS] smallest nonzero block maxima
+    volatile uint32_t* red = amax_share + 1;  // [NQ_WARPS]
     QTableM& tab = *reinterpret_cast<QTableM*>(smem + L.tab);
 
     const int warp = warp_id(), lane = lane_id();
@@ -388,7 +387,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
 
         // phase 1: block maxima as the stages land (kept for phase 2)
         uint32_t mb[MAX_ST];
-        uint32_t cmax = 0, cmin = 0xFFFFFFFFu;  // largest / smallest nonzero block max (bits)
+        uint32_t cmax = 0;
 #pragma unroll
         for (int st = 0; st < MAX_ST; ++st) {
             mb[st] = 0;
@@ -401,21 +400,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
                     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
                     mb[st] = amax_bits_16(w);
                     cmax = max(cmax, mb[st]);
-                    if (mb[st]) cmin = min(cmin, mb[st]);
                 }
             }
         }
 
         // tensor amax: CTA max, then the grid-wide max (or the caller's value)
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            cmax = max(cmax, __shfl_xor_sync(0xFFFFFFFFu, cmax, o));
-            cmin = min(cmin, __shfl_xor_sync(0xFFFFFFFFu, cmin, o));
-        }
-        if (lane == 0) {
-            red[warp - NH_WARPS] = cmax;
-            redmin[warp - NH_WARPS] = cmin;
-        }
+        for (int o = 16; o > 0; o >>= 1) cmax = max(cmax, __shfl_xor_sync(0xFFFFFFFFu, cmax, o));
+        if (lane == 0) red[warp - NH_WARPS] = cmax;
         named_bar_sync(1, NQ_THREADS);
         if (t == 0) {
             float amax_t;
@@ -447,22 +439,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
         }
         named_bar_sync(1, NQ_THREADS);
         const QTensorFast qt = make_qtensor_fast(__uint_as_float(*amax_share));
-        // the scale bytes this CTA's blocks can take (monotone in the block
-        // max): only those are checked for the multiply path
-        uint32_t bmax = 0, bmin = 0xFFFFFFFFu;
-#pragma unroll
-        for (int i = 0; i < NQ_WARPS; ++i) {
-            bmax = max(bmax, red[i]);
-            bmin = min(bmin, redmin[i]);
-        }
-        const int s_hi = (int)scale_byte_fast(__uint_as_float(bmax), qt);
-        const int s_lo = bmin == 0xFFFFFFFFu ? s_hi : (int)scale_byte_fast(__uint_as_float(bmin), qt);
         build_qtable_m1(tab, qt.g, t, NQ_THREADS);
         if (blockIdx.x == 0 && blockIdx.y == 0 && t == 0) *p.tscale = qt.g;
         named_bar_sync(1, NQ_THREADS);
-        build_qtable_m2(tab, t, NQ_THREADS, s_lo, s_hi);
+        build_qtable_m2(tab, t, NQ_THREADS);
         named_bar_sync(1, NQ_THREADS);
-        build_qtable_m3(tab, t, NQ_THREADS, s_lo, s_hi);
+        build_qtable_m3(tab, t, NQ_THREADS);
         named_bar_sync(1, NQ_THREADS);
         ok = ok && !*abort_flag;
 
