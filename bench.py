@@ -24,6 +24,7 @@ import datetime
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -243,13 +244,19 @@ class ClockSampler:
         }
 
 
+_COMMENT = re.compile(r"/\*.*?\*/|//[^\n]*", re.S)
+
+
 def kernel_source_sha(name: str) -> str:
     """Hash of a kernel's source file and the device headers every kernel
-    includes, so a recorded ncu figure lapses when any of them changes."""
+    includes, comments and blank runs left out, so a recorded ncu figure
+    lapses when any of their code changes (and not when only a comment
+    does)."""
     h = hashlib.sha256()
     for part in (name, "ft_ptx.cuh", "ft_nvfp4.cuh"):
-        with open(os.path.join(ROOT, "bit_quantized_lora_b200", "csrc", part), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "bit_quantized_lora_b200", "csrc", part)) as f:
+            code = _COMMENT.sub("", f.read())
+        h.update(" ".join(code.split()).encode())
     return h.hexdigest()[:16]
 
 

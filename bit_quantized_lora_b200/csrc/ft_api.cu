@@ -526,9 +526,9 @@ ft_status launch_qres(const ft::qres::Params& p, int mt, int splits, cudaStream_
 
 // Q(T), g_T and P = [bf16(T L1) | bf16(s T L2)] for T [M, C], with the
 // tensor amax computed on the way (amax_in == null) or taken from the caller.
-// When the CTAs' chunks fit in shared memory all at once, one cooperative
-// launch of k_qres reads T from HBM once; otherwise the amax pass (if
-// needed) is followed by k_qdown (or the plain 1x16 quantizer when r == 0).
+// When the CTAs' chunks fit in shared memory all at once, one launch of
+// k_qres reads T from HBM once; otherwise the amax pass (if needed) is
+// followed by k_qdown (or the plain 1x16 quantizer when r == 0).
 ft_status run_quant_down(const void* T, int64_t M, int64_t C, const void* L1, int64_t r1,
                          const void* L2, int64_t r2, float s, const float* amax_in, uint8_t* codes,
                          uint8_t* scales, float* tscale, void* P, uint8_t* ws, const WsPlan& w,

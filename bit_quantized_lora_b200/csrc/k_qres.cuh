@@ -16,9 +16,11 @@
 //            K = 16 step.
 //   barrier  the CTA's max is folded into one global word (an integer max on
 //            the float bits: exact, order-free); a grid-wide arrival counter
-//            (cooperative launch: every CTA is resident) releases all CTAs
-//            once every max is in.  Skipped when the caller supplies the
-//            tensor amax.
+//            releases all CTAs once every max is in.  Every CTA is resident
+//            at once: the grid never exceeds the CTAs the device holds (one
+//            per SM), and the host launches it plainly (its CTAs wait on the
+//            device for the previous kernel) or, on request, cooperatively.
+//            Skipped when the caller supplies the tensor amax.
 //   phase 2  the tensor scale and the per-scale divisor table, then every
 //            block is encoded from shared memory with the block maxima kept
 //            in registers since phase 1; codes and scales are staged in
