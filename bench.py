@@ -294,23 +294,26 @@ def run_ours(args):
     shape = workload()
     M, N, K, r_s, r_l = shape.M, shape.N, shape.K, shape.r_s, shape.r_l
 
-    # synthetic inputs (weak scaling: every rank owns its own batch)
-    inp = ft_synth.make_inputs(shape, seed=1 + rank)
+    # synthetic inputs (weak scaling): the weights are replicas (one seed for
+    # every rank), every rank owns its own batch of tokens
+    from bit_quantized_lora_b200 import dp
+    wts = ft_synth.make_inputs(shape, seed=1)
+    inp = ft_synth.make_inputs(shape, seed=dp.rank_seed(1, rank))
 
     def to_dev(u16):
         return torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).to(dev).view(torch.bfloat16)
 
     X, dY = to_dev(inp["X"]), to_dev(inp["dY"])
-    W, A, B = to_dev(inp["W"]), to_dev(inp["A"]), to_dev(inp["B"])
-    layer = ft.prepare_layer(W, r_s, A=A, B=B, s=inp["s"])  # untimed preparation
+    W, A, B = to_dev(wts["W"]), to_dev(wts["A"]), to_dev(wts["B"])
+    layer = ft.prepare_layer(W, r_s, A=A, B=B, s=wts["s"])  # untimed preparation
     ws = ft.Workspace()
     ws.get(ft.ft_workspace_bytes(M, N, K, r_s, r_l), dev)
     Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
     P = torch.empty(M, r_s + r_l, dtype=torch.bfloat16, device=dev)
     dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
-    grads = torch.empty(K * r_l + N * r_l, dtype=torch.float32, device=dev)
-    dA = grads[:K * r_l].view(K, r_l)
-    dB = grads[K * r_l:].view(N, r_l)
+    # dA, dB in one buffer: the step's only exchange is its sum over ranks
+    ag = dp.AdapterGrads(K, N, r_l, dev)
+    grads, dA, dB = ag.flat, ag.dA, ag.dB
     # L2 flush between steps: write a buffer larger than the 126 MB L2, then
     # read another one, so each step starts with a cold L2 that holds neither
     # the step's data nor dirty lines awaiting write-back
@@ -329,8 +332,7 @@ def run_ours(args):
     def step(Xs, dYs):
         ft.ft_linear_fwd(layer, Xs, Y=Y, P=P, ws=ws)
         ft.ft_linear_bwd(layer, dYs, Xs, P, dX=dX, dA=dA, dB=dB, ws=ws)
-        if dist is not None:
-            dist.all_reduce(grads)
+        ag.allreduce()
 
     def keep_host_ahead():
         # a short device-side sleep so the whole step is enqueued before the
@@ -382,11 +384,7 @@ def run_ours(args):
                                          "k_lora_grad", "k_pack_lt", "k_lora_grad_reduce"]}
     total_launches = ft.timing.read("*")[1]  # the same launches as the timed steps
     assert ft.ft_device_error() == 0, "device error during the per-kernel pass"
-    ms_step = sum(step_ms) / len(step_ms)
-    if dist is not None:
-        t = torch.tensor([ms_step], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
+    ms_step = dp.max_over_ranks(sum(step_ms) / len(step_ms), dev)
 
     # ---------------- end to end through the API with host buffers
     Xh = torch.from_numpy(np.ascontiguousarray(inp["X"]).view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -409,14 +407,10 @@ def run_ours(args):
         e1.synchronize()
         if i >= args.warmup:
             e2e_ms.append(e0.elapsed_time(e1))
-    ms_e2e = sum(e2e_ms) / len(e2e_ms)
-    if dist is not None:
-        t = torch.tensor([ms_e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = dp.max_over_ranks(sum(e2e_ms) / len(e2e_ms), dev)
 
     flops = fp4_flops_per_step(shape)
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    value = dp.job_rate(flops, world, ms_step) / 1e12
     hbm_gbs, bf16_tflops, peak_src = measured_peaks()
     fp4_peak = bf16_tflops * FP4_OVER_BF16
 
@@ -488,7 +482,7 @@ def run_ours(args):
         "wall_s_timed_region": t_wall,
         "clocks": clocks,
         "e2e": {
-            "value": world * flops / (ms_e2e * 1e-3) / 1e12,
+            "value": dp.job_rate(flops, world, ms_e2e) / 1e12,
             "unit": UNIT,
             "h2d_bytes_per_step": X.numel() * 2 + dY.numel() * 2,
             "d2h_bytes_per_step": grads.numel() * 4,

@@ -1,0 +1,132 @@
+"""The data-parallel path on the CPU: two gloo ranks (world size 2), each
+with its own batch of tokens and the same replicated weights, exchange the
+adapter gradients with the helpers bench.py uses over NCCL.
+
+Pins: the all-reduced dA, dB equal the oracle's gradients on the two batches
+stacked into one (FourTune page, section 3.2, Eq. 3: the adapter gradients
+are sums over token rows, and P_lora, Pg_lora are row-wise); the job's step
+time is the slowest rank's; the job rate counts every rank's work.  A rank
+that leaves before the exchange makes the other rank's collective fail
+within the process group's timeout instead of hanging."""
+import datetime
+import os
+import socket
+import tempfile
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+WORLD = 2
+BASE_SEED = 7
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _init(rank: int, port: int, timeout_s: float):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=WORLD,
+                            timeout=datetime.timedelta(seconds=timeout_s))
+    return dist
+
+
+def _batch(rank: int):
+    """Replicated weights (one seed for every rank) and this rank's tokens."""
+    import ft_synth
+    from bit_quantized_lora_b200 import dp
+    shape = ft_synth.TINY
+    w = ft_synth.make_inputs(shape, BASE_SEED)
+    mine = ft_synth.make_inputs(shape, dp.rank_seed(BASE_SEED + 100, rank))
+    return shape, w, mine["X"], mine["dY"]
+
+
+def _oracle_grads(shape, w, X, dY):
+    import oracle
+    U, V, Wr = oracle.svd_split(w["W"], shape.r_s)
+    qw = oracle.quantize_16x16(Wr)
+    f = oracle.linear_fwd(X, Wr, U, V, w["A"], w["B"], w["s"], rows=np.arange(1), qw=qw)
+    b = oracle.linear_bwd(dY, X, Wr, U, V, w["A"], w["B"], w["s"], f["P"], rows=np.arange(1), qw=qw)
+    return b["dA"], b["dB"]
+
+
+def _exchange_worker(rank: int, port: int, out: str):
+    dist = _init(rank, port, 60.0)
+    try:
+        from bit_quantized_lora_b200 import dp
+        shape, w, X, dY = _batch(rank)
+        dA, dB = _oracle_grads(shape, w, X, dY)
+        g = dp.AdapterGrads(shape.K, shape.N, shape.r_l, "cpu", dtype=torch.float64)
+        g.dA.copy_(torch.from_numpy(dA))
+        g.dB.copy_(torch.from_numpy(dB))
+        g.allreduce()
+        # the slowest rank sets the step time; the rate counts both ranks
+        slow = dp.max_over_ranks(1.0 + rank)
+        rate = dp.job_rate(10.0, WORLD, slow)
+        np.savez(os.path.join(out, f"rank{rank}.npz"), dA=g.dA.numpy(), dB=g.dB.numpy(),
+                 slow=slow, rate=rate)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_adapter_gradients_all_reduced_over_two_ranks_equal_the_full_batch():
+    with tempfile.TemporaryDirectory() as out:
+        mp.start_processes(_exchange_worker, args=(_free_port(), out), nprocs=WORLD, start_method="spawn")
+        r = [np.load(os.path.join(out, f"rank{k}.npz")) for k in range(WORLD)]
+    # every rank holds the same sum
+    np.testing.assert_array_equal(r[0]["dA"], r[1]["dA"])
+    np.testing.assert_array_equal(r[0]["dB"], r[1]["dB"])
+    # ... which is the gradient of the stacked batch (rows of both ranks)
+    shape, w, X0, dY0 = _batch(0)
+    _, _, X1, dY1 = _batch(1)
+    dA, dB = _oracle_grads(shape, w, np.concatenate([X0, X1]), np.concatenate([dY0, dY1]))
+    for got, ref in ((r[0]["dA"], dA), (r[0]["dB"], dB)):
+        assert np.abs(ref).max() > 0
+        np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+    # the job's step time is the slowest rank's, and the rate counts both
+    assert float(r[0]["slow"]) == float(r[1]["slow"]) == 2.0
+    assert float(r[0]["rate"]) == pytest.approx(WORLD * 10.0 / 2e-3)
+
+
+def test_job_rate_rejects_a_nonpositive_time():
+    from bit_quantized_lora_b200 import dp
+    with pytest.raises(ValueError):
+        dp.job_rate(1.0, 2, 0.0)
+
+
+def _leaver_worker(rank: int, port: int, out: str):
+    dist = _init(rank, port, 5.0)
+    from bit_quantized_lora_b200 import dp
+    g = dp.AdapterGrads(4, 4, 16, "cpu")
+    g.flat.fill_(1.0)
+    if rank == 1:
+        # leaves between steps: no collective of its own is in flight
+        return
+    try:
+        g.allreduce()
+        result = "completed"
+    except Exception as e:  # the exchange must fail, not hang
+        result = "failed: " + type(e).__name__
+    with open(os.path.join(out, "rank0.txt"), "w") as f:
+        f.write(result)
+
+
+def test_a_rank_that_leaves_makes_the_exchange_fail_not_hang():
+    import time
+    with tempfile.TemporaryDirectory() as out:
+        t0 = time.monotonic()
+        try:
+            mp.start_processes(_leaver_worker, args=(_free_port(), out), nprocs=WORLD, start_method="spawn")
+        except Exception:
+            pass  # the leaver's exit may be reported by the launcher; rank 0's record decides
+        elapsed = time.monotonic() - t0
+        with open(os.path.join(out, "rank0.txt")) as f:
+            result = f.read()
+    assert result.startswith("failed"), result
+    assert elapsed < 120.0
