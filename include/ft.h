@@ -225,7 +225,8 @@ ft_status ft_device_error(int* code, void* stream);
  *     serialization.  Its CTAs take SMs as the previous kernel's CTAs
  *     retire and wait on the device for that kernel's results; all of them
  *     are resident once it ends, unless a kernel of another stream or
- *     process keeps SMs busy meanwhile.  If that lasts longer than the
+ *     process keeps SMs busy meanwhile, or the process may use only part of
+ *     the SMs (an MPS share below 100 %, a green context).  If that lasts longer than the
  *     barrier's wait limit (1 s) the call's results are invalid and
  *     ft_device_error() reports the timeout (code 8); nothing hangs.
  *   on = 1: a cooperative launch: the driver starts the grid only when all
