@@ -163,3 +163,24 @@ def test_cooperative_quantizer_switch_is_host_only(L):
             assert L.ft_set_cooperative_quantizer(on) == 0
     finally:
         L.ft_set_cooperative_quantizer(0)
+
+
+def test_header_is_plain_c_and_the_library_links_from_c(L, tmp_path):
+    """include/ft.h compiles as strict C11 (no C++ or CUDA headers) and a C
+    program links libft_b200.so and runs its host-only entry points."""
+    import shutil
+    import subprocess
+    from bit_quantized_lora_b200 import _lib
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    lib = _lib.lib_path()
+    exe = tmp_path / "c_client"
+    cmd = [gcc, "-std=c11", "-Wall", "-Wextra", "-pedantic", "-Werror",
+           "-I", os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "c_client.c"),
+           "-o", str(exe), "-L", os.path.dirname(lib), "-l:" + os.path.basename(lib),
+           "-Wl,-rpath," + os.path.dirname(lib)]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stdout + r.stderr
