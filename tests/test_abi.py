@@ -184,3 +184,25 @@ def test_header_is_plain_c_and_the_library_links_from_c(L, tmp_path):
     assert r.returncode == 0, r.stderr
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0 and r.stdout.strip() == "ok", r.stdout + r.stderr
+
+
+def test_recorded_traffic_follows_kernel_code_not_comments(tmp_path, monkeypatch):
+    """bench.py reports a kernel's ncu DRAM traffic only while the recorded
+    source hash matches: a comment edit keeps the figure, a code edit drops
+    it (the counters were taken on other code)."""
+    import importlib.util
+    import shutil
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    csrc = tmp_path / "bit_quantized_lora_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for f in ("k_qres.cuh", "ft_ptx.cuh", "ft_nvfp4.cuh"):
+        shutil.copy(os.path.join(ROOT, "bit_quantized_lora_b200", "csrc", f), csrc / f)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.kernel_source_sha("k_qres.cuh")
+    src = (csrc / "k_qres.cuh").read_text()
+    (csrc / "k_qres.cuh").write_text(src.replace("#pragma once", "// a new comment\n/* and another */\n#pragma once", 1))
+    assert bench.kernel_source_sha("k_qres.cuh") == h0
+    (csrc / "k_qres.cuh").write_text(src.replace("constexpr int MAX_FS = 8;", "constexpr int MAX_FS = 6;", 1))
+    assert bench.kernel_source_sha("k_qres.cuh") != h0
