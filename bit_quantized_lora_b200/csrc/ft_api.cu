@@ -111,8 +111,7 @@ inline ft_status last_launch() { return cuda_ok(cudaGetLastError()); }
 // that kernel's results itself (grid_dep_wait) after its setup.
 template <typename P>
 ft_status launch_overlapped(void (*kernel)(P), dim3 grid, dim3 block, size_t smem, cudaStream_t st, const P& p) {
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
@@ -310,8 +309,7 @@ WsPlan plan_ws(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t r_l) {
 }
 
 // ------------------------------------------------------------ pieces
-ft_status run_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, float* slot,
-                   const DevInfo* d, cudaStream_t st) {
+ft_status run_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, float* slot, cudaStream_t st) {
     FT_TRY(cuda_ok(cudaMemsetAsync(slot, 0, sizeof(float), st)));
     const int64_t vecs = rows * (cols / 8);
     // one round of four 16-byte loads per thread covers a dense tensor
@@ -501,8 +499,7 @@ std::atomic<int> g_qres_cooperative{0};
 // requested and the kernel computes the tensor amax itself.
 ft_status launch_qres(const ft::qres::Params& p, int mt, int splits, cudaStream_t st) {
     namespace Q = ft::qres;
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)mt, (unsigned)splits, 1);
     cfg.blockDim = dim3(Q::NUM_THREADS, 1, 1);
     cfg.dynamicSmemBytes = Q::make_layout(p.cchunk / Q::BKC, p.ring_bytes).total;
@@ -546,7 +543,7 @@ ft_status run_quant_down(const void* T, int64_t M, int64_t C, const void* L1, in
     if (!qres_grid(M, C, qres_max_stages(p.ring_bytes), d, &mt, &splits, &cchunk) || mt > QRES_MAX_ROW_TILES) {
         const float* a = amax_in;
         if (!a) {
-            FT_TRY(run_amax(T, M, C, C, reinterpret_cast<float*>(ws + w.amax), d, st));
+            FT_TRY(run_amax(T, M, C, C, reinterpret_cast<float*>(ws + w.amax), st));
             a = reinterpret_cast<float*>(ws + w.amax);
         }
         return run_qdown(T, M, C, L1, r1, L2, r2, s, a, codes, scales, tscale, P, ws, w, d, st);
@@ -882,7 +879,7 @@ ft_status ft_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, ft_
     const float* a = amax;
     if (!a) {
         float* slot = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + 128);
-        FT_TRY(run_amax(x, rows, cols, ld, slot, d, st));
+        FT_TRY(run_amax(x, rows, cols, ld, slot, st));
         a = slot;
     }
     if (blk == FT_BLK_1x16)
@@ -920,7 +917,7 @@ ft_status ft_quantize_transpose(const void* x, int64_t rows, int64_t cols, int64
     const float* a = amax;
     if (!a) {
         float* slot = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + 128);
-        FT_TRY(run_amax(x, rows, cols, ld, slot, d, st));
+        FT_TRY(run_amax(x, rows, cols, ld, slot, st));
         a = slot;
     }
     if (blk == FT_BLK_16x16)
