@@ -6,7 +6,6 @@ run last so a stop-at-first-failure run has already covered everything else.
 """
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
