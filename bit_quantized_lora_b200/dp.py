@@ -38,10 +38,15 @@ class AdapterGrads:
         self.dA = self.flat[:K * r_l].view(K, r_l)
         self.dB = self.flat[K * r_l:].view(N, r_l)
 
-    def allreduce(self, group=None) -> None:
-        """Sum over the ranks of the group, in place."""
+    def allreduce(self, group=None, async_op: bool = False):
+        """Sum over the ranks of the group, in place.  With async_op the
+        exchange is only started and its handle returned: a training loop
+        overlaps it with the next layer's backward and calls wait() before
+        the optimizer reads dA, dB (None when there is nothing to exchange).
+        """
         if dist.is_initialized() and dist.get_world_size(group) > 1:
-            dist.all_reduce(self.flat, op=dist.ReduceOp.SUM, group=group)
+            return dist.all_reduce(self.flat, op=dist.ReduceOp.SUM, group=group, async_op=async_op)
+        return None
 
 
 def max_over_ranks(x: float, device=None, group=None) -> float:

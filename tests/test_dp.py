@@ -94,6 +94,35 @@ def test_adapter_gradients_all_reduced_over_two_ranks_equal_the_full_batch():
     assert float(r[0]["rate"]) == pytest.approx(WORLD * 10.0 / 2e-3)
 
 
+def _overlap_worker(rank: int, port: int, out: str):
+    dist = _init(rank, port, 60.0)
+    try:
+        from bit_quantized_lora_b200 import dp
+        # two layers' gradients: layer 1's exchange runs while layer 0's
+        # gradients are computed, then both are awaited
+        g1 = dp.AdapterGrads(8, 4, 16, "cpu", dtype=torch.float64)
+        g0 = dp.AdapterGrads(8, 4, 16, "cpu", dtype=torch.float64)
+        g1.flat.copy_(torch.arange(g1.flat.numel(), dtype=torch.float64) * (rank + 1))
+        h = g1.allreduce(async_op=True)
+        g0.flat.fill_(10.0 * (rank + 1))  # the next layer's backward
+        h0 = g0.allreduce(async_op=True)
+        h.wait()
+        h0.wait()
+        np.savez(os.path.join(out, f"ov{rank}.npz"), g1=g1.flat.numpy(), g0=g0.flat.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_asynchronous_exchange_overlaps_and_sums():
+    with tempfile.TemporaryDirectory() as out:
+        mp.start_processes(_overlap_worker, args=(_free_port(), out), nprocs=WORLD, start_method="spawn")
+        r = [np.load(os.path.join(out, f"ov{k}.npz")) for k in range(WORLD)]
+    n = r[0]["g1"].size
+    for k in range(WORLD):
+        np.testing.assert_array_equal(r[k]["g1"], np.arange(n, dtype=np.float64) * 3.0)
+        np.testing.assert_array_equal(r[k]["g0"], np.full(n, 30.0))
+
+
 def test_job_rate_rejects_a_nonpositive_time():
     from bit_quantized_lora_b200 import dp
     with pytest.raises(ValueError):
