@@ -36,12 +36,16 @@
 //           up-projection (kind::f16, N = 128), then four
 //           tcgen05.mma.kind::mxf4nvf4.block16 (K = 64, N = 256) per stage
 //           into the FP32 accumulator, then low-rank half 1.
-//   warp 2  scale warp: tcgen05.cp of each stage's slabs into a two-deep
-//           ring of scale columns, ahead of the MMAs (copies issued by
-//           another warp overlap the MMAs instead of queueing behind them).
-//   warps 4-11 epilogue, two groups working on the two column halves at
-//           once: tcgen05.ld accumulator and low-rank half into registers,
-//           release tensor memory, combine, stage and store Y once.
+//   warps 2-5  scale warps, one per TMEM lane quarter (2, 3, 0, 1): each
+//           lane loads its 16-byte slab row of every K step from shared
+//           memory and writes it with tcgen05.st into its own lane of a
+//           two-deep ring of scale columns -- the replicated contents a
+//           tcgen05.cp 32x128b.warpx4 per slab would leave, without the
+//           ~52 tensor-pipe cycles each of those twelve copies a stage costs.
+//   warps 6-13 epilogue, two groups working on the two column halves at
+//           once: tcgen05.ld accumulator and low-rank half into registers
+//           (16 columns at a time), release tensor memory, combine, stage
+//           and store Y once.
 // TMEM columns: [0,256) accumulator, [256,384) low-rank half 0, [384,512)
 // the scale ring (per slot: A 16 columns, B 32 columns) during the mainloop
 // and low-rank half 1 after it.
@@ -64,7 +68,9 @@ constexpr int BK_BYTES = 128;  // 256 FP4 elements of K per stage
 constexpr int KSTEPS = 4;      // MMAs of K = 64 per stage
 constexpr int MAX_STAGES = 4;
 constexpr int NUM_EPI_WARPS = 8;  // two column groups of four lane-quarter warps
-constexpr int NUM_THREADS = 128 + 32 * NUM_EPI_WARPS;
+constexpr int NUM_SF_WARPS = 4;   // one per TMEM lane quarter
+constexpr int EPI_WARP0 = 2 + NUM_SF_WARPS;
+constexpr int NUM_THREADS = 32 * (EPI_WARP0 + NUM_EPI_WARPS);
 constexpr int A_BYTES = BM * BK_BYTES;         // 16 KiB
 constexpr int B_BYTES = BN * BK_BYTES;         // 32 KiB of codes
 constexpr int SFA_STAGE_BYTES = KSTEPS * 512;  // four slabs (128 rows)
@@ -198,7 +204,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             mbar_init(&bars[B_EMPTY + i], 1);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&bars[B_SF_READY + i], 1);
+            mbar_init(&bars[B_SF_READY + i], NUM_SF_WARPS);
             mbar_init(&bars[B_SF_FREE + i], 1);
         }
         mbar_init(&bars[B_ACC_FULL], 1);
@@ -361,52 +367,59 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             mbar_wait(&bars[B_DRAIN], 0, ERR_WAIT_DRAIN, &no_abort);
         }
         __syncwarp();
-    } else if (warp == 2) {
-        // ------------------------------------------------ scale warp
-        if (lane == 0) {
-            const uint32_t hi_sf = (128u >> 4) | (1u << 14);  // 8-row groups 128 B apart
-            const uint32_t sfa_lo0 = (base + L.sfa) >> 4;     // one 16-byte column: LBO unused
-            const uint32_t sfb_lo0 = (base + L.b + B_BYTES) >> 4;  // the scales behind each B tile
-            uint32_t it = 0;
-            bool ok = true;
-            int local = 0;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
-                // the ring's columns hold the previous tile's low-rank half 1
-                // until its epilogue is done
-                if (has_lr && local > 0 &&
-                    !mbar_wait(&bars[B_ACC_EMPTY], (local - 1) & 1, ERR_WAIT_SF, abort_flag)) {
+    } else if (warp < EPI_WARP0) {
+        // ------------------------------------------------ scale warps
+        // Warp q (= warp % 4) writes TMEM lanes 32q .. 32q + 31; its lane i
+        // stores slab row i of every K step (16 bytes each) into its own
+        // lane: the contents a tcgen05.cp 32x128b.warpx4 of each slab would
+        // leave in every lane quarter, written by the TMEM store path
+        // instead of the tensor pipe.
+        const uint32_t lane_addr = (uint32_t)(32 * (warp & 3)) << 16;
+        uint32_t it = 0;
+        bool ok = true;
+        int local = 0;
+        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+            // the ring's columns hold the previous tile's low-rank half 1
+            // until its epilogue is done
+            if (has_lr && local > 0 &&
+                !mbar_wait(&bars[B_ACC_EMPTY], (local - 1) & 1, ERR_WAIT_SF, abort_flag)) {
+                ok = false;
+                break;
+            }
+            for (int kt = 0; kt < KT; ++kt, ++it) {
+                const int s = it % S;
+                const int sb = it & 1;
+                if (!mbar_wait(&bars[B_SFFULL + s], (it / S) & 1, ERR_WAIT_FULL, abort_flag) ||
+                    !mbar_wait(&bars[B_SF_FREE + sb], ((it >> 1) & 1) ^ 1, ERR_WAIT_SF, abort_flag)) {
                     ok = false;
                     break;
                 }
-                for (int kt = 0; kt < KT; ++kt, ++it) {
-                    const int s = it % S;
-                    const int sb = it & 1;
-                    if (!mbar_wait(&bars[B_SFFULL + s], (it / S) & 1, ERR_WAIT_FULL, abort_flag) ||
-                        !mbar_wait(&bars[B_SF_FREE + sb], ((it >> 1) & 1) ^ 1, ERR_WAIT_SF, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t sfa_lo = sfa_lo0 + s * (SFA_STAGE_BYTES >> 4);
-                    const uint32_t sfb_lo = sfb_lo0 + s * (B_SLOT >> 4);
-                    const uint32_t sf = tmem + R2_COL + sb * SF_SLOT_COLS;
+                tc_fence_after();
+                const uint32_t sfa = base + L.sfa + (uint32_t)s * SFA_STAGE_BYTES + 16u * (uint32_t)lane;
+                const uint32_t sfb = base + L.b + (uint32_t)s * B_SLOT + B_BYTES + 16u * (uint32_t)lane;
+                uint32_t ra[16], rb[32];
 #pragma unroll
-                    for (int j = 0; j < KSTEPS; ++j) {
-                        // A: rows 0-127; B: rows 0-127 then 128-255 (four columns each)
-                        tc_cp_32x128b_x4(sf + 4 * j, make_desc(sfa_lo + 32 * j, hi_sf));
-                        tc_cp_32x128b_x4(sf + 16 + 8 * j, make_desc(sfb_lo + 32 * j, hi_sf));
-                        tc_cp_32x128b_x4(sf + 20 + 8 * j,
-                                         make_desc(sfb_lo + (SFA_STAGE_BYTES >> 4) + 32 * j, hi_sf));
-                    }
-                    tc_commit(&bars[B_SF_READY + sb]);
+                for (int j = 0; j < KSTEPS; ++j) {
+                    const uint4 va = ld_shared_v4(sfa + 512u * j);
+                    const uint4 vl = ld_shared_v4(sfb + 512u * j);
+                    const uint4 vh = ld_shared_v4(sfb + (uint32_t)SFA_STAGE_BYTES + 512u * j);
+                    ra[4 * j] = va.x; ra[4 * j + 1] = va.y; ra[4 * j + 2] = va.z; ra[4 * j + 3] = va.w;
+                    rb[8 * j] = vl.x; rb[8 * j + 1] = vl.y; rb[8 * j + 2] = vl.z; rb[8 * j + 3] = vl.w;
+                    rb[8 * j + 4] = vh.x; rb[8 * j + 5] = vh.y; rb[8 * j + 6] = vh.z; rb[8 * j + 7] = vh.w;
                 }
+                const uint32_t sf = tmem + lane_addr + R2_COL + (uint32_t)sb * SF_SLOT_COLS;
+                tmem_st_32x32b_x16(sf, ra);
+                tmem_st_32x32b_x32(sf + 16, rb);
+                tmem_st_wait();
+                // the slab bytes were read through the generic proxy; the
+                // stage goes back to TMA after the MMAs
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[B_SF_READY + sb]);
             }
-            tc_commit(&bars[B_DRAIN_SF]);
-            volatile int no_abort = 0;
-            mbar_wait(&bars[B_DRAIN_SF], 0, ERR_WAIT_DRAIN, &no_abort);
         }
-        __syncwarp();
-    } else if (warp >= 4) {
+    } else {
         // ------------------------------------------------ epilogue
         // Each thread owns one tile row (its TMEM lane) within one of two
         // column groups working concurrently: warps 4-7 take columns 0-127
@@ -418,8 +431,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
         // whole sectors of eight rows.  (A TMA store per chunk would queue
         // in the same copy engine as the next tile's operand loads.)
         const int sp = warp & 3;  // TMEM sub-partition = rows 32*sp .. +31
-        const int grp = (warp - 4) >> 2;
-        const int et = (threadIdx.x - 128) & 127;  // tile row
+        const int grp = (warp - EPI_WARP0) >> 2;
+        const int et = 32 * sp + lane;  // tile row
         const uint32_t rsw = (uint32_t)((et >> 1) & 3);
         const uint32_t buf = base + L.stg + (uint32_t)grp * STG_BYTES;
         const uint32_t lr_col = grp == 0 ? LR0_COL : R2_COL;
@@ -459,18 +472,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                 // while they drain
                 uint32_t pk[4][16];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t v[32], lr[32];
-                    tmem_ld_32x32b_x32(tmem + lane_addr + ACC_COL + 128 * grp + 32 * c, v);
-                    if (has_lr) tmem_ld_32x32b_x32(tmem + lane_addr + lr_col + 32 * c, lr);
+                for (int c2 = 0; c2 < 8; ++c2) {
+                    const int c = c2 >> 1, h = (c2 & 1) * 8;
+                    uint32_t v[16], lr[16];
+                    tmem_ld_32x32b_x16(tmem + lane_addr + ACC_COL + 128 * grp + 16 * c2, v);
+                    if (has_lr) tmem_ld_32x32b_x16(tmem + lane_addr + lr_col + 16 * c2, lr);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) {
+                    for (int k = 0; k < 8; ++k) {
                         const float y0 = __fmaf_rn(gab, __uint_as_float(v[2 * k]), has_lr ? __uint_as_float(lr[2 * k]) : 0.0f);
                         const float y1 =
                             __fmaf_rn(gab, __uint_as_float(v[2 * k + 1]), has_lr ? __uint_as_float(lr[2 * k + 1]) : 0.0f);
                         __nv_bfloat162 t = __floats2bfloat162_rn(y0, y1);
-                        pk[c][k] = *reinterpret_cast<uint32_t*>(&t);
+                        pk[c][h + k] = *reinterpret_cast<uint32_t*>(&t);
                     }
                 }
                 // every TMEM read of this tile is done: the MMA warp may
