@@ -175,12 +175,23 @@ class Layer:
                         _ptr(self.op_n))
 
 
+def _bf16_rne(x: torch.Tensor) -> torch.Tensor:
+    """float64 -> bf16 with one round-to-nearest-even step (torch's own cast
+    goes through float32 and so rounds twice, which differs at near-ties):
+    the value is scaled so that bf16's 8 significant bits are the integer
+    part, rounded half to even, and scaled back -- exact in bf16 from there."""
+    _, e = torch.frexp(x)
+    q = torch.clamp(e.to(torch.int64) - 8, min=-133)
+    return torch.ldexp(torch.round(torch.ldexp(x, -q)), q).to(torch.float32).to(torch.bfloat16)
+
+
 def svd_split(W: torch.Tensor, r_s: int):
     """Eq. 1 on the host side (untimed, once per layer): W ~ W_res + V U^T
     with the top-r_s singular triplets, taken from the smaller Gram matrix in
     float64 (eigenvectors of W^T W are the right singular vectors, those of
     W W^T the left ones).  U = right vectors [K, r_s], V = W U [N, r_s], both
-    rounded to bf16, and W_res = W - V U^T from the rounded factors."""
+    rounded to bf16, and W_res = W - V U^T from the rounded factors (each
+    rounded once, to nearest even)."""
     Wd = W.to(torch.float64)
     N, K = Wd.shape
     if r_s == 0:
@@ -193,9 +204,9 @@ def svd_split(W: torch.Tensor, r_s: int):
         order = torch.argsort(evals, descending=True)[:r_s]
         sig = evals[order].clamp_min(0).sqrt()
         vtop = (Wd.T @ evecs[:, order]) / torch.where(sig > 0, sig, torch.ones_like(sig))
-    U = vtop.to(torch.bfloat16).contiguous()
-    V = (Wd @ U.to(torch.float64)).to(torch.bfloat16).contiguous()
-    W_res = (Wd - V.to(torch.float64) @ U.to(torch.float64).T).to(torch.bfloat16).contiguous()
+    U = _bf16_rne(vtop).contiguous()
+    V = _bf16_rne(Wd @ U.to(torch.float64)).contiguous()
+    W_res = _bf16_rne(Wd - V.to(torch.float64) @ U.to(torch.float64).T).contiguous()
     return U, V, W_res
 
 

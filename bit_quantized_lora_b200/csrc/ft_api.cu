@@ -34,16 +34,50 @@ struct DevInfo {
     int sms = 0;
     bool attr_set = false;
     int qres_ctas = 0;  // CTAs of k_qres that fit on the device at once
+    unsigned long long ctx = 0;  // the context the kernel attributes were set in
 };
 DevInfo g_dev[64];
 std::mutex g_mu;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+PFN_cuCtxGetId_v12000 g_ctx_id = nullptr;
+
+// The unique ID of the current device's context (the primary context the
+// runtime uses).  Per-device state the library caches -- kernel attributes,
+// the device address of a module variable -- belongs to one context;
+// cudaDeviceReset destroys it, and the next context has a new ID.  Caller
+// holds g_mu.
+ft_status current_ctx_id(int dev, unsigned long long* id) {
+    if (!g_ctx_current || !g_ctx_id) {
+        void* f1 = nullptr;
+        void* f2 = nullptr;
+        cudaDriverEntryPointQueryResult q1, q2;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+            q1 != cudaDriverEntryPointSuccess || !f1 ||
+            cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+            q2 != cudaDriverEntryPointSuccess || !f2)
+            return FT_ERR_CUDA;
+        g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f1);
+        g_ctx_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f2);
+    }
+    CUcontext c = nullptr;
+    if (g_ctx_current(&c) != CUDA_SUCCESS) return FT_ERR_CUDA;
+    if (!c) {
+        // no context current yet: cudaSetDevice initialises the runtime's
+        // primary context of the device and makes it current
+        if (cudaSetDevice(dev) != cudaSuccess || g_ctx_current(&c) != CUDA_SUCCESS || !c) return FT_ERR_CUDA;
+    }
+    return g_ctx_id(c, id) == CUDA_SUCCESS ? FT_OK : FT_ERR_CUDA;
+}
 
 ft_status device_info(DevInfo** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FT_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_mu);
     DevInfo& d = g_dev[dev];
+    unsigned long long ctx = 0;
+    if (current_ctx_id(dev, &ctx) != FT_OK) return FT_ERR_CUDA;
+    if (d.attr_set && d.ctx != ctx) d.attr_set = false;  // a new context: set the attributes again
     if (!d.init) {
         int major = 0, minor = 0, sms = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
@@ -98,6 +132,7 @@ ft_status device_info(DevInfo** out) {
             return FT_ERR_CUDA;
         d.qres_ctas = per_sm * d.sms;
         d.attr_set = true;
+        d.ctx = ctx;
     }
     *out = &d;
     return FT_OK;
@@ -1071,19 +1106,25 @@ constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
 __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 void* g_noalloc_scratch_dev[64] = {};
-std::mutex g_noalloc_mu;
+unsigned long long g_noalloc_ctx[64] = {};
 
 // Device address of g_noalloc_scratch on the current device.  The host
 // symbol is only a stand-in; the address has to be looked up, once per
-// device, with that device current.
+// device, with that device current -- and again after cudaDeviceReset, whose
+// new context loads the library's device image (and the array) anew.  A
+// fresh image holds the array zero-filled, as the calls' synchronisation
+// words need.
 ft_status noalloc_scratch(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FT_ERR_CUDA;
-    std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_scratch_dev[dev]) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    unsigned long long ctx = 0;
+    FT_TRY(current_ctx_id(dev, &ctx));
+    if (!g_noalloc_scratch_dev[dev] || g_noalloc_ctx[dev] != ctx) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return FT_ERR_CUDA;
         g_noalloc_scratch_dev[dev] = p;
+        g_noalloc_ctx[dev] = ctx;
     }
     *out = g_noalloc_scratch_dev[dev];
     return FT_OK;

@@ -361,6 +361,20 @@ __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
+// A kernel that took its inputs through a counter (wait_inputs with `done`)
+// never passed the grid dependency wait, so nothing holds it back until the
+// kernel before it on the stream has completed: it could complete first.
+// The next kernel's griddepcontrol.wait orders it after this kernel only, so
+// without this the next kernel could start overwriting buffers the
+// predecessor still reads (e.g. the next quantizer rewriting the workspace's
+// codes while a dgrad GEMM still reads them).  Called by every thread at the
+// end of such a kernel, after its last global write, it makes this kernel's
+// completion imply its predecessor's (a no-op after the plain dependency
+// wait, which already did the same).
+__device__ __forceinline__ void finish_after_predecessor(const unsigned long long* done) {
+    if (done) grid_dep_wait();
+}
+
 __device__ __forceinline__ void wait_inputs(const unsigned long long* done, unsigned long long epoch,
                                             unsigned int count, volatile int* abort_flag) {
     if (done) {

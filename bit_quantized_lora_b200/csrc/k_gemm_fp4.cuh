@@ -156,7 +156,6 @@ enum {
     B_LR0_READY,                       // low-rank half 0 computed
     B_LR1_READY,                       // low-rank half 1 computed
     B_DRAIN,
-    B_DRAIN_SF,
     B_COUNT
 };
 static_assert(B_COUNT * 8 + 8 <= 256, "barrier area");
@@ -214,7 +213,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
         mbar_init(&bars[B_LR0_READY], 1);
         mbar_init(&bars[B_LR1_READY], 1);
         mbar_init(&bars[B_DRAIN], 1);
-        mbar_init(&bars[B_DRAIN_SF], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -422,8 +420,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
     } else {
         // ------------------------------------------------ epilogue
         // Each thread owns one tile row (its TMEM lane) within one of two
-        // column groups working concurrently: warps 4-7 take columns 0-127
-        // (with low-rank half 0), warps 8-11 columns 128-255 (half 1).
+        // column groups working concurrently: warps 6-9 take columns 0-127
+        // (with low-rank half 0), warps 10-13 columns 128-255 (half 1).
         // Output leaves in chunks of 64 bytes per row (32 bf16 or 16 f32
         // columns): the group's rows are written into its 64-byte-swizzled
         // staging buffer, then the group copies the 128-row chunk out with
@@ -540,6 +538,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
+    finish_after_predecessor(p.dep_done);
 }
 
 }  // namespace gemm

@@ -222,26 +222,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_lora_grad(const __grid_const
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
-    if (*abort_flag) return;
-    if (threadIdx.x == 0) {
-        __threadfence();
-        const unsigned long long prev = epoch_count(&p.counters[z * p.ctiles_max + blockIdx.x], p.epoch);
-        *last_flag = (prev == (unsigned long long)(p.splits - 1)) ? 1 : 0;
+    bool last = false;
+    if (!*abort_flag) {
+        if (threadIdx.x == 0) {
+            __threadfence();
+            const unsigned long long prev = epoch_count(&p.counters[z * p.ctiles_max + blockIdx.x], p.epoch);
+            *last_flag = (prev == (unsigned long long)(p.splits - 1)) ? 1 : 0;
+        }
+        __syncthreads();
+        last = *last_flag != 0;
     }
-    __syncthreads();
-    if (!*last_flag) return;
-    __threadfence();
-    // the tile's partials, 4 floats at a time: every split's load of UNR
-    // elements is issued before the first add (one L2 round trip per pass),
-    // then the adds run in split order
-    const int n4 = BC * p.r_l / 4;
-    const int64_t stride4 = (int64_t)p.C[z] * p.r_l / 4;
-    const float4* part4 = reinterpret_cast<const float4*>(p.part[z]) + (int64_t)c0 * p.r_l / 4;
-    float4* out4 = reinterpret_cast<float4*>(p.out[z]) + (int64_t)c0 * p.r_l / 4;
-    if (p.splits <= 4)
-        reduce_splits<4, 3>(part4, stride4, n4, p.splits, out4);
-    else
-        reduce_splits<MAX_SPLITS, 1>(part4, stride4, n4, p.splits, out4);
+    if (last) {
+        __threadfence();
+        // the tile's partials, 4 floats at a time: every split's load of UNR
+        // elements is issued before the first add (one L2 round trip per
+        // pass), then the adds run in split order
+        const int n4 = BC * p.r_l / 4;
+        const int64_t stride4 = (int64_t)p.C[z] * p.r_l / 4;
+        const float4* part4 = reinterpret_cast<const float4*>(p.part[z]) + (int64_t)c0 * p.r_l / 4;
+        float4* out4 = reinterpret_cast<float4*>(p.out[z]) + (int64_t)c0 * p.r_l / 4;
+        if (p.splits <= 4)
+            reduce_splits<4, 3>(part4, stride4, n4, p.splits, out4);
+        else
+            reduce_splits<MAX_SPLITS, 1>(part4, stride4, n4, p.splits, out4);
+    }
+    // this grid completes only after the dgrad GEMM it overlapped
+    finish_after_predecessor(p.dep_done);
 }
 
 }  // namespace lgrad

@@ -46,6 +46,21 @@
  *   - NaN or Inf inputs are outside the contract; results are unspecified.
  *   - Device-side failures (a bounded wait inside a kernel that ran out) set a
  *     device error word; read and clear it with ft_device_error().
+ *   - Calls on one stream may be enqueued back to back without host
+ *     synchronisation: each kernel completes only after every kernel before
+ *     it on the stream, so a later call (or the caller's own kernel) never
+ *     overwrites or reads a buffer an earlier call still uses.
+ *   - The kernels of ft_quantize, ft_quantize_transpose (1x16, computed
+ *     amax), ft_linear_fwd and ft_linear_bwd synchronise through counter
+ *     words in the workspace, tagged with an epoch the host draws afresh for
+ *     every call and writes into the launch's parameters.  Replaying a CUDA
+ *     graph that captured such a call reuses its epochs: the counters
+ *     already hold their final values from the previous replay, so the
+ *     device waits would pass without waiting.  Do not replay captured calls.
+ *   - The library caches per-device state (kernel attributes, module
+ *     addresses) on first use and sets it up again in a new context of the
+ *     device (after cudaDeviceReset); workspaces allocated in the old
+ *     context are gone with it.
  */
 #ifndef FT_H_
 #define FT_H_
@@ -251,8 +266,9 @@ const char* ft_status_str(ft_status s);
  *   ft_workspace_bytes() exceeds it returns FT_ERR_WORKSPACE, nothing
  *   launched.  The function itself allocates nothing.
  *   The first call on a device looks up the array's device address (once
- *   per device, with that device current); make that first call before any
- *   stream capture.
+ *   per device, with that device current, and again in a new context of the
+ *   device after cudaDeviceReset); make that first call before any stream
+ *   capture.
  *   All calls on a device share its one copy of the array, which keeps the
  *   last call's contents (each call clears what must start at zero itself).
  *   Calls whose work overlaps on the same GPU (two streams, two host
