@@ -54,3 +54,48 @@ def check_lowrank_down(P_gpu_u16, P_ref_u16, Td, L1d, L2d, s):
     bound = bf16_ulp_of(ref) + K * 2.0 ** -23 * mag + bf16_ulp_of(mag * K * 2.0 ** -23)
     excess = np.abs(got - ref) - bound
     assert np.all(excess <= 0), float(excess.max())
+
+
+def check_fp32_sum_bound(got, ref, absdot, terms, slack=None):
+    """Each entry of an FP32-accumulated result within the worst-case error
+    of recursive FP32 summation of its `terms` products, terms * 2^-23 *
+    sum |products| (absdot), plus one final FP32 rounding of the value
+    (and `slack`, an allowance for operands that were themselves rounded
+    differently, when given).  A single wrong entry -- a dropped or
+    duplicated block, a stale tile -- breaks this bound even where a norm
+    over the whole output would not notice it."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    bound = terms * 2.0 ** -23 * np.asarray(absdot, np.float64) + 2.0 ** -23 * np.abs(ref) + 1e-30
+    if slack is not None:
+        bound = bound + slack
+    excess = np.abs(got - ref) - bound
+    worst = np.unravel_index(np.argmax(excess), excess.shape)
+    assert np.all(excess <= 0), (float(excess[worst]), worst, float(got[worst]), float(ref[worst]))
+
+
+def lossless_operand(rng, rows, cols, block_rows, exp_range=(-1, 1)):
+    """bf16 bits of a [rows, cols] matrix whose every block_rows x 16 block
+    holds E2M1 grid values times one power of two, with a +-6 element in
+    the block's first position, so that block quantization with tensor
+    scale 1 is lossless (drawn in whole arrays: grid indices, signs, block
+    exponents, first-element signs)."""
+    import ft_synth
+    grid = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    v = grid[rng.integers(0, 8, size=(rows, cols))] * rng.choice([-1.0, 1.0], size=(rows, cols))
+    nb = (rows // block_rows, cols // 16)
+    e = rng.integers(exp_range[0], exp_range[1] + 1, size=nb)
+    v[::block_rows, ::16] = 6.0 * rng.choice([-1.0, 1.0], size=nb)
+    v *= np.ldexp(1.0, np.repeat(np.repeat(e, block_rows, axis=0), 16, axis=1))
+    return ft_synth.to_bf16_bits(v)
+
+
+def selection_factor(rng, rows, r, exps=(-1, 0, 1)):
+    """bf16 bits of a [rows, r] factor with exactly one nonzero, +-2^e, per
+    column, in distinct rows: products with it are exact and its low-rank
+    sums have a single term."""
+    import ft_synth
+    F = np.zeros((rows, r))
+    idx = rng.choice(rows, r, replace=False)
+    F[idx, np.arange(r)] = rng.choice([-1.0, 1.0], size=r) * np.ldexp(1.0, rng.choice(exps, size=r))
+    return ft_synth.to_bf16_bits(F)

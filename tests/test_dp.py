@@ -159,3 +159,86 @@ def test_a_rank_that_leaves_makes_the_exchange_fail_not_hang():
             result = f.read()
     assert result.startswith("failed"), result
     assert elapsed < 120.0
+
+
+class _FakeLayer:
+    """The fields of a prepared layer the stack driver reads (N, K, ranks);
+    the layer's weights ride along for the stand-in backward."""
+
+    def __init__(self, shape, w):
+        self.N, self.K, self.r_s, self.r_l, self.s = shape.N, shape.K, shape.r_s, shape.r_l, w["s"]
+        self.shape, self.w = shape, w
+
+
+def _stack_worker(rank: int, port: int, out: str):
+    """The stack driver's step over two layers with the library calls
+    replaced by CPU stand-ins (the oracle's backward writes dA, dB): records
+    the call order and the quantizer launch mode each backward saw, and the
+    all-reduced per-layer gradients."""
+    dist = _init(rank, port, 60.0)
+    try:
+        import ft_synth
+        from bit_quantized_lora_b200 import dp, stack
+        log, coop = [], [False]
+
+        def to_t(u16):
+            return torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).view(torch.bfloat16)
+
+        def fake_fwd(L, X, amax_x=None, out_dtype=0, Y=None, P=None, ws=None):
+            log.append(("fwd", L.tag))
+
+        def fake_bwd(L, dY, X, P, amax_dy=None, out_dtype=0, dX=None, dA=None, dB=None, ws=None):
+            log.append(("bwd", L.tag, coop[0]))
+            Xn = X.view(torch.int16).numpy().view(np.uint16)
+            dYn = dY.view(torch.int16).numpy().view(np.uint16)
+            gA, gB = _oracle_grads(L.shape, L.w, Xn, dYn)
+            dA.copy_(torch.from_numpy(gA).float())
+            dB.copy_(torch.from_numpy(gB).float())
+
+        stack.ft_linear_fwd, stack.ft_linear_bwd = fake_fwd, fake_bwd
+        stack.ft_set_cooperative_quantizer = lambda on: coop.__setitem__(0, bool(on))
+        layers, Xs, dYs = [], [], []
+        for j in range(2):
+            shape = ft_synth.TINY
+            w = ft_synth.make_inputs(shape, BASE_SEED + 10 * j)
+            mine = ft_synth.make_inputs(shape, dp.rank_seed(BASE_SEED + 100 + 10 * j, rank))
+            L = _FakeLayer(shape, w)
+            L.tag = j
+            layers.append(L)
+            Xs.append(to_t(mine["X"]))
+            dYs.append(to_t(mine["dY"]))
+        st = stack.LinearStack(layers, ft_synth.TINY.M, "cpu")
+        st.step(Xs, dYs)
+        np.savez(os.path.join(out, f"st{rank}.npz"), grads=st.grads.numpy(),
+                 log=np.array([str(x) for x in log]), coop_after=coop[0])
+    finally:
+        dist.destroy_process_group()
+
+
+def test_stack_step_exchanges_every_layer_during_the_backward():
+    """Two ranks run the stack driver's step over two layers: forwards in
+    order, backwards in reverse order, each backward with the cooperative
+    quantizer launch on (the exchanges of earlier layers run beside it) and
+    the plain launch restored after the step; every layer's all-reduced
+    (dA, dB) slice equals the oracle's gradient of the two ranks' batches
+    stacked into one (FourTune page, section 3.2: sums over token rows)."""
+    import ft_synth
+    from bit_quantized_lora_b200 import dp
+    with tempfile.TemporaryDirectory() as out:
+        mp.start_processes(_stack_worker, args=(_free_port(), out), nprocs=WORLD, start_method="spawn")
+        r = [np.load(os.path.join(out, f"st{k}.npz")) for k in range(WORLD)]
+    np.testing.assert_array_equal(r[0]["grads"], r[1]["grads"])
+    assert list(r[0]["log"]) == [str(("fwd", 0)), str(("fwd", 1)), str(("bwd", 1, True)), str(("bwd", 0, True))]
+    assert not bool(r[0]["coop_after"])
+    shape = ft_synth.TINY
+    off = 0
+    for j in range(2):
+        w = ft_synth.make_inputs(shape, BASE_SEED + 10 * j)
+        b = [ft_synth.make_inputs(shape, dp.rank_seed(BASE_SEED + 100 + 10 * j, k)) for k in range(WORLD)]
+        dA, dB = _oracle_grads(shape, w, np.concatenate([x["X"] for x in b]), np.concatenate([x["dY"] for x in b]))
+        n = (shape.K + shape.N) * shape.r_l
+        got = r[0]["grads"][off:off + n].astype(np.float64)
+        ref = np.concatenate([dA.ravel(), dB.ravel()])
+        # each rank's FP32 gradient, summed in FP32 by the exchange
+        np.testing.assert_allclose(got, ref, rtol=0, atol=4 * 2.0 ** -24 * np.abs(ref).max() + 1e-12)
+        off += n

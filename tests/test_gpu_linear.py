@@ -2,7 +2,8 @@
 the adapter gradients) against the CPU oracle.
 
 Bar: Y, dX, dA, dB within relative Frobenius error 1e-3 of the FP64 oracle
-(FP32 output mode); exactly equal when every operand is losslessly
+(FP32 output mode), and every entry within the FP32 summation error bound of
+its reference on the same operands; exactly equal when every operand is losslessly
 representable (the FP4 GEMM then has an exact FP32 result); each entry of P
 within one bf16 rounding plus the FP32 summation error bound of its
 reference; the BF16 output mode within one bf16 ulp of the rounded oracle;
@@ -14,7 +15,8 @@ import torch
 import ft_synth
 import oracle
 import bit_quantized_lora_b200 as ft
-from gpu_util import bf16_ulp_diff, check_lowrank_down, dev_bf16, host, host_u16, scalar_dev
+from gpu_util import (bf16_ulp_diff, check_fp32_sum_bound, check_lowrank_down, dev_bf16, host, host_u16,
+                      lossless_operand, scalar_dev, selection_factor)
 
 pytestmark = pytest.mark.gpu
 
@@ -60,6 +62,7 @@ def _run_and_compare(shape, seed, M=None, rows=None, r_s=None, r_l=None, bf16_ch
     if layer.r_s + layer.r_l > 0:
         check_lowrank_down(host_u16(P), f["P"], oracle.bf16_to_f64(X), oracle.bf16_to_f64(U),
                            oracle.bf16_to_f64(A), s)
+    _check_elementwise(layer, inp, U, V, qw, f, b, rows, host_u16(P), host(Y), host(dX), host(dA), host(dB))
     if bf16_check:
         # the BF16 mode rounds the same FP32 value the FP32 mode stores
         Yb, _ = ft.ft_linear_fwd(layer, Xd, out_dtype=ft.BF16)
@@ -77,6 +80,45 @@ def _run_and_compare(shape, seed, M=None, rows=None, r_s=None, r_l=None, bf16_ch
         big = (np.abs(f["Y"]) >= np.sqrt(np.mean(f["Y"] ** 2)) / 64)[same]
         assert ulp[big].max() <= 1 and (ulp > 0).mean() < 0.01
     return layer
+
+
+def _check_elementwise(layer, inp, U, V, qw, f, b, rows, P_gpu, Y, dX, dA, dB):
+    """Every sampled entry of Y, dX and every entry of dA, dB within the FP32
+    summation bound of its own reference (check_fp32_sum_bound).  The
+    references take the operands the kernels took: the dequantized Q(X),
+    Q(dY), Q(W_res) of the oracle (bit-identical to the GPU's, checked
+    elsewhere) and the GPU's saved P where P is an operand (Y's low-rank
+    term, dB).  Pg never leaves the workspace, so dX and dA get an
+    allowance of the valid alternative roundings of Pg (one bf16 ulp plus
+    Pg's own FP32 summation bound, as for P)."""
+    from gpu_util import bf16_ulp_of
+    X, dY, A, B, s = inp["X"], inp["dY"], inp["A"], inp["B"], inp["s"]
+    N, K, r_s, r_l = layer.N, layer.K, layer.r_s, layer.r_l
+    M = X.shape[0]
+    d = oracle.bf16_to_f64
+    Xq = oracle.dequant_1x16(*f["qx"], M, K)[rows]
+    dYq = oracle.dequant_1x16(*b["qdy"], M, N)[rows]
+    Wq = oracle.dequant_16x16(qw[0], qw[2], qw[3], N, K)
+    Pd = d(P_gpu)
+    LRf = np.concatenate([d(V), d(B)], axis=1)
+    LRb = np.concatenate([d(U), d(A)], axis=1)
+    ref = Xq @ Wq.T + Pd[rows] @ LRf.T
+    absdot = np.abs(Xq) @ np.abs(Wq).T + np.abs(Pd[rows]) @ np.abs(LRf).T
+    check_fp32_sum_bound(Y[rows], ref, absdot, K)
+    Pg = d(b["Pg"])
+    dYd = d(dY)
+    mag = np.concatenate([np.abs(dYd) @ np.abs(d(V)), abs(s) * (np.abs(dYd) @ np.abs(d(B)))], axis=1)
+    dPg = bf16_ulp_of(Pg) + N * 2.0 ** -23 * mag  # Pg's valid alternative roundings
+    ref = dYq @ Wq + Pg[rows] @ LRb.T
+    absdot = np.abs(dYq) @ np.abs(Wq) + np.abs(Pg[rows]) @ np.abs(LRb).T
+    check_fp32_sum_bound(dX[rows], ref, absdot, N, slack=dPg[rows] @ np.abs(LRb).T)
+    if r_l > 0:
+        Xd = d(X)
+        P_lora = Pd[:, r_s:r_s + r_l]
+        check_fp32_sum_bound(dB, dYd.T @ P_lora, np.abs(dYd).T @ np.abs(P_lora), M)
+        Pg_lora = Pg[:, r_s:r_s + r_l]
+        check_fp32_sum_bound(dA, Xd.T @ Pg_lora, np.abs(Xd).T @ np.abs(Pg_lora), M,
+                             slack=np.abs(Xd).T @ dPg[:, r_s:r_s + r_l])
 
 
 @pytest.mark.parametrize("K", [256, 512, 768, 1024])
@@ -98,6 +140,63 @@ def test_lossless_operands_give_exact_fp32_gemm(K):
     Xf, Wf, dYf = oracle.bf16_to_f64(X), oracle.bf16_to_f64(Wr), oracle.bf16_to_f64(dY)
     np.testing.assert_array_equal(host(Y).astype(np.float64), Xf @ Wf.T)
     np.testing.assert_array_equal(host(dX).astype(np.float64), dYf @ Wf)
+
+
+@pytest.mark.parametrize("case", ["attn", "mlp_up"])
+def test_lossless_full_size_is_bit_exact(case):
+    """Full-size workloads (4608 tokens) on operands that every step of the
+    layer represents exactly: activations, gradients and the weight hold
+    E2M1 grid values times a power of two per block (quantization with
+    tensor scale 1 is lossless), and U, V, A, B select one input column per
+    rank column with a factor +-2^k (so P, Pg and the low-rank products have
+    a single exact term); s = 2.  Every sum is a multiple of 2^-4 whose
+    absolute terms add up to less than 2^20, so FP32 accumulation is exact
+    in any order.  Y, dX, dA, dB must then equal the exact result bit for
+    bit, element by element -- every tile of the persistent GEMM (each CTA
+    takes several), the low-rank epilogue's columns, the split reductions --
+    and the BF16 output mode must be the exact value rounded once."""
+    shape = ft_synth.ATTN if case == "attn" else ft_synth.MLP_UP
+    M, N, K, r_s, r_l = shape.M, shape.N, shape.K, shape.r_s, shape.r_l
+    rng = np.random.default_rng(90 if case == "attn" else 91)
+    X = lossless_operand(rng, M, K, 1)
+    dY = lossless_operand(rng, M, N, 1)
+    Wr = lossless_operand(rng, N, K, 16)
+    U, V = selection_factor(rng, K, r_s), selection_factor(rng, N, r_s)
+    A, B = selection_factor(rng, K, r_l), selection_factor(rng, N, r_l)
+    s = 2.0
+    g1 = scalar_dev(2688.0)  # tensor scale g = 1
+    layer = ft.prepare_layer(W_res=dev_bf16(Wr), U=dev_bf16(U), V=dev_bf16(V), A=dev_bf16(A), B=dev_bf16(B),
+                             s=s, amax=g1)
+    Xd, dYd = dev_bf16(X), dev_bf16(dY)
+    Y, P = ft.ft_linear_fwd(layer, Xd, amax_x=g1, out_dtype=ft.F32)
+    Yb, _ = ft.ft_linear_fwd(layer, Xd, amax_x=g1, out_dtype=ft.BF16)
+    dX, dA, dB = ft.ft_linear_bwd(layer, dYd, Xd, P, amax_dy=g1, out_dtype=ft.F32)
+    dXb, _, _ = ft.ft_linear_bwd(layer, dYd, Xd, P, amax_dy=g1, out_dtype=ft.BF16)
+    torch.cuda.synchronize()
+    assert ft.ft_device_error() == 0
+    f = oracle.bf16_to_f64
+    Xf, dYf, Wf, Uf, Vf, Af, Bf = (f(t) for t in (X, dY, Wr, U, V, A, B))
+    P_ref = np.concatenate([Xf @ Uf, s * (Xf @ Af)], axis=1)
+    Pg_ref = np.concatenate([dYf @ Vf, s * (dYf @ Bf)], axis=1)
+    for T in (P_ref, Pg_ref):
+        assert np.array_equal(f(oracle.bf16_from_f64(T)), T)  # exact in bf16
+    np.testing.assert_array_equal(host_u16(P), oracle.bf16_from_f64(P_ref))
+    LRf = np.concatenate([Vf, Bf], axis=1)
+    LRb = np.concatenate([Uf, Af], axis=1)
+    refs = {
+        "Y": (Xf @ Wf.T + P_ref @ LRf.T, np.abs(Xf) @ np.abs(Wf).T + np.abs(P_ref) @ np.abs(LRf).T),
+        "dX": (dYf @ Wf + Pg_ref @ LRb.T, np.abs(dYf) @ np.abs(Wf) + np.abs(Pg_ref) @ np.abs(LRb).T),
+        "dA": (Xf.T @ Pg_ref[:, r_s:], np.abs(Xf).T @ np.abs(Pg_ref[:, r_s:])),
+        "dB": (dYf.T @ P_ref[:, r_s:], np.abs(dYf).T @ np.abs(P_ref[:, r_s:])),
+    }
+    got = {"Y": host(Y), "dX": host(dX), "dA": host(dA), "dB": host(dB)}
+    for name, (ref, absdot) in refs.items():
+        # the precondition of exactness: multiples of 2^-4 below 2^20
+        assert absdot.max() < 2.0 ** 20 and np.array_equal(ref * 16, np.rint(ref * 16)), name
+        assert np.abs(ref).max() > 0
+        np.testing.assert_array_equal(got[name].astype(np.float64), ref, err_msg=name)
+    np.testing.assert_array_equal(host_u16(Yb), oracle.bf16_from_f64(refs["Y"][0]))
+    np.testing.assert_array_equal(host_u16(dXb), oracle.bf16_from_f64(refs["dX"][0]))
 
 
 def test_tiny_workload_fwd_bwd():
