@@ -212,16 +212,19 @@ def svd_split(W: torch.Tensor, r_s: int):
 
 def prepare_layer(W: torch.Tensor | None = None, r_s: int = 0, A: torch.Tensor | None = None,
                   B: torch.Tensor | None = None, s: float = 1.0, *, U=None, V=None, W_res=None,
-                  amax: torch.Tensor | None = None, ws: Workspace | None = None) -> Layer:
+                  amax: torch.Tensor | None = None, ws: Workspace | None = None,
+                  weight_blk: int = BLK_16x16) -> Layer:
     """Once-per-layer preparation: split W (or take a given U, V, W_res) and
-    quantize W_res with 16x16 blocks into both code layouts in one pass."""
+    quantize W_res into both code layouts in one pass: 16x16 blocks (the
+    method), or with weight_blk=BLK_1x16 the granularity ablation's 1x16
+    groups (W_res along K and, independently, W_res^T along N)."""
     if W_res is None:
         U, V, W_res = svd_split(W, r_s)
     _bf16(W_res, "W_res")
     N, K = W_res.shape
     r_s = 0 if U is None else U.shape[1]
     r_l = 0 if A is None else A.shape[1]
-    w_k, w_n = ft_quantize_transpose(W_res.contiguous(), BLK_16x16, amax=amax, ws=ws)
+    w_k, w_n = ft_quantize_transpose(W_res.contiguous(), weight_blk, amax=amax, ws=ws)
     op_k, op_n = ft_pack_weight_operands(w_k, w_n, N, K)
     return Layer(N, K, r_s, r_l, float(s), w_k, w_n, U, V,
                  None if A is None else A.contiguous(), None if B is None else B.contiguous(), op_k, op_n)
@@ -234,9 +237,14 @@ def ft_pack_weight_operands(w_k, w_n, N: int, K: int, stream=None):
     nbytes = load().ft_weight_operand_bytes(N, K)
     op_k = torch.empty(nbytes, dtype=torch.uint8, device=w_k.codes.device)
     op_n = torch.empty(nbytes, dtype=torch.uint8, device=w_k.codes.device)
-    check("ft_pack_weight_operands", load().ft_pack_weight_operands(
-        w_k.codes.data_ptr(), w_n.codes.data_ptr(), w_k.scales.data_ptr(), N, K, op_k.data_ptr(),
-        op_n.data_ptr(), _stream(stream)))
+    if w_k.blk == BLK_1x16:
+        check("ft_pack_weight_operands_1x16", load().ft_pack_weight_operands_1x16(
+            w_k.codes.data_ptr(), w_k.scales.data_ptr(), w_n.codes.data_ptr(), w_n.scales.data_ptr(), N, K,
+            op_k.data_ptr(), op_n.data_ptr(), _stream(stream)))
+    else:
+        check("ft_pack_weight_operands", load().ft_pack_weight_operands(
+            w_k.codes.data_ptr(), w_n.codes.data_ptr(), w_k.scales.data_ptr(), N, K, op_k.data_ptr(),
+            op_n.data_ptr(), _stream(stream)))
     return op_k, op_n
 
 

@@ -55,6 +55,7 @@ SIGNATURES = {
     "ft_quantize_workspace_bytes": (ctypes.c_size_t, []),
     "ft_weight_operand_bytes": (ctypes.c_size_t, [c_i64, c_i64]),
     "ft_pack_weight_operands": (ctypes.c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_vp]),
+    "ft_pack_weight_operands_1x16": (ctypes.c_int, [c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_vp]),
     "ft_workspace_qact": (ctypes.c_int, [c_i64, c_i64, c_i64, c_i64, c_i64,
                                          ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t),
                                          ctypes.POINTER(ctypes.c_size_t)]),

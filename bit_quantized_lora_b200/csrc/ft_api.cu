@@ -791,13 +791,20 @@ ft_status check_linear(const ft_linear* L) {
     if (L->N % 256 || L->K % 256) return FT_ERR_SHAPE;
     if (L->r_s % 16 || L->r_l % 16 || L->r_s + L->r_l > 128) return FT_ERR_SHAPE;
     if (L->N > (1 << 20) || L->K > (1 << 20)) return FT_ERR_SHAPE;
-    FT_TRY(check_fp4_view(&L->w_k, L->N, L->K, FT_BLK_16x16));
-    if (!L->w_n.codes) return FT_ERR_INVALID_ARG;
-    if (L->w_n.rows != L->K || L->w_n.cols != L->N || L->w_n.blk != FT_BLK_16x16) return FT_ERR_SHAPE;
-    if (!al16(L->w_n.codes)) return FT_ERR_ALIGN;
-    if ((L->w_n.scales && L->w_n.scales != L->w_k.scales) ||
-        (L->w_n.tscale && L->w_n.tscale != L->w_k.tscale))
-        return FT_ERR_INVALID_ARG;
+    if (L->w_k.blk == FT_BLK_1x16) {
+        // 1x16 weight groups: two independent quantizations, W_res along K
+        // and W_res^T along N, one tensor scale (read through w_k)
+        FT_TRY(check_fp4_view(&L->w_k, L->N, L->K, FT_BLK_1x16));
+        FT_TRY(check_fp4_view(&L->w_n, L->K, L->N, FT_BLK_1x16));
+    } else {
+        FT_TRY(check_fp4_view(&L->w_k, L->N, L->K, FT_BLK_16x16));
+        if (!L->w_n.codes) return FT_ERR_INVALID_ARG;
+        if (L->w_n.rows != L->K || L->w_n.cols != L->N || L->w_n.blk != FT_BLK_16x16) return FT_ERR_SHAPE;
+        if (!al16(L->w_n.codes)) return FT_ERR_ALIGN;
+        if ((L->w_n.scales && L->w_n.scales != L->w_k.scales) ||
+            (L->w_n.tscale && L->w_n.tscale != L->w_k.tscale))
+            return FT_ERR_INVALID_ARG;
+    }
     if (L->r_s > 0 && (!L->U || !L->V)) return FT_ERR_INVALID_ARG;
     if (L->r_l > 0 && (!L->A || !L->B)) return FT_ERR_INVALID_ARG;
     if ((L->U && !al16(L->U)) || (L->V && !al16(L->V)) || (L->A && !al16(L->A)) ||
@@ -844,9 +851,28 @@ ft_status ft_pack_weight_operands(const uint8_t* codes_k, const uint8_t* codes_n
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int64_t chunks = (int64_t)ft_weight_operand_bytes(N, K) / 16;
     const int grid_n = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(chunks, 256), (int64_t)d->sms * 16));
-    ft::k_pack_wop<<<grid_n, 256, 0, st>>>(codes_k, grid, N, K, 0, op_k);
+    ft::k_pack_wop<<<grid_n, 256, 0, st>>>(codes_k, grid, nullptr, N, K, 0, op_k);
     FT_TRY(last_launch());
-    ft::k_pack_wop<<<grid_n, 256, 0, st>>>(codes_n, grid, N, K, 1, op_n);
+    ft::k_pack_wop<<<grid_n, 256, 0, st>>>(codes_n, grid, nullptr, N, K, 1, op_n);
+    return last_launch();
+}
+
+ft_status ft_pack_weight_operands_1x16(const uint8_t* codes_k, const uint8_t* scales_k, const uint8_t* codes_n,
+                                       const uint8_t* scales_n, int64_t N, int64_t K, uint8_t* op_k,
+                                       uint8_t* op_n, void* stream) {
+    if (!codes_k || !scales_k || !codes_n || !scales_n || !op_k || !op_n || N < 0 || K < 0)
+        return FT_ERR_INVALID_ARG;
+    if (N % 256 || K % 256) return FT_ERR_SHAPE;
+    if (!al16(codes_k) || !al16(codes_n) || !al16(op_k) || !al16(op_n)) return FT_ERR_ALIGN;
+    if (N == 0 || K == 0) return FT_OK;
+    DevInfo* d;
+    FT_TRY(device_info(&d));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t chunks = (int64_t)ft_weight_operand_bytes(N, K) / 16;
+    const int grid_n = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(chunks, 256), (int64_t)d->sms * 16));
+    ft::k_pack_wop<<<grid_n, 256, 0, st>>>(codes_k, nullptr, scales_k, N, K, 0, op_k);
+    FT_TRY(last_launch());
+    ft::k_pack_wop<<<grid_n, 256, 0, st>>>(codes_n, nullptr, scales_n, N, K, 1, op_n);
     return last_launch();
 }
 

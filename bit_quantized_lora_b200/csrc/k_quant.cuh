@@ -80,8 +80,11 @@ __global__ void __launch_bounds__(256) k_amax_bf16(const uint16_t* __restrict__ 
 //   codes: the operand's codes [R, Kc/2]; grid: the 16x16 scale grid
 //   [N/16, K/16]; trans = 0: operand rows are N (op_k, Kc = K), trans = 1:
 //   operand rows are K (op_n, Kc = N) and the grid is read transposed.
+//   rows_sc (instead of grid, for 1x16 weight groups): the operand's own
+//   row-major 1x16 scales [R, Kc/16].
 __global__ void __launch_bounds__(256) k_pack_wop(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ grid,
-                                                  int64_t N, int64_t K, int trans, uint8_t* __restrict__ op) {
+                                                  const uint8_t* __restrict__ rows_sc, int64_t N, int64_t K,
+                                                  int trans, uint8_t* __restrict__ op) {
     const int64_t R = trans ? K : N, Kc = trans ? N : K;
     const int64_t KT = Kc / 256, gc = K / 16;
     const int64_t chunks = (R / 256) * KT * 288 * 8;
@@ -108,7 +111,8 @@ __global__ void __launch_bounds__(256) k_pack_wop(const uint8_t* __restrict__ co
                     const int l = e >> 4, ii = (e >> 2) & 3, b = e & 3;
                     const int64_t orow = 256 * t + 128 * h + 32 * ii + l;  // operand row
                     const int64_t kb = 16 * kt + 4 * j + b;                // 16-wide contraction block
-                    const uint32_t sb = trans ? grid[kb * gc + orow / 16] : grid[(orow / 16) * gc + kb];
+                    const uint32_t sb = rows_sc ? rows_sc[orow * (Kc / 16) + kb]
+                                        : trans ? grid[kb * gc + orow / 16] : grid[(orow / 16) * gc + kb];
                     acc |= sb << (8 * bb);
                 }
                 w[q] = acc;

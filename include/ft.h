@@ -106,6 +106,11 @@ typedef struct {
  *   w_n : the same codes transposed, rows = K, cols = N (codes packed along
  *         N).  Its scales/tscale pointers must equal w_k's: one scale grid
  *         [N/16, K/16] serves both layouts (section 3.2).
+ *   Or, for the granularity ablation (section 4, "Impact of Quantization
+ *   Granularity", Table 5), both FT_BLK_1x16: w_k = Q(W_res) in 1x16 groups
+ *   along K (scales [N, K/16]), w_n = Q(W_res^T), an independent 1x16
+ *   quantization along N (scales [K, N/16]), as ft_quantize_transpose
+ *   writes them; the tensor scale is read through w_k.
  *   U [K, r_s], V [N, r_s], A [K, r_l], B [N, r_l]: bf16, row-major, dense.
  *   r_s, r_l: multiples of 16 with r_s + r_l <= 128 (either may be 0).
  *   s: the LoRA scale.
@@ -175,6 +180,15 @@ ft_status ft_quantize_transpose(const void* x, int64_t rows, int64_t cols, int64
 size_t ft_weight_operand_bytes(int64_t N, int64_t K);
 ft_status ft_pack_weight_operands(const uint8_t* codes_k, const uint8_t* codes_n, const uint8_t* grid,
                                   int64_t N, int64_t K, uint8_t* op_k, uint8_t* op_n, void* stream);
+
+/* ft_pack_weight_operands_1x16 -- the same images for 1x16 weight groups:
+ * each operand's row-major scales (scales_k = w_k.scales [N, K/16] for
+ * op_k, scales_n = w_n.scales [K, N/16] for op_n) take the grid's place,
+ * one scale per row and 16 contraction columns already.  Arguments and
+ * errors otherwise as ft_pack_weight_operands.                             */
+ft_status ft_pack_weight_operands_1x16(const uint8_t* codes_k, const uint8_t* scales_k, const uint8_t* codes_n,
+                                       const uint8_t* scales_n, int64_t N, int64_t K, uint8_t* op_k,
+                                       uint8_t* op_n, void* stream);
 
 /* ft_linear_fwd -- Eq. 2 with LoRA fusion (section 3.3): one pass over X
  * emits Q(X) and the down-projections P = [bf16(X U) | bf16(s X A)]; one

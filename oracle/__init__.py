@@ -263,23 +263,51 @@ def _lowrank_down(Xd: np.ndarray, L1: np.ndarray, L2: np.ndarray, s: float):
     return np.concatenate(parts, axis=1)
 
 
-def linear_fwd(X, W_res, U, V, A, B, s: float, rows=None, amax_x=None, qw=None):
+def _weight_fwd(W_res, qw, weight_blk):
+    """Dequantized forward weight [N, K]: 16x16 blocks (the method's), or
+    1x16 groups along K (the granularity ablation: FourTune page, section 4,
+    "Impact of Quantization Granularity", Table 5)."""
+    N, K = W_res.shape
+    if weight_blk == "16x16":
+        qw = quantize_16x16(W_res) if qw is None else qw
+        return qw, dequant_16x16(qw[0], qw[2], qw[3], N, K)
+    if weight_blk == "1x16":
+        qw = quantize_1x16(W_res) if qw is None else qw
+        return qw, dequant_1x16(qw[0], qw[1], qw[2], N, K)
+    raise ValueError(weight_blk)
+
+
+def _weight_dgrad(W_res, qw, weight_blk):
+    """Dequantized dgrad weight as [N, K]: the 16x16 codes serve both
+    directions (their blocks are square); 1x16 groups along K do not, so
+    W_res^T is quantized again in 1x16 groups along N (same tensor scale)."""
+    N, K = W_res.shape
+    if weight_blk == "16x16":
+        qw = quantize_16x16(W_res) if qw is None else qw
+        return qw, dequant_16x16(qw[0], qw[2], qw[3], N, K)
+    if weight_blk == "1x16":
+        qw = quantize_1x16_colwise(W_res) if qw is None else qw
+        return qw, dequant_1x16(qw[0], qw[1], qw[2], K, N).T
+    raise ValueError(weight_blk)
+
+
+def linear_fwd(X, W_res, U, V, A, B, s: float, rows=None, amax_x=None, qw=None, weight_blk="16x16"):
     """Forward of the triple-branch layer (Eq. 2).
 
     X: bf16 [M, K]; W_res: bf16 [N, K]; U [K, r_s]; V [N, r_s]; A [K, r_l];
     B [N, r_l].  rows: optional row sample for Y (the quantization and P are
-    always computed on the full tensors).  qw: optional precomputed
-    quantize_16x16(W_res).  Returns a dict with Y (float64 [len(rows), N]),
-    P (bf16 [M, r_s + r_l]), qx = (codes, scales, g) and qw.
+    always computed on the full tensors).  weight_blk: "16x16" (the method)
+    or "1x16" (groups along K, the granularity ablation).  qw: optional
+    precomputed quantize_16x16(W_res) (resp. quantize_1x16(W_res)).  Returns
+    a dict with Y (float64 [len(rows), N]), P (bf16 [M, r_s + r_l]),
+    qx = (codes, scales, g) and qw.
     """
     M, K = X.shape
     N = W_res.shape[0]
     rows = np.arange(M) if rows is None else np.asarray(rows)
     qx = quantize_1x16(X, amax_x)
-    if qw is None:
-        qw = quantize_16x16(W_res)
+    qw, Wq = _weight_fwd(W_res, qw, weight_blk)
     Xq = dequant_1x16(qx[0], qx[1], qx[2], M, K)[rows]
-    Wq = dequant_16x16(qw[0], qw[2], qw[3], N, K)
     Xd = bf16_to_f64(X)
     P = _lowrank_down(Xd, U, A, s)
     Pd = bf16_to_f64(P[rows])
@@ -288,10 +316,13 @@ def linear_fwd(X, W_res, U, V, A, B, s: float, rows=None, amax_x=None, qw=None):
     return {"Y": Y, "P": P, "qx": qx, "qw": qw, "rows": rows}
 
 
-def linear_bwd(dY, X, W_res, U, V, A, B, s: float, P, rows=None, amax_dy=None, qw=None):
+def linear_bwd(dY, X, W_res, U, V, A, B, s: float, P, rows=None, amax_dy=None, qw=None,
+               weight_blk="16x16"):
     """Backward of the triple-branch layer (Eq. 3 and the LoRA gradients).
 
     dY: bf16 [M, N]; X: bf16 [M, K]; P: the forward's saved bf16 [M, r_s+r_l].
+    weight_blk as in linear_fwd; qw: optional precomputed quantize_16x16(W_res)
+    (resp. quantize_1x16_colwise(W_res), the dgrad operand of 1x16 weights).
     Returns dX (float64 [len(rows), K]), dA (float64 [K, r_l]),
     dB (float64 [N, r_l]), Pg (bf16 [M, r_s + r_l]) and qdy.
     """
@@ -300,10 +331,8 @@ def linear_bwd(dY, X, W_res, U, V, A, B, s: float, P, rows=None, amax_dy=None, q
     r_s, r_l = U.shape[1], A.shape[1]
     rows = np.arange(M) if rows is None else np.asarray(rows)
     qdy = quantize_1x16(dY, amax_dy)
-    if qw is None:
-        qw = quantize_16x16(W_res)
+    qw, Wq = _weight_dgrad(W_res, qw, weight_blk)
     dYq = dequant_1x16(qdy[0], qdy[1], qdy[2], M, N)[rows]
-    Wq = dequant_16x16(qw[0], qw[2], qw[3], N, K)
     dYd = bf16_to_f64(dY)
     Pg = _lowrank_down(dYd, V, B, s)
     Pgd = bf16_to_f64(Pg)

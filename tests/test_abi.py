@@ -206,3 +206,30 @@ def test_recorded_traffic_follows_kernel_code_not_comments(tmp_path, monkeypatch
     assert bench.kernel_source_sha("k_qres.cuh") == h0
     (csrc / "k_qres.cuh").write_text(src.replace("constexpr int MAX_FS = 8;", "constexpr int MAX_FS = 6;", 1))
     assert bench.kernel_source_sha("k_qres.cuh") != h0
+
+
+def test_1x16_weight_views_and_packing_validation(L):
+    """The granularity ablation's weights: both views 1x16 with their own
+    scales (W_res along K, W_res^T along N); a mixed pair is refused."""
+    x = 0x200000
+    ws = L.ft_workspace_bytes(128, 256, 256, 16, 16)
+    g1 = _linear()
+    g1.w_k.blk = 0
+    g1.w_n.blk = 0
+    g1.w_n.scales = 0x300000  # its own scales
+    # with M = 0 the call validates the views and returns, launching nothing
+    assert L.ft_linear_fwd(ctypes.byref(g1), x, 0, None, x, 0, x, x, ws, None) == FT_OK
+    mixed = _linear()
+    mixed.w_k.blk = 0
+    assert L.ft_linear_fwd(ctypes.byref(mixed), x, 128, None, x, 0, x, x, ws, None) == FT_ERR_SHAPE
+    no_sc = _linear()
+    no_sc.w_k.blk = 0
+    no_sc.w_n.blk = 0
+    no_sc.w_n.scales = None
+    assert L.ft_linear_fwd(ctypes.byref(no_sc), x, 128, None, x, 0, x, x, ws, None) == FT_ERR_INVALID_ARG
+    g = 0x100000
+    assert L.ft_pack_weight_operands_1x16(g, None, g, g, 256, 256, g, g, None) == FT_ERR_INVALID_ARG
+    assert L.ft_pack_weight_operands_1x16(g, g, g, None, 256, 256, g, g, None) == FT_ERR_INVALID_ARG
+    assert L.ft_pack_weight_operands_1x16(g, g, g, g, 256, 320, g, g, None) == FT_ERR_SHAPE
+    assert L.ft_pack_weight_operands_1x16(g, g, g, g, 256, 256, g, g + 8, None) == FT_ERR_ALIGN
+    assert L.ft_pack_weight_operands_1x16(g, g, g, g, 0, 256, g, g, None) == FT_OK

@@ -374,3 +374,37 @@ def test_cooperative_and_plain_quantizer_launches_agree():
     for o in outs[1:]:
         for a, b in zip(o, outs[0]):
             assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("wl", ["tiny", "attn"])
+def test_1x16_weight_groups_fwd_bwd(wl):
+    """The granularity ablation (FourTune page, section 4, "Impact of
+    Quantization Granularity", Table 5): W_res quantized in 1x16 groups along
+    K for the forward and, independently, W_res^T along N for dgrad.  The
+    weight's codes and scales are bit-exact in both orientations; Y, dX, dA,
+    dB within the same bound as the method's 16x16 layer."""
+    shape, seed = (ft_synth.TINY, 61) if wl == "tiny" else (ft_synth.ATTN, 62)
+    inp = ft_synth.make_inputs(shape, seed)
+    U, V, Wr = oracle.svd_split(inp["W"], shape.r_s)
+    layer = ft.prepare_layer(W_res=dev_bf16(Wr), U=dev_bf16(U), V=dev_bf16(V), A=dev_bf16(inp["A"]),
+                             B=dev_bf16(inp["B"]), s=inp["s"], weight_blk=ft.BLK_1x16)
+    qk = oracle.quantize_1x16(Wr)
+    qn = oracle.quantize_1x16_colwise(Wr)
+    np.testing.assert_array_equal(host(layer.w_k.codes), qk[0])
+    np.testing.assert_array_equal(host(layer.w_k.scales), qk[1])
+    np.testing.assert_array_equal(host(layer.w_n.codes), qn[0])
+    np.testing.assert_array_equal(host(layer.w_n.scales), qn[1])
+    X, dY = dev_bf16(inp["X"]), dev_bf16(inp["dY"])
+    Y, P = ft.ft_linear_fwd(layer, X, out_dtype=ft.F32)
+    dX, dA, dB = ft.ft_linear_bwd(layer, dY, X, P, out_dtype=ft.F32)
+    torch.cuda.synchronize()
+    assert ft.ft_device_error() == 0
+    M = inp["X"].shape[0]
+    rows = np.arange(M) if wl == "tiny" else np.random.default_rng(5).choice(M, 256, replace=False)
+    f = oracle.linear_fwd(inp["X"], Wr, U, V, inp["A"], inp["B"], inp["s"], rows=rows, qw=qk, weight_blk="1x16")
+    b = oracle.linear_bwd(inp["dY"], inp["X"], Wr, U, V, inp["A"], inp["B"], inp["s"], f["P"], rows=rows, qw=qn,
+                          weight_blk="1x16")
+    assert oracle.rel_fro(host(Y)[rows], f["Y"]) <= TOL
+    assert oracle.rel_fro(host(dX)[rows], b["dX"]) <= TOL
+    assert oracle.rel_fro(host(dA), b["dA"]) <= TOL
+    assert oracle.rel_fro(host(dB), b["dB"]) <= TOL

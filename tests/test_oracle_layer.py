@@ -140,3 +140,89 @@ def test_quantized_layer_is_close_to_unquantized_layer():
     exact = Xd @ oracle.bf16_to_f64(W).T + (Xd @ oracle.bf16_to_f64(A)) @ oracle.bf16_to_f64(B).T
     err = oracle.rel_fro(f["Y"], exact)
     assert 0.01 < err < 0.2
+
+
+def _lossless_both_ways(rng, rows, cols):
+    """A weight lossless under 1x16 groups along its rows and along its
+    columns: 16x16 blocks of E2M1 grid values times one power of two each,
+    with +-6 on every block's diagonal (so every 16-long row or column
+    segment of a block holds its maximum, 6 times the block's power)."""
+    grid = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    v = grid[rng.integers(0, 8, size=(rows, cols))] * rng.choice([-1.0, 1.0], size=(rows, cols))
+    for i in range(0, rows, 16):
+        for j in range(0, cols, 16):
+            blk = v[i:i + 16, j:j + 16]
+            d = np.arange(16)
+            blk[d, d] = 6.0 * rng.choice([-1.0, 1.0], size=16)
+            v[i:i + 16, j:j + 16] = blk * 2.0 ** rng.integers(-2, 3)
+    return ft_synth.to_bf16_bits(v)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_1x16_weight_layer_equals_autograd_when_quantization_is_exact(seed):
+    """The granularity ablation's layer (FourTune page, section 4, "Impact
+    of Quantization Granularity", Table 5): 1x16 weight groups along K for
+    the forward, W_res^T re-quantized in 1x16 groups along N for dgrad."""
+    c = _exact_case(seed)
+    c["Wr"] = _lossless_both_ways(np.random.default_rng(100 + seed), *c["Wr"].shape)
+    qf = oracle.quantize_1x16(c["Wr"], c["amax"])
+    qb = oracle.quantize_1x16_colwise(c["Wr"], c["amax"])
+    f = oracle.linear_fwd(c["X"], c["Wr"], c["U"], c["V"], c["A"], c["B"], c["s"],
+                          amax_x=c["amax"], qw=qf, weight_blk="1x16")
+    b = oracle.linear_bwd(c["dY"], c["X"], c["Wr"], c["U"], c["V"], c["A"], c["B"], c["s"],
+                          f["P"], amax_dy=c["amax"], qw=qb, weight_blk="1x16")
+    Y, dX, dA, dB = _torch_layer(c)
+    np.testing.assert_allclose(f["Y"], Y, rtol=1e-12, atol=1e-9)
+    np.testing.assert_allclose(b["dX"], dX, rtol=1e-12, atol=1e-9)
+    np.testing.assert_allclose(b["dA"], dA, rtol=1e-12, atol=1e-9)
+    np.testing.assert_allclose(b["dB"], dB, rtol=1e-12, atol=1e-9)
+
+
+def test_1x16_weight_groups_are_not_transposable_and_fit_closer_than_16x16():
+    """Why the method uses 16x16 blocks: 1x16 groups along K, transposed,
+    are not the 1x16 groups along N that dgrad needs (the backward must
+    quantize again), whereas 16x16 blocks serve both directions.  And why it
+    costs a little fidelity: on the workload's weight the 1x16 groups
+    reconstruct it more closely than 16x16 blocks (Table 5's premise)."""
+    W = ft_synth.make_inputs(ft_synth.TINY, 0)["W"]
+    N, K = W.shape
+    ref = oracle.bf16_to_f64(W)
+    qk = oracle.quantize_1x16(W)
+    qn = oracle.quantize_1x16_colwise(W)
+    wk = oracle.dequant_1x16(qk[0], qk[1], qk[2], N, K)
+    wn = oracle.dequant_1x16(qn[0], qn[1], qn[2], K, N).T
+    assert qk[2] == qn[2]  # one tensor scale
+    assert not np.array_equal(wk, wn)
+    q16 = oracle.quantize_16x16(W)
+    w16 = oracle.dequant_16x16(q16[0], q16[2], q16[3], N, K)
+    assert np.linalg.norm(wk - ref) < np.linalg.norm(w16 - ref)
+    assert np.linalg.norm(wn - ref) < np.linalg.norm(w16 - ref)
+
+
+def test_1x16_dgrad_reads_the_weight_quantized_along_n():
+    """One-hot gradients (one nonzero per token, 24 with the tensor amax
+    given as 2688 * 4, so g = 4 and the block scale is exactly 1: lossless)
+    read single rows of the dgrad weight out of linear_bwd: with 1x16
+    weights they are rows of dequant(Q(W_res^T))^T, not of the forward's
+    groups transposed."""
+    inp = ft_synth.make_inputs(ft_synth.TINY, 2)
+    W = inp["W"]
+    N, K = W.shape
+    M = 8
+    rng = np.random.default_rng(9)
+    cols = rng.choice(N, size=M, replace=False)
+    dY = np.zeros((M, N))
+    dY[np.arange(M), cols] = 24.0
+    dYb = ft_synth.to_bf16_bits(dY)
+    X = ft_synth.to_bf16_bits(rng.standard_normal((M, K)))
+    none_k = np.zeros((K, 0), np.uint16)
+    none_n = np.zeros((N, 0), np.uint16)
+    P = np.zeros((M, 0), np.uint16)
+    b = oracle.linear_bwd(dYb, X, W, none_k, none_n, none_k, none_n, 1.0, P, amax_dy=2688.0 * 4.0,
+                          weight_blk="1x16")
+    qn = oracle.quantize_1x16_colwise(W)
+    wn = oracle.dequant_1x16(qn[0], qn[1], qn[2], K, N).T  # [N, K]
+    qk = oracle.quantize_1x16(W)
+    wk = oracle.dequant_1x16(qk[0], qk[1], qk[2], N, K)
+    np.testing.assert_array_equal(b["dX"], 24.0 * wn[cols])
+    assert not np.array_equal(b["dX"], 24.0 * wk[cols])
