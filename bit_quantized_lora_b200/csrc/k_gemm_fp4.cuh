@@ -31,11 +31,12 @@
 //   warp 0  TMA producer: per stage, the weight block (codes + scales, one
 //           3-D box) and the activation scale slabs on one barrier, the
 //           activation code tile (128 B swizzle) on another; per tile the
-//           P / L1 / L2 panels.
-//   warp 1  TMEM owner and UMMA issuer: half 0 of the low-rank
-//           up-projection (kind::f16, N = 128), then four
+//           P / L1 / L2 panels, issued once the ring holds the tile's first
+//           stages (they are read after the tile's mainloop).
+//   warp 1  TMEM owner and UMMA issuer: four
 //           tcgen05.mma.kind::mxf4nvf4.block16 (K = 64, N = 256) per stage
-//           into the FP32 accumulator, then low-rank half 1.
+//           into the FP32 accumulator, then the low-rank up-projection
+//           (kind::f16, two halves of N = 128).
 //   warps 2-5  scale warps, one per TMEM lane quarter (2, 3, 0, 1): each
 //           lane loads its 16-byte slab row of every K step from shared
 //           memory and writes it with tcgen05.st into its own lane of a
@@ -241,28 +242,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             uint32_t it = 0;
             bool ok = true;
             int local = 0;
+            // the tile's low-rank panels are needed only after its mainloop:
+            // they are issued once the ring holds the tile's first stages
+            // (by then the previous tile's up-projection, their last
+            // reader, has been issued), so neither their latency nor that
+            // wait holds back the stages
+            const int kt_panel = min(S, KT - 1);
+            int panels_issued = 0;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
                 const int tm = tile / tiles_n, tn = tile % tiles_n;
                 const int m0 = tm * BM, n0 = tn * BN;
-                if (has_lr) {
-                    // low-rank panels first: the first half of the
-                    // up-projection runs before the tile's mainloop
-                    if (!mbar_wait(&bars[B_LR_SMEM_EMPTY], (local & 1) ^ 1, ERR_WAIT_LR, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    uint64_t* lb = &bars[B_LR_FULL];
-                    mbar_arrive_expect_tx(lb, lr_total);
-                    for (int a = 0; a < (p.f1.rf > 0 ? p.f1.natoms : 0); ++a) {
-                        tma_load_2d(smem + L.p1 + a * 128 * p.f1.row_bytes, &p.mapP1, lb, p.f1.pcol + 64 * a, m0);
-                        tma_load_2d(smem + L.l1 + a * 256 * p.f1.row_bytes, &p.mapL1, lb, 64 * a, n0);
-                    }
-                    for (int a = 0; a < (p.f2.rf > 0 ? p.f2.natoms : 0); ++a) {
-                        tma_load_2d(smem + L.p2 + a * 128 * p.f2.row_bytes, &p.mapP2, lb, p.f2.pcol + 64 * a, m0);
-                        tma_load_2d(smem + L.l2 + a * 256 * p.f2.row_bytes, &p.mapL2, lb, 64 * a, n0);
-                    }
-                }
                 for (int kt = 0; kt < KT; ++kt, ++it) {
+                    if (has_lr && kt == kt_panel) {
+                        if (!mbar_wait(&bars[B_LR_SMEM_EMPTY], (local & 1) ^ 1, ERR_WAIT_LR, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        uint64_t* lb = &bars[B_LR_FULL];
+                        mbar_arrive_expect_tx(lb, lr_total);
+                        for (int a = 0; a < (p.f1.rf > 0 ? p.f1.natoms : 0); ++a) {
+                            tma_load_2d(smem + L.p1 + a * 128 * p.f1.row_bytes, &p.mapP1, lb, p.f1.pcol + 64 * a, m0);
+                            tma_load_2d(smem + L.l1 + a * 256 * p.f1.row_bytes, &p.mapL1, lb, 64 * a, n0);
+                        }
+                        for (int a = 0; a < (p.f2.rf > 0 ? p.f2.natoms : 0); ++a) {
+                            tma_load_2d(smem + L.p2 + a * 128 * p.f2.row_bytes, &p.mapP2, lb, p.f2.pcol + 64 * a, m0);
+                            tma_load_2d(smem + L.l2 + a * 256 * p.f2.row_bytes, &p.mapL2, lb, 64 * a, n0);
+                        }
+                        ++panels_issued;
+                    }
                     const int s = it % S;
                     const uint32_t ph = (it / S) & 1;
                     if (!mbar_wait(&bars[B_EMPTY + s], ph ^ 1, ERR_WAIT_EMPTY, abort_flag)) {
@@ -271,8 +278,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     }
                     // the weight block (codes and scales in one copy) and the
                     // activation scale slabs first, on their own barrier: the
-                    // scale warp copies the scales into tensor memory while
-                    // the activation codes are still on their way
+                    // scale warps stage the scales in tensor memory while the
+                    // activation codes are still on their way
                     uint64_t* sfb_bar = &bars[B_SFFULL + s];
                     mbar_arrive_expect_tx(sfb_bar, B_SLOT + SFA_STAGE_BYTES);
                     tma_load_3d(smem + L.b + s * B_SLOT, &p.mapB, sfb_bar, 0, 0, 2 * (tn * KT + kt));
@@ -281,6 +288,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     mbar_arrive_expect_tx(fb, stage_bytes);
                     tma_load_2d(smem + L.a + s * A_BYTES, &p.mapA, fb, kt * BK_BYTES, m0);
                 }
+            }
+            if (!ok && panels_issued > 0) {
+                // the last panel copies land before the CTA exits
+                volatile int no_abort = 0;
+                mbar_wait(&bars[B_LR_FULL], (panels_issued - 1) & 1, ERR_WAIT_DRAIN, &no_abort);
             }
             if (!ok) {
                 // let copies already issued land before the CTA exits
@@ -306,19 +318,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             bool ok = true;
             int local = 0;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
-                if ((has_lr && !mbar_wait(&bars[B_LR_FULL], local & 1, ERR_WAIT_LR, abort_flag)) ||
-                    !mbar_wait(&bars[B_ACC_EMPTY], (local & 1) ^ 1, ERR_WAIT_ACC_EMPTY, abort_flag)) {
+                // the epilogue has read the previous tile's accumulator and
+                // both low-rank halves
+                if (!mbar_wait(&bars[B_ACC_EMPTY], (local & 1) ^ 1, ERR_WAIT_ACC_EMPTY, abort_flag)) {
                     ok = false;
                     break;
-                }
-                tc_fence_after();
-                if (has_lr) {
-                    // half 0 of the up-projection ahead of the mainloop (the
-                    // tensor pipe would otherwise idle waiting for data)
-                    int q = 0;
-                    if (p.f1.rf > 0) lr_mma(tmem + LR0_COL, base + L.p1, base + L.l1, p.f1, 0, idesc_lr, q);
-                    if (p.f2.rf > 0) lr_mma(tmem + LR0_COL, base + L.p2, base + L.l2, p.f2, 0, idesc_lr, q);
-                    tc_commit(&bars[B_LR0_READY]);
                 }
                 tc_fence_after();
                 for (int kt = 0; kt < KT; ++kt, ++it) {
@@ -343,10 +347,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     tc_commit(&bars[B_SF_FREE + sb]);
                 }
                 if (!ok) break;
+                if (has_lr) {
+                    // the up-projection after the mainloop: half 0 at once
+                    // (its own columns), half 1 into the scale ring's columns
+                    // once the mainloop's MMAs, their last readers, are done
+                    if (!mbar_wait(&bars[B_LR_FULL], local & 1, ERR_WAIT_LR, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    int q = 0;
+                    if (p.f1.rf > 0) lr_mma(tmem + LR0_COL, base + L.p1, base + L.l1, p.f1, 0, idesc_lr, q);
+                    if (p.f2.rf > 0) lr_mma(tmem + LR0_COL, base + L.p2, base + L.l2, p.f2, 0, idesc_lr, q);
+                    tc_commit(&bars[B_LR0_READY]);
+                }
                 tc_commit(&bars[B_ACC_FULL]);
                 if (has_lr) {
-                    // half 1 into the scale ring's columns once the mainloop's
-                    // MMAs (the last readers of the scales) have completed
                     if (!mbar_wait(&bars[B_ACC_FULL], local & 1, ERR_WAIT_ACC_FULL, abort_flag)) {
                         ok = false;
                         break;

@@ -23,8 +23,12 @@
 //            Skipped when the caller supplies the tensor amax.
 //   phase 2  the tensor scale and the per-scale divisor table, then every
 //            block is encoded from shared memory with the block maxima kept
-//            in registers since phase 1; codes and scales are staged in
-//            shared memory and leave in coalesced 16-byte / 4-byte stores.
+//            in registers since phase 1; each warp's codes leave straight
+//            from the encode as whole 32-byte sectors (a warp owns 8 rows x
+//            the 4 blocks of a stage), the scale bytes are gathered per row
+//            in shared memory and leave in 4-byte and slab stores.  With a
+//            caller-supplied tensor amax there is no barrier and no phase 1:
+//            each stage is encoded as soon as it lands.
 //   P        as soon as the accumulator is complete (during the barrier),
 //            four helper warps move TMEM (lane = token, column = P column)
 //            to FP32 split partials; in the last CTA of a row tile they add
@@ -36,8 +40,9 @@
 //
 // CTA = 128 rows x one C-range of at most 768 columns (12 stages of 64);
 // warps: 0 TMA producer, 1 TMEM owner + UMMA issuer, 0-3 then the P path
-// (one TMEM lane quarter each), 4-19 quantizers (thread t owns row t % 128
-// and block t / 128 of every 64-column stage) and then the outputs.
+// (one TMEM lane quarter each), 4-19 quantizers (quantizer warp q owns tile
+// rows 8q .. 8q + 7, lane l the block l % 4 of row 8q + l / 4 in every
+// 64-column stage).
 #pragma once
 
 #include <cuda.h>
@@ -113,7 +118,7 @@ __host__ __device__ inline Layout make_layout(int nst, uint32_t ring_bytes) {
     L.x = o;    o += (uint32_t)nst * TILE_BYTES;
     L.f = o;    o += ring_bytes;  // factor ring
     L.sst = o;  o += BM * SROW;   // staged scale bytes
-    L.tab = o;  o += (uint32_t)sizeof(QTableM);
+    L.tab = o;  o += (uint32_t)sizeof(QTable);
     L.bars = o; o += BAR_BYTES;
     L.total = o + 1024;  // slack for the 1 KiB alignment of the base
     return L;
@@ -124,8 +129,7 @@ enum {
     QB_XFULL = 0,                   // [MAX_ST] chunk stage landed (used once)
     QB_FFULL = QB_XFULL + MAX_ST,   // [MAX_FS] factor tiles landed
     QB_FEMPTY = QB_FFULL + MAX_FS,  // [MAX_FS] factor tiles consumed by the MMAs
-    QB_XDONE = QB_FEMPTY + MAX_FS,  // [MAX_ST] the MMAs are done with a chunk stage
-    QB_ACC = QB_XDONE + MAX_ST,     // accumulator complete
+    QB_ACC = QB_FEMPTY + MAX_FS,    // accumulator complete
     QB_DRAIN,                       // every tcgen05 op of the MMA warp done
     QB_COUNT
 };
@@ -213,7 +217,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
     volatile int* last_flag = abort_flag + 1;
     volatile uint32_t* amax_share = reinterpret_cast<volatile uint32_t*>(last_flag + 1);
     volatile uint32_t* red = amax_share + 1;  // [NQ_WARPS]
-    QTableM& tab = *reinterpret_cast<QTableM*>(smem + L.tab);
+    QTable& tab = *reinterpret_cast<QTable*>(smem + L.tab);
 
     const int warp = warp_id(), lane = lane_id();
     const int m0 = blockIdx.x * BM;
@@ -223,10 +227,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
     const int FS = p.fs;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < MAX_ST; ++i) {
-            mbar_init(&bars[QB_XFULL + i], 1);
-            mbar_init(&bars[QB_XDONE + i], 1);
-        }
+        for (int i = 0; i < MAX_ST; ++i) mbar_init(&bars[QB_XFULL + i], 1);
         for (int i = 0; i < MAX_FS; ++i) {
             mbar_init(&bars[QB_FFULL + i], 1);
             mbar_init(&bars[QB_FEMPTY + i], 1);
@@ -321,7 +322,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
                         umma_bf16(tmem, make_desc(a_lo + 2 * j, a_hi), make_desc(b_lo + 32 * j, b_hi), idesc,
                                   (st | j) != 0);
                     tc_commit(&bars[QB_FEMPTY + f]);
-                    tc_commit(&bars[QB_XDONE + st]);
                 }
                 if (ok) tc_commit(&bars[QB_ACC]);
                 tc_commit(&bars[QB_DRAIN]);
@@ -380,42 +380,50 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
         }
     } else {
         // ------------------------------------------------ quantizers
+        // Warp q owns tile rows 8q .. 8q + 7; lane l the block l % 4 of row
+        // 8q + l / 4 in every 64-column stage.  A warp's 32 blocks of a stage
+        // are then 8 rows x 32 contiguous code bytes: its code stores fill
+        // whole 32-byte sectors straight from the encode, and its shared
+        // loads (two 16-byte chunks a lane, 128-byte swizzle) are free of
+        // bank conflicts within each quarter warp.
         const int t = threadIdx.x - NH_THREADS;
-        const int trow = t & (BM - 1), blk = t >> 7;
+        const int qw = t >> 5;
+        const int trow = 8 * qw + (lane >> 2), blk = lane & 3;
         const uint32_t sw = (uint32_t)(trow & 7);
         const uint32_t off_lo = (uint32_t)trow * 128u + (((uint32_t)(2 * blk) ^ sw) << 4);
         const uint32_t off_hi = (uint32_t)trow * 128u + (((uint32_t)(2 * blk + 1) ^ sw) << 4);
+        const bool row_ok = m0 + trow < p.M;
+        uint8_t* crow = p.codes + (int64_t)(m0 + trow) * (p.C / 2) + c0 / 2 + 8 * blk;
+        const uint32_t sstage = base + L.sst;
         bool ok = true;
 
-        // phase 1: block maxima as the stages land (kept for phase 2)
+        // phase 1 (tensor amax computed here): block maxima as the stages
+        // land, kept in registers for phase 2
         uint32_t mb[MAX_ST];
-        uint32_t cmax = 0;
+        float amax_t = 0.0f;
+        if (!p.amax_in) {
+            uint32_t cmax = 0;
 #pragma unroll
-        for (int st = 0; st < MAX_ST; ++st) {
-            mb[st] = 0;
-            if (st < nst && ok) {
-                if (!mbar_wait(&bars[QB_XFULL + st], 0, ERR_WAIT_FULL, abort_flag)) {
-                    ok = false;
-                } else {
-                    const uint32_t ta = base + L.x + st * TILE_BYTES;
-                    const uint4 v0 = ld_shared_v4(ta + off_lo), v1 = ld_shared_v4(ta + off_hi);
-                    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-                    mb[st] = amax_bits_16(w);
-                    cmax = max(cmax, mb[st]);
+            for (int st = 0; st < MAX_ST; ++st) {
+                mb[st] = 0;
+                if (st < nst && ok) {
+                    if (!mbar_wait(&bars[QB_XFULL + st], 0, ERR_WAIT_FULL, abort_flag)) {
+                        ok = false;
+                    } else {
+                        const uint32_t ta = base + L.x + st * TILE_BYTES;
+                        const uint4 v0 = ld_shared_v4(ta + off_lo), v1 = ld_shared_v4(ta + off_hi);
+                        const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                        mb[st] = amax_bits_16(w);
+                        cmax = max(cmax, mb[st]);
+                    }
                 }
             }
-        }
-
-        // tensor amax: CTA max, then the grid-wide max (or the caller's value)
+            // CTA max, then the grid-wide max
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) cmax = max(cmax, __shfl_xor_sync(0xFFFFFFFFu, cmax, o));
-        if (lane == 0) red[warp - NH_WARPS] = cmax;
-        named_bar_sync(1, NQ_THREADS);
-        if (t == 0) {
-            float amax_t;
-            if (p.amax_in) {
-                amax_t = *p.amax_in;
-            } else {
+            for (int o = 16; o > 0; o >>= 1) cmax = max(cmax, __shfl_xor_sync(0xFFFFFFFFu, cmax, o));
+            if (lane == 0) red[qw] = cmax;
+            named_bar_sync(1, NQ_THREADS);
+            if (t == 0) {
                 uint32_t m = 0;
                 for (int i = 0; i < NQ_WARPS; ++i) m = max(m, red[i]);
                 // every CTA arrives, also one that gave up, so no other CTA
@@ -423,7 +431,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
                 // arrival
                 atomicMax(&p.sync[1], (p.epoch << 31) | m);
                 epoch_count_release(&p.sync[0], p.epoch);
-                amax_t = 0.0f;
+                float a_t = 0.0f;
                 if (!epoch_wait(&p.sync[0], p.epoch, p.num_ctas)) {
                     report_error(ERR_GRID_SYNC);
                     *abort_flag = 1;
@@ -434,47 +442,43 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
                         report_error(ERR_GRID_SYNC);
                         *abort_flag = 1;
                     }
-                    amax_t = __uint_as_float((uint32_t)(a & 0x7FFFFFFFull));
+                    a_t = __uint_as_float((uint32_t)(a & 0x7FFFFFFFull));
                 }
+                *amax_share = __float_as_uint(a_t);
             }
-            *amax_share = __float_as_uint(amax_t);
+            named_bar_sync(1, NQ_THREADS);
+            amax_t = __uint_as_float(*amax_share);
+        } else {
+            // the caller's tensor amax: the table is built while the chunk
+            // is still in flight, and each stage is encoded as it lands
+            amax_t = *p.amax_in;
         }
-        named_bar_sync(1, NQ_THREADS);
-        const QTensorFast qt = make_qtensor_fast(__uint_as_float(*amax_share));
-        build_qtable_m1(tab, qt.g, t, NQ_THREADS);
+        const QTensorFast qt = make_qtensor_fast(amax_t);
+        build_qtable(tab, qt.g, t, NQ_THREADS);
         if (blockIdx.x == 0 && blockIdx.y == 0 && t == 0) *p.tscale = qt.g;
-        named_bar_sync(1, NQ_THREADS);
-        build_qtable_m2(tab, t, NQ_THREADS);
-        named_bar_sync(1, NQ_THREADS);
-        build_qtable_m3(tab, t, NQ_THREADS);
         named_bar_sync(1, NQ_THREADS);
         ok = ok && !*abort_flag;
 
-        // phase 2: encode every block from shared memory, the loads one
-        // stage ahead.  A block's 8 code bytes go back into the first half of
-        // its own 16-byte slot once the MMAs are done with that stage (they
-        // run during phase 1 and mostly finish during the barrier), its scale
-        // byte into the [128, SROW] staging array; the output pass then
-        // writes both with coalesced stores.
-        const uint32_t sstage = base + L.sst;
+        // phase 2: encode every block; its 8 code bytes leave at once, its
+        // scale byte joins the row's word (lanes 4r .. 4r + 3) in the
+        // staging array for the scale and slab stores below
         if (ok) {
-            uint4 n0 = ld_shared_v4(base + L.x + off_lo), n1 = ld_shared_v4(base + L.x + off_hi);
 #pragma unroll
             for (int st = 0; st < MAX_ST; ++st) {
                 if (st < nst && ok) {
-                    const uint32_t ta = base + L.x + st * TILE_BYTES;
-                    const uint32_t w[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
-                    if (st + 1 < nst) {
-                        n0 = ld_shared_v4(ta + TILE_BYTES + off_lo);
-                        n1 = ld_shared_v4(ta + TILE_BYTES + off_hi);
-                    }
-                    uint32_t sbyte;
-                    const uint2 q = quant_block16_m(w, mb[st], qt, tab, sbyte);
-                    if (p.do_mma && !mbar_wait(&bars[QB_XDONE + st], 0, ERR_WAIT_ACC_FULL, abort_flag)) {
+                    if (p.amax_in && !mbar_wait(&bars[QB_XFULL + st], 0, ERR_WAIT_FULL, abort_flag)) {
                         ok = false;
                     } else {
-                        st_shared_v2(ta + off_lo, q);
-                        st_shared_u8(sstage + (uint32_t)trow * SROW + st * 4 + blk, sbyte);
+                        const uint32_t ta = base + L.x + st * TILE_BYTES;
+                        const uint4 v0 = ld_shared_v4(ta + off_lo), v1 = ld_shared_v4(ta + off_hi);
+                        const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                        uint32_t sbyte;
+                        const uint2 q = quant_block16_fast_m(w, p.amax_in ? amax_bits_16(w) : mb[st], qt, tab, sbyte);
+                        if (row_ok) *reinterpret_cast<uint2*>(crow + 32 * st) = q;
+                        uint32_t sv = sbyte << (8 * blk);
+                        sv |= __shfl_xor_sync(0xFFFFFFFFu, sv, 1);
+                        sv |= __shfl_xor_sync(0xFFFFFFFFu, sv, 2);
+                        if (blk == 0) st_shared_u32(sstage + (uint32_t)trow * SROW + st * 4, sv);
                     }
                 }
             }
@@ -485,22 +489,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
         if (ok) {
             const int ot = t, on = NQ_THREADS;
             const int rows = min(BM, p.M - m0);
-            // codes: 8-byte pieces (one block), a warp on 8 rows x the 4
-            // blocks of one stage: the pieces sit at the start of 16-byte
-            // slots whose swizzle differs from row to row, so the warp's
-            // shared loads spread over all banks (2 ways), and every row
-            // gets one full 32-byte sector
-            const int ngroups = nst * ((rows + 7) >> 3);
-            for (int i = ot; i < ngroups * 32; i += on) {
-                const int g = i >> 5, l = i & 31;
-                const int rg = g / nst, st = g - rg * nst;
-                const int r = rg * 8 + (l >> 2), b = l & 3;
-                if (r < rows) {
-                    const uint2 v = ld_shared_v2(base + L.x + st * TILE_BYTES + (uint32_t)r * 128u +
-                                                 (((uint32_t)(2 * b) ^ (uint32_t)(r & 7)) << 4));
-                    *reinterpret_cast<uint2*>(p.codes + (int64_t)(m0 + r) * (p.C / 2) + c0 / 2 + 32 * st + 8 * b) = v;
-                }
-            }
             // scales: one 4-byte word per stage of a row
             for (int i = ot; i < rows * nst; i += on) {
                 const int r = i / nst, st = i - r * nst;

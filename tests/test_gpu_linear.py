@@ -62,7 +62,8 @@ def _run_and_compare(shape, seed, M=None, rows=None, r_s=None, r_l=None, bf16_ch
     if layer.r_s + layer.r_l > 0:
         check_lowrank_down(host_u16(P), f["P"], oracle.bf16_to_f64(X), oracle.bf16_to_f64(U),
                            oracle.bf16_to_f64(A), s)
-    _check_elementwise(layer, inp, U, V, qw, f, b, rows, host_u16(P), host(Y), host(dX), host(dA), host(dB))
+    _check_elementwise(layer, inp, U, V, qw, f, b, rows, host_u16(P), host(Y), host(dX),
+                       None if dA is None else host(dA), None if dB is None else host(dB))
     if bf16_check:
         # the BF16 mode rounds the same FP32 value the FP32 mode stores
         Yb, _ = ft.ft_linear_fwd(layer, Xd, out_dtype=ft.BF16)
