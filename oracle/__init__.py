@@ -291,24 +291,51 @@ def _weight_dgrad(W_res, qw, weight_blk):
     raise ValueError(weight_blk)
 
 
-def linear_fwd(X, W_res, U, V, A, B, s: float, rows=None, amax_x=None, qw=None, weight_blk="16x16"):
+PRECISIONS = ("W4A4G4", "W4A16G4", "W4A4G16", "W4A16G16")
+
+
+def _act_bits(precision: str) -> int:
+    """Bits of the activations in the forward GEMM (FourTune page, section
+    4, "Impact of Precision Configurations", Table 4: W4A4G4 is the method;
+    W4A16G4, W4A4G16 and W4A16G16 keep activations and/or gradients at 16
+    bits, the weight always 4-bit)."""
+    if precision not in PRECISIONS:
+        raise ValueError(precision)
+    return 16 if "A16" in precision else 4
+
+
+def _grad_bits(precision: str) -> int:
+    """Bits of the output gradients in the dgrad GEMM (Table 4, as above)."""
+    if precision not in PRECISIONS:
+        raise ValueError(precision)
+    return 16 if "G16" in precision else 4
+
+
+def linear_fwd(X, W_res, U, V, A, B, s: float, rows=None, amax_x=None, qw=None, weight_blk="16x16",
+               precision="W4A4G4"):
     """Forward of the triple-branch layer (Eq. 2).
 
     X: bf16 [M, K]; W_res: bf16 [N, K]; U [K, r_s]; V [N, r_s]; A [K, r_l];
     B [N, r_l].  rows: optional row sample for Y (the quantization and P are
     always computed on the full tensors).  weight_blk: "16x16" (the method)
     or "1x16" (groups along K, the granularity ablation).  qw: optional
-    precomputed quantize_16x16(W_res) (resp. quantize_1x16(W_res)).  Returns
-    a dict with Y (float64 [len(rows), N]), P (bf16 [M, r_s + r_l]),
+    precomputed quantize_16x16(W_res) (resp. quantize_1x16(W_res)).
+    precision: one of PRECISIONS; with 16-bit activations (W4A16G*) the
+    backbone GEMM reads X itself instead of Q(X) (qx is then None).
+    Returns a dict with Y (float64 [len(rows), N]), P (bf16 [M, r_s + r_l]),
     qx = (codes, scales, g) and qw.
     """
     M, K = X.shape
     N = W_res.shape[0]
     rows = np.arange(M) if rows is None else np.asarray(rows)
-    qx = quantize_1x16(X, amax_x)
     qw, Wq = _weight_fwd(W_res, qw, weight_blk)
-    Xq = dequant_1x16(qx[0], qx[1], qx[2], M, K)[rows]
     Xd = bf16_to_f64(X)
+    if _act_bits(precision) == 16:
+        qx = None
+        Xq = Xd[rows]
+    else:
+        qx = quantize_1x16(X, amax_x)
+        Xq = dequant_1x16(qx[0], qx[1], qx[2], M, K)[rows]
     P = _lowrank_down(Xd, U, A, s)
     Pd = bf16_to_f64(P[rows])
     LR = np.concatenate([bf16_to_f64(V), bf16_to_f64(B)], axis=1)  # [N, r_s + r_l]
@@ -317,12 +344,14 @@ def linear_fwd(X, W_res, U, V, A, B, s: float, rows=None, amax_x=None, qw=None, 
 
 
 def linear_bwd(dY, X, W_res, U, V, A, B, s: float, P, rows=None, amax_dy=None, qw=None,
-               weight_blk="16x16"):
+               weight_blk="16x16", precision="W4A4G4"):
     """Backward of the triple-branch layer (Eq. 3 and the LoRA gradients).
 
     dY: bf16 [M, N]; X: bf16 [M, K]; P: the forward's saved bf16 [M, r_s+r_l].
     weight_blk as in linear_fwd; qw: optional precomputed quantize_16x16(W_res)
     (resp. quantize_1x16_colwise(W_res), the dgrad operand of 1x16 weights).
+    precision: one of PRECISIONS; with 16-bit gradients (W4A*G16) the dgrad
+    GEMM reads dY itself instead of Q(dY) (qdy is then None).
     Returns dX (float64 [len(rows), K]), dA (float64 [K, r_l]),
     dB (float64 [N, r_l]), Pg (bf16 [M, r_s + r_l]) and qdy.
     """
@@ -330,10 +359,14 @@ def linear_bwd(dY, X, W_res, U, V, A, B, s: float, P, rows=None, amax_dy=None, q
     K = X.shape[1]
     r_s, r_l = U.shape[1], A.shape[1]
     rows = np.arange(M) if rows is None else np.asarray(rows)
-    qdy = quantize_1x16(dY, amax_dy)
     qw, Wq = _weight_dgrad(W_res, qw, weight_blk)
-    dYq = dequant_1x16(qdy[0], qdy[1], qdy[2], M, N)[rows]
     dYd = bf16_to_f64(dY)
+    if _grad_bits(precision) == 16:
+        qdy = None
+        dYq = dYd[rows]
+    else:
+        qdy = quantize_1x16(dY, amax_dy)
+        dYq = dequant_1x16(qdy[0], qdy[1], qdy[2], M, N)[rows]
     Pg = _lowrank_down(dYd, V, B, s)
     Pgd = bf16_to_f64(Pg)
     LR = np.concatenate([bf16_to_f64(U), bf16_to_f64(A)], axis=1)  # [K, r_s + r_l]

@@ -106,6 +106,44 @@ def test_quantize_transpose_1x16_activations(wl):
         np.testing.assert_array_equal(host(c.scales), sc)
 
 
+@pytest.mark.parametrize("rows,cols,ld", [(16, 16, 16), (48, 144, 144), (80, 208, 216), (208, 400, 400),
+                                          (96, 256, 264), (64, 128, 128)])
+def test_quantize_transpose_ragged_tiles(rows, cols, ld):
+    """Both layouts on shapes that leave partial 64 x 128 tiles (rows or
+    columns not a multiple of the tile, row strides wider than the matrix):
+    every partial store path -- byte scales, 8-byte column-code pieces --
+    writes exactly the oracle's bytes and nothing past them (the outputs are
+    pre-filled with a marker)."""
+    rng = np.random.default_rng(rows * 1000 + cols)
+    full = ft_synth.to_bf16_bits(rng.standard_normal((rows, ld)) * np.exp(rng.standard_normal((rows, ld))))
+    xd = dev_bf16(full)[:, :cols]
+    x = np.ascontiguousarray(full[:, :cols])
+    for blk in (ft.BLK_16x16, ft.BLK_1x16):
+        out_row = ft.FP4.empty(rows, cols, blk, "cuda")
+        if blk == ft.BLK_16x16:
+            out_col = ft.FP4.empty(cols, rows, blk, "cuda", scales=out_row.scales, tscale=out_row.tscale)
+        else:
+            out_col = ft.FP4.empty(cols, rows, blk, "cuda")
+        for t in (out_row.codes, out_row.scales, out_col.codes, out_col.scales):
+            t.fill_(0xA5)
+        ft.ft_quantize_transpose(xd, blk, out_row=out_row, out_col=out_col)
+        torch.cuda.synchronize()
+        if blk == ft.BLK_16x16:
+            cr, cc, sg, g = oracle.quantize_16x16(x)
+            np.testing.assert_array_equal(host(out_row.codes), cr)
+            np.testing.assert_array_equal(host(out_col.codes), cc)
+            np.testing.assert_array_equal(host(out_row.scales), sg)
+        else:
+            cr, sr, g = oracle.quantize_1x16(x)
+            cc, sc, _ = oracle.quantize_1x16_colwise(x)
+            np.testing.assert_array_equal(host(out_row.codes), cr)
+            np.testing.assert_array_equal(host(out_row.scales), sr)
+            np.testing.assert_array_equal(host(out_col.codes), cc)
+            np.testing.assert_array_equal(host(out_col.scales), sc)
+            assert np.float32(host(out_col.tscale)[0]) == np.float32(g)
+        assert np.float32(host(out_row.tscale)[0]) == np.float32(g)
+
+
 def test_supplied_amax_matches_computed():
     rng = np.random.default_rng(32)
     x = ft_synth.to_bf16_bits(rng.standard_normal((64, 128)) * 3)

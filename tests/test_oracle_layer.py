@@ -226,3 +226,44 @@ def test_1x16_dgrad_reads_the_weight_quantized_along_n():
     wk = oracle.dequant_1x16(qk[0], qk[1], qk[2], N, K)
     np.testing.assert_array_equal(b["dX"], 24.0 * wn[cols])
     assert not np.array_equal(b["dX"], 24.0 * wk[cols])
+
+
+def _precision_case(seed, M=32, K=64, N=48, r_s=4, r_l=4, s=0.5):
+    """A weight whose 16x16 quantization is exact (so the 16-bit GEMMs of
+    the precision variants see W_res itself), selection factors (P and Pg
+    exact in bf16), and activations / gradients that are NOT on the E2M1
+    grid: their 4-bit quantization is lossy."""
+    c = _exact_case(seed, M, K, N, r_s, r_l, s)
+    rng = np.random.default_rng(100 + seed)
+    c["X"] = ft_synth.to_bf16_bits(rng.standard_normal((M, K)))
+    c["dY"] = ft_synth.to_bf16_bits(rng.standard_normal((M, N)))
+    return c
+
+
+@pytest.mark.parametrize("precision", ["W4A16G4", "W4A4G16", "W4A16G16"])
+def test_precision_variants_read_the_16bit_operands(precision):
+    """FourTune page, section 4, Table 4: with 16-bit activations the
+    forward's backbone GEMM reads X, with 16-bit gradients the dgrad GEMM
+    reads dY, the weight stays 4-bit.  On a weight whose quantization is
+    exact, each 16-bit side equals float64 autograd of the unquantized layer
+    (a quantized X or dY there would miss it by the quantization error); the
+    4-bit side does not, and the adapter gradients equal autograd's on every
+    variant (they never read a quantized tensor)."""
+    c = _precision_case(3)
+    amax = 2688.0 * 4.0
+    f = oracle.linear_fwd(c["X"], c["Wr"], c["U"], c["V"], c["A"], c["B"], c["s"], qw=c["qw"], precision=precision)
+    b = oracle.linear_bwd(c["dY"], c["X"], c["Wr"], c["U"], c["V"], c["A"], c["B"], c["s"], f["P"], qw=c["qw"],
+                          precision=precision)
+    Y, dX, dA, dB = _torch_layer(c)
+    fwd16, bwd16 = "A16" in precision, "G16" in precision
+    err_y = np.abs(f["Y"] - Y).max() / np.abs(Y).max()
+    err_dx = np.abs(b["dX"] - dX).max() / np.abs(dX).max()
+    assert (err_y < 1e-12) == fwd16 and (err_dx < 1e-12) == bwd16, (err_y, err_dx)
+    assert (f["qx"] is None) == fwd16 and (b["qdy"] is None) == bwd16
+    np.testing.assert_allclose(b["dA"], dA, rtol=1e-12, atol=1e-9)
+    np.testing.assert_allclose(b["dB"], dB, rtol=1e-12, atol=1e-9)
+    # the 4-bit method itself misses on both sides on these inputs
+    f4 = oracle.linear_fwd(c["X"], c["Wr"], c["U"], c["V"], c["A"], c["B"], c["s"], amax_x=amax, qw=c["qw"])
+    assert np.abs(f4["Y"] - Y).max() / np.abs(Y).max() > 1e-3
+    with pytest.raises(ValueError):
+        oracle.linear_fwd(c["X"], c["Wr"], c["U"], c["V"], c["A"], c["B"], c["s"], precision="W4A8G4")
