@@ -22,9 +22,14 @@ BLK_1x16 = 0
 BLK_16x16 = 1
 BF16 = 0
 F32 = 1
+# precision configurations (the FourTune page's Table 4); the weight is
+# always 4-bit, bit 0 = 16-bit activations, bit 1 = 16-bit gradients
+W4A4G4, W4A16G4, W4A4G16, W4A16G16 = 0, 1, 2, 3
+PRECISIONS = {"W4A4G4": W4A4G4, "W4A16G4": W4A16G4, "W4A4G16": W4A4G16, "W4A16G16": W4A16G16}
 
 __all__ = [
     "FP4", "Layer", "FtError", "BLK_1x16", "BLK_16x16", "BF16", "F32",
+    "W4A4G4", "W4A16G4", "W4A4G16", "W4A16G16", "PRECISIONS", "ft_dequant_weight_operands",
     "ft_quantize", "ft_quantize_transpose", "ft_linear_fwd", "ft_linear_bwd",
     "ft_workspace_bytes", "ft_quantize_workspace_bytes", "ft_device_error",
     "ft_set_cooperative_quantizer", "prepare_layer", "svd_split", "Workspace", "timing",
@@ -168,11 +173,14 @@ class Layer:
     B: torch.Tensor | None
     op_k: torch.Tensor | None = None  # the GEMM's image of w_k (codes + per-row scales)
     op_n: torch.Tensor | None = None  # ... and of w_n
+    precision: int = W4A4G4           # W4A4G4 (the method) or a 16-bit variant
+    wd_k: torch.Tensor | None = None  # bf16 image of Q(W_res) [N, K] (16-bit activations)
+    wd_n: torch.Tensor | None = None  # ... transposed [K, N] (16-bit gradients)
 
     def view(self) -> FtLinear:
         return FtLinear(self.N, self.K, self.r_s, self.r_l, self.s, self.w_k.view(), self.w_n.view(),
                         _ptr(self.U), _ptr(self.V), _ptr(self.A), _ptr(self.B), _ptr(self.op_k),
-                        _ptr(self.op_n))
+                        _ptr(self.op_n), int(self.precision), _ptr(self.wd_k), _ptr(self.wd_n))
 
 
 def _bf16_rne(x: torch.Tensor) -> torch.Tensor:
@@ -213,11 +221,13 @@ def svd_split(W: torch.Tensor, r_s: int):
 def prepare_layer(W: torch.Tensor | None = None, r_s: int = 0, A: torch.Tensor | None = None,
                   B: torch.Tensor | None = None, s: float = 1.0, *, U=None, V=None, W_res=None,
                   amax: torch.Tensor | None = None, ws: Workspace | None = None,
-                  weight_blk: int = BLK_16x16) -> Layer:
+                  weight_blk: int = BLK_16x16, precision: int | str = W4A4G4) -> Layer:
     """Once-per-layer preparation: split W (or take a given U, V, W_res) and
     quantize W_res into both code layouts in one pass: 16x16 blocks (the
     method), or with weight_blk=BLK_1x16 the granularity ablation's 1x16
-    groups (W_res along K and, independently, W_res^T along N)."""
+    groups (W_res along K and, independently, W_res^T along N).  precision:
+    W4A4G4 (the method) or a 16-bit variant ("W4A16G4", "W4A4G16",
+    "W4A16G16"), for which the bf16 weight images are built as well."""
     if W_res is None:
         U, V, W_res = svd_split(W, r_s)
     _bf16(W_res, "W_res")
@@ -226,8 +236,27 @@ def prepare_layer(W: torch.Tensor | None = None, r_s: int = 0, A: torch.Tensor |
     r_l = 0 if A is None else A.shape[1]
     w_k, w_n = ft_quantize_transpose(W_res.contiguous(), weight_blk, amax=amax, ws=ws)
     op_k, op_n = ft_pack_weight_operands(w_k, w_n, N, K)
+    prec = PRECISIONS[precision] if isinstance(precision, str) else int(precision)
+    wd_k, wd_n = ft_dequant_weight_operands(w_k, w_n, fwd=bool(prec & W4A16G4), dgrad=bool(prec & W4A4G16))
     return Layer(N, K, r_s, r_l, float(s), w_k, w_n, U, V,
-                 None if A is None else A.contiguous(), None if B is None else B.contiguous(), op_k, op_n)
+                 None if A is None else A.contiguous(), None if B is None else B.contiguous(), op_k, op_n,
+                 prec, wd_k, wd_n)
+
+
+def ft_dequant_weight_operands(w_k: FP4, w_n: FP4, fwd: bool = True, dgrad: bool = True, stream=None):
+    """bf16 images of Q(W_res) for the 16-bit GEMMs of the precision
+    variants: (wd_k [N, K] if fwd, wd_n [K, N] if dgrad), e2m1 value x block
+    scale (exact; the tensor scale stays in w_k.tscale).  (None, None) when
+    neither is asked for."""
+    if not fwd and not dgrad:
+        return None, None
+    dev = w_k.codes.device
+    wd_k = torch.empty(w_k.rows, w_k.cols, dtype=torch.bfloat16, device=dev) if fwd else None
+    wd_n = torch.empty(w_k.cols, w_k.rows, dtype=torch.bfloat16, device=dev) if dgrad else None
+    vk, vn = w_k.view(), w_n.view()
+    check("ft_dequant_weight_operands", load().ft_dequant_weight_operands(
+        ctypes.byref(vk), ctypes.byref(vn), _ptr(wd_k), _ptr(wd_n), _stream(stream)))
+    return wd_k, wd_n
 
 
 def ft_pack_weight_operands(w_k, w_n, N: int, K: int, stream=None):

@@ -37,6 +37,9 @@ class FtLinear(ctypes.Structure):
         ("B", c_vp),
         ("op_k", c_vp),
         ("op_n", c_vp),
+        ("precision", ctypes.c_int32),
+        ("wd_k", c_vp),
+        ("wd_n", c_vp),
     ]
 
 
@@ -51,6 +54,8 @@ SIGNATURES = {
                                      c_vp, c_vp, ctypes.c_size_t, c_vp]),
     "ft_linear_bwd": (ctypes.c_int, [ctypes.POINTER(FtLinear), c_vp, c_vp, c_vp, c_i64, c_vp, c_vp,
                                      ctypes.c_int, c_vp, c_vp, c_vp, ctypes.c_size_t, c_vp]),
+    "ft_dequant_weight_operands": (ctypes.c_int, [ctypes.POINTER(FtFp4), ctypes.POINTER(FtFp4), c_vp, c_vp,
+                                                  c_vp]),
     "ft_workspace_bytes": (ctypes.c_size_t, [c_i64, c_i64, c_i64, c_i64, c_i64]),
     "ft_quantize_workspace_bytes": (ctypes.c_size_t, []),
     "ft_weight_operand_bytes": (ctypes.c_size_t, [c_i64, c_i64]),

@@ -100,7 +100,9 @@ ft_status device_info(DevInfo** out) {
     }
     if (!d.attr_set) {
         const int big = 227 * 1024;
-        if (cudaFuncSetAttribute(ft::gemm::k_gemm_fp4, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(ft::gemm::k_gemm_fp4<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 big) != cudaSuccess ||
+            cudaFuncSetAttribute(ft::gemm::k_gemm_fp4<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  big) != cudaSuccess ||
             cudaFuncSetAttribute(ft::qdown::k_qdown, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)ft::qdown::SMEM_BYTES) != cudaSuccess ||
@@ -112,7 +114,8 @@ ft_status device_info(DevInfo** out) {
         // one shared-memory carveout (the largest) for every kernel of a
         // step, so that no SM has to re-partition L1 between two of them
         const void* kernels[] = {
-            reinterpret_cast<const void*>(ft::gemm::k_gemm_fp4),
+            reinterpret_cast<const void*>(ft::gemm::k_gemm_fp4<false>),
+            reinterpret_cast<const void*>(ft::gemm::k_gemm_fp4<true>),
             reinterpret_cast<const void*>(ft::qres::k_qres),
             reinterpret_cast<const void*>(ft::qdown::k_qdown),
             reinterpret_cast<const void*>(ft::lgrad::k_lora_grad),
@@ -183,11 +186,14 @@ enum KernelId {
     KID_LORA_GRAD,
     KID_LORA_REDUCE,
     KID_QRES,
+    KID_GEMM_BF16,
+    KID_DEQUANT_W,
     KID_COUNT
 };
 const char* const kKernelNames[KID_COUNT] = {
     "k_amax_bf16", "k_quant_1x16", "k_quant_tile16", "k_pack_lt", "k_qdown",
-    "k_lowrank_finalize", "k_gemm_fp4", "k_lora_grad", "k_lora_grad_reduce", "k_qres"};
+    "k_lowrank_finalize", "k_gemm_fp4", "k_lora_grad", "k_lora_grad_reduce", "k_qres",
+    "k_gemm_bf16", "k_dequant_w"};
 
 struct TimingRec {
     cudaEvent_t a, b;
@@ -374,24 +380,20 @@ ft_status run_quant_1x16(const void* x, int64_t rows, int64_t cols, int64_t ld, 
 
 ft_status run_tile16(bool mode16x16, const void* x, int64_t rows, int64_t cols, int64_t ld,
                      const float* amax, uint8_t* codes_row, uint8_t* scales_row, uint8_t* codes_col,
-                     uint8_t* scales_col, float* tscale, float* tscale2, cudaStream_t st) {
-    dim3 grid((unsigned)cdiv(cols / 16, 8), (unsigned)(rows / 16));
+                     uint8_t* scales_col, float* tscale, float* tscale2, const DevInfo* d, cudaStream_t st) {
+    // persistent CTAs over the 64 x 128 tiles, a few per SM
+    const int64_t tiles = ((rows + 63) / 64) * ((cols + 127) / 128);
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, (int64_t)d->sms * 6));
+    LaunchTimer _lt(KID_QUANT_TILE16, st);
     if (mode16x16)
-        {
-            LaunchTimer _lt(KID_QUANT_TILE16, st);
-            ft::k_quant_tile16<true><<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(x), rows, cols, ld,
-                                                           amax, codes_row, scales_row, codes_col,
-                                                           scales_col, tscale, tscale2);
-            _lt.stop();
-        }
+        ft::k_quant_tile16<true><<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(x), rows, cols, ld, amax,
+                                                       codes_row, scales_row, codes_col, scales_col, tscale,
+                                                       tscale2);
     else
-        {
-            LaunchTimer _lt(KID_QUANT_TILE16, st);
-            ft::k_quant_tile16<false><<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(x), rows, cols, ld,
-                                                            amax, codes_row, scales_row, codes_col,
-                                                            scales_col, tscale, tscale2);
-            _lt.stop();
-        }
+        ft::k_quant_tile16<false><<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(x), rows, cols, ld, amax,
+                                                        codes_row, scales_row, codes_col, scales_col, tscale,
+                                                        tscale2);
+    _lt.stop();
     return last_launch();
 }
 
@@ -665,16 +667,24 @@ CUtensorMapSwizzle swizzle_for(int wbox) {
 }
 
 // out[M, Nout] = ga gb Q(A) Q(B)^T + P[:, :r1] L1^T + P[:, r1:] L2^T, the
-// block scales of A and B given as slabs ([rows/128][Kc/64][512]).
-ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_slab, const float* ga, int64_t M,
+// block scales of A and B given as slabs ([rows/128][Kc/64][512]).  bf16:
+// the 16-bit variant, out = gb A B^T + ..., with A = a_codes a bf16 [M, Kc]
+// matrix and B = b_op the weight's bf16 image [Nout, Kc] (a_slab and ga
+// unused).
+ft_status run_gemm(bool bf16, const uint8_t* a_codes, const uint8_t* a_slab, const float* ga, int64_t M,
                    int64_t Kc, const uint8_t* b_op, const float* gb,
                    int64_t Nout, const void* P, const void* L1, int64_t r1, const void* L2, int64_t r2,
                    void* out, ft_dtype ot, const DevInfo* d, cudaStream_t st, DepFlag dep) {
     Params p;
     std::memset(&p, 0, sizeof(p));
-    FT_TRY(encode_2d(&p.mapA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, Kc / 2, M, Kc / 2, 128, 128,
-                     CU_TENSOR_MAP_SWIZZLE_128B));
-    {
+    if (bf16) {
+        FT_TRY(encode_2d(&p.mapA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a_codes, Kc, M, Kc * 2, 64, 128,
+                         CU_TENSOR_MAP_SWIZZLE_128B));
+        FT_TRY(encode_2d(&p.mapB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, b_op, Kc, Nout, Kc * 2, 64, 256,
+                         CU_TENSOR_MAP_SWIZZLE_128B));
+    } else {
+        FT_TRY(encode_2d(&p.mapA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, Kc / 2, M, Kc / 2, 128, 128,
+                         CU_TENSOR_MAP_SWIZZLE_128B));
         // the weight's operand image (ft_pack_weight_operands) as a 3-D byte
         // tensor {128, 144, 2 * blocks}: one block (codes + scales of a
         // 256-row tile for one stage) is one box of {128, 144, 2}
@@ -686,6 +696,7 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_slab, const float* g
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return FT_ERR_CUDA;
+        FT_TRY(encode_slabs(&p.mapSFA, a_slab, Kc / 64, cdiv(M, 128), 1));
     }
     const int64_t r = r1 + r2;
     p.f1 = gemm_factor(r1, 0);
@@ -706,8 +717,7 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_slab, const float* g
     p.dep_done = dep.done;
     p.dep_epoch = dep.epoch;
     p.dep_count = dep.count;
-    FT_TRY(encode_slabs(&p.mapSFA, a_slab, Kc / 64, cdiv(M, 128), 1));
-    p.ga = ga;
+    p.ga = bf16 ? nullptr : ga;
     p.gb = gb;
     p.out_f32 = (ot == FT_F32);
     p.M = (int)M;
@@ -721,8 +731,13 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_slab, const float* g
     const int tiles = cdiv(M, ft::gemm::BM) * (int)(Nout / ft::gemm::BN);
     const int grid = std::max(1, std::min(tiles, d->sms));
     {
-        LaunchTimer _lt(KID_GEMM, st);
-        FT_TRY(launch_overlapped(ft::gemm::k_gemm_fp4, dim3((unsigned)grid), dim3(ft::gemm::NUM_THREADS), smem, st, p));
+        LaunchTimer _lt(bf16 ? KID_GEMM_BF16 : KID_GEMM, st);
+        if (bf16)
+            FT_TRY(launch_overlapped(ft::gemm::k_gemm_fp4<true>, dim3((unsigned)grid), dim3(ft::gemm::NUM_THREADS),
+                                     smem, st, p));
+        else
+            FT_TRY(launch_overlapped(ft::gemm::k_gemm_fp4<false>, dim3((unsigned)grid), dim3(ft::gemm::NUM_THREADS),
+                                     smem, st, p));
         _lt.stop();
     }
     return last_launch();
@@ -812,6 +827,10 @@ ft_status check_linear(const ft_linear* L) {
         return FT_ERR_ALIGN;
     if (!L->op_k || !L->op_n) return FT_ERR_INVALID_ARG;
     if (!al16(L->op_k) || !al16(L->op_n)) return FT_ERR_ALIGN;
+    if (L->precision < FT_W4A4G4 || L->precision > FT_W4A16G16) return FT_ERR_INVALID_ARG;
+    if ((L->precision & FT_W4A16G4) && !L->wd_k) return FT_ERR_INVALID_ARG;
+    if ((L->precision & FT_W4A4G16) && !L->wd_n) return FT_ERR_INVALID_ARG;
+    if ((L->wd_k && !al16(L->wd_k)) || (L->wd_n && !al16(L->wd_n))) return FT_ERR_ALIGN;
     return FT_OK;
 }
 
@@ -874,6 +893,44 @@ ft_status ft_pack_weight_operands_1x16(const uint8_t* codes_k, const uint8_t* sc
     FT_TRY(last_launch());
     ft::k_pack_wop<<<grid_n, 256, 0, st>>>(codes_n, nullptr, scales_n, N, K, 1, op_n);
     return last_launch();
+}
+
+ft_status ft_dequant_weight_operands(const ft_fp4* w_k, const ft_fp4* w_n, void* wd_k, void* wd_n, void* stream) {
+    if (!w_k || (!wd_k && !wd_n) || (wd_n && !w_n)) return FT_ERR_INVALID_ARG;
+    const ft_block blk = w_k->blk;
+    if (blk != FT_BLK_1x16 && blk != FT_BLK_16x16) return FT_ERR_INVALID_ARG;
+    const int64_t N = w_k->rows, K = w_k->cols;
+    if (N < 0 || K < 0) return FT_ERR_INVALID_ARG;
+    if (N % 16 || K % 16) return FT_ERR_SHAPE;
+    if (!w_k->codes || !w_k->scales) return FT_ERR_INVALID_ARG;
+    if (wd_n) {
+        if (!w_n->codes || w_n->blk != blk) return FT_ERR_INVALID_ARG;
+        if (w_n->rows != K || w_n->cols != N) return FT_ERR_SHAPE;
+        if (blk == FT_BLK_1x16 && !w_n->scales) return FT_ERR_INVALID_ARG;
+        if (!al16(w_n->codes) || !al16(wd_n)) return FT_ERR_ALIGN;
+    }
+    if (!al16(w_k->codes) || (wd_k && !al16(wd_k))) return FT_ERR_ALIGN;
+    if (N == 0 || K == 0) return FT_OK;
+    DevInfo* d;
+    FT_TRY(device_info(&d));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(N * K / 8, 256), (int64_t)d->sms * 16));
+    if (wd_k) {
+        LaunchTimer _lt(KID_DEQUANT_W, st);
+        ft::k_dequant_w<<<grid, 256, 0, st>>>(w_k->codes, w_k->scales, N, K, blk == FT_BLK_16x16 ? 0 : 2,
+                                              static_cast<uint16_t*>(wd_k));
+        _lt.stop();
+        FT_TRY(last_launch());
+    }
+    if (wd_n) {
+        // 16x16: the codes packed along N with the one grid read transposed
+        LaunchTimer _lt(KID_DEQUANT_W, st);
+        ft::k_dequant_w<<<grid, 256, 0, st>>>(w_n->codes, blk == FT_BLK_16x16 ? w_k->scales : w_n->scales, K, N,
+                                              blk == FT_BLK_16x16 ? 1 : 2, static_cast<uint16_t*>(wd_n));
+        _lt.stop();
+        FT_TRY(last_launch());
+    }
+    return FT_OK;
 }
 
 size_t ft_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t r_l) {
@@ -946,7 +1003,7 @@ ft_status ft_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, ft_
     if (blk == FT_BLK_1x16)
         return run_quant_1x16(x, rows, cols, ld, a, out->codes, out->scales, out->tscale, nullptr, d, st);
     return run_tile16(true, x, rows, cols, ld, a, out->codes, out->scales, nullptr, nullptr,
-                      out->tscale, nullptr, st);
+                      out->tscale, nullptr, d, st);
 }
 
 ft_status ft_quantize_transpose(const void* x, int64_t rows, int64_t cols, int64_t ld,
@@ -983,10 +1040,10 @@ ft_status ft_quantize_transpose(const void* x, int64_t rows, int64_t cols, int64
     }
     if (blk == FT_BLK_16x16)
         return run_tile16(true, x, rows, cols, ld, a, out_row->codes, out_row->scales,
-                          out_col->codes, nullptr, out_row->tscale, nullptr, st);
+                          out_col->codes, nullptr, out_row->tscale, nullptr, d, st);
     return run_tile16(false, x, rows, cols, ld, a, out_row->codes, out_row->scales, out_col->codes,
                       out_col->scales, out_row->tscale,
-                      out_col->tscale != out_row->tscale ? out_col->tscale : nullptr, st);
+                      out_col->tscale != out_row->tscale ? out_col->tscale : nullptr, d, st);
 }
 
 ft_status ft_linear_fwd(const ft_linear* L, const void* X, int64_t M, const float* amax_x, void* Y,
@@ -1011,7 +1068,11 @@ ft_status ft_linear_fwd(const ft_linear* L, const void* X, int64_t M, const floa
     DepFlag dep;
     FT_TRY(run_quant_down(X, M, L->K, L->U, L->r_s, L->A, L->r_l, L->s, amax_x, codes, scales, g_x,
                           P_save, wsb, w, d, st, &dep));
-    return run_gemm(codes, wsb + w.sfslab, g_x, M, L->K, L->op_k, L->w_k.tscale, L->N,
+    if (L->precision & FT_W4A16G4)  // 16-bit activations: the GEMM reads X itself
+        return run_gemm(true, static_cast<const uint8_t*>(X), nullptr, nullptr, M, L->K,
+                        static_cast<const uint8_t*>(L->wd_k), L->w_k.tscale, L->N, P_save, L->V, L->r_s, L->B,
+                        L->r_l, Y, yt, d, st, dep);
+    return run_gemm(false, codes, wsb + w.sfslab, g_x, M, L->K, L->op_k, L->w_k.tscale, L->N,
                     P_save, L->V, L->r_s, L->B, L->r_l, Y, yt, d, st, dep);
 }
 
@@ -1051,8 +1112,13 @@ ft_status ft_linear_bwd(const ft_linear* L, const void* dY, const void* X, const
     DepFlag dep;
     FT_TRY(run_quant_down(dY, M, L->N, L->V, L->r_s, L->B, L->r_l, L->s, amax_dy, codes, scales, g_dy,
                           Pg, wsb, w, d, st, &dep));
-    FT_TRY(run_gemm(codes, wsb + w.sfslab, g_dy, M, L->N, L->op_n, L->w_k.tscale, L->K,
-                    Pg, L->U, L->r_s, L->A, L->r_l, dX, xt, d, st, dep));
+    if (L->precision & FT_W4A4G16)  // 16-bit gradients: the dgrad GEMM reads dY itself
+        FT_TRY(run_gemm(true, static_cast<const uint8_t*>(dY), nullptr, nullptr, M, L->N,
+                        static_cast<const uint8_t*>(L->wd_n), L->w_k.tscale, L->K, Pg, L->U, L->r_s, L->A, L->r_l,
+                        dX, xt, d, st, dep));
+    else
+        FT_TRY(run_gemm(false, codes, wsb + w.sfslab, g_dy, M, L->N, L->op_n, L->w_k.tscale, L->K,
+                        Pg, L->U, L->r_s, L->A, L->r_l, dX, xt, d, st, dep));
     // the adapter gradients read dY, X, P_save and Pg: nothing the dgrad GEMM
     // (the kernel they overlap) writes, so they wait on the quantizer's
     // counter for Pg, not on the GEMM

@@ -179,6 +179,15 @@ __device__ __forceinline__ void lr_mma(uint32_t tmem_d, uint32_t pa, uint32_t pb
     }
 }
 
+// kBf16 = false: the 4-bit backbone GEMM (both operands NVFP4, block
+// scales staged in tensor memory); a 256-deep stage is four K = 64 MMAs.
+// kBf16 = true: the 16-bit variant of the precision ablation (FourTune
+// page, section 4, Table 4): A = a bf16 activation or gradient, B = the
+// weight's bf16 image (E2M1 value x block scale, exact in bf16; the tensor
+// scale stays apart as gb), tcgen05 kind::f16; a stage holds 64 columns of
+// K in the same 128-byte rows, four K = 16 MMAs.  No scale factors: the
+// scale warps idle.  Tiles, epilogue and low-rank terms are shared.
+template <bool kBf16>
 __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
@@ -195,7 +204,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
     const int tiles_m = (p.M + BM - 1) / BM;
     const int tiles_n = p.Nout / BN;
     const int num_tiles = tiles_m * tiles_n;
-    const int KT = p.Kc / 256;  // stages per tile
+    const int KT = kBf16 ? p.Kc / 64 : p.Kc / 256;  // stages per tile
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < MAX_STAGES; ++i) {
@@ -220,7 +229,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&p.mapA);
         tma_prefetch_desc(&p.mapB);
-        tma_prefetch_desc(&p.mapSFA);
+        if (!kBf16) tma_prefetch_desc(&p.mapSFA);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, TMEM_COLS);
@@ -276,6 +285,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                         ok = false;
                         break;
                     }
+                    if (kBf16) {
+                        // A [128 rows x 64 columns] and B [256 x 64], bf16
+                        uint64_t* fb = &bars[B_FULL + s];
+                        mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
+                        tma_load_2d(smem + L.b + s * B_SLOT, &p.mapB, fb, kt * 64, n0);
+                        tma_load_2d(smem + L.a + s * A_BYTES, &p.mapA, fb, kt * 64, m0);
+                        continue;
+                    }
                     // the weight block (codes and scales in one copy) and the
                     // activation scale slabs first, on their own barrier: the
                     // scale warps stage the scales in tensor memory while the
@@ -299,7 +316,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                 for (int d = 0; d < S && d < (int)it; ++d) {
                     uint32_t j = it - 1 - d;
                     volatile int no_abort = 0;
-                    mbar_wait(&bars[B_SFFULL + (j % S)], (j / S) & 1, ERR_WAIT_DRAIN, &no_abort);
+                    if (!kBf16) mbar_wait(&bars[B_SFFULL + (j % S)], (j / S) & 1, ERR_WAIT_DRAIN, &no_abort);
                     mbar_wait(&bars[B_FULL + (j % S)], (j / S) & 1, ERR_WAIT_DRAIN, &no_abort);
                 }
             }
@@ -307,7 +324,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
     } else if (warp == 1) {
         // ------------------------------------------------ UMMA issuer
         if (lane == 0) {
-            const uint32_t idesc = idesc_nvfp4(BM, BN);
+            const uint32_t idesc = kBf16 ? idesc_bf16(BM, BN, 0, 0) : idesc_nvfp4(BM, BN);
             const uint32_t idesc_lr = idesc_bf16(BM, 128, 0, 0);
             // descriptor words: lo = start >> 4 | (LBO >> 4) << 16;
             // hi = SBO >> 4 | version 1 << 14 | layout << 29
@@ -329,14 +346,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     const int s = it % S;
                     const int sb = it & 1;
                     if (!mbar_wait(&bars[B_FULL + s], (it / S) & 1, ERR_WAIT_FULL, abort_flag) ||
-                        !mbar_wait(&bars[B_SFFULL + s], (it / S) & 1, ERR_WAIT_FULL, abort_flag) ||
-                        !mbar_wait(&bars[B_SF_READY + sb], (it >> 1) & 1, ERR_WAIT_SF, abort_flag)) {
+                        (!kBf16 && (!mbar_wait(&bars[B_SFFULL + s], (it / S) & 1, ERR_WAIT_FULL, abort_flag) ||
+                                    !mbar_wait(&bars[B_SF_READY + sb], (it >> 1) & 1, ERR_WAIT_SF, abort_flag)))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t a_lo = a_lo0 + s * (A_BYTES >> 4);
                     const uint32_t b_lo = b_lo0 + s * (B_SLOT >> 4);
+                    if (kBf16) {
+                        // a K = 16 step is 32 bytes of each 128-byte row
+#pragma unroll
+                        for (int j = 0; j < KSTEPS; ++j)
+                            umma_bf16(tmem + ACC_COL, make_desc(a_lo + 2 * j, hi_sw128),
+                                      make_desc(b_lo + 2 * j, hi_sw128), idesc, (kt | j) != 0);
+                        tc_commit(&bars[B_EMPTY + s]);
+                        continue;
+                    }
                     const uint32_t sf = tmem + R2_COL + sb * SF_SLOT_COLS;
 #pragma unroll
                     for (int j = 0; j < KSTEPS; ++j)
@@ -382,55 +408,57 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
         }
         __syncwarp();
     } else if (warp < EPI_WARP0) {
-        // ------------------------------------------------ scale warps
-        // Warp q (= warp % 4) writes TMEM lanes 32q .. 32q + 31; its lane i
-        // stores slab row i of every K step (16 bytes each) into its own
-        // lane: the contents a tcgen05.cp 32x128b.warpx4 of each slab would
-        // leave in every lane quarter, written by the TMEM store path
-        // instead of the tensor pipe.
-        const uint32_t lane_addr = (uint32_t)(32 * (warp & 3)) << 16;
-        uint32_t it = 0;
-        bool ok = true;
-        int local = 0;
-        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
-            // the ring's columns hold the previous tile's low-rank half 1
-            // until its epilogue is done
-            if (has_lr && local > 0 &&
-                !mbar_wait(&bars[B_ACC_EMPTY], (local - 1) & 1, ERR_WAIT_SF, abort_flag)) {
-                ok = false;
-                break;
-            }
-            for (int kt = 0; kt < KT; ++kt, ++it) {
-                const int s = it % S;
-                const int sb = it & 1;
-                if (!mbar_wait(&bars[B_SFFULL + s], (it / S) & 1, ERR_WAIT_FULL, abort_flag) ||
-                    !mbar_wait(&bars[B_SF_FREE + sb], ((it >> 1) & 1) ^ 1, ERR_WAIT_SF, abort_flag)) {
+        if constexpr (!kBf16) {  // no block scales in the 16-bit variant
+            // ------------------------------------------------ scale warps
+            // Warp q (= warp % 4) writes TMEM lanes 32q .. 32q + 31; its lane i
+            // stores slab row i of every K step (16 bytes each) into its own
+            // lane: the contents a tcgen05.cp 32x128b.warpx4 of each slab would
+            // leave in every lane quarter, written by the TMEM store path
+            // instead of the tensor pipe.
+            const uint32_t lane_addr = (uint32_t)(32 * (warp & 3)) << 16;
+            uint32_t it = 0;
+            bool ok = true;
+            int local = 0;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+                // the ring's columns hold the previous tile's low-rank half 1
+                // until its epilogue is done
+                if (has_lr && local > 0 &&
+                    !mbar_wait(&bars[B_ACC_EMPTY], (local - 1) & 1, ERR_WAIT_SF, abort_flag)) {
                     ok = false;
                     break;
                 }
-                tc_fence_after();
-                const uint32_t sfa = base + L.sfa + (uint32_t)s * SFA_STAGE_BYTES + 16u * (uint32_t)lane;
-                const uint32_t sfb = base + L.b + (uint32_t)s * B_SLOT + B_BYTES + 16u * (uint32_t)lane;
-                uint32_t ra[16], rb[32];
-#pragma unroll
-                for (int j = 0; j < KSTEPS; ++j) {
-                    const uint4 va = ld_shared_v4(sfa + 512u * j);
-                    const uint4 vl = ld_shared_v4(sfb + 512u * j);
-                    const uint4 vh = ld_shared_v4(sfb + (uint32_t)SFA_STAGE_BYTES + 512u * j);
-                    ra[4 * j] = va.x; ra[4 * j + 1] = va.y; ra[4 * j + 2] = va.z; ra[4 * j + 3] = va.w;
-                    rb[8 * j] = vl.x; rb[8 * j + 1] = vl.y; rb[8 * j + 2] = vl.z; rb[8 * j + 3] = vl.w;
-                    rb[8 * j + 4] = vh.x; rb[8 * j + 5] = vh.y; rb[8 * j + 6] = vh.z; rb[8 * j + 7] = vh.w;
+                for (int kt = 0; kt < KT; ++kt, ++it) {
+                    const int s = it % S;
+                    const int sb = it & 1;
+                    if (!mbar_wait(&bars[B_SFFULL + s], (it / S) & 1, ERR_WAIT_FULL, abort_flag) ||
+                        !mbar_wait(&bars[B_SF_FREE + sb], ((it >> 1) & 1) ^ 1, ERR_WAIT_SF, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sfa = base + L.sfa + (uint32_t)s * SFA_STAGE_BYTES + 16u * (uint32_t)lane;
+                    const uint32_t sfb = base + L.b + (uint32_t)s * B_SLOT + B_BYTES + 16u * (uint32_t)lane;
+                    uint32_t ra[16], rb[32];
+    #pragma unroll
+                    for (int j = 0; j < KSTEPS; ++j) {
+                        const uint4 va = ld_shared_v4(sfa + 512u * j);
+                        const uint4 vl = ld_shared_v4(sfb + 512u * j);
+                        const uint4 vh = ld_shared_v4(sfb + (uint32_t)SFA_STAGE_BYTES + 512u * j);
+                        ra[4 * j] = va.x; ra[4 * j + 1] = va.y; ra[4 * j + 2] = va.z; ra[4 * j + 3] = va.w;
+                        rb[8 * j] = vl.x; rb[8 * j + 1] = vl.y; rb[8 * j + 2] = vl.z; rb[8 * j + 3] = vl.w;
+                        rb[8 * j + 4] = vh.x; rb[8 * j + 5] = vh.y; rb[8 * j + 6] = vh.z; rb[8 * j + 7] = vh.w;
+                    }
+                    const uint32_t sf = tmem + lane_addr + R2_COL + (uint32_t)sb * SF_SLOT_COLS;
+                    tmem_st_32x32b_x16(sf, ra);
+                    tmem_st_32x32b_x32(sf + 16, rb);
+                    tmem_st_wait();
+                    // the slab bytes were read through the generic proxy; the
+                    // stage goes back to TMA after the MMAs
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars[B_SF_READY + sb]);
                 }
-                const uint32_t sf = tmem + lane_addr + R2_COL + (uint32_t)sb * SF_SLOT_COLS;
-                tmem_st_32x32b_x16(sf, ra);
-                tmem_st_32x32b_x32(sf + 16, rb);
-                tmem_st_wait();
-                // the slab bytes were read through the generic proxy; the
-                // stage goes back to TMA after the MMAs
-                fence_proxy_async_smem();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars[B_SF_READY + sb]);
             }
         }
     } else {
@@ -454,7 +482,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
         bool ok = true;
         int local = 0;
         const int64_t ldo = (int64_t)p.Nout * (p.out_f32 ? 4 : 2);  // output row bytes
-        const float gab = __fmul_rn(*p.ga, *p.gb);
+        // the FP32 tensor scales of the operands (a bf16 activation has none)
+        const float gab = p.ga ? __fmul_rn(*p.ga, *p.gb) : *p.gb;
         for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
             const int m0 = (tile / tiles_n) * BM;
             const int n0 = (tile % tiles_n) * BN;

@@ -118,7 +118,7 @@ __host__ __device__ inline Layout make_layout(int nst, uint32_t ring_bytes) {
     L.x = o;    o += (uint32_t)nst * TILE_BYTES;
     L.f = o;    o += ring_bytes;  // factor ring
     L.sst = o;  o += BM * SROW;   // staged scale bytes
-    L.tab = o;  o += (uint32_t)sizeof(QTable);
+    L.tab = o;  o += (uint32_t)sizeof(QTableM);
     L.bars = o; o += BAR_BYTES;
     L.total = o + 1024;  // slack for the 1 KiB alignment of the base
     return L;
@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
     volatile int* last_flag = abort_flag + 1;
     volatile uint32_t* amax_share = reinterpret_cast<volatile uint32_t*>(last_flag + 1);
     volatile uint32_t* red = amax_share + 1;  // [NQ_WARPS]
-    QTable& tab = *reinterpret_cast<QTable*>(smem + L.tab);
+    QTableM& tab = *reinterpret_cast<QTableM*>(smem + L.tab);
 
     const int warp = warp_id(), lane = lane_id();
     const int m0 = blockIdx.x * BM;
@@ -454,8 +454,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
             amax_t = *p.amax_in;
         }
         const QTensorFast qt = make_qtensor_fast(amax_t);
-        build_qtable(tab, qt.g, t, NQ_THREADS);
+        build_qtable_m1(tab, qt.g, t, NQ_THREADS);
         if (blockIdx.x == 0 && blockIdx.y == 0 && t == 0) *p.tscale = qt.g;
+        named_bar_sync(1, NQ_THREADS);
+        build_qtable_m2(tab, t, NQ_THREADS);
+        named_bar_sync(1, NQ_THREADS);
+        build_qtable_m3(tab, t, NQ_THREADS);
         named_bar_sync(1, NQ_THREADS);
         ok = ok && !*abort_flag;
 
@@ -473,7 +477,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qres(const __grid_constant__
                         const uint4 v0 = ld_shared_v4(ta + off_lo), v1 = ld_shared_v4(ta + off_hi);
                         const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
                         uint32_t sbyte;
-                        const uint2 q = quant_block16_fast_m(w, p.amax_in ? amax_bits_16(w) : mb[st], qt, tab, sbyte);
+                        const uint2 q = quant_block16_m(w, p.amax_in ? amax_bits_16(w) : mb[st], qt, tab, sbyte);
                         if (row_ok) *reinterpret_cast<uint2*>(crow + 32 * st) = q;
                         uint32_t sv = sbyte << (8 * blk);
                         sv |= __shfl_xor_sync(0xFFFFFFFFu, sv, 1);

@@ -123,6 +123,39 @@ __global__ void __launch_bounds__(256) k_pack_wop(const uint8_t* __restrict__ co
     }
 }
 
+// ------------------------------------------------- bf16 weight images
+// The 16-bit GEMMs of the precision ablation read the 4-bit weight through
+// a bf16 image of one orientation: value = e2m1(code) x E4M3 block scale,
+// exact in bf16 (at most 2 + 4 significant bits, exponents within range);
+// the FP32 tensor scale is applied in the GEMM's epilogue, as for the 4-bit
+// GEMM.  codes: [R, C/2], packed along C.  Scales: mode 0 = 16x16 grid
+// [R/16, C/16]; mode 1 = 16x16 grid read transposed ([C/16, R/16], the
+// codes being the grid's transposed layout); mode 2 = 1x16 row scales
+// [R, C/16].  Each thread writes 8 bf16 (16 bytes) per step.
+__global__ void __launch_bounds__(256) k_dequant_w(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                                                   int64_t R, int64_t C, int mode, uint16_t* __restrict__ out) {
+    const float e2m1[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+    const int64_t n8 = R * (C / 8);
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / (C / 8), c = (i - r * (C / 8)) * 8;
+        const uint32_t q = *reinterpret_cast<const uint32_t*>(codes + r * (C / 2) + c / 2);
+        const uint32_t sb = mode == 0 ? scales[(r / 16) * (C / 16) + c / 16]
+                          : mode == 1 ? scales[(c / 16) * (R / 16) + r / 16]
+                                      : scales[r * (C / 16) + c / 16];
+        const float sd = e4m3_decode(sb);
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t n0 = (q >> (8 * k)) & 0xFu, n1 = (q >> (8 * k + 4)) & 0xFu;
+            const float v0 = __fmul_rn((n0 & 8u) ? -e2m1[n0 & 7u] : e2m1[n0 & 7u], sd);
+            const float v1 = __fmul_rn((n1 & 8u) ? -e2m1[n1 & 7u] : e2m1[n1 & 7u], sd);
+            const __nv_bfloat162 b = __floats2bfloat162_rn(v0, v1);
+            w[k] = *reinterpret_cast<const uint32_t*>(&b);
+        }
+        *reinterpret_cast<uint4*>(out + r * C + c) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
 // ------------------------------------------------------- 1x16 row-wise
 // Two 16-element blocks per thread per iteration (four 16-byte loads in
 // flight); stores are 8 bytes of codes and one scale byte per block;
@@ -168,119 +201,192 @@ __global__ void __launch_bounds__(256) k_quant_1x16(const uint16_t* __restrict__
     }
 }
 
-// ---------------------------------------------------- 16x16 tile kernel
-// One warp per 16x16 tile.  Lane l holds row (l & 15), columns 8*(l >> 4)
-// .. +7 of the tile (one 16-byte load).
-//
-// kMode16x16 = true : one scale per tile (weights).  Writes codes packed
-//   along rows (codes_row, [rows, cols/2]) and, if codes_col != nullptr,
-//   the same codes packed along columns ([cols, rows/2]); scale grid
+// ---------------------------------------------------- tile kernel (both layouts)
+// Persistent CTAs over 64 x 128 tiles of x (a 16-wide block never straddles
+// a tile edge: rows and cols are multiples of 16).  A tile is read once with
+// coalesced 16-byte loads into shared memory (rows padded to 272 bytes, so
+// the column pass reads conflict-free), then:
+//   row pass    thread t takes blocks (row, b) = (j / 8, j % 8) for j = t and
+//               t + 256: a warp covers 4 rows x 8 blocks, so its 8-byte code
+//               stores fill whole 64-byte row pieces;
+//   column pass thread t takes columns 2 (t % 64) and 2 (t % 64) + 1, rows
+//               16 (t / 64) .. + 15; column codes and scales are staged in
+//               shared memory and leave as 32-byte column pieces (16-byte
+//               stores) and 4-byte scale words.
+// kMode16x16 = true : one scale per 16x16 tile (weights).  Writes codes
+//   packed along rows (codes_row, [rows, cols/2]) and, if codes_col !=
+//   nullptr, the same codes packed along columns ([cols, rows/2]) -- the
+//   nibbles transposed through shared memory, no second encode; scale grid
 //   [rows/16, cols/16].
 // kMode16x16 = false: 1x16 blocks (activations).  Row blocks -> codes_row /
 //   scales_row ([rows, cols/16]); column blocks (16 consecutive rows of one
 //   column) -> codes_col / scales_col ([cols, rows/16]); both share g.
+constexpr int QTT_R = 64, QTT_C = 128;
+constexpr int QTT_LDW = QTT_C / 2 + 4;  // shared row stride in words (272 bytes)
+
+struct QTileSmem {
+    uint32_t x[QTT_R * QTT_LDW];  // the tile, bf16 pairs
+    uint8_t crow[QTT_R * 64];     // 16x16 mode: the row codes, for the transpose
+    uint8_t ccol[QTT_C * 32];     // column codes, 32 bytes (64 rows) per column
+    uint8_t cscale[QTT_C * 4];    // 1x16 mode: column scales, 4 per column
+    uint32_t rbmax[QTT_R * 8];    // 16x16 mode: max bits of each row block
+    uint32_t tmax[4 * 8];         // 16x16 mode: max bits of each 16x16 tile
+    QTable tab;
+};
+
 template <bool kMode16x16>
 __global__ void __launch_bounds__(256) k_quant_tile16(
     const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
     const float* __restrict__ amax, uint8_t* __restrict__ codes_row,
     uint8_t* __restrict__ scales_row, uint8_t* __restrict__ codes_col,
     uint8_t* __restrict__ scales_col, float* __restrict__ tscale, float* __restrict__ tscale2) {
-    __shared__ uint32_t tile[8][16][9];  // per warp: 16 rows x 8 bf16 pairs (+1 pad)
-    const QTensor t = make_qtensor(*amax);
-    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
-        *tscale = t.g;
-        if (tscale2) *tscale2 = t.g;
+    __shared__ __align__(16) QTileSmem sm;
+    const QTensorFast qt = make_qtensor_fast(*amax);
+    build_qtable(sm.tab, qt.g, threadIdx.x, blockDim.x);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        *tscale = qt.g;
+        if (tscale2) *tscale2 = qt.g;
     }
-    const int w = warp_id(), l = lane_id();
-    const int64_t tiles_c = cols / 16;
-    const int64_t tr = blockIdx.y;                            // tile row
-    const int64_t tc = (int64_t)blockIdx.x * 8 + w;           // tile column
-    if (tc >= tiles_c) return;
-    const int r = l & 15, h = l >> 4;
-    const int64_t row = tr * 16 + r;
-    const int64_t col = tc * 16 + h * 8;
-    uint4 v = ld_nc_v4(x + row * ld + col);
-    uint32_t mine[4] = {v.x, v.y, v.z, v.w};
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int64_t ntc = (cols + QTT_C - 1) / QTT_C;
+    const int64_t ntiles = ((rows + QTT_R - 1) / QTT_R) * ntc;
+    const uint32_t xs = smem_u32(sm.x);
+    // whole-word stores are aligned only for these shapes; else byte stores
+    const bool rs8 = (cols % QTT_C) == 0;   // 8 row scales of a tile row: one 8-byte store
+    const bool cc16 = (rows % 32) == 0;     // column codes: 16-byte pieces
+    const bool cs4 = (rows % QTT_R) == 0;   // column scales: 4-byte words
 
-    if (kMode16x16) {
-        uint32_t m = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) m = __vmaxu2(m, mine[i] & 0x7FFF7FFFu);
-        m = max(m & 0xFFFFu, m >> 16);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-        float amax_b = __uint_as_float(m << 16);
-        uint32_t s;
-        BlockDiv bd;
-        uint32_t code8 = 0;
-        if (block_divisor(amax_b, t, s, bd))
-            code8 = encode8(mine[0], mine[1], mine[2], mine[3], bd.d, bd.y, bd.fast);
-        *reinterpret_cast<uint32_t*>(codes_row + row * (cols / 2) + col / 2) = code8;
-        if (l == 0) scales_row[tr * tiles_c + tc] = (uint8_t)s;
-        if (codes_col) {
-            // transpose the 16x16 nibble tile through shared memory
-            uint32_t* tw = &tile[w][0][0];
-            tw[r * 9 + h] = code8;  // row r, columns 8h..8h+7 (nibbles)
-            __syncwarp();
-            // lane l: column c = l & 15, rows 8*(l>>4) .. +7
-            const int c = l & 15, rh = l >> 4;
-            uint32_t out = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                int rr = rh * 8 + i;
-                uint32_t word = tw[rr * 9 + (c >> 3)];
-                uint32_t nib = (word >> (4 * (c & 7))) & 0xFu;
-                out |= nib << (4 * i);
-            }
-            *reinterpret_cast<uint32_t*>(codes_col + (tc * 16 + c) * (rows / 2) + tr * 8 + rh * 4) =
-                out;
-        }
-    } else {
-        // row blocks: lanes r and r+16 hold the two halves of row r
-        uint32_t m = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) m = __vmaxu2(m, mine[i] & 0x7FFF7FFFu);
-        m = max(m & 0xFFFFu, m >> 16);
-        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 16));
+    for (int64_t ti = blockIdx.x; ti < ntiles; ti += gridDim.x) {
+        const int64_t r0 = (ti / ntc) * QTT_R, c0 = (ti % ntc) * QTT_C;
+        const int vr = (int)min((int64_t)QTT_R, rows - r0);  // multiples of 16
+        const int vc = (int)min((int64_t)QTT_C, cols - c0);
+        __syncthreads();  // the previous tile's shared reads are done (and the table is built)
         {
-            float amax_b = __uint_as_float(m << 16);
-            uint32_t s;
-            BlockDiv bd;
-            uint32_t code8 = 0;
-            if (block_divisor(amax_b, t, s, bd))
-                code8 = encode8(mine[0], mine[1], mine[2], mine[3], bd.d, bd.y, bd.fast);
-            *reinterpret_cast<uint32_t*>(codes_row + row * (cols / 2) + col / 2) = code8;
-            if (h == 0) scales_row[row * tiles_c + tc] = (uint8_t)s;
+            uint4 v[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int i = tid + 256 * k, r = i >> 4, ch = i & 15;
+                v[k] = (r < vr && 8 * ch < vc) ? ld_nc_v4(x + (r0 + r) * ld + c0 + 8 * ch) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int i = tid + 256 * k, r = i >> 4, ch = i & 15;
+                st_shared_v4(xs + (uint32_t)(r * QTT_LDW + 4 * ch) * 4u, v[k]);
+            }
         }
-        // column blocks: gather column c (rows 8h'..8h'+7) through shared memory
-        uint32_t* tw = &tile[w][0][0];
+        __syncthreads();
+
+        // ---------------- row pass
+        uint32_t w[2][8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) tw[r * 9 + h * 4 + i] = mine[i];
-        __syncwarp();
-        const int c = l & 15, rh = l >> 4;
-        uint32_t cw[4];  // 8 bf16 of column c, rows rh*8 .. +7, packed in pairs
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            int r0 = rh * 8 + 2 * i;
-            uint32_t a = tw[r0 * 9 + (c >> 1)];
-            uint32_t b = tw[(r0 + 1) * 9 + (c >> 1)];
-            uint32_t ea = (c & 1) ? (a >> 16) : (a & 0xFFFFu);
-            uint32_t eb = (c & 1) ? (b >> 16) : (b & 0xFFFFu);
-            cw[i] = ea | (eb << 16);
+        for (int k = 0; k < 2; ++k) {
+            const int j = tid + 256 * k, row = j >> 3, b = j & 7;
+            const uint32_t a = xs + (uint32_t)(row * QTT_LDW + 8 * b) * 4u;
+            const uint4 lo = ld_shared_v4(a), hi = ld_shared_v4(a + 16);
+            w[k][0] = lo.x; w[k][1] = lo.y; w[k][2] = lo.z; w[k][3] = lo.w;
+            w[k][4] = hi.x; w[k][5] = hi.y; w[k][6] = hi.z; w[k][7] = hi.w;
         }
-        uint32_t mc = 0;
+        if (kMode16x16) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) mc = __vmaxu2(mc, cw[i] & 0x7FFF7FFFu);
-        mc = max(mc & 0xFFFFu, mc >> 16);
-        mc = max(mc, __shfl_xor_sync(0xFFFFFFFFu, mc, 16));
-        float amax_c = __uint_as_float(mc << 16);
-        uint32_t s;
-        BlockDiv bd;
-        uint32_t code8 = 0;
-        if (block_divisor(amax_c, t, s, bd)) code8 = encode8(cw[0], cw[1], cw[2], cw[3], bd.d, bd.y, bd.fast);
-        const int64_t ccol = tc * 16 + c;
-        *reinterpret_cast<uint32_t*>(codes_col + ccol * (rows / 2) + tr * 8 + rh * 4) = code8;
-        if (rh == 0) scales_col[ccol * (rows / 16) + tr] = (uint8_t)s;
+            for (int k = 0; k < 2; ++k) sm.rbmax[tid + 256 * k] = amax_bits_16(w[k]);
+            __syncthreads();
+            if (tid < 32) {
+                const int tr = tid >> 3, tc = tid & 7;
+                uint32_t m = 0;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) m = max(m, sm.rbmax[(16 * tr + i) * 8 + tc]);
+                sm.tmax[tid] = m;
+            }
+            __syncthreads();
+        }
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int j = tid + 256 * k, row = j >> 3, b = j & 7;
+            const bool valid = row < vr && 16 * b < vc;
+            uint32_t sbyte;
+            const uint32_t mbits = kMode16x16 ? sm.tmax[(row >> 4) * 8 + b] : amax_bits_16(w[k]);
+            const uint2 q = quant_block16_fast_m(w[k], mbits, qt, sm.tab, sbyte);
+            if (valid) *reinterpret_cast<uint2*>(codes_row + (r0 + row) * (cols / 2) + c0 / 2 + 8 * b) = q;
+            if (kMode16x16) {
+                *reinterpret_cast<uint2*>(sm.crow + row * 64 + 8 * b) = q;
+                if (valid && (row & 15) == 0) scales_row[((r0 + row) >> 4) * (cols / 16) + c0 / 16 + b] = (uint8_t)sbyte;
+            } else {
+                // the 8 scale bytes of a row are lanes 8 (row % 4) .. + 7
+                uint32_t sv = sbyte << (8 * (b & 3));
+                sv |= __shfl_xor_sync(0xFFFFFFFFu, sv, 1);
+                sv |= __shfl_xor_sync(0xFFFFFFFFu, sv, 2);
+                const uint32_t hi = __shfl_down_sync(0xFFFFFFFFu, sv, 4);
+                uint8_t* srow = scales_row + (r0 + row) * (cols / 16) + c0 / 16;
+                if (rs8 && vc == QTT_C) {
+                    if (b == 0 && row < vr) *reinterpret_cast<uint2*>(srow) = make_uint2(sv, hi);
+                } else if (valid) {
+                    srow[b] = (uint8_t)sbyte;
+                }
+            }
+        }
+        (void)lane;
+        if (kMode16x16 && !codes_col) continue;
+        if (kMode16x16) __syncthreads();  // the row codes are staged
+
+        // ---------------- column pass: columns 2 cp, 2 cp + 1, rows 16 rb ..
+        {
+            const int cp = tid & 63, rb = tid >> 6;
+            uint2 q0 = make_uint2(0u, 0u), q1 = make_uint2(0u, 0u);
+            uint32_t s0 = 0, s1 = 0;
+            if (kMode16x16) {
+                // transpose the nibbles: byte cp of a row holds columns 2 cp
+                // (low nibble) and 2 cp + 1 (high nibble)
+                uint32_t e[4] = {0, 0, 0, 0}, o[4] = {0, 0, 0, 0};
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const uint32_t byte = sm.crow[(16 * rb + i) * 64 + cp];
+                    e[i >> 2] |= (byte & 0xFu) << (4 * (i & 7));
+                    o[i >> 2] |= (byte >> 4) << (4 * (i & 7));
+                }
+                q0 = make_uint2(e[0] | e[1], e[2] | e[3]);
+                q1 = make_uint2(o[0] | o[1], o[2] | o[3]);
+            } else {
+                uint32_t wc[2][8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint32_t a = sm.x[(16 * rb + 2 * i) * QTT_LDW + cp];
+                    const uint32_t b = sm.x[(16 * rb + 2 * i + 1) * QTT_LDW + cp];
+                    wc[0][i] = __byte_perm(a, b, 0x5410);  // column 2 cp, rows 2i, 2i + 1
+                    wc[1][i] = __byte_perm(a, b, 0x7632);  // column 2 cp + 1
+                }
+                q0 = quant_block16_fast_m(wc[0], amax_bits_16(wc[0]), qt, sm.tab, s0);
+                q1 = quant_block16_fast_m(wc[1], amax_bits_16(wc[1]), qt, sm.tab, s1);
+                sm.cscale[(2 * cp) * 4 + rb] = (uint8_t)s0;
+                sm.cscale[(2 * cp + 1) * 4 + rb] = (uint8_t)s1;
+            }
+            *reinterpret_cast<uint2*>(sm.ccol + (2 * cp) * 32 + 8 * rb) = q0;
+            *reinterpret_cast<uint2*>(sm.ccol + (2 * cp + 1) * 32 + 8 * rb) = q1;
+        }
+        __syncthreads();
+        {
+            // column c's 32 code bytes (64 rows): two 16-byte pieces
+            const int c = tid >> 1, h = tid & 1;
+            if (c < vc) {
+                uint8_t* dst = codes_col + (c0 + c) * (rows / 2) + r0 / 2 + 16 * h;
+                const uint8_t* src = sm.ccol + c * 32 + 16 * h;
+                if (cc16 && 32 * h + 32 <= vr) {
+                    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 2; ++k)
+                        if (32 * h + 16 * k < vr)
+                            *reinterpret_cast<uint2*>(dst + 8 * k) = *reinterpret_cast<const uint2*>(src + 8 * k);
+                }
+            }
+            if (!kMode16x16 && tid < QTT_C && tid < vc) {
+                uint8_t* dst = scales_col + (c0 + tid) * (rows / 16) + r0 / 16;
+                if (cs4 && vr == QTT_R) {
+                    *reinterpret_cast<uint32_t*>(dst) = *reinterpret_cast<const uint32_t*>(sm.cscale + tid * 4);
+                } else {
+                    for (int k = 0; 16 * k < vr; ++k) dst[k] = sm.cscale[tid * 4 + k];
+                }
+            }
+        }
     }
 }
 

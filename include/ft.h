@@ -86,6 +86,17 @@ typedef enum {
 typedef enum { FT_BLK_1x16 = 0, FT_BLK_16x16 = 1 } ft_block;
 typedef enum { FT_BF16 = 0, FT_F32 = 1 } ft_dtype;
 
+/* Precision configuration of a layer (section 4, "Impact of Precision
+ * Configurations", Table 4).  The weight is always 4-bit.  FT_W4A4G4 (the
+ * method): both backbone GEMMs are NVFP4 x NVFP4.  Bit 0 (FT_W4A16G4): the
+ * forward GEMM reads the bf16 activation X with the weight's bf16 image
+ * (ft_linear.wd_k).  Bit 1 (FT_W4A4G16): the dgrad GEMM reads the bf16
+ * output gradient dY with the transposed image (wd_n).  FT_W4A16G16: both.
+ * The 16-bit GEMMs run on tcgen05 kind::f16 with FP32 accumulation; the
+ * low-rank branches and the adapter gradients are the same in every
+ * configuration (they never read a quantized tensor).                      */
+typedef enum { FT_W4A4G4 = 0, FT_W4A16G4 = 1, FT_W4A4G16 = 2, FT_W4A16G16 = 3 } ft_precision;
+
 /* Non-owning view of an NVFP4 tensor of logical shape rows x cols.
  *   codes : rows x cols/2 bytes, row-major, two E2M1 codes per byte packed
  *           along the row (column 2i in the low nibble of byte i).
@@ -118,7 +129,13 @@ typedef struct {
  *         scales of each 256 x 256 block side by side, the scales one per
  *         row (ft_pack_weight_operands fills them from w_k, w_n and the
  *         grid; ft_weight_operand_bytes(N, K) bytes each, 16-byte aligned).
- *         A layout of the same codes and scales, not a new quantization.  */
+ *         A layout of the same codes and scales, not a new quantization.
+ *   precision: an ft_precision (0 = FT_W4A4G4, the method).
+ *   wd_k, wd_n: the weight's bf16 images for the 16-bit GEMMs
+ *         (ft_dequant_weight_operands): wd_k [N, K] read by the forward
+ *         when precision has FT_W4A16G4, wd_n [K, N] (the same values
+ *         transposed) read by dgrad when it has FT_W4A4G16; NULL otherwise.
+ *         16-byte aligned.                                                 */
 typedef struct {
     int64_t N, K, r_s, r_l;
     float s;
@@ -130,6 +147,9 @@ typedef struct {
     const void* B;
     const uint8_t* op_k;
     const uint8_t* op_n;
+    int32_t precision;
+    const void* wd_k;
+    const void* wd_n;
 } ft_linear;
 
 /* ft_quantize -- Q(x) for a bf16 matrix (section 3.2 block quantization).
@@ -189,6 +209,18 @@ ft_status ft_pack_weight_operands(const uint8_t* codes_k, const uint8_t* codes_n
 ft_status ft_pack_weight_operands_1x16(const uint8_t* codes_k, const uint8_t* scales_k, const uint8_t* codes_n,
                                        const uint8_t* scales_n, int64_t N, int64_t K, uint8_t* op_k,
                                        uint8_t* op_n, void* stream);
+
+/* ft_dequant_weight_operands -- once per weight, for the 16-bit GEMMs of
+ * the precision configurations (section 4, Table 4): bf16 images of Q(W_res)
+ * holding e2m1(code) x block scale (exact in bf16; the tensor scale stays in
+ * w_k.tscale and is applied by the GEMM).  A layout of the same quantized
+ * values, not a new quantization.
+ *   w_k   : Q(W_res) [N, K] as in ft_linear (16x16 blocks, or 1x16 groups).
+ *   w_n   : its dgrad orientation [K, N] (needed when wd_n is given; for
+ *           16x16 blocks its scales are w_k's grid).
+ *   wd_k  : bf16 [N, K] out, or NULL.   wd_n : bf16 [K, N] out, or NULL.
+ *   N, K multiples of 16; 16-byte aligned pointers.  At least one output.  */
+ft_status ft_dequant_weight_operands(const ft_fp4* w_k, const ft_fp4* w_n, void* wd_k, void* wd_n, void* stream);
 
 /* ft_linear_fwd -- Eq. 2 with LoRA fusion (section 3.3): one pass over X
  * emits Q(X) and the down-projections P = [bf16(X U) | bf16(s X A)]; one

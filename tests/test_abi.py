@@ -40,7 +40,7 @@ def test_every_declared_symbol_is_exported_and_bound(L):
 def test_struct_layouts_match_c():
     # int64 x4, float (+4 pad), two 48-byte views, six pointers
     assert ctypes.sizeof(FtFp4) == 48
-    assert ctypes.sizeof(FtLinear) == 32 + 8 + 2 * 48 + 6 * 8
+    assert ctypes.sizeof(FtLinear) == 32 + 8 + 2 * 48 + 6 * 8 + 8 + 2 * 8
 
 
 def test_status_strings(L):
@@ -233,3 +233,39 @@ def test_1x16_weight_views_and_packing_validation(L):
     assert L.ft_pack_weight_operands_1x16(g, g, g, g, 256, 320, g, g, None) == FT_ERR_SHAPE
     assert L.ft_pack_weight_operands_1x16(g, g, g, g, 256, 256, g, g + 8, None) == FT_ERR_ALIGN
     assert L.ft_pack_weight_operands_1x16(g, g, g, g, 0, 256, g, g, None) == FT_OK
+
+
+def test_precision_field_is_validated_on_the_host(L):
+    """The precision configuration of a layer (the FourTune page's Table 4):
+    out-of-range values and a 16-bit GEMM without its bf16 weight image are
+    refused before any launch, as is a misaligned image."""
+    x = 0x200000
+    ws = L.ft_workspace_bytes(128, 256, 256, 16, 16)
+    for prec, wd_k, wd_n, want in [(4, 0, 0, FT_ERR_INVALID_ARG), (-1, 0, 0, FT_ERR_INVALID_ARG),
+                                   (1, 0, 0, FT_ERR_INVALID_ARG), (2, x, 0, FT_ERR_INVALID_ARG),
+                                   (3, x, 0, FT_ERR_INVALID_ARG), (1, x + 8, 0, FT_ERR_ALIGN),
+                                   (2, 0, x + 4, FT_ERR_ALIGN)]:
+        lin = _linear()
+        lin.precision, lin.wd_k, lin.wd_n = prec, wd_k or None, wd_n or None
+        assert L.ft_linear_fwd(ctypes.byref(lin), x, 128, None, x, 0, x, x, ws, None) == want, prec
+        assert L.ft_linear_bwd(ctypes.byref(lin), x, x, x, 128, None, x, 0, x, x, x, ws, None) == want, prec
+    # a complete 16-bit configuration passes validation (M = 0: nothing runs)
+    lin = _linear()
+    lin.precision, lin.wd_k, lin.wd_n = 3, x, x
+    assert L.ft_linear_fwd(ctypes.byref(lin), x, 0, None, x, 0, x, x, ws, None) == FT_OK
+
+
+def test_dequant_weight_operands_validation(L):
+    p = 0x100000
+    wk = FtFp4(p, p, p, 256, 512, 1)
+    wn = FtFp4(p, p, p, 512, 256, 1)
+    assert L.ft_dequant_weight_operands(None, ctypes.byref(wn), p, p, None) == FT_ERR_INVALID_ARG
+    assert L.ft_dequant_weight_operands(ctypes.byref(wk), ctypes.byref(wn), None, None, None) == FT_ERR_INVALID_ARG
+    assert L.ft_dequant_weight_operands(ctypes.byref(wk), None, None, p, None) == FT_ERR_INVALID_ARG
+    bad = FtFp4(p, p, p, 256, 520, 1)
+    assert L.ft_dequant_weight_operands(ctypes.byref(bad), None, p, None, None) == FT_ERR_SHAPE
+    swapped = FtFp4(p, p, p, 256, 512, 1)
+    assert L.ft_dequant_weight_operands(ctypes.byref(wk), ctypes.byref(swapped), None, p, None) == FT_ERR_SHAPE
+    assert L.ft_dequant_weight_operands(ctypes.byref(wk), ctypes.byref(wn), p + 8, None, None) == FT_ERR_ALIGN
+    empty = FtFp4(p, p, p, 0, 512, 1)
+    assert L.ft_dequant_weight_operands(ctypes.byref(empty), None, p, None, None) == FT_OK
