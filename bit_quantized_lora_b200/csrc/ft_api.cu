@@ -350,11 +350,14 @@ WsPlan plan_ws(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t r_l) {
 }
 
 // ------------------------------------------------------------ pieces
-ft_status run_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, float* slot, cudaStream_t st) {
+ft_status run_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, float* slot, const DevInfo* d,
+                   cudaStream_t st) {
     FT_TRY(cuda_ok(cudaMemsetAsync(slot, 0, sizeof(float), st)));
     const int64_t vecs = rows * (cols / 8);
-    // one round of four 16-byte loads per thread covers a dense tensor
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(vecs, 4 * 256), 1 << 30));
+    // a few CTAs per SM, each thread looping with eight 16-byte loads in
+    // flight: every CTA ends in one same-address atomic, which serialise in
+    // L2, so thousands of short CTAs would queue on it
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(vecs, 8 * 256), (int64_t)d->sms * 4));
     {
         LaunchTimer _lt(KID_AMAX, st);
         ft::k_amax_bf16<<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(x), rows, cols, ld,
@@ -368,7 +371,8 @@ ft_status run_quant_1x16(const void* x, int64_t rows, int64_t cols, int64_t ld, 
                          uint8_t* codes, uint8_t* scales, float* tscale, uint8_t* slab,
                          const DevInfo* d, cudaStream_t st) {
     const int64_t blocks = rows * (cols / 16);
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(blocks, 256), (int64_t)d->sms * 16));
+    // one wave of persistent CTAs (each builds its encode table once)
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(blocks, 512), (int64_t)d->sms * 6));
     {
         LaunchTimer _lt(KID_QUANT_1X16, st);
         ft::k_quant_1x16<<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(x), rows, cols, ld, amax,
@@ -580,7 +584,7 @@ ft_status run_quant_down(const void* T, int64_t M, int64_t C, const void* L1, in
     if (!qres_grid(M, C, qres_max_stages(p.ring_bytes), d, &mt, &splits, &cchunk) || mt > QRES_MAX_ROW_TILES) {
         const float* a = amax_in;
         if (!a) {
-            FT_TRY(run_amax(T, M, C, C, reinterpret_cast<float*>(ws + w.amax), st));
+            FT_TRY(run_amax(T, M, C, C, reinterpret_cast<float*>(ws + w.amax), d, st));
             a = reinterpret_cast<float*>(ws + w.amax);
         }
         return run_qdown(T, M, C, L1, r1, L2, r2, s, a, codes, scales, tscale, P, ws, w, d, st);
@@ -997,7 +1001,7 @@ ft_status ft_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, ft_
     const float* a = amax;
     if (!a) {
         float* slot = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + 128);
-        FT_TRY(run_amax(x, rows, cols, ld, slot, st));
+        FT_TRY(run_amax(x, rows, cols, ld, slot, d, st));
         a = slot;
     }
     if (blk == FT_BLK_1x16)
@@ -1035,7 +1039,7 @@ ft_status ft_quantize_transpose(const void* x, int64_t rows, int64_t cols, int64
     const float* a = amax;
     if (!a) {
         float* slot = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + 128);
-        FT_TRY(run_amax(x, rows, cols, ld, slot, st));
+        FT_TRY(run_amax(x, rows, cols, ld, slot, d, st));
         a = slot;
     }
     if (blk == FT_BLK_16x16)

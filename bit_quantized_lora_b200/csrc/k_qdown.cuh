@@ -17,9 +17,12 @@
 // P with all of its loads in flight at once.
 //
 // CTA = 128 rows of T x one C-range; warps: 0 TMA producer, 1 UMMA issuer,
-// 2-9 quantizers (thread t owns row t % 128, blocks 2(t/128), 2(t/128)+1 of
-// each 128 x 64 stage, read from the same swizzled shared-memory tile the MMA
-// consumes) and then the epilogue (TMEM -> partial).
+// 2-17 quantizers (quantizer warp q owns tile rows 8q .. 8q + 7, lane l the
+// block l % 4 of row 8q + l / 4 in each 128 x 64 stage, read from the same
+// swizzled shared-memory tile the MMA consumes: a warp's codes of a stage
+// are 8 rows x 32 contiguous bytes, whole sectors, and its scales one 4-byte
+// word per row, in the row-major and the slab layout alike); warps 2-9 then
+// move the down-projection from TMEM to the FP32 partial.
 #pragma once
 
 #include <cuda.h>
@@ -32,7 +35,7 @@ namespace qdown {
 constexpr int BM = 128;
 constexpr int BKC = 64;  // columns of T per stage (128 bytes of bf16)
 constexpr int STAGES = 4;
-constexpr int NQ_WARPS = 8;  // quantizer / epilogue warps
+constexpr int NQ_WARPS = 16;  // quantizer warps (the first 8 also the epilogue)
 constexpr int NUM_THREADS = 64 + NQ_WARPS * 32;
 constexpr int TILE_BYTES = BM * BKC * 2;  // 16 KiB
 constexpr uint32_t TMEM_COLS = 128;
@@ -55,7 +58,7 @@ struct Params {
     int direct;  // 1: read L1 / L2 directly (r1, r2 <= 64); 0: packed Lt
 };
 
-constexpr uint32_t SMEM_BYTES = STAGES * 2 * TILE_BYTES + sizeof(QTable) + 256 + 1024;
+constexpr uint32_t SMEM_BYTES = STAGES * 2 * TILE_BYTES + sizeof(QTableM) + 256 + 1024;
 
 __global__ void __launch_bounds__(NUM_THREADS, 1) k_qdown(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
@@ -63,8 +66,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qdown(const __grid_constant_
     const uint32_t base = (raw_base + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (base - raw_base);
     const uint32_t off_x = 0, off_l = STAGES * TILE_BYTES, off_tab = 2 * STAGES * TILE_BYTES;
-    const uint32_t off_bar = off_tab + sizeof(QTable);
-    QTable& tab = *reinterpret_cast<QTable*>(smem + off_tab);
+    const uint32_t off_bar = off_tab + sizeof(QTableM);
+    QTableM& tab = *reinterpret_cast<QTableM*>(smem + off_tab);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + off_bar);
     uint64_t* empty = full + STAGES;
     uint64_t* accfull = empty + STAGES;
@@ -84,16 +87,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qdown(const __grid_constant_
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
             mbar_init(&full[i], 1);
-            // every quantizer thread releases the stage after its own loads
+            // every quantizer warp releases the stage after its own loads
             // (behind a proxy fence, see below), plus the MMA commit
-            mbar_init(&empty[i], NQ_WARPS * 32 + (p.do_mma ? 1 : 0));
+            mbar_init(&empty[i], NQ_WARPS + (p.do_mma ? 1 : 0));
         }
         mbar_init(accfull, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp >= 2) build_qtable(tab, qt.g, threadIdx.x - 64, NUM_THREADS - 64);
     if (warp == 1 && p.do_mma) {
         tmem_alloc(tmem_slot, TMEM_COLS);
         tmem_relinquish();
@@ -170,13 +172,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qdown(const __grid_constant_
         }
         __syncwarp();
     } else {
-        // quantizers: thread t owns row (t & 127), 16-element blocks 2h, 2h+1
+        // quantizers
         const int t = threadIdx.x - 64;
-        const int trow = t & (BM - 1), h = t >> 7;
+        const int qw = t >> 5;
+        const int trow = 8 * qw + (lane >> 2), blk = lane & 3;
         const int row = m0 + trow;
         if (blockIdx.x == 0 && blockIdx.y == 0 && t == 0) *p.tscale = qt.g;
+        // the multiply-path table, built while the first stages land
+        build_qtable_m1(tab, qt.g, t, NQ_WARPS * 32);
+        named_bar_sync(1, NQ_WARPS * 32);
+        build_qtable_m2(tab, t, NQ_WARPS * 32);
+        named_bar_sync(1, NQ_WARPS * 32);
+        build_qtable_m3(tab, t, NQ_WARPS * 32);
+        named_bar_sync(1, NQ_WARPS * 32);
         bool ok = true;
         const uint32_t sw = (uint32_t)(trow & 7);
+        const uint32_t off_lo = (uint32_t)trow * 128u + (((uint32_t)(2 * blk) ^ sw) << 4);
+        const uint32_t off_hi = (uint32_t)trow * 128u + (((uint32_t)(2 * blk + 1) ^ sw) << 4);
         for (int st = 0; st < nst; ++st) {
             const int s = st % STAGES;
             const uint32_t ph = (st / STAGES) & 1;
@@ -184,31 +196,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qdown(const __grid_constant_
                 ok = false;
                 break;
             }
-            const uint32_t rowaddr = base + off_x + s * TILE_BYTES + trow * 128;
-            uint4 v[4];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) v[c] = ld_shared_v4(rowaddr + (((uint32_t)(4 * h + c) ^ sw) << 4));
+            const uint32_t ta = base + off_x + s * TILE_BYTES;
+            const uint4 v0 = ld_shared_v4(ta + off_lo), v1 = ld_shared_v4(ta + off_hi);
             // the next TMA copy into this stage is an async-proxy write: the
             // generic-proxy loads above must be ordered before it explicitly
             // (without this fence the copy was seen to overtake them)
             fence_proxy_async_smem();
-            mbar_arrive(&empty[s]);
-            uint32_t w0[8] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w};
-            uint32_t w1[8] = {v[2].x, v[2].y, v[2].z, v[2].w, v[3].x, v[3].y, v[3].z, v[3].w};
-            uint32_t s0, s1;
-            const uint2 q0 = quant_block16_fast(w0, qt, tab, s0);
-            const uint2 q1 = quant_block16_fast(w1, qt, tab, s1);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+            const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            uint32_t sbyte;
+            const uint2 q = quant_block16_m(w, amax_bits_16(w), qt, tab, sbyte);
+            // the row's four scale bytes of this stage (lanes 4r .. 4r + 3)
+            uint32_t sv = sbyte << (8 * blk);
+            sv |= __shfl_xor_sync(0xFFFFFFFFu, sv, 1);
+            sv |= __shfl_xor_sync(0xFFFFFFFFu, sv, 2);
             if (row < p.M) {
-                const int col = c0 + st * BKC + 32 * h;
-                *reinterpret_cast<uint4*>(p.codes + (int64_t)row * (p.C / 2) + col / 2) =
-                    make_uint4(q0.x, q0.y, q1.x, q1.y);
-                *reinterpret_cast<uint16_t*>(p.scales + (int64_t)row * (p.C / 16) + col / 16) =
-                    (uint16_t)(s0 | (s1 << 8));
-                *reinterpret_cast<uint16_t*>(p.slab + slab_offset(row, col / 16, p.C)) =
-                    (uint16_t)(s0 | (s1 << 8));
+                const int col = c0 + st * BKC;
+                *reinterpret_cast<uint2*>(p.codes + (int64_t)row * (p.C / 2) + col / 2 + 8 * blk) = q;
+                if (blk == 0) {
+                    *reinterpret_cast<uint32_t*>(p.scales + (int64_t)row * (p.C / 16) + col / 16) = sv;
+                    *reinterpret_cast<uint32_t*>(p.slab + slab_offset(row, col / 16, p.C)) = sv;
+                }
             }
         }
-        if (p.do_mma && ok) {
+        if (p.do_mma && ok && warp < 10) {
             // TMEM lane = rank index j, column = tile row; warps 2-5 take tile
             // rows 0-63, warps 6-9 rows 64-127
             const int sp = warp & 3;

@@ -157,8 +157,9 @@ __global__ void __launch_bounds__(256) k_dequant_w(const uint8_t* __restrict__ c
 }
 
 // ------------------------------------------------------- 1x16 row-wise
-// Two 16-element blocks per thread per iteration (four 16-byte loads in
-// flight); stores are 8 bytes of codes and one scale byte per block;
+// Persistent CTAs (one wave); each builds the multiply-path table once, then
+// takes two 16-element blocks per thread per iteration (four 16-byte loads
+// in flight); stores are 8 bytes of codes and one scale byte per block;
 // consecutive threads touch consecutive blocks, so accesses are coalesced.
 // slab (optional, cols % 64 == 0): the scales again in the GEMM slab layout.
 __global__ void __launch_bounds__(256) k_quant_1x16(const uint16_t* __restrict__ x, int64_t rows,
@@ -168,9 +169,13 @@ __global__ void __launch_bounds__(256) k_quant_1x16(const uint16_t* __restrict__
                                                     uint8_t* __restrict__ scales,
                                                     float* __restrict__ tscale,
                                                     uint8_t* __restrict__ slab) {
-    __shared__ QTable tab;
+    __shared__ QTableM tab;
     const QTensorFast t = make_qtensor_fast(*amax);
-    build_qtable(tab, t.g, threadIdx.x, blockDim.x);
+    build_qtable_m1(tab, t.g, threadIdx.x, blockDim.x);
+    __syncthreads();
+    build_qtable_m2(tab, threadIdx.x, blockDim.x);
+    __syncthreads();
+    build_qtable_m3(tab, threadIdx.x, blockDim.x);
     __syncthreads();
     if (blockIdx.x == 0 && threadIdx.x == 0) *tscale = t.g;
     const int64_t nb = cols / 16;
@@ -187,13 +192,13 @@ __global__ void __launch_bounds__(256) k_quant_1x16(const uint16_t* __restrict__
         const uint4 u0 = ld_nc_v4(p2), u1 = ld_nc_v4(p2 + 8);
         uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
         uint32_t s;
-        const uint2 q = quant_block16_fast(w, t, tab, s);
+        const uint2 q = quant_block16_m(w, amax_bits_16(w), t, tab, s);
         *reinterpret_cast<uint2*>(codes + r * (cols / 2) + c * 8) = q;
         scales[r * nb + c] = (uint8_t)s;
         if (slab) slab[slab_offset(r, c, cols)] = (uint8_t)s;
         if (two) {
             uint32_t w2[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-            const uint2 q2 = quant_block16_fast(w2, t, tab, s);
+            const uint2 q2 = quant_block16_m(w2, amax_bits_16(w2), t, tab, s);
             *reinterpret_cast<uint2*>(codes + r2 * (cols / 2) + c2 * 8) = q2;
             scales[r2 * nb + c2] = (uint8_t)s;
             if (slab) slab[slab_offset(r2, c2, cols)] = (uint8_t)s;
@@ -231,7 +236,7 @@ struct QTileSmem {
     uint8_t cscale[QTT_C * 4];    // 1x16 mode: column scales, 4 per column
     uint32_t rbmax[QTT_R * 8];    // 16x16 mode: max bits of each row block
     uint32_t tmax[4 * 8];         // 16x16 mode: max bits of each 16x16 tile
-    QTable tab;
+    QTableM tab;
 };
 
 template <bool kMode16x16>
@@ -242,7 +247,11 @@ __global__ void __launch_bounds__(256) k_quant_tile16(
     uint8_t* __restrict__ scales_col, float* __restrict__ tscale, float* __restrict__ tscale2) {
     __shared__ __align__(16) QTileSmem sm;
     const QTensorFast qt = make_qtensor_fast(*amax);
-    build_qtable(sm.tab, qt.g, threadIdx.x, blockDim.x);
+    build_qtable_m1(sm.tab, qt.g, threadIdx.x, blockDim.x);
+    __syncthreads();
+    build_qtable_m2(sm.tab, threadIdx.x, blockDim.x);
+    __syncthreads();
+    build_qtable_m3(sm.tab, threadIdx.x, blockDim.x);
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         *tscale = qt.g;
         if (tscale2) *tscale2 = qt.g;
@@ -305,7 +314,7 @@ __global__ void __launch_bounds__(256) k_quant_tile16(
             const bool valid = row < vr && 16 * b < vc;
             uint32_t sbyte;
             const uint32_t mbits = kMode16x16 ? sm.tmax[(row >> 4) * 8 + b] : amax_bits_16(w[k]);
-            const uint2 q = quant_block16_fast_m(w[k], mbits, qt, sm.tab, sbyte);
+            const uint2 q = quant_block16_m(w[k], mbits, qt, sm.tab, sbyte);
             if (valid) *reinterpret_cast<uint2*>(codes_row + (r0 + row) * (cols / 2) + c0 / 2 + 8 * b) = q;
             if (kMode16x16) {
                 *reinterpret_cast<uint2*>(sm.crow + row * 64 + 8 * b) = q;
@@ -354,8 +363,8 @@ __global__ void __launch_bounds__(256) k_quant_tile16(
                     wc[0][i] = __byte_perm(a, b, 0x5410);  // column 2 cp, rows 2i, 2i + 1
                     wc[1][i] = __byte_perm(a, b, 0x7632);  // column 2 cp + 1
                 }
-                q0 = quant_block16_fast_m(wc[0], amax_bits_16(wc[0]), qt, sm.tab, s0);
-                q1 = quant_block16_fast_m(wc[1], amax_bits_16(wc[1]), qt, sm.tab, s1);
+                q0 = quant_block16_m(wc[0], amax_bits_16(wc[0]), qt, sm.tab, s0);
+                q1 = quant_block16_m(wc[1], amax_bits_16(wc[1]), qt, sm.tab, s1);
                 sm.cscale[(2 * cp) * 4 + rb] = (uint8_t)s0;
                 sm.cscale[(2 * cp + 1) * 4 + rb] = (uint8_t)s1;
             }

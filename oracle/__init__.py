@@ -378,6 +378,59 @@ def linear_bwd(dY, X, W_res, U, V, A, B, s: float, P, rows=None, amax_dy=None, q
     return {"dX": dX, "dA": dA, "dB": dB, "Pg": Pg, "qdy": qdy, "rows": rows}
 
 
+# -------------------------------------------------------------- MLP fusion
+_GELU_TABLE = None
+
+
+def gelu_bf16(y: np.ndarray) -> np.ndarray:
+    """GELU of bf16 values, rounded once to bf16 (RNE): for each bf16 bit
+    pattern y, h = bf16(0.5 y erfc(-y / sqrt 2)) from float64 (the erfc form
+    stays accurate where 1 + erf would cancel, y << 0).  A bf16 input takes
+    one of 65536 values, so the function is a table over every bit pattern
+    (pinned against a 50-digit evaluation).  GELU is the activation between
+    a DiT block's MLP linears (FourTune page, section 3.3, MLP fusion)."""
+    global _GELU_TABLE
+    if _GELU_TABLE is None:
+        import math
+        v = bf16_to_f64(np.arange(65536, dtype=np.uint32).astype(np.uint16))
+        out = np.empty(65536, np.float64)
+        for i, x in enumerate(v):
+            out[i] = 0.5 * x * math.erfc(-x / math.sqrt(2.0)) if np.isfinite(x) else x
+        t = bf16_from_f64(out)
+        # A float64 result exactly halfway between two bf16 values arises
+        # only for subnormal y, where it is y / 2 with the y^2 / sqrt(2 pi)
+        # term rounded away; the true value lies above it (GELU(y) - y / 2 =
+        # y (Phi(y) - 1/2) > 0 for y != 0), so such a tie rounds up.
+        lo = bf16_to_f64(t)
+        up = bf16_to_f64(((t.astype(np.int32) + np.where(lo >= 0, 1, -1)) & 0xFFFF).astype(np.uint16))
+        tie = np.isfinite(out) & (out != lo) & (np.abs(out - lo) == np.abs(up - out)) & (up > lo)
+        t[tie] = bf16_from_f64(up[tie])
+        _GELU_TABLE = t
+    return _GELU_TABLE[np.asarray(y, np.uint16)]
+
+
+def mlp_fwd(X, up: dict, down: dict, amax_h: float, amax_x=None):
+    """Forward of a DiT MLP whose two linears are triple-branch layers, with
+    the FC1 GEMM fused with the FC2 quantization (FourTune page, section 3.3,
+    "MLP Fusion"): Y_up = the up layer's Eq. 2 output rounded to bf16, H =
+    GELU(Y_up) rounded to bf16, and the down layer's forward on H, whose
+    NVFP4 tensor scale comes from the supplied amax_h (the fused kernel
+    quantizes H as the tiles leave the FC1 GEMM, before the whole of H
+    exists, so the tensor amax cannot come from H itself).  Every step is
+    row-local given amax_x (the tensor amax of X, else X's own) and amax_h,
+    so X may be a sample of token rows.  up / down: dicts of W_res, U, V, A,
+    B, s and optionally qw (the 16x16 quantization of W_res).  Returns Y_up
+    (bf16), H (bf16), P_up, P_down (bf16), qh = (codes, scales, g) of Q(H)
+    and Y (float64) of the down layer."""
+    f_up = linear_fwd(X, up["W_res"], up["U"], up["V"], up["A"], up["B"], up["s"], amax_x=amax_x,
+                      qw=up.get("qw"))
+    Y_up = bf16_from_f64(f_up["Y"])
+    H = gelu_bf16(Y_up)
+    f_dn = linear_fwd(H, down["W_res"], down["U"], down["V"], down["A"], down["B"], down["s"], amax_x=amax_h,
+                      qw=down.get("qw"))
+    return {"Y_up": Y_up, "H": H, "P_up": f_up["P"], "P_down": f_dn["P"], "qh": f_dn["qx"], "Y": f_dn["Y"]}
+
+
 def rel_fro(a: np.ndarray, b: np.ndarray) -> float:
     """||a - b||_F / ||b||_F (0 when both are zero)."""
     a = np.asarray(a, np.float64)
