@@ -574,6 +574,72 @@ def run_attn_secondary(torch, ft, dev, flush, steps, warmup, fp4_peak, hbm_gbs):
     return res
 
 
+def bench_mlp(torch, ft, dev, flush, reps=10):
+    """MLP fusion (the FourTune page's section 3.3; its Fig. 9 credits it
+    with a further 1.10x): one DiT block's MLP forward, X [4608, 3072] ->
+    up [12288, 3072] -> GELU -> down [3072, 12288], fused (FC1's GEMM
+    epilogue applies GELU and quantizes H for FC2 with a supplied tensor
+    amax) against the same calls unfused (FC1, the GELU kernel, FC2 with its
+    own quantizer, with the amax supplied or computed).  CUDA events around
+    each forward, L2 flushed before each."""
+    import ft_synth
+    sh_up, sh_dn = stack_shapes()[2], stack_shapes()[3]
+
+    def to_dev(u16):
+        return torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    iu = ft_synth.make_inputs(sh_up, seed=SEED + 2)
+    wd = ft_synth.make_inputs(dataclasses_replace(sh_dn, M=16), seed=SEED + 3)
+    up = ft.prepare_layer(to_dev(iu["W"]), sh_up.r_s, A=to_dev(iu["A"]), B=to_dev(iu["B"]), s=iu["s"])
+    dn = ft.prepare_layer(to_dev(wd["W"]), sh_dn.r_s, A=to_dev(wd["A"]), B=to_dev(wd["B"]), s=wd["s"])
+    X = to_dev(iu["X"])
+    M = sh_up.M
+    Y_up, _ = ft.ft_linear_fwd(up, X)
+    H = ft.ft_gelu_bf16(Y_up)
+    amax_h = H.abs().max().float().reshape(1)
+    ws_f, ws_u = ft.Workspace(), ft.Workspace()
+    Yd = torch.empty(M, sh_dn.N, dtype=torch.bfloat16, device=dev)
+    Pu = torch.empty(M, sh_up.r_s + sh_up.r_l, dtype=torch.bfloat16, device=dev)
+    Pd = torch.empty(M, sh_dn.r_s + sh_dn.r_l, dtype=torch.bfloat16, device=dev)
+    Hf = torch.empty_like(H)
+
+    def fused():
+        ft.ft_mlp_fwd(up, dn, X, amax_h, H=Hf, Y=Yd, P_up=Pu, P_down=Pd, ws=ws_f)
+
+    def unfused(amax):
+        ft.ft_linear_fwd(up, X, Y=Y_up, P=Pu, ws=ws_u)
+        ft.ft_gelu_bf16(Y_up, out=H)
+        ft.ft_linear_fwd(dn, H, amax_x=amax, Y=Yd, P=Pd, ws=ws_u)
+
+    stream = torch.cuda.current_stream()
+    out = {}
+    for name, fn in (("fused", fused), ("unfused_supplied_amax", lambda: unfused(amax_h)),
+                     ("unfused_computed_amax", lambda: unfused(None))):
+        fn()
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(reps):
+            flush()
+            keep_host_ahead(torch, 1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        out[name + "_ms"] = statistics.median(ms)
+    assert ft.ft_device_error() == 0, "device error in the MLP section"
+    out["speedup_vs_unfused_supplied"] = out["unfused_supplied_amax_ms"] / out["fused_ms"]
+    out["speedup_vs_unfused_computed"] = out["unfused_computed_amax_ms"] / out["fused_ms"]
+    out["workload"] = "X [4608,3072] -> up [12288,3072] -> GELU -> down [3072,12288], r_s = r_l = 32, bf16 outputs"
+    return out
+
+
+def dataclasses_replace(obj, **kw):
+    import dataclasses
+    return dataclasses.replace(obj, **kw)
+
+
 def run_ours(args):
     import torch
 
@@ -723,6 +789,7 @@ def run_ours(args):
     if dist is None and not args.skip_extras:
         out["attn_proj"] = run_attn_secondary(torch, ft, dev, flush, args.steps, args.warmup, fp4_peak, hbm_gbs)
         out["quantize"] = bench_quantizers(torch, ft, dev, hbm_gbs, flush)
+        out["mlp_fusion"] = bench_mlp(torch, ft, dev, flush)
 
     # ---------------- end to end through the API with host buffers: every
     # linear's X and dY copied in from pinned host memory, the step, and the

@@ -29,7 +29,8 @@ PRECISIONS = {"W4A4G4": W4A4G4, "W4A16G4": W4A16G4, "W4A4G16": W4A4G16, "W4A16G1
 
 __all__ = [
     "FP4", "Layer", "FtError", "BLK_1x16", "BLK_16x16", "BF16", "F32",
-    "W4A4G4", "W4A16G4", "W4A4G16", "W4A16G16", "PRECISIONS", "ft_dequant_weight_operands",
+    "W4A4G4", "W4A16G4", "W4A4G16", "W4A16G16", "PRECISIONS", "ft_dequant_weight_operands", "ft_gelu_bf16",
+    "ft_mlp_fwd", "ft_mlp_workspace_bytes",
     "ft_quantize", "ft_quantize_transpose", "ft_linear_fwd", "ft_linear_bwd",
     "ft_workspace_bytes", "ft_quantize_workspace_bytes", "ft_device_error",
     "ft_set_cooperative_quantizer", "prepare_layer", "svd_split", "Workspace", "timing",
@@ -319,6 +320,47 @@ def ft_linear_bwd(layer: Layer, dY: torch.Tensor, X: torch.Tensor, P: torch.Tens
         ctypes.byref(v), dY.data_ptr(), _ptr(X), P.data_ptr() if r > 0 else None, M, _ptr(amax_dy),
         dX.data_ptr(), out_dtype, _ptr(dA), _ptr(dB), wbuf.data_ptr(), wbuf.numel(), _stream(stream)))
     return dX, dA, dB
+
+
+def ft_mlp_workspace_bytes(up: Layer, down: Layer, M: int) -> int:
+    vu, vd = up.view(), down.view()
+    return load().ft_mlp_workspace_bytes(ctypes.byref(vu), ctypes.byref(vd), M)
+
+
+def ft_mlp_fwd(up: Layer, down: Layer, X: torch.Tensor, amax_h: torch.Tensor, amax_x: torch.Tensor | None = None,
+               out_dtype: int = BF16, H: torch.Tensor | None = None, Y: torch.Tensor | None = None,
+               P_up: torch.Tensor | None = None, P_down: torch.Tensor | None = None,
+               ws: Workspace | None = None, stream=None):
+    """The MLP forward with FC1's GEMM fused with FC2's quantization: H =
+    GELU(bf16(FC1(X))) and Y = FC2(H), Q(H) made by FC1's epilogue with the
+    tensor scale of the supplied amax_h.  Returns (Y, H, P_up, P_down)."""
+    _bf16(X, "X")
+    M = X.shape[0]
+    dev = X.device
+    H = torch.empty(M, up.N, dtype=torch.bfloat16, device=dev) if H is None else H
+    if Y is None:
+        Y = torch.empty(M, down.N, device=dev, dtype=torch.float32 if out_dtype == F32 else torch.bfloat16)
+    ru, rd = up.r_s + up.r_l, down.r_s + down.r_l
+    P_up = torch.empty(M, max(ru, 0), dtype=torch.bfloat16, device=dev) if P_up is None else P_up
+    P_down = torch.empty(M, max(rd, 0), dtype=torch.bfloat16, device=dev) if P_down is None else P_down
+    wbuf = _ws(ws, ft_mlp_workspace_bytes(up, down, M), dev)
+    vu, vd = up.view(), down.view()
+    check("ft_mlp_fwd", load().ft_mlp_fwd(
+        ctypes.byref(vu), ctypes.byref(vd), X.data_ptr(), M, _ptr(amax_x), amax_h.data_ptr(), H.data_ptr(),
+        Y.data_ptr(), out_dtype, P_up.data_ptr() if ru > 0 else None, P_down.data_ptr() if rd > 0 else None,
+        wbuf.data_ptr(), wbuf.numel(), _stream(stream)))
+    return Y, H, P_up, P_down
+
+
+def ft_gelu_bf16(y: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """h = GELU(y) on bf16, each value correctly rounded (the activation the
+    fused MLP applies between its linears)."""
+    _bf16(y, "y")
+    if not y.is_contiguous():
+        raise ValueError("y must be contiguous")
+    out = torch.empty_like(y) if out is None else out
+    check("ft_gelu_bf16", load().ft_gelu_bf16(y.data_ptr(), out.data_ptr(), y.numel(), _stream(stream)))
+    return out
 
 
 def ft_device_error(stream=None) -> int:

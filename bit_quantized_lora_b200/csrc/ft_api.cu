@@ -104,6 +104,8 @@ ft_status device_info(DevInfo** out) {
                                  big) != cudaSuccess ||
             cudaFuncSetAttribute(ft::gemm::k_gemm_fp4<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  big) != cudaSuccess ||
+            cudaFuncSetAttribute(ft::gemm::k_gemm_fp4<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 big) != cudaSuccess ||
             cudaFuncSetAttribute(ft::qdown::k_qdown, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)ft::qdown::SMEM_BYTES) != cudaSuccess ||
             cudaFuncSetAttribute(ft::lgrad::k_lora_grad, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -116,6 +118,7 @@ ft_status device_info(DevInfo** out) {
         const void* kernels[] = {
             reinterpret_cast<const void*>(ft::gemm::k_gemm_fp4<false>),
             reinterpret_cast<const void*>(ft::gemm::k_gemm_fp4<true>),
+            reinterpret_cast<const void*>(ft::gemm::k_gemm_fp4<false, true>),
             reinterpret_cast<const void*>(ft::qres::k_qres),
             reinterpret_cast<const void*>(ft::qdown::k_qdown),
             reinterpret_cast<const void*>(ft::lgrad::k_lora_grad),
@@ -188,12 +191,13 @@ enum KernelId {
     KID_QRES,
     KID_GEMM_BF16,
     KID_DEQUANT_W,
+    KID_GELU,
     KID_COUNT
 };
 const char* const kKernelNames[KID_COUNT] = {
     "k_amax_bf16", "k_quant_1x16", "k_quant_tile16", "k_pack_lt", "k_qdown",
     "k_lowrank_finalize", "k_gemm_fp4", "k_lora_grad", "k_lora_grad_reduce", "k_qres",
-    "k_gemm_bf16", "k_dequant_w"};
+    "k_gemm_bf16", "k_dequant_w", "k_gelu_bf16"};
 
 struct TimingRec {
     cudaEvent_t a, b;
@@ -371,8 +375,7 @@ ft_status run_quant_1x16(const void* x, int64_t rows, int64_t cols, int64_t ld, 
                          uint8_t* codes, uint8_t* scales, float* tscale, uint8_t* slab,
                          const DevInfo* d, cudaStream_t st) {
     const int64_t blocks = rows * (cols / 16);
-    // one wave of persistent CTAs (each builds its encode table once)
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(blocks, 512), (int64_t)d->sms * 6));
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(blocks, 256), (int64_t)d->sms * 16));
     {
         LaunchTimer _lt(KID_QUANT_1X16, st);
         ft::k_quant_1x16<<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(x), rows, cols, ld, amax,
@@ -403,13 +406,14 @@ ft_status run_tile16(bool mode16x16, const void* x, int64_t rows, int64_t cols, 
 
 // Q(T) and P = [bf16(T L1) | bf16(s T L2)] in one pass over T [M, C].
 // Also zeroes its row-tile completion counters.
+// quant = false: P alone (T's quantized form is produced elsewhere).
 ft_status run_qdown(const void* T, int64_t M, int64_t C, const void* L1, int64_t r1, const void* L2,
                     int64_t r2, float s, const float* amax, uint8_t* codes, uint8_t* scales,
                     float* tscale, void* P, uint8_t* ws, const WsPlan& w, const DevInfo* d,
-                    cudaStream_t st) {
+                    cudaStream_t st, bool quant = true) {
     const int64_t r = r1 + r2;
     uint8_t* slab = ws + w.sfslab;
-    if (r == 0) return run_quant_1x16(T, M, C, C, amax, codes, scales, tscale, slab, d, st);
+    if (r == 0) return quant ? run_quant_1x16(T, M, C, C, amax, codes, scales, tscale, slab, d, st) : FT_OK;
     float* part = reinterpret_cast<float*>(ws + w.part);
     unsigned int* counters = reinterpret_cast<unsigned int*>(ws + w.counters);
     FT_TRY(cuda_ok(cudaMemsetAsync(counters, 0, (size_t)w.n_qd_counters * 4, st)));
@@ -458,6 +462,7 @@ ft_status run_qdown(const void* T, int64_t M, int64_t C, const void* L1, int64_t
     p.splits = splits;
     p.s = s;
     p.do_mma = 1;
+    p.quant = quant ? 1 : 0;
     {
         LaunchTimer _lt(KID_QDOWN, st);
         ft::qdown::k_qdown<<<dim3((unsigned)mt, (unsigned)splits), ft::qdown::NUM_THREADS,
@@ -675,12 +680,30 @@ CUtensorMapSwizzle swizzle_for(int wbox) {
 // the 16-bit variant, out = gb A B^T + ..., with A = a_codes a bf16 [M, Kc]
 // matrix and B = b_op the weight's bf16 image [Nout, Kc] (a_slab and ga
 // unused).
+// MLP fusion: the epilogue's GELU and the quantized copy of its output.
+struct MlpOut {
+    const float* amax_h;
+    uint8_t* codes;
+    uint8_t* scales;
+    uint8_t* slab;
+    float* tscale;
+};
+
 ft_status run_gemm(bool bf16, const uint8_t* a_codes, const uint8_t* a_slab, const float* ga, int64_t M,
                    int64_t Kc, const uint8_t* b_op, const float* gb,
                    int64_t Nout, const void* P, const void* L1, int64_t r1, const void* L2, int64_t r2,
-                   void* out, ft_dtype ot, const DevInfo* d, cudaStream_t st, DepFlag dep) {
+                   void* out, ft_dtype ot, const DevInfo* d, cudaStream_t st, DepFlag dep,
+                   const MlpOut* mlp = nullptr) {
     Params p;
     std::memset(&p, 0, sizeof(p));
+    if (mlp) {
+        p.mlp = 1;
+        p.amax_h = mlp->amax_h;
+        p.q_codes = mlp->codes;
+        p.q_scales = mlp->scales;
+        p.q_slab = mlp->slab;
+        p.q_tscale = mlp->tscale;
+    }
     if (bf16) {
         FT_TRY(encode_2d(&p.mapA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a_codes, Kc, M, Kc * 2, 64, 128,
                          CU_TENSOR_MAP_SWIZZLE_128B));
@@ -728,10 +751,10 @@ ft_status run_gemm(bool bf16, const uint8_t* a_codes, const uint8_t* a_slab, con
     p.Nout = (int)Nout;
     p.Kc = (int)Kc;
     int stages = ft::gemm::MAX_STAGES;
-    while (stages > 1 && ft::gemm::make_layout(stages, p.f1, p.f2).total > 227u * 1024u) --stages;
-    if (ft::gemm::make_layout(stages, p.f1, p.f2).total > 227u * 1024u) return FT_ERR_SHAPE;
+    while (stages > 1 && ft::gemm::make_layout(stages, p.f1, p.f2, p.mlp).total > 227u * 1024u) --stages;
+    if (ft::gemm::make_layout(stages, p.f1, p.f2, p.mlp).total > 227u * 1024u) return FT_ERR_SHAPE;
     p.stages = stages;
-    const uint32_t smem = ft::gemm::make_layout(stages, p.f1, p.f2).total;
+    const uint32_t smem = ft::gemm::make_layout(stages, p.f1, p.f2, p.mlp).total;
     const int tiles = cdiv(M, ft::gemm::BM) * (int)(Nout / ft::gemm::BN);
     const int grid = std::max(1, std::min(tiles, d->sms));
     {
@@ -739,6 +762,9 @@ ft_status run_gemm(bool bf16, const uint8_t* a_codes, const uint8_t* a_slab, con
         if (bf16)
             FT_TRY(launch_overlapped(ft::gemm::k_gemm_fp4<true>, dim3((unsigned)grid), dim3(ft::gemm::NUM_THREADS),
                                      smem, st, p));
+        else if (mlp)
+            FT_TRY(launch_overlapped(ft::gemm::k_gemm_fp4<false, true>, dim3((unsigned)grid),
+                                     dim3(ft::gemm::NUM_THREADS), smem, st, p));
         else
             FT_TRY(launch_overlapped(ft::gemm::k_gemm_fp4<false>, dim3((unsigned)grid), dim3(ft::gemm::NUM_THREADS),
                                      smem, st, p));
@@ -937,6 +963,21 @@ ft_status ft_dequant_weight_operands(const ft_fp4* w_k, const ft_fp4* w_n, void*
     return FT_OK;
 }
 
+ft_status ft_gelu_bf16(const void* y, void* h, int64_t n, void* stream) {
+    if (n < 0 || (n > 0 && (!y || !h))) return FT_ERR_INVALID_ARG;
+    if (n % 8) return FT_ERR_SHAPE;
+    if (!al16(y) || !al16(h)) return FT_ERR_ALIGN;
+    if (n == 0) return FT_OK;
+    DevInfo* d;
+    FT_TRY(device_info(&d));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(n / 8, 256), (int64_t)d->sms * 8));
+    LaunchTimer _lt(KID_GELU, st);
+    ft::k_gelu_bf16<<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(y), static_cast<uint16_t*>(h), n);
+    _lt.stop();
+    return last_launch();
+}
+
 size_t ft_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t r_l) {
     if (M < 0 || N < 0 || K < 0 || r_s < 0 || r_l < 0) return 0;
     return plan_ws(M, N, K, r_s, r_l).total;
@@ -1129,6 +1170,59 @@ ft_status ft_linear_bwd(const ft_linear* L, const void* dY, const void* X, const
     if (L->r_l > 0)
         FT_TRY(run_lora_grads(dY, X, P_save, Pg, M, L->N, L->K, L->r_s, L->r_l, dA, dB, wsb, w, d, st, dep));
     return FT_OK;
+}
+
+size_t ft_mlp_workspace_bytes(const ft_linear* up, const ft_linear* down, int64_t M) {
+    if (!up || !down || M < 0) return 0;
+    return up256(plan_ws(M, up->N, up->K, up->r_s, up->r_l).total) +
+           plan_ws(M, down->N, down->K, down->r_s, down->r_l).total;
+}
+
+ft_status ft_mlp_fwd(const ft_linear* up, const ft_linear* down, const void* X, int64_t M, const float* amax_x,
+                     const float* amax_h, void* H, void* Y, ft_dtype yt, void* P_up, void* P_down, void* ws,
+                     size_t ws_bytes, void* stream) {
+    FT_TRY(check_linear(up));
+    FT_TRY(check_linear(down));
+    if (down->K != up->N) return FT_ERR_SHAPE;
+    if (up->precision != FT_W4A4G4 || down->precision != FT_W4A4G4) return FT_ERR_INVALID_ARG;
+    if (M < 0) return FT_ERR_INVALID_ARG;
+    if (yt != FT_BF16 && yt != FT_F32) return FT_ERR_INVALID_ARG;
+    if (M > (1 << 24)) return FT_ERR_SHAPE;
+    if (M == 0) return FT_OK;
+    const int64_t r_up = up->r_s + up->r_l, r_dn = down->r_s + down->r_l;
+    if (!X || !amax_h || !H || !Y || (r_up > 0 && !P_up) || (r_dn > 0 && !P_down)) return FT_ERR_INVALID_ARG;
+    if (!al16(X) || !al16(H) || !al16(Y) || (P_up && !al16(P_up)) || (P_down && !al16(P_down)) ||
+        (reinterpret_cast<uintptr_t>(amax_h) & 3u))
+        return FT_ERR_ALIGN;
+    const WsPlan wu = plan_ws(M, up->N, up->K, up->r_s, up->r_l);
+    const WsPlan wd = plan_ws(M, down->N, down->K, down->r_s, down->r_l);
+    if (!ws || ws_bytes < up256(wu.total) + wd.total || !al16(ws)) return FT_ERR_WORKSPACE;
+    DevInfo* d;
+    FT_TRY(device_info(&d));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* wsu = static_cast<uint8_t*>(ws);
+    uint8_t* wsd = wsu + up256(wu.total);
+    // FC1: Q(X) and P_up in one pass over X
+    DepFlag dep;
+    FT_TRY(run_quant_down(X, M, up->K, up->U, up->r_s, up->A, up->r_l, up->s, amax_x, wsu + wu.codes,
+                          wsu + wu.scales, reinterpret_cast<float*>(wsu + wu.gact), P_up, wsu, wu, d, st, &dep));
+    // FC1's GEMM with the fused epilogue: H = GELU(bf16(Y_up)) and Q(H) in
+    // the down layer's workspace, as its own quantizer would lay it out
+    MlpOut mo;
+    mo.amax_h = amax_h;
+    mo.codes = wsd + wd.codes;
+    mo.scales = wsd + wd.scales;
+    mo.slab = wsd + wd.sfslab;
+    mo.tscale = reinterpret_cast<float*>(wsd + wd.gact);
+    FT_TRY(run_gemm(false, wsu + wu.codes, wsu + wu.sfslab, reinterpret_cast<float*>(wsu + wu.gact), M, up->K,
+                    up->op_k, up->w_k.tscale, up->N, P_up, up->V, up->r_s, up->B, up->r_l, H, FT_BF16, d, st, dep,
+                    &mo));
+    // FC2: its down-projections of H (no second quantization), then its GEMM on Q(H)
+    FT_TRY(run_qdown(H, M, down->K, down->U, down->r_s, down->A, down->r_l, down->s, nullptr, nullptr, nullptr,
+                     nullptr, P_down, wsd, wd, d, st, false));
+    return run_gemm(false, wsd + wd.codes, wsd + wd.sfslab, reinterpret_cast<float*>(wsd + wd.gact), M, down->K,
+                    down->op_k, down->w_k.tscale, down->N, P_down, down->V, down->r_s, down->B, down->r_l, Y, yt, d,
+                    st, DepFlag());
 }
 
 ft_status ft_timing_enable(int on) {

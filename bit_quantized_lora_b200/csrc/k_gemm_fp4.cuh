@@ -58,6 +58,8 @@
 
 #include <cuda.h>
 
+#include "ft_gelu.cuh"
+#include "ft_nvfp4.cuh"
 #include "ft_ptx.cuh"
 
 namespace ft {
@@ -112,12 +114,23 @@ struct Params {
     int M, Nout, Kc;
     LrFactor f1, f2;
     int stages;
+    // MLP fusion (section 3.3; bf16 output only): the output is H =
+    // GELU(bf16(y)), and the epilogue also quantizes H for the next linear
+    // with the tensor scale of the caller's amax_h: 1x16 codes [M, Nout/2],
+    // scales [M, Nout/16], the same scales in the GEMM slab layout, and the
+    // decode scale (written by CTA 0)
+    int mlp;
+    const float* amax_h;
+    uint8_t* q_codes;
+    uint8_t* q_scales;
+    uint8_t* q_slab;
+    float* q_tscale;
 };
 
 struct Layout {
-    uint32_t a, b, sfa, p1, p2, l1, l2, stg, bars, total;
+    uint32_t a, b, sfa, p1, p2, l1, l2, stg, tab, bars, total;
 };
-constexpr uint32_t STG_BYTES = 128 * 64;  // one staged output chunk: 128 rows x 64 bytes
+constexpr uint32_t STG_BYTES = 128 * 32;  // one staged output chunk: 128 rows x 32 bytes
 
 // bytes of a factor's P panel (128 rows) and L panel (256 rows)
 __host__ __device__ inline uint32_t p_bytes(const LrFactor& f) {
@@ -127,7 +140,7 @@ __host__ __device__ inline uint32_t l_bytes(const LrFactor& f) {
     return f.rf > 0 ? (uint32_t)f.natoms * 256u * f.row_bytes : 0u;
 }
 
-__host__ __device__ inline Layout make_layout(int stages, const LrFactor& f1, const LrFactor& f2) {
+__host__ __device__ inline Layout make_layout(int stages, const LrFactor& f1, const LrFactor& f2, int mlp) {
     Layout L;
     uint32_t o = 0;
     L.a = o;    o += stages * A_BYTES;
@@ -138,6 +151,8 @@ __host__ __device__ inline Layout make_layout(int stages, const LrFactor& f1, co
     L.l2 = o;   o += l_bytes(f2);
     L.sfa = o;  o += stages * SFA_STAGE_BYTES;
     L.stg = o;  o += 2 * STG_BYTES;  // output staging, one buffer per column group
+    L.tab = o;  o += mlp ? (uint32_t)sizeof(QTableM) : 0u;  // the encode table of Q(H)
+    o = (o + 15u) & ~15u;
     L.bars = o; o += 256;  // barriers, TMEM slot, abort flag
     L.total = o + 1024;    // slack for 1 KiB alignment of the base
     return L;
@@ -187,13 +202,14 @@ __device__ __forceinline__ void lr_mma(uint32_t tmem_d, uint32_t pa, uint32_t pb
 // scale stays apart as gb), tcgen05 kind::f16; a stage holds 64 columns of
 // K in the same 128-byte rows, four K = 16 MMAs.  No scale factors: the
 // scale warps idle.  Tiles, epilogue and low-rank terms are shared.
-template <bool kBf16>
+// kMlp: the MLP-fusion epilogue (Params::mlp), for the 4-bit GEMM.
+template <bool kBf16, bool kMlp = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (base - raw_base);
-    const Layout L = make_layout(p.stages, p.f1, p.f2);
+    const Layout L = make_layout(p.stages, p.f1, p.f2, kMlp ? 1 : 0);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.bars + B_COUNT * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.bars + B_COUNT * 8 + 4);
@@ -466,16 +482,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
         // Each thread owns one tile row (its TMEM lane) within one of two
         // column groups working concurrently: warps 6-9 take columns 0-127
         // (with low-rank half 0), warps 10-13 columns 128-255 (half 1).
-        // Output leaves in chunks of 64 bytes per row (32 bf16 or 16 f32
-        // columns): the group's rows are written into its 64-byte-swizzled
-        // staging buffer, then the group copies the 128-row chunk out with
-        // 16-byte stores, four threads per row, so every warp store covers
-        // whole sectors of eight rows.  (A TMA store per chunk would queue
-        // in the same copy engine as the next tile's operand loads.)
+        // Output leaves in chunks of 32 bytes per row (16 bf16 or 8 f32
+        // columns): the group's rows are written into its staging buffer
+        // (the two 16-byte halves of a row swapped on every other group of
+        // four rows, so eight consecutive rows' stores hit distinct banks),
+        // then the group copies the 128-row chunk out with 16-byte stores,
+        // two threads per row, so every warp store covers whole sectors of
+        // sixteen rows.  (A TMA store per chunk would queue in the same copy
+        // engine as the next tile's operand loads.)  The small staging
+        // buffer keeps three operand stages resident at rank 64.
         const int sp = warp & 3;  // TMEM sub-partition = rows 32*sp .. +31
         const int grp = (warp - EPI_WARP0) >> 2;
         const int et = 32 * sp + lane;  // tile row
-        const uint32_t rsw = (uint32_t)((et >> 1) & 3);
+        const uint32_t rsw = (uint32_t)((et >> 2) & 1);
         const uint32_t buf = base + L.stg + (uint32_t)grp * STG_BYTES;
         const uint32_t lr_col = grp == 0 ? LR0_COL : R2_COL;
         uint64_t* lr_ready = &bars[grp == 0 ? B_LR0_READY : B_LR1_READY];
@@ -484,6 +503,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
         const int64_t ldo = (int64_t)p.Nout * (p.out_f32 ? 4 : 2);  // output row bytes
         // the FP32 tensor scales of the operands (a bf16 activation has none)
         const float gab = p.ga ? __fmul_rn(*p.ga, *p.gb) : *p.gb;
+        // MLP fusion: the encode table of Q(H) for the caller's tensor amax,
+        // built by the 256 epilogue threads before the first accumulator
+        QTableM& tab = *reinterpret_cast<QTableM*>(smem + L.tab);
+        QTensorFast qt;
+        qt.g = qt.six_g = qt.y6 = 0.0f;
+        if (kMlp) {
+            const int et2 = threadIdx.x - 32 * EPI_WARP0;
+            qt = make_qtensor_fast(*p.amax_h);
+            build_qtable_m1(tab, qt.g, et2, 32 * NUM_EPI_WARPS);
+            named_bar_sync(3, 32 * NUM_EPI_WARPS);
+            build_qtable_m2(tab, et2, 32 * NUM_EPI_WARPS);
+            named_bar_sync(3, 32 * NUM_EPI_WARPS);
+            build_qtable_m3(tab, et2, 32 * NUM_EPI_WARPS);
+            named_bar_sync(3, 32 * NUM_EPI_WARPS);
+            if (blockIdx.x == 0 && et2 == 0) *p.q_tscale = qt.g;
+        }
         for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
             const int m0 = (tile / tiles_n) * BM;
             const int n0 = (tile % tiles_n) * BN;
@@ -494,17 +529,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             }
             tc_fence_after();
             const uint32_t lane_addr = (uint32_t)(32 * sp) << 16;
-            const uint32_t rowa = buf + (uint32_t)et * 64u;
-            // the staged chunk at tile column `col` leaves the buffer: piece
-            // i is row i / 4, 16-byte column i % 4
+            const uint32_t rowa = buf + (uint32_t)et * 32u;
+            // stage one 32-byte piece of this thread's row ...
+            auto stage = [&](uint4 lo, uint4 hi) {
+                st_shared_v4(rowa + (rsw << 4), lo);
+                st_shared_v4(rowa + ((rsw ^ 1u) << 4), hi);
+            };
+            // ... and copy the group's staged chunk at tile column `col` out:
+            // piece i is row i / 2, 16-byte half i % 2
             auto copy_out = [&](int col) {
                 uint8_t* obase = p.out + (int64_t)m0 * ldo + (int64_t)(n0 + col) * (p.out_f32 ? 4 : 2);
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
+                for (int k = 0; k < 2; ++k) {
                     const int i = et + 128 * k;
-                    const int row = i >> 2, q = i & 3;
-                    const uint4 v =
-                        ld_shared_v4(buf + (uint32_t)row * 64u + (((uint32_t)q ^ (uint32_t)((row >> 1) & 3)) << 4));
+                    const int row = i >> 1, q = i & 1;
+                    const uint4 v = ld_shared_v4(buf + (uint32_t)row * 32u +
+                                                 (((uint32_t)q ^ (uint32_t)((row >> 2) & 1)) << 4));
                     if (m0 + row < p.M) *reinterpret_cast<uint4*>(obase + (int64_t)row * ldo + 16 * q) = v;
                 }
             };
@@ -513,13 +553,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                 // tensor memory and packed first, so the accumulator is
                 // released before the stores and the next tile's MMAs run
                 // while they drain
-                uint32_t pk[4][16];
+                uint32_t pk[8][8];
 #pragma unroll
-                for (int c2 = 0; c2 < 8; ++c2) {
-                    const int c = c2 >> 1, h = (c2 & 1) * 8;
+                for (int c = 0; c < 8; ++c) {
                     uint32_t v[16], lr[16];
-                    tmem_ld_32x32b_x16(tmem + lane_addr + ACC_COL + 128 * grp + 16 * c2, v);
-                    if (has_lr) tmem_ld_32x32b_x16(tmem + lane_addr + lr_col + 16 * c2, lr);
+                    tmem_ld_32x32b_x16(tmem + lane_addr + ACC_COL + 128 * grp + 16 * c, v);
+                    if (has_lr) tmem_ld_32x32b_x16(tmem + lane_addr + lr_col + 16 * c, lr);
                     tmem_ld_wait();
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
@@ -527,7 +566,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                         const float y1 =
                             __fmaf_rn(gab, __uint_as_float(v[2 * k + 1]), has_lr ? __uint_as_float(lr[2 * k + 1]) : 0.0f);
                         __nv_bfloat162 t = __floats2bfloat162_rn(y0, y1);
-                        pk[c][h + k] = *reinterpret_cast<uint32_t*>(&t);
+                        pk[c][k] = *reinterpret_cast<uint32_t*>(&t);
                     }
                 }
                 // every TMEM read of this tile is done: the MMA warp may
@@ -535,20 +574,48 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[B_ACC_EMPTY]);
+                if (kMlp) {
+                    // MLP fusion: H = GELU(y) per bf16 value; a 16-column
+                    // chunk of the row is exactly one 1x16 block of Q(H)
+                    const int row = m0 + et;
+                    const int64_t qcol = n0 + 128 * grp;  // first column of the group
+                    uint32_t sw0 = 0, sw1 = 0;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    // the group's previous chunk has been copied out of the buffer
-                    named_bar_sync(1 + grp, 128);
+                    for (int c = 0; c < 8; ++c) {
+                        uint32_t w[8];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        st_shared_v4(rowa + (((uint32_t)q ^ rsw) << 4),
-                                     make_uint4(pk[c][4 * q], pk[c][4 * q + 1], pk[c][4 * q + 2], pk[c][4 * q + 3]));
-                    named_bar_sync(1 + grp, 128);
-                    copy_out(128 * grp + 32 * c);
+                        for (int k = 0; k < 8; ++k) w[k] = gelu_bf16x2(pk[c][k]);
+                        uint32_t sbyte;
+                        const uint2 q = quant_block16_m(w, amax_bits_16(w), qt, tab, sbyte);
+                        if (row < p.M)
+                            *reinterpret_cast<uint2*>(p.q_codes + (int64_t)row * (p.Nout / 2) + (qcol + 16 * c) / 2) = q;
+                        if (c < 4) sw0 |= sbyte << (8 * c);
+                        else sw1 |= sbyte << (8 * (c - 4));
+                        named_bar_sync(1 + grp, 128);
+                        stage(make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]));
+                        named_bar_sync(1 + grp, 128);
+                        copy_out(128 * grp + 16 * c);
+                    }
+                    if (row < p.M)
+                        *reinterpret_cast<uint2*>(p.q_scales + (int64_t)row * (p.Nout / 16) + qcol / 16) =
+                            make_uint2(sw0, sw1);
+                    // slab rows past M hold the (zero) scales of the zero-filled rows
+                    *reinterpret_cast<uint32_t*>(p.q_slab + slab_offset(row, qcol / 16, p.Nout)) = sw0;
+                    *reinterpret_cast<uint32_t*>(p.q_slab + slab_offset(row, qcol / 16 + 4, p.Nout)) = sw1;
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        // the group's previous chunk has been copied out of the buffer
+                        named_bar_sync(1 + grp, 128);
+                        stage(make_uint4(pk[c][0], pk[c][1], pk[c][2], pk[c][3]),
+                              make_uint4(pk[c][4], pk[c][5], pk[c][6], pk[c][7]));
+                        named_bar_sync(1 + grp, 128);
+                        copy_out(128 * grp + 16 * c);
+                    }
                 }
             } else {
-                // FP32: eight chunks of 16 columns, the accumulator released
-                // after the last
+                // FP32: eight reads of 16 columns, each leaving as two chunks
+                // of 8; the accumulator released after the last
 #pragma unroll 1
                 for (int c = 0; c < 8; ++c) {
                     const int lcol = 16 * c;          // column within the group's half
@@ -557,18 +624,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     tmem_ld_32x32b_x16(tmem + lane_addr + ACC_COL + col, v);
                     if (has_lr) tmem_ld_32x32b_x16(tmem + lane_addr + lr_col + lcol, lr);
                     tmem_ld_wait();
-                    float y[16];
+                    uint32_t y[16];
 #pragma unroll
                     for (int k = 0; k < 16; ++k)
-                        y[k] = __fmaf_rn(gab, __uint_as_float(v[k]), has_lr ? __uint_as_float(lr[k]) : 0.0f);
-                    named_bar_sync(1 + grp, 128);
+                        y[k] = __float_as_uint(
+                            __fmaf_rn(gab, __uint_as_float(v[k]), has_lr ? __uint_as_float(lr[k]) : 0.0f));
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        st_shared_v4(rowa + (((uint32_t)q ^ rsw) << 4),
-                                     make_uint4(__float_as_uint(y[4 * q]), __float_as_uint(y[4 * q + 1]),
-                                                __float_as_uint(y[4 * q + 2]), __float_as_uint(y[4 * q + 3])));
-                    named_bar_sync(1 + grp, 128);
-                    copy_out(col);
+                    for (int h = 0; h < 2; ++h) {
+                        named_bar_sync(1 + grp, 128);
+                        stage(make_uint4(y[8 * h], y[8 * h + 1], y[8 * h + 2], y[8 * h + 3]),
+                              make_uint4(y[8 * h + 4], y[8 * h + 5], y[8 * h + 6], y[8 * h + 7]));
+                        named_bar_sync(1 + grp, 128);
+                        copy_out(col + 8 * h);
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();

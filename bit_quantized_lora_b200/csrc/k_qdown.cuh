@@ -56,6 +56,7 @@ struct Params {
     float s;
     int do_mma;
     int direct;  // 1: read L1 / L2 directly (r1, r2 <= 64); 0: packed Lt
+    int quant;   // 1: Q(T) and P; 0: P alone (T already quantized elsewhere)
 };
 
 constexpr uint32_t SMEM_BYTES = STAGES * 2 * TILE_BYTES + sizeof(QTableM) + 256 + 1024;
@@ -82,14 +83,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qdown(const __grid_constant_
     const int c0 = split * p.cchunk;
     const int cn = min(p.cchunk, p.C - c0);
     const int nst = cn / BKC;
-    const QTensorFast qt = make_qtensor_fast(*p.amax);
+    const QTensorFast qt = make_qtensor_fast(p.quant ? *p.amax : 0.0f);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
             mbar_init(&full[i], 1);
             // every quantizer warp releases the stage after its own loads
             // (behind a proxy fence, see below), plus the MMA commit
-            mbar_init(&empty[i], NQ_WARPS + (p.do_mma ? 1 : 0));
+            mbar_init(&empty[i], (p.quant ? NQ_WARPS : 0) + (p.do_mma ? 1 : 0));
         }
         mbar_init(accfull, 1);
         mbar_init(drain, 1);
@@ -177,7 +178,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qdown(const __grid_constant_
         const int qw = t >> 5;
         const int trow = 8 * qw + (lane >> 2), blk = lane & 3;
         const int row = m0 + trow;
-        if (blockIdx.x == 0 && blockIdx.y == 0 && t == 0) *p.tscale = qt.g;
+        if (p.quant && blockIdx.x == 0 && blockIdx.y == 0 && t == 0) *p.tscale = qt.g;
         // the multiply-path table, built while the first stages land
         build_qtable_m1(tab, qt.g, t, NQ_WARPS * 32);
         named_bar_sync(1, NQ_WARPS * 32);
@@ -189,7 +190,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_qdown(const __grid_constant_
         const uint32_t sw = (uint32_t)(trow & 7);
         const uint32_t off_lo = (uint32_t)trow * 128u + (((uint32_t)(2 * blk) ^ sw) << 4);
         const uint32_t off_hi = (uint32_t)trow * 128u + (((uint32_t)(2 * blk + 1) ^ sw) << 4);
-        for (int st = 0; st < nst; ++st) {
+        for (int st = 0; st < (p.quant ? nst : 0); ++st) {
             const int s = st % STAGES;
             const uint32_t ph = (st / STAGES) & 1;
             if (!mbar_wait(&full[s], ph, ERR_WAIT_FULL, abort_flag)) {

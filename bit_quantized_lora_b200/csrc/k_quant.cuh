@@ -8,9 +8,23 @@
 // group-wise granularity).
 #pragma once
 
+#include "ft_gelu.cuh"
 #include "ft_nvfp4.cuh"
 
 namespace ft {
+
+// ------------------------------------------------------------------ GELU
+// h = GELU(y) elementwise on bf16 (ft_gelu.cuh), 8 values per 16-byte load;
+// n a multiple of 8, pointers 16-byte aligned.
+__global__ void __launch_bounds__(256) k_gelu_bf16(const uint16_t* __restrict__ y, uint16_t* __restrict__ h,
+                                                   int64_t n) {
+    const int64_t n8 = n / 8;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+        const uint4 v = ld_nc_v4(y + 8 * i);
+        *reinterpret_cast<uint4*>(h + 8 * i) =
+            make_uint4(gelu_bf16x2(v.x), gelu_bf16x2(v.y), gelu_bf16x2(v.z), gelu_bf16x2(v.w));
+    }
+}
 
 // ------------------------------------------------------------------ amax
 // max|x| over a bf16 matrix (cols % 8 == 0, rows 16-byte aligned).  Each
@@ -157,10 +171,13 @@ __global__ void __launch_bounds__(256) k_dequant_w(const uint8_t* __restrict__ c
 }
 
 // ------------------------------------------------------- 1x16 row-wise
-// Persistent CTAs (one wave); each builds the multiply-path table once, then
-// takes two 16-element blocks per thread per iteration (four 16-byte loads
-// in flight); stores are 8 bytes of codes and one scale byte per block;
+// Two 16-element blocks per thread per iteration (four 16-byte loads in
+// flight); stores are 8 bytes of codes and one scale byte per block;
 // consecutive threads touch consecutive blocks, so accesses are coalesced.
+// Many short CTAs, each with the one-step divisor table (Markstein-corrected
+// quotients): measured faster here than persistent CTAs with the
+// multiply-path table, whose longer build and serial loop cost more than
+// the cheaper per-element encode saves.
 // slab (optional, cols % 64 == 0): the scales again in the GEMM slab layout.
 __global__ void __launch_bounds__(256) k_quant_1x16(const uint16_t* __restrict__ x, int64_t rows,
                                                     int64_t cols, int64_t ld,
@@ -169,13 +186,9 @@ __global__ void __launch_bounds__(256) k_quant_1x16(const uint16_t* __restrict__
                                                     uint8_t* __restrict__ scales,
                                                     float* __restrict__ tscale,
                                                     uint8_t* __restrict__ slab) {
-    __shared__ QTableM tab;
+    __shared__ QTable tab;
     const QTensorFast t = make_qtensor_fast(*amax);
-    build_qtable_m1(tab, t.g, threadIdx.x, blockDim.x);
-    __syncthreads();
-    build_qtable_m2(tab, threadIdx.x, blockDim.x);
-    __syncthreads();
-    build_qtable_m3(tab, threadIdx.x, blockDim.x);
+    build_qtable(tab, t.g, threadIdx.x, blockDim.x);
     __syncthreads();
     if (blockIdx.x == 0 && threadIdx.x == 0) *tscale = t.g;
     const int64_t nb = cols / 16;
@@ -192,13 +205,13 @@ __global__ void __launch_bounds__(256) k_quant_1x16(const uint16_t* __restrict__
         const uint4 u0 = ld_nc_v4(p2), u1 = ld_nc_v4(p2 + 8);
         uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
         uint32_t s;
-        const uint2 q = quant_block16_m(w, amax_bits_16(w), t, tab, s);
+        const uint2 q = quant_block16_fast(w, t, tab, s);
         *reinterpret_cast<uint2*>(codes + r * (cols / 2) + c * 8) = q;
         scales[r * nb + c] = (uint8_t)s;
         if (slab) slab[slab_offset(r, c, cols)] = (uint8_t)s;
         if (two) {
             uint32_t w2[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-            const uint2 q2 = quant_block16_m(w2, amax_bits_16(w2), t, tab, s);
+            const uint2 q2 = quant_block16_fast(w2, t, tab, s);
             *reinterpret_cast<uint2*>(codes + r2 * (cols / 2) + c2 * 8) = q2;
             scales[r2 * nb + c2] = (uint8_t)s;
             if (slab) slab[slab_offset(r2, c2, cols)] = (uint8_t)s;
@@ -247,11 +260,6 @@ __global__ void __launch_bounds__(256) k_quant_tile16(
     uint8_t* __restrict__ scales_col, float* __restrict__ tscale, float* __restrict__ tscale2) {
     __shared__ __align__(16) QTileSmem sm;
     const QTensorFast qt = make_qtensor_fast(*amax);
-    build_qtable_m1(sm.tab, qt.g, threadIdx.x, blockDim.x);
-    __syncthreads();
-    build_qtable_m2(sm.tab, threadIdx.x, blockDim.x);
-    __syncthreads();
-    build_qtable_m3(sm.tab, threadIdx.x, blockDim.x);
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         *tscale = qt.g;
         if (tscale2) *tscale2 = qt.g;
@@ -269,13 +277,21 @@ __global__ void __launch_bounds__(256) k_quant_tile16(
         const int64_t r0 = (ti / ntc) * QTT_R, c0 = (ti % ntc) * QTT_C;
         const int vr = (int)min((int64_t)QTT_R, rows - r0);  // multiples of 16
         const int vc = (int)min((int64_t)QTT_C, cols - c0);
-        __syncthreads();  // the previous tile's shared reads are done (and the table is built)
+        __syncthreads();  // the previous tile's shared reads are done
         {
             uint4 v[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int i = tid + 256 * k, r = i >> 4, ch = i & 15;
                 v[k] = (r < vr && 8 * ch < vc) ? ld_nc_v4(x + (r0 + r) * ld + c0 + 8 * ch) : make_uint4(0, 0, 0, 0);
+            }
+            if (ti == blockIdx.x) {
+                // the encode table, built while the first tile's loads are in flight
+                build_qtable_m1(sm.tab, qt.g, tid, blockDim.x);
+                __syncthreads();
+                build_qtable_m2(sm.tab, tid, blockDim.x);
+                __syncthreads();
+                build_qtable_m3(sm.tab, tid, blockDim.x);
             }
 #pragma unroll
             for (int k = 0; k < 4; ++k) {

@@ -222,6 +222,14 @@ ft_status ft_pack_weight_operands_1x16(const uint8_t* codes_k, const uint8_t* sc
  *   N, K multiples of 16; 16-byte aligned pointers.  At least one output.  */
 ft_status ft_dequant_weight_operands(const ft_fp4* w_k, const ft_fp4* w_n, void* wd_k, void* wd_n, void* stream);
 
+/* ft_gelu_bf16 -- h = GELU(y) = y Phi(y) elementwise on bf16, each result
+ * the correctly rounded bf16 of the exact GELU (round to nearest even): the
+ * activation the fused MLP applies between its linears (section 3.3, "MLP
+ * Fusion"), for callers that apply it outside the fused path.
+ *   y, h : bf16 [n] device pointers, 16-byte aligned (may be equal); n a
+ *          multiple of 8.  NaN inputs are outside the contract.            */
+ft_status ft_gelu_bf16(const void* y, void* h, int64_t n, void* stream);
+
 /* ft_linear_fwd -- Eq. 2 with LoRA fusion (section 3.3): one pass over X
  * emits Q(X) and the down-projections P = [bf16(X U) | bf16(s X A)]; one
  * FP4 GEMM on tcgen05 block-scaled tensor cores adds P [V | B]^T in its
@@ -246,6 +254,35 @@ ft_status ft_linear_fwd(const ft_linear* L, const void* X, int64_t M, const floa
 ft_status ft_linear_bwd(const ft_linear* L, const void* dY, const void* X, const void* P_save,
                         int64_t M, const float* amax_dy, void* dX, ft_dtype xt, float* dA,
                         float* dB, void* ws, size_t ws_bytes, void* stream);
+
+/* ft_mlp_fwd -- the forward of a DiT MLP whose two linears are triple-
+ * branch layers, with MLP fusion (section 3.3, "MLP Fusion"): FC1's GEMM
+ * applies GELU in its epilogue and quantizes its output for FC2 as the
+ * tiles leave, so FC2 runs no quantization pass of its own.
+ *   Y_up = up's Eq. 2 output (FP32) rounded to bf16; H = GELU(Y_up) rounded
+ *   to bf16 (as ft_gelu_bf16); Y = down's Eq. 2 output on H.
+ *   up     : [N_up, K] layer; down: [N, N_up] layer (down->K == up->N);
+ *            both FT_W4A4G4.
+ *   X      : bf16 [M, K] dense;  amax_x: device max|X|, or NULL (computed).
+ *   amax_h : device float, required: the tensor amax that fixes the tensor
+ *            scale of Q(H).  The fused kernel quantizes H tile by tile,
+ *            before all of H exists, so max|H| cannot be measured first: the
+ *            caller passes a bound (e.g. the previous step's max|H|).  Values
+ *            above it saturate (block scale 448, codes +-6).
+ *   H      : bf16 [M, N_up] out: the down layer's input, for its backward.
+ *   Y      : [M, N] out, FT_BF16 or FT_F32 (yt).
+ *   P_up [M, up r_s + r_l], P_down [M, down r_s + r_l]: bf16 out, the
+ *            layers' saved down-projections (NULL when the rank is 0).
+ *   ws     : ft_mlp_workspace_bytes(up, down, M) bytes, zero-filled once.
+ *            After the call it holds Q(H) as the down layer's quantized
+ *            activation: at byte offset ft_workspace_bytes(M, up->N, up->K,
+ *            up->r_s, up->r_l) rounded up to a multiple of 256 lies the down
+ *            layer's workspace, laid out as ft_workspace_qact describes for
+ *            (M, down->N, down->K, down->r_s, down->r_l).                  */
+ft_status ft_mlp_fwd(const ft_linear* up, const ft_linear* down, const void* X, int64_t M, const float* amax_x,
+                     const float* amax_h, void* H, void* Y, ft_dtype yt, void* P_up, void* P_down, void* ws,
+                     size_t ws_bytes, void* stream);
+size_t ft_mlp_workspace_bytes(const ft_linear* up, const ft_linear* down, int64_t M);
 
 /* Workspace sizes (bytes) for the calls above.  Zero-fill a workspace once
  * after allocating it (e.g. cudaMemsetAsync); calls keep their
