@@ -8,22 +8,33 @@
 // The erfc form keeps its relative accuracy in the tail (1 + erf(t) would
 // cancel for y << 0).  A bf16 input takes one of 65536 values; the result
 // must be the correctly rounded bf16 of the exact GELU for every one of them.
-//   y >= 10        : y itself (1 - Phi(y) < 8e-24, far below half a bf16 ulp
-//                    of y).
-//   -10 <= y < 10  : FP32 first.  The FP32 evaluation's relative error is
-//                    below 2^-16 (erfcf's few ulps plus the argument's
-//                    rounding amplified by erfc's slope, 2 t^2 2^-23 at
-//                    t = 7.07); unless the FP32 value lies within 256 FP32
-//                    ulps (2^-15 relative) of a bf16 rounding midpoint, its
-//                    RNE rounding to bf16 is the correct one.
-//   otherwise      : double, rounded to bf16 from its exact binary value;
-//                    that covers the midpoint neighbourhoods, y < -10 and
-//                    results near or below the FP32 normal range (bf16
-//                    subnormals).  A double result exactly on a midpoint
-//                    arises only for subnormal y, where it is y / 2 with the
-//                    y^2 / sqrt(2 pi) term rounded away; the true value lies
-//                    above it (GELU(y) - y / 2 = y (Phi(y) - 1/2) > 0), so such
-//                    a tie rounds up.
+// An FP32 evaluation is accepted unless it lies within a margin of a bf16
+// rounding midpoint (where its own error could move it across), or near the
+// FP32 subnormal range; those cases are recomputed in double.  The margins
+// bound the FP32 evaluation's error on each range, in FP32 ulps of the
+// result:
+//   y >= 10        : y itself (1 - Phi(y) < 8e-24, far below half a bf16 ulp).
+//   0 <= y < 10    : 0.5 y erfcf(-y / sqrt 2): erfcf's few ulps and two
+//                    roundings; erfc(-t) in [1, 2] barely amplifies the
+//                    argument's rounding.  Margin 32 ulps.
+//   -3.125 <= y < 0: the same formula; erfc(t) amplifies the argument's
+//                    relative rounding (~2^-23.4) by up to 2 t^2 < 10.
+//                    Margin 32 ulps.
+//   -10 <= y < -3.125: the same, amplification up to 2 t^2 = 100.  Margin
+//                    128 ulps.
+//   y < -10        : with x = -y, Phi(y) = phi(x) / x (1 - 1/x^2 + 3/x^4 -
+//                    15/x^6 + 105/x^8 - ...), an alternating asymptotic
+//                    series whose first omitted term bounds the error (945 /
+//                    x^10 < 2^-23.3); so GELU(y) = -phi(x) S(1/x^2) with
+//                    phi(x) = exp(-x^2/2) / sqrt(2 pi), x^2 exact in FP32.
+//                    Margin 64 ulps; results below 2^-120 (x > ~12.9, bf16
+//                    subnormals and underflow) go to double.
+// In double, the value is rounded to bf16 from its exact binary value.  A
+// double result exactly on a midpoint arises only for subnormal y, where it
+// is y / 2 with the y^2 / sqrt(2 pi) term rounded away; the true value lies
+// above it (GELU(y) - y / 2 = y (Phi(y) - 1/2) > 0), so such a tie rounds up.
+// Every bf16 input is checked against a 50-digit reference through the
+// library's tests.
 #pragma once
 
 #include <cstdint>
@@ -56,11 +67,22 @@ __device__ __forceinline__ uint32_t gelu_bf16(uint32_t ybits) {
     ybits &= 0xFFFFu;
     const float y = __uint_as_float(ybits << 16);
     if (!(y < 10.0f)) return ybits;  // y >= 10 (and +inf); NaN is outside the contract
-    if (y < -10.0f) return gelu_bf16_slow(y);
-    const float h = __fmul_rn(__fmul_rn(0.5f, y), erfcf(__fmul_rn(-y, 0.70710678118654752f)));
+    float h;
+    uint32_t margin;
+    if (y >= -10.0f) {
+        h = __fmul_rn(__fmul_rn(0.5f, y), erfcf(__fmul_rn(-y, 0.70710678118654752f)));
+        margin = y >= -3.125f ? 32u : 128u;
+    } else {
+        const float x2 = __fmul_rn(y, y);  // exact: y has 8 significant bits
+        const float u = __frcp_rn(x2);
+        const float s = __fmaf_rn(-u, __fmaf_rn(-3.0f * u, __fmaf_rn(-5.0f * u, __fmaf_rn(-7.0f, u, 1.0f), 1.0f), 1.0f),
+                                  1.0f);
+        h = -__fmul_rn(__fmul_rn(expf(-0.5f * x2), 0.39894228040143268f), s);
+        margin = 64u;
+    }
     const uint32_t hb = __float_as_uint(h);
     const uint32_t low = hb & 0xFFFFu;
-    if ((hb & 0x7F800000u) < (7u << 23) || (low > 0x8000u - 256u && low < 0x8000u + 256u))
+    if ((hb & 0x7F800000u) < (7u << 23) || (low > 0x8000u - margin && low < 0x8000u + margin))
         return gelu_bf16_slow(y);
     return (hb + 0x7FFFu + ((hb >> 16) & 1u)) >> 16;
 }
