@@ -62,6 +62,9 @@ def parse_args():
                     help="token rows per linear per oracle step (reference arm / cpu baseline)")
     ap.add_argument("--skip-cpu-baseline", action="store_true",
                     help="omit the oracle timing (for profiler runs)")
+    ap.add_argument("--single", choices=["qkv", "out", "up", "down"], default=None,
+                    help="profiling: prepare one DiT-stack linear and run its forward and backward --steps "
+                         "times (prints 'ok', no timing)")
     ap.add_argument("--skip-extras", action="store_true",
                     help="omit the secondary figures (attention projection, standalone quantizers) "
                          "and the end-to-end leg (for profiler runs)")
@@ -840,10 +843,42 @@ def run_ours(args):
     return 0
 
 
+def run_single(args):
+    """One linear of the DiT stack, forward then backward, --steps times: a
+    short, fixed launch sequence for ncu captures (per step: the input's
+    quantizer -- k_qres, or k_amax_bf16 + k_qdown --, the forward GEMM, the
+    output gradient's quantizer, the dgrad GEMM, k_lora_grad)."""
+    import torch
+
+    import ft_synth
+    import bit_quantized_lora_b200 as ft
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    j = ["qkv", "out", "up", "down"].index(args.single)
+    sh = stack_shapes()[j]
+    inp = ft_synth.make_inputs(sh, seed=SEED + j)
+
+    def to_dev(u16):
+        return torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    layer = ft.prepare_layer(to_dev(inp["W"]), sh.r_s, A=to_dev(inp["A"]), B=to_dev(inp["B"]), s=inp["s"])
+    from bit_quantized_lora_b200.stack import LinearStack
+    st = LinearStack([layer], sh.M, dev)
+    X, dY = to_dev(inp["X"]), to_dev(inp["dY"])
+    for _ in range(args.steps):
+        st.step([X], [dY])
+    torch.cuda.synchronize()
+    assert ft.ft_device_error() == 0, "device error"
+    print("ok", flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.single:
+        return run_single(args)
     return run_ours(args)
 
 

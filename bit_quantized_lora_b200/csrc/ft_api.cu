@@ -787,9 +787,25 @@ ft_status run_lora_grads(const void* dY, const void* X, const void* P, const voi
     FT_TRY(encode_2d(&p.mapS[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Pg, r, M, r * 2, 64, LG::BMR,
                      CU_TENSOR_MAP_SWIZZLE_128B));
     const int ctiles = (int)(N / ft::lgrad::BC + K / ft::lgrad::BC);
-    int splits = std::max(1, std::min(LG_MAX_SPLITS, d->sms / std::max(1, ctiles)));
-    int mrows = cdiv(M, (int64_t)splits * ft::lgrad::BMR) * ft::lgrad::BMR;
-    splits = std::max(1, cdiv(M, mrows));
+    // token splits: the count that minimises (waves of CTAs, one per SM) x
+    // (128-token stages per CTA), plus a stage's worth per extra split for
+    // the partial sums; fewer splits on a tie
+    int splits = 1, mrows = cdiv(M, ft::lgrad::BMR) * ft::lgrad::BMR;
+    {
+        int64_t best = -1;
+        for (int s = 1; s <= LG_MAX_SPLITS; ++s) {
+            const int mr = cdiv(M, (int64_t)s * ft::lgrad::BMR) * ft::lgrad::BMR;
+            const int sp = std::max(1, cdiv(M, mr));
+            if (sp != s) continue;  // the same split as a smaller s
+            const int64_t waves = cdiv((int64_t)ctiles * sp, d->sms);
+            const int64_t cost = waves * (mr / ft::lgrad::BMR) + (sp - 1);
+            if (best < 0 || cost < best) {
+                best = cost;
+                splits = sp;
+                mrows = mr;
+            }
+        }
+    }
     float* partB = reinterpret_cast<float*>(ws + w.lgpart);
     float* partA = partB + (size_t)splits * N * r_l;
     p.part[0] = partB;
@@ -971,7 +987,7 @@ ft_status ft_gelu_bf16(const void* y, void* h, int64_t n, void* stream) {
     DevInfo* d;
     FT_TRY(device_info(&d));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(n / 8, 256), (int64_t)d->sms * 8));
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(n / 8, 256), (int64_t)d->sms * 4));
     LaunchTimer _lt(KID_GELU, st);
     ft::k_gelu_bf16<<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(y), static_cast<uint16_t*>(h), n);
     _lt.stop();

@@ -92,4 +92,46 @@ __device__ __forceinline__ uint32_t gelu_bf16x2(uint32_t w) {
     return gelu_bf16(w) | (gelu_bf16(w >> 16) << 16);
 }
 
+// ---------------------------------------------------------------- table form
+// The kernels that apply GELU to many values read the results for the 2048
+// bf16 inputs with 2^-4 <= |y| < 2^4 (8 exponents x 128 mantissas x 2
+// signs: the bulk of any activation) from a 4 KB shared-memory table,
+// filled once per CTA by the double path above.  Outside it:
+//   |y| >= 16      : y for y > 0; -0 for y < 0 (|GELU(y)| < 2^-134, below
+//                    half the smallest bf16 subnormal).
+//   |y| < 2^-4     : GELU(y) = y/2 + phi(0) y^2 (1 - y^2/6) + O(y^6), the
+//                    Taylor series of y Phi(y) at 0; the omitted terms are
+//                    below 2^-25 of the value, FP32 evaluation adds a few
+//                    ulps: margin 16 ulps, else (and for subnormal or
+//                    FP32-subnormal results) the double path.
+constexpr int kGeluTab = 2048;
+
+__device__ __forceinline__ void gelu_table_build(uint16_t* tab, int tid, int nthreads) {
+    for (int i = tid; i < kGeluTab; i += nthreads) {
+        const uint32_t b = ((uint32_t)(i >> 10) << 15) | ((123u + ((uint32_t)i >> 7 & 7u)) << 7) | ((uint32_t)i & 127u);
+        tab[i] = (uint16_t)gelu_bf16_slow(__uint_as_float(b << 16));
+    }
+}
+
+__device__ __forceinline__ uint32_t gelu_bf16_tab(uint32_t ybits, const uint16_t* tab) {
+    ybits &= 0xFFFFu;
+    const uint32_t e = (ybits >> 7) & 0xFFu;
+    if (e - 123u <= 7u) return tab[((ybits >> 5) & 0x400u) | ((e - 123u) << 7) | (ybits & 0x7Fu)];
+    if (e > 130u) return (ybits & 0x8000u) ? 0x8000u : ybits;
+    if (e == 0u) return gelu_bf16_slow(__uint_as_float(ybits << 16));
+    const float y = __uint_as_float(ybits << 16);
+    const float y2 = __fmul_rn(y, y);
+    const float c = __fmaf_rn(y2, -0.066490380066905446f, 0.39894228040143268f);  // phi(0) (1 - y^2 / 6)
+    const float h = __fmul_rn(__fmaf_rn(c, y, 0.5f), y);
+    const uint32_t hb = __float_as_uint(h);
+    const uint32_t low = hb & 0xFFFFu;
+    if ((hb & 0x7F800000u) < (7u << 23) || (low > 0x8000u - 16u && low < 0x8000u + 16u))
+        return gelu_bf16_slow(y);
+    return (hb + 0x7FFFu + ((hb >> 16) & 1u)) >> 16;
+}
+
+__device__ __forceinline__ uint32_t gelu_bf16x2_tab(uint32_t w, const uint16_t* tab) {
+    return gelu_bf16_tab(w, tab) | (gelu_bf16_tab(w >> 16, tab) << 16);
+}
+
 }  // namespace ft

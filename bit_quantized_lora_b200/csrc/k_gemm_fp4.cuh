@@ -151,7 +151,7 @@ __host__ __device__ inline Layout make_layout(int stages, const LrFactor& f1, co
     L.l2 = o;   o += l_bytes(f2);
     L.sfa = o;  o += stages * SFA_STAGE_BYTES;
     L.stg = o;  o += 2 * STG_BYTES;  // output staging, one buffer per column group
-    L.tab = o;  o += mlp ? (uint32_t)sizeof(QTableM) : 0u;  // the encode table of Q(H)
+    L.tab = o;  o += mlp ? (uint32_t)sizeof(QTableM) + 2u * kGeluTab : 0u;  // Q(H)'s encode table, GELU's
     o = (o + 15u) & ~15u;
     L.bars = o; o += 256;  // barriers, TMEM slot, abort flag
     L.total = o + 1024;    // slack for 1 KiB alignment of the base
@@ -506,6 +506,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
         // MLP fusion: the encode table of Q(H) for the caller's tensor amax,
         // built by the 256 epilogue threads before the first accumulator
         QTableM& tab = *reinterpret_cast<QTableM*>(smem + L.tab);
+        uint16_t* gtab = reinterpret_cast<uint16_t*>(smem + L.tab + sizeof(QTableM));
         QTensorFast qt;
         qt.g = qt.six_g = qt.y6 = 0.0f;
         if (kMlp) {
@@ -518,6 +519,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             build_qtable_m3(tab, et2, 32 * NUM_EPI_WARPS);
             named_bar_sync(3, 32 * NUM_EPI_WARPS);
             if (blockIdx.x == 0 && et2 == 0) *p.q_tscale = qt.g;
+            // GELU's table (the first tile's mainloop runs meanwhile)
+            gelu_table_build(gtab, et2, 32 * NUM_EPI_WARPS);
+            named_bar_sync(3, 32 * NUM_EPI_WARPS);
         }
         for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
             const int m0 = (tile / tiles_n) * BM;
@@ -584,7 +588,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     for (int c = 0; c < 8; ++c) {
                         uint32_t w[8];
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) w[k] = gelu_bf16x2(pk[c][k]);
+                        for (int k = 0; k < 8; ++k) w[k] = gelu_bf16x2_tab(pk[c][k], gtab);
                         uint32_t sbyte;
                         const uint2 q = quant_block16_m(w, amax_bits_16(w), qt, tab, sbyte);
                         if (row < p.M)

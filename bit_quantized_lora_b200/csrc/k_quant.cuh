@@ -14,15 +14,23 @@
 namespace ft {
 
 // ------------------------------------------------------------------ GELU
-// h = GELU(y) elementwise on bf16 (ft_gelu.cuh), 8 values per 16-byte load;
-// n a multiple of 8, pointers 16-byte aligned.
+// h = GELU(y) elementwise on bf16 (ft_gelu.cuh, the table form), 8 values
+// per 16-byte load; persistent CTAs, each filling its table once (its first
+// loads are in flight meanwhile); n a multiple of 8, pointers 16-byte aligned.
 __global__ void __launch_bounds__(256) k_gelu_bf16(const uint16_t* __restrict__ y, uint16_t* __restrict__ h,
                                                    int64_t n) {
+    __shared__ uint16_t tab[kGeluTab];
     const int64_t n8 = n / 8;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
-        const uint4 v = ld_nc_v4(y + 8 * i);
-        *reinterpret_cast<uint4*>(h + 8 * i) =
-            make_uint4(gelu_bf16x2(v.x), gelu_bf16x2(v.y), gelu_bf16x2(v.z), gelu_bf16x2(v.w));
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    uint4 v = i < n8 ? ld_nc_v4(y + 8 * i) : make_uint4(0, 0, 0, 0);
+    gelu_table_build(tab, threadIdx.x, blockDim.x);
+    __syncthreads();
+    for (; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t j = i + (int64_t)gridDim.x * blockDim.x;
+        const uint4 nv = j < n8 ? ld_nc_v4(y + 8 * j) : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(h + 8 * i) = make_uint4(gelu_bf16x2_tab(v.x, tab), gelu_bf16x2_tab(v.y, tab),
+                                                          gelu_bf16x2_tab(v.z, tab), gelu_bf16x2_tab(v.w, tab));
+        v = nv;
     }
 }
 
@@ -32,7 +40,7 @@ __global__ void __launch_bounds__(256) k_gelu_bf16(const uint16_t* __restrict__ 
 // the float bits (non-negative floats order like their bit patterns), so the
 // result is exact and independent of scheduling.  *out must be 0 on entry.
 // The grid is kept to a few blocks per SM (same-address atomics serialise in
-// L2); each thread keeps eight independent 16-byte loads in flight.
+// L2); each thread keeps eight to sixteen independent 16-byte loads in flight.
 __global__ void __launch_bounds__(256) k_amax_bf16(const uint16_t* __restrict__ x, int64_t rows,
                                                    int64_t cols, int64_t ld,
                                                    unsigned int* __restrict__ out) {
@@ -43,12 +51,19 @@ __global__ void __launch_bounds__(256) k_amax_bf16(const uint16_t* __restrict__ 
     uint32_t m = 0;
     int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (ld == cols) {
+        // software-pipelined: the next eight loads are issued before the
+        // current eight are reduced, so a thread always has a batch in flight
         const uint4* xv = reinterpret_cast<const uint4*>(x);
+        uint4 v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            v[u] = (i + u * nthr < total) ? ld_nc_v4(xv + i + u * nthr) : make_uint4(0, 0, 0, 0);
         for (; i < total; i += U * nthr) {
-            uint4 v[U];
+            const int64_t j = i + U * nthr;
+            uint4 nv[U];
 #pragma unroll
             for (int u = 0; u < U; ++u)
-                v[u] = (i + u * nthr < total) ? ld_nc_v4(xv + i + u * nthr) : make_uint4(0, 0, 0, 0);
+                nv[u] = (j + u * nthr < total) ? ld_nc_v4(xv + j + u * nthr) : make_uint4(0, 0, 0, 0);
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 m = __vmaxu2(m, v[u].x & 0x7FFF7FFFu);
@@ -56,6 +71,8 @@ __global__ void __launch_bounds__(256) k_amax_bf16(const uint16_t* __restrict__ 
                 m = __vmaxu2(m, v[u].z & 0x7FFF7FFFu);
                 m = __vmaxu2(m, v[u].w & 0x7FFF7FFFu);
             }
+#pragma unroll
+            for (int u = 0; u < U; ++u) v[u] = nv[u];
         }
         i = total;
     }
