@@ -48,7 +48,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 N_BLOCKS = 8
 SEED = 100  # linear type j of the stack draws its tensors from seed SEED + j (weights) / rank_seed(.., rank)
 KERNELS = ["k_gemm_fp4", "k_qres", "k_qdown", "k_amax_bf16", "k_lora_grad", "k_pack_lt", "k_quant_1x16",
-           "k_quant_tile16"]
+           "k_quant_tile16", "k_gelu_bf16"]
 
 
 def parse_args():
@@ -62,7 +62,7 @@ def parse_args():
                     help="token rows per linear per oracle step (reference arm / cpu baseline)")
     ap.add_argument("--skip-cpu-baseline", action="store_true",
                     help="omit the oracle timing (for profiler runs)")
-    ap.add_argument("--single", choices=["qkv", "out", "up", "down"], default=None,
+    ap.add_argument("--single", choices=["qkv", "out", "up", "down", "mlp"], default=None,
                     help="profiling: prepare one DiT-stack linear and run its forward and backward --steps "
                          "times (prints 'ok', no timing)")
     ap.add_argument("--skip-extras", action="store_true",
@@ -621,6 +621,8 @@ def bench_mlp(torch, ft, dev, flush, reps=10):
         fn()
         torch.cuda.synchronize()
         ms = []
+        ft.timing.reset()
+        ft.timing.enable(True)
         for _ in range(reps):
             flush()
             keep_host_ahead(torch, 1)
@@ -630,7 +632,11 @@ def bench_mlp(torch, ft, dev, flush, reps=10):
             e1.record(stream)
             e1.synchronize()
             ms.append(e0.elapsed_time(e1))
+        ft.timing.enable(False)
         out[name + "_ms"] = statistics.median(ms)
+        kern = {k: ft.timing.read(k) for k in KERNELS}
+        # per forward: the summed time of each kernel's launches in it
+        out[name + "_kernels_us"] = {k: round(v[0] / reps * 1e3, 2) for k, v in kern.items() if v[1]}
     assert ft.ft_device_error() == 0, "device error in the MLP section"
     out["speedup_vs_unfused_supplied"] = out["unfused_supplied_amax_ms"] / out["fused_ms"]
     out["speedup_vs_unfused_computed"] = out["unfused_computed_amax_ms"] / out["fused_ms"]
@@ -847,13 +853,18 @@ def run_single(args):
     """One linear of the DiT stack, forward then backward, --steps times: a
     short, fixed launch sequence for ncu captures (per step: the input's
     quantizer -- k_qres, or k_amax_bf16 + k_qdown --, the forward GEMM, the
-    output gradient's quantizer, the dgrad GEMM, k_lora_grad)."""
+    output gradient's quantizer, the dgrad GEMM, k_lora_grad).  With
+    "mlp": one DiT block's fused MLP forward per step (k_qres of X, FC1's
+    GEMM with the GELU + Q(H) epilogue, k_qdown's P-only pass over H, FC2's
+    GEMM)."""
     import torch
 
     import ft_synth
     import bit_quantized_lora_b200 as ft
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
+    if args.single == "mlp":
+        return run_single_mlp(args, torch, ft, dev)
     j = ["qkv", "out", "up", "down"].index(args.single)
     sh = stack_shapes()[j]
     inp = ft_synth.make_inputs(sh, seed=SEED + j)
@@ -867,6 +878,32 @@ def run_single(args):
     X, dY = to_dev(inp["X"]), to_dev(inp["dY"])
     for _ in range(args.steps):
         st.step([X], [dY])
+    torch.cuda.synchronize()
+    assert ft.ft_device_error() == 0, "device error"
+    print("ok", flush=True)
+    return 0
+
+
+def run_single_mlp(args, torch, ft, dev):
+    import ft_synth
+    sh_up, sh_dn = stack_shapes()[2], stack_shapes()[3]
+
+    def to_dev(u16):
+        return torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    iu = ft_synth.make_inputs(sh_up, seed=SEED + 2)
+    wd = ft_synth.make_inputs(dataclasses_replace(sh_dn, M=16), seed=SEED + 3)
+    up = ft.prepare_layer(to_dev(iu["W"]), sh_up.r_s, A=to_dev(iu["A"]), B=to_dev(iu["B"]), s=iu["s"])
+    dn = ft.prepare_layer(to_dev(wd["W"]), sh_dn.r_s, A=to_dev(wd["A"]), B=to_dev(wd["B"]), s=wd["s"])
+    X = to_dev(iu["X"])
+    # H's tensor amax from one unfused FC1 + GELU (one k_gemm_fp4 launch
+    # before the loop's)
+    Y_up, _ = ft.ft_linear_fwd(up, X)
+    amax_h = ft.ft_gelu_bf16(Y_up).abs().max().float().reshape(1)
+    del Y_up
+    ws = ft.Workspace()
+    for _ in range(args.steps):
+        ft.ft_mlp_fwd(up, dn, X, amax_h, ws=ws)
     torch.cuda.synchronize()
     assert ft.ft_device_error() == 0, "device error"
     print("ok", flush=True)

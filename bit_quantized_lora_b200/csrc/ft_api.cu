@@ -787,25 +787,9 @@ ft_status run_lora_grads(const void* dY, const void* X, const void* P, const voi
     FT_TRY(encode_2d(&p.mapS[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Pg, r, M, r * 2, 64, LG::BMR,
                      CU_TENSOR_MAP_SWIZZLE_128B));
     const int ctiles = (int)(N / ft::lgrad::BC + K / ft::lgrad::BC);
-    // token splits: the count that minimises (waves of CTAs, one per SM) x
-    // (128-token stages per CTA), plus a stage's worth per extra split for
-    // the partial sums; fewer splits on a tie
-    int splits = 1, mrows = cdiv(M, ft::lgrad::BMR) * ft::lgrad::BMR;
-    {
-        int64_t best = -1;
-        for (int s = 1; s <= LG_MAX_SPLITS; ++s) {
-            const int mr = cdiv(M, (int64_t)s * ft::lgrad::BMR) * ft::lgrad::BMR;
-            const int sp = std::max(1, cdiv(M, mr));
-            if (sp != s) continue;  // the same split as a smaller s
-            const int64_t waves = cdiv((int64_t)ctiles * sp, d->sms);
-            const int64_t cost = waves * (mr / ft::lgrad::BMR) + (sp - 1);
-            if (best < 0 || cost < best) {
-                best = cost;
-                splits = sp;
-                mrows = mr;
-            }
-        }
-    }
+    int splits = std::max(1, std::min(LG_MAX_SPLITS, d->sms / std::max(1, ctiles)));
+    int mrows = cdiv(M, (int64_t)splits * ft::lgrad::BMR) * ft::lgrad::BMR;
+    splits = std::max(1, cdiv(M, mrows));
     float* partB = reinterpret_cast<float*>(ws + w.lgpart);
     float* partA = partB + (size_t)splits * N * r_l;
     p.part[0] = partB;
@@ -1207,8 +1191,9 @@ ft_status ft_mlp_fwd(const ft_linear* up, const ft_linear* down, const void* X, 
     if (M == 0) return FT_OK;
     const int64_t r_up = up->r_s + up->r_l, r_dn = down->r_s + down->r_l;
     if (!X || !amax_h || !H || !Y || (r_up > 0 && !P_up) || (r_dn > 0 && !P_down)) return FT_ERR_INVALID_ARG;
-    if (!al16(X) || !al16(H) || !al16(Y) || (P_up && !al16(P_up)) || (P_down && !al16(P_down)) ||
-        (reinterpret_cast<uintptr_t>(amax_h) & 3u))
+    // H leaves the fused epilogue in whole 32-byte sectors
+    if (!al16(X) || (reinterpret_cast<uintptr_t>(H) & 31u) || !al16(Y) || (P_up && !al16(P_up)) ||
+        (P_down && !al16(P_down)) || (reinterpret_cast<uintptr_t>(amax_h) & 3u))
         return FT_ERR_ALIGN;
     const WsPlan wu = plan_ws(M, up->N, up->K, up->r_s, up->r_l);
     const WsPlan wd = plan_ws(M, down->N, down->K, down->r_s, down->r_l);

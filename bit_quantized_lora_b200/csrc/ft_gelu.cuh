@@ -87,37 +87,38 @@ __device__ __forceinline__ uint32_t gelu_bf16(uint32_t ybits) {
     return (hb + 0x7FFFu + ((hb >> 16) & 1u)) >> 16;
 }
 
-// GELU of two bf16 values packed in a word (element 0 in the low half).
-__device__ __forceinline__ uint32_t gelu_bf16x2(uint32_t w) {
-    return gelu_bf16(w) | (gelu_bf16(w >> 16) << 16);
-}
-
 // ---------------------------------------------------------------- table form
-// The kernels that apply GELU to many values read the results for the 2048
-// bf16 inputs with 2^-4 <= |y| < 2^4 (8 exponents x 128 mantissas x 2
-// signs: the bulk of any activation) from a 4 KB shared-memory table,
-// filled once per CTA by the double path above.  Outside it:
+// The kernels that apply GELU to many values read the results for the 4096
+// bf16 inputs with 2^-12 <= |y| < 2^4 (16 exponents x 128 mantissas x 2
+// signs: all but a sliver of any activation) from an 8 KB shared-memory
+// table, filled once per CTA by gelu_bf16 above (FP32, double near a
+// rounding midpoint: correctly rounded either way).  Outside it:
 //   |y| >= 16      : y for y > 0; -0 for y < 0 (|GELU(y)| < 2^-134, below
 //                    half the smallest bf16 subnormal).
-//   |y| < 2^-4     : GELU(y) = y/2 + phi(0) y^2 (1 - y^2/6) + O(y^6), the
+//   y = +-0        : y.
+//   |y| < 2^-12    : GELU(y) = y/2 + phi(0) y^2 (1 - y^2/6) + O(y^6), the
 //                    Taylor series of y Phi(y) at 0; the omitted terms are
-//                    below 2^-25 of the value, FP32 evaluation adds a few
-//                    ulps: margin 16 ulps, else (and for subnormal or
+//                    far below 2^-25 of the value, FP32 evaluation adds a few
+//                    ulps: margin 16 ulps, else (and for subnormal inputs or
 //                    FP32-subnormal results) the double path.
-constexpr int kGeluTab = 2048;
+// Table entry s << 11 | (e - 115) << 7 | m holds GELU of the bf16 with sign
+// s, biased exponent e (115..130) and mantissa m.
+constexpr int kGeluTab = 4096;
 
 __device__ __forceinline__ void gelu_table_build(uint16_t* tab, int tid, int nthreads) {
     for (int i = tid; i < kGeluTab; i += nthreads) {
-        const uint32_t b = ((uint32_t)(i >> 10) << 15) | ((123u + ((uint32_t)i >> 7 & 7u)) << 7) | ((uint32_t)i & 127u);
-        tab[i] = (uint16_t)gelu_bf16_slow(__uint_as_float(b << 16));
+        const uint32_t b = ((uint32_t)(i >> 11) << 15) | ((115u + ((uint32_t)i >> 7 & 15u)) << 7) | ((uint32_t)i & 127u);
+        tab[i] = (uint16_t)gelu_bf16(b);
     }
 }
 
+// One value (low 16 bits of ybits) by the table and the cases around it.
 __device__ __forceinline__ uint32_t gelu_bf16_tab(uint32_t ybits, const uint16_t* tab) {
     ybits &= 0xFFFFu;
     const uint32_t e = (ybits >> 7) & 0xFFu;
-    if (e - 123u <= 7u) return tab[((ybits >> 5) & 0x400u) | ((e - 123u) << 7) | (ybits & 0x7Fu)];
+    if (e - 115u <= 15u) return tab[((ybits >> 4) & 0x800u) | ((e - 115u) << 7) | (ybits & 0x7Fu)];
     if (e > 130u) return (ybits & 0x8000u) ? 0x8000u : ybits;
+    if ((ybits & 0x7FFFu) == 0u) return ybits;
     if (e == 0u) return gelu_bf16_slow(__uint_as_float(ybits << 16));
     const float y = __uint_as_float(ybits << 16);
     const float y2 = __fmul_rn(y, y);
@@ -130,8 +131,24 @@ __device__ __forceinline__ uint32_t gelu_bf16_tab(uint32_t ybits, const uint16_t
     return (hb + 0x7FFFu + ((hb >> 16) & 1u)) >> 16;
 }
 
-__device__ __forceinline__ uint32_t gelu_bf16x2_tab(uint32_t w, const uint16_t* tab) {
+// Both halves of a word, one at a time: the rare case of the packed form,
+// kept out of line so that the common path stays short.
+__device__ __noinline__ uint32_t gelu_bf16x2_rare(uint32_t w, const uint16_t* tab) {
     return gelu_bf16_tab(w, tab) | (gelu_bf16_tab(w >> 16, tab) << 16);
+}
+
+// Two bf16 values packed in a word (element 0 in the low half).  Both
+// exponents are offset by 141 in their own 16-bit lanes (no carry between
+// them: 255 + 141 < 2^16), so each lies in [256, 272) exactly when its value
+// is inside the table, and both table indices are assembled in one word.
+// The indices are in range whatever the exponents; the loads go first and
+// the rare case replaces their result.
+__device__ __forceinline__ uint32_t gelu_bf16x2_tab(uint32_t w, const uint16_t* tab) {
+    const uint32_t v = ((w >> 7) & 0x00FF00FFu) + 0x008D008Du;
+    const uint32_t i = ((w >> 4) & 0x08000800u) | ((v & 0x000F000Fu) << 7) | (w & 0x007F007Fu);
+    uint32_t r = (uint32_t)tab[i & 0xFFFFu] | ((uint32_t)tab[i >> 16] << 16);
+    if ((v & 0xFFF0FFF0u) != 0x01000100u) r = gelu_bf16x2_rare(w, tab);
+    return r;
 }
 
 }  // namespace ft

@@ -150,7 +150,7 @@ __host__ __device__ inline Layout make_layout(int stages, const LrFactor& f1, co
     L.p2 = o;   o += p_bytes(f2);
     L.l2 = o;   o += l_bytes(f2);
     L.sfa = o;  o += stages * SFA_STAGE_BYTES;
-    L.stg = o;  o += 2 * STG_BYTES;  // output staging, one buffer per column group
+    L.stg = o;  o += mlp ? 0u : 2 * STG_BYTES;  // output staging, one buffer per column group (H: none)
     L.tab = o;  o += mlp ? (uint32_t)sizeof(QTableM) + 2u * kGeluTab : 0u;  // Q(H)'s encode table, GELU's
     o = (o + 15u) & ~15u;
     L.bars = o; o += 256;  // barriers, TMEM slot, abort flag
@@ -552,7 +552,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     if (m0 + row < p.M) *reinterpret_cast<uint4*>(obase + (int64_t)row * ldo + 16 * q) = v;
                 }
             };
-            if (!p.out_f32) {
+            if (kMlp || !p.out_f32) {
                 // bf16: the group's 128 columns of this row are read out of
                 // tensor memory and packed first, so the accumulator is
                 // released before the stores and the next tile's MMAs run
@@ -579,10 +579,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[B_ACC_EMPTY]);
                 if (kMlp) {
-                    // MLP fusion: H = GELU(y) per bf16 value; a 16-column
-                    // chunk of the row is exactly one 1x16 block of Q(H)
+                    // MLP fusion: H = GELU(y) per bf16 value.  A 16-column
+                    // chunk of the row is one 1x16 block of Q(H), and its 32
+                    // bytes of H are one whole sector, stored straight from
+                    // registers (no staging, no barriers between the group's
+                    // warps).
                     const int row = m0 + et;
+                    const bool in = row < p.M;
                     const int64_t qcol = n0 + 128 * grp;  // first column of the group
+                    uint8_t* hrow = p.out + (int64_t)row * ldo + qcol * 2;
+                    uint8_t* crow = p.q_codes + (int64_t)row * (p.Nout / 2) + qcol / 2;
                     uint32_t sw0 = 0, sw1 = 0;
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
@@ -591,16 +597,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                         for (int k = 0; k < 8; ++k) w[k] = gelu_bf16x2_tab(pk[c][k], gtab);
                         uint32_t sbyte;
                         const uint2 q = quant_block16_m(w, amax_bits_16(w), qt, tab, sbyte);
-                        if (row < p.M)
-                            *reinterpret_cast<uint2*>(p.q_codes + (int64_t)row * (p.Nout / 2) + (qcol + 16 * c) / 2) = q;
+                        if (in) {
+                            st_global_v8(hrow + 32 * c, w);
+                            *reinterpret_cast<uint2*>(crow + 8 * c) = q;
+                        }
                         if (c < 4) sw0 |= sbyte << (8 * c);
                         else sw1 |= sbyte << (8 * (c - 4));
-                        named_bar_sync(1 + grp, 128);
-                        stage(make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]));
-                        named_bar_sync(1 + grp, 128);
-                        copy_out(128 * grp + 16 * c);
                     }
-                    if (row < p.M)
+                    if (in)
                         *reinterpret_cast<uint2*>(p.q_scales + (int64_t)row * (p.Nout / 16) + qcol / 16) =
                             make_uint2(sw0, sw1);
                     // slab rows past M hold the (zero) scales of the zero-filled rows

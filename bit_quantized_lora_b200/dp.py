@@ -43,6 +43,16 @@ class AdapterGrads:
         exchange is only started and its handle returned: a training loop
         overlaps it with the next layer's backward and calls wait() before
         the optimizer reads dA, dB (None when there is nothing to exchange).
+
+        An exchange in flight occupies SMs.  The library's single-pass
+        quantizer (a layer call with no tensor amax supplied) joins its CTAs
+        at a grid-wide barrier, so launched plainly beside a running
+        all-reduce it can find some of its CTAs unscheduled: its bounded wait
+        then gives up and ft_device_error() reports a timeout.  While
+        exchanges overlap layer calls, either switch the quantizer to a
+        cooperative launch (ft_set_cooperative_quantizer(True), as
+        stack.LinearStack.step does), supply the tensor amax, or read
+        ft_device_error() after the step.
         """
         if dist.is_initialized() and dist.get_world_size(group) > 1:
             return dist.all_reduce(self.flat, op=dist.ReduceOp.SUM, group=group, async_op=async_op)

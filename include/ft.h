@@ -269,7 +269,8 @@ ft_status ft_linear_bwd(const ft_linear* L, const void* dY, const void* X, const
  *            before all of H exists, so max|H| cannot be measured first: the
  *            caller passes a bound (e.g. the previous step's max|H|).  Values
  *            above it saturate (block scale 448, codes +-6).
- *   H      : bf16 [M, N_up] out: the down layer's input, for its backward.
+ *   H      : bf16 [M, N_up] out: the down layer's input, for its backward;
+ *            32-byte aligned (FT_ERR_ALIGN otherwise).
  *   Y      : [M, N] out, FT_BF16 or FT_F32 (yt).
  *   P_up [M, up r_s + r_l], P_down [M, down r_s + r_l]: bf16 out, the
  *            layers' saved down-projections (NULL when the rank is 0).
