@@ -971,9 +971,10 @@ ft_status ft_gelu_bf16(const void* y, void* h, int64_t n, void* stream) {
     DevInfo* d;
     FT_TRY(device_info(&d));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(n / 8, 256), (int64_t)d->sms * 4));
+    // one CTA of 1024 threads per SM: each CTA fills its own GELU table
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(n / 8, 1024), (int64_t)d->sms));
     LaunchTimer _lt(KID_GELU, st);
-    ft::k_gelu_bf16<<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(y), static_cast<uint16_t*>(h), n);
+    ft::k_gelu_bf16<<<grid, 1024, 0, st>>>(static_cast<const uint16_t*>(y), static_cast<uint16_t*>(h), n);
     _lt.stop();
     return last_launch();
 }

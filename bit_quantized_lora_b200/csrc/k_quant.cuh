@@ -17,7 +17,7 @@ namespace ft {
 // h = GELU(y) elementwise on bf16 (ft_gelu.cuh, the table form), 8 values
 // per 16-byte load; persistent CTAs, each filling its table once (its first
 // loads are in flight meanwhile); n a multiple of 8, pointers 16-byte aligned.
-__global__ void __launch_bounds__(256) k_gelu_bf16(const uint16_t* __restrict__ y, uint16_t* __restrict__ h,
+__global__ void __launch_bounds__(1024) k_gelu_bf16(const uint16_t* __restrict__ y, uint16_t* __restrict__ h,
                                                    int64_t n) {
     __shared__ uint16_t tab[kGeluTab];
     const int64_t n8 = n / 8;
