@@ -68,6 +68,9 @@ def parse_args():
     ap.add_argument("--skip-extras", action="store_true",
                     help="omit the secondary figures (attention projection, standalone quantizers) "
                          "and the end-to-end leg (for profiler runs)")
+    ap.add_argument("--gemm-mode", choices=["pairs", "single"], default="pairs",
+                    help="tiling of the 4-bit GEMMs: CTA pairs on 256 x 256 tiles (default) or one CTA per "
+                         "128 x 256 tile (same results)")
     return ap.parse_args()
 
 
@@ -773,6 +776,7 @@ def run_ours(args):
             "global_batch": M * world,
             "seq_len": M,
             "parallelism": f"dp{world}" if world > 1 else "single",
+            "gemm_tiling": "CTA pairs, 256 x 256 tiles" if args.gemm_mode == "pairs" else "one CTA per 128 x 256 tile",
             "l2": "inputs larger than L2 (the step touches several GB) and flushed between steps "
                   "(256 MB write then 256 MB read, outside the step events)",
         },
@@ -914,6 +918,9 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.gemm_mode == "single":
+        import bit_quantized_lora_b200 as ft
+        ft.ft_set_gemm_mode(ft.GEMM_SINGLE)
     if args.single:
         return run_single(args)
     return run_ours(args)

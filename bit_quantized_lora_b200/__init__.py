@@ -33,7 +33,7 @@ __all__ = [
     "ft_mlp_fwd", "ft_mlp_workspace_bytes",
     "ft_quantize", "ft_quantize_transpose", "ft_linear_fwd", "ft_linear_bwd",
     "ft_workspace_bytes", "ft_quantize_workspace_bytes", "ft_device_error",
-    "ft_set_cooperative_quantizer", "prepare_layer", "svd_split", "Workspace", "timing",
+    "ft_set_cooperative_quantizer", "ft_set_gemm_mode", "GEMM_PAIRS", "GEMM_SINGLE", "prepare_layer", "svd_split", "Workspace", "timing",
 ]
 
 
@@ -376,6 +376,16 @@ def ft_set_cooperative_quantizer(on: bool) -> None:
     default) = plain launch, True = cooperative launch (safe next to other
     streams' long-running kernels, ~3 us later start per call)."""
     check("ft_set_cooperative_quantizer", load().ft_set_cooperative_quantizer(1 if on else 0))
+
+
+GEMM_PAIRS, GEMM_SINGLE = 0, 1
+
+
+def ft_set_gemm_mode(mode: int) -> None:
+    """Tiling of the 4-bit GEMMs: GEMM_PAIRS (the default: CTA pairs share
+    256 x 256 tiles when the activation has more than 128 rows) or
+    GEMM_SINGLE (one CTA per 128 x 256 tile).  Same results either way."""
+    check("ft_set_gemm_mode", load().ft_set_gemm_mode(int(mode)))
 
 
 class timing:

@@ -70,6 +70,7 @@ SIGNATURES = {
                                          ctypes.POINTER(ctypes.c_size_t)]),
     "ft_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int), c_vp]),
     "ft_set_cooperative_quantizer": (ctypes.c_int, [ctypes.c_int]),
+    "ft_set_gemm_mode": (ctypes.c_int, [ctypes.c_int]),
     "ft_status_str": (ctypes.c_char_p, [ctypes.c_int]),
     "ft_linear_fwd_noalloc": (ctypes.c_int, [ctypes.POINTER(FtLinear), c_vp, c_i64, c_vp, c_vp,
                                              ctypes.c_int, c_vp, c_vp]),

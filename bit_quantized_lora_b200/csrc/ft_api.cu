@@ -106,6 +106,10 @@ ft_status device_info(DevInfo** out) {
                                  big) != cudaSuccess ||
             cudaFuncSetAttribute(ft::gemm::k_gemm_fp4<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  big) != cudaSuccess ||
+            cudaFuncSetAttribute(ft::gemm::k_gemm_fp4<false, false, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, big) != cudaSuccess ||
+            cudaFuncSetAttribute(ft::gemm::k_gemm_fp4<false, true, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, big) != cudaSuccess ||
             cudaFuncSetAttribute(ft::qdown::k_qdown, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)ft::qdown::SMEM_BYTES) != cudaSuccess ||
             cudaFuncSetAttribute(ft::lgrad::k_lora_grad, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -119,6 +123,8 @@ ft_status device_info(DevInfo** out) {
             reinterpret_cast<const void*>(ft::gemm::k_gemm_fp4<false>),
             reinterpret_cast<const void*>(ft::gemm::k_gemm_fp4<true>),
             reinterpret_cast<const void*>(ft::gemm::k_gemm_fp4<false, true>),
+            reinterpret_cast<const void*>(ft::gemm::k_gemm_fp4<false, false, true>),
+            reinterpret_cast<const void*>(ft::gemm::k_gemm_fp4<false, true, true>),
             reinterpret_cast<const void*>(ft::qres::k_qres),
             reinterpret_cast<const void*>(ft::qdown::k_qdown),
             reinterpret_cast<const void*>(ft::lgrad::k_lora_grad),
@@ -150,18 +156,28 @@ inline ft_status last_launch() { return cuda_ok(cudaGetLastError()); }
 // Launches `kernel` so that it may begin while the previous kernel on the
 // stream finishes (programmatic stream serialization): the kernel waits for
 // that kernel's results itself (grid_dep_wait) after its setup.
+// cluster_x > 1: thread-block clusters of that many CTAs along x (the
+// GEMM's CTA pairs).
 template <typename P>
-ft_status launch_overlapped(void (*kernel)(P), dim3 grid, dim3 block, size_t smem, cudaStream_t st, const P& p) {
+ft_status launch_overlapped(void (*kernel)(P), dim3 grid, dim3 block, size_t smem, cudaStream_t st, const P& p,
+                            int cluster_x = 1) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (cluster_x > 1) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = (unsigned)cluster_x;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
+    }
+    cfg.attrs = attr;
     return cuda_ok(cudaLaunchKernelEx(&cfg, kernel, p));
 }
 inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -541,6 +557,10 @@ int qres_max_stages(uint32_t ring_bytes) {
 // cooperative.  See ft_set_cooperative_quantizer.
 std::atomic<int> g_qres_cooperative{0};
 
+// GEMM tiling: 0 = CTA pairs whenever the activation has more than 128
+// rows, 1 = one CTA per tile always.  See ft_set_gemm_mode.
+std::atomic<int> g_gemm_mode{0};
+
 // Launches k_qres with programmatic stream serialization; cooperative when
 // requested and the kernel computes the tensor amax itself.
 ft_status launch_qres(const ft::qres::Params& p, int mt, int splits, cudaStream_t st) {
@@ -696,6 +716,9 @@ ft_status run_gemm(bool bf16, const uint8_t* a_codes, const uint8_t* a_slab, con
                    const MlpOut* mlp = nullptr) {
     Params p;
     std::memset(&p, 0, sizeof(p));
+    // CTA pairs for the 4-bit GEMM unless a tile's 128 rows hold every row
+    const bool pair = !bf16 && M > ft::gemm::BM && g_gemm_mode.load(std::memory_order_relaxed) == 0;
+    const int lrows = pair ? 64 : ft::gemm::BN;  // rows of an L panel box
     if (mlp) {
         p.mlp = 1;
         p.amax_h = mlp->amax_h;
@@ -709,6 +732,18 @@ ft_status run_gemm(bool bf16, const uint8_t* a_codes, const uint8_t* a_slab, con
                          CU_TENSOR_MAP_SWIZZLE_128B));
         FT_TRY(encode_2d(&p.mapB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, b_op, Kc, Nout, Kc * 2, 64, 256,
                          CU_TENSOR_MAP_SWIZZLE_128B));
+    } else if (pair) {
+        FT_TRY(encode_2d(&p.mapA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, Kc / 2, M, Kc / 2, 128, 128,
+                         CU_TENSOR_MAP_SWIZZLE_128B));
+        // the weight's operand image as rows of 128 bytes, 288 per block
+        // (256 code rows, 32 scale rows): one CTA's 128 code rows are one
+        // box, the block's scale rows another
+        const int64_t img_rows = (Nout / 256) * (Kc / 256) * ft::gemm::IMG_BLOCK_ROWS;
+        FT_TRY(encode_2d(&p.mapB, CU_TENSOR_MAP_DATA_TYPE_UINT8, b_op, 128, img_rows, 128, 128, 128,
+                         CU_TENSOR_MAP_SWIZZLE_128B));
+        FT_TRY(encode_2d(&p.mapBs, CU_TENSOR_MAP_DATA_TYPE_UINT8, b_op, 128, img_rows, 128, 128, 32,
+                         CU_TENSOR_MAP_SWIZZLE_128B));
+        FT_TRY(encode_slabs(&p.mapSFA, a_slab, Kc / 64, cdiv(M, 128), 1));
     } else {
         FT_TRY(encode_2d(&p.mapA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, Kc / 2, M, Kc / 2, 128, 128,
                          CU_TENSOR_MAP_SWIZZLE_128B));
@@ -731,14 +766,14 @@ ft_status run_gemm(bool bf16, const uint8_t* a_codes, const uint8_t* a_slab, con
     if (r1 > 0) {
         FT_TRY(encode_2d(&p.mapP1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P, r, M, r * 2, p.f1.wbox, 128,
                          swizzle_for(p.f1.wbox)));
-        FT_TRY(encode_2d(&p.mapL1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1, r1, Nout, r1 * 2, p.f1.wbox,
-                         ft::gemm::BN, swizzle_for(p.f1.wbox)));
+        FT_TRY(encode_2d(&p.mapL1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1, r1, Nout, r1 * 2, p.f1.wbox, lrows,
+                         swizzle_for(p.f1.wbox)));
     }
     if (r2 > 0) {
         FT_TRY(encode_2d(&p.mapP2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P, r, M, r * 2, p.f2.wbox, 128,
                          swizzle_for(p.f2.wbox)));
-        FT_TRY(encode_2d(&p.mapL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2, r2, Nout, r2 * 2, p.f2.wbox,
-                         ft::gemm::BN, swizzle_for(p.f2.wbox)));
+        FT_TRY(encode_2d(&p.mapL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2, r2, Nout, r2 * 2, p.f2.wbox, lrows,
+                         swizzle_for(p.f2.wbox)));
     }
     p.out = static_cast<uint8_t*>(out);
     p.dep_done = dep.done;
@@ -750,24 +785,31 @@ ft_status run_gemm(bool bf16, const uint8_t* a_codes, const uint8_t* a_slab, con
     p.M = (int)M;
     p.Nout = (int)Nout;
     p.Kc = (int)Kc;
+    const int pr = pair ? 1 : 0;
     int stages = ft::gemm::MAX_STAGES;
-    while (stages > 1 && ft::gemm::make_layout(stages, p.f1, p.f2, p.mlp).total > 227u * 1024u) --stages;
-    if (ft::gemm::make_layout(stages, p.f1, p.f2, p.mlp).total > 227u * 1024u) return FT_ERR_SHAPE;
+    while (stages > 1 && ft::gemm::make_layout(stages, p.f1, p.f2, p.mlp, pr).total > 227u * 1024u) --stages;
+    if (ft::gemm::make_layout(stages, p.f1, p.f2, p.mlp, pr).total > 227u * 1024u) return FT_ERR_SHAPE;
     p.stages = stages;
-    const uint32_t smem = ft::gemm::make_layout(stages, p.f1, p.f2, p.mlp).total;
-    const int tiles = cdiv(M, ft::gemm::BM) * (int)(Nout / ft::gemm::BN);
-    const int grid = std::max(1, std::min(tiles, d->sms));
+    const uint32_t smem = ft::gemm::make_layout(stages, p.f1, p.f2, p.mlp, pr).total;
+    const int tiles = cdiv(M, pair ? 2 * ft::gemm::BM : ft::gemm::BM) * (int)(Nout / ft::gemm::BN);
+    // persistent: one CTA (pair: two, one per SM of a TPC) per tile, at most
+    // the device's SMs
+    const int grid = pair ? 2 * std::max(1, std::min(tiles, d->sms / 2)) : std::max(1, std::min(tiles, d->sms));
     {
         LaunchTimer _lt(bf16 ? KID_GEMM_BF16 : KID_GEMM, st);
+        const dim3 blk(ft::gemm::NUM_THREADS);
         if (bf16)
-            FT_TRY(launch_overlapped(ft::gemm::k_gemm_fp4<true>, dim3((unsigned)grid), dim3(ft::gemm::NUM_THREADS),
-                                     smem, st, p));
+            FT_TRY(launch_overlapped(ft::gemm::k_gemm_fp4<true>, dim3((unsigned)grid), blk, smem, st, p));
+        else if (pair && mlp)
+            FT_TRY(launch_overlapped(ft::gemm::k_gemm_fp4<false, true, true>, dim3((unsigned)grid), blk, smem, st, p,
+                                     2));
+        else if (pair)
+            FT_TRY(launch_overlapped(ft::gemm::k_gemm_fp4<false, false, true>, dim3((unsigned)grid), blk, smem, st,
+                                     p, 2));
         else if (mlp)
-            FT_TRY(launch_overlapped(ft::gemm::k_gemm_fp4<false, true>, dim3((unsigned)grid),
-                                     dim3(ft::gemm::NUM_THREADS), smem, st, p));
+            FT_TRY(launch_overlapped(ft::gemm::k_gemm_fp4<false, true>, dim3((unsigned)grid), blk, smem, st, p));
         else
-            FT_TRY(launch_overlapped(ft::gemm::k_gemm_fp4<false>, dim3((unsigned)grid), dim3(ft::gemm::NUM_THREADS),
-                                     smem, st, p));
+            FT_TRY(launch_overlapped(ft::gemm::k_gemm_fp4<false>, dim3((unsigned)grid), blk, smem, st, p));
         _lt.stop();
     }
     return last_launch();
@@ -997,6 +1039,12 @@ ft_status ft_workspace_qact(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_
 
 ft_status ft_set_cooperative_quantizer(int on) {
     g_qres_cooperative.store(on ? 1 : 0, std::memory_order_relaxed);
+    return FT_OK;
+}
+
+ft_status ft_set_gemm_mode(int mode) {
+    if (mode != 0 && mode != 1) return FT_ERR_INVALID_ARG;
+    g_gemm_mode.store(mode, std::memory_order_relaxed);
     return FT_OK;
 }
 

@@ -81,11 +81,23 @@ constexpr int SFB_STAGE_BYTES = 2 * KSTEPS * 512;  // two row halves x four slab
 // one block of the weight's operand image: the B tile's codes, then its
 // scale slabs (they arrive in one copy)
 constexpr int B_SLOT = B_BYTES + SFB_STAGE_BYTES;  // 36 KiB
+// CTA pairs: each CTA holds its 128-row half of the B tile's codes and the
+// scale slabs of all 256 rows (its accumulator spans every column)
+constexpr int B_HALF_BYTES = (BN / 2) * BK_BYTES;          // 16 KiB
+constexpr int B_SLOT_P = B_HALF_BYTES + SFB_STAGE_BYTES;    // 20 KiB
+// rows of one 256-row block of the weight's operand image: 256 code rows of
+// 128 bytes, then its 32 rows of scale slabs
+constexpr int IMG_BLOCK_ROWS = 288;
 constexpr uint32_t TMEM_COLS = 512;
 // TMEM columns: [0,256) accumulator; [256,384) low-rank half 0; [384,512)
 // shared in time: the scale ring while the mainloop runs, low-rank half 1
 // after it (the next tile's first scale copy waits for the epilogue).
 constexpr uint32_t ACC_COL = 0, LR0_COL = 256, R2_COL = 384, SF_SLOT_COLS = 48;
+// CTA pairs: the scale ring takes [256, 496), five slots, during the
+// mainloop (a slot's refill waits on the other SM's signals, so the ring is
+// deeper); both low-rank halves are computed after it, into [256, 512).
+constexpr int SF_SLOTS = 2, SF_SLOTS_P = 5;
+constexpr uint32_t RING_COL_P = LR0_COL;
 
 // One low-rank factor's panels: P columns [pcol, pcol + rf) for the tile's
 // 128 rows (A operand) and L [256 output rows, rf] (B operand), both K-major.
@@ -104,6 +116,10 @@ struct Params {
     // as 3-D tensors {256 B, 2 * Kc / 64, tiles}: one stage's four slabs are
     // one box (8 x 256 B) of one tile (A) or of two (B)
     CUtensorMap mapSFA;
+    // CTA pairs: mapB covers one CTA's 128 code rows of an image block,
+    // mapBs the block's 32 rows of scale slabs; mapL1 / mapL2 boxes are 64
+    // rows (one CTA's share of a 128-column half)
+    CUtensorMap mapBs;
     const float* ga;
     const float* gb;
     uint8_t* out;        // output [M, Nout], bf16 or FP32, rows contiguous
@@ -132,7 +148,8 @@ struct Layout {
 };
 constexpr uint32_t STG_BYTES = 128 * 32;  // one staged output chunk: 128 rows x 32 bytes
 
-// bytes of a factor's P panel (128 rows) and L panel (256 rows)
+// bytes of a factor's P panel (128 rows) and L panel (256 rows; a CTA of a
+// pair holds 128 of them)
 __host__ __device__ inline uint32_t p_bytes(const LrFactor& f) {
     return f.rf > 0 ? (uint32_t)f.natoms * 128u * f.row_bytes : 0u;
 }
@@ -140,15 +157,17 @@ __host__ __device__ inline uint32_t l_bytes(const LrFactor& f) {
     return f.rf > 0 ? (uint32_t)f.natoms * 256u * f.row_bytes : 0u;
 }
 
-__host__ __device__ inline Layout make_layout(int stages, const LrFactor& f1, const LrFactor& f2, int mlp) {
+__host__ __device__ inline Layout make_layout(int stages, const LrFactor& f1, const LrFactor& f2, int mlp,
+                                              int pair = 0) {
     Layout L;
     uint32_t o = 0;
+    const uint32_t lsh = pair ? 1u : 0u;
     L.a = o;    o += stages * A_BYTES;
-    L.b = o;    o += stages * B_SLOT;
+    L.b = o;    o += stages * (pair ? B_SLOT_P : B_SLOT);
     L.p1 = o;   o += p_bytes(f1);
-    L.l1 = o;   o += l_bytes(f1);
+    L.l1 = o;   o += l_bytes(f1) >> lsh;
     L.p2 = o;   o += p_bytes(f2);
-    L.l2 = o;   o += l_bytes(f2);
+    L.l2 = o;   o += l_bytes(f2) >> lsh;
     L.sfa = o;  o += stages * SFA_STAGE_BYTES;
     L.stg = o;  o += mlp ? 0u : 2 * STG_BYTES;  // output staging, one buffer per column group (H: none)
     L.tab = o;  o += mlp ? (uint32_t)sizeof(QTableM) + 2u * kGeluTab : 0u;  // Q(H)'s encode table, GELU's
@@ -163,34 +182,43 @@ enum {
     B_FULL = 0,                        // [MAX_STAGES] TMA landed
     B_EMPTY = B_FULL + MAX_STAGES,     // [MAX_STAGES] stage consumed by the MMAs
     B_SFFULL = B_EMPTY + MAX_STAGES,   // [MAX_STAGES] the stage's scale slabs landed
-    B_SF_READY = B_SFFULL + MAX_STAGES, // [2] scale slot copied into TMEM
-    B_SF_FREE = B_SF_READY + 2,        // [2] scale slot read by its MMAs
-    B_ACC_FULL = B_SF_FREE + 2,
+    B_SF_READY = B_SFFULL + MAX_STAGES, // [SF_SLOTS_P] scale slot copied into TMEM
+    B_SF_FREE = B_SF_READY + SF_SLOTS_P, // [SF_SLOTS_P] scale slot read by its MMAs
+    B_ACC_FULL = B_SF_FREE + SF_SLOTS_P,
     B_ACC_EMPTY,                       // every epilogue warp done with the tile
     B_LR_FULL,                         // panels landed
     B_LR_SMEM_EMPTY,                   // panels consumed
     B_LR0_READY,                       // low-rank half 0 computed
     B_LR1_READY,                       // low-rank half 1 computed
     B_DRAIN,
+    B_EPI_DONE,                        // this CTA's epilogue done with the tile (CTA pairs)
     B_COUNT
 };
 static_assert(B_COUNT * 8 + 8 <= 256, "barrier area");
 
-// The K = 16 MMAs of one factor's up-projection for output rows
+// The K = 16 MMAs of one factor's up-projection for output columns
 // [128 h, 128 h + 128) of the tile: D (+)= P_f x L_f[half h]^T.
 // Descriptor words are built once per call (lo = start >> 4 | 1 << 16,
 // hi = SBO >> 4 | version 1 << 14 | swizzle << 29); a K step adds 32 bytes
 // inside an atom, the second 64-wide atom (rf > 64) starts a panel later.
+// kPair: the pair's MMA (M = 256); each CTA's L panel holds its 64 rows of
+// each half, so halves are 64 rows apart and atoms 128.
+template <bool kPair>
 __device__ __forceinline__ void lr_mma(uint32_t tmem_d, uint32_t pa, uint32_t pb, const LrFactor& f, int h,
                                        uint32_t idesc, int& q) {
+    constexpr uint32_t HALF = kPair ? 64u : 128u;
     const uint32_t hi = ((8u * f.row_bytes) >> 4) | (1u << 14) | (f.swz << 29);
     const uint32_t a_lo = (pa >> 4) | (1u << 16);
-    const uint32_t b_lo = ((pb + (uint32_t)h * 128u * f.row_bytes) >> 4) | (1u << 16);
-    const uint32_t a_atom = (128u * f.row_bytes) >> 4, b_atom = (256u * f.row_bytes) >> 4;
+    const uint32_t b_lo = ((pb + (uint32_t)h * HALF * f.row_bytes) >> 4) | (1u << 16);
+    const uint32_t a_atom = (128u * f.row_bytes) >> 4, b_atom = (2u * HALF * f.row_bytes) >> 4;
     for (int j = 0; j < f.rf; j += 16, ++q) {
         const uint32_t a = (uint32_t)(j >> 6), k = ((uint32_t)(j & (f.wbox - 1)) * 2u) >> 4;
-        umma_bf16(tmem_d, make_desc(a_lo + a * a_atom + k, hi), make_desc(b_lo + a * b_atom + k, hi), idesc,
-                  q != 0);
+        if (kPair)
+            umma_bf16_pair(tmem_d, make_desc(a_lo + a * a_atom + k, hi), make_desc(b_lo + a * b_atom + k, hi), idesc,
+                           q != 0);
+        else
+            umma_bf16(tmem_d, make_desc(a_lo + a * a_atom + k, hi), make_desc(b_lo + a * b_atom + k, hi), idesc,
+                      q != 0);
     }
 }
 
@@ -203,13 +231,19 @@ __device__ __forceinline__ void lr_mma(uint32_t tmem_d, uint32_t pa, uint32_t pb
 // K in the same 128-byte rows, four K = 16 MMAs.  No scale factors: the
 // scale warps idle.  Tiles, epilogue and low-rank terms are shared.
 // kMlp: the MLP-fusion epilogue (Params::mlp), for the 4-bit GEMM.
-template <bool kBf16, bool kMlp = false>
+// kPair: the 4-bit GEMM on CTA pairs (clusters of two): 256 x 256 tiles,
+// CTA r of a pair owns output rows 128 r .. 128 r + 127 of the tile and
+// loads its own A rows, its half of the B codes and all of the tile's
+// scales; the leader's MMAs (M = 256) read both CTAs' operands, so each SM
+// waits for 38 KB per stage instead of 54 KB for the same work.
+template <bool kBf16, bool kMlp = false, bool kPair = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_constant__ Params p) {
+    static_assert(!(kBf16 && kPair), "CTA pairs are for the 4-bit GEMM");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (base - raw_base);
-    const Layout L = make_layout(p.stages, p.f1, p.f2, kMlp ? 1 : 0);
+    const Layout L = make_layout(p.stages, p.f1, p.f2, kMlp ? 1 : 0, kPair ? 1 : 0);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.bars + B_COUNT * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.bars + B_COUNT * 8 + 4);
@@ -217,7 +251,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
     const int warp = warp_id(), lane = lane_id();
     const int S = p.stages;
     const bool has_lr = p.f1.rf + p.f2.rf > 0;
-    const int tiles_m = (p.M + BM - 1) / BM;
+    // output rows per tile: the CTA's 128, or the pair's 256 (this CTA's
+    // rows start at 128 rank); both CTAs of a pair walk the same tiles
+    constexpr int TM = kPair ? 2 * BM : BM;
+    const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+    const int unit = kPair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int nunits = kPair ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+    const int tiles_m = (p.M + TM - 1) / TM;
     const int tiles_n = p.Nout / BN;
     const int num_tiles = tiles_m * tiles_n;
     const int KT = kBf16 ? p.Kc / 64 : p.Kc / 256;  // stages per tile
@@ -228,12 +268,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             mbar_init(&bars[B_SFFULL + i], 1);
             mbar_init(&bars[B_EMPTY + i], 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&bars[B_SF_READY + i], NUM_SF_WARPS);
+        // a pair's leader counts both CTAs' scale and epilogue warps
+        for (int i = 0; i < SF_SLOTS_P; ++i) {
+            mbar_init(&bars[B_SF_READY + i], (kPair ? 2 : 1) * NUM_SF_WARPS);
             mbar_init(&bars[B_SF_FREE + i], 1);
         }
         mbar_init(&bars[B_ACC_FULL], 1);
-        mbar_init(&bars[B_ACC_EMPTY], NUM_EPI_WARPS);
+        mbar_init(&bars[B_ACC_EMPTY], (kPair ? 2 : 1) * NUM_EPI_WARPS);
+        mbar_init(&bars[B_EPI_DONE], NUM_EPI_WARPS);
         mbar_init(&bars[B_LR_FULL], 1);
         mbar_init(&bars[B_LR_SMEM_EMPTY], 1);
         mbar_init(&bars[B_LR0_READY], 1);
@@ -247,12 +289,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
         tma_prefetch_desc(&p.mapB);
         if (!kBf16) tma_prefetch_desc(&p.mapSFA);
     }
+    // both CTAs' barriers exist before either signals the other's
+    if constexpr (kPair) cluster_sync();
     if (warp == 1) {
-        tmem_alloc(tmem_slot, TMEM_COLS);
-        tmem_relinquish();
+        if (kPair) {
+            tmem_alloc_pair(tmem_slot, TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_slot, TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if constexpr (kPair) cluster_sync();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     // the inputs written by the previous kernel are complete from here on;
@@ -261,7 +311,77 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
-        if (lane == 0) {
+        if (kPair && lane == 0) {
+            // Per stage: this CTA's A rows and B code half, with their bytes
+            // counted on the leader's FULL barrier (the leader expects both
+            // CTAs' bytes); the tile's weight scale slabs (all 256 rows) and
+            // this CTA's activation slabs on its own SFFULL barrier, for its
+            // scale warps.  Panels likewise: this CTA's 128 rows of P and its
+            // 64 rows of each half of L, counted on the leader's LR_FULL.
+            const uint32_t lead_full = mapa_shared(smem_u32(&bars[B_FULL]), 0);
+            const uint32_t lead_lr = mapa_shared(smem_u32(&bars[B_LR_FULL]), 0);
+            const uint32_t lr_share = p_bytes(p.f1) + (l_bytes(p.f1) >> 1) + p_bytes(p.f2) + (l_bytes(p.f2) >> 1);
+            uint32_t it = 0;
+            bool ok = true;
+            int local = 0;
+            const int kt_panel = min(S, KT - 1);
+            for (int tile = unit; tile < num_tiles && ok; tile += nunits, ++local) {
+                const int tm = tile / tiles_n, tn = tile % tiles_n;
+                const int m0 = tm * TM + BM * (int)rank, n0 = tn * BN;
+                for (int kt = 0; kt < KT; ++kt, ++it) {
+                    if (has_lr && kt == kt_panel) {
+                        if (!mbar_wait_cluster(&bars[B_LR_SMEM_EMPTY], (local & 1) ^ 1, ERR_WAIT_LR, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        if (rank == 0) mbar_arrive_expect_tx(&bars[B_LR_FULL], 2u * lr_share);
+                        const LrFactor* fs[2] = {&p.f1, &p.f2};
+                        const CUtensorMap* pm[2] = {&p.mapP1, &p.mapP2};
+                        const CUtensorMap* lm[2] = {&p.mapL1, &p.mapL2};
+                        const uint32_t po[2] = {L.p1, L.p2}, lo[2] = {L.l1, L.l2};
+                        for (int f = 0; f < 2; ++f) {
+                            const LrFactor& F = *fs[f];
+                            for (int a = 0; a < (F.rf > 0 ? F.natoms : 0); ++a) {
+                                tma_load_2d_pair(smem + po[f] + a * 128 * F.row_bytes, pm[f], lead_lr,
+                                                 F.pcol + 64 * a, m0);
+                                for (int h = 0; h < 2; ++h)
+                                    tma_load_2d_pair(smem + lo[f] + (a * 128 + h * 64) * F.row_bytes, lm[f], lead_lr,
+                                                     64 * a, n0 + 128 * h + 64 * (int)rank);
+                            }
+                        }
+                    }
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1;
+                    if (!mbar_wait_cluster(&bars[B_EMPTY + s], ph ^ 1, ERR_WAIT_EMPTY, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const int blk_row = IMG_BLOCK_ROWS * (tn * KT + kt);
+                    uint64_t* sfb_bar = &bars[B_SFFULL + s];
+                    mbar_arrive_expect_tx(sfb_bar, SFB_STAGE_BYTES + SFA_STAGE_BYTES);
+                    tma_load_2d(smem + L.b + s * B_SLOT_P + B_HALF_BYTES, &p.mapBs, sfb_bar, 0, blk_row + BN);
+                    tma_load_3d(smem + L.sfa + s * SFA_STAGE_BYTES, &p.mapSFA, sfb_bar, 0, 8 * kt, 2 * tm + (int)rank);
+                    if (rank == 0) mbar_arrive_expect_tx(&bars[B_FULL + s], 2u * (A_BYTES + B_HALF_BYTES));
+                    tma_load_2d_pair(smem + L.b + s * B_SLOT_P, &p.mapB, lead_full + 8u * s, 0,
+                                     blk_row + (BN / 2) * (int)rank);
+                    tma_load_2d_pair(smem + L.a + s * A_BYTES, &p.mapA, lead_full + 8u * s, kt * BK_BYTES, m0);
+                }
+            }
+            if (!ok) {
+                // this CTA's scale copies land on its own barriers; its code
+                // and panel copies count on the leader's, so give those time
+                // to land before the CTA can exit (both CTAs pass a cluster
+                // barrier at the end)
+                for (int d = 0; d < S && d < (int)it; ++d) {
+                    uint32_t j = it - 1 - d;
+                    volatile int no_abort = 0;
+                    mbar_wait(&bars[B_SFFULL + (j % S)], (j / S) & 1, ERR_WAIT_DRAIN, &no_abort);
+                }
+                const uint64_t t0 = globaltimer_ns();
+                while (globaltimer_ns() - t0 < 200000ull) {
+                }
+            }
+        } else if (!kPair && lane == 0) {
             const uint32_t stage_bytes = A_BYTES;
             const uint32_t lr_total = p_bytes(p.f1) + l_bytes(p.f1) + p_bytes(p.f2) + l_bytes(p.f2);
             uint32_t it = 0;
@@ -274,7 +394,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             // wait holds back the stages
             const int kt_panel = min(S, KT - 1);
             int panels_issued = 0;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+            for (int tile = unit; tile < num_tiles && ok; tile += nunits, ++local) {
                 const int tm = tile / tiles_n, tn = tile % tiles_n;
                 const int m0 = tm * BM, n0 = tn * BN;
                 for (int kt = 0; kt < KT; ++kt, ++it) {
@@ -339,7 +459,79 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
         }
     } else if (warp == 1) {
         // ------------------------------------------------ UMMA issuer
-        if (lane == 0) {
+        if (kPair && lane == 0 && rank == 0) {
+            // the pair's leader: M = 256 MMAs over both CTAs' operands into
+            // both CTAs' tensor memory; every completion is committed to
+            // the barrier of each CTA that waits for it
+            const uint32_t idesc = idesc_nvfp4(2 * BM, BN);
+            const uint32_t idesc_lr = idesc_bf16(2 * BM, 128, 0, 0);
+            const uint32_t hi_sw128 = (1024u >> 4) | (1u << 14) | (SWZ_128B << 29);
+            const uint32_t a_lo0 = ((base + L.a) >> 4) | (1u << 16);
+            const uint32_t b_lo0 = ((base + L.b) >> 4) | (1u << 16);
+            const uint32_t own0 = smem_u32(&bars[0]);
+            const uint32_t peer0 = mapa_shared(own0, 1);
+            auto commit_both = [&](int b) {
+                tc_commit_pair(own0 + 8u * (uint32_t)b);
+                tc_commit_pair(peer0 + 8u * (uint32_t)b);
+            };
+            uint32_t it = 0;
+            bool ok = true;
+            int local = 0;
+            for (int tile = unit; tile < num_tiles && ok; tile += nunits, ++local) {
+                // both CTAs' epilogues have read the previous tile
+                if (!mbar_wait_cluster(&bars[B_ACC_EMPTY], (local & 1) ^ 1, ERR_WAIT_ACC_EMPTY, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (int kt = 0; kt < KT; ++kt, ++it) {
+                    const int s = it % S;
+                    const int sb = it % SF_SLOTS_P;
+                    if (!mbar_wait_cluster(&bars[B_FULL + s], (it / S) & 1, ERR_WAIT_FULL, abort_flag) ||
+                        !mbar_wait_cluster(&bars[B_SF_READY + sb], (it / SF_SLOTS_P) & 1, ERR_WAIT_SF, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_lo = a_lo0 + s * (A_BYTES >> 4);
+                    const uint32_t b_lo = b_lo0 + s * (B_SLOT_P >> 4);
+                    const uint32_t sf = tmem + RING_COL_P + sb * SF_SLOT_COLS;
+#pragma unroll
+                    for (int j = 0; j < KSTEPS; ++j)
+                        umma_nvfp4_pair(tmem + ACC_COL, make_desc(a_lo + 2 * j, hi_sw128),
+                                        make_desc(b_lo + 2 * j, hi_sw128), idesc, sf + 4 * j, sf + 16 + 8 * j,
+                                        (kt | j) != 0);
+                    commit_both(B_EMPTY + s);
+                    commit_both(B_SF_FREE + sb);
+                }
+                if (!ok) break;
+                commit_both(B_ACC_FULL);
+                if (has_lr) {
+                    // both halves go into the ring's columns, once the
+                    // mainloop's MMAs (their last readers) are done
+                    if (!mbar_wait_cluster(&bars[B_LR_FULL], local & 1, ERR_WAIT_LR, abort_flag) ||
+                        !mbar_wait_cluster(&bars[B_ACC_FULL], local & 1, ERR_WAIT_ACC_FULL, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    int q = 0;
+                    if (p.f1.rf > 0) lr_mma<true>(tmem + LR0_COL, base + L.p1, base + L.l1, p.f1, 0, idesc_lr, q);
+                    if (p.f2.rf > 0) lr_mma<true>(tmem + LR0_COL, base + L.p2, base + L.l2, p.f2, 0, idesc_lr, q);
+                    commit_both(B_LR0_READY);
+                    q = 0;
+                    if (p.f1.rf > 0) lr_mma<true>(tmem + R2_COL, base + L.p1, base + L.l1, p.f1, 1, idesc_lr, q);
+                    if (p.f2.rf > 0) lr_mma<true>(tmem + R2_COL, base + L.p2, base + L.l2, p.f2, 1, idesc_lr, q);
+                    commit_both(B_LR1_READY);
+                    commit_both(B_LR_SMEM_EMPTY);
+                }
+            }
+            // every tcgen05 op issued by this thread completes before TMEM is
+            // freed and before either CTA can exit
+            tc_commit_pair(own0 + 8u * B_DRAIN);
+            volatile int no_abort = 0;
+            mbar_wait(&bars[B_DRAIN], 0, ERR_WAIT_DRAIN, &no_abort);
+        } else if (!kPair && lane == 0) {
             const uint32_t idesc = kBf16 ? idesc_bf16(BM, BN, 0, 0) : idesc_nvfp4(BM, BN);
             const uint32_t idesc_lr = idesc_bf16(BM, 128, 0, 0);
             // descriptor words: lo = start >> 4 | (LBO >> 4) << 16;
@@ -350,7 +542,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             uint32_t it = 0;
             bool ok = true;
             int local = 0;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+            for (int tile = unit; tile < num_tiles && ok; tile += nunits, ++local) {
                 // the epilogue has read the previous tile's accumulator and
                 // both low-rank halves
                 if (!mbar_wait(&bars[B_ACC_EMPTY], (local & 1) ^ 1, ERR_WAIT_ACC_EMPTY, abort_flag)) {
@@ -399,8 +591,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     }
                     tc_fence_after();
                     int q = 0;
-                    if (p.f1.rf > 0) lr_mma(tmem + LR0_COL, base + L.p1, base + L.l1, p.f1, 0, idesc_lr, q);
-                    if (p.f2.rf > 0) lr_mma(tmem + LR0_COL, base + L.p2, base + L.l2, p.f2, 0, idesc_lr, q);
+                    if (p.f1.rf > 0) lr_mma<false>(tmem + LR0_COL, base + L.p1, base + L.l1, p.f1, 0, idesc_lr, q);
+                    if (p.f2.rf > 0) lr_mma<false>(tmem + LR0_COL, base + L.p2, base + L.l2, p.f2, 0, idesc_lr, q);
                     tc_commit(&bars[B_LR0_READY]);
                 }
                 tc_commit(&bars[B_ACC_FULL]);
@@ -411,8 +603,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     }
                     tc_fence_after();
                     int q = 0;
-                    if (p.f1.rf > 0) lr_mma(tmem + R2_COL, base + L.p1, base + L.l1, p.f1, 1, idesc_lr, q);
-                    if (p.f2.rf > 0) lr_mma(tmem + R2_COL, base + L.p2, base + L.l2, p.f2, 1, idesc_lr, q);
+                    if (p.f1.rf > 0) lr_mma<false>(tmem + R2_COL, base + L.p1, base + L.l1, p.f1, 1, idesc_lr, q);
+                    if (p.f2.rf > 0) lr_mma<false>(tmem + R2_COL, base + L.p2, base + L.l2, p.f2, 1, idesc_lr, q);
                     tc_commit(&bars[B_LR1_READY]);
                     tc_commit(&bars[B_LR_SMEM_EMPTY]);
                 }
@@ -435,25 +627,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             uint32_t it = 0;
             bool ok = true;
             int local = 0;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+            for (int tile = unit; tile < num_tiles && ok; tile += nunits, ++local) {
                 // the ring's columns hold the previous tile's low-rank half 1
-                // until its epilogue is done
+                // until its epilogue (this CTA's) is done
                 if (has_lr && local > 0 &&
-                    !mbar_wait(&bars[B_ACC_EMPTY], (local - 1) & 1, ERR_WAIT_SF, abort_flag)) {
+                    !mbar_wait(&bars[kPair ? B_EPI_DONE : B_ACC_EMPTY], (local - 1) & 1, ERR_WAIT_SF, abort_flag)) {
                     ok = false;
                     break;
                 }
                 for (int kt = 0; kt < KT; ++kt, ++it) {
                     const int s = it % S;
-                    const int sb = it & 1;
+                    constexpr int NSL = kPair ? SF_SLOTS_P : SF_SLOTS;
+                    const int sb = it % NSL;
+                    const uint32_t fph = ((it / NSL) & 1) ^ 1;
                     if (!mbar_wait(&bars[B_SFFULL + s], (it / S) & 1, ERR_WAIT_FULL, abort_flag) ||
-                        !mbar_wait(&bars[B_SF_FREE + sb], ((it >> 1) & 1) ^ 1, ERR_WAIT_SF, abort_flag)) {
+                        !(kPair ? mbar_wait_cluster(&bars[B_SF_FREE + sb], fph, ERR_WAIT_SF, abort_flag)
+                                : mbar_wait(&bars[B_SF_FREE + sb], fph, ERR_WAIT_SF, abort_flag))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t sfa = base + L.sfa + (uint32_t)s * SFA_STAGE_BYTES + 16u * (uint32_t)lane;
-                    const uint32_t sfb = base + L.b + (uint32_t)s * B_SLOT + B_BYTES + 16u * (uint32_t)lane;
+                    const uint32_t sfb = kPair ? base + L.b + (uint32_t)s * B_SLOT_P + B_HALF_BYTES + 16u * (uint32_t)lane
+                                               : base + L.b + (uint32_t)s * B_SLOT + B_BYTES + 16u * (uint32_t)lane;
                     uint32_t ra[16], rb[32];
     #pragma unroll
                     for (int j = 0; j < KSTEPS; ++j) {
@@ -464,7 +660,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                         rb[8 * j] = vl.x; rb[8 * j + 1] = vl.y; rb[8 * j + 2] = vl.z; rb[8 * j + 3] = vl.w;
                         rb[8 * j + 4] = vh.x; rb[8 * j + 5] = vh.y; rb[8 * j + 6] = vh.z; rb[8 * j + 7] = vh.w;
                     }
-                    const uint32_t sf = tmem + lane_addr + R2_COL + (uint32_t)sb * SF_SLOT_COLS;
+                    const uint32_t sf = tmem + lane_addr + (kPair ? RING_COL_P : R2_COL) + (uint32_t)sb * SF_SLOT_COLS;
                     tmem_st_32x32b_x16(sf, ra);
                     tmem_st_32x32b_x32(sf + 16, rb);
                     tmem_st_wait();
@@ -473,7 +669,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     fence_proxy_async_smem();
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars[B_SF_READY + sb]);
+                    if (lane == 0) {
+                        if (kPair) mbar_arrive_cluster(mapa_shared(smem_u32(&bars[B_SF_READY + sb]), 0));
+                        else mbar_arrive(&bars[B_SF_READY + sb]);
+                    }
                 }
             }
         }
@@ -498,6 +697,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
         const uint32_t buf = base + L.stg + (uint32_t)grp * STG_BYTES;
         const uint32_t lr_col = grp == 0 ? LR0_COL : R2_COL;
         uint64_t* lr_ready = &bars[grp == 0 ? B_LR0_READY : B_LR1_READY];
+        // this warp is done reading the tile's tensor memory: the MMA warp
+        // (the pair's leader) may overwrite it, this CTA's scale warps may
+        // reuse the ring columns
+        auto release_acc = [&]() {
+            if (kPair) {
+                mbar_arrive(&bars[B_EPI_DONE]);
+                mbar_arrive_cluster(mapa_shared(smem_u32(&bars[B_ACC_EMPTY]), 0));
+            } else {
+                mbar_arrive(&bars[B_ACC_EMPTY]);
+            }
+        };
         bool ok = true;
         int local = 0;
         const int64_t ldo = (int64_t)p.Nout * (p.out_f32 ? 4 : 2);  // output row bytes
@@ -523,11 +733,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             gelu_table_build(gtab, et2, 32 * NUM_EPI_WARPS);
             named_bar_sync(3, 32 * NUM_EPI_WARPS);
         }
-        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
-            const int m0 = (tile / tiles_n) * BM;
+        for (int tile = unit; tile < num_tiles && ok; tile += nunits, ++local) {
+            const int m0 = (tile / tiles_n) * TM + BM * (int)rank;
             const int n0 = (tile % tiles_n) * BN;
-            if (!mbar_wait(&bars[B_ACC_FULL], local & 1, ERR_WAIT_ACC_FULL, abort_flag) ||
-                (has_lr && !mbar_wait(lr_ready, local & 1, ERR_WAIT_LR, abort_flag))) {
+            if (kPair ? (!mbar_wait_cluster(&bars[B_ACC_FULL], local & 1, ERR_WAIT_ACC_FULL, abort_flag) ||
+                         (has_lr && !mbar_wait_cluster(lr_ready, local & 1, ERR_WAIT_LR, abort_flag)))
+                      : (!mbar_wait(&bars[B_ACC_FULL], local & 1, ERR_WAIT_ACC_FULL, abort_flag) ||
+                         (has_lr && !mbar_wait(lr_ready, local & 1, ERR_WAIT_LR, abort_flag)))) {
                 ok = false;
                 break;
             }
@@ -577,7 +789,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                 // overwrite the accumulator and both low-rank halves
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars[B_ACC_EMPTY]);
+                if (lane == 0) release_acc();
                 if (kMlp) {
                     // MLP fusion: H = GELU(y) per bf16 value.  A 16-column
                     // chunk of the row is one 1x16 block of Q(H), and its 32
@@ -607,9 +819,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     if (in)
                         *reinterpret_cast<uint2*>(p.q_scales + (int64_t)row * (p.Nout / 16) + qcol / 16) =
                             make_uint2(sw0, sw1);
-                    // slab rows past M hold the (zero) scales of the zero-filled rows
-                    *reinterpret_cast<uint32_t*>(p.q_slab + slab_offset(row, qcol / 16, p.Nout)) = sw0;
-                    *reinterpret_cast<uint32_t*>(p.q_slab + slab_offset(row, qcol / 16 + 4, p.Nout)) = sw1;
+                    // slab rows past M hold the (zero) scales of the zero-filled
+                    // rows, up to the slabs' 128-row padding (a pair's second
+                    // CTA may lie wholly past it)
+                    if (row < ((p.M + BM - 1) / BM) * BM) {
+                        *reinterpret_cast<uint32_t*>(p.q_slab + slab_offset(row, qcol / 16, p.Nout)) = sw0;
+                        *reinterpret_cast<uint32_t*>(p.q_slab + slab_offset(row, qcol / 16 + 4, p.Nout)) = sw1;
+                    }
                 } else {
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
@@ -648,16 +864,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars[B_ACC_EMPTY]);
+                if (lane == 0) release_acc();
             }
         }
     }
 
     tc_fence_before();
     __syncthreads();
+    // neither CTA of a pair leaves while the other may still read its shared
+    // memory or signal its barriers
+    if constexpr (kPair) cluster_sync();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, TMEM_COLS);
+        if (kPair) tmem_dealloc_pair(tmem, TMEM_COLS);
+        else tmem_dealloc(tmem, TMEM_COLS);
     }
     finish_after_predecessor(p.dep_done);
 }

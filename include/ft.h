@@ -335,6 +335,19 @@ ft_status ft_device_error(int* code, void* stream);
  * Process-wide, for calls made after it returns.  Host-only; always FT_OK. */
 ft_status ft_set_cooperative_quantizer(int on);
 
+/* ft_set_gemm_mode -- tiling of the 4-bit GEMMs inside ft_linear_fwd,
+ * ft_linear_bwd and ft_mlp_fwd (no counterpart in the paper: a choice of
+ * how the hardware runs the same sums).
+ *   mode = 0 (the default): pairs of CTAs on the two SMs of a TPC share
+ *     each 256 x 256 output tile (a thread-block cluster of two; the MMAs
+ *     of the pair read half of the weight tile from each SM), whenever the
+ *     activation has more than 128 rows; one CTA per 128 x 256 tile
+ *     otherwise.
+ *   mode = 1: one CTA per 128 x 256 tile always.
+ * Both give the same results.  Process-wide, for calls made after it
+ * returns.  Host-only; FT_ERR_INVALID_ARG for another mode. */
+ft_status ft_set_gemm_mode(int mode);
+
 /* Human-readable name of a status. */
 const char* ft_status_str(ft_status s);
 

@@ -165,6 +165,19 @@ def test_cooperative_quantizer_switch_is_host_only(L):
         L.ft_set_cooperative_quantizer(0)
 
 
+def test_gemm_mode_switch_is_host_only(L):
+    """The GEMM tiling switch touches no device: modes 0 (CTA pairs) and 1
+    (one CTA per tile) answer FT_OK without a GPU; any other mode is
+    rejected and leaves the setting alone."""
+    try:
+        for mode in (1, 0, 1):
+            assert L.ft_set_gemm_mode(mode) == 0
+        for bad in (2, -1, 7):
+            assert L.ft_set_gemm_mode(bad) == FT_ERR_INVALID_ARG
+    finally:
+        L.ft_set_gemm_mode(0)
+
+
 def test_header_is_plain_c_and_the_library_links_from_c(L, tmp_path):
     """include/ft.h compiles as strict C11 (no C++ or CUDA headers) and a C
     program links libft_b200.so and runs its host-only entry points."""
