@@ -647,6 +647,68 @@ def bench_mlp(torch, ft, dev, flush, reps=10):
     return out
 
 
+def bench_lora_fusion(torch, ft, dev, flush, reps=10):
+    """LoRA fusion (the FourTune page's section 3.3; its Fig. 9 credits it
+    with 1.82x): one forward of the DiT MLP-up linear (X [4608, 3072],
+    W [12288, 3072], r_s = r_l = 32, bf16 Y) as the library runs it -- P =
+    [X U | s X A] made by the quantizer's pass over X, P [V | B]^T added in
+    the GEMM's epilogue, Y written once -- against the same layer unfused:
+    the 4-bit GEMM alone (rank 0, FP32 Y), then the low-rank branch as
+    separate bf16 matmuls (torch), the add and the cast to bf16.  CUDA events
+    around each forward, L2 flushed before each."""
+    import ft_synth
+    sh = stack_shapes()[2]
+
+    def to_dev(u16):
+        return torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    inp = ft_synth.make_inputs(sh, seed=SEED + 2)
+    U, V, Wr = ft.svd_split(to_dev(inp["W"]), sh.r_s)
+    A, B, s = to_dev(inp["A"]), to_dev(inp["B"]), float(inp["s"])
+    fused = ft.prepare_layer(W_res=Wr, U=U, V=V, A=A, B=B, s=s)
+    bare = ft.prepare_layer(W_res=Wr)
+    X = to_dev(inp["X"])
+    M, N = X.shape[0], Wr.shape[0]
+    r = U.shape[1] + A.shape[1]
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    P = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
+    Y32 = torch.empty(M, N, dtype=torch.float32, device=dev)
+    UA = torch.cat([U, A * s], dim=1).contiguous()   # [K, r], s folded into A
+    LR = torch.cat([V, B], dim=1).contiguous()       # [N, r]
+    ws_f, ws_b = ft.Workspace(), ft.Workspace()
+
+    def run_fused():
+        ft.ft_linear_fwd(fused, X, Y=Y, P=P, ws=ws_f)
+
+    def run_unfused():
+        ft.ft_linear_fwd(bare, X, out_dtype=ft.F32, Y=Y32, ws=ws_b)
+        Pu = X @ UA
+        Y32.add_(Pu @ LR.T)
+        Y.copy_(Y32)
+
+    stream = torch.cuda.current_stream()
+    out = {}
+    for name, fn in (("fused", run_fused), ("unfused", run_unfused)):
+        fn()
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(reps):
+            flush()
+            keep_host_ahead(torch, 1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        out[name + "_ms"] = statistics.median(ms)
+    assert ft.ft_device_error() == 0, "device error in the LoRA-fusion section"
+    out["speedup"] = out["unfused_ms"] / out["fused_ms"]
+    out["workload"] = ("X [4608,3072], W [12288,3072], r_s = r_l = 32, bf16 Y; unfused = rank-0 4-bit GEMM (FP32 Y) "
+                       "+ torch bf16 matmuls X [U | sA], P [V | B]^T + add + cast")
+    return out
+
+
 def dataclasses_replace(obj, **kw):
     import dataclasses
     return dataclasses.replace(obj, **kw)
@@ -803,6 +865,7 @@ def run_ours(args):
         out["attn_proj"] = run_attn_secondary(torch, ft, dev, flush, args.steps, args.warmup, fp4_peak, hbm_gbs)
         out["quantize"] = bench_quantizers(torch, ft, dev, hbm_gbs, flush)
         out["mlp_fusion"] = bench_mlp(torch, ft, dev, flush)
+        out["lora_fusion"] = bench_lora_fusion(torch, ft, dev, flush)
 
     # ---------------- end to end through the API with host buffers: every
     # linear's X and dY copied in from pinned host memory, the step, and the

@@ -280,9 +280,11 @@ def ft_pack_weight_operands(w_k, w_n, N: int, K: int, stream=None):
 
 def ft_linear_fwd(layer: Layer, X: torch.Tensor, amax_x: torch.Tensor | None = None,
                   out_dtype: int = BF16, Y: torch.Tensor | None = None, P: torch.Tensor | None = None,
-                  ws: Workspace | None = None, stream=None):
+                  ws: Workspace | None = None, stream=None, amax_y: torch.Tensor | None = None):
     """Y = Q(X) Q(W_res)^T + (X U) V^T + s (X A) B^T.  Returns (Y, P) where
-    P = [bf16(X U) | bf16(s X A)] is saved for the backward."""
+    P = [bf16(X U) | bf16(s X A)] is saved for the backward.  amax_y: an
+    optional float32 device scalar (>= 0) raised to max|Y| by the GEMM's
+    epilogue."""
     _bf16(X, "X")
     M = X.shape[0]
     r = layer.r_s + layer.r_l
@@ -295,7 +297,7 @@ def ft_linear_fwd(layer: Layer, X: torch.Tensor, amax_x: torch.Tensor | None = N
     v = layer.view()
     check("ft_linear_fwd", load().ft_linear_fwd(
         ctypes.byref(v), X.data_ptr(), M, _ptr(amax_x), Y.data_ptr(), out_dtype,
-        P.data_ptr() if r > 0 else None, wbuf.data_ptr(), wbuf.numel(), _stream(stream)))
+        P.data_ptr() if r > 0 else None, _ptr(amax_y), wbuf.data_ptr(), wbuf.numel(), _stream(stream)))
     return Y, P
 
 
@@ -330,10 +332,12 @@ def ft_mlp_workspace_bytes(up: Layer, down: Layer, M: int) -> int:
 def ft_mlp_fwd(up: Layer, down: Layer, X: torch.Tensor, amax_h: torch.Tensor, amax_x: torch.Tensor | None = None,
                out_dtype: int = BF16, H: torch.Tensor | None = None, Y: torch.Tensor | None = None,
                P_up: torch.Tensor | None = None, P_down: torch.Tensor | None = None,
-               ws: Workspace | None = None, stream=None):
+               ws: Workspace | None = None, stream=None, amax_h_out: torch.Tensor | None = None):
     """The MLP forward with FC1's GEMM fused with FC2's quantization: H =
     GELU(bf16(FC1(X))) and Y = FC2(H), Q(H) made by FC1's epilogue with the
-    tensor scale of the supplied amax_h.  Returns (Y, H, P_up, P_down)."""
+    tensor scale of the supplied amax_h.  amax_h_out: an optional float32
+    device scalar (>= 0) raised to max|H| (the next step's amax_h).
+    Returns (Y, H, P_up, P_down)."""
     _bf16(X, "X")
     M = X.shape[0]
     dev = X.device
@@ -348,7 +352,7 @@ def ft_mlp_fwd(up: Layer, down: Layer, X: torch.Tensor, amax_h: torch.Tensor, am
     check("ft_mlp_fwd", load().ft_mlp_fwd(
         ctypes.byref(vu), ctypes.byref(vd), X.data_ptr(), M, _ptr(amax_x), amax_h.data_ptr(), H.data_ptr(),
         Y.data_ptr(), out_dtype, P_up.data_ptr() if ru > 0 else None, P_down.data_ptr() if rd > 0 else None,
-        wbuf.data_ptr(), wbuf.numel(), _stream(stream)))
+        _ptr(amax_h_out), wbuf.data_ptr(), wbuf.numel(), _stream(stream)))
     return Y, H, P_up, P_down
 
 

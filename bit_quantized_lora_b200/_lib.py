@@ -51,14 +51,14 @@ SIGNATURES = {
                                              ctypes.POINTER(FtFp4), ctypes.POINTER(FtFp4), c_vp,
                                              ctypes.c_size_t, c_vp]),
     "ft_linear_fwd": (ctypes.c_int, [ctypes.POINTER(FtLinear), c_vp, c_i64, c_vp, c_vp, ctypes.c_int,
-                                     c_vp, c_vp, ctypes.c_size_t, c_vp]),
+                                     c_vp, c_vp, c_vp, ctypes.c_size_t, c_vp]),
     "ft_linear_bwd": (ctypes.c_int, [ctypes.POINTER(FtLinear), c_vp, c_vp, c_vp, c_i64, c_vp, c_vp,
                                      ctypes.c_int, c_vp, c_vp, c_vp, ctypes.c_size_t, c_vp]),
     "ft_dequant_weight_operands": (ctypes.c_int, [ctypes.POINTER(FtFp4), ctypes.POINTER(FtFp4), c_vp, c_vp,
                                                   c_vp]),
     "ft_gelu_bf16": (ctypes.c_int, [c_vp, c_vp, c_i64, c_vp]),
     "ft_mlp_fwd": (ctypes.c_int, [ctypes.POINTER(FtLinear), ctypes.POINTER(FtLinear), c_vp, c_i64, c_vp, c_vp,
-                                  c_vp, c_vp, ctypes.c_int, c_vp, c_vp, c_vp, ctypes.c_size_t, c_vp]),
+                                  c_vp, c_vp, ctypes.c_int, c_vp, c_vp, c_vp, c_vp, ctypes.c_size_t, c_vp]),
     "ft_mlp_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(FtLinear), ctypes.POINTER(FtLinear), c_i64]),
     "ft_workspace_bytes": (ctypes.c_size_t, [c_i64, c_i64, c_i64, c_i64, c_i64]),
     "ft_quantize_workspace_bytes": (ctypes.c_size_t, []),

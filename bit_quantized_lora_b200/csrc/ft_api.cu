@@ -713,9 +713,10 @@ ft_status run_gemm(bool bf16, const uint8_t* a_codes, const uint8_t* a_slab, con
                    int64_t Kc, const uint8_t* b_op, const float* gb,
                    int64_t Nout, const void* P, const void* L1, int64_t r1, const void* L2, int64_t r2,
                    void* out, ft_dtype ot, const DevInfo* d, cudaStream_t st, DepFlag dep,
-                   const MlpOut* mlp = nullptr) {
+                   const MlpOut* mlp = nullptr, float* amax_out = nullptr) {
     Params p;
     std::memset(&p, 0, sizeof(p));
+    p.amax_out = reinterpret_cast<unsigned int*>(amax_out);
     // CTA pairs for the 4-bit GEMM unless a tile's 128 rows hold every row
     const bool pair = !bf16 && M > ft::gemm::BM && g_gemm_mode.load(std::memory_order_relaxed) == 0;
     const int lrows = pair ? 64 : ft::gemm::BN;  // rows of an L panel box
@@ -1141,7 +1142,7 @@ ft_status ft_quantize_transpose(const void* x, int64_t rows, int64_t cols, int64
 }
 
 ft_status ft_linear_fwd(const ft_linear* L, const void* X, int64_t M, const float* amax_x, void* Y,
-                        ft_dtype yt, void* P_save, void* ws, size_t ws_bytes, void* stream) {
+                        ft_dtype yt, void* P_save, float* amax_y, void* ws, size_t ws_bytes, void* stream) {
     FT_TRY(check_linear(L));
     if (M < 0) return FT_ERR_INVALID_ARG;
     if (yt != FT_BF16 && yt != FT_F32) return FT_ERR_INVALID_ARG;
@@ -1149,7 +1150,8 @@ ft_status ft_linear_fwd(const ft_linear* L, const void* X, int64_t M, const floa
     const int64_t r = L->r_s + L->r_l;
     if (M == 0) return FT_OK;
     if (!X || !Y || (r > 0 && !P_save)) return FT_ERR_INVALID_ARG;
-    if (!al16(X) || !al16(Y) || (P_save && !al16(P_save))) return FT_ERR_ALIGN;
+    if (!al16(X) || !al16(Y) || (P_save && !al16(P_save)) || (reinterpret_cast<uintptr_t>(amax_y) & 3u))
+        return FT_ERR_ALIGN;
     const WsPlan w = plan_ws(M, L->N, L->K, L->r_s, L->r_l);
     if (!ws || ws_bytes < w.total || !al16(ws)) return FT_ERR_WORKSPACE;
     DevInfo* d;
@@ -1165,9 +1167,9 @@ ft_status ft_linear_fwd(const ft_linear* L, const void* X, int64_t M, const floa
     if (L->precision & FT_W4A16G4)  // 16-bit activations: the GEMM reads X itself
         return run_gemm(true, static_cast<const uint8_t*>(X), nullptr, nullptr, M, L->K,
                         static_cast<const uint8_t*>(L->wd_k), L->w_k.tscale, L->N, P_save, L->V, L->r_s, L->B,
-                        L->r_l, Y, yt, d, st, dep);
+                        L->r_l, Y, yt, d, st, dep, nullptr, amax_y);
     return run_gemm(false, codes, wsb + w.sfslab, g_x, M, L->K, L->op_k, L->w_k.tscale, L->N,
-                    P_save, L->V, L->r_s, L->B, L->r_l, Y, yt, d, st, dep);
+                    P_save, L->V, L->r_s, L->B, L->r_l, Y, yt, d, st, dep, nullptr, amax_y);
 }
 
 ft_status ft_linear_bwd(const ft_linear* L, const void* dY, const void* X, const void* P_save,
@@ -1228,8 +1230,8 @@ size_t ft_mlp_workspace_bytes(const ft_linear* up, const ft_linear* down, int64_
 }
 
 ft_status ft_mlp_fwd(const ft_linear* up, const ft_linear* down, const void* X, int64_t M, const float* amax_x,
-                     const float* amax_h, void* H, void* Y, ft_dtype yt, void* P_up, void* P_down, void* ws,
-                     size_t ws_bytes, void* stream) {
+                     const float* amax_h, void* H, void* Y, ft_dtype yt, void* P_up, void* P_down, float* amax_h_out,
+                     void* ws, size_t ws_bytes, void* stream) {
     FT_TRY(check_linear(up));
     FT_TRY(check_linear(down));
     if (down->K != up->N) return FT_ERR_SHAPE;
@@ -1242,7 +1244,8 @@ ft_status ft_mlp_fwd(const ft_linear* up, const ft_linear* down, const void* X, 
     if (!X || !amax_h || !H || !Y || (r_up > 0 && !P_up) || (r_dn > 0 && !P_down)) return FT_ERR_INVALID_ARG;
     // H leaves the fused epilogue in whole 32-byte sectors
     if (!al16(X) || (reinterpret_cast<uintptr_t>(H) & 31u) || !al16(Y) || (P_up && !al16(P_up)) ||
-        (P_down && !al16(P_down)) || (reinterpret_cast<uintptr_t>(amax_h) & 3u))
+        (P_down && !al16(P_down)) || (reinterpret_cast<uintptr_t>(amax_h) & 3u) ||
+        (reinterpret_cast<uintptr_t>(amax_h_out) & 3u))
         return FT_ERR_ALIGN;
     const WsPlan wu = plan_ws(M, up->N, up->K, up->r_s, up->r_l);
     const WsPlan wd = plan_ws(M, down->N, down->K, down->r_s, down->r_l);
@@ -1266,7 +1269,7 @@ ft_status ft_mlp_fwd(const ft_linear* up, const ft_linear* down, const void* X, 
     mo.tscale = reinterpret_cast<float*>(wsd + wd.gact);
     FT_TRY(run_gemm(false, wsu + wu.codes, wsu + wu.sfslab, reinterpret_cast<float*>(wsu + wu.gact), M, up->K,
                     up->op_k, up->w_k.tscale, up->N, P_up, up->V, up->r_s, up->B, up->r_l, H, FT_BF16, d, st, dep,
-                    &mo));
+                    &mo, amax_h_out));
     // FC2: its down-projections of H (no second quantization), then its GEMM on Q(H)
     FT_TRY(run_qdown(H, M, down->K, down->U, down->r_s, down->A, down->r_l, down->s, nullptr, nullptr, nullptr,
                      nullptr, P_down, wsd, wd, d, st, false));
@@ -1379,7 +1382,7 @@ extern "C" ft_status ft_linear_fwd_noalloc(const ft_linear* L, const void* X, in
     if (ft_workspace_bytes(M, L->N, L->K, L->r_s, L->r_l) > kNoAllocScratchBytes) return FT_ERR_WORKSPACE;
     void* scratch = nullptr;
     FT_TRY(noalloc_scratch(&scratch));
-    return ft_linear_fwd(L, X, M, amax_x, Y, yt, P_save, scratch, kNoAllocScratchBytes, stream);
+    return ft_linear_fwd(L, X, M, amax_x, Y, yt, P_save, nullptr, scratch, kNoAllocScratchBytes, stream);
 }
 
 extern "C" size_t ft_linear_fwd_noalloc_max_bytes(void) { return kNoAllocScratchBytes; }

@@ -141,6 +141,10 @@ struct Params {
     uint8_t* q_scales;
     uint8_t* q_slab;
     float* q_tscale;
+    // null, or a float (as its bits) raised to the largest |value| the
+    // epilogue writes (bf16 Y or H as rounded, FP32 Y as stored): the next
+    // quantizer's tensor amax, found without another pass
+    unsigned int* amax_out;
 };
 
 struct Layout {
@@ -711,6 +715,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
         bool ok = true;
         int local = 0;
         const int64_t ldo = (int64_t)p.Nout * (p.out_f32 ? 4 : 2);  // output row bytes
+        // running max of |output| over this thread's values (bf16 pairs as
+        // two 16-bit lanes, or FP32 bits), for p.amax_out
+        uint32_t am2 = 0, am32 = 0;
         // the FP32 tensor scales of the operands (a bf16 activation has none)
         const float gab = p.ga ? __fmul_rn(*p.ga, *p.gb) : *p.gb;
         // MLP fusion: the encode table of Q(H) for the caller's tensor amax,
@@ -783,6 +790,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                             __fmaf_rn(gab, __uint_as_float(v[2 * k + 1]), has_lr ? __uint_as_float(lr[2 * k + 1]) : 0.0f);
                         __nv_bfloat162 t = __floats2bfloat162_rn(y0, y1);
                         pk[c][k] = *reinterpret_cast<uint32_t*>(&t);
+                        if (!kMlp) am2 = __vmaxu2(am2, pk[c][k] & 0x7FFF7FFFu);
                     }
                 }
                 // every TMEM read of this tile is done: the MMA warp may
@@ -806,7 +814,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     for (int c = 0; c < 8; ++c) {
                         uint32_t w[8];
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) w[k] = gelu_bf16x2_tab(pk[c][k], gtab);
+                        for (int k = 0; k < 8; ++k) {
+                            w[k] = gelu_bf16x2_tab(pk[c][k], gtab);
+                            am2 = __vmaxu2(am2, w[k] & 0x7FFF7FFFu);
+                        }
                         uint32_t sbyte;
                         const uint2 q = quant_block16_m(w, amax_bits_16(w), qt, tab, sbyte);
                         if (in) {
@@ -851,8 +862,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     uint32_t y[16];
 #pragma unroll
                     for (int k = 0; k < 16; ++k)
+                    {
                         y[k] = __float_as_uint(
                             __fmaf_rn(gab, __uint_as_float(v[k]), has_lr ? __uint_as_float(lr[k]) : 0.0f));
+                        am32 = max(am32, y[k] & 0x7FFFFFFFu);
+                    }
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         named_bar_sync(1 + grp, 128);
@@ -866,6 +880,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                 __syncwarp();
                 if (lane == 0) release_acc();
             }
+        }
+        if (p.amax_out) {
+            // rows past M and padding columns hold zeros; one reduction per
+            // warp and launch (non-negative floats order like their bits)
+            uint32_t a = max(max(am2 & 0xFFFFu, am2 >> 16) << 16, am32);
+            a = __reduce_max_sync(0xFFFFFFFFu, a);
+            if (lane == 0 && a != 0u) atomicMax(p.amax_out, a);
         }
     }
 

@@ -238,10 +238,16 @@ ft_status ft_gelu_bf16(const void* y, void* h, int64_t n, void* stream);
  *   amax_x : device float max|X|, or NULL to compute it.
  *   Y      : [M, N] dense, FT_BF16 or FT_F32 (yt).
  *   P_save : bf16 [M, r_s + r_l] dense, written; the backward reads it.
+ *   amax_y : NULL, or a device float >= 0 that the call raises to
+ *            max(*amax_y, max|Y|) over Y as stored: the tensor amax of the
+ *            next layer's input, found by the GEMM's epilogue without
+ *            another pass over Y (section 3.3's fusion, the amax for a
+ *            single-pass quantize next).  Zero it before the call to get
+ *            max|Y| itself.  4-byte aligned (FT_ERR_ALIGN otherwise).
  *   N, K   : multiples of 256 (the scale rows stay 16-byte aligned for TMA).
  *   ws     : at least ft_workspace_bytes(M, N, K, r_s, r_l) bytes.         */
 ft_status ft_linear_fwd(const ft_linear* L, const void* X, int64_t M, const float* amax_x,
-                        void* Y, ft_dtype yt, void* P_save, void* ws, size_t ws_bytes,
+                        void* Y, ft_dtype yt, void* P_save, float* amax_y, void* ws, size_t ws_bytes,
                         void* stream);
 
 /* ft_linear_bwd -- Eq. 3 and the adapter gradients (section 3.2).
@@ -274,6 +280,10 @@ ft_status ft_linear_bwd(const ft_linear* L, const void* dY, const void* X, const
  *   Y      : [M, N] out, FT_BF16 or FT_F32 (yt).
  *   P_up [M, up r_s + r_l], P_down [M, down r_s + r_l]: bf16 out, the
  *            layers' saved down-projections (NULL when the rank is 0).
+ *   amax_h_out: NULL, or a device float >= 0 raised to max(*amax_h_out,
+ *            max|H|): the exact amax of this call's H, from FC1's
+ *            epilogue, to pass as amax_h on the next step (delayed
+ *            scaling).  4-byte aligned.
  *   ws     : ft_mlp_workspace_bytes(up, down, M) bytes, zero-filled once.
  *            After the call it holds Q(H) as the down layer's quantized
  *            activation: at byte offset ft_workspace_bytes(M, up->N, up->K,
@@ -281,8 +291,8 @@ ft_status ft_linear_bwd(const ft_linear* L, const void* dY, const void* X, const
  *            layer's workspace, laid out as ft_workspace_qact describes for
  *            (M, down->N, down->K, down->r_s, down->r_l).                  */
 ft_status ft_mlp_fwd(const ft_linear* up, const ft_linear* down, const void* X, int64_t M, const float* amax_x,
-                     const float* amax_h, void* H, void* Y, ft_dtype yt, void* P_up, void* P_down, void* ws,
-                     size_t ws_bytes, void* stream);
+                     const float* amax_h, void* H, void* Y, ft_dtype yt, void* P_up, void* P_down, float* amax_h_out,
+                     void* ws, size_t ws_bytes, void* stream);
 size_t ft_mlp_workspace_bytes(const ft_linear* up, const ft_linear* down, int64_t M);
 
 /* Workspace sizes (bytes) for the calls above.  Zero-fill a workspace once

@@ -38,7 +38,7 @@ int main(void) {
     ft_fp4 out;
     memset(&out, 0, sizeof(out));
     CHECK(ft_quantize(NULL, 128, 256, 256, FT_BLK_1x16, NULL, &out, NULL, 0, NULL) == FT_ERR_INVALID_ARG);
-    CHECK(ft_linear_fwd(NULL, NULL, 128, NULL, NULL, FT_BF16, NULL, NULL, 0, NULL) == FT_ERR_INVALID_ARG);
+    CHECK(ft_linear_fwd(NULL, NULL, 128, NULL, NULL, FT_BF16, NULL, NULL, NULL, 0, NULL) == FT_ERR_INVALID_ARG);
 
     /* the quantizer's launch mode switch is host-only */
     CHECK(ft_set_cooperative_quantizer(1) == FT_OK);

@@ -99,28 +99,30 @@ def test_linear_validation_happens_on_the_host(L):
     ws = L.ft_workspace_bytes(128, 256, 256, 16, 16)
     ok = _linear()
     bad_n = _linear(N=320)
-    assert L.ft_linear_fwd(ctypes.byref(bad_n), x, 128, None, x, 0, x, x, ws, None) == FT_ERR_SHAPE
+    assert L.ft_linear_fwd(ctypes.byref(bad_n), x, 128, None, x, 0, x, None, x, ws, None) == FT_ERR_SHAPE
     bad_r = _linear(r_s=8)
-    assert L.ft_linear_fwd(ctypes.byref(bad_r), x, 128, None, x, 0, x, x, ws, None) == FT_ERR_SHAPE
+    assert L.ft_linear_fwd(ctypes.byref(bad_r), x, 128, None, x, 0, x, None, x, ws, None) == FT_ERR_SHAPE
     big_r = _linear(r_s=80, r_l=64)
-    assert L.ft_linear_fwd(ctypes.byref(big_r), x, 128, None, x, 0, x, x, ws, None) == FT_ERR_SHAPE
-    assert L.ft_linear_fwd(None, x, 128, None, x, 0, x, x, ws, None) == FT_ERR_INVALID_ARG
-    assert L.ft_linear_fwd(ctypes.byref(ok), x, 128, None, x, 5, x, x, ws, None) == FT_ERR_INVALID_ARG
-    assert L.ft_linear_fwd(ctypes.byref(ok), x, 128, None, x, 0, x, x, ws - 1, None) == FT_ERR_WORKSPACE
-    assert L.ft_linear_fwd(ctypes.byref(ok), x + 8, 128, None, x, 0, x, x, ws, None) == FT_ERR_ALIGN
+    assert L.ft_linear_fwd(ctypes.byref(big_r), x, 128, None, x, 0, x, None, x, ws, None) == FT_ERR_SHAPE
+    assert L.ft_linear_fwd(None, x, 128, None, x, 0, x, None, x, ws, None) == FT_ERR_INVALID_ARG
+    assert L.ft_linear_fwd(ctypes.byref(ok), x, 128, None, x, 5, x, None, x, ws, None) == FT_ERR_INVALID_ARG
+    assert L.ft_linear_fwd(ctypes.byref(ok), x, 128, None, x, 0, x, None, x, ws - 1, None) == FT_ERR_WORKSPACE
+    assert L.ft_linear_fwd(ctypes.byref(ok), x + 8, 128, None, x, 0, x, None, x, ws, None) == FT_ERR_ALIGN
+    # the epilogue's amax word must be 4-byte aligned
+    assert L.ft_linear_fwd(ctypes.byref(ok), x, 128, None, x, 0, x, x + 2, x, ws, None) == FT_ERR_ALIGN
     # the transposed weight view must share the scale grid
     shared = _linear()
     shared.w_n.scales = 0x300000
-    assert L.ft_linear_fwd(ctypes.byref(shared), x, 128, None, x, 0, x, x, ws, None) == FT_ERR_INVALID_ARG
+    assert L.ft_linear_fwd(ctypes.byref(shared), x, 128, None, x, 0, x, None, x, ws, None) == FT_ERR_INVALID_ARG
     # the weight operand images are required and 16-byte aligned
     no_sf = _linear()
     no_sf.op_n = None
-    assert L.ft_linear_fwd(ctypes.byref(no_sf), x, 128, None, x, 0, x, x, ws, None) == FT_ERR_INVALID_ARG
+    assert L.ft_linear_fwd(ctypes.byref(no_sf), x, 128, None, x, 0, x, None, x, ws, None) == FT_ERR_INVALID_ARG
     odd_sf = _linear()
     odd_sf.op_k = 0x100008
-    assert L.ft_linear_fwd(ctypes.byref(odd_sf), x, 128, None, x, 0, x, x, ws, None) == FT_ERR_ALIGN
+    assert L.ft_linear_fwd(ctypes.byref(odd_sf), x, 128, None, x, 0, x, None, x, ws, None) == FT_ERR_ALIGN
     # M = 0: nothing to do
-    assert L.ft_linear_fwd(ctypes.byref(ok), x, 0, None, x, 0, x, x, ws, None) == FT_OK
+    assert L.ft_linear_fwd(ctypes.byref(ok), x, 0, None, x, 0, x, None, x, ws, None) == FT_OK
     assert L.ft_linear_bwd(ctypes.byref(bad_n), x, x, x, 128, None, x, 0, x, x, x, ws, None) == FT_ERR_SHAPE
     assert L.ft_linear_bwd(ctypes.byref(ok), x, x, x, 128, None, x, 9, x, x, x, ws, None) == FT_ERR_INVALID_ARG
 
@@ -231,15 +233,15 @@ def test_1x16_weight_views_and_packing_validation(L):
     g1.w_n.blk = 0
     g1.w_n.scales = 0x300000  # its own scales
     # with M = 0 the call validates the views and returns, launching nothing
-    assert L.ft_linear_fwd(ctypes.byref(g1), x, 0, None, x, 0, x, x, ws, None) == FT_OK
+    assert L.ft_linear_fwd(ctypes.byref(g1), x, 0, None, x, 0, x, None, x, ws, None) == FT_OK
     mixed = _linear()
     mixed.w_k.blk = 0
-    assert L.ft_linear_fwd(ctypes.byref(mixed), x, 128, None, x, 0, x, x, ws, None) == FT_ERR_SHAPE
+    assert L.ft_linear_fwd(ctypes.byref(mixed), x, 128, None, x, 0, x, None, x, ws, None) == FT_ERR_SHAPE
     no_sc = _linear()
     no_sc.w_k.blk = 0
     no_sc.w_n.blk = 0
     no_sc.w_n.scales = None
-    assert L.ft_linear_fwd(ctypes.byref(no_sc), x, 128, None, x, 0, x, x, ws, None) == FT_ERR_INVALID_ARG
+    assert L.ft_linear_fwd(ctypes.byref(no_sc), x, 128, None, x, 0, x, None, x, ws, None) == FT_ERR_INVALID_ARG
     g = 0x100000
     assert L.ft_pack_weight_operands_1x16(g, None, g, g, 256, 256, g, g, None) == FT_ERR_INVALID_ARG
     assert L.ft_pack_weight_operands_1x16(g, g, g, None, 256, 256, g, g, None) == FT_ERR_INVALID_ARG
@@ -260,12 +262,12 @@ def test_precision_field_is_validated_on_the_host(L):
                                    (2, 0, x + 4, FT_ERR_ALIGN)]:
         lin = _linear()
         lin.precision, lin.wd_k, lin.wd_n = prec, wd_k or None, wd_n or None
-        assert L.ft_linear_fwd(ctypes.byref(lin), x, 128, None, x, 0, x, x, ws, None) == want, prec
+        assert L.ft_linear_fwd(ctypes.byref(lin), x, 128, None, x, 0, x, None, x, ws, None) == want, prec
         assert L.ft_linear_bwd(ctypes.byref(lin), x, x, x, 128, None, x, 0, x, x, x, ws, None) == want, prec
     # a complete 16-bit configuration passes validation (M = 0: nothing runs)
     lin = _linear()
     lin.precision, lin.wd_k, lin.wd_n = 3, x, x
-    assert L.ft_linear_fwd(ctypes.byref(lin), x, 0, None, x, 0, x, x, ws, None) == FT_OK
+    assert L.ft_linear_fwd(ctypes.byref(lin), x, 0, None, x, 0, x, None, x, ws, None) == FT_OK
 
 
 def test_dequant_weight_operands_validation(L):

@@ -464,3 +464,22 @@ def test_precision_variants(precision, wl):
         Xr = d(inp["X"])[rows]
         check_fp32_sum_bound(host(Y)[rows], Xr @ Wq.T + Pd @ LRf.T,
                              np.abs(Xr) @ np.abs(Wq).T + np.abs(Pd) @ np.abs(LRf).T, shape.K)
+
+
+@pytest.mark.parametrize("out_dtype", ["bf16", "f32"])
+def test_epilogue_amax_is_exact(out_dtype):
+    """amax_y: the GEMM epilogue raises the word to max|Y| over Y as stored
+    (the next quantizer's tensor amax); a larger value already there stays."""
+    shape = ft_synth.LinearShape("amax", 300, 512, 768, 32, 32, outlier_channels=4, outlier_factor=20.0)
+    inp, U, V, Wr, layer = _prep(shape, 81, None, None, None)
+    X = dev_bf16(inp["X"])
+    ot = ft.BF16 if out_dtype == "bf16" else ft.F32
+    am = torch.zeros(1, dtype=torch.float32, device="cuda")
+    Y, _ = ft.ft_linear_fwd(layer, X, out_dtype=ot, amax_y=am)
+    torch.cuda.synchronize()
+    assert ft.ft_device_error() == 0
+    assert am.item() == Y.abs().max().float().item()
+    big = torch.full((1,), 1e30, dtype=torch.float32, device="cuda")
+    ft.ft_linear_fwd(layer, X, out_dtype=ot, amax_y=big)
+    torch.cuda.synchronize()
+    assert big.item() == np.float32(1e30)

@@ -111,3 +111,31 @@ def test_fused_mlp_forward(case):
         m = oracle.mlp_fwd(np.ascontiguousarray(up_inp["X"][rows]), dict(up_o, qw=oracle.quantize_16x16(up_o["W_res"])),
                            dict(dn_o, qw=qw), amax_h, amax_x=oracle.amax_bf16(up_inp["X"]))
         assert oracle.rel_fro(Yg, m["Y"]) <= TOL
+
+
+def test_fused_mlp_reports_amax_of_h_for_delayed_scaling():
+    """amax_h_out = max|H| exactly (FC1's epilogue); passed back as amax_h
+    (the next step's tensor scale) it quantizes H as the oracle does with the
+    true amax."""
+    M = 300
+    up_shape = ft_synth.LinearShape("mlp_up", M, 256, 512, 16, 16, outlier_channels=4, outlier_factor=20.0)
+    dn_shape = ft_synth.LinearShape("mlp_dn", M, 512, 256, 16, 32, w_std=0.05)
+    up_inp, _, up = _layer(up_shape, 41)
+    _, _, down = _layer(dn_shape, 42)
+    X = dev_bf16(up_inp["X"])
+    am = torch.zeros(1, dtype=torch.float32, device="cuda")
+    _, H, _, _ = ft.ft_mlp_fwd(up, down, X, scalar_dev(1.0), ws=ft.Workspace(), amax_h_out=am)
+    torch.cuda.synchronize()
+    assert ft.ft_device_error() == 0
+    H_host = host_u16(H)
+    true_amax = float(np.abs(oracle.bf16_to_f64(H_host)).max())
+    assert am.item() == true_amax
+    ws = ft.Workspace()
+    _, H2, _, _ = ft.ft_mlp_fwd(up, down, X, am.clone(), ws=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(H2, H)
+    codes, scales, g = _q_h(ws, M, up, down)
+    rc, rs, rg = oracle.quantize_1x16(H_host, true_amax)
+    assert np.float32(g) == np.float32(rg)
+    np.testing.assert_array_equal(scales, rs)
+    np.testing.assert_array_equal(codes, rc)
