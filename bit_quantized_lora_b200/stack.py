@@ -80,21 +80,30 @@ class LinearStack:
         ft_linear_bwd(self.layers[j], dY, X, b.P, amax_dy=amax, out_dtype=self.out_dtype, dX=b.dX, dA=b.dA,
                       dB=b.dB, ws=self.ws)
 
-    def step(self, Xs: list[torch.Tensor], dYs: list[torch.Tensor], group=None) -> None:
+    def step(self, Xs: list[torch.Tensor], dYs: list[torch.Tensor], group=None, x_ready=None,
+             dy_ready=None) -> None:
         """Forward of every layer in order, then backward in reverse order.
         With a process group of more than one rank, each layer's adapter
         gradients are summed over the ranks by an all-reduce started right
         after its backward; the step returns once the current stream has
-        been made to wait for all of them."""
+        been made to wait for all of them.  x_ready / dy_ready: optional
+        CUDA events, one per layer, that the layer's forward / backward
+        waits for first (inputs arriving on another stream, e.g. host copies
+        overlapped with the layers before)."""
         import torch.distributed as dist
         exchange = dist.is_initialized() and dist.get_world_size(group) > 1
+        stream = torch.cuda.current_stream() if (x_ready is not None or dy_ready is not None) else None
         for j in range(len(self.layers)):
+            if x_ready is not None:
+                stream.wait_event(x_ready[j])
             self.forward_layer(j, Xs[j])
         handles = []
         if exchange:
             ft_set_cooperative_quantizer(True)
         try:
             for j in reversed(range(len(self.layers))):
+                if dy_ready is not None:
+                    stream.wait_event(dy_ready[j])
                 self.backward_layer(j, dYs[j], Xs[j])
                 if exchange and self.grad_slices[j] is not None:
                     handles.append(dist.all_reduce(self.grad_slices[j], op=dist.ReduceOp.SUM, group=group,
