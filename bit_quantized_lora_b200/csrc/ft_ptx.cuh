@@ -84,12 +84,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking check that the phase of `bar` with the given parity is complete.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Waits for the phase of `bar` with the given parity to complete.  Gives up
 // when *abort becomes nonzero (another role failed) or after kWaitLimitNs;
 // in the latter case it records `code` in the device error word and sets
 // *abort.  Returns true when the phase completed.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int code,
                                           volatile int* abort) {
+    // a phase that is already complete costs a few cycles this way; the
+    // potentially suspending try_wait costs tens even then, which the GEMM's
+    // MMA thread pays in tensor-pipe time (its MMA queue is shallow)
+    if (mbar_test_wait(bar, parity)) return true;
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {

@@ -268,7 +268,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < MAX_STAGES; ++i) {
-            mbar_init(&bars[B_FULL + i], 1);
+            // CTA pairs: the leader's FULL also counts both CTAs' scale warps
+            // (the stage's scales are in tensor memory), so the MMA thread
+            // waits on one barrier per stage
+            mbar_init(&bars[B_FULL + i], kPair ? 1 + 2 * NUM_SF_WARPS : 1);
             mbar_init(&bars[B_SFFULL + i], 1);
             mbar_init(&bars[B_EMPTY + i], 1);
         }
@@ -479,6 +482,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                 tc_commit_pair(peer0 + 8u * (uint32_t)b);
             };
             uint32_t it = 0;
+            // ring positions of `it`, advanced by increments (the MMA
+            // thread's per-stage work costs tensor-pipe time; no divisions)
+            int s = 0;
+            uint32_t ph = 0;
             bool ok = true;
             int local = 0;
             for (int tile = unit; tile < num_tiles && ok; tile += nunits, ++local) {
@@ -489,24 +496,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                 }
                 tc_fence_after();
                 for (int kt = 0; kt < KT; ++kt, ++it) {
-                    const int s = it % S;
-                    const int sb = it % SF_SLOTS_P;
-                    if (!mbar_wait_cluster(&bars[B_FULL + s], (it / S) & 1, ERR_WAIT_FULL, abort_flag) ||
-                        !mbar_wait_cluster(&bars[B_SF_READY + sb], (it / SF_SLOTS_P) & 1, ERR_WAIT_SF, abort_flag)) {
+                    if (!mbar_wait_cluster(&bars[B_FULL + s], ph, ERR_WAIT_FULL, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t a_lo = a_lo0 + s * (A_BYTES >> 4);
                     const uint32_t b_lo = b_lo0 + s * (B_SLOT_P >> 4);
-                    const uint32_t sf = tmem + RING_COL_P + sb * SF_SLOT_COLS;
+                    const uint32_t sf = tmem + RING_COL_P + s * SF_SLOT_COLS;
 #pragma unroll
                     for (int j = 0; j < KSTEPS; ++j)
                         umma_nvfp4_pair(tmem + ACC_COL, make_desc(a_lo + 2 * j, hi_sw128),
                                         make_desc(b_lo + 2 * j, hi_sw128), idesc, sf + 4 * j, sf + 16 + 8 * j,
                                         (kt | j) != 0);
+                    // the stage's buffers and its scale columns are free again
                     commit_both(B_EMPTY + s);
-                    commit_both(B_SF_FREE + sb);
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
                 if (!ok) break;
                 commit_both(B_ACC_FULL);
@@ -544,6 +552,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
             const uint32_t a_lo0 = ((base + L.a) >> 4) | (1u << 16);
             const uint32_t b_lo0 = ((base + L.b) >> 4) | (1u << 16);
             uint32_t it = 0;
+            int s = 0;  // it % S and (it / S) & 1, advanced by increments
+            uint32_t ph = 0;
             bool ok = true;
             int local = 0;
             for (int tile = unit; tile < num_tiles && ok; tile += nunits, ++local) {
@@ -555,10 +565,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                 }
                 tc_fence_after();
                 for (int kt = 0; kt < KT; ++kt, ++it) {
-                    const int s = it % S;
                     const int sb = it & 1;
-                    if (!mbar_wait(&bars[B_FULL + s], (it / S) & 1, ERR_WAIT_FULL, abort_flag) ||
-                        (!kBf16 && (!mbar_wait(&bars[B_SFFULL + s], (it / S) & 1, ERR_WAIT_FULL, abort_flag) ||
+                    if (!mbar_wait(&bars[B_FULL + s], ph, ERR_WAIT_FULL, abort_flag) ||
+                        (!kBf16 && (!mbar_wait(&bars[B_SFFULL + s], ph, ERR_WAIT_FULL, abort_flag) ||
                                     !mbar_wait(&bars[B_SF_READY + sb], (it >> 1) & 1, ERR_WAIT_SF, abort_flag)))) {
                         ok = false;
                         break;
@@ -573,6 +582,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                             umma_bf16(tmem + ACC_COL, make_desc(a_lo + 2 * j, hi_sw128),
                                       make_desc(b_lo + 2 * j, hi_sw128), idesc, (kt | j) != 0);
                         tc_commit(&bars[B_EMPTY + s]);
+                        if (++s == S) {
+                            s = 0;
+                            ph ^= 1u;
+                        }
                         continue;
                     }
                     const uint32_t sf = tmem + R2_COL + sb * SF_SLOT_COLS;
@@ -583,6 +596,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                                    (kt | j) != 0);
                     tc_commit(&bars[B_EMPTY + s]);
                     tc_commit(&bars[B_SF_FREE + sb]);
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
                 if (!ok) break;
                 if (has_lr) {
@@ -641,12 +658,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                 }
                 for (int kt = 0; kt < KT; ++kt, ++it) {
                     const int s = it % S;
-                    constexpr int NSL = kPair ? SF_SLOTS_P : SF_SLOTS;
-                    const int sb = it % NSL;
-                    const uint32_t fph = ((it / NSL) & 1) ^ 1;
+                    // one-CTA tiles: a two-slot ring freed by the MMAs'
+                    // commits; CTA pairs: the stage's own slot, whose last
+                    // readers (the MMAs of stage it - S) finished before this
+                    // CTA's producer refilled the stage
+                    const int sb = kPair ? s : (int)(it & 1);
                     if (!mbar_wait(&bars[B_SFFULL + s], (it / S) & 1, ERR_WAIT_FULL, abort_flag) ||
-                        !(kPair ? mbar_wait_cluster(&bars[B_SF_FREE + sb], fph, ERR_WAIT_SF, abort_flag)
-                                : mbar_wait(&bars[B_SF_FREE + sb], fph, ERR_WAIT_SF, abort_flag))) {
+                        (!kPair && !mbar_wait(&bars[B_SF_FREE + sb], ((it >> 1) & 1) ^ 1, ERR_WAIT_SF, abort_flag))) {
                         ok = false;
                         break;
                     }
@@ -674,7 +692,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_gemm_fp4(const __grid_consta
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) {
-                        if (kPair) mbar_arrive_cluster(mapa_shared(smem_u32(&bars[B_SF_READY + sb]), 0));
+                        if (kPair) mbar_arrive_cluster(mapa_shared(smem_u32(&bars[B_FULL + sb]), 0));
                         else mbar_arrive(&bars[B_SF_READY + sb]);
                     }
                 }
