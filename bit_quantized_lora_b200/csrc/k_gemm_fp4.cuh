@@ -27,7 +27,11 @@
 //
 // Blackwell mapping: one CTA per SM, persistent over 128x256 output tiles
 // (a tcgen05 MMA costs about the same for N = 128 as for N = 256, so the
-// wide tile doubles the work per instruction).
+// wide tile doubles the work per instruction); or, the default for more
+// than 128 rows, CTA pairs on 256x256 tiles (kPair, below).  The MMA queue
+// is shallow: every instruction the MMA thread runs between MMAs costs
+// tensor-pipe time, so its per-stage path is kept to one non-suspending
+// barrier check, the MMAs and the commits (ring slots advance by increments).
 //   warp 0  TMA producer: per stage, the weight block (codes + scales, one
 //           3-D box) and the activation scale slabs on one barrier, the
 //           activation code tile (128 B swizzle) on another; per tile the
