@@ -97,9 +97,10 @@ constexpr uint32_t TMEM_COLS = 512;
 // shared in time: the scale ring while the mainloop runs, low-rank half 1
 // after it (the next tile's first scale copy waits for the epilogue).
 constexpr uint32_t ACC_COL = 0, LR0_COL = 256, R2_COL = 384, SF_SLOT_COLS = 48;
-// CTA pairs: the scale ring takes [256, 496), five slots, during the
-// mainloop (a slot's refill waits on the other SM's signals, so the ring is
-// deeper); both low-rank halves are computed after it, into [256, 512).
+// CTA pairs: each stage slot s keeps its scales in columns
+// [256 + 48 s, 256 + 48 s + 48) during the mainloop (at most four stages,
+// [256, 448)); both low-rank halves are computed after it, into [256, 512).
+// The barrier arrays below are sized for SF_SLOTS_P slots.
 constexpr int SF_SLOTS = 2, SF_SLOTS_P = 5;
 constexpr uint32_t RING_COL_P = LR0_COL;
 
