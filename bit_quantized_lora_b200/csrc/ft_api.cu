@@ -180,6 +180,22 @@ ft_status launch_overlapped(void (*kernel)(P), dim3 grid, dim3 block, size_t sme
     cfg.attrs = attr;
     return cuda_ok(cudaLaunchKernelEx(&cfg, kernel, p));
 }
+// The same launch for a kernel taking plain arguments.
+template <typename... KArgs, typename... Args>
+ft_status launch_overlapped_args(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                 Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cuda_ok(cudaLaunchKernelEx(&cfg, kernel, args...));
+}
 inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 inline int cdiv(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
@@ -372,7 +388,9 @@ WsPlan plan_ws(int64_t M, int64_t N, int64_t K, int64_t r_s, int64_t r_l) {
 // ------------------------------------------------------------ pieces
 ft_status run_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, float* slot, const DevInfo* d,
                    cudaStream_t st) {
-    FT_TRY(cuda_ok(cudaMemsetAsync(slot, 0, sizeof(float), st)));
+    // slot: the first half of an 8-byte-aligned 64-bit word that the kernel
+    // tags with this launch's epoch (no clearing, no memset between kernels)
+    if (reinterpret_cast<uintptr_t>(slot) & 7u) return FT_ERR_ALIGN;
     const int64_t vecs = rows * (cols / 8);
     // a few CTAs per SM, each thread looping with eight 16-byte loads in
     // flight: every CTA ends in one same-address atomic, which serialise in
@@ -380,8 +398,9 @@ ft_status run_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, float*
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(vecs, 8 * 256), (int64_t)d->sms * 4));
     {
         LaunchTimer _lt(KID_AMAX, st);
-        ft::k_amax_bf16<<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(x), rows, cols, ld,
-                                              reinterpret_cast<unsigned int*>(slot));
+        FT_TRY(launch_overlapped_args(ft::k_amax_bf16, dim3((unsigned)grid), dim3(256), 0, st,
+                                 static_cast<const uint16_t*>(x), rows, cols, ld,
+                                 reinterpret_cast<unsigned long long*>(slot), next_epoch()));
         _lt.stop();
     }
     return last_launch();

@@ -36,14 +36,21 @@ __global__ void __launch_bounds__(1024) k_gelu_bf16(const uint16_t* __restrict__
 
 // ------------------------------------------------------------------ amax
 // max|x| over a bf16 matrix (cols % 8 == 0, rows 16-byte aligned).  Each
-// block reduces its share and folds it into *out with an integer atomicMax on
-// the float bits (non-negative floats order like their bit patterns), so the
-// result is exact and independent of scheduling.  *out must be 0 on entry.
-// The grid is kept to a few blocks per SM (same-address atomics serialise in
-// L2); each thread keeps eight to sixteen independent 16-byte loads in flight.
+// block reduces its share and folds it into the 64-bit word *out as
+// (epoch << 32) | float bits with an integer atomicMax (non-negative floats
+// order like their bit patterns), so the result is exact and independent of
+// scheduling; the tag makes any value an earlier launch left there smaller
+// than this launch's, so the word needs no clearing, and every block
+// publishes, a zero block included.  The low 32 bits (the word's first four
+// bytes) are then the float max|x|.  The grid is kept to a few blocks per SM
+// (same-address atomics serialise in L2); each thread keeps eight 16-byte
+// loads in flight.  Launched with programmatic serialization: it waits for
+// the kernel before it, whose output it may read, after its own launch.
 __global__ void __launch_bounds__(256) k_amax_bf16(const uint16_t* __restrict__ x, int64_t rows,
                                                    int64_t cols, int64_t ld,
-                                                   unsigned int* __restrict__ out) {
+                                                   unsigned long long* __restrict__ out,
+                                                   unsigned long long epoch) {
+    grid_dep_wait();
     constexpr int U = 8;
     const int64_t vec_per_row = cols / 8;
     const int64_t total = rows * vec_per_row;
@@ -93,7 +100,7 @@ __global__ void __launch_bounds__(256) k_amax_bf16(const uint16_t* __restrict__ 
     if (threadIdx.x == 0) {
         uint32_t b = 0;
         for (int w = 0; w < (int)(blockDim.x >> 5); ++w) b = max(b, red[w]);
-        if (b) atomicMax(out, b << 16);
+        atomicMax(out, (epoch << 32) | (unsigned long long)(b << 16));
     }
 }
 
