@@ -472,7 +472,8 @@ def clone_layer(ft, L):
 
 
 def bench_quantizers(torch, ft, dev, hbm_gbs, flush, reps=10):
-    """The standalone quantize kernels (SURVEY's quantize metric): per case
+    """The standalone quantize kernels (the GB/s-against-HBM half of the
+    metric): per case
     the algorithmic bytes of one call, its time (CUDA events around the call,
     L2 flushed before each) and the fraction of the HBM peak.  'supplied'
     runs take the tensor amax from the caller (single pass); 'computed' runs
